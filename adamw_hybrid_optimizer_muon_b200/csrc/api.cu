@@ -1,0 +1,787 @@
+// C ABI of the MuonAdamW library: validation, workspace layout, the per-step
+// orchestration of the kernels, and the plan over a parameter table.
+//
+// Structure of one step ("How nanochat Combines Muon and AdamW in a Single
+// Optimizer", "The MuonAdamW Class Architecture": one step() that dispatches
+// on each group's kind):
+//   1. one multi-tensor AdamW launch over every AdamW tensor (adamw.cu)
+//   2. per Muon bucket of same-shape matrices ("Muon Step Implementation":
+//      stacked batches): momentum + norm (muon_prep.cu), norm finalize, then
+//      the Newton-Schulz chain (ns_tc.cu, or ns_simt.cu in fp32 mode), whose
+//      last GEMM writes the decayed, updated weights.
+// The host never synchronises. Every argument is checked before the first
+// launch, so a failing call changes nothing.
+#include <algorithm>
+#include <climits>
+#include <cmath>
+#include <cstdlib>
+#include <cstring>
+#include <new>
+#include <vector>
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace ma {
+
+__device__ int g_status = 0;
+
+static long long g_host_wait_limit_ns = 2000000000LL;
+long long host_wait_limit_ns() { return g_host_wait_limit_ns; }
+
+int* device_status_ptr() {
+    static int* cached[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!cached[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) return nullptr;
+        cached[dev] = reinterpret_cast<int*>(ptr);
+    }
+    return cached[dev];
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// sm_100a code runs only on compute capability 10.0; cache per device.
+int device_ok_and_sms(int* sms) {
+    static int cached_sms[64] = {0};
+    static int cached_ok[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MA_ERR_CUDA;
+    if (dev < 0 || dev >= 64) return MA_ERR_UNSUPPORTED;
+    if (!cached_ok[dev]) {
+        int maj = 0, min = 0, n = 0;
+        if (cudaDeviceGetAttribute(&maj, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&min, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return MA_ERR_CUDA;
+        if (maj != 10 || min != 0) return MA_ERR_UNSUPPORTED;
+        cached_sms[dev] = n;
+        cached_ok[dev] = 1;
+    }
+    if (sms) *sms = cached_sms[dev];
+    return MA_OK;
+}
+
+// ------------------------------------------------------------------ Muon geometry
+
+struct MuonGeom {
+    int64_t R, C, Rh;
+    int heads, transposed;
+    int64_t m, n, ldx, ldg;
+    int64_t units;
+    int64_t parts;
+    int esz;
+    bool quintic;
+    size_t off_x0, off_x1, off_g, off_g2, off_part, off_scale, total;
+};
+
+bool any_c(const ma_muon_hparams_t& hp) {
+    const int nc = hp.n_coeffs;
+    for (int k = 0; k < nc && k < MA_MAX_NS_STEPS; ++k)
+        if (hp.coeffs[k][2] != 0.f) return true;
+    return false;
+}
+
+int check_muon_hp(const ma_muon_hparams_t* hp) {
+    if (!hp) return MA_ERR_NULL;
+    if (hp->ns_steps < 1 || hp->ns_steps > MA_MAX_NS_STEPS) return MA_ERR_ARG;
+    if (!(hp->n_coeffs == 1 || hp->n_coeffs == hp->ns_steps)) return MA_ERR_ARG;
+    if (hp->scale_mode < 0 || hp->scale_mode > 2) return MA_ERR_ARG;
+    if (hp->precision < 0 || hp->precision > 1) return MA_ERR_ARG;
+    if (hp->heads < 1) return MA_ERR_SHAPE;
+    if (!(hp->beta >= 0.f && hp->beta <= 1.f)) return MA_ERR_ARG;
+    if (!(hp->eps >= 0.f) || !std::isfinite(hp->lr) || !std::isfinite(hp->weight_decay)) return MA_ERR_ARG;
+    for (int k = 0; k < hp->n_coeffs; ++k)
+        for (int j = 0; j < 3; ++j)
+            if (!std::isfinite(hp->coeffs[k][j])) return MA_ERR_ARG;
+    return MA_OK;
+}
+
+int muon_geom(int batch, int64_t R, int64_t C, const ma_muon_hparams_t& hp, MuonGeom* g) {
+    if (batch < 0 || R < 0 || C < 0) return MA_ERR_SHAPE;
+    if (hp.heads < 1 || (R > 0 && R % hp.heads != 0)) return MA_ERR_SHAPE;
+    g->R = R;
+    g->C = C;
+    g->heads = hp.heads;
+    g->Rh = R / hp.heads;
+    g->transposed = g->Rh > C ? 1 : 0;
+    g->m = std::min(g->Rh, C);
+    g->n = std::max(g->Rh, C);
+    g->ldx = round8(g->n);
+    g->ldg = round8(g->m);
+    g->units = (int64_t)batch * hp.heads;
+    g->parts = (g->Rh > 0 && C > 0) ? prep_parts_per_unit(g->Rh, C, g->transposed) : 0;
+    g->esz = hp.precision ? 4 : 2;
+    g->quintic = any_c(hp);
+    size_t off = 0;
+    const size_t xbytes = (size_t)g->units * g->m * g->ldx * g->esz;
+    const size_t gbytes = (size_t)g->units * g->m * g->ldg * g->esz;
+    g->off_x0 = off;
+    off = align_up(off + xbytes, kAlign);
+    g->off_x1 = off;
+    if (hp.ns_steps >= 2) off = align_up(off + xbytes, kAlign);
+    g->off_g = off;
+    off = align_up(off + gbytes, kAlign);
+    g->off_g2 = off;
+    if (g->quintic) off = align_up(off + gbytes, kAlign);
+    g->off_part = off;
+    off = align_up(off + (size_t)g->units * g->parts * sizeof(double), kAlign);
+    g->off_scale = off;
+    off = align_up(off + (size_t)g->units * sizeof(float), kAlign);
+    g->total = (batch == 0 || R == 0 || C == 0) ? 0 : off;
+    return MA_OK;
+}
+
+float shape_scale(int64_t R, int64_t C, int mode) {
+    const double r = (double)R / (double)C;
+    if (mode == 0) return (float)std::sqrt(std::max(1.0, r));
+    if (mode == 1) return (float)std::sqrt(r);
+    return 1.f;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? MA_OK : MA_ERR_CUDA; }
+
+// All checks passed; launch the whole Muon chain for one batch.
+int run_muon(int batch, const MuonGeom& g, float* const* W, const void* const* G, int gdt, float* const* M,
+             const ma_muon_hparams_t& hp, void* ws, cudaStream_t s, int sms, int* launches) {
+    if (g.total == 0) return MA_OK;
+    uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+    void* X0 = base + g.off_x0;
+    void* X1 = base + g.off_x1;
+    void* Gb = base + g.off_g;
+    void* G2 = base + g.off_g2;
+    double* part = reinterpret_cast<double*>(base + g.off_part);
+    float* scale = reinterpret_cast<float*>(base + g.off_scale);
+
+    MuonPrepLaunch P;
+    std::memset(&P, 0, sizeof(P));
+    P.batch = batch;
+    P.heads = g.heads;
+    P.transposed = g.transposed;
+    P.gdt = gdt;
+    P.nesterov = hp.nesterov ? 1 : 0;
+    P.x_f32 = hp.precision ? 1 : 0;
+    P.C = g.C;
+    P.Rh = g.Rh;
+    P.ldx = g.ldx;
+    P.x_unit = g.m * g.ldx;
+    P.parts = g.parts;
+    P.tiles_c = (g.C + kPrepTile - 1) / kPrepTile;
+    P.beta = hp.beta;
+    P.omb = 1.f - hp.beta;
+    P.X = X0;
+    P.partials = part;
+    for (int b = 0; b < batch; ++b) {
+        P.G[b] = G[b];
+        P.M[b] = M[b];
+    }
+    int st = cuda_status(launch_muon_prep(P, s));
+    if (st) return st;
+    st = cuda_status(launch_norm_finalize(part, g.parts, (int)g.units, hp.eps, scale, s));
+    if (st) return st;
+    *launches += 2;
+
+    NsParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.units = (int)g.units;
+    p.m = (int)g.m;
+    p.n = (int)g.n;
+    p.ldx = g.ldx;
+    p.ldg = g.ldg;
+    p.x_unit = g.m * g.ldx;
+    p.g_unit = g.m * g.ldg;
+    p.scale = scale;
+    p.transposed = g.transposed;
+    p.heads = g.heads;
+    p.Rh = g.Rh;
+    p.C = g.C;
+    p.decay = 1.f - hp.lr * hp.weight_decay;
+    p.lr_s = hp.lr * shape_scale(g.Rh, g.C, hp.scale_mode);
+    p.wait_limit_ns = host_wait_limit_ns();
+    p.status = device_status_ptr();
+    for (int b = 0; b < batch; ++b) p.W[b] = W[b];
+
+    auto launch = [&](int mode, const void* xb, const void* gb) -> int {
+        cudaError_t e = hp.precision ? launch_ns_simt(mode, p, xb, gb, s) : launch_ns_tc(mode, p, xb, gb, sms, s);
+        ++*launches;
+        return cuda_status(e);
+    };
+
+    void* cur = X0;
+    void* nxt = X1;
+    for (int k = 0; k < hp.ns_steps; ++k) {
+        const float* cf = hp.coeffs[hp.n_coeffs == 1 ? 0 : k];
+        p.a = cf[0];
+        p.b = cf[1];
+        p.c = cf[2];
+        p.first = (k == 0) ? 1 : 0;
+        const bool quint = cf[2] != 0.f;
+        p.coef_gram = quint ? 1.f : cf[1];
+        p.out = Gb;
+        if ((st = launch(NS_GRAM, cur, Gb))) return st;
+        void* Bbuf = Gb;
+        if (quint) {
+            p.xin = Gb;
+            p.out = G2;
+            if ((st = launch(NS_GRAMSQ, cur, Gb))) return st;
+            Bbuf = G2;
+        }
+        p.xin = cur;
+        if (k + 1 < hp.ns_steps) {
+            p.out = nxt;
+            if ((st = launch(NS_APPLY, cur, Bbuf))) return st;
+            std::swap(cur, nxt);
+        } else {
+            p.out = nullptr;
+            if ((st = launch(NS_FINAL, cur, Bbuf))) return st;
+        }
+    }
+    return MA_OK;
+}
+
+int check_ptr_array(const void* const* a, int n, size_t align) {
+    if (!a) return MA_ERR_NULL;
+    for (int i = 0; i < n; ++i) {
+        if (!a[i]) return MA_ERR_NULL;
+        if (!aligned(a[i], align)) return MA_ERR_ALIGN;
+    }
+    return MA_OK;
+}
+
+int check_muon_call(int batch, int64_t R, int64_t C, float* const* W, const void* const* G, int gdt,
+                    float* const* M, const ma_muon_hparams_t* hp, MuonGeom* g) {
+    int st = check_muon_hp(hp);
+    if (st) return st;
+    if (batch < 0 || R < 0 || C < 0) return MA_ERR_SHAPE;
+    if (batch > MA_MAX_BATCH) return MA_ERR_UNSUPPORTED;
+    if (gdt != MA_F32 && gdt != MA_BF16) return MA_ERR_DTYPE;
+    if ((st = muon_geom(batch, R, C, *hp, g))) return st;
+    if (batch == 0 || R == 0 || C == 0) return MA_OK;
+    if ((st = check_ptr_array(reinterpret_cast<const void* const*>(W), batch, 16))) return st;
+    if ((st = check_ptr_array(G, batch, 16))) return st;
+    if ((st = check_ptr_array(reinterpret_cast<const void* const*>(M), batch, 16))) return st;
+    if (C % 8 != 0) return MA_ERR_ALIGN;
+    if (g->units > 65535 || g->m > INT_MAX || g->n > INT_MAX || g->parts > INT_MAX) return MA_ERR_UNSUPPORTED;
+    return MA_OK;
+}
+
+// ------------------------------------------------------------------ AdamW helpers
+
+AdamwGroupConst adamw_const(const ma_adamw_hparams_t& h) {
+    AdamwGroupConst c;
+    const double bc1 = 1.0 - std::pow((double)h.beta1, (double)h.step);
+    const double bc2 = 1.0 - std::pow((double)h.beta2, (double)h.step);
+    c.decay = (float)(1.0 - (double)h.lr * (double)h.weight_decay);
+    c.step_size = (float)((double)h.lr / bc1);
+    c.inv_sqrt_bc2 = (float)(1.0 / std::sqrt(bc2));
+    c.beta1 = h.beta1;
+    c.beta2 = h.beta2;
+    c.omb1 = (float)(1.0 - (double)h.beta1);
+    c.omb2 = (float)(1.0 - (double)h.beta2);
+    c.eps = h.eps;
+    return c;
+}
+
+int check_adamw_hp(const ma_adamw_hparams_t* h) {
+    if (!h) return MA_ERR_NULL;
+    if (h->step < 1) return MA_ERR_ARG;
+    if (!(h->beta1 >= 0.f && h->beta1 < 1.f) || !(h->beta2 >= 0.f && h->beta2 < 1.f)) return MA_ERR_ARG;
+    if (!(h->eps >= 0.f) || !std::isfinite(h->lr) || !std::isfinite(h->weight_decay)) return MA_ERR_ARG;
+    return MA_OK;
+}
+
+struct AdamwItem {
+    float* p;
+    const void* g;
+    float* m;
+    float* v;
+    int64_t numel;
+    int group;
+};
+
+// Launch AdamW over items (all with gradient dtype gdt) in parameter-block batches.
+int run_adamw(const std::vector<AdamwItem>& items, int gdt, const AdamwGroupConst* grp, int ngroups, cudaStream_t s,
+              int* launches) {
+    static thread_local AdamwLaunch L;  // ~19 KB parameter block, copied at launch
+    size_t i = 0;
+    while (i < items.size()) {
+        std::memset(&L, 0, sizeof(L));
+        L.gdt = gdt;
+        for (int k = 0; k < ngroups; ++k) L.grp[k] = grp[k];
+        int64_t chunk = 0;
+        int nt = 0;
+        while (i < items.size() && nt < kAdamwMaxTensorsPerLaunch) {
+            const AdamwItem& it = items[i++];
+            if (it.numel == 0) continue;
+            AdamwTensorDesc& d = L.t[nt++];
+            d.p = it.p;
+            d.g = it.g;
+            d.m = it.m;
+            d.v = it.v;
+            d.numel = it.numel;
+            d.chunk0 = chunk;
+            d.group = it.group;
+            const size_t gal = gdt == MA_BF16 ? 8 : 16;
+            d.vec = aligned(it.p, 16) && aligned(it.m, 16) && aligned(it.v, 16) && aligned(it.g, gal);
+            chunk += (it.numel + kAdamwChunk - 1) / kAdamwChunk;
+            if (chunk > (int64_t)INT_MAX - kAdamwMaxTensorsPerLaunch) break;
+        }
+        L.ntensors = nt;
+        L.nchunks = chunk;
+        if (nt > 0) {
+            cudaError_t e = launch_adamw(L, s);
+            if (e != cudaSuccess) return MA_ERR_CUDA;
+            ++*launches;
+        }
+    }
+    return MA_OK;
+}
+
+__global__ void wait_selftest_kernel(long long limit_ns, int* status) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        // nothing ever arrives on `bar`: this wait must give up after limit_ns
+        mbar_wait_bounded(&bar, 0, &abort_flag, limit_ns, status);
+    }
+    __syncthreads();
+}
+
+}  // namespace
+
+cudaError_t launch_wait_selftest(long long limit_ns, int* status, cudaStream_t s) {
+    wait_selftest_kernel<<<1, 32, 0, s>>>(limit_ns, status);
+    return cudaGetLastError();
+}
+
+}  // namespace ma
+
+// ====================================================================== C ABI
+
+using namespace ma;
+
+struct ma_plan {
+    std::vector<ma_tensor_t> t;
+    std::vector<int32_t> kind;
+    std::vector<int32_t> group_kind;
+    std::vector<int> adamw_idx;
+    struct Bucket {
+        int group;
+        int64_t R, C;
+        std::vector<int> members;
+        int sub;  // matrices per sub-batch
+    };
+    std::vector<Bucket> buckets;
+    size_t ws_bytes = 0;
+    int last_launches = 0;
+};
+
+extern "C" {
+
+const char* ma_status_string(int s) {
+    switch (s) {
+        case MA_OK: return "ok";
+        case MA_ERR_NULL: return "null pointer";
+        case MA_ERR_SHAPE: return "bad shape or size";
+        case MA_ERR_DTYPE: return "bad dtype";
+        case MA_ERR_ALIGN: return "misaligned pointer or row length";
+        case MA_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case MA_ERR_UNSUPPORTED: return "unsupported request";
+        case MA_ERR_CUDA: return "CUDA runtime error";
+        case MA_ERR_TIMEOUT: return "device wait timed out";
+        case MA_ERR_ARG: return "hyperparameter out of range";
+        default: return "unknown status";
+    }
+}
+
+int ma_version(void) { return MA_VERSION; }
+
+size_t ma_struct_size(int which) {
+    switch (which) {
+        case 0: return sizeof(ma_tensor_t);
+        case 1: return sizeof(ma_group_t);
+        case 2: return sizeof(ma_muon_hparams_t);
+        case 3: return sizeof(ma_adamw_hparams_t);
+        default: return 0;
+    }
+}
+
+int ma_partition(const ma_tensor_t* t, int n, int32_t* kind_out) {
+    if (n < 0) return MA_ERR_SHAPE;
+    if (n == 0) return MA_OK;
+    if (!t || !kind_out) return MA_ERR_NULL;
+    for (int i = 0; i < n; ++i) {
+        if (t[i].ndim < 0) return MA_ERR_SHAPE;
+        if (t[i].ndim >= 3) return MA_ERR_UNSUPPORTED;
+        if (t[i].role < MA_ROLE_HIDDEN || t[i].role > MA_ROLE_FORCE_ADAMW) return MA_ERR_ARG;
+    }
+    for (int i = 0; i < n; ++i) {
+        int k = MA_ADAMW;
+        if (t[i].ndim == 2 && t[i].role == MA_ROLE_HIDDEN) k = MA_MUON;
+        kind_out[i] = k;
+    }
+    return MA_OK;
+}
+
+int ma_assign_owners(const ma_tensor_t* t, int n, const ma_group_t* groups, int ngroups, int world_size,
+                     int32_t* owner_out) {
+    if (n < 0 || ngroups < 0) return MA_ERR_SHAPE;
+    if (world_size < 1) return MA_ERR_ARG;
+    if (n == 0) return MA_OK;
+    if (!t || !owner_out || !groups) return MA_ERR_NULL;
+    std::vector<int32_t> kind(n);
+    int st = ma_partition(t, n, kind.data());
+    if (st) return st;
+    std::vector<double> cost(n, 0.0);
+    for (int i = 0; i < n; ++i) {
+        if (t[i].group < 0 || t[i].group >= ngroups) return MA_ERR_ARG;
+        double numel = 1.0;
+        for (int d = 0; d < t[i].ndim; ++d) {
+            if (t[i].shape[d] < 0) return MA_ERR_SHAPE;
+            numel *= (double)t[i].shape[d];
+        }
+        if (kind[i] == MA_MUON) {
+            const ma_muon_hparams_t& hp = groups[t[i].group].muon;
+            const int heads = hp.heads < 1 ? 1 : hp.heads;
+            const double Rh = (double)t[i].shape[0] / heads, C = (double)t[i].shape[1];
+            const double m = std::min(Rh, C), nn = std::max(Rh, C);
+            const int steps = hp.ns_steps < 1 ? 1 : hp.ns_steps;
+            cost[i] = heads * steps * (m * (m + 1) * nn + 2 * m * m * nn) + numel;
+        } else {
+            cost[i] = numel;
+        }
+    }
+    for (int pass = 0; pass < 2; ++pass) {
+        const int want = pass == 0 ? MA_MUON : MA_ADAMW;
+        std::vector<int> idx;
+        for (int i = 0; i < n; ++i)
+            if (kind[i] == want) idx.push_back(i);
+        std::stable_sort(idx.begin(), idx.end(), [&](int a, int b) { return cost[a] > cost[b]; });
+        std::vector<double> load(world_size, 0.0);
+        for (int i : idx) {
+            int best = 0;
+            for (int r = 1; r < world_size; ++r)
+                if (load[r] < load[best]) best = r;
+            owner_out[i] = best;
+            load[best] += cost[i];
+        }
+    }
+    return MA_OK;
+}
+
+size_t muon_workspace_bytes(int batch, int64_t R, int64_t C, const ma_muon_hparams_t* hp) {
+    if (check_muon_hp(hp) != MA_OK) return SIZE_MAX;
+    MuonGeom g;
+    if (muon_geom(batch, R, C, *hp, &g) != MA_OK) return SIZE_MAX;
+    return g.total;
+}
+
+int muon_step_batched(int batch, int64_t R, int64_t C, float* const* W, const void* const* G, int gdt,
+                      float* const* M, const ma_muon_hparams_t* hp, void* ws, size_t ws_bytes, void* stream) {
+    MuonGeom g;
+    int st = check_muon_call(batch, R, C, W, G, gdt, M, hp, &g);
+    if (st) return st;
+    if (g.total == 0) return MA_OK;
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < g.total) return MA_ERR_WORKSPACE;
+    int sms = 0;
+    if ((st = device_ok_and_sms(&sms))) return st;
+    int launches = 0;
+    return run_muon(batch, g, W, G, gdt, M, *hp, ws, reinterpret_cast<cudaStream_t>(stream), sms, &launches);
+}
+
+size_t ns_iterate_workspace_bytes(int batch, int64_t m, int64_t n) {
+    if (batch < 0 || m < 0 || n < 0) return SIZE_MAX;
+    const size_t x = align_up((size_t)batch * m * n * 2, kAlign);
+    const size_t gm = align_up((size_t)batch * m * round8(m) * 2, kAlign);
+    return x + 2 * gm;
+}
+
+int ns_iterate_bf16(int batch, int64_t m, int64_t n, const uint16_t* X_in, uint16_t* X_out, const float* coeffs,
+                    int n_coeffs, int steps, void* ws, size_t ws_bytes, void* stream) {
+    if (batch < 0 || m < 0 || n < 0) return MA_ERR_SHAPE;
+    if (steps < 1 || steps > MA_MAX_NS_STEPS || !(n_coeffs == 1 || n_coeffs == steps)) return MA_ERR_ARG;
+    if (!coeffs) return MA_ERR_NULL;
+    for (int k = 0; k < 3 * n_coeffs; ++k)
+        if (!std::isfinite(coeffs[k])) return MA_ERR_ARG;
+    if (batch == 0 || m == 0 || n == 0) return MA_OK;
+    if (!X_in || !X_out) return MA_ERR_NULL;
+    if (m > n) return MA_ERR_SHAPE;
+    if (n % 8 != 0 || !aligned(X_in, 16) || !aligned(X_out, 16)) return MA_ERR_ALIGN;
+    if (batch > 65535 || n > INT_MAX) return MA_ERR_UNSUPPORTED;
+    const size_t need = ns_iterate_workspace_bytes(batch, m, n);
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < need) return MA_ERR_WORKSPACE;
+    int sms = 0;
+    int st = device_ok_and_sms(&sms);
+    if (st) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+    void* T = base;
+    void* Gb = base + align_up((size_t)batch * m * n * 2, kAlign);
+    void* G2 = reinterpret_cast<uint8_t*>(Gb) + align_up((size_t)batch * m * round8(m) * 2, kAlign);
+    NsParams p;
+    std::memset(&p, 0, sizeof(p));
+    p.units = batch;
+    p.m = (int)m;
+    p.n = (int)n;
+    p.ldx = n;
+    p.ldg = round8(m);
+    p.x_unit = m * n;
+    p.g_unit = m * round8(m);
+    p.first = 0;
+    p.heads = 1;
+    p.wait_limit_ns = host_wait_limit_ns();
+    p.status = device_status_ptr();
+    const void* cur = X_in;
+    for (int k = 0; k < steps; ++k) {
+        const float* cf = coeffs + 3 * (n_coeffs == 1 ? 0 : k);
+        p.a = cf[0];
+        p.b = cf[1];
+        p.c = cf[2];
+        const bool quint = cf[2] != 0.f;
+        p.coef_gram = quint ? 1.f : cf[1];
+        p.out = Gb;
+        if (cuda_status(launch_ns_tc(NS_GRAM, p, cur, Gb, sms, s))) return MA_ERR_CUDA;
+        void* Bbuf = Gb;
+        if (quint) {
+            p.xin = Gb;
+            p.out = G2;
+            if (cuda_status(launch_ns_tc(NS_GRAMSQ, p, cur, Gb, sms, s))) return MA_ERR_CUDA;
+            Bbuf = G2;
+        }
+        // the last iteration writes X_out; earlier ones alternate so that no GEMM
+        // reads and writes the same buffer
+        void* dst = ((steps - 1 - k) % 2 == 0) ? static_cast<void*>(X_out) : T;
+        p.xin = cur;
+        p.out = dst;
+        if (cuda_status(launch_ns_tc(NS_APPLY, p, cur, Bbuf, sms, s))) return MA_ERR_CUDA;
+        cur = dst;
+    }
+    return MA_OK;
+}
+
+int adamw_step_fused(int n, float* const* P, const void* const* G, int gdt, float* const* M, float* const* V,
+                     const int64_t* numel, const ma_adamw_hparams_t* hp, void* stream) {
+    if (n < 0) return MA_ERR_SHAPE;
+    int st = check_adamw_hp(hp);
+    if (st) return st;
+    if (gdt != MA_F32 && gdt != MA_BF16) return MA_ERR_DTYPE;
+    if (n == 0) return MA_OK;
+    if (!P || !G || !M || !V || !numel) return MA_ERR_NULL;
+    std::vector<AdamwItem> items;
+    items.reserve(n);
+    for (int i = 0; i < n; ++i) {
+        if (numel[i] < 0) return MA_ERR_SHAPE;
+        if (numel[i] == 0) continue;
+        if (!P[i] || !G[i] || !M[i] || !V[i]) return MA_ERR_NULL;
+        if (!aligned(P[i], 4) || !aligned(M[i], 4) || !aligned(V[i], 4) || !aligned(G[i], gdt == MA_BF16 ? 2 : 4))
+            return MA_ERR_ALIGN;
+        items.push_back({P[i], G[i], M[i], V[i], numel[i], 0});
+    }
+    if (items.empty()) return MA_OK;
+    if ((st = device_ok_and_sms(nullptr))) return st;
+    AdamwGroupConst c = adamw_const(*hp);
+    int launches = 0;
+    return run_adamw(items, gdt, &c, 1, reinterpret_cast<cudaStream_t>(stream), &launches);
+}
+
+int ma_plan_create(const ma_tensor_t* t, int n, const ma_group_t* groups, int ngroups, ma_plan_t** out,
+                   size_t* ws_bytes) {
+    if (!out || !ws_bytes) return MA_ERR_NULL;
+    *out = nullptr;
+    if (n < 0 || ngroups < 0) return MA_ERR_SHAPE;
+    if (ngroups > MA_MAX_GROUPS) return MA_ERR_UNSUPPORTED;
+    if ((n > 0 && !t) || (ngroups > 0 && !groups)) return MA_ERR_NULL;
+    const size_t cap = *ws_bytes;
+    std::vector<int32_t> kind(n);
+    int st = ma_partition(t, n, kind.data());
+    if (st) return st;
+    for (int k = 0; k < ngroups; ++k) {
+        if (groups[k].kind == MA_MUON) {
+            if ((st = check_muon_hp(&groups[k].muon))) return st;
+        } else if (groups[k].kind == MA_ADAMW) {
+            if ((st = check_adamw_hp(&groups[k].adamw))) return st;
+        } else {
+            return MA_ERR_ARG;
+        }
+    }
+    ma_plan* plan = new (std::nothrow) ma_plan();
+    if (!plan) return MA_ERR_UNSUPPORTED;
+    plan->t.assign(t, t + n);
+    plan->kind = kind;
+    for (int k = 0; k < ngroups; ++k) plan->group_kind.push_back(groups[k].kind);
+    auto fail = [&](int code) {
+        delete plan;
+        return code;
+    };
+    for (int i = 0; i < n; ++i) {
+        const ma_tensor_t& x = t[i];
+        if (x.group < 0 || x.group >= ngroups) return fail(MA_ERR_ARG);
+        if (groups[x.group].kind != kind[i]) return fail(MA_ERR_ARG);
+        if (x.grad_dtype != MA_F32 && x.grad_dtype != MA_BF16) return fail(MA_ERR_DTYPE);
+        int64_t numel = 1;
+        for (int d = 0; d < x.ndim; ++d) {
+            if (x.shape[d] < 0) return fail(MA_ERR_SHAPE);
+            numel *= x.shape[d];
+        }
+        if (numel == 0) continue;
+        if (!x.param || !x.grad || !x.state0) return fail(MA_ERR_NULL);
+        if (kind[i] == MA_ADAMW) {
+            if (!x.state1) return fail(MA_ERR_NULL);
+            if (!aligned(x.param, 4) || !aligned(x.state0, 4) || !aligned(x.state1, 4) ||
+                !aligned(x.grad, x.grad_dtype == MA_BF16 ? 2 : 4))
+                return fail(MA_ERR_ALIGN);
+            plan->adamw_idx.push_back(i);
+        } else {
+            if (!aligned(x.param, 16) || !aligned(x.state0, 16) || !aligned(x.grad, 16)) return fail(MA_ERR_ALIGN);
+            if (x.shape[1] % 8 != 0) return fail(MA_ERR_ALIGN);
+            const ma_muon_hparams_t& hp = groups[x.group].muon;
+            if (x.shape[0] % hp.heads != 0) return fail(MA_ERR_SHAPE);
+            bool found = false;
+            for (auto& b : plan->buckets) {
+                if (b.group == x.group && b.R == x.shape[0] && b.C == x.shape[1]) {
+                    // one gradient dtype per bucket: a different dtype starts a new bucket
+                    if (t[b.members[0]].grad_dtype != x.grad_dtype) continue;
+                    b.members.push_back(i);
+                    found = true;
+                    break;
+                }
+            }
+            if (!found) plan->buckets.push_back({x.group, x.shape[0], x.shape[1], {i}, 0});
+        }
+    }
+    size_t need = 0;
+    for (auto& b : plan->buckets) {
+        const ma_muon_hparams_t& hp = groups[b.group].muon;
+        const int nb = (int)b.members.size();
+        int sub = std::min(nb, (int)MA_MAX_BATCH);
+        MuonGeom g;
+        if ((st = muon_geom(sub, b.R, b.C, hp, &g))) return fail(st);
+        while (cap > 0 && g.total > cap && sub > 1) {
+            sub = std::max(1, sub / 2);
+            muon_geom(sub, b.R, b.C, hp, &g);
+        }
+        if (cap > 0 && g.total > cap) return fail(MA_ERR_WORKSPACE);
+        if (g.units > 65535 || g.m > INT_MAX || g.n > INT_MAX || g.parts > INT_MAX) return fail(MA_ERR_UNSUPPORTED);
+        b.sub = sub;
+        need = std::max(need, g.total);
+    }
+    plan->ws_bytes = need;
+    *ws_bytes = need;
+    *out = plan;
+    return MA_OK;
+}
+
+int muonadamw_step(ma_plan_t* plan, const ma_group_t* groups, void* ws, size_t ws_bytes, void* stream) {
+    if (!plan) return MA_ERR_NULL;
+    const int ngroups = (int)plan->group_kind.size();
+    if (ngroups > 0 && !groups) return MA_ERR_NULL;
+    int st;
+    for (int k = 0; k < ngroups; ++k) {
+        if (groups[k].kind != plan->group_kind[k]) return MA_ERR_ARG;
+        if (groups[k].kind == MA_MUON) {
+            if ((st = check_muon_hp(&groups[k].muon))) return st;
+        } else if ((st = check_adamw_hp(&groups[k].adamw))) {
+            return st;
+        }
+    }
+    // the plan's bucket geometry depends on heads, steps, precision and c != 0
+    for (auto& b : plan->buckets) {
+        MuonGeom g;
+        if ((st = muon_geom(b.sub, b.R, b.C, groups[b.group].muon, &g))) return st;
+        if (g.total > plan->ws_bytes) return MA_ERR_ARG;
+    }
+    if (plan->ws_bytes > 0 && (!ws || !aligned(ws, kAlign) || ws_bytes < plan->ws_bytes)) return MA_ERR_WORKSPACE;
+    int sms = 0;
+    if (!plan->adamw_idx.empty() || !plan->buckets.empty()) {
+        if ((st = device_ok_and_sms(&sms))) return st;
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    int launches = 0;
+    if (!plan->adamw_idx.empty()) {
+        AdamwGroupConst gc[MA_MAX_GROUPS];
+        std::memset(gc, 0, sizeof(gc));
+        for (int k = 0; k < ngroups; ++k)
+            if (groups[k].kind == MA_ADAMW) gc[k] = adamw_const(groups[k].adamw);
+        for (int dt = 0; dt < 2; ++dt) {
+            std::vector<AdamwItem> items;
+            for (int i : plan->adamw_idx) {
+                const ma_tensor_t& x = plan->t[i];
+                if (x.grad_dtype != dt) continue;
+                int64_t numel = 1;
+                for (int d = 0; d < x.ndim; ++d) numel *= x.shape[d];
+                items.push_back({x.param, x.grad, x.state0, x.state1, numel, x.group});
+            }
+            if (!items.empty() && (st = run_adamw(items, dt, gc, ngroups, s, &launches))) return st;
+        }
+    }
+    for (auto& b : plan->buckets) {
+        const ma_muon_hparams_t& hp = groups[b.group].muon;
+        const int nb = (int)b.members.size();
+        const int gdt = plan->t[b.members[0]].grad_dtype;
+        for (int s0 = 0; s0 < nb; s0 += b.sub) {
+            const int cnt = std::min(b.sub, nb - s0);
+            float* W[MA_MAX_BATCH];
+            const void* G[MA_MAX_BATCH];
+            float* M[MA_MAX_BATCH];
+            for (int k = 0; k < cnt; ++k) {
+                const ma_tensor_t& x = plan->t[b.members[s0 + k]];
+                W[k] = x.param;
+                G[k] = x.grad;
+                M[k] = x.state0;
+            }
+            MuonGeom g;
+            muon_geom(cnt, b.R, b.C, hp, &g);
+            if ((st = run_muon(cnt, g, W, G, gdt, M, hp, ws, s, sms, &launches))) return st;
+        }
+    }
+    plan->last_launches = launches;
+    return MA_OK;
+}
+
+int ma_plan_last_launches(const ma_plan_t* plan) { return plan ? plan->last_launches : 0; }
+
+void ma_plan_destroy(ma_plan_t* plan) { delete plan; }
+
+int ma_device_status(void* stream, int reset) {
+    if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MA_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return MA_ERR_CUDA;
+    if (reset) {
+        const int z = 0;
+        if (cudaMemcpyToSymbol(g_status, &z, sizeof(int)) != cudaSuccess) return MA_ERR_CUDA;
+    }
+    return v;
+}
+
+int ma_set_wait_limit_ns(int64_t limit_ns) {
+    if (limit_ns <= 0) return MA_ERR_ARG;
+    g_host_wait_limit_ns = limit_ns;
+    return MA_OK;
+}
+
+int ma_selftest_wait_timeout(int64_t limit_ns, void* stream) {
+    if (limit_ns <= 0 || limit_ns > 10000000000LL) return MA_ERR_ARG;
+    int st = device_ok_and_sms(nullptr);
+    if (st) return st;
+    int* status = device_status_ptr();
+    if (!status) return MA_ERR_CUDA;
+    return launch_wait_selftest(limit_ns, status, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MA_OK
+               : MA_ERR_CUDA;
+}
+
+}  // extern "C"

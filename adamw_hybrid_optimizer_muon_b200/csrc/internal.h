@@ -1,0 +1,113 @@
+// Launch descriptors shared between the host entry points (api.cu) and the
+// kernel files. Every table a kernel needs travels in its parameter block
+// (up to 32 KB on sm_70+ with CUDA >= 12.1), so no call allocates device
+// memory and every launch can be replayed from a CUDA graph as captured.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/muonadamw.h"
+
+namespace ma {
+
+// ------------------------------------------------------------------ AdamW
+
+constexpr int kAdamwChunk = 8192;              // elements per block
+constexpr int kAdamwMaxTensorsPerLaunch = 320;  // parameter-block capacity
+
+struct AdamwTensorDesc {
+    float* p;
+    const void* g;
+    float* m;
+    float* v;
+    int64_t numel;
+    int64_t chunk0;  // first global chunk index of this tensor
+    int32_t group;
+    int32_t vec;     // 1 when p, m, v are 16-byte aligned and g is aligned for 4-wide loads
+};
+
+struct AdamwGroupConst {
+    float decay;         // 1 - lr * wd
+    float step_size;     // lr / (1 - beta1^t)
+    float inv_sqrt_bc2;  // 1 / sqrt(1 - beta2^t)
+    float beta1, beta2, omb1, omb2, eps;
+};
+
+struct AdamwLaunch {
+    int32_t ntensors;
+    int32_t gdt;  // ma_dtype_t of every gradient in this launch
+    int64_t nchunks;
+    AdamwGroupConst grp[MA_MAX_GROUPS];
+    AdamwTensorDesc t[kAdamwMaxTensorsPerLaunch];
+};
+
+cudaError_t launch_adamw(const AdamwLaunch& L, cudaStream_t s);
+
+// ------------------------------------------------------------------ Muon: momentum + norm
+
+constexpr int kPrepChunk = 8192;  // elements per block, flat path
+constexpr int kPrepTile = 64;     // tile edge, transposing path
+
+struct MuonPrepLaunch {
+    int32_t batch, heads, transposed, gdt, nesterov, x_f32;
+    int64_t C, Rh;        // matrix columns, rows per head slice
+    int64_t ldx;          // row stride (elements) of the NS operand X
+    int64_t x_unit;       // elements between consecutive units of X
+    int64_t parts;        // partial sums per unit
+    int64_t tiles_c;      // transposing path: tiles along C
+    float beta, omb;
+    void* X;
+    double* partials;
+    const void* G[MA_MAX_BATCH];
+    float* M[MA_MAX_BATCH];
+};
+
+// Number of per-block partial sums the momentum pass writes for one unit.
+int64_t prep_parts_per_unit(int64_t Rh, int64_t C, int transposed);
+
+cudaError_t launch_muon_prep(const MuonPrepLaunch& L, cudaStream_t s);
+// scale[u] = 1 / (sqrt(sum of the unit's partials) + eps), deterministic order.
+cudaError_t launch_norm_finalize(const double* partials, int64_t parts, int units, float eps, float* scale,
+                                 cudaStream_t s);
+
+// ------------------------------------------------------------------ Newton-Schulz
+
+enum NsMode { NS_GRAM = 0, NS_APPLY = 1, NS_FINAL = 2, NS_GRAMSQ = 3 };
+
+struct NsParams {
+    int32_t units, m, n;
+    int64_t ldx, ldg;        // row strides (elements) of X and of the Gram
+    int64_t x_unit, g_unit;  // elements between consecutive units
+    int32_t first;           // 1: fold the per-unit normalisation scale in
+    float a, b, c;           // this iteration's polynomial coefficients
+    float coef_gram;         // GRAM epilogue multiplier (b, or 1 when c != 0)
+    const float* scale;      // per-unit 1 / (||u|| + eps); may be NULL when first == 0
+    const void* xin;         // APPLY/FINAL: X of this iteration; GRAMSQ: the Gram input
+    void* out;               // GRAM/GRAMSQ: Gram output; APPLY: next X
+    // FINAL: W <- W * decay - lr_s * X_N, written through W[] in the original orientation
+    int32_t transposed, heads;
+    int64_t Rh, C;
+    float decay, lr_s;
+    long long wait_limit_ns;
+    int* status;             // per-device status word
+    float* W[MA_MAX_BATCH];
+};
+
+// bf16 tcgen05 path: X, Gram buffers are bf16 with 16-byte-multiple strides.
+size_t ns_tc_smem_bytes();
+cudaError_t launch_ns_tc(int mode, const NsParams& p, const void* x_buf, const void* g_buf, int num_sms,
+                         cudaStream_t s);
+
+// fp32 SIMT path (precision mode 1).
+cudaError_t launch_ns_simt(int mode, const NsParams& p, const void* x_buf, const void* g_buf, cudaStream_t s);
+
+// ------------------------------------------------------------------ misc
+
+cudaError_t launch_wait_selftest(long long limit_ns, int* status, cudaStream_t s);
+long long host_wait_limit_ns();
+int* device_status_ptr();  // address of this device's status word, NULL on failure
+
+}  // namespace ma

@@ -1,0 +1,473 @@
+// Newton-Schulz GEMMs on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// One iteration of the odd polynomial ("MuonClip Optimizer",
+// "Newton-Schulz Orthogonalization": X <- 1.5 X - 0.5 X (X^T X); in general
+// X <- aX + b X(X^T X) + c X(X^T X)^2) runs on the short side of X, which is
+// the same thing because X (X^T X) = (X X^T) X:
+//
+//   GRAM    A = X X^T             (m x m, symmetric; only tiles touching the
+//                                  upper triangle are computed, and each one
+//                                  writes its elements and their mirror)
+//           epilogue: B = coef * A, coef = b * s^2 on the first iteration
+//           (s = 1/(||u||_F + eps), the Frobenius normalisation), else b.
+//   GRAMSQ  (only when c != 0) B = b*A + c*A*A, with A*A = A A^T by symmetry
+//   APPLY   X' = s * (a X + B X)  (s only on the first iteration)
+//   FINAL   the last APPLY. Its epilogue does the decoupled decay and the
+//           update, W <- W*(1 - lr*wd) - lr*scale*X_N, straight into the
+//           caller's fp32 weights, transposing back when the unit was tall.
+//           X_N is never rounded or stored.
+//
+// Kernel structure (one CTA per SM, persistent over the tiles of all units of
+// a batch):
+//   warp 0      TMA producer: 128B-swizzled 3-D bulk tensor loads into a
+//               4-stage ring (A tile 128x64, B tile 256x64 bf16 = 48 KB per stage)
+//   warp 1      TMEM allocator and MMA issuer: tcgen05.mma kind::f16, M=128,
+//               N=256, K=16 per instruction, fp32 accumulators in TMEM, two
+//               accumulator buffers (2 x 256 columns) so the epilogue of one
+//               tile overlaps the main loop of the next
+//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, fused polynomial
+//               combine, bf16 rounding, stores
+// Every mbarrier wait is bounded (see common.cuh). On a timeout the block
+// records MA_ERR_TIMEOUT, lets in-flight copies and MMAs drain (also bounded),
+// frees its TMEM and returns.
+//
+// B operand major-ness: for GRAM and GRAMSQ both operands are K-major rows of
+// the same matrix. For APPLY the B operand is X itself, read MN-major (the
+// contraction runs over X's rows), so no transposed copy is ever made.
+#include "common.cuh"
+#include "internal.h"
+
+namespace ma {
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr uint32_t A_BYTES = BM * BK * 2;             // 16 KB
+constexpr uint32_t B_BYTES = BN * BK * 2;             // 32 KB
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;   // 48 KB
+constexpr uint32_t TMEM_COLS = 2 * BN;                // two fp32 accumulators
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+
+struct TileCoord {
+    int u, ti, tj;
+};
+
+// Tiles of one unit. GRAM/GRAMSQ: only (ti, tj) whose 128x256 block holds an
+// element with row <= col, i.e. ti <= 2*tj + 1, enumerated column by column.
+__device__ __forceinline__ TileCoord decode_tile(int mode, int t, int tiles_per_unit, int mt, int nt) {
+    TileCoord c;
+    c.u = t / tiles_per_unit;
+    int r = t - c.u * tiles_per_unit;
+    if (mode == NS_GRAM || mode == NS_GRAMSQ) {
+        int tj = 0;
+        for (;; ++tj) {
+            const int cnt = min(2 * tj + 2, mt);
+            if (r < cnt || tj == nt - 1) break;
+            r -= cnt;
+        }
+        c.ti = r;
+        c.tj = tj;
+    } else {
+        c.ti = r / nt;
+        c.tj = r - c.ti * nt;
+    }
+    return c;
+}
+
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32], float mul) {
+    uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        uint4 w;
+        w.x = pack_bf16x2(v[8 * q + 0] * mul, v[8 * q + 1] * mul);
+        w.y = pack_bf16x2(v[8 * q + 2] * mul, v[8 * q + 3] * mul);
+        w.z = pack_bf16x2(v[8 * q + 4] * mul, v[8 * q + 5] * mul);
+        w.w = pack_bf16x2(v[8 * q + 6] * mul, v[8 * q + 7] * mul);
+        d[q] = w;
+    }
+}
+
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&x)[32]) {
+    const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const uint4 w = s[q];
+        x[8 * q + 0] = bf16_lo(w.x); x[8 * q + 1] = bf16_hi(w.x);
+        x[8 * q + 2] = bf16_lo(w.y); x[8 * q + 3] = bf16_hi(w.y);
+        x[8 * q + 4] = bf16_lo(w.z); x[8 * q + 5] = bf16_hi(w.z);
+        x[8 * q + 6] = bf16_lo(w.w); x[8 * q + 7] = bf16_hi(w.w);
+    }
+}
+
+template <int MODE>
+__device__ __forceinline__ void epilogue_chunk(const NsParams& p, const TileCoord& tc, int row, int col0,
+                                               const float (&v)[32]) {
+    const int m = p.m, n = p.n;
+    if (MODE == NS_GRAM || MODE == NS_GRAMSQ) {
+        if (row >= m) return;
+        float coef = p.coef_gram;
+        if (MODE == NS_GRAM && p.first) {
+            const float s = p.scale[tc.u];
+            coef *= s * s;
+        }
+        __nv_bfloat16* G = reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)tc.u * p.g_unit;
+        const __nv_bfloat16* Gin =
+            MODE == NS_GRAMSQ ? reinterpret_cast<const __nv_bfloat16*>(p.xin) + (int64_t)tc.u * p.g_unit : nullptr;
+        float o[32];
+        if (MODE == NS_GRAMSQ) {
+            // B = b*A + c*A^2, with acc = A^2 and A read back from the Gram buffer
+            float a_in[32];
+            if (col0 + 32 <= m) {
+                load_bf16x32(Gin + (int64_t)row * p.ldg + col0, a_in);
+            } else {
+#pragma unroll
+                for (int t = 0; t < 32; ++t)
+                    a_in[t] = (col0 + t < m) ? __bfloat162float(Gin[(int64_t)row * p.ldg + col0 + t]) : 0.f;
+            }
+#pragma unroll
+            for (int t = 0; t < 32; ++t) o[t] = p.b * a_in[t] + p.c * v[t];
+            coef = 1.f;
+        } else {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) o[t] = v[t];
+        }
+        if (col0 >= row && col0 + 32 <= m) {
+            store_bf16x32(G + (int64_t)row * p.ldg + col0, o, coef);
+        } else {
+#pragma unroll
+            for (int t = 0; t < 32; ++t) {
+                const int j = col0 + t;
+                if (j >= row && j < m) G[(int64_t)row * p.ldg + j] = __float2bfloat16_rn(o[t] * coef);
+            }
+        }
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            const int j = col0 + t;
+            if (j > row && j < m) G[(int64_t)j * p.ldg + row] = __float2bfloat16_rn(o[t] * coef);
+        }
+    } else {
+        if (row >= m) return;
+        const float sa = p.first ? p.scale[tc.u] : 1.f;
+        const __nv_bfloat16* Xin = reinterpret_cast<const __nv_bfloat16*>(p.xin) + (int64_t)tc.u * p.x_unit;
+        float x[32];
+        const bool full = col0 + 32 <= n;
+        if (full) {
+            load_bf16x32(Xin + (int64_t)row * p.ldx + col0, x);
+        } else {
+#pragma unroll
+            for (int t = 0; t < 32; ++t)
+                x[t] = (col0 + t < n) ? __bfloat162float(Xin[(int64_t)row * p.ldx + col0 + t]) : 0.f;
+        }
+        float o[32];
+#pragma unroll
+        for (int t = 0; t < 32; ++t) o[t] = sa * (p.a * x[t] + v[t]);
+        if (MODE == NS_APPLY) {
+            __nv_bfloat16* Xo = reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)tc.u * p.x_unit;
+            if (full) {
+                store_bf16x32(Xo + (int64_t)row * p.ldx + col0, o, 1.f);
+            } else {
+#pragma unroll
+                for (int t = 0; t < 32; ++t)
+                    if (col0 + t < n) Xo[(int64_t)row * p.ldx + col0 + t] = __float2bfloat16_rn(o[t]);
+            }
+        } else {  // NS_FINAL
+            const int bidx = tc.u / p.heads, h = tc.u - bidx * p.heads;
+            float* Wb = p.W[bidx] + (int64_t)h * p.Rh * p.C;
+            const float decay = p.decay, lrs = p.lr_s;
+            if (!p.transposed) {
+                float* w = Wb + (int64_t)row * p.C + col0;
+                if (full && (p.C & 3) == 0) {
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        float4 wv = reinterpret_cast<float4*>(w)[q];
+                        wv.x = wv.x * decay - lrs * o[4 * q + 0];
+                        wv.y = wv.y * decay - lrs * o[4 * q + 1];
+                        wv.z = wv.z * decay - lrs * o[4 * q + 2];
+                        wv.w = wv.w * decay - lrs * o[4 * q + 3];
+                        reinterpret_cast<float4*>(w)[q] = wv;
+                    }
+                } else {
+#pragma unroll
+                    for (int t = 0; t < 32; ++t)
+                        if (col0 + t < n) w[t] = w[t] * decay - lrs * o[t];
+                }
+            } else {
+                // X_N[row][j] is W[j][row]: lanes hold consecutive rows, so each
+                // column j is one coalesced 128-byte access across the warp.
+#pragma unroll
+                for (int t = 0; t < 32; ++t) {
+                    const int j = col0 + t;
+                    if (j < n) {
+                        float* w = Wb + (int64_t)j * p.C + row;
+                        *w = *w * decay - lrs * o[t];
+                    }
+                }
+            }
+        }
+    }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(192, 1)
+    ns_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
+                 const __grid_constant__ NsParams p, int tiles_per_unit, int mt, int nt, int kblocks) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* acc_full = empty + STAGES;
+    uint64_t* acc_empty = acc_full + 2;
+    uint64_t* drain = acc_empty + 2;
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    int* counters = const_cast<int*>(abort_flag) + 1;  // [0] loads issued, [1] loads consumed
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int total_tiles = p.units * tiles_per_unit;
+    const long long limit = p.wait_limit_ns;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        for (int a = 0; a < 2; ++a) {
+            mbar_init(&acc_full[a], 1);
+            mbar_init(&acc_empty[a], 4);
+        }
+        mbar_init(drain, 1);
+        *abort_flag = 0;
+        counters[0] = 0;
+        counters[1] = 0;
+        fence_barrier_init();
+        prefetch_tensormap(&mapA);
+        prefetch_tensormap(&mapB);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_holder, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_holder;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+                const TileCoord tc = decode_tile(MODE, t, tiles_per_unit, mt, nt);
+                bool ok = true;
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    uint8_t* sa = smem + stage * STAGE_BYTES;
+                    uint8_t* sb = sa + A_BYTES;
+                    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
+                    tma_load_3d(sa, &mapA, &full[stage], kb * BK, tc.ti * BM, tc.u);
+                    if (MODE == NS_GRAM || MODE == NS_GRAMSQ) {
+                        tma_load_3d(sb, &mapB, &full[stage], kb * BK, tc.tj * BN, tc.u);
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < BN / 64; ++q)
+                            tma_load_3d(sb + q * (64 * BK * 2), &mapB, &full[stage], tc.tj * BN + q * 64, kb * BK,
+                                        tc.u);
+                    }
+                    ++issued;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+            }
+            counters[0] = issued;
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, (MODE == NS_APPLY || MODE == NS_FINAL) ? 1 : 0);
+            int stage = 0;
+            uint32_t phase = 0;
+            int consumed = 0;
+            int lt = 0;
+            bool ok = true;
+            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++lt) {
+                const int acc = lt & 1;
+                const uint32_t use = (uint32_t)(lt >> 1);
+                if (!mbar_wait_bounded(&acc_empty[acc], (use & 1u) ^ 1u, abort_flag, limit, p.status)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                for (int kb = 0; kb < kblocks; ++kb) {
+                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, limit, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a0 = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint32_t b0 = a0 + A_BYTES;
+#pragma unroll
+                    for (int kk = 0; kk < BK / 16; ++kk) {
+                        const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
+                        uint64_t bdesc;
+                        if (MODE == NS_APPLY || MODE == NS_FINAL)
+                            bdesc = smem_desc_sw128(b0 + kk * (16 * 128), 64 * BK * 2, 1024);
+                        else
+                            bdesc = smem_desc_sw128(b0 + kk * 32, 16, 1024);
+                        tc_mma_f16(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                    }
+                    tc_commit(&empty[stage]);
+                    ++consumed;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit(&acc_full[acc]);
+            }
+            counters[1] = consumed;
+            if (!ok) {
+                // let every MMA issued so far finish before TMEM is released
+                tc_commit(drain);
+                mbar_wait_bounded(drain, 0, abort_flag, limit, p.status);
+            }
+        }
+    } else {
+        const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad + 32)
+        int lt = 0;
+        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++lt) {
+            const TileCoord tc = decode_tile(MODE, t, tiles_per_unit, mt, nt);
+            const int acc = lt & 1;
+            const uint32_t use = (uint32_t)(lt >> 1);
+            int ok = 1;
+            if (lane == 0) ok = mbar_wait_bounded(&acc_full[acc], use & 1u, abort_flag, limit, p.status) ? 1 : 0;
+            ok = __shfl_sync(0xffffffffu, ok, 0);
+            if (!ok) break;
+            tc_fence_after();
+            const int row = tc.ti * BM + quad * 32 + lane;
+            const int row_lo = tc.ti * BM + quad * 32;
+            const int limit_cols = (MODE == NS_APPLY || MODE == NS_FINAL) ? p.n : p.m;
+#pragma unroll 1
+            for (int cc = 0; cc < BN / 32; ++cc) {
+                const int col0 = tc.tj * BN + cc * 32;
+                if (col0 >= limit_cols) break;                                            // warp-uniform
+                if ((MODE == NS_GRAM || MODE == NS_GRAMSQ) && col0 + 31 < row_lo) continue;  // below diagonal
+                float v[32];
+                tmem_ld32(tmem_base + (uint32_t)(acc * BN + cc * 32) + ((uint32_t)(quad * 32) << 16), v);
+                epilogue_chunk<MODE>(p, tc, row, col0, v);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        }
+    }
+
+    __syncthreads();
+    if (threadIdx.x == 0 && *abort_flag) {
+        // loads that were issued but never consumed must land before the block exits
+        for (int k = counters[1]; k < counters[0]; ++k)
+            mbar_wait_bounded(&full[k % STAGES], (uint32_t)((k / STAGES) & 1), abort_flag, limit, p.status);
+    }
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, TMEM_COLS);
+    }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(ptr);
+    }
+    return fn;
+}
+
+// 3-D bf16 map over [units][rows][inner] with row stride `ld` and unit stride
+// `unit` (elements), 128-byte swizzle, zero fill out of bounds.
+bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t units, uint64_t ld,
+              uint64_t unit, uint32_t box_inner, uint32_t box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {inner, rows, units};
+    cuuint64_t strides[2] = {ld * 2, unit * 2};
+    cuuint32_t box[3] = {box_inner, box_rows, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MODE>
+cudaError_t launch_mode(const NsParams& p, const void* x_buf, const void* g_buf, int num_sms, cudaStream_t s) {
+    CUtensorMap mA, mB;
+    int kblocks, mt, nt, tiles;
+    mt = (p.m + BM - 1) / BM;
+    if (MODE == NS_GRAM || MODE == NS_GRAMSQ) {
+        nt = (p.m + BN - 1) / BN;
+        tiles = 0;
+        for (int tj = 0; tj < nt; ++tj) tiles += (2 * tj + 2 < mt) ? 2 * tj + 2 : mt;
+        if (MODE == NS_GRAM) {
+            kblocks = (p.n + BK - 1) / BK;
+            if (!make_map(&mA, x_buf, p.n, p.m, p.units, p.ldx, p.x_unit, BK, BM)) return cudaErrorInvalidValue;
+            if (!make_map(&mB, x_buf, p.n, p.m, p.units, p.ldx, p.x_unit, BK, BN)) return cudaErrorInvalidValue;
+        } else {
+            kblocks = (p.m + BK - 1) / BK;
+            if (!make_map(&mA, p.xin, p.m, p.m, p.units, p.ldg, p.g_unit, BK, BM)) return cudaErrorInvalidValue;
+            if (!make_map(&mB, p.xin, p.m, p.m, p.units, p.ldg, p.g_unit, BK, BN)) return cudaErrorInvalidValue;
+        }
+    } else {
+        nt = (p.n + BN - 1) / BN;
+        tiles = mt * nt;
+        kblocks = (p.m + BK - 1) / BK;
+        if (!make_map(&mA, g_buf, p.m, p.m, p.units, p.ldg, p.g_unit, BK, BM)) return cudaErrorInvalidValue;
+        if (!make_map(&mB, x_buf, p.n, p.m, p.units, p.ldx, p.x_unit, 64, BK)) return cudaErrorInvalidValue;
+    }
+    const long long total = (long long)tiles * p.units;
+    if (total <= 0) return cudaSuccess;
+    const int grid = (int)(total < num_sms ? total : num_sms);
+    static unsigned long long attr_set = 0;  // one bit per device
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!(attr_set & (1ull << dev))) {
+        e = cudaFuncSetAttribute(ns_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+        attr_set |= 1ull << dev;
+    }
+    ns_tc_kernel<MODE><<<grid, 192, SMEM_BYTES, s>>>(mA, mB, p, tiles, mt, nt, kblocks);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t ns_tc_smem_bytes() { return SMEM_BYTES; }
+
+cudaError_t launch_ns_tc(int mode, const NsParams& p, const void* x_buf, const void* g_buf, int num_sms,
+                         cudaStream_t s) {
+    switch (mode) {
+        case NS_GRAM: return launch_mode<NS_GRAM>(p, x_buf, g_buf, num_sms, s);
+        case NS_GRAMSQ: return launch_mode<NS_GRAMSQ>(p, x_buf, g_buf, num_sms, s);
+        case NS_APPLY: return launch_mode<NS_APPLY>(p, x_buf, g_buf, num_sms, s);
+        case NS_FINAL: return launch_mode<NS_FINAL>(p, x_buf, g_buf, num_sms, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace ma

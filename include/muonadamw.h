@@ -1,0 +1,241 @@
+/*
+ * muonadamw.h - C ABI of the B200 (sm_100a) MuonAdamW optimizer-step library.
+ *
+ * The library updates optimizer state and parameters in place, on the GPU.
+ * Every argument is a plain pointer or size. A pointer marked "device" must
+ * point into memory that the calling context's current CUDA device can read
+ * and write. "host" pointers are read by the CPU during the call and are not
+ * kept afterwards. Streams are passed as `void*` holding a `cudaStream_t`
+ * (NULL = the legacy default stream).
+ *
+ * Ownership: the caller owns every tensor, optimizer-state buffer, workspace
+ * and stream. A plan (ma_plan_t) owns only host metadata.
+ *
+ * Errors: every entry point validates all of its arguments before it launches
+ * anything, so a call that returns an error has changed nothing. Launches are
+ * asynchronous on the given stream and the host never blocks. A kernel that
+ * hits an internal time limit (a bounded wait that ran out) records
+ * MA_ERR_TIMEOUT in a per-device status word, which ma_device_status() reads.
+ * No entry point ever falls back to the CPU.
+ *
+ * Method sources (cited by page title and section):
+ *  [P1] "How nanochat Combines Muon and AdamW in a Single Optimizer":
+ *       "Parameter Grouping Strategy", "The MuonAdamW Class Architecture",
+ *       "AdamW Step Implementation", "Muon Step Implementation".
+ *  [P2] "Qwen Training Details: Full-Network Muon Optimizer and Residual
+ *       Stream Design", "Confirmed".
+ *  [P3] "nemo_automodel.components.optim.muown_triton", API of _prepare,
+ *       _finish and _supported.
+ *  [P4] "Guidelines for whether to use muon for parameters" (Muon issue 31).
+ *  [P5] "MuonClip Optimizer": "Newton-Schulz Orthogonalization", "Momentum",
+ *       "Design Decisions".
+ */
+#ifndef MUONADAMW_H
+#define MUONADAMW_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MA_VERSION 1
+
+typedef enum {
+    MA_OK = 0,
+    MA_ERR_NULL = 1,        /* a required pointer is NULL                        */
+    MA_ERR_SHAPE = 2,       /* a size or shape is negative or inconsistent        */
+    MA_ERR_DTYPE = 3,       /* unknown dtype code                                 */
+    MA_ERR_ALIGN = 4,       /* a pointer or row length breaks an alignment rule   */
+    MA_ERR_WORKSPACE = 5,   /* workspace NULL, too small or misaligned            */
+    MA_ERR_UNSUPPORTED = 6, /* a valid request this build does not implement      */
+    MA_ERR_CUDA = 7,        /* a CUDA runtime call failed                         */
+    MA_ERR_TIMEOUT = 8,     /* a device-side bounded wait ran out (status word)   */
+    MA_ERR_ARG = 9          /* a hyperparameter is out of its domain              */
+} ma_status_t;
+
+typedef enum { MA_F32 = 0, MA_BF16 = 1 } ma_dtype_t;
+typedef enum { MA_MUON = 0, MA_ADAMW = 1 } ma_kind_t;
+
+/* Role of a tensor in the model. Muon is meant for hidden matrices whose input
+ * and output are RMS-normed [P4]. Embedding and unembedding (head) matrices are
+ * 2-D but belong with AdamW [P1 "AdamW Step Implementation"; P4]. Some
+ * projections are forced onto AdamW for stability [P2]. */
+typedef enum {
+    MA_ROLE_HIDDEN = 0,
+    MA_ROLE_EMBED = 1,
+    MA_ROLE_UNEMBED = 2,
+    MA_ROLE_FORCE_ADAMW = 3
+} ma_role_t;
+
+#define MA_MAX_NS_STEPS 16      /* Newton-Schulz iterations per step             */
+#define MA_MAX_GROUPS 32        /* parameter groups per plan                     */
+#define MA_MAX_BATCH 256        /* matrices per muon_step_batched call           */
+
+/* Muon hyperparameters [P1 "Muon Step Implementation"; P5].
+ *  lr, weight_decay: W <- W*(1 - lr*weight_decay) - lr*s*O (decoupled decay).
+ *  beta: EMA momentum m <- beta*m + (1-beta)*g (0.95 default [P5 "Momentum"]).
+ *  nesterov: direction u = beta*m + (1-beta)*g when nonzero, else u = m.
+ *  eps: X0 = u / (||u||_F + eps).
+ *  ns_steps: Newton-Schulz iterations, 1..MA_MAX_NS_STEPS (5 [P5]).
+ *  coeffs: polynomial X <- aX + b(XX^T)X + c(XX^T)^2 X per iteration; with
+ *      n_coeffs == 1 row 0 is used for every iteration, otherwise n_coeffs must
+ *      equal ns_steps. The cubic of [P5] is (1.5, -0.5, 0).
+ *  scale_mode: 0: s = sqrt(max(1, R/C)); 1: s = sqrt(R/C); 2: s = 1, with R x C
+ *      the global shape of the matrix (or head slice) [P3 _finish].
+ *  heads: rows split into `heads` equal slices, each orthogonalised on its own
+ *      [P2 per-head orthogonalisation]; 1 = the whole matrix.
+ *  precision: 0 = bf16 tensor-core operands with fp32 accumulation;
+ *      1 = fp32 arithmetic throughout (a correctness mode). */
+typedef struct {
+    float lr, beta, weight_decay, eps;
+    int32_t nesterov, ns_steps, n_coeffs;
+    float coeffs[MA_MAX_NS_STEPS][3];
+    int32_t scale_mode, heads, precision;
+} ma_muon_hparams_t;
+
+/* AdamW hyperparameters [P1 "AdamW Step Implementation"; P3 _finish: bias
+ * corrections are runtime scalars]. `step` is the 1-based index of the step
+ * being taken; the bias corrections 1 - beta^step are formed in double on the
+ * host. Update: m <- b1 m + (1-b1) g; v <- b2 v + (1-b2) g^2;
+ * p <- p (1 - lr wd) - lr (m / (1-b1^t)) / (sqrt(v / (1-b2^t)) + eps). */
+typedef struct {
+    float lr, beta1, beta2, eps, weight_decay;
+    int64_t step;
+} ma_adamw_hparams_t;
+
+/* A parameter group: `kind` dispatch as in [P1 "The MuonAdamW Class Architecture"]. */
+typedef struct {
+    int32_t kind;                /* ma_kind_t */
+    ma_muon_hparams_t muon;      /* used when kind == MA_MUON  */
+    ma_adamw_hparams_t adamw;    /* used when kind == MA_ADAMW */
+} ma_group_t;
+
+/* One tensor of the model. All buffers are device, fp32 row-major contiguous,
+ * 16-byte aligned, except grad, which is fp32 or bf16 (grad_dtype).
+ * state0/state1: Muon: momentum (state1 unused, may be NULL);
+ *                AdamW: exp_avg, exp_avg_sq. State starts at zero. */
+typedef struct {
+    float* param;
+    const void* grad;
+    int32_t grad_dtype;          /* ma_dtype_t */
+    float* state0;
+    float* state1;
+    int32_t ndim;                /* 0, 1 or 2 */
+    int64_t shape[2];
+    int32_t role;                /* ma_role_t */
+    int32_t group;               /* index into the group table */
+} ma_tensor_t;
+
+typedef struct ma_plan ma_plan_t;
+
+/* ---------------------------------------------------------------- host-only */
+
+const char* ma_status_string(int status);
+int ma_version(void);
+
+/* sizeof of the ABI structs, for bindings to check their layouts:
+ * 0 ma_tensor_t, 1 ma_group_t, 2 ma_muon_hparams_t, 3 ma_adamw_hparams_t; else 0. */
+size_t ma_struct_size(int which);
+
+/* Partition by tensor rank [P1 "Parameter Grouping Strategy"; P4]:
+ * ndim <= 1 -> MA_ADAMW; ndim == 2 with role HIDDEN -> MA_MUON; ndim == 2 with
+ * role EMBED / UNEMBED / FORCE_ADAMW -> MA_ADAMW; ndim >= 3 -> MA_ERR_UNSUPPORTED.
+ * t: host array of n tensors (only ndim and role are read). kind_out: host
+ * array of n ints. Host-only, no CUDA call, bit-exact and deterministic. */
+int ma_partition(const ma_tensor_t* t, int n, int32_t* kind_out);
+
+/* Owner rank per tensor for a data-parallel step over `world_size` ranks: Muon
+ * matrices by greedy largest-Newton-Schulz-flops-first onto the least-loaded
+ * rank, AdamW tensors the same way by element count, ties to the lower rank and
+ * the lower tensor index. Every tensor gets exactly one owner. Host-only. */
+int ma_assign_owners(const ma_tensor_t* t, int n, const ma_group_t* groups, int ngroups,
+                     int world_size, int32_t* owner_out);
+
+/* ---------------------------------------------------------------- Muon */
+
+/* Workspace bytes that muon_step_batched needs for `batch` matrices of R x C
+ * with these hyperparameters (0 for an empty batch; SIZE_MAX for invalid input). */
+size_t muon_workspace_bytes(int batch, int64_t R, int64_t C, const ma_muon_hparams_t* hp);
+
+/* One Muon step on `batch` same-shape R x C matrices [P1 "Muon Step
+ * Implementation": stacked matrices, momentum, orthogonalisation, decay, write
+ * back; P3 _prepare/_finish: fp32 weights and momentum mutated in place,
+ * gradients preserved, scale from the global shape; P5: EMA momentum and the
+ * Newton-Schulz cubic].
+ *  W, M: host arrays of `batch` device pointers to fp32 R x C row-major
+ *        (weights, momentum), updated in place.
+ *  G:    host array of `batch` device pointers to R x C gradients (gdt), read only.
+ *  hp:   host pointer. ws: device workspace of ws_bytes >= muon_workspace_bytes(),
+ *        256-byte aligned, contents scratch.
+ * Requires C % 8 == 0 and 16-byte aligned W/M/G; R % hp->heads == 0. */
+int muon_step_batched(int batch, int64_t R, int64_t C, float* const* W, const void* const* G,
+                      int gdt, float* const* M, const ma_muon_hparams_t* hp, void* ws,
+                      size_t ws_bytes, void* stream);
+
+/* Newton-Schulz iterations alone, no normalisation [P5 "Newton-Schulz
+ * Orthogonalization"]: for each of `batch` bf16 m x n row-major matrices with
+ * m <= n, X <- aX + b(XX^T)X (+ c(XX^T)^2 X) for `steps` iterations.
+ * X_in (device, read only) and X_out (device) hold batch*m*n bf16 values
+ * (uint16 bit patterns), n % 8 == 0, 16-byte aligned. coeffs: host array of
+ * n_coeffs triples (1 or steps). ws: device, >= ns_iterate_workspace_bytes(). */
+size_t ns_iterate_workspace_bytes(int batch, int64_t m, int64_t n);
+int ns_iterate_bf16(int batch, int64_t m, int64_t n, const uint16_t* X_in, uint16_t* X_out,
+                    const float* coeffs, int n_coeffs, int steps, void* ws, size_t ws_bytes,
+                    void* stream);
+
+/* ---------------------------------------------------------------- AdamW */
+
+/* One AdamW step on n tensors in one multi-tensor launch sequence
+ * [P1 "AdamW Step Implementation"]. P, M, V: host arrays of n device pointers
+ * to fp32 (param, exp_avg, exp_avg_sq), updated in place. G: host array of n
+ * device pointers to gradients of dtype gdt, read only. numel: host array of n
+ * element counts (0 allowed). hp: host pointer. */
+int adamw_step_fused(int n, float* const* P, const void* const* G, int gdt, float* const* M,
+                     float* const* V, const int64_t* numel, const ma_adamw_hparams_t* hp,
+                     void* stream);
+
+/* ---------------------------------------------------------------- whole step */
+
+/* Build a plan for a parameter table [P1 "The MuonAdamW Class Architecture"]:
+ * partition, same-shape Muon buckets (first-appearance order), batching and
+ * workspace sizing. t, groups: host arrays, copied. *ws_bytes: in = largest
+ * workspace the caller will provide (0 = no limit), out = the bytes that
+ * muonadamw_step needs (Muon buckets are split into sub-batches to fit). */
+int ma_plan_create(const ma_tensor_t* t, int n, const ma_group_t* groups, int ngroups,
+                   ma_plan_t** out, size_t* ws_bytes);
+
+/* One MuonAdamW step over the planned table: one multi-tensor AdamW pass over
+ * every AdamW tensor, then each Muon bucket. groups: host array with this
+ * step's hyperparameters (same count and kinds as at plan time; lr schedules
+ * and the AdamW step counter change here). ws: device, >= the planned size. */
+int muonadamw_step(ma_plan_t* plan, const ma_group_t* groups, void* ws, size_t ws_bytes,
+                   void* stream);
+
+/* Number of kernel launches the last muonadamw_step issued (for benchmarks). */
+int ma_plan_last_launches(const ma_plan_t* plan);
+
+void ma_plan_destroy(ma_plan_t* plan);
+
+/* ---------------------------------------------------------------- status */
+
+/* Synchronise `stream`, return the per-device status word (MA_OK or the first
+ * device-side error recorded since the last reset) and, if reset != 0, clear it. */
+int ma_device_status(void* stream, int reset);
+
+/* Set the limit, in nanoseconds, of every device-side bounded wait (default
+ * 2e9). Takes effect for launches issued after the call. */
+int ma_set_wait_limit_ns(int64_t limit_ns);
+
+/* Self-test of the bounded wait: launch one block that waits on a barrier
+ * phase that nothing completes, with a wait limit of limit_ns. The kernel
+ * returns after the limit and records MA_ERR_TIMEOUT in the status word;
+ * the context stays usable. Returns the launch status (MA_OK if launched). */
+int ma_selftest_wait_timeout(int64_t limit_ns, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUONADAMW_H */

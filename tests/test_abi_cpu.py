@@ -1,0 +1,200 @@
+"""C-ABI boundary tests that need no GPU.
+
+The library must load, export every function that include/muonadamw.h
+declares, agree with the binding on struct layouts, partition bit-exactly
+like the oracle, and reject bad arguments with the documented status code
+before it touches any memory. With valid arguments and no usable device, the
+call must fail loudly (MA_ERR_CUDA / MA_ERR_UNSUPPORTED), never fall back.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+import adamw_hybrid_optimizer_muon_b200 as ma
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "muonadamw.h")
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s+\**([a-z_][a-z0-9_]*)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_symbols_exported():
+    names = declared_functions()
+    assert len(names) >= 15
+    L = ma.lib()
+    for n in names:
+        assert hasattr(L, n), f"{n} declared in muonadamw.h but not exported"
+
+
+def test_struct_layouts_match():
+    L = ma.lib()
+    for which, cls in enumerate((ma.Tensor, ma.Group, ma.MuonHParams, ma.AdamWHParams)):
+        assert L.ma_struct_size(which) == ctypes.sizeof(cls)
+    assert L.ma_version() == 1
+    assert L.ma_status_string(8) == b"device wait timed out"
+
+
+def _desc(shape, role, group=0):
+    t = ma.Tensor()
+    t.ndim = len(shape)
+    for d, s in enumerate(shape[:2]):
+        t.shape[d] = s
+    t.role = role
+    t.group = group
+    return t
+
+
+@pytest.mark.parametrize("name", ["tiny", "d20", "7b", "aspect", "square"])
+def test_partition_bit_exact_vs_oracle(name):
+    wl = synth.WORKLOADS[name]()
+    descs = [_desc(t.shape, t.role, t.group) for t in wl.tensors]
+    assert ma.ma_partition(descs) == oracle.partition([(t.shape, t.role) for t in wl.tensors])
+
+
+def test_partition_random_tables():
+    r = np.random.default_rng(0)
+    for _ in range(50):
+        n = int(r.integers(1, 40))
+        table = []
+        for _ in range(n):
+            nd = int(r.integers(0, 3))
+            shape = tuple(int(x) for x in r.integers(0, 9, size=nd))
+            table.append((shape, int(r.integers(0, 4))))
+        got = ma.ma_partition([_desc(s, ro) for s, ro in table])
+        assert got == oracle.partition(table)
+
+
+def test_partition_rejects_rank3():
+    with pytest.raises(ma.MAError) as e:
+        ma.ma_partition([_desc((2, 3), 0), _desc((2, 3, 4), 0)])
+    assert e.value.code == ma.MA_ERR_UNSUPPORTED
+
+
+def _groups_for(wl):
+    gs = []
+    for g in wl.groups:
+        G = ma.Group()
+        G.kind = g.kind
+        if g.kind == ma.MA_MUON:
+            h = g.muon
+            G.muon = ma.muon_hparams(h.lr, h.beta, h.weight_decay, h.eps, h.nesterov, h.ns_steps, h.coeffs,
+                                     h.scale_mode, h.heads, h.precision)
+        else:
+            h = g.adamw
+            G.adamw = ma.adamw_hparams(h.lr, h.beta1, h.beta2, h.eps, h.weight_decay, 1)
+        gs.append(G)
+    return gs
+
+
+@pytest.mark.parametrize("name,world", [("7b", 1), ("7b", 2), ("7b", 8), ("d20", 3), ("aspect", 4), ("tiny", 2)])
+def test_owner_assignment_exactly_once_and_balanced(name, world):
+    wl = synth.WORKLOADS[name]()
+    descs = [_desc(t.shape, t.role, t.group) for t in wl.tensors]
+    owners = ma.ma_assign_owners(descs, _groups_for(wl), world)
+    assert len(owners) == len(descs)
+    assert all(0 <= o < world for o in owners)
+    assert owners == ma.ma_assign_owners(descs, _groups_for(wl), world)  # deterministic
+    # greedy bound: the heaviest rank exceeds the average by at most the largest item
+    kinds = oracle.partition([(t.shape, t.role) for t in wl.tensors])
+    for kind in (0, 1):
+        items = [t.numel for t, k in zip(wl.tensors, kinds) if k == kind]
+        if not items or kind == 0:
+            continue
+        load = [0] * world
+        for t, k, o in zip(wl.tensors, kinds, owners):
+            if k == kind:
+                load[o] += t.numel
+        assert max(load) <= sum(items) / world + max(items)
+
+
+def test_validation_before_any_device_call():
+    hp = ma.muon_hparams()
+    L = ma.lib()
+    fake = ctypes.c_void_p(0x1000)
+    arr = (ctypes.c_void_p * 1)(0x1000)
+    null = (ctypes.c_void_p * 1)(0)
+    # C % 8 != 0
+    rc = L.muon_step_batched(1, 16, 12, arr, arr, ma.MA_F32, arr, ctypes.byref(hp), fake, 1 << 30, None)
+    assert rc == ma.MA_ERR_ALIGN
+    # null pointer entry
+    rc = L.muon_step_batched(1, 16, 16, null, arr, ma.MA_F32, arr, ctypes.byref(hp), fake, 1 << 30, None)
+    assert rc == ma.MA_ERR_NULL
+    # heads must divide R
+    hp3 = ma.muon_hparams(heads=3)
+    rc = L.muon_step_batched(1, 16, 16, arr, arr, ma.MA_F32, arr, ctypes.byref(hp3), fake, 1 << 30, None)
+    assert rc == ma.MA_ERR_SHAPE
+    # bad dtype, bad steps, bad coefficient count
+    assert L.muon_step_batched(1, 16, 16, arr, arr, 7, arr, ctypes.byref(hp), fake, 1 << 30, None) == ma.MA_ERR_DTYPE
+    bad = ma.muon_hparams(ns_steps=0)
+    assert L.muon_step_batched(1, 16, 16, arr, arr, 0, arr, ctypes.byref(bad), fake, 1 << 30, None) == ma.MA_ERR_ARG
+    bad = ma.muon_hparams(ns_steps=3, coeffs=((1.5, -0.5, 0), (1.5, -0.5, 0)))
+    assert L.muon_step_batched(1, 16, 16, arr, arr, 0, arr, ctypes.byref(bad), fake, 1 << 30, None) == ma.MA_ERR_ARG
+    # workspace too small / misaligned
+    assert L.muon_step_batched(1, 16, 16, arr, arr, 0, arr, ctypes.byref(hp), fake, 16, None) == ma.MA_ERR_WORKSPACE
+    assert L.muon_step_batched(1, 16, 16, arr, arr, 0, arr, ctypes.byref(hp), ctypes.c_void_p(0x1008), 1 << 30,
+                               None) == ma.MA_ERR_WORKSPACE
+    # empty batch is a no-op
+    assert L.muon_step_batched(0, 16, 16, arr, arr, 0, arr, ctypes.byref(hp), None, 0, None) == ma.MA_OK
+    # AdamW: bad step, bad betas
+    ahp = ma.adamw_hparams(step=0)
+    n1 = (ctypes.c_int64 * 1)(4)
+    assert L.adamw_step_fused(1, arr, arr, 0, arr, arr, n1, ctypes.byref(ahp), None) == ma.MA_ERR_ARG
+    ahp = ma.adamw_hparams(beta2=1.0)
+    assert L.adamw_step_fused(1, arr, arr, 0, arr, arr, n1, ctypes.byref(ahp), None) == ma.MA_ERR_ARG
+    ahp = ma.adamw_hparams()
+    assert L.adamw_step_fused(1, null, arr, 0, arr, arr, n1, ctypes.byref(ahp), None) == ma.MA_ERR_NULL
+
+
+def test_valid_call_without_gpu_fails_loudly():
+    try:
+        import torch
+        if torch.cuda.is_available():
+            pytest.skip("a GPU is present")
+    except ImportError:
+        pass
+    hp = ma.muon_hparams()
+    L = ma.lib()
+    arr = (ctypes.c_void_p * 1)(0x1000)
+    rc = L.muon_step_batched(1, 16, 16, arr, arr, 0, arr, ctypes.byref(hp), ctypes.c_void_p(0x10000), 1 << 30, None)
+    assert rc in (ma.MA_ERR_CUDA, ma.MA_ERR_UNSUPPORTED)
+
+
+def test_plan_sizing_on_host():
+    wl = synth.llama7b()
+    descs = []
+    for i, t in enumerate(wl.tensors):
+        d = _desc(t.shape, t.role, t.group)
+        d.param = d.state0 = d.state1 = d.grad = 0x100000 + 0x1000 * i
+        d.grad_dtype = ma.MA_BF16
+        descs.append(d)
+    plan, ws = ma.ma_plan_create(descs, _groups_for(wl))
+    hp = ma.muon_hparams()
+    expect = max(ma.muon_workspace_bytes(128, 4096, 4096, hp), ma.muon_workspace_bytes(64, 4096, 11008, hp),
+                 ma.muon_workspace_bytes(32, 11008, 4096, hp))
+    assert ws == expect
+    ma.ma_plan_destroy(plan)
+    # a cap splits buckets into sub-batches
+    plan, ws2 = ma.ma_plan_create(descs, _groups_for(wl), ws_cap=4 << 30)
+    assert 0 < ws2 <= 4 << 30
+    ma.ma_plan_destroy(plan)
+    with pytest.raises(ma.MAError) as e:
+        ma.ma_plan_create(descs, _groups_for(wl), ws_cap=1 << 20)
+    assert e.value.code == ma.MA_ERR_WORKSPACE
+
+
+def test_plan_rejects_kind_mismatch():
+    wl = synth.tiny()
+    d0 = _desc((256, 512), ma.ROLE_HIDDEN, 1)  # a Muon matrix in the AdamW group
+    d0.param = d0.state0 = d0.state1 = d0.grad = 0x100000
+    with pytest.raises(ma.MAError) as e:
+        ma.ma_plan_create([d0], _groups_for(wl))
+    assert e.value.code == ma.MA_ERR_ARG

@@ -1,0 +1,143 @@
+"""The whole MuonAdamW step through the plan (muonadamw_step) against the oracle.
+
+* tiny: every element of every tensor, two steps.
+* d20 and the 7B-shaped set at full size, in the same launch configuration
+  bench.py times. The oracle recomputes sampled matrices in full (one of each
+  bucket) and sampled elements of the AdamW tensors and of every momentum
+  buffer, two steps from zero state.
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle
+import synth
+import synth.device as sdev
+import adamw_hybrid_optimizer_muon_b200 as ma
+from gpu_helpers import TOL_BF16, TOL_F32, check_muon, check_state, host, momentum_terms
+
+pytestmark = pytest.mark.gpu
+
+
+def build_optimizer(wl, params, precision=0):
+    groups = []
+    for g in wl.groups:
+        if g.kind == synth.KIND_MUON:
+            h = g.muon
+            groups.append(("muon", ma.muon_hparams(h.lr, h.beta, h.weight_decay, h.eps, h.nesterov, h.ns_steps,
+                                                   h.coeffs, h.scale_mode, h.heads, precision)))
+        else:
+            h = g.adamw
+            groups.append(("adamw", ma.adamw_hparams(h.lr, h.beta1, h.beta2, h.eps, h.weight_decay, 1)))
+    return ma.MuonAdamW([(p, t.role, t.group) for p, t in zip(params, wl.tensors)], groups)
+
+
+def oracle_groups(wl, precision=0):
+    out = []
+    for g in wl.groups:
+        if g.kind == synth.KIND_MUON:
+            h = g.muon
+            out.append(dict(kind=0, lr=h.lr, beta=h.beta, weight_decay=h.weight_decay, eps=h.eps,
+                            nesterov=h.nesterov, ns_steps=h.ns_steps, coeffs=h.coeffs, scale_mode=h.scale_mode,
+                            heads=h.heads))
+        else:
+            h = g.adamw
+            out.append(dict(kind=1, lr=h.lr, beta1=h.beta1, beta2=h.beta2, eps=h.eps,
+                            weight_decay=h.weight_decay))
+    return out
+
+
+@pytest.mark.parametrize("precision", [0, 1])
+def test_tiny_two_steps_every_element(precision):
+    wl = synth.tiny()
+    W0 = [synth.initial_weight(t, i) for i, t in enumerate(wl.tensors)]
+    params = [torch.from_numpy(w).cuda() for w in W0]
+    opt = build_optimizer(wl, params, precision)
+    tensors = [dict(shape=t.shape, role=t.role, group=t.group) for t in wl.tensors]
+    groups = oracle_groups(wl)
+    state = [{} for _ in wl.tensors]
+    ref = [w.astype(np.float64) for w in W0]
+    for step in (1, 2):
+        G = [synth.gradient(wl, i, step) for i in range(len(wl.tensors))]
+        gd = [torch.from_numpy(g).cuda() for g in G]  # fp32 gradients in this config
+        before_p = [host(p) for p in params]
+        before_s = [(host(s0), None if s1 is None else host(s1)) for s0, s1 in opt.state]
+        opt.step(gd)
+        torch.cuda.synchronize()
+        assert ma.ma_device_status() == ma.MA_OK
+        # one oracle step from exactly the GPU's pre-step values
+        st = [{"m": before_s[0][0]}, {"exp_avg": before_s[1][0], "exp_avg_sq": before_s[1][1]}]
+        ref = oracle.muonadamw_step(tensors, groups, before_p, G, st, step)
+        m = wl.groups[0].muon
+        check_muon(before_p[0], host(params[0]), ref[0], m.lr, m.weight_decay, TOL_F32 if precision else TOL_BF16)
+        check_state(host(opt.state[0][0]), st[0]["m"], momentum_terms(before_s[0][0], G[0], m.beta), what="m")
+        a = wl.groups[1].adamw
+        tp, tm, tv = oracle.adamw_term_magnitudes(before_p[1], G[1], before_s[1][0], before_s[1][1], step, a.lr,
+                                                  a.beta1, a.beta2, a.eps, a.weight_decay)
+        check_state(host(params[1]), ref[1], tp, what="gain")
+        check_state(host(opt.state[1][0]), st[1]["exp_avg"], tm, what="exp_avg")
+        check_state(host(opt.state[1][1]), st[1]["exp_avg_sq"], tv, what="exp_avg_sq")
+    assert opt.launches == 1 + 2 + 2 * 5  # AdamW, momentum+norm, finalize, 5 x (Gram, apply)
+
+
+def _full_size_check(name, n_muon_samples=1, adamw_samples=200_000, seed=0):
+    wl = synth.WORKLOADS[name]()
+    params = sdev.weights(wl)
+    opt = build_optimizer(wl, params)
+    kinds = oracle.partition([(t.shape, t.role) for t in wl.tensors])
+    buckets = oracle.muon_buckets([(t.shape, t.role) for t in wl.tensors], [t.group for t in wl.tensors])
+    sample_mats = [idx for b in buckets for idx in b[3][:n_muon_samples]]
+    r = np.random.default_rng(seed)
+    grads = None
+    for step in (1, 2):
+        grads = sdev.gradients(wl, step, out=grads)
+        snap = {}
+        for i in sample_mats:
+            snap[i] = (host(params[i]), host(grads[i]), host(opt.state[i][0]))
+        # sampled elements of everything else
+        idx = {}
+        for i, t in enumerate(wl.tensors):
+            n = t.numel
+            k = min(n, adamw_samples if kinds[i] == 1 else 4096)
+            sel = torch.from_numpy(r.choice(n, size=k, replace=False) if k < n else np.arange(n)).cuda()
+            flat = lambda x: x.reshape(-1)[sel]  # noqa: E731
+            s0, s1 = opt.state[i]
+            idx[i] = (sel, host(flat(params[i])), host(flat(grads[i])), host(flat(s0)),
+                      None if s1 is None else host(flat(s1)))
+        opt.step(grads)
+        torch.cuda.synchronize()
+        assert ma.ma_device_status() == ma.MA_OK
+        for i in sample_mats:
+            w0, g, m0 = snap[i]
+            grp = wl.groups[wl.tensors[i].group].muon
+            rw, rm = oracle.muon_update(w0, g, m0, grp.lr, grp.beta, grp.weight_decay, grp.nesterov, grp.ns_steps,
+                                        grp.coeffs, grp.eps, grp.scale_mode, grp.heads)
+            check_muon(w0, host(params[i]), rw, grp.lr, grp.weight_decay, TOL_BF16, what=wl.tensors[i].name)
+            check_state(host(opt.state[i][0]), rm, momentum_terms(m0, g, grp.beta), what="momentum")
+        for i, t in enumerate(wl.tensors):
+            sel, p0, g, s0, s1 = idx[i]
+            flat = lambda x: x.reshape(-1)[sel]  # noqa: E731
+            if kinds[i] == 1:
+                a = wl.groups[t.group].adamw
+                rp, rm, rv = oracle.adamw_update(p0, g, s0, s1, step, a.lr, a.beta1, a.beta2, a.eps, a.weight_decay)
+                tp, tm, tv = oracle.adamw_term_magnitudes(p0, g, s0, s1, step, a.lr, a.beta1, a.beta2, a.eps,
+                                                          a.weight_decay)
+                check_state(host(flat(params[i])), rp, tp, what=t.name)
+                check_state(host(flat(opt.state[i][0])), rm, tm, what=t.name + ".exp_avg")
+                check_state(host(flat(opt.state[i][1])), rv, tv, what=t.name + ".exp_avg_sq")
+            else:
+                grp = wl.groups[t.group].muon
+                rm, _ = oracle.momentum_update(s0, g, grp.beta, grp.nesterov)
+                check_state(host(flat(opt.state[i][0])), rm, momentum_terms(s0, g, grp.beta),
+                            what=t.name + ".m")
+    return opt
+
+
+def test_d20_full_size_sampled():
+    _full_size_check("d20", n_muon_samples=2)
+
+
+@pytest.mark.slow
+def test_7b_full_size_sampled():
+    _full_size_check("7b", n_muon_samples=1, adamw_samples=100_000)
