@@ -286,16 +286,20 @@ def rel_frobenius(x, ref):
 
 
 def adamw_term_magnitudes(p, g, m, v, step, lr, beta1, beta2, eps, weight_decay):
-    """Per-element sum of |addends| in each updated quantity, for the cancellation-safe bound."""
+    """Per-element sum of |addends| in each updated quantity, for the cancellation-safe bound.
+
+    The step term lr * m_hat / (sqrt(v_hat) + eps) contains the sum
+    beta1*m + (1-beta1)*g, which can cancel. Its addends enter in absolute
+    value, so the bound follows the magnitudes that the computation handles
+    (forward error propagation), not just the magnitude of the final result.
+    """
     p = np.asarray(p, dtype=np.float64)
     g = np.asarray(g, dtype=np.float64)
     m = np.asarray(m, dtype=np.float64)
     v = np.asarray(v, dtype=np.float64)
-    m_new = beta1 * m + (1.0 - beta1) * g
     v_new = beta2 * v + (1.0 - beta2) * g * g
-    m_hat = m_new / (1.0 - beta1 ** step)
     v_hat = v_new / (1.0 - beta2 ** step)
     t_m = np.abs(beta1 * m) + np.abs((1.0 - beta1) * g)
     t_v = np.abs(beta2 * v) + np.abs((1.0 - beta2) * g * g)
-    t_p = np.abs(p * (1.0 - lr * weight_decay)) + np.abs(lr * m_hat / (np.sqrt(v_hat) + eps))
+    t_p = np.abs(p * (1.0 - lr * weight_decay)) + lr * (t_m / (1.0 - beta1 ** step)) / (np.sqrt(v_hat) + eps)
     return t_p, t_m, t_v
