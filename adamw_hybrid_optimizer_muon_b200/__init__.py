@@ -18,7 +18,7 @@ __all__ = [
     "ROLE_FORCE_ADAMW", "ma_partition", "ma_assign_owners", "muon_workspace_bytes", "muon_step_batched",
     "ns_iterate_workspace_bytes", "ns_iterate_bf16", "adamw_step_fused", "ma_plan_create", "muonadamw_step",
     "ma_plan_destroy", "ma_device_status", "ma_set_wait_limit_ns", "ma_selftest_wait_timeout", "Plan",
-    "MuonAdamW", "muon_hparams", "adamw_hparams",
+    "MuonAdamW", "muon_hparams", "adamw_hparams", "ma_profile_enable", "ma_profile_collect", "PROF_CLASSES",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -106,6 +106,9 @@ def lib() -> ctypes.CDLL:
         "ma_device_status": (i32, [vp, i32]),
         "ma_set_wait_limit_ns": (i32, [i64]),
         "ma_selftest_wait_timeout": (i32, [i64, vp]),
+        "ma_profile_enable": (i32, [i32]),
+        "ma_profile_collect": (i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64),
+                                     ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(L, name)
@@ -283,6 +286,23 @@ def ma_set_wait_limit_ns(limit_ns: int) -> None:
 
 def ma_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
     _check(lib().ma_selftest_wait_timeout(int(limit_ns), _stream(stream)), "ma_selftest_wait_timeout")
+
+
+PROF_CLASSES = ("adamw", "momentum", "finalize", "ns_gram", "ns_apply", "ns_gramsq")
+
+
+def ma_profile_enable(on: bool) -> None:
+    _check(lib().ma_profile_enable(int(bool(on))), "ma_profile_enable")
+
+
+def ma_profile_collect() -> dict:
+    """Per kernel class: {"ms", "launches", "flops", "bytes"} summed since the last collect."""
+    k = len(PROF_CLASSES)
+    ms, cnt = (ctypes.c_double * k)(), (ctypes.c_int64 * k)()
+    fl, by = (ctypes.c_double * k)(), (ctypes.c_double * k)()
+    _check(lib().ma_profile_collect(ms, cnt, fl, by), "ma_profile_collect")
+    return {name: {"ms": ms[i], "launches": int(cnt[i]), "flops": fl[i], "bytes": by[i]}
+            for i, name in enumerate(PROF_CLASSES)}
 
 
 # ---------------------------------------------------------------------------- user-level wrappers

@@ -43,6 +43,43 @@ int* device_status_ptr() {
 
 namespace {
 
+// ------------------------------------------------------------------ launch profiler
+
+struct ProfRec {
+    int ev;  // index of the event pair in the pool
+    int cls;
+    double flops, bytes;
+};
+thread_local bool g_prof_on = false;
+thread_local std::vector<std::pair<cudaEvent_t, cudaEvent_t>> g_prof_pool;
+thread_local std::vector<ProfRec> g_prof_recs;
+
+// Returns the record index, or -1 when profiling is off or an event is unavailable.
+int prof_begin(int cls, cudaStream_t s) {
+    if (!g_prof_on) return -1;
+    const size_t k = g_prof_recs.size();
+    if (k >= g_prof_pool.size()) {
+        cudaEvent_t a, b;
+        if (cudaEventCreate(&a) != cudaSuccess) return -1;
+        if (cudaEventCreate(&b) != cudaSuccess) {
+            cudaEventDestroy(a);
+            return -1;
+        }
+        g_prof_pool.push_back({a, b});
+    }
+    if (cudaEventRecord(g_prof_pool[k].first, s) != cudaSuccess) return -1;
+    g_prof_recs.push_back({(int)k, cls, 0.0, 0.0});
+    return (int)k;
+}
+
+void prof_end(int rec, cudaStream_t s, double flops, double bytes) {
+    if (rec < 0) return;
+    ProfRec& r = g_prof_recs[rec];
+    r.flops = flops;
+    r.bytes = bytes;
+    cudaEventRecord(g_prof_pool[r.ev].second, s);
+}
+
 constexpr size_t kAlign = 256;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -149,6 +186,20 @@ float shape_scale(int64_t R, int64_t C, int mode) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? MA_OK : MA_ERR_CUDA; }
 
+int ns_prof_class(int mode) {
+    return mode == NS_GRAM ? MA_PROF_NS_GRAM : mode == NS_GRAMSQ ? MA_PROF_NS_GRAMSQ : MA_PROF_NS_APPLY;
+}
+
+// Algorithmic flops of one Newton-Schulz launch. A symmetric Gram X X^T has
+// m(m+1)/2 distinct entries of n multiply-adds each: m(m+1)n flops (A A^T:
+// m(m+1)m). The apply B X costs 2 m^2 n.
+double ns_flops(int mode, int64_t units, int64_t m, int64_t n) {
+    const double u = (double)units, M = (double)m, N = (double)n;
+    if (mode == NS_GRAM) return u * M * (M + 1.0) * N;
+    if (mode == NS_GRAMSQ) return u * M * (M + 1.0) * M;
+    return u * 2.0 * M * M * N;
+}
+
 // All checks passed; launch the whole Muon chain for one batch.
 int run_muon(int batch, const MuonGeom& g, float* const* W, const void* const* G, int gdt, float* const* M,
              const ma_muon_hparams_t& hp, void* ws, cudaStream_t s, int sms, int* launches) {
@@ -183,9 +234,14 @@ int run_muon(int batch, const MuonGeom& g, float* const* W, const void* const* G
         P.G[b] = G[b];
         P.M[b] = M[b];
     }
+    const double elems = (double)g.units * (double)g.Rh * (double)g.C;
+    int pr = prof_begin(MA_PROF_MOMENTUM, s);
     int st = cuda_status(launch_muon_prep(P, s));
+    prof_end(pr, s, 0.0, elems * ((gdt == MA_BF16 ? 2 : 4) + 8 + (hp.precision ? 4 : 2)));
     if (st) return st;
+    pr = prof_begin(MA_PROF_FINALIZE, s);
     st = cuda_status(launch_norm_finalize(part, g.parts, (int)g.units, hp.eps, scale, s));
+    prof_end(pr, s, 0.0, (double)g.units * g.parts * 8.0 + g.units * 4.0);
     if (st) return st;
     *launches += 2;
 
@@ -210,7 +266,9 @@ int run_muon(int batch, const MuonGeom& g, float* const* W, const void* const* G
     for (int b = 0; b < batch; ++b) p.W[b] = W[b];
 
     auto launch = [&](int mode, const void* xb, const void* gb) -> int {
+        const int pr = prof_begin(ns_prof_class(mode), s);
         cudaError_t e = hp.precision ? launch_ns_simt(mode, p, xb, gb, s) : launch_ns_tc(mode, p, xb, gb, sms, s);
+        prof_end(pr, s, ns_flops(mode, g.units, g.m, g.n), 0.0);
         ++*launches;
         return cuda_status(e);
     };
@@ -337,7 +395,11 @@ int run_adamw(const std::vector<AdamwItem>& items, int gdt, const AdamwGroupCons
         L.ntensors = nt;
         L.nchunks = chunk;
         if (nt > 0) {
+            double elems = 0.0;
+            for (int k = 0; k < nt; ++k) elems += (double)L.t[k].numel;
+            const int pr = prof_begin(MA_PROF_ADAMW, s);
             cudaError_t e = launch_adamw(L, s);
+            prof_end(pr, s, 0.0, elems * (gdt == MA_BF16 ? 26.0 : 28.0));
             if (e != cudaSuccess) return MA_ERR_CUDA;
             ++*launches;
         }
@@ -553,13 +615,19 @@ int ns_iterate_bf16(int batch, int64_t m, int64_t n, const uint16_t* X_in, uint1
         p.c = cf[2];
         const bool quint = cf[2] != 0.f;
         p.coef_gram = quint ? 1.f : cf[1];
+        auto launch = [&](int mode, const void* xb, const void* gb) -> int {
+            const int pr = prof_begin(ns_prof_class(mode), s);
+            cudaError_t e = launch_ns_tc(mode, p, xb, gb, sms, s);
+            prof_end(pr, s, ns_flops(mode, batch, m, n), 0.0);
+            return cuda_status(e);
+        };
         p.out = Gb;
-        if (cuda_status(launch_ns_tc(NS_GRAM, p, cur, Gb, sms, s))) return MA_ERR_CUDA;
+        if (launch(NS_GRAM, cur, Gb)) return MA_ERR_CUDA;
         void* Bbuf = Gb;
         if (quint) {
             p.xin = Gb;
             p.out = G2;
-            if (cuda_status(launch_ns_tc(NS_GRAMSQ, p, cur, Gb, sms, s))) return MA_ERR_CUDA;
+            if (launch(NS_GRAMSQ, cur, Gb)) return MA_ERR_CUDA;
             Bbuf = G2;
         }
         // the last iteration writes X_out; earlier ones alternate so that no GEMM
@@ -567,7 +635,7 @@ int ns_iterate_bf16(int batch, int64_t m, int64_t n, const uint16_t* X_in, uint1
         void* dst = ((steps - 1 - k) % 2 == 0) ? static_cast<void*>(X_out) : T;
         p.xin = cur;
         p.out = dst;
-        if (cuda_status(launch_ns_tc(NS_APPLY, p, cur, Bbuf, sms, s))) return MA_ERR_CUDA;
+        if (launch(NS_APPLY, cur, Bbuf)) return MA_ERR_CUDA;
         cur = dst;
     }
     return MA_OK;
@@ -755,6 +823,41 @@ int muonadamw_step(ma_plan_t* plan, const ma_group_t* groups, void* ws, size_t w
 int ma_plan_last_launches(const ma_plan_t* plan) { return plan ? plan->last_launches : 0; }
 
 void ma_plan_destroy(ma_plan_t* plan) { delete plan; }
+
+int ma_profile_enable(int on) {
+    g_prof_on = on != 0;
+    return MA_OK;
+}
+
+int ma_profile_collect(double* ms_out, int64_t* launches_out, double* flops_out, double* bytes_out) {
+    double ms[MA_PROF_CLASSES] = {0}, fl[MA_PROF_CLASSES] = {0}, by[MA_PROF_CLASSES] = {0};
+    int64_t cnt[MA_PROF_CLASSES] = {0};
+    int st = MA_OK;
+    for (const ProfRec& r : g_prof_recs) {
+        const auto& ev = g_prof_pool[r.ev];
+        if (cudaEventSynchronize(ev.second) != cudaSuccess) {
+            st = MA_ERR_CUDA;
+            continue;
+        }
+        float t = 0.f;
+        if (cudaEventElapsedTime(&t, ev.first, ev.second) != cudaSuccess) {
+            st = MA_ERR_CUDA;
+            continue;
+        }
+        ms[r.cls] += t;
+        cnt[r.cls] += 1;
+        fl[r.cls] += r.flops;
+        by[r.cls] += r.bytes;
+    }
+    g_prof_recs.clear();
+    for (int c = 0; c < MA_PROF_CLASSES; ++c) {
+        if (ms_out) ms_out[c] = ms[c];
+        if (launches_out) launches_out[c] = cnt[c];
+        if (flops_out) flops_out[c] = fl[c];
+        if (bytes_out) bytes_out[c] = by[c];
+    }
+    return st;
+}
 
 int ma_device_status(void* stream, int reset) {
     if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MA_ERR_CUDA;

@@ -1,0 +1,394 @@
+#!/usr/bin/env python
+"""Benchmark of one MuonAdamW optimizer step on a B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 7b|d20|square|aspect|tiny]
+                    [--impl ours|reference] [--no-e2e]
+
+A step is one muonadamw_step over a synthetic parameter set. Each step runs
+AdamW on every 0-D/1-D tensor and on the embedding/unembedding, and the
+momentum/norm pass plus 5 Newton-Schulz iterations on every hidden matrix,
+with the final decay and apply. The default workload is the 7B-shaped set.
+Its inputs (params, grads, state: ~80 GB) are far larger than the 126 MB L2,
+so no flush is needed between steps.
+
+Printed (rank 0): one JSON line with the metric (params/s), ms per step, the
+end-to-end number through the C ABI with host buffers, the roofline of the
+dominant kernel (Newton-Schulz GEMMs, measured live with CUDA events on their
+launch stream), the clocks seen during the timed region, and a CPU baseline
+(the fp64 oracle on a bounded sample, host cores).
+
+``--impl reference`` times that same oracle (there is no other implementation
+of this method to run) on a bounded sample per step and prints the same line
+with ``"impl": "reference"``.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "MuonAdamW step ms & params/s; NS TFLOP/s vs bf16 peak; AdamW GB/s vs HBM"
+UNIT = "params/s"
+
+# ncu DRAM traffic per launch of the dominant kernel, from the capture summarised
+# under profiles/ (None until a capture of the current kernel exists).
+NS_TRAFFIC_BYTES_PER_LAUNCH = None
+
+
+def env_int(name, default):
+    try:
+        return int(os.environ.get(name, default))
+    except ValueError:
+        return default
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return {"hbm_gbs": float(p["hbm_gbs"]), "bf16_tflops": float(p["bf16_tflops"]),
+                "bf16_tflops_sustained": float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.path = os.path.join("/tmp", f"ma_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.fh = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu_id), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.fh,
+                                         stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            self.proc.wait(5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.fh.close()
+        sm, smax, reasons = [], [], set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def gpu_id_for(device_index):
+    import torch
+    try:
+        uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+        return uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+    except Exception:
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+        if vis:
+            return vis.split(",")[device_index]
+        return device_index
+
+
+# ----------------------------------------------------------------------------- oracle timing (CPU baseline)
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = [i for i in threadpool_info() if i.get("user_api") == "blas"]
+        if info:
+            return int(info[0]["num_threads"])
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+def oracle_sample(wl):
+    """A bounded slice of the workload for the oracle: one Muon matrix of the most
+    common shape plus AdamW elements in the workload's AdamW:Muon proportion."""
+    import oracle
+    kinds = oracle.partition([(t.shape, t.role) for t in wl.tensors])
+    muon = [i for i, k in enumerate(kinds) if k == 0]
+    adamw = [i for i, k in enumerate(kinds) if k == 1]
+    shapes = {}
+    for i in muon:
+        shapes.setdefault(wl.tensors[i].shape, []).append(i)
+    mi = max(shapes.values(), key=len)[0] if muon else None
+    n_muon = sum(wl.tensors[i].numel for i in muon)
+    n_adamw = sum(wl.tensors[i].numel for i in adamw)
+    mat = wl.tensors[mi].numel if mi is not None else 0
+    k_adamw = int(round(n_adamw * mat / n_muon)) if n_muon else min(n_adamw, 4_000_000)
+    return mi, adamw, k_adamw
+
+
+def time_oracle_step(wl, mi, adamw, k_adamw, step=2):
+    import oracle
+    elapsed = 0.0
+    params = 0
+    if mi is not None:
+        spec = wl.tensors[mi]
+        g = wl.groups[spec.group].muon
+        W = synth.initial_weight(spec, mi)
+        G = synth.gradient(wl, mi, step)
+        M = np.zeros(spec.shape)
+        t0 = time.perf_counter()
+        oracle.muon_update(W, G, M, g.lr, g.beta, g.weight_decay, g.nesterov, g.ns_steps, g.coeffs, g.eps,
+                           g.scale_mode, g.heads)
+        elapsed += time.perf_counter() - t0
+        params += spec.numel
+    left = k_adamw
+    for i in adamw:
+        if left <= 0:
+            break
+        spec = wl.tensors[i]
+        n = min(spec.numel, left)
+        r = synth.rng(i, step, synth.STREAM_GRAD)
+        p = (r.standard_normal(n) * 0.02)
+        gr = r.standard_normal(n) * 1e-3
+        a = wl.groups[spec.group].adamw
+        t0 = time.perf_counter()
+        oracle.adamw_update(p, gr, np.zeros(n), np.zeros(n), step, a.lr, a.beta1, a.beta2, a.eps, a.weight_decay)
+        elapsed += time.perf_counter() - t0
+        params += n
+        left -= n
+    return params, elapsed
+
+
+def cpu_baseline(wl):
+    mi, adamw, k = oracle_sample(wl)
+    params, secs = time_oracle_step(wl, mi, adamw, k)
+    desc = (f"oracle fp64 on 1 Muon matrix {wl.tensors[mi].shape} + {k} AdamW elements "
+            f"({params} params, {secs:.1f} s)") if mi is not None else f"oracle fp64 on {params} AdamW elements"
+    return {"value": params / secs, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": desc}
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    wl = synth.WORKLOADS[args.workload]()
+    mi, adamw, k = oracle_sample(wl)
+    for _ in range(args.warmup):
+        time_oracle_step(wl, mi, adamw, k)
+    tot_params, tot_s = 0, 0.0
+    for _ in range(args.steps):
+        p, s = time_oracle_step(wl, mi, adamw, k)
+        tot_params += p
+        tot_s += s
+    value = tot_params / tot_s
+    sample = f"per step: oracle fp64 on 1 Muon matrix {wl.tensors[mi].shape} + {k} AdamW elements"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * tot_s / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": workload_config(wl, args.gpus),
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def workload_config(wl, n_gpus):
+    import oracle
+    kinds = oracle.partition([(t.shape, t.role) for t in wl.tensors])
+    return {"workload": f"{wl.name}: {wl.description}", "params": wl.numel,
+            "muon_matrices": kinds.count(0), "adamw_tensors": kinds.count(1),
+            "ns_steps": wl.groups[0].muon.ns_steps if wl.groups[0].kind == 0 else None,
+            "l2": "inputs larger than L2 (no flush needed)", "parallelism": f"replicas x{n_gpus}"}
+
+
+# ----------------------------------------------------------------------------- our arm
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="7b", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    rank, world, local = env_int("RANK", 0), env_int("WORLD_SIZE", 1), env_int("LOCAL_RANK", 0)
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+
+    import torch
+    import torch.distributed as dist
+
+    import adamw_hybrid_optimizer_muon_b200 as ma
+    import synth.device as sdev
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    wl = synth.WORKLOADS[args.workload]()
+    params = sdev.weights(wl, device=dev, base=rank)
+    grads = sdev.gradients(wl, 1, device=dev, base=rank)
+    groups = []
+    for g in wl.groups:
+        if g.kind == synth.KIND_MUON:
+            h = g.muon
+            groups.append(("muon", ma.muon_hparams(h.lr, h.beta, h.weight_decay, h.eps, h.nesterov, h.ns_steps,
+                                                   h.coeffs, h.scale_mode, h.heads, h.precision)))
+        else:
+            h = g.adamw
+            groups.append(("adamw", ma.adamw_hparams(h.lr, h.beta1, h.beta2, h.eps, h.weight_decay, 1)))
+    opt = ma.MuonAdamW([(p, t.role, t.group) for p, t in zip(params, wl.tensors)], groups)
+    stream = torch.cuda.current_stream(dev)
+
+    for _ in range(args.warmup):
+        opt.step(grads)
+    torch.cuda.synchronize(dev)
+    st = ma.ma_device_status(stream)
+    if st != ma.MA_OK:
+        raise SystemExit(f"device status after warm-up: {st}")
+
+    # ---- timed region: K steps, inputs resident in HBM
+    clocks = ClockSampler(gpu_id_for(local))
+    clocks.start()
+    time.sleep(0.5)
+    barrier()
+    torch.cuda.synchronize(dev)
+    ma.ma_profile_enable(True)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        opt.step(grads)
+    t1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    ma.ma_profile_enable(False)
+    prof = ma.ma_profile_collect()
+    clk = clocks.stop()
+    ms = t0.elapsed_time(t1) / args.steps
+    launches_per_step = opt.launches
+    if world > 1:
+        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    st = ma.ma_device_status(stream)
+    if st != ma.MA_OK:
+        raise SystemExit(f"device status after the timed steps: {st}")
+    n_params = wl.numel
+    value = world * n_params / (ms / 1000.0)
+
+    # ---- end to end through the public API: gradients from pinned host memory,
+    # the step, and a read of the device status word (the step's result) each step
+    e2e = None
+    if not args.no_e2e:
+        host_grads = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in grads]
+        for hg, g in zip(host_grads, grads):
+            hg.copy_(g)
+        h2d = sum(g.numel() * g.element_size() for g in grads)
+        k_e2e = max(1, min(args.steps, 5))
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(k_e2e):
+            for g, hg in zip(grads, host_grads):
+                g.copy_(hg, non_blocking=True)
+            opt.step(grads)
+            if ma.ma_device_status(stream) != ma.MA_OK:
+                raise SystemExit("device status error in the end-to-end loop")
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        ems = e0.elapsed_time(e1) / k_e2e
+        if world > 1:
+            tt = torch.tensor([ems], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ems = float(tt.item())
+        e2e = {"value": world * n_params / (ems / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": 4, "ms_per_step": ems}
+        del host_grads
+
+    if rank == 0:
+        peaks = load_peaks()
+        ns_ms = sum(prof[c]["ms"] for c in ("ns_gram", "ns_apply", "ns_gramsq"))
+        ns_fl = sum(prof[c]["flops"] for c in ("ns_gram", "ns_apply", "ns_gramsq"))
+        ns_launches = sum(prof[c]["launches"] for c in ("ns_gram", "ns_apply", "ns_gramsq"))
+        ns_tflops = ns_fl / (ns_ms / 1000.0) / 1e12 if ns_ms > 0 else None
+        peak_t = peaks["bf16_tflops_sustained"]
+        roofline = {"kernel": "ns_tc_kernel (Newton-Schulz Gram + apply, tcgen05)", "bound": "tensor",
+                    "achieved": ns_tflops, "peak": peak_t, "unit": "TFLOP/s",
+                    "frac": ns_tflops / peak_t if ns_tflops else None,
+                    "peak_kind": f"bf16 dense, sustained ({peaks['source']})",
+                    "traffic": NS_TRAFFIC_BYTES_PER_LAUNCH,
+                    "launches": ns_launches, "avg_launch_ms": ns_ms / max(1, ns_launches),
+                    "flops_per_launch": ns_fl / max(1, ns_launches)}
+        kernels = {}
+        for c in ma.PROF_CLASSES:
+            pc = prof[c]
+            if pc["launches"] == 0:
+                continue
+            d = {"ms_per_step": pc["ms"] / args.steps, "launches_per_step": pc["launches"] / args.steps}
+            if pc["flops"] > 0:
+                d["tflops"] = pc["flops"] / (pc["ms"] / 1000.0) / 1e12
+            if pc["bytes"] > 0:
+                d["gbs"] = pc["bytes"] / (pc["ms"] / 1000.0) / 1e9
+                d["frac_hbm"] = d["gbs"] / peaks["hbm_gbs"]
+            kernels[c] = d
+        line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,0.02^2) weights, "
+                "N(0,1e-3^2) bf16 grads)", "config": workload_config(wl, world),
+                "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "roofline": roofline,
+                "kernels": kernels, "clocks": clk,
+                "precision": {"ns_operands": "bf16", "accumulate": "fp32", "state": "fp32"}}
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(wl)
+        print(json.dumps(line))
+    opt._plan.close()
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -218,6 +218,31 @@ int ma_plan_last_launches(const ma_plan_t* plan);
 
 void ma_plan_destroy(ma_plan_t* plan);
 
+/* ---------------------------------------------------------------- profiling */
+
+/* Kernel classes for ma_profile_collect. */
+#define MA_PROF_ADAMW 0         /* multi-tensor AdamW                          */
+#define MA_PROF_MOMENTUM 1      /* momentum + Nesterov + norm partials         */
+#define MA_PROF_FINALIZE 2      /* norm finalize                               */
+#define MA_PROF_NS_GRAM 3       /* Newton-Schulz A = X X^T (tcgen05 or fp32)   */
+#define MA_PROF_NS_APPLY 4      /* Newton-Schulz X' = aX + BX, final apply too */
+#define MA_PROF_NS_GRAMSQ 5     /* Newton-Schulz A^2 (c != 0 only)             */
+#define MA_PROF_CLASSES 6
+
+/* When on != 0, every kernel the library launches on this thread's current
+ * device is bracketed by two CUDA events recorded on its launch stream. Off by
+ * default; costs two event records per launch when on. */
+int ma_profile_enable(int on);
+
+/* Wait for the recorded events, then, per class (arrays of MA_PROF_CLASSES,
+ * host, any may be NULL), store the summed device time in ms, the launch
+ * count, and the algorithmic work of those launches: flops for the
+ * Newton-Schulz classes (symmetric Gram counted as m(m+1)n, apply as 2m^2n,
+ * per unit), DRAM bytes for the memory-bound classes (AdamW 26 B/element with
+ * bf16 gradients and 28 with fp32; momentum pass 12 / 14 B/element, +2 when X
+ * is fp32). Clears the record. */
+int ma_profile_collect(double* ms_out, int64_t* launches_out, double* flops_out, double* bytes_out);
+
 /* ---------------------------------------------------------------- status */
 
 /* Synchronise `stream`, return the per-device status word (MA_OK or the first

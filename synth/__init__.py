@@ -213,7 +213,9 @@ def aspect(d: int = 4096, ff: int = 14336, heads: int = 32) -> Workload:
                     "bf16 grads N(0,1e-3^2), 10% of units rank-64")
 
 
-WORKLOADS = {"tiny": tiny, "d20": d20, "square": square, "aspect": aspect, "7b": llama7b}
+WORKLOADS = {"tiny": tiny, "d20": d20, "square": square, "aspect": aspect, "7b": llama7b,
+             # 8 square 4096x4096 matrices: a few-GB case for profiler captures
+             "square8": lambda: square(8)}
 
 
 # ---------------------------------------------------------------------------

@@ -22,6 +22,25 @@ TOL_F32 = 1e-5
 TOL_STATE = 1e-6
 
 
+def f32(x: float) -> float:
+    """A hyperparameter as the library receives it: rounded to fp32, then exact in fp64."""
+    return float(np.float32(x))
+
+
+def hp32(hp):
+    """Copy of a synth MuonHP / AdamWHP with every float field rounded to fp32."""
+    import dataclasses
+    kw = {}
+    for f in dataclasses.fields(hp):
+        v = getattr(hp, f.name)
+        if isinstance(v, float):
+            v = f32(v)
+        elif f.name == "coeffs":
+            v = tuple(tuple(f32(x) for x in c) for c in v)
+        kw[f.name] = v
+    return type(hp)(**kw)
+
+
 def dev_f32(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(np.ascontiguousarray(a, dtype=np.float32)).cuda()
 

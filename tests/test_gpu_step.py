@@ -15,7 +15,7 @@ import oracle
 import synth
 import synth.device as sdev
 import adamw_hybrid_optimizer_muon_b200 as ma
-from gpu_helpers import TOL_BF16, TOL_F32, check_muon, check_state, host, momentum_terms
+from gpu_helpers import TOL_BF16, TOL_F32, check_muon, check_state, host, hp32, momentum_terms
 
 pytestmark = pytest.mark.gpu
 
@@ -37,12 +37,12 @@ def oracle_groups(wl, precision=0):
     out = []
     for g in wl.groups:
         if g.kind == synth.KIND_MUON:
-            h = g.muon
+            h = hp32(g.muon)
             out.append(dict(kind=0, lr=h.lr, beta=h.beta, weight_decay=h.weight_decay, eps=h.eps,
                             nesterov=h.nesterov, ns_steps=h.ns_steps, coeffs=h.coeffs, scale_mode=h.scale_mode,
                             heads=h.heads))
         else:
-            h = g.adamw
+            h = hp32(g.adamw)
             out.append(dict(kind=1, lr=h.lr, beta1=h.beta1, beta2=h.beta2, eps=h.eps,
                             weight_decay=h.weight_decay))
     return out
@@ -69,10 +69,10 @@ def test_tiny_two_steps_every_element(precision):
         # one oracle step from exactly the GPU's pre-step values
         st = [{"m": before_s[0][0]}, {"exp_avg": before_s[1][0], "exp_avg_sq": before_s[1][1]}]
         ref = oracle.muonadamw_step(tensors, groups, before_p, G, st, step)
-        m = wl.groups[0].muon
+        m = hp32(wl.groups[0].muon)
         check_muon(before_p[0], host(params[0]), ref[0], m.lr, m.weight_decay, TOL_F32 if precision else TOL_BF16)
         check_state(host(opt.state[0][0]), st[0]["m"], momentum_terms(before_s[0][0], G[0], m.beta), what="m")
-        a = wl.groups[1].adamw
+        a = hp32(wl.groups[1].adamw)
         tp, tm, tv = oracle.adamw_term_magnitudes(before_p[1], G[1], before_s[1][0], before_s[1][1], step, a.lr,
                                                   a.beta1, a.beta2, a.eps, a.weight_decay)
         check_state(host(params[1]), ref[1], tp, what="gain")
@@ -110,7 +110,7 @@ def _full_size_check(name, n_muon_samples=1, adamw_samples=200_000, seed=0):
         assert ma.ma_device_status() == ma.MA_OK
         for i in sample_mats:
             w0, g, m0 = snap[i]
-            grp = wl.groups[wl.tensors[i].group].muon
+            grp = hp32(wl.groups[wl.tensors[i].group].muon)
             rw, rm = oracle.muon_update(w0, g, m0, grp.lr, grp.beta, grp.weight_decay, grp.nesterov, grp.ns_steps,
                                         grp.coeffs, grp.eps, grp.scale_mode, grp.heads)
             check_muon(w0, host(params[i]), rw, grp.lr, grp.weight_decay, TOL_BF16, what=wl.tensors[i].name)
@@ -119,7 +119,7 @@ def _full_size_check(name, n_muon_samples=1, adamw_samples=200_000, seed=0):
             sel, p0, g, s0, s1 = idx[i]
             flat = lambda x: x.reshape(-1)[sel]  # noqa: E731
             if kinds[i] == 1:
-                a = wl.groups[t.group].adamw
+                a = hp32(wl.groups[t.group].adamw)
                 rp, rm, rv = oracle.adamw_update(p0, g, s0, s1, step, a.lr, a.beta1, a.beta2, a.eps, a.weight_decay)
                 tp, tm, tv = oracle.adamw_term_magnitudes(p0, g, s0, s1, step, a.lr, a.beta1, a.beta2, a.eps,
                                                           a.weight_decay)
@@ -127,7 +127,7 @@ def _full_size_check(name, n_muon_samples=1, adamw_samples=200_000, seed=0):
                 check_state(host(flat(opt.state[i][0])), rm, tm, what=t.name + ".exp_avg")
                 check_state(host(flat(opt.state[i][1])), rv, tv, what=t.name + ".exp_avg_sq")
             else:
-                grp = wl.groups[t.group].muon
+                grp = hp32(wl.groups[t.group].muon)
                 rm, _ = oracle.momentum_update(s0, g, grp.beta, grp.nesterov)
                 check_state(host(flat(opt.state[i][0])), rm, momentum_terms(s0, g, grp.beta),
                             what=t.name + ".m")
