@@ -19,6 +19,7 @@ __all__ = [
     "ns_iterate_workspace_bytes", "ns_iterate_bf16", "adamw_step_fused", "ma_plan_create", "muonadamw_step",
     "ma_plan_destroy", "ma_device_status", "ma_set_wait_limit_ns", "ma_selftest_wait_timeout", "Plan",
     "MuonAdamW", "muon_hparams", "adamw_hparams", "ma_profile_enable", "ma_profile_collect", "PROF_CLASSES",
+    "muon_step_batched_noalloc", "STATIC_SCRATCH_BYTES",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -106,6 +107,7 @@ def lib() -> ctypes.CDLL:
         "ma_device_status": (i32, [vp, i32]),
         "ma_set_wait_limit_ns": (i32, [i64]),
         "ma_selftest_wait_timeout": (i32, [i64, vp]),
+        "muon_step_batched_noalloc": (i32, [i32, i64, i64, pp, pp, i32, pp, ctypes.POINTER(MuonHParams), vp]),
         "ma_profile_enable": (i32, [i32]),
         "ma_profile_collect": (i32, [ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_int64),
                                      ctypes.POINTER(ctypes.c_double), ctypes.POINTER(ctypes.c_double)]),
@@ -229,6 +231,27 @@ def muon_step_batched(W, G, M, hp: MuonHParams, ws, ws_bytes: int | None = None,
     _check(lib().muon_step_batched(batch, R, C, _ptr_array(W), _ptr_array(G), int(gdt), _ptr_array(M),
                                    ctypes.byref(hp), _ptr(ws), int(ws_bytes), _stream(stream)),
            "muon_step_batched")
+
+
+STATIC_SCRATCH_BYTES = 64 << 20  # MA_STATIC_SCRATCH_BYTES
+
+
+def muon_step_batched_noalloc(W, G, M, hp: MuonHParams, stream=None, gdt: int | None = None, shape=None) -> None:
+    """muon_step_batched without a workspace argument: for callers that cannot
+    allocate device memory. Its scratch is the library's fixed device array of
+    STATIC_SCRATCH_BYTES per GPU, shared by every call: calls that overlap on
+    the GPU race. The first call on a device looks up the array's address and
+    should come before any stream capture. Raises MAError(MA_ERR_WORKSPACE)
+    when the step needs more scratch than the array holds."""
+    batch = len(W)
+    if shape is None:
+        R, C = (int(W[0].shape[0]), int(W[0].shape[1])) if batch else (0, 0)
+    else:
+        R, C = int(shape[0]), int(shape[1])
+    if gdt is None:
+        gdt = _dtype_code(G[0]) if batch else MA_F32
+    _check(lib().muon_step_batched_noalloc(batch, R, C, _ptr_array(W), _ptr_array(G), int(gdt), _ptr_array(M),
+                                           ctypes.byref(hp), _stream(stream)), "muon_step_batched_noalloc")
 
 
 def ns_iterate_workspace_bytes(batch: int, m: int, n: int) -> int:

@@ -888,3 +888,42 @@ int ma_selftest_wait_timeout(int64_t limit_ns, void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------- allocation-free Muon step
+//
+// For callers that cannot call cudaMalloc (see muonadamw.h): the scratch that
+// muon_step_batched takes from the caller lives here, in one file-scope
+// device array per GPU. The kernels and their order are exactly those of
+// muon_step_batched; only the scratch base pointer differs.
+
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MA_STATIC_SCRATCH_BYTES];
+
+// Device address of g_noalloc_scratch on the current device, looked up once per
+// device (host code only has a host-side stand-in for the symbol, which must
+// never be handed to a kernel). NULL if the lookup fails.
+static void* noalloc_scratch_ptr() {
+    static void* cached[64] = {nullptr};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!cached[dev]) {
+        void* ptr = nullptr;
+        if (cudaGetSymbolAddress((void**)&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
+        cached[dev] = ptr;
+    }
+    return cached[dev];
+}
+
+extern "C" int muon_step_batched_noalloc(int batch, int64_t R, int64_t C, float* const* W, const void* const* G,
+                                         int gdt, float* const* M, const ma_muon_hparams_t* hp, void* stream) {
+    MuonGeom g;
+    int st = check_muon_call(batch, R, C, W, G, gdt, M, hp, &g);
+    if (st) return st;
+    if (g.total == 0) return MA_OK;
+    if (g.total > MA_STATIC_SCRATCH_BYTES) return MA_ERR_WORKSPACE;
+    int sms = 0;
+    if ((st = device_ok_and_sms(&sms))) return st;
+    void* scratch = noalloc_scratch_ptr();
+    if (!scratch) return MA_ERR_CUDA;
+    int launches = 0;
+    return run_muon(batch, g, W, G, gdt, M, *hp, scratch, reinterpret_cast<cudaStream_t>(stream), sms, &launches);
+}

@@ -185,6 +185,29 @@ int ns_iterate_bf16(int batch, int64_t m, int64_t n, const uint16_t* X_in, uint1
                     const float* coeffs, int n_coeffs, int steps, void* ws, size_t ws_bytes,
                     void* stream);
 
+/* Muon step without a caller workspace. The paper has no counterpart; this
+ * entry point exists for callers that cannot call cudaMalloc: plugins and hooks
+ * inside a host framework that owns the device allocator and hands out no
+ * scratch buffer, processes that reserve all their memory up front under a
+ * fixed budget, and loops that cannot accept the device-wide synchronisation a
+ * cudaMalloc may cause. Same arguments and results as muon_step_batched, minus
+ * ws/ws_bytes. Its scratch is a file-scope device array of
+ * MA_STATIC_SCRATCH_BYTES, which every GPU that loads the library holds until
+ * the process exits.
+ *  - Limit: returns MA_ERR_WORKSPACE, before launching anything, when
+ *    muon_workspace_bytes(batch, R, C, hp) > MA_STATIC_SCRATCH_BYTES.
+ *  - Set-up: the first call on each device looks up the array's device
+ *    address (cudaGetSymbolAddress) with that device current; make that first
+ *    call before any stream capture begins.
+ *  - Sharing: every call on a device uses the same array and leaves its
+ *    contents behind. Nothing in it needs to start at zero (each call writes
+ *    every scratch value before reading it), but calls that overlap on the GPU
+ *    (different streams, or different host threads) race on it.
+ *  - Allocates nothing: no cudaMalloc, cudaFree or allocating library call. */
+#define MA_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
+int muon_step_batched_noalloc(int batch, int64_t R, int64_t C, float* const* W, const void* const* G,
+                              int gdt, float* const* M, const ma_muon_hparams_t* hp, void* stream);
+
 /* ---------------------------------------------------------------- AdamW */
 
 /* One AdamW step on n tensors in one multi-tensor launch sequence
