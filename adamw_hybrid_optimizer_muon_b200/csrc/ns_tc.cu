@@ -17,20 +17,22 @@
 //           caller's fp32 weights, transposing back when the unit was tall.
 //           X_N is never rounded or stored.
 //
-// Kernel structure (one CTA per SM, persistent over the tiles of all units of
-// a batch):
-//   warp 0      TMA producer: 128B-swizzled 3-D bulk tensor loads into a
-//               4-stage ring (A tile 128x64, B tile 256x64 bf16 = 48 KB per stage)
-//   warp 1      TMEM allocator and MMA issuer: tcgen05.mma kind::f16, M=128,
-//               N=256, K=16 per instruction, fp32 accumulators in TMEM, two
-//               accumulator buffers (2 x 256 columns) so the epilogue of one
-//               tile overlaps the main loop of the next
-//   warps 2..5  epilogue: tcgen05.ld 32 columns at a time, fused polynomial
-//               combine, bf16 rounding, stores
-// Every mbarrier wait is bounded (see common.cuh). On a timeout the block
-// records MA_ERR_TIMEOUT, lets in-flight copies and MMAs drain (also bounded),
-// frees its TMEM and returns.
-//
+// Kernel structure: CTA pairs (clusters of 2), persistent over the 256 x 256
+// output tiles of all units of a batch, 320 threads per CTA:
+//   warp 0      TMA producer in each CTA: this CTA's half of the A tile
+//               (128 rows x 64) and of the B tile (128 columns x 64), bf16,
+//               128B swizzle, 6 stages of 32 KB. Both CTAs' loads complete on
+//               the leader CTA's stage barrier; there is no multicast.
+//   warp 1      TMEM allocation in both CTAs (cta_group::2, 2 x 256 fp32
+//               columns). In the leader only, MMA issue:
+//               tcgen05.mma.cta_group::2.kind::f16, M = 256 (128 rows in each
+//               CTA), N = 256, K = 16. Commits are multicast to both CTAs'
+//               barriers: stage release and accumulator full.
+//   warps 2..9  epilogue in both CTAs: each TMEM lane quadrant is read by two
+//               warps, each taking half of the 256 columns, 32 at a time.
+// Per unit of tile work, the pair moves (256 + 256) x 64 x 2 bytes from L2 for
+// 256 x 256 x 64 multiply-adds: one third fewer bytes per flop than a
+// single-CTA 128 x 256 tile.
 // B operand major-ness: for GRAM and GRAMSQ both operands are K-major rows of
 // the same matrix. For APPLY the B operand is X itself, read MN-major (the
 // contraction runs over X's rows), so no transposed copy is ever made.
@@ -41,29 +43,31 @@ namespace ma {
 
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr uint32_t A_BYTES = BM * BK * 2;             // 16 KB
-constexpr uint32_t B_BYTES = BN * BK * 2;             // 32 KB
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;   // 48 KB
-constexpr uint32_t TMEM_COLS = 2 * BN;                // two fp32 accumulators
+constexpr int BM = 256, BN = 256, BK = 64, STAGES = 6;
+constexpr int HM = BM / 2, HN = BN / 2;                // rows of A / columns of B held by each CTA
+constexpr uint32_t A_BYTES = HM * BK * 2;              // 16 KB
+constexpr uint32_t B_BYTES = HN * BK * 2;              // 16 KB
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;    // 32 KB per CTA
+constexpr uint32_t TMEM_COLS = 2 * BN;                 // two fp32 accumulators
+constexpr int EPI_WARPS = 8;
+constexpr int THREADS = 32 * (2 + EPI_WARPS);
 constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 
 struct TileCoord {
     int u, ti, tj;
 };
 
-// Tiles of one unit. GRAM/GRAMSQ: only (ti, tj) whose 128x256 block holds an
-// element with row <= col, i.e. ti <= 2*tj + 1, enumerated column by column.
+// Tiles of one unit. GRAM/GRAMSQ: only the tiles (ti, tj) with ti <= tj, the
+// ones that hold an element with row <= col, enumerated column by column.
 __device__ __forceinline__ TileCoord decode_tile(int mode, int t, int tiles_per_unit, int mt, int nt) {
     TileCoord c;
     c.u = t / tiles_per_unit;
     int r = t - c.u * tiles_per_unit;
     if (mode == NS_GRAM || mode == NS_GRAMSQ) {
         int tj = 0;
-        for (;; ++tj) {
-            const int cnt = min(2 * tj + 2, mt);
-            if (r < cnt || tj == nt - 1) break;
-            r -= cnt;
+        while (r >= tj + 1 && tj < nt - 1) {
+            r -= tj + 1;
+            ++tj;
         }
         c.ti = r;
         c.tj = tj;
@@ -208,7 +212,7 @@ __device__ __forceinline__ void epilogue_chunk(const NsParams& p, const TileCoor
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(THREADS, 1)
     ns_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
                  const __grid_constant__ NsParams p, int tiles_per_unit, int mt, int nt, int kblocks) {
     extern __shared__ uint8_t smem_raw[];
@@ -220,35 +224,36 @@ __global__ void __launch_bounds__(192, 1)
     uint64_t* drain = acc_empty + 2;
     uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-    int* counters = const_cast<int*>(abort_flag) + 1;  // [0] loads issued, [1] loads consumed
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();  // 0 = leader of the pair
+    const bool leader = rank == 0;
+    const int pair = (int)cluster_id_x(), npairs = (int)cluster_count_x();
     const int total_tiles = p.units * tiles_per_unit;
     const long long limit = p.wait_limit_ns;
+    constexpr bool kApply = (MODE == NS_APPLY || MODE == NS_FINAL);
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], 1);
+            mbar_init(&full[s], 1);   // leader: its own arrive.expect_tx + both CTAs' bytes
+            mbar_init(&empty[s], 1);  // both: one multicast commit per use
         }
         for (int a = 0; a < 2; ++a) {
-            mbar_init(&acc_full[a], 1);
-            mbar_init(&acc_empty[a], 4);
+            mbar_init(&acc_full[a], 1);                  // both: one multicast commit per tile
+            mbar_init(&acc_empty[a], 2 * EPI_WARPS);     // leader: every epilogue warp of the pair
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
-        counters[0] = 0;
-        counters[1] = 0;
         fence_barrier_init();
         prefetch_tensormap(&mapA);
         prefetch_tensormap(&mapB);
     }
     if (warp == 1) {
-        tmem_alloc(tmem_holder, TMEM_COLS);
-        tmem_relinquish();
+        tmem_alloc_pair(tmem_holder, TMEM_COLS);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated in both
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
@@ -256,10 +261,11 @@ __global__ void __launch_bounds__(192, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            int issued = 0;
-            for (int t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+            bool ok = true;
+            for (int t = pair; t < total_tiles && ok; t += npairs) {
                 const TileCoord tc = decode_tile(MODE, t, tiles_per_unit, mt, nt);
-                bool ok = true;
+                const int arow = tc.ti * BM + (int)rank * HM;
+                const int bcol = tc.tj * BN + (int)rank * HN;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit, p.status)) {
                         ok = false;
@@ -267,35 +273,40 @@ __global__ void __launch_bounds__(192, 1)
                     }
                     uint8_t* sa = smem + stage * STAGE_BYTES;
                     uint8_t* sb = sa + A_BYTES;
-                    mbar_arrive_expect_tx(&full[stage], STAGE_BYTES);
-                    tma_load_3d(sa, &mapA, &full[stage], kb * BK, tc.ti * BM, tc.u);
-                    if (MODE == NS_GRAM || MODE == NS_GRAMSQ) {
-                        tma_load_3d(sb, &mapB, &full[stage], kb * BK, tc.tj * BN, tc.u);
+                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+                    const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+                    tma_load_3d_pair(sa, &mapA, fb, kb * BK, arow, tc.u);
+                    if (!kApply) {
+                        tma_load_3d_pair(sb, &mapB, fb, kb * BK, bcol, tc.u);
                     } else {
 #pragma unroll
-                        for (int q = 0; q < BN / 64; ++q)
-                            tma_load_3d(sb + q * (64 * BK * 2), &mapB, &full[stage], tc.tj * BN + q * 64, kb * BK,
-                                        tc.u);
+                        for (int q = 0; q < HN / 64; ++q)
+                            tma_load_3d_pair(sb + q * (64 * BK * 2), &mapB, fb, bcol + q * 64, kb * BK, tc.u);
                     }
-                    ++issued;
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
-                if (!ok) break;
             }
-            counters[0] = issued;
+            // Tail: wait until the MMAs have released every stage this CTA filled,
+            // so that no commit arrives on this CTA's barriers after it exits.
+            for (int i = 0; i < STAGES && ok; ++i) {
+                ok = mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit, p.status);
+                if (++stage == STAGES) {
+                    stage = 0;
+                    phase ^= 1u;
+                }
+            }
         }
     } else if (warp == 1) {
-        if (lane == 0) {
-            constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, (MODE == NS_APPLY || MODE == NS_FINAL) ? 1 : 0);
+        if (lane == 0 && leader) {
+            constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, kApply ? 1 : 0);
             int stage = 0;
             uint32_t phase = 0;
-            int consumed = 0;
             int lt = 0;
             bool ok = true;
-            for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++lt) {
+            for (int t = pair; t < total_tiles && ok; t += npairs, ++lt) {
                 const int acc = lt & 1;
                 const uint32_t use = (uint32_t)(lt >> 1);
                 if (!mbar_wait_bounded(&acc_empty[acc], (use & 1u) ^ 1u, abort_flag, limit, p.status)) {
@@ -316,33 +327,34 @@ __global__ void __launch_bounds__(192, 1)
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
                         uint64_t bdesc;
-                        if (MODE == NS_APPLY || MODE == NS_FINAL)
+                        if (kApply)
                             bdesc = smem_desc_sw128(b0 + kk * (16 * 128), 64 * BK * 2, 1024);
                         else
                             bdesc = smem_desc_sw128(b0 + kk * 32, 16, 1024);
-                        tc_mma_f16(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                        tc_mma_f16_pair(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
                     }
-                    tc_commit(&empty[stage]);
-                    ++consumed;
+                    tc_commit_pair_mc(&empty[stage], 0x3);
                     if (++stage == STAGES) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                tc_commit(&acc_full[acc]);
+                tc_commit_pair_mc(&acc_full[acc], 0x3);
             }
-            counters[1] = consumed;
             if (!ok) {
                 // let every MMA issued so far finish before TMEM is released
-                tc_commit(drain);
+                tc_commit_pair(drain);
                 mbar_wait_bounded(drain, 0, abort_flag, limit, p.status);
             }
         }
     } else {
-        const int quad = warp & 3;  // TMEM lanes [32*quad, 32*quad + 32)
+        const int quad = warp & 3;              // TMEM lanes [32*quad, 32*quad + 32)
+        const int half = (warp - 2) / 4;        // which half of the 256 columns
+        const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
+        const uint32_t acc_empty_leader1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
         int lt = 0;
-        for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++lt) {
+        for (int t = pair; t < total_tiles; t += npairs, ++lt) {
             const TileCoord tc = decode_tile(MODE, t, tiles_per_unit, mt, nt);
             const int acc = lt & 1;
             const uint32_t use = (uint32_t)(lt >> 1);
@@ -351,34 +363,36 @@ __global__ void __launch_bounds__(192, 1)
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after();
-            const int row = tc.ti * BM + quad * 32 + lane;
-            const int row_lo = tc.ti * BM + quad * 32;
-            const int limit_cols = (MODE == NS_APPLY || MODE == NS_FINAL) ? p.n : p.m;
+            const int row_lo = tc.ti * BM + (int)rank * HM + quad * 32;
+            const int row = row_lo + lane;
+            const int limit_cols = kApply ? p.n : p.m;
 #pragma unroll 1
-            for (int cc = 0; cc < BN / 32; ++cc) {
+            for (int cc = half * 4; cc < half * 4 + 4; ++cc) {
                 const int col0 = tc.tj * BN + cc * 32;
-                if (col0 >= limit_cols) break;                                            // warp-uniform
-                if ((MODE == NS_GRAM || MODE == NS_GRAMSQ) && col0 + 31 < row_lo) continue;  // below diagonal
+                if (col0 >= limit_cols) break;                                    // warp-uniform
+                if (!kApply && col0 + 31 < row_lo) continue;                     // below the diagonal
                 float v[32];
                 tmem_ld32(tmem_base + (uint32_t)(acc * BN + cc * 32) + ((uint32_t)(quad * 32) << 16), v);
                 epilogue_chunk<MODE>(p, tc, row, col0, v);
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[acc]);
+            if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);
         }
     }
 
     __syncthreads();
     if (threadIdx.x == 0 && *abort_flag) {
-        // loads that were issued but never consumed must land before the block exits
-        for (int k = counters[1]; k < counters[0]; ++k)
-            mbar_wait_bounded(&full[k % STAGES], (uint32_t)((k / STAGES) & 1), abort_flag, limit, p.status);
+        // give this CTA's own bulk copies that may still be in flight time to land
+        const uint64_t t0 = globaltimer();
+        while (globaltimer() - t0 < 200000ull) {
+        }
     }
-    __syncthreads();
+    tc_fence_before();
+    cluster_sync_all();  // neither CTA leaves while the pair may still touch its memory
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, TMEM_COLS);
+        tmem_dealloc_pair(tmem_base, TMEM_COLS);
     }
 }
 
@@ -419,29 +433,27 @@ cudaError_t launch_mode(const NsParams& p, const void* x_buf, const void* g_buf,
     int kblocks, mt, nt, tiles;
     mt = (p.m + BM - 1) / BM;
     if (MODE == NS_GRAM || MODE == NS_GRAMSQ) {
-        nt = (p.m + BN - 1) / BN;
-        tiles = 0;
-        for (int tj = 0; tj < nt; ++tj) tiles += (2 * tj + 2 < mt) ? 2 * tj + 2 : mt;
+        nt = mt;
+        tiles = nt * (nt + 1) / 2;
         if (MODE == NS_GRAM) {
             kblocks = (p.n + BK - 1) / BK;
-            if (!make_map(&mA, x_buf, p.n, p.m, p.units, p.ldx, p.x_unit, BK, BM)) return cudaErrorInvalidValue;
-            if (!make_map(&mB, x_buf, p.n, p.m, p.units, p.ldx, p.x_unit, BK, BN)) return cudaErrorInvalidValue;
+            if (!make_map(&mA, x_buf, p.n, p.m, p.units, p.ldx, p.x_unit, BK, HM)) return cudaErrorInvalidValue;
         } else {
             kblocks = (p.m + BK - 1) / BK;
-            if (!make_map(&mA, p.xin, p.m, p.m, p.units, p.ldg, p.g_unit, BK, BM)) return cudaErrorInvalidValue;
-            if (!make_map(&mB, p.xin, p.m, p.m, p.units, p.ldg, p.g_unit, BK, BN)) return cudaErrorInvalidValue;
+            if (!make_map(&mA, p.xin, p.m, p.m, p.units, p.ldg, p.g_unit, BK, HM)) return cudaErrorInvalidValue;
         }
+        mB = mA;  // both operands are 128-row, 64-deep K-major boxes of the same matrix
     } else {
         nt = (p.n + BN - 1) / BN;
         tiles = mt * nt;
         kblocks = (p.m + BK - 1) / BK;
-        if (!make_map(&mA, g_buf, p.m, p.m, p.units, p.ldg, p.g_unit, BK, BM)) return cudaErrorInvalidValue;
+        if (!make_map(&mA, g_buf, p.m, p.m, p.units, p.ldg, p.g_unit, BK, HM)) return cudaErrorInvalidValue;
         if (!make_map(&mB, x_buf, p.n, p.m, p.units, p.ldx, p.x_unit, 64, BK)) return cudaErrorInvalidValue;
     }
     const long long total = (long long)tiles * p.units;
     if (total <= 0) return cudaSuccess;
-    const int grid = (int)(total < num_sms ? total : num_sms);
     static unsigned long long attr_set = 0;  // one bit per device
+    static int max_pairs[64] = {0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -449,10 +461,40 @@ cudaError_t launch_mode(const NsParams& p, const void* x_buf, const void* g_buf,
     if (!(attr_set & (1ull << dev))) {
         e = cudaFuncSetAttribute(ns_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
         if (e != cudaSuccess) return e;
+        e = cudaFuncSetAttribute(ns_tc_kernel<MODE>, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
+        if (e != cudaSuccess) return e;
+        cudaLaunchConfig_t qc = {};
+        cudaLaunchAttribute qa[1];
+        qa[0].id = cudaLaunchAttributeClusterDimension;
+        qa[0].val.clusterDim.x = 2;
+        qa[0].val.clusterDim.y = 1;
+        qa[0].val.clusterDim.z = 1;
+        qc.gridDim = dim3(2 * (unsigned)(num_sms / 2));
+        qc.blockDim = dim3(THREADS);
+        qc.dynamicSmemBytes = SMEM_BYTES;
+        qc.attrs = qa;
+        qc.numAttrs = 1;
+        int nclusters = 0;
+        e = cudaOccupancyMaxActiveClusters(&nclusters, ns_tc_kernel<MODE>, &qc);
+        if (e != cudaSuccess) return e;
+        if (nclusters < 1) return cudaErrorInvalidConfiguration;
+        max_pairs[dev] = nclusters;
         attr_set |= 1ull << dev;
     }
-    ns_tc_kernel<MODE><<<grid, 192, SMEM_BYTES, s>>>(mA, mB, p, tiles, mt, nt, kblocks);
-    return cudaGetLastError();
+    const long long pairs = total < max_pairs[dev] ? total : max_pairs[dev];
+    cudaLaunchConfig_t cfg = {};
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 2;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    cfg.blockDim = dim3(THREADS);
+    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.stream = s;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, ns_tc_kernel<MODE>, mA, mB, p, tiles, mt, nt, kblocks);
 }
 
 }  // namespace
