@@ -42,8 +42,55 @@ __device__ __forceinline__ float block_sum_256(float v, float* red) {
     return t;
 }
 
+template <bool GBF16>
+__device__ __forceinline__ void load_g8(const void* G, int64_t i, float (&g)[8]) {
+    if (GBF16) {
+        const uint4 w = __ldcs(reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(G) + i));
+        g[0] = bf16_lo(w.x); g[1] = bf16_hi(w.x); g[2] = bf16_lo(w.y); g[3] = bf16_hi(w.y);
+        g[4] = bf16_lo(w.z); g[5] = bf16_hi(w.z); g[6] = bf16_lo(w.w); g[7] = bf16_hi(w.w);
+    } else {
+        const float4* gp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(G) + i);
+        const float4 a = __ldcs(gp), c = __ldcs(gp + 1);
+        g[0] = a.x; g[1] = a.y; g[2] = a.z; g[3] = a.w; g[4] = c.x; g[5] = c.y; g[6] = c.z; g[7] = c.w;
+    }
+}
+
+// m <- beta*m + (1-beta)*g on 8 elements; d <- the direction; returns sum of d^2.
+__device__ __forceinline__ float momentum8(float (&m)[8], const float (&g)[8], float (&d)[8], float beta, float omb,
+                                           bool nesterov) {
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        m[k] = beta * m[k] + omb * g[k];
+        d[k] = nesterov ? beta * m[k] + omb * g[k] : m[k];
+        ss += d[k] * d[k];
+    }
+    return ss;
+}
+
+template <bool XF32>
+__device__ __forceinline__ void store_x8(void* X, int64_t i, const float (&d)[8]) {
+    if (XF32) {
+        float4* xp = reinterpret_cast<float4*>(reinterpret_cast<float*>(X) + i);
+        __stcs(xp, make_float4(d[0], d[1], d[2], d[3]));
+        __stcs(xp + 1, make_float4(d[4], d[5], d[6], d[7]));
+    } else {
+        uint4 w;
+        w.x = pack_bf16x2(d[0], d[1]);
+        w.y = pack_bf16x2(d[2], d[3]);
+        w.z = pack_bf16x2(d[4], d[5]);
+        w.w = pack_bf16x2(d[6], d[7]);
+        __stcs(reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(X) + i), w);
+    }
+}
+
+// Flat path: one block per 8192-element chunk of one unit. A full chunk issues
+// all of its loads (4 groups of 8 elements per thread) before any arithmetic,
+// so each thread keeps 12 independent 16-byte loads in flight.
+template <bool GBF16, bool XF32>
 __global__ void __launch_bounds__(256) prep_flat_kernel(const __grid_constant__ MuonPrepLaunch L) {
     __shared__ float red[8];
+    constexpr int kIter = kPrepChunk / (8 * 256);
     const int u = blockIdx.y;
     const int b = u / L.heads, h = u % L.heads;
     const int64_t unit_elems = L.Rh * L.C;
@@ -51,91 +98,144 @@ __global__ void __launch_bounds__(256) prep_flat_kernel(const __grid_constant__ 
     const int64_t start = (int64_t)blockIdx.x * kPrepChunk;
     const int64_t end = min(start + (int64_t)kPrepChunk, unit_elems);
     float* M = L.M[b] + off;
+    const void* G = GBF16 ? static_cast<const void*>(reinterpret_cast<const uint16_t*>(L.G[b]) + off)
+                          : static_cast<const void*>(reinterpret_cast<const float*>(L.G[b]) + off);
+    void* X = XF32 ? static_cast<void*>(reinterpret_cast<float*>(L.X) + (int64_t)u * L.x_unit)
+                   : static_cast<void*>(reinterpret_cast<uint16_t*>(L.X) + (int64_t)u * L.x_unit);
     const float beta = L.beta, omb = L.omb;
+    const bool nest = L.nesterov != 0;
     float ss = 0.f;
-    for (int64_t i = start + 8 * (int64_t)threadIdx.x; i < end; i += 8 * 256) {
-        float g[8];
-        if (L.gdt == MA_BF16) {
-            const uint4 w = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(L.G[b]) + off + i);
-            g[0] = bf16_lo(w.x); g[1] = bf16_hi(w.x); g[2] = bf16_lo(w.y); g[3] = bf16_hi(w.y);
-            g[4] = bf16_lo(w.z); g[5] = bf16_hi(w.z); g[6] = bf16_lo(w.w); g[7] = bf16_hi(w.w);
-        } else {
-            const float* gp = reinterpret_cast<const float*>(L.G[b]) + off + i;
-            const float4 a = *reinterpret_cast<const float4*>(gp);
-            const float4 c = *reinterpret_cast<const float4*>(gp + 4);
-            g[0] = a.x; g[1] = a.y; g[2] = a.z; g[3] = a.w; g[4] = c.x; g[5] = c.y; g[6] = c.z; g[7] = c.w;
-        }
-        float4 m0 = *reinterpret_cast<const float4*>(M + i);
-        float4 m1 = *reinterpret_cast<const float4*>(M + i + 4);
-        float m[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
-        float d[8];
+    if (end - start == kPrepChunk) {
+        float g[kIter][8], m[kIter][8];
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
-            m[k] = beta * m[k] + omb * g[k];
-            d[k] = L.nesterov ? beta * m[k] + omb * g[k] : m[k];
-            ss += d[k] * d[k];
+        for (int k = 0; k < kIter; ++k) {
+            const int64_t i = start + 8 * ((int64_t)k * 256 + threadIdx.x);
+            load_g8<GBF16>(G, i, g[k]);
+            const float4 a = __ldcs(reinterpret_cast<const float4*>(M + i));
+            const float4 c = __ldcs(reinterpret_cast<const float4*>(M + i + 4));
+            m[k][0] = a.x; m[k][1] = a.y; m[k][2] = a.z; m[k][3] = a.w;
+            m[k][4] = c.x; m[k][5] = c.y; m[k][6] = c.z; m[k][7] = c.w;
         }
-        *reinterpret_cast<float4*>(M + i) = make_float4(m[0], m[1], m[2], m[3]);
-        *reinterpret_cast<float4*>(M + i + 4) = make_float4(m[4], m[5], m[6], m[7]);
-        if (L.x_f32) {
-            float* X = reinterpret_cast<float*>(L.X) + (int64_t)u * L.x_unit + i;
-            *reinterpret_cast<float4*>(X) = make_float4(d[0], d[1], d[2], d[3]);
-            *reinterpret_cast<float4*>(X + 4) = make_float4(d[4], d[5], d[6], d[7]);
-        } else {
-            uint16_t* X = reinterpret_cast<uint16_t*>(L.X) + (int64_t)u * L.x_unit + i;
-            uint4 w;
-            w.x = pack_bf16x2(d[0], d[1]);
-            w.y = pack_bf16x2(d[2], d[3]);
-            w.z = pack_bf16x2(d[4], d[5]);
-            w.w = pack_bf16x2(d[6], d[7]);
-            *reinterpret_cast<uint4*>(X) = w;
+#pragma unroll
+        for (int k = 0; k < kIter; ++k) {
+            const int64_t i = start + 8 * ((int64_t)k * 256 + threadIdx.x);
+            float d[8];
+            ss += momentum8(m[k], g[k], d, beta, omb, nest);
+            __stcs(reinterpret_cast<float4*>(M + i), make_float4(m[k][0], m[k][1], m[k][2], m[k][3]));
+            __stcs(reinterpret_cast<float4*>(M + i + 4), make_float4(m[k][4], m[k][5], m[k][6], m[k][7]));
+            store_x8<XF32>(X, i, d);
+        }
+    } else {
+        for (int64_t i = start + 8 * (int64_t)threadIdx.x; i < end; i += 8 * 256) {
+            float g[8], m[8], d[8];
+            load_g8<GBF16>(G, i, g);
+            const float4 a = __ldcs(reinterpret_cast<const float4*>(M + i));
+            const float4 c = __ldcs(reinterpret_cast<const float4*>(M + i + 4));
+            m[0] = a.x; m[1] = a.y; m[2] = a.z; m[3] = a.w; m[4] = c.x; m[5] = c.y; m[6] = c.z; m[7] = c.w;
+            ss += momentum8(m, g, d, beta, omb, nest);
+            __stcs(reinterpret_cast<float4*>(M + i), make_float4(m[0], m[1], m[2], m[3]));
+            __stcs(reinterpret_cast<float4*>(M + i + 4), make_float4(m[4], m[5], m[6], m[7]));
+            store_x8<XF32>(X, i, d);
         }
     }
     const float tot = block_sum_256(ss, red);
     if (threadIdx.x == 0) L.partials[(int64_t)u * L.parts + blockIdx.x] = (double)tot;
 }
 
+// Transposing path (tall units, X = u^T). A 64 x 64 tile: each thread reads
+// four 4-wide vectors along a row of u (a warp covers two 256-byte row
+// segments), the tile turns in shared memory, and each row of X gets 64
+// consecutive values (128 bytes of bf16) written as 16-byte vectors.
+template <bool GBF16, bool XF32>
 __global__ void __launch_bounds__(256) prep_transpose_kernel(const __grid_constant__ MuonPrepLaunch L) {
-    __shared__ float tile[kPrepTile][kPrepTile + 1];
+    __shared__ float tile[kPrepTile][kPrepTile + 1];  // [column of u][row of u]
     __shared__ float red[8];
     const int u = blockIdx.y;
     const int b = u / L.heads, h = u % L.heads;
     const int64_t off = (int64_t)h * L.Rh * L.C;
     const int64_t tr = blockIdx.x / L.tiles_c, tc = blockIdx.x % L.tiles_c;
     const int64_t r0 = tr * kPrepTile, c0 = tc * kPrepTile;
-    const int col = threadIdx.x & 63, rsub = threadIdx.x >> 6;
+    const int t = threadIdx.x;
     float* M = L.M[b] + off;
     const float beta = L.beta, omb = L.omb;
+    const bool nest = L.nesterov != 0;
     float ss = 0.f;
-#pragma unroll 4
-    for (int k = 0; k < 16; ++k) {
-        const int rl = rsub + 4 * k;
-        const int64_t r = r0 + rl, c = c0 + col;
-        float d = 0.f;
-        if (r < L.Rh && c < L.C) {
-            const int64_t idx = r * L.C + c;
-            float g;
-            if (L.gdt == MA_BF16)
-                g = __uint_as_float(uint32_t(reinterpret_cast<const uint16_t*>(L.G[b])[off + idx]) << 16);
-            else
-                g = reinterpret_cast<const float*>(L.G[b])[off + idx];
-            float m = beta * M[idx] + omb * g;
-            M[idx] = m;
-            d = L.nesterov ? beta * m + omb * g : m;
-            ss += d * d;
+    {
+        const int cl = (t & 15) * 4;  // C % 8 == 0, so a 4-wide vector never straddles the row end
+        const int64_t c = c0 + cl;
+        float g[4][4], m[4][4];
+        bool in[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int rl = (t >> 4) + 16 * k;
+            const int64_t r = r0 + rl;
+            in[k] = (r < L.Rh) && (c < L.C);
+            if (in[k]) {
+                const int64_t idx = r * L.C + c;
+                if (GBF16) {
+                    const uint2 w = __ldcs(reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(L.G[b]) +
+                                                                          off + idx));
+                    g[k][0] = bf16_lo(w.x); g[k][1] = bf16_hi(w.x); g[k][2] = bf16_lo(w.y); g[k][3] = bf16_hi(w.y);
+                } else {
+                    const float4 w =
+                        __ldcs(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(L.G[b]) + off + idx));
+                    g[k][0] = w.x; g[k][1] = w.y; g[k][2] = w.z; g[k][3] = w.w;
+                }
+                const float4 mv = __ldcs(reinterpret_cast<const float4*>(M + idx));
+                m[k][0] = mv.x; m[k][1] = mv.y; m[k][2] = mv.z; m[k][3] = mv.w;
+            }
         }
-        tile[rl][col] = d;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int rl = (t >> 4) + 16 * k;
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            if (in[k]) {
+                const int64_t idx = (r0 + rl) * L.C + c;
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    m[k][j] = beta * m[k][j] + omb * g[k][j];
+                    d[j] = nest ? beta * m[k][j] + omb * g[k][j] : m[k][j];
+                    ss += d[j] * d[j];
+                }
+                __stcs(reinterpret_cast<float4*>(M + idx), make_float4(m[k][0], m[k][1], m[k][2], m[k][3]));
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) tile[cl + j][rl] = d[j];
+        }
     }
     __syncthreads();
-#pragma unroll 4
-    for (int k = 0; k < 16; ++k) {
-        const int cl = rsub + 4 * k;
-        const int64_t xr = c0 + cl, xc = r0 + col;  // X = u^T: row = original column
-        if (xr < L.C && xc < L.Rh) {
-            const float d = tile[col][cl];
+    {
+        const int xr_l = t >> 2;         // row of X within the tile (a column of u)
+        const int seg = (t & 3) * 16;    // 16 consecutive values of that row
+        const int64_t xr = c0 + xr_l, xc = r0 + seg;
+        if (xr < L.C) {
+            float d[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) d[j] = tile[xr_l][seg + j];
             const int64_t xi = (int64_t)u * L.x_unit + xr * L.ldx + xc;
-            if (L.x_f32) reinterpret_cast<float*>(L.X)[xi] = d;
-            else reinterpret_cast<__nv_bfloat16*>(L.X)[xi] = __float2bfloat16_rn(d);
+            if (xc + 16 <= L.Rh) {
+                if (XF32) {
+                    float4* xp = reinterpret_cast<float4*>(reinterpret_cast<float*>(L.X) + xi);
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) __stcs(xp + q, make_float4(d[4 * q], d[4 * q + 1], d[4 * q + 2], d[4 * q + 3]));
+                } else {
+                    uint4* xp = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(L.X) + xi);
+#pragma unroll
+                    for (int q = 0; q < 2; ++q) {
+                        uint4 w;
+                        w.x = pack_bf16x2(d[8 * q + 0], d[8 * q + 1]);
+                        w.y = pack_bf16x2(d[8 * q + 2], d[8 * q + 3]);
+                        w.z = pack_bf16x2(d[8 * q + 4], d[8 * q + 5]);
+                        w.w = pack_bf16x2(d[8 * q + 6], d[8 * q + 7]);
+                        __stcs(xp + q, w);
+                    }
+                }
+            } else {
+                for (int j = 0; j < 16 && xc + j < L.Rh; ++j) {
+                    if (XF32) reinterpret_cast<float*>(L.X)[xi + j] = d[j];
+                    else reinterpret_cast<__nv_bfloat16*>(L.X)[xi + j] = __float2bfloat16_rn(d[j]);
+                }
+            }
         }
     }
     const float tot = block_sum_256(ss, red);
@@ -167,8 +267,18 @@ cudaError_t launch_muon_prep(const MuonPrepLaunch& L, cudaStream_t s) {
     const int units = L.batch * L.heads;
     if (units == 0 || L.parts == 0) return cudaSuccess;
     dim3 grid((unsigned)L.parts, (unsigned)units);
-    if (L.transposed) prep_transpose_kernel<<<grid, 256, 0, s>>>(L);
-    else prep_flat_kernel<<<grid, 256, 0, s>>>(L);
+    const bool gb = L.gdt == MA_BF16, xf = L.x_f32 != 0;
+    if (L.transposed) {
+        if (gb && !xf) prep_transpose_kernel<true, false><<<grid, 256, 0, s>>>(L);
+        else if (gb) prep_transpose_kernel<true, true><<<grid, 256, 0, s>>>(L);
+        else if (!xf) prep_transpose_kernel<false, false><<<grid, 256, 0, s>>>(L);
+        else prep_transpose_kernel<false, true><<<grid, 256, 0, s>>>(L);
+    } else {
+        if (gb && !xf) prep_flat_kernel<true, false><<<grid, 256, 0, s>>>(L);
+        else if (gb) prep_flat_kernel<true, true><<<grid, 256, 0, s>>>(L);
+        else if (!xf) prep_flat_kernel<false, false><<<grid, 256, 0, s>>>(L);
+        else prep_flat_kernel<false, true><<<grid, 256, 0, s>>>(L);
+    }
     return cudaGetLastError();
 }
 

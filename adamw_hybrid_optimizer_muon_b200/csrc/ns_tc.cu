@@ -43,7 +43,10 @@ namespace ma {
 
 namespace {
 
-constexpr int BM = 256, BN = 256, BK = 64, STAGES = 6;
+#ifndef MA_NS_STAGES
+#define MA_NS_STAGES 6
+#endif
+constexpr int BM = 256, BN = 256, BK = 64, STAGES = MA_NS_STAGES;
 constexpr int HM = BM / 2, HN = BN / 2;                // rows of A / columns of B held by each CTA
 constexpr uint32_t A_BYTES = HM * BK * 2;              // 16 KB
 constexpr uint32_t B_BYTES = HN * BK * 2;              // 16 KB
