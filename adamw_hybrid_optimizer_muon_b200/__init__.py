@@ -19,7 +19,7 @@ __all__ = [
     "ns_iterate_workspace_bytes", "ns_iterate_bf16", "adamw_step_fused", "ma_plan_create", "muonadamw_step",
     "ma_plan_destroy", "ma_device_status", "ma_set_wait_limit_ns", "ma_selftest_wait_timeout", "Plan",
     "MuonAdamW", "muon_hparams", "adamw_hparams", "ma_profile_enable", "ma_profile_collect", "PROF_CLASSES",
-    "muon_step_batched_noalloc", "STATIC_SCRATCH_BYTES",
+    "muon_step_batched_noalloc", "STATIC_SCRATCH_BYTES", "muonadamw_step_from_host",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -102,6 +102,7 @@ def lib() -> ctypes.CDLL:
         "ma_plan_create": (i32, [ctypes.POINTER(Tensor), i32, ctypes.POINTER(Group), i32, ctypes.POINTER(vp),
                                  ctypes.POINTER(sz)]),
         "muonadamw_step": (i32, [vp, ctypes.POINTER(Group), vp, sz, vp]),
+        "muonadamw_step_from_host": (i32, [vp, ctypes.POINTER(Group), pp, vp, sz, vp, vp]),
         "ma_plan_last_launches": (i32, [vp]),
         "ma_plan_destroy": (None, [vp]),
         "ma_device_status": (i32, [vp, i32]),
@@ -295,6 +296,16 @@ def muonadamw_step(plan, groups: Sequence[Group], ws, ws_bytes: int, stream=None
     _check(lib().muonadamw_step(plan, garr, _ptr(ws), int(ws_bytes), _stream(stream)), "muonadamw_step")
 
 
+def muonadamw_step_from_host(plan, groups: Sequence[Group], host_grads, ws, ws_bytes: int, stream=None,
+                             copy_stream=None) -> None:
+    """One step whose gradients are copied from host memory (pinned tensors or host pointers) on copy_stream,
+    overlapped with the compute on stream."""
+    garr = (Group * max(1, len(groups)))(*groups)
+    _check(lib().muonadamw_step_from_host(plan, garr, _ptr_array(host_grads), _ptr(ws), int(ws_bytes),
+                                          _stream(stream), _stream(copy_stream) if copy_stream is not None
+                                          else _stream(stream)), "muonadamw_step_from_host")
+
+
 def ma_plan_destroy(plan) -> None:
     lib().ma_plan_destroy(plan)
 
@@ -342,6 +353,11 @@ class Plan:
 
     def step(self, groups: Sequence[Group] | None = None, stream=None) -> None:
         muonadamw_step(self.handle, groups if groups is not None else self.groups, self.ws, self.ws.numel(), stream)
+
+    def step_from_host(self, host_grads, groups: Sequence[Group] | None = None, stream=None,
+                       copy_stream=None) -> None:
+        muonadamw_step_from_host(self.handle, groups if groups is not None else self.groups, host_grads, self.ws,
+                                 self.ws.numel(), stream, copy_stream)
 
     @property
     def launches(self) -> int:
@@ -419,15 +435,36 @@ class MuonAdamW:
         self._plan = Plan(descs, self.groups, self._ws_cap, device=self.entries[0][0].device)
         self._grad_ptrs = ptrs
 
-    def step(self, grads=None, stream=None) -> None:
-        if grads is None:
-            grads = [p.grad for p, _, _ in self.entries]
-        self._ensure_plan(grads)
+    def _advance(self):
         self.step_count += 1
         for g in self.groups:
             if g.kind == MA_ADAMW:
                 g.adamw.step = self.step_count
+
+    def step(self, grads=None, stream=None) -> None:
+        if grads is None:
+            grads = [p.grad for p, _, _ in self.entries]
+        self._ensure_plan(grads)
+        self._advance()
         self._plan.step(self.groups, stream)
+
+    def step_from_host(self, host_grads, device_grads, stream=None, copy_stream=None) -> None:
+        """One step whose gradients arrive from host memory.
+
+        host_grads: pinned CPU tensors (or host pointers), one per entry.
+        device_grads: the device buffers that receive them (same shapes and
+        dtypes); the library copies each group of gradients on copy_stream
+        (default: a stream owned by this optimizer) and overlaps the copies
+        with the compute on stream.
+        """
+        import torch
+        self._ensure_plan(device_grads)
+        if copy_stream is None:
+            if getattr(self, "_copy_stream", None) is None:
+                self._copy_stream = torch.cuda.Stream(device=self.entries[0][0].device)
+            copy_stream = self._copy_stream
+        self._advance()
+        self._plan.step_from_host(host_grads, self.groups, stream, copy_stream)
 
     @property
     def launches(self) -> int:

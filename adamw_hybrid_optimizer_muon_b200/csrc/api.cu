@@ -81,6 +81,11 @@ void prof_end(int rec, cudaStream_t s, double flops, double bytes) {
 }
 
 constexpr size_t kAlign = 256;
+// Muon sub-batch sizes when gradients stream in from the host: the first
+// sub-batch is small so that compute starts after a short copy, the others
+// large enough to keep every GEMM launch many waves deep.
+constexpr int kFromHostFirstBatch = 8;
+constexpr int kFromHostBatch = 32;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
@@ -450,7 +455,118 @@ struct ma_plan {
     std::vector<Bucket> buckets;
     size_t ws_bytes = 0;
     int last_launches = 0;
+    std::vector<cudaEvent_t> events;  // segment-ready events of muonadamw_step_from_host
+    ~ma_plan() {
+        for (cudaEvent_t e : events) cudaEventDestroy(e);
+    }
 };
+
+namespace ma {
+namespace {
+
+// A unit of launch work inside one step: every AdamW tensor, or one sub-batch
+// of one Muon bucket.
+struct Segment {
+    int adamw;  // 1: the AdamW tensors; 0: a Muon sub-batch
+    int bucket, start, count;
+};
+
+int64_t tensor_numel(const ma_tensor_t& x) {
+    int64_t n = 1;
+    for (int d = 0; d < x.ndim; ++d) n *= x.shape[d];
+    return n;
+}
+
+// Shared checks of a step over a plan; fills *sms.
+int check_step(ma_plan* plan, const ma_group_t* groups, void* ws, size_t ws_bytes, int* sms) {
+    if (!plan) return MA_ERR_NULL;
+    const int ngroups = (int)plan->group_kind.size();
+    if (ngroups > 0 && !groups) return MA_ERR_NULL;
+    int st;
+    for (int k = 0; k < ngroups; ++k) {
+        if (groups[k].kind != plan->group_kind[k]) return MA_ERR_ARG;
+        if (groups[k].kind == MA_MUON) {
+            if ((st = check_muon_hp(&groups[k].muon))) return st;
+        } else if ((st = check_adamw_hp(&groups[k].adamw))) {
+            return st;
+        }
+    }
+    // the plan's bucket geometry depends on heads, steps, precision and c != 0
+    for (auto& b : plan->buckets) {
+        MuonGeom g;
+        if ((st = muon_geom(b.sub, b.R, b.C, groups[b.group].muon, &g))) return st;
+        if (g.total > plan->ws_bytes) return MA_ERR_ARG;
+    }
+    if (plan->ws_bytes > 0 && (!ws || !aligned(ws, kAlign) || ws_bytes < plan->ws_bytes)) return MA_ERR_WORKSPACE;
+    *sms = 0;
+    if (!plan->adamw_idx.empty() || !plan->buckets.empty()) {
+        if ((st = device_ok_and_sms(sms))) return st;
+    }
+    return MA_OK;
+}
+
+// Segments in launch order. first_cap / cap bound the Muon sub-batch sizes
+// (0 = the plan's own sub-batch size); AdamW goes first or last.
+std::vector<Segment> step_segments(const ma_plan* plan, int first_cap, int cap, bool adamw_last) {
+    std::vector<Segment> segs;
+    if (!adamw_last && !plan->adamw_idx.empty()) segs.push_back({1, -1, 0, 0});
+    bool first = true;
+    for (int bi = 0; bi < (int)plan->buckets.size(); ++bi) {
+        const auto& b = plan->buckets[bi];
+        const int nb = (int)b.members.size();
+        for (int s0 = 0; s0 < nb;) {
+            int lim = b.sub;
+            if (cap > 0) lim = std::min(lim, cap);
+            if (first && first_cap > 0) lim = std::min(lim, first_cap);
+            const int cnt = std::min(lim, nb - s0);
+            segs.push_back({0, bi, s0, cnt});
+            s0 += cnt;
+            first = false;
+        }
+    }
+    if (adamw_last && !plan->adamw_idx.empty()) segs.push_back({1, -1, 0, 0});
+    return segs;
+}
+
+int launch_segment(ma_plan* plan, const ma_group_t* groups, const Segment& sg, void* ws, cudaStream_t s, int sms,
+                   int* launches) {
+    const int ngroups = (int)plan->group_kind.size();
+    int st;
+    if (sg.adamw) {
+        AdamwGroupConst gc[MA_MAX_GROUPS];
+        std::memset(gc, 0, sizeof(gc));
+        for (int k = 0; k < ngroups; ++k)
+            if (groups[k].kind == MA_ADAMW) gc[k] = adamw_const(groups[k].adamw);
+        for (int dt = 0; dt < 2; ++dt) {
+            std::vector<AdamwItem> items;
+            for (int i : plan->adamw_idx) {
+                const ma_tensor_t& x = plan->t[i];
+                if (x.grad_dtype != dt) continue;
+                items.push_back({x.param, x.grad, x.state0, x.state1, tensor_numel(x), x.group});
+            }
+            if (!items.empty() && (st = run_adamw(items, dt, gc, ngroups, s, launches))) return st;
+        }
+        return MA_OK;
+    }
+    const auto& b = plan->buckets[sg.bucket];
+    const ma_muon_hparams_t& hp = groups[b.group].muon;
+    const int gdt = plan->t[b.members[0]].grad_dtype;
+    float* W[MA_MAX_BATCH];
+    const void* G[MA_MAX_BATCH];
+    float* M[MA_MAX_BATCH];
+    for (int k = 0; k < sg.count; ++k) {
+        const ma_tensor_t& x = plan->t[b.members[sg.start + k]];
+        W[k] = x.param;
+        G[k] = x.grad;
+        M[k] = x.state0;
+    }
+    MuonGeom g;
+    muon_geom(sg.count, b.R, b.C, hp, &g);
+    return run_muon(sg.count, g, W, G, gdt, M, hp, ws, s, sms, launches);
+}
+
+}  // namespace
+}  // namespace ma
 
 extern "C" {
 
@@ -754,67 +870,65 @@ int ma_plan_create(const ma_tensor_t* t, int n, const ma_group_t* groups, int ng
 }
 
 int muonadamw_step(ma_plan_t* plan, const ma_group_t* groups, void* ws, size_t ws_bytes, void* stream) {
-    if (!plan) return MA_ERR_NULL;
-    const int ngroups = (int)plan->group_kind.size();
-    if (ngroups > 0 && !groups) return MA_ERR_NULL;
-    int st;
-    for (int k = 0; k < ngroups; ++k) {
-        if (groups[k].kind != plan->group_kind[k]) return MA_ERR_ARG;
-        if (groups[k].kind == MA_MUON) {
-            if ((st = check_muon_hp(&groups[k].muon))) return st;
-        } else if ((st = check_adamw_hp(&groups[k].adamw))) {
-            return st;
-        }
-    }
-    // the plan's bucket geometry depends on heads, steps, precision and c != 0
-    for (auto& b : plan->buckets) {
-        MuonGeom g;
-        if ((st = muon_geom(b.sub, b.R, b.C, groups[b.group].muon, &g))) return st;
-        if (g.total > plan->ws_bytes) return MA_ERR_ARG;
-    }
-    if (plan->ws_bytes > 0 && (!ws || !aligned(ws, kAlign) || ws_bytes < plan->ws_bytes)) return MA_ERR_WORKSPACE;
     int sms = 0;
-    if (!plan->adamw_idx.empty() || !plan->buckets.empty()) {
-        if ((st = device_ok_and_sms(&sms))) return st;
-    }
+    int st = check_step(plan, groups, ws, ws_bytes, &sms);
+    if (st) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     int launches = 0;
-    if (!plan->adamw_idx.empty()) {
-        AdamwGroupConst gc[MA_MAX_GROUPS];
-        std::memset(gc, 0, sizeof(gc));
-        for (int k = 0; k < ngroups; ++k)
-            if (groups[k].kind == MA_ADAMW) gc[k] = adamw_const(groups[k].adamw);
-        for (int dt = 0; dt < 2; ++dt) {
-            std::vector<AdamwItem> items;
-            for (int i : plan->adamw_idx) {
-                const ma_tensor_t& x = plan->t[i];
-                if (x.grad_dtype != dt) continue;
-                int64_t numel = 1;
-                for (int d = 0; d < x.ndim; ++d) numel *= x.shape[d];
-                items.push_back({x.param, x.grad, x.state0, x.state1, numel, x.group});
-            }
-            if (!items.empty() && (st = run_adamw(items, dt, gc, ngroups, s, &launches))) return st;
-        }
+    for (const Segment& sg : step_segments(plan, 0, 0, false))
+        if ((st = launch_segment(plan, groups, sg, ws, s, sms, &launches))) return st;
+    plan->last_launches = launches;
+    return MA_OK;
+}
+
+int muonadamw_step_from_host(ma_plan_t* plan, const ma_group_t* groups, const void* const* host_grads, void* ws,
+                             size_t ws_bytes, void* stream, void* copy_stream) {
+    int sms = 0;
+    int st = check_step(plan, groups, ws, ws_bytes, &sms);
+    if (st) return st;
+    const int n = (int)plan->t.size();
+    if (n > 0 && !host_grads) return MA_ERR_NULL;
+    for (int i = 0; i < n; ++i)
+        if (tensor_numel(plan->t[i]) > 0 && !host_grads[i]) return MA_ERR_NULL;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(copy_stream);
+    // Muon sub-batches first (the first one small, so the compute starts early),
+    // the AdamW tensors last: every later copy overlaps earlier compute.
+    const std::vector<Segment> segs = step_segments(plan, kFromHostFirstBatch, kFromHostBatch, true);
+    while (plan->events.size() < segs.size() + 1) {
+        cudaEvent_t e;
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return MA_ERR_CUDA;
+        plan->events.push_back(e);
     }
-    for (auto& b : plan->buckets) {
-        const ma_muon_hparams_t& hp = groups[b.group].muon;
-        const int nb = (int)b.members.size();
-        const int gdt = plan->t[b.members[0]].grad_dtype;
-        for (int s0 = 0; s0 < nb; s0 += b.sub) {
-            const int cnt = std::min(b.sub, nb - s0);
-            float* W[MA_MAX_BATCH];
-            const void* G[MA_MAX_BATCH];
-            float* M[MA_MAX_BATCH];
-            for (int k = 0; k < cnt; ++k) {
-                const ma_tensor_t& x = plan->t[b.members[s0 + k]];
-                W[k] = x.param;
-                G[k] = x.grad;
-                M[k] = x.state0;
-            }
-            MuonGeom g;
-            muon_geom(cnt, b.R, b.C, hp, &g);
-            if ((st = run_muon(cnt, g, W, G, gdt, M, hp, ws, s, sms, &launches))) return st;
+    // the copies overwrite the device gradients: wait for earlier work on `stream`
+    cudaEvent_t prior = plan->events[segs.size()];
+    if (cudaEventRecord(prior, s) != cudaSuccess || cudaStreamWaitEvent(cs, prior, 0) != cudaSuccess)
+        return MA_ERR_CUDA;
+    auto copy_tensor = [&](int i) -> int {
+        const ma_tensor_t& x = plan->t[i];
+        const size_t bytes = (size_t)tensor_numel(x) * (x.grad_dtype == MA_BF16 ? 2 : 4);
+        if (bytes == 0) return MA_OK;
+        return cudaMemcpyAsync(const_cast<void*>(x.grad), host_grads[i], bytes, cudaMemcpyHostToDevice, cs) ==
+                       cudaSuccess
+                   ? MA_OK
+                   : MA_ERR_CUDA;
+    };
+    for (size_t k = 0; k < segs.size(); ++k) {
+        const Segment& sg = segs[k];
+        if (sg.adamw) {
+            for (int i : plan->adamw_idx)
+                if ((st = copy_tensor(i))) return st;
+        } else {
+            const auto& b = plan->buckets[sg.bucket];
+            for (int j = 0; j < sg.count; ++j)
+                if ((st = copy_tensor(b.members[sg.start + j]))) return st;
         }
+        if (cudaEventRecord(plan->events[k], cs) != cudaSuccess) return MA_ERR_CUDA;
+    }
+    int launches = 0;
+    for (size_t k = 0; k < segs.size(); ++k) {
+        if (cudaStreamWaitEvent(s, plan->events[k], 0) != cudaSuccess) return MA_ERR_CUDA;
+        if ((st = launch_segment(plan, groups, segs[k], ws, s, sms, &launches))) return st;
     }
     plan->last_launches = launches;
     return MA_OK;

@@ -236,7 +236,23 @@ int ma_plan_create(const ma_tensor_t* t, int n, const ma_group_t* groups, int ng
 int muonadamw_step(ma_plan_t* plan, const ma_group_t* groups, void* ws, size_t ws_bytes,
                    void* stream);
 
-/* Number of kernel launches the last muonadamw_step issued (for benchmarks). */
+/* One MuonAdamW step whose gradients start in host memory (for example
+ * gradients offloaded to the CPU). host_grads: host array of n pointers, one
+ * per planned tensor in table order, each to that tensor's gradient in its
+ * grad_dtype (numel elements; page-locked memory makes the copies
+ * asynchronous). The library copies each gradient into the tensor's device
+ * grad buffer on copy_stream, in the order the step consumes them (Muon
+ * sub-batches first, the AdamW tensors last), records an event after each
+ * group of copies, and makes `stream` wait for that event before the group's
+ * kernels: later copies overlap earlier compute. The copies wait for all work
+ * queued on `stream` before the call, since they overwrite the device
+ * gradients. copy_stream may equal stream (no overlap). Results equal those of
+ * muonadamw_step on the same gradients. Host buffers must stay valid and
+ * unchanged until the step completes. */
+int muonadamw_step_from_host(ma_plan_t* plan, const ma_group_t* groups, const void* const* host_grads, void* ws,
+                             size_t ws_bytes, void* stream, void* copy_stream);
+
+/* Number of kernel launches the last muonadamw_step or muonadamw_step_from_host issued (for benchmarks). */
 int ma_plan_last_launches(const ma_plan_t* plan);
 
 void ma_plan_destroy(ma_plan_t* plan);

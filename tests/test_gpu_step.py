@@ -141,3 +141,26 @@ def test_d20_full_size_sampled():
 @pytest.mark.slow
 def test_7b_full_size_sampled():
     _full_size_check("7b", n_muon_samples=1, adamw_samples=100_000)
+
+
+@pytest.mark.parametrize("name", ["tiny", "d20"])
+def test_step_from_host_equals_resident_step(name):
+    # gradients copied from pinned host memory, overlapped with compute, give
+    # bit-identical parameters and state to the step on resident gradients
+    wl = synth.WORKLOADS[name]()
+    pa = sdev.weights(wl)
+    pb = [p.clone() for p in pa]
+    opt_a, opt_b = build_optimizer(wl, pa), build_optimizer(wl, pb)
+    dev_a = sdev.gradients(wl, 1)
+    dev_b = [torch.zeros_like(g) for g in dev_a]
+    for step in (1, 2):
+        g = sdev.gradients(wl, step, out=dev_a)
+        host_g = [x.cpu().pin_memory() for x in g]
+        opt_a.step(dev_a)
+        opt_b.step_from_host(host_g, dev_b)
+        torch.cuda.synchronize()
+        assert ma.ma_device_status() == ma.MA_OK
+        for x, y in zip(pa, pb):
+            assert torch.equal(x, y)
+        for (s0, s1), (t0, t1) in zip(opt_a.state, opt_b.state):
+            assert torch.equal(s0, t0) and (s1 is None or torch.equal(s1, t1))
