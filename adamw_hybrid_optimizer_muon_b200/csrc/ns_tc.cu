@@ -36,6 +36,8 @@
 // B operand major-ness: for GRAM and GRAMSQ both operands are K-major rows of
 // the same matrix. For APPLY the B operand is X itself, read MN-major (the
 // contraction runs over X's rows), so no transposed copy is ever made.
+#include <cstring>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -54,7 +56,19 @@ constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;    // 32 KB per CTA
 constexpr uint32_t TMEM_COLS = 2 * BN;                 // two fp32 accumulators
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 32 * (2 + EPI_WARPS);
-constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+// Epilogue staging: per epilogue warp one 32 x 32 bf16 block for the tile and
+// one for its mirror (2 KB each, 64-byte rows, 64-byte swizzle), written out
+// with bulk tensor stores.
+constexpr uint32_t STG_BLOCK = 32 * 32 * 2;
+// The epilogue warps wait for a whole tile's main loop; they sleep in the
+// barrier wait rather than poll it (polling costs power, hence clock, on a
+// power-capped part).
+#ifndef MA_EPI_SLEEP_NS
+#define MA_EPI_SLEEP_NS 20000
+#endif
+constexpr uint32_t kEpiSleepNs = MA_EPI_SLEEP_NS;
+constexpr uint32_t STG_BYTES = EPI_WARPS * 2 * STG_BLOCK;  // 32 KB
+constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + STG_BYTES + 1024 /*align*/ + 256 /*barriers*/;
 
 struct TileCoord {
     int u, ti, tj;
@@ -81,19 +95,6 @@ __device__ __forceinline__ TileCoord decode_tile(int mode, int t, int tiles_per_
     return c;
 }
 
-__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32], float mul) {
-    uint4* d = reinterpret_cast<uint4*>(dst);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        uint4 w;
-        w.x = pack_bf16x2(v[8 * q + 0] * mul, v[8 * q + 1] * mul);
-        w.y = pack_bf16x2(v[8 * q + 2] * mul, v[8 * q + 3] * mul);
-        w.z = pack_bf16x2(v[8 * q + 4] * mul, v[8 * q + 5] * mul);
-        w.w = pack_bf16x2(v[8 * q + 6] * mul, v[8 * q + 7] * mul);
-        d[q] = w;
-    }
-}
-
 __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&x)[32]) {
     const uint4* s = reinterpret_cast<const uint4*>(src);
 #pragma unroll
@@ -106,121 +107,103 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&x
     }
 }
 
+// This lane's 32 output values of one 32-column chunk (row `row`, columns
+// col0..col0+31), before rounding: GRAM b*A (x s^2 on the first iteration),
+// GRAMSQ b*A + c*A^2, APPLY/FINAL s*(a*X + B*X).
 template <int MODE>
-__device__ __forceinline__ void epilogue_chunk(const NsParams& p, const TileCoord& tc, int row, int col0,
-                                               const float (&v)[32]) {
-    const int m = p.m, n = p.n;
-    if (MODE == NS_GRAM || MODE == NS_GRAMSQ) {
-        if (row >= m) return;
+__device__ __forceinline__ void epilogue_values(const NsParams& p, const TileCoord& tc, int row, int col0,
+                                                const float (&v)[32], float (&o)[32]) {
+    if (MODE == NS_GRAM) {
         float coef = p.coef_gram;
-        if (MODE == NS_GRAM && p.first) {
+        if (p.first) {
             const float s = p.scale[tc.u];
             coef *= s * s;
         }
-        __nv_bfloat16* G = reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)tc.u * p.g_unit;
-        const __nv_bfloat16* Gin =
-            MODE == NS_GRAMSQ ? reinterpret_cast<const __nv_bfloat16*>(p.xin) + (int64_t)tc.u * p.g_unit : nullptr;
-        float o[32];
-        if (MODE == NS_GRAMSQ) {
-            // B = b*A + c*A^2, with acc = A^2 and A read back from the Gram buffer
-            float a_in[32];
-            if (col0 + 32 <= m) {
-                load_bf16x32(Gin + (int64_t)row * p.ldg + col0, a_in);
-            } else {
 #pragma unroll
-                for (int t = 0; t < 32; ++t)
-                    a_in[t] = (col0 + t < m) ? __bfloat162float(Gin[(int64_t)row * p.ldg + col0 + t]) : 0.f;
-            }
-#pragma unroll
-            for (int t = 0; t < 32; ++t) o[t] = p.b * a_in[t] + p.c * v[t];
-            coef = 1.f;
+        for (int t = 0; t < 32; ++t) o[t] = coef * v[t];
+    } else if (MODE == NS_GRAMSQ) {
+        // acc = A^2; A is read back from the Gram buffer
+        const int m = p.m;
+        const __nv_bfloat16* Gin = reinterpret_cast<const __nv_bfloat16*>(p.xin) + (int64_t)tc.u * p.g_unit;
+        float a_in[32];
+        if (row < m && col0 + 32 <= m) {
+            load_bf16x32(Gin + (int64_t)row * p.ldg + col0, a_in);
         } else {
 #pragma unroll
-            for (int t = 0; t < 32; ++t) o[t] = v[t];
-        }
-        if (col0 >= row && col0 + 32 <= m) {
-            store_bf16x32(G + (int64_t)row * p.ldg + col0, o, coef);
-        } else {
-#pragma unroll
-            for (int t = 0; t < 32; ++t) {
-                const int j = col0 + t;
-                if (j >= row && j < m) G[(int64_t)row * p.ldg + j] = __float2bfloat16_rn(o[t] * coef);
-            }
+            for (int t = 0; t < 32; ++t)
+                a_in[t] = (row < m && col0 + t < m) ? __bfloat162float(Gin[(int64_t)row * p.ldg + col0 + t]) : 0.f;
         }
 #pragma unroll
-        for (int t = 0; t < 32; ++t) {
-            const int j = col0 + t;
-            if (j > row && j < m) G[(int64_t)j * p.ldg + row] = __float2bfloat16_rn(o[t] * coef);
-        }
+        for (int t = 0; t < 32; ++t) o[t] = p.b * a_in[t] + p.c * v[t];
     } else {
-        if (row >= m) return;
+        const int m = p.m, n = p.n;
         const float sa = p.first ? p.scale[tc.u] : 1.f;
-        const __nv_bfloat16* Xin = reinterpret_cast<const __nv_bfloat16*>(p.xin) + (int64_t)tc.u * p.x_unit;
         float x[32];
-        const bool full = col0 + 32 <= n;
-        if (full) {
+        const __nv_bfloat16* Xin = reinterpret_cast<const __nv_bfloat16*>(p.xin) + (int64_t)tc.u * p.x_unit;
+        if (row < m && col0 + 32 <= n) {
             load_bf16x32(Xin + (int64_t)row * p.ldx + col0, x);
         } else {
 #pragma unroll
             for (int t = 0; t < 32; ++t)
-                x[t] = (col0 + t < n) ? __bfloat162float(Xin[(int64_t)row * p.ldx + col0 + t]) : 0.f;
+                x[t] = (row < m && col0 + t < n) ? __bfloat162float(Xin[(int64_t)row * p.ldx + col0 + t]) : 0.f;
         }
-        float o[32];
 #pragma unroll
         for (int t = 0; t < 32; ++t) o[t] = sa * (p.a * x[t] + v[t]);
-        if (MODE == NS_APPLY) {
-            __nv_bfloat16* Xo = reinterpret_cast<__nv_bfloat16*>(p.out) + (int64_t)tc.u * p.x_unit;
-            if (full) {
-                store_bf16x32(Xo + (int64_t)row * p.ldx + col0, o, 1.f);
-            } else {
+    }
+}
+
+// Final apply: W <- W*(1 - lr*wd) - lr*scale*X_N in the caller's fp32 weights.
+__device__ __forceinline__ void epilogue_final(const NsParams& p, const TileCoord& tc, int row, int col0,
+                                               const float (&o)[32]) {
+    const int m = p.m, n = p.n;
+    if (row >= m) return;
+    const int bidx = tc.u / p.heads, h = tc.u - bidx * p.heads;
+    float* Wb = p.W[bidx] + (int64_t)h * p.Rh * p.C;
+    const float decay = p.decay, lrs = p.lr_s;
+    if (!p.transposed) {
+        float* w = Wb + (int64_t)row * p.C + col0;
+        if (col0 + 32 <= n && (p.C & 3) == 0) {
 #pragma unroll
-                for (int t = 0; t < 32; ++t)
-                    if (col0 + t < n) Xo[(int64_t)row * p.ldx + col0 + t] = __float2bfloat16_rn(o[t]);
+            for (int q = 0; q < 8; ++q) {
+                float4 wv = reinterpret_cast<float4*>(w)[q];
+                wv.x = wv.x * decay - lrs * o[4 * q + 0];
+                wv.y = wv.y * decay - lrs * o[4 * q + 1];
+                wv.z = wv.z * decay - lrs * o[4 * q + 2];
+                wv.w = wv.w * decay - lrs * o[4 * q + 3];
+                reinterpret_cast<float4*>(w)[q] = wv;
             }
-        } else {  // NS_FINAL
-            const int bidx = tc.u / p.heads, h = tc.u - bidx * p.heads;
-            float* Wb = p.W[bidx] + (int64_t)h * p.Rh * p.C;
-            const float decay = p.decay, lrs = p.lr_s;
-            if (!p.transposed) {
-                float* w = Wb + (int64_t)row * p.C + col0;
-                if (full && (p.C & 3) == 0) {
+        } else {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) {
-                        float4 wv = reinterpret_cast<float4*>(w)[q];
-                        wv.x = wv.x * decay - lrs * o[4 * q + 0];
-                        wv.y = wv.y * decay - lrs * o[4 * q + 1];
-                        wv.z = wv.z * decay - lrs * o[4 * q + 2];
-                        wv.w = wv.w * decay - lrs * o[4 * q + 3];
-                        reinterpret_cast<float4*>(w)[q] = wv;
-                    }
-                } else {
+            for (int t = 0; t < 32; ++t)
+                if (col0 + t < n) w[t] = w[t] * decay - lrs * o[t];
+        }
+    } else {
+        // X_N[row][j] is W[j][row]: lanes hold consecutive rows, so each column
+        // j is one coalesced 128-byte access across the warp.
 #pragma unroll
-                    for (int t = 0; t < 32; ++t)
-                        if (col0 + t < n) w[t] = w[t] * decay - lrs * o[t];
-                }
-            } else {
-                // X_N[row][j] is W[j][row]: lanes hold consecutive rows, so each
-                // column j is one coalesced 128-byte access across the warp.
-#pragma unroll
-                for (int t = 0; t < 32; ++t) {
-                    const int j = col0 + t;
-                    if (j < n) {
-                        float* w = Wb + (int64_t)j * p.C + row;
-                        *w = *w * decay - lrs * o[t];
-                    }
-                }
+        for (int t = 0; t < 32; ++t) {
+            const int j = col0 + t;
+            if (j < n) {
+                float* w = Wb + (int64_t)j * p.C + row;
+                *w = *w * decay - lrs * o[t];
             }
         }
     }
 }
 
+// Byte offset of 16-byte chunk q of row r in a 64-byte-row block with the
+// 64-byte swizzle that the bulk tensor store expects.
+__device__ __forceinline__ uint32_t sw64(uint32_t r, uint32_t q) { return r * 64u + ((q ^ ((r >> 1) & 3u)) << 4); }
+
 template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
     ns_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                 const __grid_constant__ NsParams p, int tiles_per_unit, int mt, int nt, int kblocks) {
+                 const __grid_constant__ CUtensorMap mapOut, const __grid_constant__ NsParams p, int tiles_per_unit,
+                 int mt, int nt, int kblocks) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + STAGES * STAGE_BYTES);
+    uint8_t* staging = smem + STAGES * STAGE_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(staging + STG_BYTES);
     uint64_t* empty = full + STAGES;
     uint64_t* acc_full = empty + STAGES;
     uint64_t* acc_empty = acc_full + 2;
@@ -250,6 +233,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         fence_barrier_init();
         prefetch_tensormap(&mapA);
         prefetch_tensormap(&mapB);
+        if (MODE != NS_FINAL) prefetch_tensormap(&mapOut);
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_holder, TMEM_COLS);
@@ -354,6 +338,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     } else {
         const int quad = warp & 3;              // TMEM lanes [32*quad, 32*quad + 32)
         const int half = (warp - 2) / 4;        // which half of the 256 columns
+        uint8_t* stg = staging + (warp - 2) * 2 * STG_BLOCK;
         const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
         const uint32_t acc_empty_leader1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
         int lt = 0;
@@ -361,27 +346,62 @@ __global__ void __launch_bounds__(THREADS, 1)
             const TileCoord tc = decode_tile(MODE, t, tiles_per_unit, mt, nt);
             const int acc = lt & 1;
             const uint32_t use = (uint32_t)(lt >> 1);
+            const int row_lo = tc.ti * BM + (int)rank * HM + quad * 32;
+            const int row = row_lo + lane;
             int ok = 1;
-            if (lane == 0) ok = mbar_wait_bounded(&acc_full[acc], use & 1u, abort_flag, limit, p.status) ? 1 : 0;
+            if (lane == 0)
+                ok = mbar_wait_bounded(&acc_full[acc], use & 1u, abort_flag, limit, p.status, kEpiSleepNs) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after();
-            const int row_lo = tc.ti * BM + (int)rank * HM + quad * 32;
-            const int row = row_lo + lane;
             const int limit_cols = kApply ? p.n : p.m;
 #pragma unroll 1
-            for (int cc = half * 4; cc < half * 4 + 4; ++cc) {
+            for (int c = 0; c < 4; ++c) {
+                const int cc = half * 4 + c;
                 const int col0 = tc.tj * BN + cc * 32;
-                if (col0 >= limit_cols) break;                                    // warp-uniform
-                if (!kApply && col0 + 31 < row_lo) continue;                     // below the diagonal
-                float v[32];
+                if (col0 >= limit_cols || row_lo >= p.m) break;                  // warp-uniform
+                if (!kApply && col0 < row_lo) continue;                          // below the diagonal
+                float v[32], o[32];
                 tmem_ld32(tmem_base + (uint32_t)(acc * BN + cc * 32) + ((uint32_t)(quad * 32) << 16), v);
-                epilogue_chunk<MODE>(p, tc, row, col0, v);
+                epilogue_values<MODE>(p, tc, row, col0, v, o);
+                if (MODE == NS_FINAL) {
+                    epilogue_final(p, tc, row, col0, o);
+                    continue;
+                }
+                // Stage this warp's 32 x 32 block (and, for an off-diagonal Gram
+                // chunk, its transpose), then write both with bulk tensor stores:
+                // each leaves shared memory as contiguous 64-byte rows.
+                const bool mirror = !kApply && col0 > row_lo;
+                if (lane == 0) bulk_wait_group_read0();  // the previous chunk's stores have read their source
+                __syncwarp();
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint4 w;
+                    w.x = pack_bf16x2(o[8 * q + 0], o[8 * q + 1]);
+                    w.y = pack_bf16x2(o[8 * q + 2], o[8 * q + 3]);
+                    w.z = pack_bf16x2(o[8 * q + 4], o[8 * q + 5]);
+                    w.w = pack_bf16x2(o[8 * q + 6], o[8 * q + 7]);
+                    *reinterpret_cast<uint4*>(stg + sw64(lane, q)) = w;
+                }
+                if (mirror) {
+                    const uint32_t lo = ((uint32_t)lane & 7u) << 1, qq = (uint32_t)lane >> 3;
+#pragma unroll
+                    for (int t = 0; t < 32; ++t)
+                        *reinterpret_cast<__nv_bfloat16*>(stg + STG_BLOCK + sw64(t, qq) + lo) = __float2bfloat16_rn(o[t]);
+                }
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_3d(&mapOut, stg, col0, row_lo, tc.u);
+                    if (mirror) tma_store_3d(&mapOut, stg + STG_BLOCK, row_lo, col0, tc.u);
+                    bulk_commit_group();
+                }
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);
         }
+        if (lane == 0) bulk_wait_group0();  // every bulk store of this warp has completed
     }
 
     __syncthreads();
@@ -416,9 +436,10 @@ EncodeTiledFn encode_fn() {
 }
 
 // 3-D bf16 map over [units][rows][inner] with row stride `ld` and unit stride
-// `unit` (elements), 128-byte swizzle, zero fill out of bounds.
+// `unit` (elements), zero fill out of bounds (loads) / clipping (stores).
 bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint64_t units, uint64_t ld,
-              uint64_t unit, uint32_t box_inner, uint32_t box_rows) {
+              uint64_t unit, uint32_t box_inner, uint32_t box_rows,
+              CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     cuuint64_t dims[3] = {inner, rows, units};
@@ -426,13 +447,14 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
     cuuint32_t box[3] = {box_inner, box_rows, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 template <int MODE>
 cudaError_t launch_mode(const NsParams& p, const void* x_buf, const void* g_buf, int num_sms, cudaStream_t s) {
-    CUtensorMap mA, mB;
+    CUtensorMap mA, mB, mO;
+    std::memset(&mO, 0, sizeof(mO));
     int kblocks, mt, nt, tiles;
     mt = (p.m + BM - 1) / BM;
     if (MODE == NS_GRAM || MODE == NS_GRAMSQ) {
@@ -446,12 +468,17 @@ cudaError_t launch_mode(const NsParams& p, const void* x_buf, const void* g_buf,
             if (!make_map(&mA, p.xin, p.m, p.m, p.units, p.ldg, p.g_unit, BK, HM)) return cudaErrorInvalidValue;
         }
         mB = mA;  // both operands are 128-row, 64-deep K-major boxes of the same matrix
+        if (!make_map(&mO, p.out, p.m, p.m, p.units, p.ldg, p.g_unit, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+            return cudaErrorInvalidValue;
     } else {
         nt = (p.n + BN - 1) / BN;
         tiles = mt * nt;
         kblocks = (p.m + BK - 1) / BK;
         if (!make_map(&mA, g_buf, p.m, p.m, p.units, p.ldg, p.g_unit, BK, HM)) return cudaErrorInvalidValue;
         if (!make_map(&mB, x_buf, p.n, p.m, p.units, p.ldx, p.x_unit, 64, BK)) return cudaErrorInvalidValue;
+        if (MODE == NS_APPLY &&
+            !make_map(&mO, p.out, p.n, p.m, p.units, p.ldx, p.x_unit, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+            return cudaErrorInvalidValue;
     }
     const long long total = (long long)tiles * p.units;
     if (total <= 0) return cudaSuccess;
@@ -497,7 +524,7 @@ cudaError_t launch_mode(const NsParams& p, const void* x_buf, const void* g_buf,
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, ns_tc_kernel<MODE>, mA, mB, p, tiles, mt, nt, kblocks);
+    return cudaLaunchKernelEx(&cfg, ns_tc_kernel<MODE>, mA, mB, mO, p, tiles, mt, nt, kblocks);
 }
 
 }  // namespace
