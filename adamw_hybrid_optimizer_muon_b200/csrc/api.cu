@@ -192,7 +192,10 @@ float shape_scale(int64_t R, int64_t C, int mode) {
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? MA_OK : MA_ERR_CUDA; }
 
 int ns_prof_class(int mode) {
-    return mode == NS_GRAM ? MA_PROF_NS_GRAM : mode == NS_GRAMSQ ? MA_PROF_NS_GRAMSQ : MA_PROF_NS_APPLY;
+    return mode == NS_GRAM     ? MA_PROF_NS_GRAM
+           : mode == NS_GRAMSQ ? MA_PROF_NS_GRAMSQ
+           : mode == NS_FINAL  ? MA_PROF_NS_FINAL
+                               : MA_PROF_NS_APPLY;
 }
 
 // Algorithmic flops of one Newton-Schulz launch. A symmetric Gram X X^T has

@@ -152,41 +152,57 @@ __device__ __forceinline__ void epilogue_values(const NsParams& p, const TileCoo
     }
 }
 
+// Byte offset of 16-byte chunk q of row r in a 128-byte-row block with a
+// 128-byte XOR swizzle (conflict-free for the row-wise and column-wise
+// accesses of the final apply).
+__device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t q) { return r * 128u + ((q ^ (r & 7u)) << 4); }
+
 // Final apply: W <- W*(1 - lr*wd) - lr*scale*X_N in the caller's fp32 weights.
-__device__ __forceinline__ void epilogue_final(const NsParams& p, const TileCoord& tc, int row, int col0,
-                                               const float (&o)[32]) {
+// The warp's 32 x 32 fp32 block of X_N is staged in shared memory in the
+// orientation of W (transposed back when the unit was tall), then each lane
+// handles 4 consecutive elements of one W row: every read and write of W is
+// a 16-byte access and each group of 8 lanes covers one 128-byte row segment.
+__device__ __forceinline__ void epilogue_final(const NsParams& p, const TileCoord& tc, int row_lo, int col0,
+                                               const float (&o)[32], uint8_t* stg, int lane) {
+    __syncwarp();  // the previous chunk's reads of the staging block are done
+    if (!p.transposed) {
+#pragma unroll
+        for (int q = 0; q < 8; ++q)
+            *reinterpret_cast<float4*>(stg + sw128(lane, q)) =
+                make_float4(o[4 * q + 0], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
+    } else {
+#pragma unroll
+        for (int t = 0; t < 32; ++t)
+            *reinterpret_cast<float*>(stg + sw128(t, (uint32_t)lane >> 2) + (lane & 3) * 4) = o[t];
+    }
+    __syncwarp();
     const int m = p.m, n = p.n;
-    if (row >= m) return;
     const int bidx = tc.u / p.heads, h = tc.u - bidx * p.heads;
     float* Wb = p.W[bidx] + (int64_t)h * p.Rh * p.C;
     const float decay = p.decay, lrs = p.lr_s;
-    if (!p.transposed) {
-        float* w = Wb + (int64_t)row * p.C + col0;
-        if (col0 + 32 <= n && (p.C & 3) == 0) {
-#pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                float4 wv = reinterpret_cast<float4*>(w)[q];
-                wv.x = wv.x * decay - lrs * o[4 * q + 0];
-                wv.y = wv.y * decay - lrs * o[4 * q + 1];
-                wv.z = wv.z * decay - lrs * o[4 * q + 2];
-                wv.w = wv.w * decay - lrs * o[4 * q + 3];
-                reinterpret_cast<float4*>(w)[q] = wv;
-            }
-        } else {
-#pragma unroll
-            for (int t = 0; t < 32; ++t)
-                if (col0 + t < n) w[t] = w[t] * decay - lrs * o[t];
+    const int sub = lane >> 3, cq = lane & 7;
+#pragma unroll 2
+    for (int i = 0; i < 8; ++i) {
+        const int rr = 4 * i + sub;  // row of the staged block (a row of W)
+        const float4 ov = *reinterpret_cast<const float4*>(stg + sw128(rr, cq));
+        int wrow, wcol, nrows, ncols;
+        if (!p.transposed) {  // W row = X row, W column = X column
+            wrow = row_lo + rr; wcol = col0 + cq * 4; nrows = m; ncols = n;
+        } else {              // W row = X column, W column = X row
+            wrow = col0 + rr; wcol = row_lo + cq * 4; nrows = n; ncols = m;
         }
-    } else {
-        // X_N[row][j] is W[j][row]: lanes hold consecutive rows, so each column
-        // j is one coalesced 128-byte access across the warp.
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-            const int j = col0 + t;
-            if (j < n) {
-                float* w = Wb + (int64_t)j * p.C + row;
-                *w = *w * decay - lrs * o[t];
-            }
+        if (wrow >= nrows) continue;
+        float* w = Wb + (int64_t)wrow * p.C + wcol;
+        if (wcol + 4 <= ncols) {
+            float4 wv = *reinterpret_cast<float4*>(w);
+            wv.x = wv.x * decay - lrs * ov.x;
+            wv.y = wv.y * decay - lrs * ov.y;
+            wv.z = wv.z * decay - lrs * ov.z;
+            wv.w = wv.w * decay - lrs * ov.w;
+            *reinterpret_cast<float4*>(w) = wv;
+        } else {
+            const float oe[4] = {ov.x, ov.y, ov.z, ov.w};
+            for (int e = 0; e < 4 && wcol + e < ncols; ++e) w[e] = w[e] * decay - lrs * oe[e];
         }
     }
 }
@@ -365,7 +381,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 tmem_ld32(tmem_base + (uint32_t)(acc * BN + cc * 32) + ((uint32_t)(quad * 32) << 16), v);
                 epilogue_values<MODE>(p, tc, row, col0, v, o);
                 if (MODE == NS_FINAL) {
-                    epilogue_final(p, tc, row, col0, o);
+                    epilogue_final(p, tc, row_lo, col0, o, stg, lane);
                     continue;
                 }
                 // Stage this warp's 32 x 32 block (and, for an off-diagonal Gram

@@ -352,9 +352,10 @@ def main():
 
     if rank == 0:
         peaks = load_peaks()
-        ns_ms = sum(prof[c]["ms"] for c in ("ns_gram", "ns_apply", "ns_gramsq"))
-        ns_fl = sum(prof[c]["flops"] for c in ("ns_gram", "ns_apply", "ns_gramsq"))
-        ns_launches = sum(prof[c]["launches"] for c in ("ns_gram", "ns_apply", "ns_gramsq"))
+        ns_cls = ("ns_gram", "ns_apply", "ns_gramsq", "ns_final")
+        ns_ms = sum(prof[c]["ms"] for c in ns_cls)
+        ns_fl = sum(prof[c]["flops"] for c in ns_cls)
+        ns_launches = sum(prof[c]["launches"] for c in ns_cls)
         ns_tflops = ns_fl / (ns_ms / 1000.0) / 1e12 if ns_ms > 0 else None
         peak_t = peaks["bf16_tflops_sustained"]
         roofline = {"kernel": "ns_tc_kernel (Newton-Schulz Gram + apply, tcgen05)", "bound": "tensor",

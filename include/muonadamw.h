@@ -264,9 +264,10 @@ void ma_plan_destroy(ma_plan_t* plan);
 #define MA_PROF_MOMENTUM 1      /* momentum + Nesterov + norm partials         */
 #define MA_PROF_FINALIZE 2      /* norm finalize                               */
 #define MA_PROF_NS_GRAM 3       /* Newton-Schulz A = X X^T (tcgen05 or fp32)   */
-#define MA_PROF_NS_APPLY 4      /* Newton-Schulz X' = aX + BX, final apply too */
+#define MA_PROF_NS_APPLY 4      /* Newton-Schulz X' = aX + BX (not the last)   */
 #define MA_PROF_NS_GRAMSQ 5     /* Newton-Schulz A^2 (c != 0 only)             */
-#define MA_PROF_CLASSES 6
+#define MA_PROF_NS_FINAL 6      /* last apply, fused with decay and W update   */
+#define MA_PROF_CLASSES 7
 
 /* When on != 0, every kernel the library launches on this thread's current
  * device is bracketed by two CUDA events recorded on its launch stream. Off by
