@@ -181,28 +181,43 @@ __device__ __forceinline__ void epilogue_final(const NsParams& p, const TileCoor
     float* Wb = p.W[bidx] + (int64_t)h * p.Rh * p.C;
     const float decay = p.decay, lrs = p.lr_s;
     const int sub = lane >> 3, cq = lane & 7;
-#pragma unroll 2
-    for (int i = 0; i < 8; ++i) {
-        const int rr = 4 * i + sub;  // row of the staged block (a row of W)
-        const float4 ov = *reinterpret_cast<const float4*>(stg + sw128(rr, cq));
-        int wrow, wcol, nrows, ncols;
-        if (!p.transposed) {  // W row = X row, W column = X column
-            wrow = row_lo + rr; wcol = col0 + cq * 4; nrows = m; ncols = n;
-        } else {              // W row = X column, W column = X row
-            wrow = col0 + rr; wcol = row_lo + cq * 4; nrows = n; ncols = m;
+    // This lane's 8 groups of 4 W elements lie 4 rows apart in W in either
+    // orientation. They are loaded in two batches of 4 (all loads of a batch
+    // in flight together), so the chunk waits for DRAM twice.
+    int r0, c0, nrows, ncols;
+    if (!p.transposed) {  // W row = X row, W column = X column
+        r0 = row_lo + sub; c0 = col0 + cq * 4; nrows = m; ncols = n;
+    } else {              // W row = X column, W column = X row
+        r0 = col0 + sub; c0 = row_lo + cq * 4; nrows = n; ncols = m;
+    }
+    float* wbase = Wb + (int64_t)r0 * p.C + c0;
+    const int64_t wstep = 4 * (int64_t)p.C;
+    if (c0 + 4 <= ncols) {
+#pragma unroll 1
+        for (int i0 = 0; i0 < 8; i0 += 4) {
+            float4 wv[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+                if (r0 + 4 * (i0 + k) < nrows) wv[k] = *reinterpret_cast<const float4*>(wbase + (i0 + k) * wstep);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const int i = i0 + k;
+                if (r0 + 4 * i >= nrows) continue;
+                const float4 ov = *reinterpret_cast<const float4*>(stg + sw128(4 * i + sub, cq));
+                float4 w = wv[k];
+                w.x = w.x * decay - lrs * ov.x;
+                w.y = w.y * decay - lrs * ov.y;
+                w.z = w.z * decay - lrs * ov.z;
+                w.w = w.w * decay - lrs * ov.w;
+                *reinterpret_cast<float4*>(wbase + i * wstep) = w;
+            }
         }
-        if (wrow >= nrows) continue;
-        float* w = Wb + (int64_t)wrow * p.C + wcol;
-        if (wcol + 4 <= ncols) {
-            float4 wv = *reinterpret_cast<float4*>(w);
-            wv.x = wv.x * decay - lrs * ov.x;
-            wv.y = wv.y * decay - lrs * ov.y;
-            wv.z = wv.z * decay - lrs * ov.z;
-            wv.w = wv.w * decay - lrs * ov.w;
-            *reinterpret_cast<float4*>(w) = wv;
-        } else {
-            const float oe[4] = {ov.x, ov.y, ov.z, ov.w};
-            for (int e = 0; e < 4 && wcol + e < ncols; ++e) w[e] = w[e] * decay - lrs * oe[e];
+    } else {  // ragged right edge of W
+        for (int i = 0; i < 8; ++i) {
+            if (r0 + 4 * i >= nrows) continue;
+            const float* ov = reinterpret_cast<const float*>(stg + sw128(4 * i + sub, cq));
+            float* w = wbase + i * wstep;
+            for (int e = 0; e < 4 && c0 + e < ncols; ++e) w[e] = w[e] * decay - lrs * ov[e];
         }
     }
 }
