@@ -1,0 +1,184 @@
+"""Edge cases of the whole step on the GPU, against the oracle or bit for bit.
+
+* a mixed parameter table: bf16 and fp32 gradients of one shape (separate
+  buckets), a per-head fp32-mode group, an embedding, a bias, a 0-D scalar in
+  a group without weight decay, and empty tensors;
+* a workspace cap that splits buckets into sub-batches, and a bucket of more
+  than 256 matrices: results bit-identical to the unsplit plan;
+* 1 and 16 Newton-Schulz iterations;
+* resume: k steps, state copied into fresh buffers, more steps, bit for bit;
+* fp32 mode on larger matrices (1e-5).
+"""
+import numpy as np
+import pytest
+
+torch = pytest.importorskip("torch")
+
+import oracle
+import synth
+import adamw_hybrid_optimizer_muon_b200 as ma
+from gpu_helpers import (TOL_BF16, TOL_F32, bf16_round, check_muon, check_state, dev_f32, dev_grad, f32, host,
+                         momentum_terms)
+
+pytestmark = pytest.mark.gpu
+
+
+def _mhp(**kw):
+    base = dict(lr=0.02, beta=0.95, weight_decay=0.01, eps=1e-7, nesterov=True, ns_steps=5,
+                coeffs=((1.5, -0.5, 0.0),), scale_mode=0, heads=1, precision=0)
+    base.update(kw)
+    return base
+
+
+def _ahp(**kw):
+    base = dict(lr=0.01, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.01)
+    base.update(kw)
+    return base
+
+
+def _as32(d):
+    return {k: (f32(v) if isinstance(v, float) else v) for k, v in d.items()}
+
+
+def test_mixed_table_two_steps():
+    r = np.random.default_rng(200)
+    H, E = ma.ROLE_HIDDEN, ma.ROLE_EMBED
+    # (shape, role, group, grad dtype)
+    table = [((256, 512), H, 0, "bf16"), ((256, 512), H, 0, "f32"), ((384, 128), H, 1, "bf16"),
+             ((1000, 64), E, 2, "bf16"), ((37,), H, 2, "bf16"), ((), H, 3, "f32"), ((0,), H, 2, "bf16"),
+             ((0, 16), H, 0, "bf16"), ((256, 512), H, 0, "bf16")]
+    mg = [_mhp(), _mhp(heads=2, precision=1, nesterov=False, scale_mode=1)]
+    ag = [_ahp(), _ahp(lr=0.003, weight_decay=0.0)]
+    groups = [("muon", ma.muon_hparams(**mg[0])), ("muon", ma.muon_hparams(**mg[1])),
+              ("adamw", ma.adamw_hparams(**ag[0])), ("adamw", ma.adamw_hparams(**ag[1]))]
+    P0 = [(r.standard_normal(s) * 0.02).astype(np.float32) for s, *_ in table]
+    params = [dev_f32(p) for p in P0]
+    opt = ma.MuonAdamW([(p, role, g) for p, (s, role, g, _) in zip(params, table)], groups)
+    og = [dict(kind=0, **_as32(mg[0])), dict(kind=0, **_as32(mg[1])), dict(kind=1, **_as32(ag[0])),
+          dict(kind=1, **_as32(ag[1]))]
+    for step in (1, 2):
+        G = [bf16_round(r.standard_normal(s) * 1e-3) for s, *_ in table]
+        Gd = [dev_grad(g, dt) for g, (_, _, _, dt) in zip(G, table)]
+        before_p = [host(p) for p in params]
+        before_s = [(host(a), None if b is None else host(b)) for a, b in opt.state]
+        opt.step(Gd)
+        torch.cuda.synchronize()
+        assert ma.ma_device_status() == ma.MA_OK
+        for i, ((shape, role, g, _), p) in enumerate(zip(table, params)):
+            grp = og[g]
+            if grp["kind"] == 0:
+                if before_p[i].size == 0:
+                    continue
+                rw, rm = oracle.muon_update(before_p[i], G[i], before_s[i][0], grp["lr"], grp["beta"],
+                                            grp["weight_decay"], grp["nesterov"], grp["ns_steps"], grp["coeffs"],
+                                            grp["eps"], grp["scale_mode"], grp["heads"])
+                check_muon(before_p[i], host(p), rw, grp["lr"], grp["weight_decay"],
+                           TOL_F32 if grp["precision"] else TOL_BF16, what=f"tensor {i}")
+                check_state(host(opt.state[i][0]), rm, momentum_terms(before_s[i][0], G[i], grp["beta"]))
+            else:
+                args = (step, grp["lr"], grp["beta1"], grp["beta2"], grp["eps"], grp["weight_decay"])
+                rp, rm, rv = oracle.adamw_update(before_p[i], G[i], before_s[i][0], before_s[i][1], *args)
+                tp, tm, tv = oracle.adamw_term_magnitudes(before_p[i], G[i], before_s[i][0], before_s[i][1], *args)
+                check_state(host(p).reshape(-1), rp.reshape(-1), tp.reshape(-1), what=f"tensor {i}")
+                check_state(host(opt.state[i][0]).reshape(-1), rm.reshape(-1), tm.reshape(-1))
+                check_state(host(opt.state[i][1]).reshape(-1), rv.reshape(-1), tv.reshape(-1))
+
+
+def _run_bucket(shapes_count, steps, ws_cap=0, seed=1):
+    (R, C), n = shapes_count
+    r = np.random.default_rng(seed)
+    params = [dev_f32(r.standard_normal((R, C)) * 0.02) for _ in range(n)]
+    opt = ma.MuonAdamW([(p, ma.ROLE_HIDDEN, 0) for p in params], [("muon", ma.muon_hparams())], ws_cap=ws_cap)
+    for s in range(steps):
+        gr = np.random.default_rng(seed * 100 + s)
+        opt.step([dev_grad(bf16_round(gr.standard_normal((R, C)) * 1e-3), "bf16") for _ in range(n)])
+    torch.cuda.synchronize()
+    assert ma.ma_device_status() == ma.MA_OK
+    return params, opt
+
+
+def test_workspace_cap_sub_batches_are_bit_identical():
+    full, _ = _run_bucket(((256, 512), 7), 2)
+    per2 = ma.muon_workspace_bytes(2, 256, 512, ma.muon_hparams())
+    capped, opt = _run_bucket(((256, 512), 7), 2, ws_cap=per2)
+    assert opt._plan.ws_bytes <= per2
+    for a, b in zip(full, capped):
+        assert torch.equal(a, b)
+
+
+def test_bucket_of_more_than_256_matrices():
+    params, _ = _run_bucket(((64, 128), 300), 1, seed=3)
+    r = np.random.default_rng(3)
+    W0 = [r.standard_normal((64, 128)) * 0.02 for _ in range(300)]
+    gr = np.random.default_rng(300)
+    G = [bf16_round(gr.standard_normal((64, 128)) * 1e-3) for _ in range(300)]
+    hp = synth.MuonHP()
+    for i in (0, 255, 256, 299):  # both sides of the 256-matrix launch split
+        w0 = W0[i].astype(np.float32).astype(np.float64)
+        rw, _ = oracle.muon_update(w0, G[i], np.zeros((64, 128)), f32(hp.lr), f32(hp.beta), f32(hp.weight_decay),
+                                   eps=f32(hp.eps))
+        check_muon(w0, host(params[i]), rw, f32(hp.lr), f32(hp.weight_decay), TOL_BF16, what=f"matrix {i}")
+
+
+@pytest.mark.parametrize("steps", [1, 16])
+def test_ns_step_counts(steps):
+    R, C = 256, 512
+    r = np.random.default_rng(10 + steps)
+    W0 = (r.standard_normal((R, C)) * 0.02).astype(np.float32)
+    g = bf16_round(r.standard_normal((R, C)) * 1e-3)
+    hp = ma.muon_hparams(ns_steps=steps)
+    Wd, Md = [dev_f32(W0)], [torch.zeros((R, C), device="cuda")]
+    ws = torch.empty(ma.muon_workspace_bytes(1, R, C, hp), dtype=torch.uint8, device="cuda")
+    ma.muon_step_batched(Wd, [dev_grad(g, "bf16")], Md, hp, ws)
+    torch.cuda.synchronize()
+    rw, _ = oracle.muon_update(W0, g, np.zeros((R, C)), f32(0.02), f32(0.95), f32(0.01), steps=steps, eps=f32(1e-7))
+    check_muon(W0, host(Wd[0]), rw, f32(0.02), f32(0.01), TOL_BF16)
+
+
+def test_resume_from_copied_state_is_bit_identical():
+    wl = synth.tiny()
+    W0 = [synth.initial_weight(t, i) for i, t in enumerate(wl.tensors)]
+    grads = [[torch.from_numpy(synth.gradient(wl, i, s)).cuda() for i in range(2)] for s in (1, 2, 3)]
+
+    def make(params):
+        gm, ga = wl.groups[0].muon, wl.groups[1].adamw
+        return ma.MuonAdamW([(p, t.role, t.group) for p, t in zip(params, wl.tensors)],
+                            [("muon", ma.muon_hparams()), ("adamw", ma.adamw_hparams(ga.lr, ga.beta1, ga.beta2,
+                                                                                      ga.eps, ga.weight_decay))])
+    pa = [torch.from_numpy(w).cuda() for w in W0]
+    oa = make(pa)
+    for g in grads:
+        oa.step(g)
+    pb = [torch.from_numpy(w).cuda() for w in W0]
+    ob = make(pb)
+    for g in grads[:2]:
+        ob.step(g)
+    torch.cuda.synchronize()
+    # fresh buffers holding the copied parameters and state
+    pc = [p.clone() for p in pb]
+    oc = make(pc)
+    for (s0, s1), (t0, t1) in zip(ob.state, oc.state):
+        t0.copy_(s0)
+        if s1 is not None:
+            t1.copy_(s1)
+    oc.step_count = ob.step_count
+    oc.step(grads[2])
+    torch.cuda.synchronize()
+    for x, y in zip(pa, pc):
+        assert torch.equal(x, y)
+    for (s0, s1), (t0, t1) in zip(oa.state, oc.state):
+        assert torch.equal(s0, t0) and (s1 is None or torch.equal(s1, t1))
+
+
+@pytest.mark.parametrize("shape", [(1024, 2048), (2048, 1024)])
+def test_fp32_mode_larger(shape):
+    r = np.random.default_rng(20)
+    W0 = (r.standard_normal(shape) * 0.02).astype(np.float32)
+    g = (r.standard_normal(shape) * 1e-3).astype(np.float32)
+    hp = ma.muon_hparams(precision=1)
+    Wd, Md = [dev_f32(W0)], [torch.zeros(shape, device="cuda")]
+    ws = torch.empty(ma.muon_workspace_bytes(1, *shape, hp), dtype=torch.uint8, device="cuda")
+    ma.muon_step_batched(Wd, [dev_f32(g)], Md, hp, ws)
+    torch.cuda.synchronize()
+    rw, _ = oracle.muon_update(W0, g, np.zeros(shape), f32(0.02), f32(0.95), f32(0.01), eps=f32(1e-7))
+    check_muon(W0, host(Wd[0]), rw, f32(0.02), f32(0.01), TOL_F32)

@@ -143,6 +143,19 @@ def test_7b_full_size_sampled():
     _full_size_check("7b", n_muon_samples=1, adamw_samples=100_000)
 
 
+@pytest.mark.slow
+def test_aspect_full_size_sampled():
+    # MLP 4096x14336 (wide) and 14336x4096 (transpose path), Q/K/V as 32 heads of
+    # 128x4096, 10 % of units with rank-64 gradients
+    _full_size_check("aspect", n_muon_samples=1)
+
+
+@pytest.mark.slow
+def test_square_full_size_sampled():
+    # 64 matrices 4096^2, gradient scales spread over three decades
+    _full_size_check("square", n_muon_samples=2)
+
+
 @pytest.mark.parametrize("name", ["tiny", "d20"])
 def test_step_from_host_equals_resident_step(name):
     # gradients copied from pinned host memory, overlapped with compute, give
