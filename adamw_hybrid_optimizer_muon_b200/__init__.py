@@ -52,7 +52,8 @@ class MuonHParams(ctypes.Structure):
     _fields_ = [("lr", ctypes.c_float), ("beta", ctypes.c_float), ("weight_decay", ctypes.c_float),
                 ("eps", ctypes.c_float), ("nesterov", ctypes.c_int32), ("ns_steps", ctypes.c_int32),
                 ("n_coeffs", ctypes.c_int32), ("coeffs", (ctypes.c_float * 3) * MAX_NS_STEPS),
-                ("scale_mode", ctypes.c_int32), ("heads", ctypes.c_int32), ("precision", ctypes.c_int32)]
+                ("scale_mode", ctypes.c_int32), ("heads", ctypes.c_int32), ("precision", ctypes.c_int32),
+                ("cautious", ctypes.c_int32)]
 
 
 class AdamWHParams(ctypes.Structure):
@@ -173,7 +174,7 @@ def _dtype_code(t) -> int:
 
 
 def muon_hparams(lr=0.02, beta=0.95, weight_decay=0.01, eps=1e-7, nesterov=True, ns_steps=5,
-                 coeffs=((1.5, -0.5, 0.0),), scale_mode=0, heads=1, precision=0) -> MuonHParams:
+                 coeffs=((1.5, -0.5, 0.0),), scale_mode=0, heads=1, precision=0, cautious=False) -> MuonHParams:
     hp = MuonHParams()
     hp.lr, hp.beta, hp.weight_decay, hp.eps = lr, beta, weight_decay, eps
     hp.nesterov, hp.ns_steps, hp.n_coeffs = int(bool(nesterov)), int(ns_steps), len(coeffs)
@@ -182,6 +183,7 @@ def muon_hparams(lr=0.02, beta=0.95, weight_decay=0.01, eps=1e-7, nesterov=True,
     for k, (a, b, c) in enumerate(coeffs):
         hp.coeffs[k][0], hp.coeffs[k][1], hp.coeffs[k][2] = a, b, c
     hp.scale_mode, hp.heads, hp.precision = int(scale_mode), int(heads), int(precision)
+    hp.cautious = int(bool(cautious))
     return hp
 
 

@@ -269,6 +269,8 @@ int run_muon(int batch, const MuonGeom& g, float* const* W, const void* const* G
     p.C = g.C;
     p.decay = 1.f - hp.lr * hp.weight_decay;
     p.lr_s = hp.lr * shape_scale(g.Rh, g.C, hp.scale_mode);
+    p.lr_wd = hp.lr * hp.weight_decay;
+    p.cautious = hp.cautious ? 1 : 0;
     p.wait_limit_ns = host_wait_limit_ns();
     p.status = device_status_ptr();
     for (int b = 0; b < batch; ++b) p.W[b] = W[b];

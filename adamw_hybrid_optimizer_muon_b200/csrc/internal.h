@@ -91,6 +91,8 @@ struct NsParams {
     int32_t transposed, heads;
     int64_t Rh, C;
     float decay, lr_s;
+    float lr_wd;             // lr * wd, for cautious decay
+    int32_t cautious;        // decay only where X_N * W > 0
     long long wait_limit_ns;
     int* status;             // per-device status word
     float* W[MA_MAX_BATCH];

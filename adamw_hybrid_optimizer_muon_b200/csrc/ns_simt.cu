@@ -110,7 +110,8 @@ __global__ void __launch_bounds__(256) ns_simt_kernel(const __grid_constant__ Ns
                     const int bidx = u / p.heads, h = u - bidx * p.heads;
                     float* Wb = p.W[bidx] + (int64_t)h * p.Rh * p.C;
                     float* w = p.transposed ? Wb + (int64_t)j * p.C + i : Wb + (int64_t)i * p.C + j;
-                    *w = *w * p.decay - p.lr_s * o;
+                    const float wv = *w;
+                    *w = p.cautious ? (o * wv > 0.f ? wv - p.lr_wd * wv : wv) - p.lr_s * o : wv * p.decay - p.lr_s * o;
                 }
             }
         }

@@ -152,6 +152,13 @@ __device__ __forceinline__ void epilogue_values(const NsParams& p, const TileCoo
     }
 }
 
+// One weight: decoupled decay (optionally only where the update x and w agree in
+// sign, the cautious reading), then the scaled orthogonalised update.
+__device__ __forceinline__ float apply_update(float w, float x, float decay, float lrs, const NsParams& p) {
+    if (p.cautious) return (x * w > 0.f ? w - p.lr_wd * w : w) - lrs * x;
+    return w * decay - lrs * x;
+}
+
 // Byte offset of 16-byte chunk q of row r in a 128-byte-row block with a
 // 128-byte XOR swizzle (conflict-free for the row-wise and column-wise
 // accesses of the final apply).
@@ -205,10 +212,10 @@ __device__ __forceinline__ void epilogue_final(const NsParams& p, const TileCoor
                 if (r0 + 4 * i >= nrows) continue;
                 const float4 ov = *reinterpret_cast<const float4*>(stg + sw128(4 * i + sub, cq));
                 float4 w = wv[k];
-                w.x = w.x * decay - lrs * ov.x;
-                w.y = w.y * decay - lrs * ov.y;
-                w.z = w.z * decay - lrs * ov.z;
-                w.w = w.w * decay - lrs * ov.w;
+                w.x = apply_update(w.x, ov.x, decay, lrs, p);
+                w.y = apply_update(w.y, ov.y, decay, lrs, p);
+                w.z = apply_update(w.z, ov.z, decay, lrs, p);
+                w.w = apply_update(w.w, ov.w, decay, lrs, p);
                 *reinterpret_cast<float4*>(wbase + i * wstep) = w;
             }
         }
@@ -217,7 +224,7 @@ __device__ __forceinline__ void epilogue_final(const NsParams& p, const TileCoor
             if (r0 + 4 * i >= nrows) continue;
             const float* ov = reinterpret_cast<const float*>(stg + sw128(4 * i + sub, cq));
             float* w = wbase + i * wstep;
-            for (int e = 0; e < 4 && c0 + e < ncols; ++e) w[e] = w[e] * decay - lrs * ov[e];
+            for (int e = 0; e < 4 && c0 + e < ncols; ++e) w[e] = apply_update(w[e], ov[e], decay, lrs, p);
         }
     }
 }

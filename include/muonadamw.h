@@ -87,12 +87,17 @@ typedef enum {
  *  heads: rows split into `heads` equal slices, each orthogonalised on its own
  *      [P2 per-head orthogonalisation]; 1 = the whole matrix.
  *  precision: 0 = bf16 tensor-core operands with fp32 accumulation;
- *      1 = fp32 arithmetic throughout (a correctness mode). */
+ *      1 = fp32 arithmetic throughout (a correctness mode).
+ *  cautious: nonzero applies the weight decay only where the orthogonalised
+ *      update O and the weight W have the same sign (O*W > 0), i.e. where the
+ *      update already moves W towards zero. [P1 "Muon Step Implementation"]
+ *      names "cautious weight decay" without defining it; this is a reading. */
 typedef struct {
     float lr, beta, weight_decay, eps;
     int32_t nesterov, ns_steps, n_coeffs;
     float coeffs[MA_MAX_NS_STEPS][3];
     int32_t scale_mode, heads, precision;
+    int32_t cautious;
 } ma_muon_hparams_t;
 
 /* AdamW hyperparameters [P1 "AdamW Step Implementation"; P3 _finish: bias

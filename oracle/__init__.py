@@ -31,7 +31,8 @@ Readings where the pages are silent (each one is listed in the design notes):
 * Nesterov form ``u = beta*m_new + (1-beta)*g``.
 * Shape scale ``s = sqrt(max(1, R/C))`` (mode 0), ``sqrt(R/C)`` (mode 1),
   or 1 (mode 2).
-* Decoupled weight decay ``W*(1 - lr*wd)``, applied to the pre-update weight.
+* Decoupled weight decay ``W*(1 - lr*wd)``, applied to the pre-update weight;
+  the cautious option decays only where the update and the weight share a sign.
 * AdamW eps is added after the bias-corrected square root.
 * Head h of an R x C matrix split into H heads is rows [h*R/H, (h+1)*R/H).
 
@@ -214,7 +215,7 @@ def shape_scale(R, C, mode=0):
 
 
 def muon_update(W, g, m, lr, beta, weight_decay, nesterov=True, steps=DEFAULT_NS_STEPS,
-                coeffs=(CUBIC,), eps=1e-7, scale_mode=0, heads=1):
+                coeffs=(CUBIC,), eps=1e-7, scale_mode=0, heads=1, cautious=False):
     """One Muon step on one R x C matrix. Returns new (W, m) as float64.
 
     Steps, in the order of "Muon Step Implementation": momentum (plus
@@ -222,6 +223,11 @@ def muon_update(W, g, m, lr, beta, weight_decay, nesterov=True, steps=DEFAULT_NS
     back. With ``heads > 1`` each block of R/heads rows is orthogonalised on
     its own (Qwen "Confirmed": per-head orthogonalisation), and the scale uses
     the slice shape.
+
+    ``cautious``: the same page names "cautious weight decay" without defining
+    it. The reading taken: decay only the elements where the orthogonalised
+    update O and the pre-update weight W have the same sign (O*W > 0). Parity
+    of this reading is unpinned by the pages.
     """
     W = np.asarray(W, dtype=np.float64)
     R, C = W.shape
@@ -233,7 +239,10 @@ def muon_update(W, g, m, lr, beta, weight_decay, nesterov=True, steps=DEFAULT_NS
     for h in range(heads):
         sl = slice(h * rh, (h + 1) * rh)
         O[sl] = shape_scale(rh, C, scale_mode) * orthogonalize(u[sl], coeffs, steps, eps)
-    W_new = W * (1.0 - lr * weight_decay) - lr * O
+    if cautious:
+        W_new = W - lr * weight_decay * W * (O * W > 0) - lr * O
+    else:
+        W_new = W * (1.0 - lr * weight_decay) - lr * O
     return W_new, m_new
 
 
@@ -269,7 +278,8 @@ def muonadamw_step(tensors, groups, params, grads, state, step):
             m = st.get("m", np.zeros_like(p))
             p, st["m"] = muon_update(
                 p, g, m, grp["lr"], grp["beta"], grp["weight_decay"], grp["nesterov"],
-                grp["ns_steps"], grp["coeffs"], grp["eps"], grp["scale_mode"], grp["heads"])
+                grp["ns_steps"], grp["coeffs"], grp["eps"], grp["scale_mode"], grp["heads"],
+                grp.get("cautious", False))
         out.append(p)
     return out
 

@@ -57,6 +57,7 @@ class MuonHP:
     scale_mode: int = 0  # 0: sqrt(max(1,R/C)), 1: sqrt(R/C), 2: 1
     heads: int = 1
     precision: int = 0  # 0: bf16 operands, 1: fp32 compute
+    cautious: bool = False  # decay only where update and weight share a sign
 
 
 @dataclasses.dataclass

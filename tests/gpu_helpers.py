@@ -90,7 +90,7 @@ def check_muon(W_old, W_new_gpu, W_new_ref, lr, wd, tol, what="muon"):
 
 def oracle_muon(W, g, m, hp: synth.MuonHP):
     return oracle.muon_update(W, g, m, hp.lr, hp.beta, hp.weight_decay, hp.nesterov, hp.ns_steps, hp.coeffs,
-                              hp.eps, hp.scale_mode, hp.heads)
+                              hp.eps, hp.scale_mode, hp.heads, hp.cautious)
 
 
 def momentum_terms(m_old, g, beta):

@@ -134,16 +134,18 @@ MUON_CASES = [
 ]
 
 
-def _muon_run(shape, heads, nesterov, mode, coeffs, precision, gdt, batch=2, steps=2, seed=0):
+def _muon_run(shape, heads, nesterov, mode, coeffs, precision, gdt, batch=2, steps=2, seed=0, cautious=False,
+              wd=0.01):
     R, C = shape
     hp = hp32(synth.MuonHP(nesterov=nesterov, scale_mode=mode, heads=heads, precision=precision,
-                           coeffs=tuple(coeffs), ns_steps=len(coeffs) if len(coeffs) > 1 else 5))
+                           coeffs=tuple(coeffs), ns_steps=len(coeffs) if len(coeffs) > 1 else 5, cautious=cautious,
+                           weight_decay=wd))
     r = np.random.default_rng(seed)
     W = [(r.standard_normal(shape) * 0.02).astype(np.float32) for _ in range(batch)]
     Wd = [dev_f32(w) for w in W]
     Md = [torch.zeros(shape, device="cuda") for _ in range(batch)]
     mhp = ma.muon_hparams(hp.lr, hp.beta, hp.weight_decay, hp.eps, hp.nesterov, hp.ns_steps, hp.coeffs,
-                          hp.scale_mode, hp.heads, hp.precision)
+                          hp.scale_mode, hp.heads, hp.precision, hp.cautious)
     ws = torch.empty(ma.muon_workspace_bytes(batch, R, C, mhp), dtype=torch.uint8, device="cuda")
     errs = []
     for step in range(steps):
@@ -171,6 +173,36 @@ def test_muon_fp32_mode_parity(case):
 @pytest.mark.parametrize("gdt", ["bf16", "f32"])
 def test_muon_bf16_parity(case, gdt):
     _muon_run(*case, precision=0, gdt=gdt)
+
+
+@pytest.mark.parametrize("shape", [(256, 512), (512, 256), (200, 136)])
+@pytest.mark.parametrize("precision", [0, 1])
+def test_muon_cautious_decay(shape, precision):
+    # The decay mask (O*W > 0) is decided in floating point, so where O is near
+    # zero the GPU and the fp64 oracle may decide differently. The test reads
+    # the GPU's decision back, requires it to match the oracle wherever |O| is
+    # not small, and checks values under the GPU's own decision. A large decay
+    # makes the two candidate values of every element far apart.
+    R, C = shape
+    lr, beta, wd, eps = f32(0.02), f32(0.95), f32(5.0), f32(1e-7)
+    r = np.random.default_rng(40)
+    W0 = (r.standard_normal(shape) * 0.02).astype(np.float32).astype(np.float64)
+    g = bf16_round(r.standard_normal(shape) * 1e-3)
+    hp = ma.muon_hparams(lr=lr, beta=beta, weight_decay=wd, eps=eps, precision=precision, cautious=True)
+    Wd, Md = [dev_f32(W0)], [torch.zeros(shape, device="cuda")]
+    ws = torch.empty(ma.muon_workspace_bytes(1, R, C, hp), dtype=torch.uint8, device="cuda")
+    ma.muon_step_batched(Wd, [dev_grad(g, "bf16")], Md, hp, ws)
+    torch.cuda.synchronize()
+    got = host(Wd[0])
+    W_nodecay, _ = oracle.muon_update(W0, g, np.zeros(shape), lr, beta, 0.0, eps=eps)
+    O = (W0 - W_nodecay) / lr                       # scaled orthogonalised update
+    decayed = (1 - lr * wd) * W0 - lr * O
+    kept = W0 - lr * O
+    gpu_mask = np.abs(got - decayed) < np.abs(got - kept)
+    ref_mask = O * W0 > 0
+    clear = np.abs(O) > 0.05 * np.sqrt(np.mean(O * O))
+    assert np.array_equal(gpu_mask[clear], ref_mask[clear])
+    check_muon(W0, got, np.where(gpu_mask, decayed, kept), lr, wd, TOL_F32 if precision else TOL_BF16)
 
 
 @pytest.mark.parametrize("precision", [0, 1])

@@ -312,3 +312,26 @@ def test_bf16_storage_roundtrip_is_exact():
     # ties go to even
     t = np.array([np.float32(1.0) + np.float32(2 ** -8)], dtype=np.float32)
     assert synth.bf16_bits_to_f32(synth.f32_to_bf16_bits(t))[0] == 1.0
+
+
+@pytest.mark.parametrize("shape", [(16, 40), (40, 16)])
+def test_cautious_decay_closed_form(shape):
+    # O from the SVD closed form; the decay mask follows the sign agreement of O and W
+    lr, beta, wd, eps = 0.02, 0.95, 0.1, 1e-7
+    r = rng(30)
+    g = r.standard_normal(shape) * 1e-3
+    U, S, Vt = np.linalg.svd(g, full_matrices=False)
+    c = (1 - beta) * (1 + beta)
+    R, C = shape
+    O = math.sqrt(max(1.0, R / C)) * (U * p_scalar(c * S / (c * np.linalg.norm(g) + eps), [oracle.CUBIC], 5)) @ Vt
+    mag = np.abs(r.standard_normal(shape)) * 0.02
+    for W0, expect in ((np.sign(O) * mag, (1 - lr * wd) * np.sign(O) * mag - lr * O),     # all agree: full decay
+                       (-np.sign(O) * mag, -np.sign(O) * mag - lr * O)):                    # none agree: no decay
+        W1, _ = oracle.muon_update(W0, g, np.zeros(shape), lr, beta, wd, cautious=True)
+        assert np.allclose(W1, expect, rtol=1e-12, atol=1e-15)
+    W0 = r.standard_normal(shape) * 0.02   # mixed signs
+    W1, _ = oracle.muon_update(W0, g, np.zeros(shape), lr, beta, wd, cautious=True)
+    agree = O * W0 > 0
+    assert 0 < agree.sum() < agree.size
+    assert np.allclose(W1[agree], ((1 - lr * wd) * W0 - lr * O)[agree], rtol=1e-12, atol=1e-15)
+    assert np.allclose(W1[~agree], (W0 - lr * O)[~agree], rtol=1e-12, atol=1e-15)
