@@ -232,6 +232,7 @@ def workload_config(wl, n_gpus):
     return {"workload": f"{wl.name}: {wl.description}", "params": wl.numel,
             "muon_matrices": kinds.count(0), "adamw_tensors": kinds.count(1),
             "ns_steps": wl.groups[0].muon.ns_steps if wl.groups[0].kind == 0 else None,
+            "ns_coeffs": [list(c) for c in wl.groups[0].muon.coeffs] if wl.groups[0].kind == 0 else None,
             "l2": "inputs larger than L2 (no flush needed)", "parallelism": f"replicas x{n_gpus}"}
 
 
@@ -246,6 +247,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--coeffs", default=None,
+                    help="Newton-Schulz polynomial per iteration, 'a,b,c[;a,b,c...]' (default: the cubic 1.5,-0.5,0)")
     args = ap.parse_args()
     rank, world, local = env_int("RANK", 0), env_int("WORLD_SIZE", 1), env_int("LOCAL_RANK", 0)
     if args.impl == "reference":
@@ -267,6 +270,13 @@ def main():
             dist.barrier()
 
     wl = synth.WORKLOADS[args.workload]()
+    if args.coeffs:
+        co = tuple(tuple(float(x) for x in t.split(",")) for t in args.coeffs.split(";"))
+        for g in wl.groups:
+            if g.kind == synth.KIND_MUON:
+                g.muon.coeffs = co
+                if len(co) > 1:
+                    g.muon.ns_steps = len(co)
     params = sdev.weights(wl, device=dev, base=rank)
     grads = sdev.gradients(wl, 1, device=dev, base=rank)
     groups = []
