@@ -68,7 +68,17 @@ constexpr uint32_t STG_BLOCK = 32 * 32 * 2;
 #endif
 constexpr uint32_t kEpiSleepNs = MA_EPI_SLEEP_NS;
 constexpr uint32_t STG_BYTES = EPI_WARPS * 2 * STG_BLOCK;  // 32 KB
-constexpr size_t SMEM_BYTES = (size_t)STAGES * STAGE_BYTES + STG_BYTES + 1024 /*align*/ + 256 /*barriers*/;
+// Final apply: each epilogue warp double-buffers 32 x 32 fp32 blocks of W,
+// rows padded to 144 bytes (conflict-free row and column access).
+constexpr uint32_t WROW = 144;
+constexpr uint32_t WBUF = 32 * WROW;                        // 4.5 KB
+constexpr uint32_t WBUF_BYTES = EPI_WARPS * 2 * WBUF;       // 72 KB
+constexpr int kStages(int mode) { return mode == NS_FINAL ? 4 : STAGES; }
+constexpr uint32_t kEpiBytes(int mode) { return mode == NS_FINAL ? WBUF_BYTES : STG_BYTES; }
+constexpr size_t kSmemBytes(int mode) {
+    return (size_t)kStages(mode) * STAGE_BYTES + kEpiBytes(mode) + 1024 /*align*/ + 512 /*barriers*/;
+}
+constexpr size_t SMEM_BYTES = kSmemBytes(NS_GRAM);
 
 struct TileCoord {
     int u, ti, tj;
@@ -159,74 +169,115 @@ __device__ __forceinline__ float apply_update(float w, float x, float decay, flo
     return w * decay - lrs * x;
 }
 
-// Byte offset of 16-byte chunk q of row r in a 128-byte-row block with a
-// 128-byte XOR swizzle (conflict-free for the row-wise and column-wise
-// accesses of the final apply).
-__device__ __forceinline__ uint32_t sw128(uint32_t r, uint32_t q) { return r * 128u + ((q ^ (r & 7u)) << 4); }
 
-// Final apply: W <- W*(1 - lr*wd) - lr*scale*X_N in the caller's fp32 weights.
-// The warp's 32 x 32 fp32 block of X_N is staged in shared memory in the
-// orientation of W (transposed back when the unit was tall), then each lane
-// handles 4 consecutive elements of one W row: every read and write of W is
-// a 16-byte access and each group of 8 lanes covers one 128-byte row segment.
-__device__ __forceinline__ void epilogue_final(const NsParams& p, const TileCoord& tc, int row_lo, int col0,
-                                               const float (&o)[32], uint8_t* stg, int lane) {
-    __syncwarp();  // the previous chunk's reads of the staging block are done
-    if (!p.transposed) {
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-            *reinterpret_cast<float4*>(stg + sw128(lane, q)) =
-                make_float4(o[4 * q + 0], o[4 * q + 1], o[4 * q + 2], o[4 * q + 3]);
-    } else {
-#pragma unroll
-        for (int t = 0; t < 32; ++t)
-            *reinterpret_cast<float*>(stg + sw128(t, (uint32_t)lane >> 2) + (lane & 3) * 4) = o[t];
-    }
-    __syncwarp();
+// Final apply: W <- W*(1 - lr*wd) - lr*scale*X_N in the caller's fp32 weights,
+// run by each epilogue warp over its four 32-column chunks of every tile.
+//
+// The chunk's 32 x 32 block of W (in W's own orientation: transposed back
+// when the unit was tall) comes into one of two shared-memory buffers by
+// 16-byte asynchronous copies, 8 lanes per 128-byte row. The first two chunks
+// of a tile are fetched before the accumulator is ready, and each later chunk
+// while the one before it is being computed, so the weights' DRAM latency
+// hides behind the main loop without holding registers. Each lane then
+// updates its own row (or, transposed, its own column) of the block in place
+// from X_N in its registers, and the block goes back to W with coalesced
+// 16-byte stores.
+__device__ __forceinline__ void final_epilogue(const NsParams& p, int tiles_per_unit, int mt, int nt, int pair,
+                                               int npairs, int total_tiles, uint32_t rank, uint32_t tmem_base,
+                                               int warp, int lane, uint8_t* wbuf, uint64_t* wbar,
+                                               uint64_t* acc_full, uint64_t* acc_empty, volatile int* abort_flag,
+                                               long long limit) {
+    const int quad = warp & 3, half = (warp - 2) / 4;
     const int m = p.m, n = p.n;
-    const int bidx = tc.u / p.heads, h = tc.u - bidx * p.heads;
-    float* Wb = p.W[bidx] + (int64_t)h * p.Rh * p.C;
+    const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
+    const uint32_t acc_empty_leader1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
     const float decay = p.decay, lrs = p.lr_s;
-    const int sub = lane >> 3, cq = lane & 7;
-    // This lane's 8 groups of 4 W elements lie 4 rows apart in W in either
-    // orientation. They are loaded in two batches of 4 (all loads of a batch
-    // in flight together), so the chunk waits for DRAM twice.
-    int r0, c0, nrows, ncols;
-    if (!p.transposed) {  // W row = X row, W column = X column
-        r0 = row_lo + sub; c0 = col0 + cq * 4; nrows = m; ncols = n;
-    } else {              // W row = X column, W column = X row
-        r0 = col0 + sub; c0 = row_lo + cq * 4; nrows = n; ncols = m;
-    }
-    float* wbase = Wb + (int64_t)r0 * p.C + c0;
-    const int64_t wstep = 4 * (int64_t)p.C;
-    if (c0 + 4 <= ncols) {
-#pragma unroll 1
-        for (int i0 = 0; i0 < 8; i0 += 4) {
-            float4 wv[4];
+    int lt = 0;
+    for (int t = pair; t < total_tiles; t += npairs, ++lt) {
+        const TileCoord tc = decode_tile(NS_FINAL, t, tiles_per_unit, mt, nt);
+        const int acc = lt & 1;
+        const uint32_t use = (uint32_t)(lt >> 1);
+        const int row_lo = tc.ti * BM + (int)rank * HM + quad * 32;
+        const int bidx = tc.u / p.heads, h = tc.u - bidx * p.heads;
+        float* Wb = p.W[bidx] + (int64_t)h * p.Rh * p.C;
+        // geometry of chunk c's W block: its first W row, first W column, and extents
+        auto block = [&](int c, int& r0, int& c0, int& nr, int& rb) -> bool {
+            const int col0 = tc.tj * BN + (half * 4 + c) * 32;
+            if (row_lo >= m || col0 >= n) return false;
+            if (!p.transposed) { r0 = row_lo; c0 = col0; nr = min(32, m - row_lo); rb = min(32, n - col0) * 4; }
+            else { r0 = col0; c0 = row_lo; nr = min(32, n - col0); rb = min(32, m - row_lo) * 4; }
+            return true;
+        };
+        auto fetch = [&](int c) {
+            int r0, c0, nr, rb;
+            if (c < 4 && block(c, r0, c0, nr, rb)) {
+                uint8_t* buf = wbuf + (c & 1) * WBUF;
 #pragma unroll
-            for (int k = 0; k < 4; ++k)
-                if (r0 + 4 * (i0 + k) < nrows) wv[k] = *reinterpret_cast<const float4*>(wbase + (i0 + k) * wstep);
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-                const int i = i0 + k;
-                if (r0 + 4 * i >= nrows) continue;
-                const float4 ov = *reinterpret_cast<const float4*>(stg + sw128(4 * i + sub, cq));
-                float4 w = wv[k];
-                w.x = apply_update(w.x, ov.x, decay, lrs, p);
-                w.y = apply_update(w.y, ov.y, decay, lrs, p);
-                w.z = apply_update(w.z, ov.z, decay, lrs, p);
-                w.w = apply_update(w.w, ov.w, decay, lrs, p);
-                *reinterpret_cast<float4*>(wbase + i * wstep) = w;
+                for (int i = 0; i < 8; ++i) {
+                    const int row = 4 * i + (lane >> 3), q = lane & 7;
+                    if (row < nr && q * 16 < rb)
+                        cp_async16(buf + row * WROW + q * 16, Wb + (int64_t)(r0 + row) * p.C + c0 + q * 4);
+                }
             }
+            cp_async_commit();  // one group per chunk, empty or not, so the counts line up
+        };
+        fetch(0);
+        fetch(1);
+        int ok = 1;
+        if (lane == 0) ok = mbar_wait_bounded(&acc_full[acc], use & 1u, abort_flag, limit, p.status, kEpiSleepNs) ? 1 : 0;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) break;
+        tc_fence_after();
+#pragma unroll 1
+        for (int c = 0; c < 4; ++c) {
+            int r0, c0, nr, rb;
+            if (!block(c, r0, c0, nr, rb)) break;  // warp-uniform
+            const int col0 = tc.tj * BN + (half * 4 + c) * 32;
+            uint8_t* buf = wbuf + (c & 1) * WBUF;
+            float v[32], o[32];
+            tmem_ld32(tmem_base + (uint32_t)(acc * BN + (half * 4 + c) * 32) + ((uint32_t)(quad * 32) << 16), v);
+            epilogue_values<NS_FINAL>(p, tc, row_lo + lane, col0, v, o);
+            // chunk c's copies are the oldest group but one (chunk c + 1 was issued after it)
+            cp_async_wait<1>();
+            __syncwarp();
+            if (!p.transposed) {
+                // lane = row of W: 32 consecutive elements
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    float4* wq = reinterpret_cast<float4*>(buf + lane * WROW + q * 16);
+                    float4 w = *wq;
+                    w.x = apply_update(w.x, o[4 * q + 0], decay, lrs, p);
+                    w.y = apply_update(w.y, o[4 * q + 1], decay, lrs, p);
+                    w.z = apply_update(w.z, o[4 * q + 2], decay, lrs, p);
+                    w.w = apply_update(w.w, o[4 * q + 3], decay, lrs, p);
+                    *wq = w;
+                }
+            } else {
+                // lane = column of W: element t of the lane's X_N row is W[t][lane]
+#pragma unroll
+                for (int q = 0; q < 32; ++q) {
+                    float* wq = reinterpret_cast<float*>(buf + q * WROW + lane * 4);
+                    *wq = apply_update(*wq, o[q], decay, lrs, p);
+                }
+            }
+            __syncwarp();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int row = 4 * i + (lane >> 3), q = lane & 7;
+                if (row < nr && q * 16 < rb)
+                    *reinterpret_cast<float4*>(Wb + (int64_t)(r0 + row) * p.C + c0 + q * 4) =
+                        *reinterpret_cast<const float4*>(buf + row * WROW + q * 16);
+            }
+            __syncwarp();  // the buffer is free again
+            fetch(c + 2);
         }
-    } else {  // ragged right edge of W
-        for (int i = 0; i < 8; ++i) {
-            if (r0 + 4 * i >= nrows) continue;
-            const float* ov = reinterpret_cast<const float*>(stg + sw128(4 * i + sub, cq));
-            float* w = wbase + i * wstep;
-            for (int e = 0; e < 4 && c0 + e < ncols; ++e) w[e] = apply_update(w[e], ov[e], decay, lrs, p);
-        }
+        cp_async_wait<0>();  // drop the copies of chunks this tile does not use
+        if (!ok) break;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);
     }
+    cp_async_wait<0>();
 }
 
 // Byte offset of 16-byte chunk q of row r in a 64-byte-row block with the
@@ -240,13 +291,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                  int mt, int nt, int kblocks) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* staging = smem + STAGES * STAGE_BYTES;
-    uint64_t* full = reinterpret_cast<uint64_t*>(staging + STG_BYTES);
-    uint64_t* empty = full + STAGES;
-    uint64_t* acc_full = empty + STAGES;
+    constexpr int NST = kStages(MODE);
+    uint8_t* staging = smem + NST * STAGE_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(staging + kEpiBytes(MODE));
+    uint64_t* empty = full + NST;
+    uint64_t* acc_full = empty + NST;
     uint64_t* acc_empty = acc_full + 2;
     uint64_t* drain = acc_empty + 2;
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* wbar = drain + 1;  // final apply: 2 per epilogue warp
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(wbar + 2 * EPI_WARPS);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -258,10 +311,11 @@ __global__ void __launch_bounds__(THREADS, 1)
     constexpr bool kApply = (MODE == NS_APPLY || MODE == NS_FINAL);
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < NST; ++s) {
             mbar_init(&full[s], 1);   // leader: its own arrive.expect_tx + both CTAs' bytes
             mbar_init(&empty[s], 1);  // both: one multicast commit per use
         }
+        for (int w = 0; w < 2 * EPI_WARPS; ++w) mbar_init(&wbar[w], 1);
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);                  // both: one multicast commit per tile
             mbar_init(&acc_empty[a], 2 * EPI_WARPS);     // leader: every epilogue warp of the pair
@@ -308,7 +362,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         for (int q = 0; q < HN / 64; ++q)
                             tma_load_3d_pair(sb + q * (64 * BK * 2), &mapB, fb, bcol + q * 64, kb * BK, tc.u);
                     }
-                    if (++stage == STAGES) {
+                    if (++stage == NST) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -316,9 +370,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             // Tail: wait until the MMAs have released every stage this CTA filled,
             // so that no commit arrives on this CTA's barriers after it exits.
-            for (int i = 0; i < STAGES && ok; ++i) {
+            for (int i = 0; i < NST && ok; ++i) {
                 ok = mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit, p.status);
-                if (++stage == STAGES) {
+                if (++stage == NST) {
                     stage = 0;
                     phase ^= 1u;
                 }
@@ -359,7 +413,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         tc_mma_f16_pair(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
                     }
                     tc_commit_pair_mc(&empty[stage], 0x3);
-                    if (++stage == STAGES) {
+                    if (++stage == NST) {
                         stage = 0;
                         phase ^= 1u;
                     }
@@ -373,6 +427,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 mbar_wait_bounded(drain, 0, abort_flag, limit, p.status);
             }
         }
+    } else if (MODE == NS_FINAL) {
+        final_epilogue(p, tiles_per_unit, mt, nt, pair, npairs, total_tiles, rank, tmem_base, warp, lane,
+                       staging + (warp - 2) * 2 * WBUF, &wbar[2 * (warp - 2)], acc_full, acc_empty, abort_flag, limit);
     } else {
         const int quad = warp & 3;              // TMEM lanes [32*quad, 32*quad + 32)
         const int half = (warp - 2) / 4;        // which half of the 256 columns
@@ -402,10 +459,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                 float v[32], o[32];
                 tmem_ld32(tmem_base + (uint32_t)(acc * BN + cc * 32) + ((uint32_t)(quad * 32) << 16), v);
                 epilogue_values<MODE>(p, tc, row, col0, v, o);
-                if (MODE == NS_FINAL) {
-                    epilogue_final(p, tc, row_lo, col0, o, stg, lane);
-                    continue;
-                }
                 // Stage this warp's 32 x 32 block (and, for an off-diagonal Gram
                 // chunk, its transpose), then write both with bulk tensor stores:
                 // each leaves shared memory as contiguous 64-byte rows.
@@ -527,7 +580,7 @@ cudaError_t launch_mode(const NsParams& p, const void* x_buf, const void* g_buf,
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     if (!(attr_set & (1ull << dev))) {
-        e = cudaFuncSetAttribute(ns_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_BYTES);
+        e = cudaFuncSetAttribute(ns_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes(MODE));
         if (e != cudaSuccess) return e;
         e = cudaFuncSetAttribute(ns_tc_kernel<MODE>, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
         if (e != cudaSuccess) return e;
@@ -539,7 +592,7 @@ cudaError_t launch_mode(const NsParams& p, const void* x_buf, const void* g_buf,
         qa[0].val.clusterDim.z = 1;
         qc.gridDim = dim3(2 * (unsigned)(num_sms / 2));
         qc.blockDim = dim3(THREADS);
-        qc.dynamicSmemBytes = SMEM_BYTES;
+        qc.dynamicSmemBytes = kSmemBytes(MODE);
         qc.attrs = qa;
         qc.numAttrs = 1;
         int nclusters = 0;
@@ -558,7 +611,7 @@ cudaError_t launch_mode(const NsParams& p, const void* x_buf, const void* g_buf,
     attr[0].val.clusterDim.z = 1;
     cfg.gridDim = dim3((unsigned)(2 * pairs));
     cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = SMEM_BYTES;
+    cfg.dynamicSmemBytes = kSmemBytes(MODE);
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
