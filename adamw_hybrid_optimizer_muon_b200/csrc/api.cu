@@ -86,6 +86,9 @@ constexpr size_t kAlign = 256;
 // large enough to keep every GEMM launch many waves deep.
 constexpr int kFromHostFirstBatch = 8;
 constexpr int kFromHostBatch = 32;
+// Workspace that a plan may use, beyond its largest sub-batch, to run small
+// Muon buckets through shared Newton-Schulz launches.
+constexpr size_t kGroupWsBytes = size_t(4) << 30;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 int64_t round8(int64_t x) { return (x + 7) / 8 * 8; }
@@ -208,24 +211,45 @@ double ns_flops(int mode, int64_t units, int64_t m, int64_t n) {
     return u * 2.0 * M * M * N;
 }
 
-// All checks passed; launch the whole Muon chain for one batch.
-int run_muon(int batch, const MuonGeom& g, float* const* W, const void* const* G, int gdt, float* const* M,
-             const ma_muon_hparams_t& hp, void* ws, cudaStream_t s, int sms, int* launches) {
-    if (g.total == 0) return MA_OK;
-    uint8_t* base = reinterpret_cast<uint8_t*>(ws);
-    void* X0 = base + g.off_x0;
-    void* X1 = base + g.off_x1;
-    void* Gb = base + g.off_g;
-    void* G2 = base + g.off_g2;
-    double* part = reinterpret_cast<double*>(base + g.off_part);
-    float* scale = reinterpret_cast<float*>(base + g.off_scale);
+// One Muon batch of same-shape matrices with its own workspace (g.total bytes).
+struct MuonJob {
+    int batch;
+    MuonGeom g;
+    float* const* W;
+    const void* const* G;
+    int gdt;
+    float* const* M;
+    const ma_muon_hparams_t* hp;
+    uint8_t* ws;
+};
 
+// Bit k set: Newton-Schulz iteration k has c != 0 (it needs the A^2 term).
+uint32_t quint_mask(const ma_muon_hparams_t& hp) {
+    uint32_t mask = 0;
+    for (int k = 0; k < hp.ns_steps && k < MA_MAX_NS_STEPS; ++k)
+        if (hp.coeffs[hp.n_coeffs == 1 ? 0 : k][2] != 0.f) mask |= 1u << k;
+    return mask;
+}
+
+// Jobs can share Newton-Schulz launches when they take the same sequence of
+// kernels: the tensor-core path, the same number of iterations and the same
+// iterations with an A^2 term. Coefficients, learning rates and decay may differ.
+bool ns_compatible(const ma_muon_hparams_t& x, const ma_muon_hparams_t& y) {
+    return x.precision == 0 && y.precision == 0 && x.ns_steps == y.ns_steps && quint_mask(x) == quint_mask(y);
+}
+
+// Momentum + norm partials, then the norm finalize, of one job.
+int muon_prep(const MuonJob& j, cudaStream_t s, int* launches) {
+    const MuonGeom& g = j.g;
+    const ma_muon_hparams_t& hp = *j.hp;
+    double* part = reinterpret_cast<double*>(j.ws + g.off_part);
+    float* scale = reinterpret_cast<float*>(j.ws + g.off_scale);
     MuonPrepLaunch P;
     std::memset(&P, 0, sizeof(P));
-    P.batch = batch;
+    P.batch = j.batch;
     P.heads = g.heads;
     P.transposed = g.transposed;
-    P.gdt = gdt;
+    P.gdt = j.gdt;
     P.nesterov = hp.nesterov ? 1 : 0;
     P.x_f32 = hp.precision ? 1 : 0;
     P.C = g.C;
@@ -236,83 +260,137 @@ int run_muon(int batch, const MuonGeom& g, float* const* W, const void* const* G
     P.tiles_c = (g.C + kPrepTile - 1) / kPrepTile;
     P.beta = hp.beta;
     P.omb = 1.f - hp.beta;
-    P.X = X0;
+    P.X = j.ws + g.off_x0;
     P.partials = part;
-    for (int b = 0; b < batch; ++b) {
-        P.G[b] = G[b];
-        P.M[b] = M[b];
+    for (int b = 0; b < j.batch; ++b) {
+        P.G[b] = j.G[b];
+        P.M[b] = j.M[b];
     }
     const double elems = (double)g.units * (double)g.Rh * (double)g.C;
     int pr = prof_begin(MA_PROF_MOMENTUM, s);
     int st = cuda_status(launch_muon_prep(P, s));
-    prof_end(pr, s, 0.0, elems * ((gdt == MA_BF16 ? 2 : 4) + 8 + (hp.precision ? 4 : 2)));
+    prof_end(pr, s, 0.0, elems * ((j.gdt == MA_BF16 ? 2 : 4) + 8 + (hp.precision ? 4 : 2)));
     if (st) return st;
     pr = prof_begin(MA_PROF_FINALIZE, s);
     st = cuda_status(launch_norm_finalize(part, g.parts, (int)g.units, hp.eps, scale, s));
     prof_end(pr, s, 0.0, (double)g.units * g.parts * 8.0 + g.units * 4.0);
     if (st) return st;
     *launches += 2;
+    return MA_OK;
+}
 
-    NsParams p;
-    std::memset(&p, 0, sizeof(p));
-    p.units = (int)g.units;
-    p.m = (int)g.m;
-    p.n = (int)g.n;
-    p.ldx = g.ldx;
-    p.ldg = g.ldg;
-    p.x_unit = g.m * g.ldx;
-    p.g_unit = g.m * g.ldg;
-    p.scale = scale;
-    p.transposed = g.transposed;
-    p.heads = g.heads;
-    p.Rh = g.Rh;
-    p.C = g.C;
-    p.decay = 1.f - hp.lr * hp.weight_decay;
-    p.lr_s = hp.lr * shape_scale(g.Rh, g.C, hp.scale_mode);
-    p.lr_wd = hp.lr * hp.weight_decay;
-    p.cautious = hp.cautious ? 1 : 0;
-    p.wait_limit_ns = host_wait_limit_ns();
-    p.status = device_status_ptr();
-    for (int b = 0; b < batch; ++b) p.W[b] = W[b];
+// All checks passed; launch the whole Muon chain for a set of jobs that are
+// pairwise ns_compatible (or a single job). Each Newton-Schulz step is one
+// launch over every job's tiles on the tensor-core path; per job in fp32 mode.
+// A tile's arithmetic does not depend on the launch it is in, so grouping
+// gives the same bits as running the jobs one by one.
+int run_muon_jobs(const MuonJob* jobs_in, int njobs_in, cudaStream_t s, int sms, int* launches) {
+    std::vector<const MuonJob*> jobs;
+    for (int j = 0; j < njobs_in; ++j)
+        if (jobs_in[j].g.total > 0) jobs.push_back(&jobs_in[j]);
+    const int nj = (int)jobs.size();
+    if (nj == 0) return MA_OK;
+    if (nj > ns_tc_max_jobs()) return MA_ERR_UNSUPPORTED;
+    int st;
+    for (const MuonJob* j : jobs)
+        if ((st = muon_prep(*j, s, launches))) return st;
 
-    auto launch = [&](int mode, const void* xb, const void* gb) -> int {
+    const ma_muon_hparams_t& hp0 = *jobs[0]->hp;
+    std::vector<NsParams> p(nj);
+    std::vector<void*> cur(nj), nxt(nj), Gb(nj), G2(nj);
+    for (int i = 0; i < nj; ++i) {
+        const MuonJob& J = *jobs[i];
+        const MuonGeom& g = J.g;
+        const ma_muon_hparams_t& hp = *J.hp;
+        NsParams& q = p[i];
+        std::memset(&q, 0, sizeof(q));
+        q.units = (int)g.units;
+        q.m = (int)g.m;
+        q.n = (int)g.n;
+        q.ldx = g.ldx;
+        q.ldg = g.ldg;
+        q.x_unit = g.m * g.ldx;
+        q.g_unit = g.m * g.ldg;
+        q.scale = reinterpret_cast<float*>(J.ws + g.off_scale);
+        q.transposed = g.transposed;
+        q.heads = g.heads;
+        q.Rh = g.Rh;
+        q.C = g.C;
+        q.decay = 1.f - hp.lr * hp.weight_decay;
+        q.lr_s = hp.lr * shape_scale(g.Rh, g.C, hp.scale_mode);
+        q.lr_wd = hp.lr * hp.weight_decay;
+        q.cautious = hp.cautious ? 1 : 0;
+        q.wait_limit_ns = host_wait_limit_ns();
+        q.status = device_status_ptr();
+        for (int b = 0; b < J.batch; ++b) q.W[b] = J.W[b];
+        cur[i] = J.ws + g.off_x0;
+        nxt[i] = J.ws + g.off_x1;
+        Gb[i] = J.ws + g.off_g;
+        G2[i] = J.ws + g.off_g2;
+    }
+
+    std::vector<NsJobIn> in(nj);
+    auto launch = [&](int mode, const std::vector<void*>& xb, const std::vector<void*>& gb) -> int {
         const int pr = prof_begin(ns_prof_class(mode), s);
-        cudaError_t e = hp.precision ? launch_ns_simt(mode, p, xb, gb, s) : launch_ns_tc(mode, p, xb, gb, sms, s);
-        prof_end(pr, s, ns_flops(mode, g.units, g.m, g.n), 0.0);
-        ++*launches;
+        double flops = 0.0;
+        cudaError_t e = cudaSuccess;
+        for (int i = 0; i < nj; ++i) {
+            in[i] = {&p[i], xb[i], gb[i]};
+            flops += ns_flops(mode, jobs[i]->g.units, jobs[i]->g.m, jobs[i]->g.n);
+        }
+        if (hp0.precision) {
+            for (int i = 0; i < nj && e == cudaSuccess; ++i) {
+                e = launch_ns_simt(mode, p[i], xb[i], gb[i], s);
+                ++*launches;
+            }
+        } else {
+            e = launch_ns_tc_group(mode, in.data(), nj, sms, s);
+            ++*launches;
+        }
+        prof_end(pr, s, flops, 0.0);
         return cuda_status(e);
     };
 
-    void* cur = X0;
-    void* nxt = X1;
-    for (int k = 0; k < hp.ns_steps; ++k) {
-        const float* cf = hp.coeffs[hp.n_coeffs == 1 ? 0 : k];
-        p.a = cf[0];
-        p.b = cf[1];
-        p.c = cf[2];
-        p.first = (k == 0) ? 1 : 0;
-        const bool quint = cf[2] != 0.f;
-        p.coef_gram = quint ? 1.f : cf[1];
-        p.out = Gb;
+    for (int k = 0; k < hp0.ns_steps; ++k) {
+        bool quint = false;
+        for (int i = 0; i < nj; ++i) {
+            const ma_muon_hparams_t& hp = *jobs[i]->hp;
+            const float* cf = hp.coeffs[hp.n_coeffs == 1 ? 0 : k];
+            NsParams& q = p[i];
+            q.a = cf[0];
+            q.b = cf[1];
+            q.c = cf[2];
+            q.first = (k == 0) ? 1 : 0;
+            quint = cf[2] != 0.f;  // the same for every job of the set
+            q.coef_gram = quint ? 1.f : cf[1];
+            q.out = Gb[i];
+        }
         if ((st = launch(NS_GRAM, cur, Gb))) return st;
-        void* Bbuf = Gb;
+        std::vector<void*>* Bbuf = &Gb;
         if (quint) {
-            p.xin = Gb;
-            p.out = G2;
+            for (int i = 0; i < nj; ++i) {
+                p[i].xin = Gb[i];
+                p[i].out = G2[i];
+            }
             if ((st = launch(NS_GRAMSQ, cur, Gb))) return st;
-            Bbuf = G2;
+            Bbuf = &G2;
         }
-        p.xin = cur;
-        if (k + 1 < hp.ns_steps) {
-            p.out = nxt;
-            if ((st = launch(NS_APPLY, cur, Bbuf))) return st;
-            std::swap(cur, nxt);
-        } else {
-            p.out = nullptr;
-            if ((st = launch(NS_FINAL, cur, Bbuf))) return st;
+        const bool last = k + 1 == hp0.ns_steps;
+        for (int i = 0; i < nj; ++i) {
+            p[i].xin = cur[i];
+            p[i].out = last ? nullptr : nxt[i];
         }
+        if ((st = launch(last ? NS_FINAL : NS_APPLY, cur, *Bbuf))) return st;
+        if (!last) std::swap(cur, nxt);
     }
     return MA_OK;
+}
+
+// One batch with workspace ws.
+int run_muon(int batch, const MuonGeom& g, float* const* W, const void* const* G, int gdt, float* const* M,
+             const ma_muon_hparams_t& hp, void* ws, cudaStream_t s, int sms, int* launches) {
+    const MuonJob j{batch, g, W, G, gdt, M, &hp, reinterpret_cast<uint8_t*>(ws)};
+    return run_muon_jobs(&j, 1, s, sms, launches);
 }
 
 int check_ptr_array(const void* const* a, int n, size_t align) {
@@ -469,11 +547,14 @@ struct ma_plan {
 namespace ma {
 namespace {
 
-// A unit of launch work inside one step: every AdamW tensor, or one sub-batch
-// of one Muon bucket.
-struct Segment {
-    int adamw;  // 1: the AdamW tensors; 0: a Muon sub-batch
+// A unit of launch work inside one step: every AdamW tensor, or one or more
+// Muon sub-batches (parts) whose Newton-Schulz steps share launches.
+struct Part {
     int bucket, start, count;
+};
+struct Segment {
+    int adamw;  // 1: the AdamW tensors; 0: Muon parts
+    std::vector<Part> parts;
 };
 
 int64_t tensor_numel(const ma_tensor_t& x) {
@@ -510,12 +591,25 @@ int check_step(ma_plan* plan, const ma_group_t* groups, void* ws, size_t ws_byte
     return MA_OK;
 }
 
+size_t part_ws(const ma_plan* plan, const ma_group_t* groups, const Part& pt) {
+    const auto& b = plan->buckets[pt.bucket];
+    MuonGeom g;
+    if (muon_geom(pt.count, b.R, b.C, groups[b.group].muon, &g)) return SIZE_MAX;
+    return g.total;
+}
+
 // Segments in launch order. first_cap / cap bound the Muon sub-batch sizes
-// (0 = the plan's own sub-batch size); AdamW goes first or last.
-std::vector<Segment> step_segments(const ma_plan* plan, int first_cap, int cap, bool adamw_last) {
+// (0 = the plan's own sub-batch size); AdamW goes first or last. With
+// group_limit > 0, consecutive sub-batches whose Newton-Schulz chains take
+// the same kernels are merged into one segment while their summed workspace
+// stays within group_limit and the launch tables have room (jobs, weights).
+std::vector<Segment> step_segments(const ma_plan* plan, const ma_group_t* groups, int first_cap, int cap,
+                                   bool adamw_last, size_t group_limit) {
     std::vector<Segment> segs;
-    if (!adamw_last && !plan->adamw_idx.empty()) segs.push_back({1, -1, 0, 0});
+    if (!adamw_last && !plan->adamw_idx.empty()) segs.push_back({1, {}});
     bool first = true;
+    size_t seg_ws = 0;
+    int seg_w = 0;
     for (int bi = 0; bi < (int)plan->buckets.size(); ++bi) {
         const auto& b = plan->buckets[bi];
         const int nb = (int)b.members.size();
@@ -524,12 +618,31 @@ std::vector<Segment> step_segments(const ma_plan* plan, int first_cap, int cap, 
             if (cap > 0) lim = std::min(lim, cap);
             if (first && first_cap > 0) lim = std::min(lim, first_cap);
             const int cnt = std::min(lim, nb - s0);
-            segs.push_back({0, bi, s0, cnt});
+            const Part pt{bi, s0, cnt};
+            const size_t ws = part_ws(plan, groups, pt);
+            const int nw = cnt;
+            bool merge = false;
+            if (group_limit > 0 && !segs.empty() && !segs.back().adamw) {
+                const Segment& last = segs.back();
+                const auto& lb = plan->buckets[last.parts.back().bucket];
+                merge = ns_compatible(groups[lb.group].muon, groups[b.group].muon) &&
+                        (int)last.parts.size() < ns_tc_max_jobs() && seg_w + nw <= ns_tc_max_weights() &&
+                        ws <= group_limit && seg_ws <= group_limit - ws;
+            }
+            if (merge) {
+                segs.back().parts.push_back(pt);
+                seg_ws += ws;
+                seg_w += nw;
+            } else {
+                segs.push_back({0, {pt}});
+                seg_ws = ws;
+                seg_w = nw;
+            }
             s0 += cnt;
             first = false;
         }
     }
-    if (adamw_last && !plan->adamw_idx.empty()) segs.push_back({1, -1, 0, 0});
+    if (adamw_last && !plan->adamw_idx.empty()) segs.push_back({1, {}});
     return segs;
 }
 
@@ -553,21 +666,39 @@ int launch_segment(ma_plan* plan, const ma_group_t* groups, const Segment& sg, v
         }
         return MA_OK;
     }
-    const auto& b = plan->buckets[sg.bucket];
-    const ma_muon_hparams_t& hp = groups[b.group].muon;
-    const int gdt = plan->t[b.members[0]].grad_dtype;
-    float* W[MA_MAX_BATCH];
-    const void* G[MA_MAX_BATCH];
-    float* M[MA_MAX_BATCH];
-    for (int k = 0; k < sg.count; ++k) {
-        const ma_tensor_t& x = plan->t[b.members[sg.start + k]];
-        W[k] = x.param;
-        G[k] = x.grad;
-        M[k] = x.state0;
+    const int np = (int)sg.parts.size();
+    std::vector<MuonJob> jobs(np);
+    std::vector<float*> W, M;
+    std::vector<const void*> G;
+    int total = 0;
+    for (const Part& pt : sg.parts) total += pt.count;
+    W.reserve(total);
+    M.reserve(total);
+    G.reserve(total);
+    uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+    for (int q = 0; q < np; ++q) {
+        const Part& pt = sg.parts[q];
+        const auto& b = plan->buckets[pt.bucket];
+        const ma_muon_hparams_t& hp = groups[b.group].muon;
+        MuonJob& J = jobs[q];
+        J.batch = pt.count;
+        muon_geom(pt.count, b.R, b.C, hp, &J.g);
+        J.gdt = plan->t[b.members[0]].grad_dtype;
+        J.hp = &hp;
+        J.ws = base;
+        base += J.g.total;  // a multiple of the workspace alignment
+        const size_t off = W.size();
+        for (int k = 0; k < pt.count; ++k) {
+            const ma_tensor_t& x = plan->t[b.members[pt.start + k]];
+            W.push_back(x.param);
+            G.push_back(x.grad);
+            M.push_back(x.state0);
+        }
+        J.W = W.data() + off;
+        J.G = G.data() + off;
+        J.M = M.data() + off;
     }
-    MuonGeom g;
-    muon_geom(sg.count, b.R, b.C, hp, &g);
-    return run_muon(sg.count, g, W, G, gdt, M, hp, ws, s, sms, launches);
+    return run_muon_jobs(jobs.data(), np, s, sms, launches);
 }
 
 }  // namespace
@@ -868,6 +999,15 @@ int ma_plan_create(const ma_tensor_t* t, int n, const ma_group_t* groups, int ng
         b.sub = sub;
         need = std::max(need, g.total);
     }
+    // Small buckets share Newton-Schulz launches (more tiles per launch, fewer
+    // launches) when the grouped workspace stays within the cap, or without a
+    // cap within the larger of the biggest single sub-batch and kGroupWsBytes.
+    const size_t limit = cap > 0 ? cap : std::max(need, kGroupWsBytes);
+    for (const Segment& sg : step_segments(plan, groups, 0, 0, false, limit)) {
+        size_t tot = 0;
+        for (const Part& pt : sg.parts) tot += part_ws(plan, groups, pt);
+        need = std::max(need, tot);
+    }
     plan->ws_bytes = need;
     *ws_bytes = need;
     *out = plan;
@@ -880,7 +1020,7 @@ int muonadamw_step(ma_plan_t* plan, const ma_group_t* groups, void* ws, size_t w
     if (st) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     int launches = 0;
-    for (const Segment& sg : step_segments(plan, 0, 0, false))
+    for (const Segment& sg : step_segments(plan, groups, 0, 0, false, plan->ws_bytes))
         if ((st = launch_segment(plan, groups, sg, ws, s, sms, &launches))) return st;
     plan->last_launches = launches;
     return MA_OK;
@@ -899,7 +1039,7 @@ int muonadamw_step_from_host(ma_plan_t* plan, const ma_group_t* groups, const vo
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(copy_stream);
     // Muon sub-batches first (the first one small, so the compute starts early),
     // the AdamW tensors last: every later copy overlaps earlier compute.
-    const std::vector<Segment> segs = step_segments(plan, kFromHostFirstBatch, kFromHostBatch, true);
+    const std::vector<Segment> segs = step_segments(plan, groups, kFromHostFirstBatch, kFromHostBatch, true, 0);
     while (plan->events.size() < segs.size() + 1) {
         cudaEvent_t e;
         if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return MA_ERR_CUDA;
@@ -924,9 +1064,9 @@ int muonadamw_step_from_host(ma_plan_t* plan, const ma_group_t* groups, const vo
             for (int i : plan->adamw_idx)
                 if ((st = copy_tensor(i))) return st;
         } else {
-            const auto& b = plan->buckets[sg.bucket];
-            for (int j = 0; j < sg.count; ++j)
-                if ((st = copy_tensor(b.members[sg.start + j]))) return st;
+            for (const Part& pt : sg.parts)
+                for (int j = 0; j < pt.count; ++j)
+                    if ((st = copy_tensor(plan->buckets[pt.bucket].members[pt.start + j]))) return st;
         }
         if (cudaEventRecord(plan->events[k], cs) != cudaSuccess) return MA_ERR_CUDA;
     }

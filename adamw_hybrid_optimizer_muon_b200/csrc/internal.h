@@ -102,6 +102,16 @@ struct NsParams {
 size_t ns_tc_smem_bytes();
 cudaError_t launch_ns_tc(int mode, const NsParams& p, const void* x_buf, const void* g_buf, int num_sms,
                          cudaStream_t s);
+// Several jobs (same mode) in one persistent launch: at most ns_tc_max_jobs()
+// jobs and, for the final apply, ns_tc_max_weights() weight matrices in total.
+struct NsJobIn {
+    const NsParams* p;
+    const void* x_buf;
+    const void* g_buf;
+};
+cudaError_t launch_ns_tc_group(int mode, const NsJobIn* jobs, int njobs, int num_sms, cudaStream_t s);
+int ns_tc_max_jobs();
+int ns_tc_max_weights();
 
 // fp32 SIMT path (precision mode 1).
 cudaError_t launch_ns_simt(int mode, const NsParams& p, const void* x_buf, const void* g_buf, cudaStream_t s);

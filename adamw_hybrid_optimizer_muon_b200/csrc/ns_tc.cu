@@ -36,6 +36,7 @@
 // B operand major-ness: for GRAM and GRAMSQ both operands are K-major rows of
 // the same matrix. For APPLY the B operand is X itself, read MN-major (the
 // contraction runs over X's rows), so no transposed copy is ever made.
+#include <climits>
 #include <cstring>
 
 #include "common.cuh"
@@ -84,6 +85,39 @@ struct TileCoord {
     int u, ti, tj;
 };
 
+// One job of a launch: a batch of same-shape units sharing this iteration's
+// polynomial. A launch covers up to kMaxJobs jobs (same mode), so that small
+// buckets fill the machine together.
+constexpr int kMaxJobs = 8;
+constexpr int kMaxW = 512;  // weight pointers over all jobs of a final-apply launch
+
+struct NsJob {
+    int32_t units, m, n, first;
+    int64_t ldx, ldg, x_unit, g_unit;
+    float a, b, c, coef_gram;
+    const float* scale;
+    const void* xin;
+    void* out;
+    int32_t transposed, heads, cautious, w0;
+    int64_t Rh, C;
+    float decay, lr_s, lr_wd;
+    int32_t tiles_per_unit, mt, nt, kblocks, tile0;
+};
+
+struct NsLaunch {
+    CUtensorMap mA[kMaxJobs], mB[kMaxJobs], mO[kMaxJobs];
+    NsJob job[kMaxJobs];
+    int32_t njobs, total_tiles;
+    long long wait_limit_ns;
+    int* status;
+    float* W[kMaxW];
+};
+
+struct JobTile {
+    int j;
+    TileCoord tc;
+};
+
 // Tiles of one unit. GRAM/GRAMSQ: only the tiles (ti, tj) with ti <= tj, the
 // ones that hold an element with row <= col, enumerated column by column.
 __device__ __forceinline__ TileCoord decode_tile(int mode, int t, int tiles_per_unit, int mt, int nt) {
@@ -105,15 +139,39 @@ __device__ __forceinline__ TileCoord decode_tile(int mode, int t, int tiles_per_
     return c;
 }
 
-__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&x)[32]) {
-    const uint4* s = reinterpret_cast<const uint4*>(src);
+// Global tile index of a launch -> (job, unit, tile row, tile column).
+__device__ __forceinline__ JobTile decode_job_tile(const NsLaunch& L, int mode, int t) {
+    JobTile r;
+    int j = 0;
+    while (j + 1 < L.njobs && t >= L.job[j + 1].tile0) ++j;
+    const NsJob& J = L.job[j];
+    r.j = j;
+    r.tc = decode_tile(mode, t - J.tile0, J.tiles_per_unit, J.mt, J.nt);
+    return r;
+}
+
+// o[t] = ca * in[t] + cv * v[t] for the 32 bf16 values in[0..31] of one row
+// (zero where the row is out of range or t >= cols_left). o may alias v.
+__device__ __forceinline__ void combine_row(const __nv_bfloat16* in, bool row_ok, int cols_left, float ca, float cv,
+                                            const float (&v)[32], float (&o)[32]) {
+    if (row_ok && cols_left >= 32) {
+        const uint4* s = reinterpret_cast<const uint4*>(in);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-        const uint4 w = s[q];
-        x[8 * q + 0] = bf16_lo(w.x); x[8 * q + 1] = bf16_hi(w.x);
-        x[8 * q + 2] = bf16_lo(w.y); x[8 * q + 3] = bf16_hi(w.y);
-        x[8 * q + 4] = bf16_lo(w.z); x[8 * q + 5] = bf16_hi(w.z);
-        x[8 * q + 6] = bf16_lo(w.w); x[8 * q + 7] = bf16_hi(w.w);
+        for (int q = 0; q < 4; ++q) {
+            const uint4 w = s[q];
+            const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                o[8 * q + 2 * e] = ca * bf16_lo(wv[e]) + cv * v[8 * q + 2 * e];
+                o[8 * q + 2 * e + 1] = ca * bf16_hi(wv[e]) + cv * v[8 * q + 2 * e + 1];
+            }
+        }
+    } else {
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+            const float x = (row_ok && t < cols_left) ? __bfloat162float(in[t]) : 0.f;
+            o[t] = ca * x + cv * v[t];
+        }
     }
 }
 
@@ -121,8 +179,8 @@ __device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&x
 // col0..col0+31), before rounding: GRAM b*A (x s^2 on the first iteration),
 // GRAMSQ b*A + c*A^2, APPLY/FINAL s*(a*X + B*X).
 template <int MODE>
-__device__ __forceinline__ void epilogue_values(const NsParams& p, const TileCoord& tc, int row, int col0,
-                                                const float (&v)[32], float (&o)[32]) {
+__device__ __forceinline__ void epilogue_values(const NsJob& p, const TileCoord& tc, int row, int col0,
+                                                const float (&v)[32], float (&o)[32]) {  // o may alias v
     if (MODE == NS_GRAM) {
         float coef = p.coef_gram;
         if (p.first) {
@@ -132,39 +190,22 @@ __device__ __forceinline__ void epilogue_values(const NsParams& p, const TileCoo
 #pragma unroll
         for (int t = 0; t < 32; ++t) o[t] = coef * v[t];
     } else if (MODE == NS_GRAMSQ) {
-        // acc = A^2; A is read back from the Gram buffer
+        // acc = A^2; A is read back from the Gram buffer, 8 values at a time
         const int m = p.m;
+        const float b = p.b, c = p.c;
         const __nv_bfloat16* Gin = reinterpret_cast<const __nv_bfloat16*>(p.xin) + (int64_t)tc.u * p.g_unit;
-        float a_in[32];
-        if (row < m && col0 + 32 <= m) {
-            load_bf16x32(Gin + (int64_t)row * p.ldg + col0, a_in);
-        } else {
-#pragma unroll
-            for (int t = 0; t < 32; ++t)
-                a_in[t] = (row < m && col0 + t < m) ? __bfloat162float(Gin[(int64_t)row * p.ldg + col0 + t]) : 0.f;
-        }
-#pragma unroll
-        for (int t = 0; t < 32; ++t) o[t] = p.b * a_in[t] + p.c * v[t];
+        combine_row(Gin + (int64_t)row * p.ldg + col0, row < m, m - col0, b, c, v, o);
     } else {
         const int m = p.m, n = p.n;
         const float sa = p.first ? p.scale[tc.u] : 1.f;
-        float x[32];
         const __nv_bfloat16* Xin = reinterpret_cast<const __nv_bfloat16*>(p.xin) + (int64_t)tc.u * p.x_unit;
-        if (row < m && col0 + 32 <= n) {
-            load_bf16x32(Xin + (int64_t)row * p.ldx + col0, x);
-        } else {
-#pragma unroll
-            for (int t = 0; t < 32; ++t)
-                x[t] = (row < m && col0 + t < n) ? __bfloat162float(Xin[(int64_t)row * p.ldx + col0 + t]) : 0.f;
-        }
-#pragma unroll
-        for (int t = 0; t < 32; ++t) o[t] = sa * (p.a * x[t] + v[t]);
+        combine_row(Xin + (int64_t)row * p.ldx + col0, row < m, n - col0, sa * p.a, sa, v, o);
     }
 }
 
 // One weight: decoupled decay (optionally only where the update x and w agree in
 // sign, the cautious reading), then the scaled orthogonalised update.
-__device__ __forceinline__ float apply_update(float w, float x, float decay, float lrs, const NsParams& p) {
+__device__ __forceinline__ float apply_update(float w, float x, float decay, float lrs, const NsJob& p) {
     if (p.cautious) return (x * w > 0.f ? w - p.lr_wd * w : w) - lrs * x;
     return w * decay - lrs * x;
 }
@@ -182,24 +223,25 @@ __device__ __forceinline__ float apply_update(float w, float x, float decay, flo
 // updates its own row (or, transposed, its own column) of the block in place
 // from X_N in its registers, and the block goes back to W with coalesced
 // 16-byte stores.
-__device__ __forceinline__ void final_epilogue(const NsParams& p, int tiles_per_unit, int mt, int nt, int pair,
-                                               int npairs, int total_tiles, uint32_t rank, uint32_t tmem_base,
-                                               int warp, int lane, uint8_t* wbuf, uint64_t* wbar,
-                                               uint64_t* acc_full, uint64_t* acc_empty, volatile int* abort_flag,
-                                               long long limit) {
+__device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int npairs, uint32_t rank,
+                                               uint32_t tmem_base, int warp, int lane, uint8_t* wbuf,
+                                               uint64_t* acc_full, uint64_t* acc_empty, volatile int* abort_flag) {
     const int quad = warp & 3, half = (warp - 2) / 4;
-    const int m = p.m, n = p.n;
+    const long long limit = L.wait_limit_ns;
     const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
     const uint32_t acc_empty_leader1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
-    const float decay = p.decay, lrs = p.lr_s;
     int lt = 0;
-    for (int t = pair; t < total_tiles; t += npairs, ++lt) {
-        const TileCoord tc = decode_tile(NS_FINAL, t, tiles_per_unit, mt, nt);
+    for (int t = pair; t < L.total_tiles; t += npairs, ++lt) {
+        const JobTile jt = decode_job_tile(L, NS_FINAL, t);
+        const NsJob& p = L.job[jt.j];
+        const TileCoord tc = jt.tc;
+        const int m = p.m, n = p.n;
+        const float decay = p.decay, lrs = p.lr_s;
         const int acc = lt & 1;
         const uint32_t use = (uint32_t)(lt >> 1);
         const int row_lo = tc.ti * BM + (int)rank * HM + quad * 32;
         const int bidx = tc.u / p.heads, h = tc.u - bidx * p.heads;
-        float* Wb = p.W[bidx] + (int64_t)h * p.Rh * p.C;
+        float* Wb = L.W[p.w0 + bidx] + (int64_t)h * p.Rh * p.C;
         // geometry of chunk c's W block: its first W row, first W column, and extents
         auto block = [&](int c, int& r0, int& c0, int& nr, int& rb) -> bool {
             const int col0 = tc.tj * BN + (half * 4 + c) * 32;
@@ -224,7 +266,7 @@ __device__ __forceinline__ void final_epilogue(const NsParams& p, int tiles_per_
         fetch(0);
         fetch(1);
         int ok = 1;
-        if (lane == 0) ok = mbar_wait_bounded(&acc_full[acc], use & 1u, abort_flag, limit, p.status, kEpiSleepNs) ? 1 : 0;
+        if (lane == 0) ok = mbar_wait_bounded(&acc_full[acc], use & 1u, abort_flag, limit, L.status, kEpiSleepNs) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         tc_fence_after();
@@ -286,9 +328,7 @@ __device__ __forceinline__ uint32_t sw64(uint32_t r, uint32_t q) { return r * 64
 
 template <int MODE>
 __global__ void __launch_bounds__(THREADS, 1)
-    ns_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__ CUtensorMap mapB,
-                 const __grid_constant__ CUtensorMap mapOut, const __grid_constant__ NsParams p, int tiles_per_unit,
-                 int mt, int nt, int kblocks) {
+    ns_tc_kernel(const __grid_constant__ NsLaunch L) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int NST = kStages(MODE);
@@ -306,8 +346,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     const uint32_t rank = cluster_ctarank();  // 0 = leader of the pair
     const bool leader = rank == 0;
     const int pair = (int)cluster_id_x(), npairs = (int)cluster_count_x();
-    const int total_tiles = p.units * tiles_per_unit;
-    const long long limit = p.wait_limit_ns;
+    const int total_tiles = L.total_tiles;
+    const long long limit = L.wait_limit_ns;
     constexpr bool kApply = (MODE == NS_APPLY || MODE == NS_FINAL);
 
     if (threadIdx.x == 0) {
@@ -323,9 +363,11 @@ __global__ void __launch_bounds__(THREADS, 1)
         mbar_init(drain, 1);
         *abort_flag = 0;
         fence_barrier_init();
-        prefetch_tensormap(&mapA);
-        prefetch_tensormap(&mapB);
-        if (MODE != NS_FINAL) prefetch_tensormap(&mapOut);
+        for (int j = 0; j < L.njobs; ++j) {
+            prefetch_tensormap(&L.mA[j]);
+            prefetch_tensormap(&L.mB[j]);
+            if (MODE != NS_FINAL) prefetch_tensormap(&L.mO[j]);
+        }
     }
     if (warp == 1) {
         tmem_alloc_pair(tmem_holder, TMEM_COLS);
@@ -342,11 +384,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint32_t phase = 0;
             bool ok = true;
             for (int t = pair; t < total_tiles && ok; t += npairs) {
-                const TileCoord tc = decode_tile(MODE, t, tiles_per_unit, mt, nt);
+                const JobTile jt = decode_job_tile(L, MODE, t);
+                const TileCoord tc = jt.tc;
+                const CUtensorMap* mapA = &L.mA[jt.j];
+                const CUtensorMap* mapB = &L.mB[jt.j];
+                const int kblocks = L.job[jt.j].kblocks;
                 const int arow = tc.ti * BM + (int)rank * HM;
                 const int bcol = tc.tj * BN + (int)rank * HN;
                 for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit, p.status)) {
+                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit, L.status)) {
                         ok = false;
                         break;
                     }
@@ -354,13 +400,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                     uint8_t* sb = sa + A_BYTES;
                     if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
                     const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
-                    tma_load_3d_pair(sa, &mapA, fb, kb * BK, arow, tc.u);
+                    tma_load_3d_pair(sa, mapA, fb, kb * BK, arow, tc.u);
                     if (!kApply) {
-                        tma_load_3d_pair(sb, &mapB, fb, kb * BK, bcol, tc.u);
+                        tma_load_3d_pair(sb, mapB, fb, kb * BK, bcol, tc.u);
                     } else {
 #pragma unroll
                         for (int q = 0; q < HN / 64; ++q)
-                            tma_load_3d_pair(sb + q * (64 * BK * 2), &mapB, fb, bcol + q * 64, kb * BK, tc.u);
+                            tma_load_3d_pair(sb + q * (64 * BK * 2), mapB, fb, bcol + q * 64, kb * BK, tc.u);
                     }
                     if (++stage == NST) {
                         stage = 0;
@@ -371,7 +417,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             // Tail: wait until the MMAs have released every stage this CTA filled,
             // so that no commit arrives on this CTA's barriers after it exits.
             for (int i = 0; i < NST && ok; ++i) {
-                ok = mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit, p.status);
+                ok = mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit, L.status);
                 if (++stage == NST) {
                     stage = 0;
                     phase ^= 1u;
@@ -388,14 +434,15 @@ __global__ void __launch_bounds__(THREADS, 1)
             for (int t = pair; t < total_tiles && ok; t += npairs, ++lt) {
                 const int acc = lt & 1;
                 const uint32_t use = (uint32_t)(lt >> 1);
-                if (!mbar_wait_bounded(&acc_empty[acc], (use & 1u) ^ 1u, abort_flag, limit, p.status)) {
+                if (!mbar_wait_bounded(&acc_empty[acc], (use & 1u) ^ 1u, abort_flag, limit, L.status)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                const int kblocks = L.job[decode_job_tile(L, MODE, t).j].kblocks;
                 for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, limit, p.status)) {
+                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, limit, L.status)) {
                         ok = false;
                         break;
                     }
@@ -424,12 +471,12 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (!ok) {
                 // let every MMA issued so far finish before TMEM is released
                 tc_commit_pair(drain);
-                mbar_wait_bounded(drain, 0, abort_flag, limit, p.status);
+                mbar_wait_bounded(drain, 0, abort_flag, limit, L.status);
             }
         }
     } else if (MODE == NS_FINAL) {
-        final_epilogue(p, tiles_per_unit, mt, nt, pair, npairs, total_tiles, rank, tmem_base, warp, lane,
-                       staging + (warp - 2) * 2 * WBUF, &wbar[2 * (warp - 2)], acc_full, acc_empty, abort_flag, limit);
+        final_epilogue(L, pair, npairs, rank, tmem_base, warp, lane, staging + (warp - 2) * 2 * WBUF, acc_full,
+                       acc_empty, abort_flag);
     } else {
         const int quad = warp & 3;              // TMEM lanes [32*quad, 32*quad + 32)
         const int half = (warp - 2) / 4;        // which half of the 256 columns
@@ -438,14 +485,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t acc_empty_leader1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
         int lt = 0;
         for (int t = pair; t < total_tiles; t += npairs, ++lt) {
-            const TileCoord tc = decode_tile(MODE, t, tiles_per_unit, mt, nt);
+            const JobTile jt = decode_job_tile(L, MODE, t);
+            const NsJob& p = L.job[jt.j];
+            const CUtensorMap* mapOut = &L.mO[jt.j];
+            const TileCoord tc = jt.tc;
             const int acc = lt & 1;
             const uint32_t use = (uint32_t)(lt >> 1);
             const int row_lo = tc.ti * BM + (int)rank * HM + quad * 32;
             const int row = row_lo + lane;
             int ok = 1;
             if (lane == 0)
-                ok = mbar_wait_bounded(&acc_full[acc], use & 1u, abort_flag, limit, p.status, kEpiSleepNs) ? 1 : 0;
+                ok = mbar_wait_bounded(&acc_full[acc], use & 1u, abort_flag, limit, L.status, kEpiSleepNs) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after();
@@ -456,9 +506,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int col0 = tc.tj * BN + cc * 32;
                 if (col0 >= limit_cols || row_lo >= p.m) break;                  // warp-uniform
                 if (!kApply && col0 < row_lo) continue;                          // below the diagonal
-                float v[32], o[32];
-                tmem_ld32(tmem_base + (uint32_t)(acc * BN + cc * 32) + ((uint32_t)(quad * 32) << 16), v);
-                epilogue_values<MODE>(p, tc, row, col0, v, o);
+                float o[32];
+                tmem_ld32(tmem_base + (uint32_t)(acc * BN + cc * 32) + ((uint32_t)(quad * 32) << 16), o);
+                epilogue_values<MODE>(p, tc, row, col0, o, o);  // in place
                 // Stage this warp's 32 x 32 block (and, for an off-diagonal Gram
                 // chunk, its transpose), then write both with bulk tensor stores:
                 // each leaves shared memory as contiguous 64-byte rows.
@@ -483,8 +533,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_3d(&mapOut, stg, col0, row_lo, tc.u);
-                    if (mirror) tma_store_3d(&mapOut, stg + STG_BLOCK, row_lo, col0, tc.u);
+                    tma_store_3d(mapOut, stg, col0, row_lo, tc.u);
+                    if (mirror) tma_store_3d(mapOut, stg + STG_BLOCK, row_lo, col0, tc.u);
                     bulk_commit_group();
                 }
             }
@@ -543,36 +593,66 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
 }
 
 template <int MODE>
-cudaError_t launch_mode(const NsParams& p, const void* x_buf, const void* g_buf, int num_sms, cudaStream_t s) {
-    CUtensorMap mA, mB, mO;
-    std::memset(&mO, 0, sizeof(mO));
-    int kblocks, mt, nt, tiles;
-    mt = (p.m + BM - 1) / BM;
-    if (MODE == NS_GRAM || MODE == NS_GRAMSQ) {
-        nt = mt;
-        tiles = nt * (nt + 1) / 2;
-        if (MODE == NS_GRAM) {
-            kblocks = (p.n + BK - 1) / BK;
-            if (!make_map(&mA, x_buf, p.n, p.m, p.units, p.ldx, p.x_unit, BK, HM)) return cudaErrorInvalidValue;
+cudaError_t launch_mode(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_t s) {
+    if (njobs < 1 || njobs > kMaxJobs) return cudaErrorInvalidValue;
+    static thread_local NsLaunch L;  // ~9 KB parameter block, copied at launch
+    std::memset(&L, 0, sizeof(L));
+    int tile0 = 0, w0 = 0;
+    for (int j = 0; j < njobs; ++j) {
+        const NsParams& p = *jobs[j].p;
+        const void* x_buf = jobs[j].x_buf;
+        const void* g_buf = jobs[j].g_buf;
+        NsJob& J = L.job[j];
+        int kblocks, mt, nt, tiles;
+        mt = (p.m + BM - 1) / BM;
+        if (MODE == NS_GRAM || MODE == NS_GRAMSQ) {
+            nt = mt;
+            tiles = nt * (nt + 1) / 2;
+            if (MODE == NS_GRAM) {
+                kblocks = (p.n + BK - 1) / BK;
+                if (!make_map(&L.mA[j], x_buf, p.n, p.m, p.units, p.ldx, p.x_unit, BK, HM)) return cudaErrorInvalidValue;
+            } else {
+                kblocks = (p.m + BK - 1) / BK;
+                if (!make_map(&L.mA[j], p.xin, p.m, p.m, p.units, p.ldg, p.g_unit, BK, HM))
+                    return cudaErrorInvalidValue;
+            }
+            L.mB[j] = L.mA[j];  // both operands are 128-row, 64-deep K-major boxes of the same matrix
+            if (!make_map(&L.mO[j], p.out, p.m, p.m, p.units, p.ldg, p.g_unit, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+                return cudaErrorInvalidValue;
         } else {
+            nt = (p.n + BN - 1) / BN;
+            tiles = mt * nt;
             kblocks = (p.m + BK - 1) / BK;
-            if (!make_map(&mA, p.xin, p.m, p.m, p.units, p.ldg, p.g_unit, BK, HM)) return cudaErrorInvalidValue;
+            if (!make_map(&L.mA[j], g_buf, p.m, p.m, p.units, p.ldg, p.g_unit, BK, HM)) return cudaErrorInvalidValue;
+            if (!make_map(&L.mB[j], x_buf, p.n, p.m, p.units, p.ldx, p.x_unit, 64, BK)) return cudaErrorInvalidValue;
+            if (MODE == NS_APPLY &&
+                !make_map(&L.mO[j], p.out, p.n, p.m, p.units, p.ldx, p.x_unit, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
+                return cudaErrorInvalidValue;
         }
-        mB = mA;  // both operands are 128-row, 64-deep K-major boxes of the same matrix
-        if (!make_map(&mO, p.out, p.m, p.m, p.units, p.ldg, p.g_unit, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
-            return cudaErrorInvalidValue;
-    } else {
-        nt = (p.n + BN - 1) / BN;
-        tiles = mt * nt;
-        kblocks = (p.m + BK - 1) / BK;
-        if (!make_map(&mA, g_buf, p.m, p.m, p.units, p.ldg, p.g_unit, BK, HM)) return cudaErrorInvalidValue;
-        if (!make_map(&mB, x_buf, p.n, p.m, p.units, p.ldx, p.x_unit, 64, BK)) return cudaErrorInvalidValue;
-        if (MODE == NS_APPLY &&
-            !make_map(&mO, p.out, p.n, p.m, p.units, p.ldx, p.x_unit, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
-            return cudaErrorInvalidValue;
+        J.units = p.units; J.m = p.m; J.n = p.n; J.first = p.first;
+        J.ldx = p.ldx; J.ldg = p.ldg; J.x_unit = p.x_unit; J.g_unit = p.g_unit;
+        J.a = p.a; J.b = p.b; J.c = p.c; J.coef_gram = p.coef_gram;
+        J.scale = p.scale; J.xin = p.xin; J.out = p.out;
+        J.transposed = p.transposed; J.heads = p.heads; J.cautious = p.cautious;
+        J.Rh = p.Rh; J.C = p.C; J.decay = p.decay; J.lr_s = p.lr_s; J.lr_wd = p.lr_wd;
+        J.tiles_per_unit = tiles; J.mt = mt; J.nt = nt; J.kblocks = kblocks;
+        J.tile0 = tile0;
+        J.w0 = w0;
+        if (MODE == NS_FINAL) {
+            const int batch = p.heads > 0 ? p.units / p.heads : 0;
+            if (w0 + batch > kMaxW) return cudaErrorInvalidValue;
+            for (int b = 0; b < batch; ++b) L.W[w0 + b] = p.W[b];
+            w0 += batch;
+        }
+        const long long t = (long long)tile0 + (long long)tiles * p.units;
+        if (t > INT_MAX) return cudaErrorInvalidValue;
+        tile0 = (int)t;
     }
-    const long long total = (long long)tiles * p.units;
-    if (total <= 0) return cudaSuccess;
+    L.njobs = njobs;
+    L.total_tiles = tile0;
+    L.wait_limit_ns = jobs[0].p->wait_limit_ns;
+    L.status = jobs[0].p->status;
+    if (tile0 <= 0) return cudaSuccess;
     static unsigned long long attr_set = 0;  // one bit per device
     static int max_pairs[64] = {0};
     int dev = 0;
@@ -602,7 +682,7 @@ cudaError_t launch_mode(const NsParams& p, const void* x_buf, const void* g_buf,
         max_pairs[dev] = nclusters;
         attr_set |= 1ull << dev;
     }
-    const long long pairs = total < max_pairs[dev] ? total : max_pairs[dev];
+    const long long pairs = tile0 < max_pairs[dev] ? tile0 : max_pairs[dev];
     cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -615,22 +695,29 @@ cudaError_t launch_mode(const NsParams& p, const void* x_buf, const void* g_buf,
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, ns_tc_kernel<MODE>, mA, mB, mO, p, tiles, mt, nt, kblocks);
+    return cudaLaunchKernelEx(&cfg, ns_tc_kernel<MODE>, L);
 }
 
 }  // namespace
 
 size_t ns_tc_smem_bytes() { return SMEM_BYTES; }
+int ns_tc_max_jobs() { return kMaxJobs; }
+int ns_tc_max_weights() { return kMaxW; }
+
+cudaError_t launch_ns_tc_group(int mode, const NsJobIn* jobs, int njobs, int num_sms, cudaStream_t s) {
+    switch (mode) {
+        case NS_GRAM: return launch_mode<NS_GRAM>(jobs, njobs, num_sms, s);
+        case NS_GRAMSQ: return launch_mode<NS_GRAMSQ>(jobs, njobs, num_sms, s);
+        case NS_APPLY: return launch_mode<NS_APPLY>(jobs, njobs, num_sms, s);
+        case NS_FINAL: return launch_mode<NS_FINAL>(jobs, njobs, num_sms, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
 
 cudaError_t launch_ns_tc(int mode, const NsParams& p, const void* x_buf, const void* g_buf, int num_sms,
                          cudaStream_t s) {
-    switch (mode) {
-        case NS_GRAM: return launch_mode<NS_GRAM>(p, x_buf, g_buf, num_sms, s);
-        case NS_GRAMSQ: return launch_mode<NS_GRAMSQ>(p, x_buf, g_buf, num_sms, s);
-        case NS_APPLY: return launch_mode<NS_APPLY>(p, x_buf, g_buf, num_sms, s);
-        case NS_FINAL: return launch_mode<NS_FINAL>(p, x_buf, g_buf, num_sms, s);
-        default: return cudaErrorInvalidValue;
-    }
+    NsJobIn j{&p, x_buf, g_buf};
+    return launch_ns_tc_group(mode, &j, 1, num_sms, s);
 }
 
 }  // namespace ma

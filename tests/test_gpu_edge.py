@@ -182,3 +182,50 @@ def test_fp32_mode_larger(shape):
     torch.cuda.synchronize()
     rw, _ = oracle.muon_update(W0, g, np.zeros(shape), f32(0.02), f32(0.95), f32(0.01), eps=f32(1e-7))
     check_muon(W0, host(Wd[0]), rw, f32(0.02), f32(0.01), TOL_F32)
+
+
+def test_grouped_newton_schulz_launches_match_per_bucket_calls():
+    """A plan runs small Muon buckets through shared Newton-Schulz launches;
+    every tile is computed as in a launch of its own bucket alone, so the
+    result must equal one muon_step_batched call per bucket, bit for bit.
+    Nine buckets (tall, wide, square, per-head; two cubic schedules) exceed
+    the eight jobs one launch takes; two more with an A^2 term (c != 0) take
+    a different kernel sequence and form a group of their own."""
+    H = ma.ROLE_HIDDEN
+    shapes = [(64, 128), (128, 64), (256, 512), (512, 256), (128, 128), (192, 64), (64, 320), (384, 128),
+              (96, 96), (320, 64), (256, 256)]
+    counts = [3, 2, 1, 2, 4, 1, 2, 1, 3, 2, 1]
+    cubic2 = ((2.0, -1.25, 0.0), (1.7, -0.6, 0.0), (1.5, -0.5, 0.0), (1.5, -0.5, 0.0), (1.6, -0.55, 0.0))
+    hps = [ma.muon_hparams(),
+           ma.muon_hparams(coeffs=cubic2, lr=0.01, weight_decay=0.1, heads=2),
+           ma.muon_hparams(coeffs=((3.4445, -4.7750, 2.0315),), scale_mode=1)]
+    which = [0, 1, 0, 1, 0, 1, 0, 1, 0, 2, 2]
+    r = np.random.default_rng(41)
+    table, P0, G = [], [], []
+    for bi, (shape, cnt) in enumerate(zip(shapes, counts)):
+        for _ in range(cnt):
+            table.append((shape, which[bi]))
+            P0.append((r.standard_normal(shape) * 0.02).astype(np.float32))
+            G.append(bf16_round(r.standard_normal(shape) * 1e-3))
+    params = [dev_f32(p) for p in P0]
+    opt = ma.MuonAdamW([(p, H, g) for p, (_, g) in zip(params, table)], [("muon", h) for h in hps])
+    opt.step([dev_grad(g, "bf16") for g in G])
+    torch.cuda.synchronize()
+    assert ma.ma_device_status() == ma.MA_OK
+    grouped = opt.launches
+    i = 0
+    for bi, (shape, cnt) in enumerate(zip(shapes, counts)):
+        hp = hps[which[bi]]
+        Wd = [dev_f32(P0[i + k]) for k in range(cnt)]
+        Md = [torch.zeros(shape, device="cuda") for _ in range(cnt)]
+        ws = torch.empty(ma.muon_workspace_bytes(cnt, *shape, hp), dtype=torch.uint8, device="cuda")
+        ma.muon_step_batched(Wd, [dev_grad(G[i + k], "bf16") for k in range(cnt)], Md, hp, ws)
+        torch.cuda.synchronize()
+        for k in range(cnt):
+            assert torch.equal(Wd[k], params[i + k]), f"bucket {bi} matrix {k}"
+            assert torch.equal(Md[k], opt.state[i + k][0]), f"bucket {bi} momentum {k}"
+        i += cnt
+    # two launches of momentum and norm per bucket; Newton-Schulz: 8 cubic
+    # buckets in one set, the ninth alone (2 launches a step each), the two
+    # quintic buckets together (3 a step)
+    assert grouped == 2 * len(shapes) + 2 * 5 + 2 * 5 + 3 * 5
