@@ -344,8 +344,7 @@ int run_muon_jobs(const MuonJob* jobs_in, int njobs_in, cudaStream_t s, int sms,
                 ++*launches;
             }
         } else {
-            e = launch_ns_tc_group(mode, in.data(), nj, sms, s);
-            ++*launches;
+            e = launch_ns_tc_group(mode, in.data(), nj, sms, s, launches);
         }
         prof_end(pr, s, flops, 0.0);
         return cuda_status(e);

@@ -109,7 +109,10 @@ struct NsJobIn {
     const void* x_buf;
     const void* g_buf;
 };
-cudaError_t launch_ns_tc_group(int mode, const NsJobIn* jobs, int njobs, int num_sms, cudaStream_t s);
+// *launched (may be null) is increased by the number of kernels launched: one
+// for jobs with m > 128, one for jobs with m <= 128 (single-CTA tiles).
+cudaError_t launch_ns_tc_group(int mode, const NsJobIn* jobs, int njobs, int num_sms, cudaStream_t s,
+                               int* launched);
 int ns_tc_max_jobs();
 int ns_tc_max_weights();
 

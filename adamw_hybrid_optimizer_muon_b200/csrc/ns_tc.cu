@@ -54,7 +54,6 @@ constexpr int HM = BM / 2, HN = BN / 2;                // rows of A / columns of
 constexpr uint32_t A_BYTES = HM * BK * 2;              // 16 KB
 constexpr uint32_t B_BYTES = HN * BK * 2;              // 16 KB
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;    // 32 KB per CTA
-constexpr uint32_t TMEM_COLS = 2 * BN;                 // two fp32 accumulators
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 32 * (2 + EPI_WARPS);
 // Epilogue staging: per epilogue warp one 32 x 32 bf16 block for the tile and
@@ -80,6 +79,27 @@ constexpr size_t kSmemBytes(int mode) {
     return (size_t)kStages(mode) * STAGE_BYTES + kEpiBytes(mode) + 1024 /*align*/ + 512 /*barriers*/;
 }
 constexpr size_t SMEM_BYTES = kSmemBytes(NS_GRAM);
+
+// Tile shape of one kernel instance. PAIR: a CTA pair computes a 256 x 256
+// tile (cta_group::2, each CTA holding 128 rows of A and 128 columns of B).
+// Single CTA (for units with m <= 128, where a 256-row tile would be half
+// empty): a 128-row tile, 256 columns for the applies and 128 for the Gram,
+// cta_group::1.
+template <int MODE, bool PAIR>
+struct Shape {
+    static constexpr bool kApply = MODE == NS_APPLY || MODE == NS_FINAL;
+    static constexpr int TM = PAIR ? BM : HM;                       // output tile rows
+    static constexpr int TN = PAIR ? BN : (kApply ? BN : HN);       // output tile columns
+    static constexpr int CN = PAIR ? TN / 2 : TN;                   // B columns staged by each CTA
+    static constexpr uint32_t STAGE = A_BYTES + (uint32_t)CN * BK * 2;
+    static constexpr uint32_t EPI = kEpiBytes(MODE);
+    static constexpr int FIT = (int)((232448u - EPI - 1536u) / STAGE);  // 227 KB of shared memory per CTA
+    static constexpr int NST = PAIR ? kStages(MODE) : (FIT < STAGES ? FIT : STAGES);
+    static constexpr uint32_t TMEM = 2 * TN;                        // two fp32 accumulators
+    static constexpr int CPW = TN / 64;                             // 32-column chunks per epilogue warp
+    static constexpr size_t SMEM = (size_t)NST * STAGE + EPI + 1024 + 512;
+    static_assert(SMEM <= 232448, "shared memory");
+};
 
 struct TileCoord {
     int u, ti, tj;
@@ -223,13 +243,16 @@ __device__ __forceinline__ float apply_update(float w, float x, float decay, flo
 // updates its own row (or, transposed, its own column) of the block in place
 // from X_N in its registers, and the block goes back to W with coalesced
 // 16-byte stores.
+template <bool PAIR>
 __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int npairs, uint32_t rank,
                                                uint32_t tmem_base, int warp, int lane, uint8_t* wbuf,
                                                uint64_t* acc_full, uint64_t* acc_empty, volatile int* abort_flag) {
+    using S = Shape<NS_FINAL, PAIR>;
+    constexpr int CPW = S::CPW;
     const int quad = warp & 3, half = (warp - 2) / 4;
     const long long limit = L.wait_limit_ns;
-    const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
-    const uint32_t acc_empty_leader1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
+    const uint32_t acc_empty_leader0 = PAIR ? mapa_shared(smem_u32(&acc_empty[0]), 0) : 0u;
+    const uint32_t acc_empty_leader1 = PAIR ? mapa_shared(smem_u32(&acc_empty[1]), 0) : 0u;
     int lt = 0;
     for (int t = pair; t < L.total_tiles; t += npairs, ++lt) {
         const JobTile jt = decode_job_tile(L, NS_FINAL, t);
@@ -239,12 +262,12 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int 
         const float decay = p.decay, lrs = p.lr_s;
         const int acc = lt & 1;
         const uint32_t use = (uint32_t)(lt >> 1);
-        const int row_lo = tc.ti * BM + (int)rank * HM + quad * 32;
+        const int row_lo = tc.ti * S::TM + (int)rank * HM + quad * 32;
         const int bidx = tc.u / p.heads, h = tc.u - bidx * p.heads;
         float* Wb = L.W[p.w0 + bidx] + (int64_t)h * p.Rh * p.C;
         // geometry of chunk c's W block: its first W row, first W column, and extents
         auto block = [&](int c, int& r0, int& c0, int& nr, int& rb) -> bool {
-            const int col0 = tc.tj * BN + (half * 4 + c) * 32;
+            const int col0 = tc.tj * S::TN + (half * CPW + c) * 32;
             if (row_lo >= m || col0 >= n) return false;
             if (!p.transposed) { r0 = row_lo; c0 = col0; nr = min(32, m - row_lo); rb = min(32, n - col0) * 4; }
             else { r0 = col0; c0 = row_lo; nr = min(32, n - col0); rb = min(32, m - row_lo) * 4; }
@@ -252,7 +275,7 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int 
         };
         auto fetch = [&](int c) {
             int r0, c0, nr, rb;
-            if (c < 4 && block(c, r0, c0, nr, rb)) {
+            if (c < CPW && block(c, r0, c0, nr, rb)) {
                 uint8_t* buf = wbuf + (c & 1) * WBUF;
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
@@ -271,13 +294,13 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int 
         if (!ok) break;
         tc_fence_after();
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < CPW; ++c) {
             int r0, c0, nr, rb;
             if (!block(c, r0, c0, nr, rb)) break;  // warp-uniform
-            const int col0 = tc.tj * BN + (half * 4 + c) * 32;
+            const int col0 = tc.tj * S::TN + (half * CPW + c) * 32;
             uint8_t* buf = wbuf + (c & 1) * WBUF;
             float v[32], o[32];
-            tmem_ld32(tmem_base + (uint32_t)(acc * BN + (half * 4 + c) * 32) + ((uint32_t)(quad * 32) << 16), v);
+            tmem_ld32(tmem_base + (uint32_t)(acc * S::TN + (half * CPW + c) * 32) + ((uint32_t)(quad * 32) << 16), v);
             epilogue_values<NS_FINAL>(p, tc, row_lo + lane, col0, v, o);
             // chunk c's copies are the oldest group but one (chunk c + 1 was issued after it)
             cp_async_wait<1>();
@@ -317,7 +340,10 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int 
         if (!ok) break;
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);
+        if (lane == 0) {
+            if (PAIR) mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);
+            else mbar_arrive(&acc_empty[acc]);
+        }
     }
     cp_async_wait<0>();
 }
@@ -326,14 +352,15 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int 
 // 64-byte swizzle that the bulk tensor store expects.
 __device__ __forceinline__ uint32_t sw64(uint32_t r, uint32_t q) { return r * 64u + ((q ^ ((r >> 1) & 3u)) << 4); }
 
-template <int MODE>
+template <int MODE, bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
     ns_tc_kernel(const __grid_constant__ NsLaunch L) {
+    using S = Shape<MODE, PAIR>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    constexpr int NST = kStages(MODE);
-    uint8_t* staging = smem + NST * STAGE_BYTES;
-    uint64_t* full = reinterpret_cast<uint64_t*>(staging + kEpiBytes(MODE));
+    constexpr int NST = S::NST;
+    uint8_t* staging = smem + NST * S::STAGE;
+    uint64_t* full = reinterpret_cast<uint64_t*>(staging + S::EPI);
     uint64_t* empty = full + NST;
     uint64_t* acc_full = empty + NST;
     uint64_t* acc_empty = acc_full + 2;
@@ -343,9 +370,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const uint32_t rank = cluster_ctarank();  // 0 = leader of the pair
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = leader of the pair
     const bool leader = rank == 0;
-    const int pair = (int)cluster_id_x(), npairs = (int)cluster_count_x();
+    const int pair = PAIR ? (int)cluster_id_x() : (int)blockIdx.x;
+    const int npairs = PAIR ? (int)cluster_count_x() : (int)gridDim.x;
     const int total_tiles = L.total_tiles;
     const long long limit = L.wait_limit_ns;
     constexpr bool kApply = (MODE == NS_APPLY || MODE == NS_FINAL);
@@ -358,7 +386,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int w = 0; w < 2 * EPI_WARPS; ++w) mbar_init(&wbar[w], 1);
         for (int a = 0; a < 2; ++a) {
             mbar_init(&acc_full[a], 1);                  // both: one multicast commit per tile
-            mbar_init(&acc_empty[a], 2 * EPI_WARPS);     // leader: every epilogue warp of the pair
+            mbar_init(&acc_empty[a], (PAIR ? 2 : 1) * EPI_WARPS);  // leader: every epilogue warp of the pair
         }
         mbar_init(drain, 1);
         *abort_flag = 0;
@@ -370,11 +398,17 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     }
     if (warp == 1) {
-        tmem_alloc_pair(tmem_holder, TMEM_COLS);
-        tmem_relinquish_pair();
+        if (PAIR) {
+            tmem_alloc_pair(tmem_holder, S::TMEM);
+            tmem_relinquish_pair();
+        } else {
+            tmem_alloc(tmem_holder, S::TMEM);
+            tmem_relinquish();
+        }
     }
     tc_fence_before();
-    cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated in both
+    if (PAIR) cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated in both
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
 
@@ -389,24 +423,36 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const CUtensorMap* mapA = &L.mA[jt.j];
                 const CUtensorMap* mapB = &L.mB[jt.j];
                 const int kblocks = L.job[jt.j].kblocks;
-                const int arow = tc.ti * BM + (int)rank * HM;
-                const int bcol = tc.tj * BN + (int)rank * HN;
+                const int arow = tc.ti * S::TM + (int)rank * HM;
+                const int bcol = tc.tj * S::TN + (int)rank * S::CN;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit, L.status)) {
                         ok = false;
                         break;
                     }
-                    uint8_t* sa = smem + stage * STAGE_BYTES;
+                    uint8_t* sa = smem + stage * S::STAGE;
                     uint8_t* sb = sa + A_BYTES;
-                    if (leader) mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
-                    const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
-                    tma_load_3d_pair(sa, mapA, fb, kb * BK, arow, tc.u);
-                    if (!kApply) {
-                        tma_load_3d_pair(sb, mapB, fb, kb * BK, bcol, tc.u);
-                    } else {
+                    if (PAIR) {
+                        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * S::STAGE);
+                        const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+                        tma_load_3d_pair(sa, mapA, fb, kb * BK, arow, tc.u);
+                        if (!kApply) {
+                            tma_load_3d_pair(sb, mapB, fb, kb * BK, bcol, tc.u);
+                        } else {
 #pragma unroll
-                        for (int q = 0; q < HN / 64; ++q)
-                            tma_load_3d_pair(sb + q * (64 * BK * 2), mapB, fb, bcol + q * 64, kb * BK, tc.u);
+                            for (int q = 0; q < S::CN / 64; ++q)
+                                tma_load_3d_pair(sb + q * (64 * BK * 2), mapB, fb, bcol + q * 64, kb * BK, tc.u);
+                        }
+                    } else {
+                        mbar_arrive_expect_tx(&full[stage], S::STAGE);
+                        tma_load_3d(sa, mapA, &full[stage], kb * BK, arow, tc.u);
+                        if (!kApply) {
+                            tma_load_3d(sb, mapB, &full[stage], kb * BK, bcol, tc.u);  // CN = 128 rows
+                        } else {
+#pragma unroll
+                            for (int q = 0; q < S::CN / 64; ++q)
+                                tma_load_3d(sb + q * (64 * BK * 2), mapB, &full[stage], bcol + q * 64, kb * BK, tc.u);
+                        }
                     }
                     if (++stage == NST) {
                         stage = 0;
@@ -426,7 +472,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     } else if (warp == 1) {
         if (lane == 0 && leader) {
-            constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, kApply ? 1 : 0);
+            constexpr uint32_t IDESC = idesc_bf16_f32(S::TM, S::TN, kApply ? 1 : 0);
             int stage = 0;
             uint32_t phase = 0;
             int lt = 0;
@@ -439,7 +485,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+                const uint32_t d_tmem = tmem_base + (uint32_t)(acc * S::TN);
                 const int kblocks = L.job[decode_job_tile(L, MODE, t).j].kblocks;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag, limit, L.status)) {
@@ -447,7 +493,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t a0 = smem_u32(smem + stage * STAGE_BYTES);
+                    const uint32_t a0 = smem_u32(smem + stage * S::STAGE);
                     const uint32_t b0 = a0 + A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
@@ -457,32 +503,36 @@ __global__ void __launch_bounds__(THREADS, 1)
                             bdesc = smem_desc_sw128(b0 + kk * (16 * 128), 64 * BK * 2, 1024);
                         else
                             bdesc = smem_desc_sw128(b0 + kk * 32, 16, 1024);
-                        tc_mma_f16_pair(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                        if (PAIR) tc_mma_f16_pair(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
+                        else tc_mma_f16(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
                     }
-                    tc_commit_pair_mc(&empty[stage], 0x3);
+                    if (PAIR) tc_commit_pair_mc(&empty[stage], 0x3);
+                    else tc_commit(&empty[stage]);
                     if (++stage == NST) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                tc_commit_pair_mc(&acc_full[acc], 0x3);
+                if (PAIR) tc_commit_pair_mc(&acc_full[acc], 0x3);
+                else tc_commit(&acc_full[acc]);
             }
             if (!ok) {
                 // let every MMA issued so far finish before TMEM is released
-                tc_commit_pair(drain);
+                if (PAIR) tc_commit_pair(drain);
+                else tc_commit(drain);
                 mbar_wait_bounded(drain, 0, abort_flag, limit, L.status);
             }
         }
     } else if (MODE == NS_FINAL) {
-        final_epilogue(L, pair, npairs, rank, tmem_base, warp, lane, staging + (warp - 2) * 2 * WBUF, acc_full,
-                       acc_empty, abort_flag);
+        final_epilogue<PAIR>(L, pair, npairs, rank, tmem_base, warp, lane, staging + (warp - 2) * 2 * WBUF,
+                             acc_full, acc_empty, abort_flag);
     } else {
         const int quad = warp & 3;              // TMEM lanes [32*quad, 32*quad + 32)
         const int half = (warp - 2) / 4;        // which half of the 256 columns
         uint8_t* stg = staging + (warp - 2) * 2 * STG_BLOCK;
-        const uint32_t acc_empty_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0);
-        const uint32_t acc_empty_leader1 = mapa_shared(smem_u32(&acc_empty[1]), 0);
+        const uint32_t acc_empty_leader0 = PAIR ? mapa_shared(smem_u32(&acc_empty[0]), 0) : 0u;
+        const uint32_t acc_empty_leader1 = PAIR ? mapa_shared(smem_u32(&acc_empty[1]), 0) : 0u;
         int lt = 0;
         for (int t = pair; t < total_tiles; t += npairs, ++lt) {
             const JobTile jt = decode_job_tile(L, MODE, t);
@@ -491,7 +541,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const TileCoord tc = jt.tc;
             const int acc = lt & 1;
             const uint32_t use = (uint32_t)(lt >> 1);
-            const int row_lo = tc.ti * BM + (int)rank * HM + quad * 32;
+            const int row_lo = tc.ti * S::TM + (int)rank * HM + quad * 32;
             const int row = row_lo + lane;
             int ok = 1;
             if (lane == 0)
@@ -501,13 +551,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             tc_fence_after();
             const int limit_cols = kApply ? p.n : p.m;
 #pragma unroll 1
-            for (int c = 0; c < 4; ++c) {
-                const int cc = half * 4 + c;
-                const int col0 = tc.tj * BN + cc * 32;
+            for (int c = 0; c < S::CPW; ++c) {
+                const int cc = half * S::CPW + c;
+                const int col0 = tc.tj * S::TN + cc * 32;
                 if (col0 >= limit_cols || row_lo >= p.m) break;                  // warp-uniform
                 if (!kApply && col0 < row_lo) continue;                          // below the diagonal
                 float o[32];
-                tmem_ld32(tmem_base + (uint32_t)(acc * BN + cc * 32) + ((uint32_t)(quad * 32) << 16), o);
+                tmem_ld32(tmem_base + (uint32_t)(acc * S::TN + cc * 32) + ((uint32_t)(quad * 32) << 16), o);
                 epilogue_values<MODE>(p, tc, row, col0, o, o);  // in place
                 // Stage this warp's 32 x 32 block (and, for an off-diagonal Gram
                 // chunk, its transpose), then write both with bulk tensor stores:
@@ -540,7 +590,10 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);
+            if (lane == 0) {
+                if (PAIR) mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);
+                else mbar_arrive(&acc_empty[acc]);
+            }
         }
         if (lane == 0) bulk_wait_group0();  // every bulk store of this warp has completed
     }
@@ -553,10 +606,12 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
     }
     tc_fence_before();
-    cluster_sync_all();  // neither CTA leaves while the pair may still touch its memory
+    if (PAIR) cluster_sync_all();  // neither CTA leaves while the pair may still touch its memory
+    else __syncthreads();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc_pair(tmem_base, TMEM_COLS);
+        if (PAIR) tmem_dealloc_pair(tmem_base, S::TMEM);
+        else tmem_dealloc(tmem_base, S::TMEM);
     }
 }
 
@@ -592,8 +647,9 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int MODE>
+template <int MODE, bool PAIR>
 cudaError_t launch_mode(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_t s) {
+    using S = Shape<MODE, PAIR>;
     if (njobs < 1 || njobs > kMaxJobs) return cudaErrorInvalidValue;
     static thread_local NsLaunch L;  // ~9 KB parameter block, copied at launch
     std::memset(&L, 0, sizeof(L));
@@ -604,9 +660,9 @@ cudaError_t launch_mode(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_
         const void* g_buf = jobs[j].g_buf;
         NsJob& J = L.job[j];
         int kblocks, mt, nt, tiles;
-        mt = (p.m + BM - 1) / BM;
+        mt = (p.m + S::TM - 1) / S::TM;
         if (MODE == NS_GRAM || MODE == NS_GRAMSQ) {
-            nt = mt;
+            nt = (p.m + S::TN - 1) / S::TN;  // S::TN == S::TM for the Gram
             tiles = nt * (nt + 1) / 2;
             if (MODE == NS_GRAM) {
                 kblocks = (p.n + BK - 1) / BK;
@@ -620,7 +676,7 @@ cudaError_t launch_mode(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_
             if (!make_map(&L.mO[j], p.out, p.m, p.m, p.units, p.ldg, p.g_unit, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
                 return cudaErrorInvalidValue;
         } else {
-            nt = (p.n + BN - 1) / BN;
+            nt = (p.n + S::TN - 1) / S::TN;
             tiles = mt * nt;
             kblocks = (p.m + BK - 1) / BK;
             if (!make_map(&L.mA[j], g_buf, p.m, p.m, p.units, p.ldg, p.g_unit, BK, HM)) return cudaErrorInvalidValue;
@@ -654,48 +710,76 @@ cudaError_t launch_mode(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_
     L.status = jobs[0].p->status;
     if (tile0 <= 0) return cudaSuccess;
     static unsigned long long attr_set = 0;  // one bit per device
-    static int max_pairs[64] = {0};
+    static int max_units[64] = {0};          // resident pairs (or CTAs) per device
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!(attr_set & (1ull << dev))) {
-        e = cudaFuncSetAttribute(ns_tc_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes(MODE));
-        if (e != cudaSuccess) return e;
-        e = cudaFuncSetAttribute(ns_tc_kernel<MODE>, cudaFuncAttributeNonPortableClusterSizeAllowed, 0);
-        if (e != cudaSuccess) return e;
-        cudaLaunchConfig_t qc = {};
-        cudaLaunchAttribute qa[1];
-        qa[0].id = cudaLaunchAttributeClusterDimension;
-        qa[0].val.clusterDim.x = 2;
-        qa[0].val.clusterDim.y = 1;
-        qa[0].val.clusterDim.z = 1;
-        qc.gridDim = dim3(2 * (unsigned)(num_sms / 2));
-        qc.blockDim = dim3(THREADS);
-        qc.dynamicSmemBytes = kSmemBytes(MODE);
-        qc.attrs = qa;
-        qc.numAttrs = 1;
-        int nclusters = 0;
-        e = cudaOccupancyMaxActiveClusters(&nclusters, ns_tc_kernel<MODE>, &qc);
-        if (e != cudaSuccess) return e;
-        if (nclusters < 1) return cudaErrorInvalidConfiguration;
-        max_pairs[dev] = nclusters;
-        attr_set |= 1ull << dev;
-    }
-    const long long pairs = tile0 < max_pairs[dev] ? tile0 : max_pairs[dev];
-    cudaLaunchConfig_t cfg = {};
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    cfg.gridDim = dim3((unsigned)(2 * pairs));
+    if (!(attr_set & (1ull << dev))) {
+        e = cudaFuncSetAttribute(ns_tc_kernel<MODE, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM);
+        if (e != cudaSuccess) return e;
+        if (PAIR) {
+            cudaLaunchConfig_t qc = {};
+            qc.gridDim = dim3(2 * (unsigned)(num_sms / 2));
+            qc.blockDim = dim3(THREADS);
+            qc.dynamicSmemBytes = S::SMEM;
+            qc.attrs = attr;
+            qc.numAttrs = 1;
+            int nclusters = 0;
+            e = cudaOccupancyMaxActiveClusters(&nclusters, ns_tc_kernel<MODE, PAIR>, &qc);
+            if (e != cudaSuccess) return e;
+            if (nclusters < 1) return cudaErrorInvalidConfiguration;
+            max_units[dev] = nclusters;
+        } else {
+            int per_sm = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ns_tc_kernel<MODE, PAIR>, THREADS, S::SMEM);
+            if (e != cudaSuccess) return e;
+            if (per_sm < 1) return cudaErrorInvalidConfiguration;
+            max_units[dev] = per_sm * num_sms;
+        }
+        attr_set |= 1ull << dev;
+    }
+    const long long units = tile0 < max_units[dev] ? tile0 : max_units[dev];
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)((PAIR ? 2 : 1) * units));
     cfg.blockDim = dim3(THREADS);
-    cfg.dynamicSmemBytes = kSmemBytes(MODE);
+    cfg.dynamicSmemBytes = S::SMEM;
     cfg.stream = s;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, ns_tc_kernel<MODE>, L);
+    cfg.attrs = PAIR ? attr : nullptr;
+    cfg.numAttrs = PAIR ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, ns_tc_kernel<MODE, PAIR>, L);
+}
+
+// Units with m <= 128 fill only half of a pair's 256-row tile: they take the
+// single-CTA kernel.
+bool single_cta(const NsParams& p) { return p.m <= HM; }
+
+template <int MODE>
+cudaError_t launch_split(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_t s, int* launched) {
+    NsJobIn big[kMaxJobs], small[kMaxJobs];
+    int nb = 0, ns = 0;
+    for (int j = 0; j < njobs && j < kMaxJobs; ++j) {
+        if (single_cta(*jobs[j].p)) small[ns++] = jobs[j];
+        else big[nb++] = jobs[j];
+    }
+    if (njobs > kMaxJobs) return cudaErrorInvalidValue;
+    cudaError_t e = cudaSuccess;
+    if (nb > 0) {
+        e = launch_mode<MODE, true>(big, nb, num_sms, s);
+        if (e != cudaSuccess) return e;
+        ++*launched;
+    }
+    if (ns > 0) {
+        e = launch_mode<MODE, false>(small, ns, num_sms, s);
+        if (e != cudaSuccess) return e;
+        ++*launched;
+    }
+    return cudaSuccess;
 }
 
 }  // namespace
@@ -704,12 +788,15 @@ size_t ns_tc_smem_bytes() { return SMEM_BYTES; }
 int ns_tc_max_jobs() { return kMaxJobs; }
 int ns_tc_max_weights() { return kMaxW; }
 
-cudaError_t launch_ns_tc_group(int mode, const NsJobIn* jobs, int njobs, int num_sms, cudaStream_t s) {
+cudaError_t launch_ns_tc_group(int mode, const NsJobIn* jobs, int njobs, int num_sms, cudaStream_t s,
+                               int* launched) {
+    int dummy = 0;
+    if (!launched) launched = &dummy;
     switch (mode) {
-        case NS_GRAM: return launch_mode<NS_GRAM>(jobs, njobs, num_sms, s);
-        case NS_GRAMSQ: return launch_mode<NS_GRAMSQ>(jobs, njobs, num_sms, s);
-        case NS_APPLY: return launch_mode<NS_APPLY>(jobs, njobs, num_sms, s);
-        case NS_FINAL: return launch_mode<NS_FINAL>(jobs, njobs, num_sms, s);
+        case NS_GRAM: return launch_split<NS_GRAM>(jobs, njobs, num_sms, s, launched);
+        case NS_GRAMSQ: return launch_split<NS_GRAMSQ>(jobs, njobs, num_sms, s, launched);
+        case NS_APPLY: return launch_split<NS_APPLY>(jobs, njobs, num_sms, s, launched);
+        case NS_FINAL: return launch_split<NS_FINAL>(jobs, njobs, num_sms, s, launched);
         default: return cudaErrorInvalidValue;
     }
 }
@@ -717,7 +804,7 @@ cudaError_t launch_ns_tc_group(int mode, const NsJobIn* jobs, int njobs, int num
 cudaError_t launch_ns_tc(int mode, const NsParams& p, const void* x_buf, const void* g_buf, int num_sms,
                          cudaStream_t s) {
     NsJobIn j{&p, x_buf, g_buf};
-    return launch_ns_tc_group(mode, &j, 1, num_sms, s);
+    return launch_ns_tc_group(mode, &j, 1, num_sms, s, nullptr);
 }
 
 }  // namespace ma

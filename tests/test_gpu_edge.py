@@ -225,7 +225,12 @@ def test_grouped_newton_schulz_launches_match_per_bucket_calls():
             assert torch.equal(Wd[k], params[i + k]), f"bucket {bi} matrix {k}"
             assert torch.equal(Md[k], opt.state[i + k][0]), f"bucket {bi} momentum {k}"
         i += cnt
-    # two launches of momentum and norm per bucket; Newton-Schulz: 8 cubic
-    # buckets in one set, the ninth alone (2 launches a step each), the two
-    # quintic buckets together (3 a step)
-    assert grouped == 2 * len(shapes) + 2 * 5 + 2 * 5 + 3 * 5
+    # Two launches of momentum and norm per bucket. Newton-Schulz: 8 cubic
+    # buckets in one set, the ninth alone (2 kernels a step), the two quintic
+    # buckets together (3 a step); a set with units of m <= 128 and of
+    # m > 128 takes one kernel of each tile shape per kernel of the chain.
+    def kinds(bis):
+        small = [min(shapes[b][0] // hps[which[b]].heads, shapes[b][1]) <= 128 for b in bis]
+        return int(any(small)) + int(not all(small))
+    sets = [(range(0, 8), 2), (range(8, 9), 2), (range(9, 11), 3)]
+    assert grouped == 2 * len(shapes) + sum(5 * per * kinds(b) for b, per in sets)

@@ -131,6 +131,8 @@ MUON_CASES = [
     ((256, 512), 4, True, 0, (oracle.CUBIC,)),      # per-head, wide slices 64 x 512
     ((512, 128), 2, True, 0, (oracle.CUBIC,)),      # per-head, tall slices 256 x 128
     ((128, 384), 1, True, 0, ((2.0, -1.5, 0.5), (1.5, -0.5, 0.0))),  # c != 0 schedule
+    ((96, 200), 1, True, 0, (oracle.CUBIC,)),       # ragged, m < 128 (single-CTA tiles)
+    ((384, 120), 1, True, 0, ((2.0, -1.5, 0.5), (1.5, -0.5, 0.0))),  # tall, m = 120, c != 0
 ]
 
 
