@@ -68,11 +68,14 @@ constexpr uint32_t STG_BLOCK = 32 * 32 * 2;
 #endif
 constexpr uint32_t kEpiSleepNs = MA_EPI_SLEEP_NS;
 constexpr uint32_t STG_BYTES = EPI_WARPS * 2 * STG_BLOCK;  // 32 KB
-// Final apply: each epilogue warp double-buffers 32 x 32 fp32 blocks of W,
-// rows padded to 144 bytes (conflict-free row and column access).
-constexpr uint32_t WROW = 144;
-constexpr uint32_t WBUF = 32 * WROW;                        // 4.5 KB
-constexpr uint32_t WBUF_BYTES = EPI_WARPS * 2 * WBUF;       // 72 KB
+// Final apply: each epilogue warp double-buffers a 32 x 32 fp32 block of W
+// (128-byte rows) and the matching 32 x 32 bf16 block of X (64-byte rows).
+// The 16-byte chunks of each row are XOR-swizzled by the row index, which
+// keeps row-wise and column-wise accesses free of bank conflicts.
+constexpr uint32_t WBUF = 32 * 128;                              // 4 KB
+constexpr uint32_t XBUF = 32 * 64;                               // 2 KB
+constexpr uint32_t FIN_WARP_BYTES = 2 * WBUF + 2 * XBUF;         // 12 KB
+constexpr uint32_t WBUF_BYTES = EPI_WARPS * FIN_WARP_BYTES;      // 96 KB
 constexpr int kStages(int mode) { return mode == NS_FINAL ? 4 : STAGES; }
 constexpr uint32_t kEpiBytes(int mode) { return mode == NS_FINAL ? WBUF_BYTES : STG_BYTES; }
 constexpr size_t kSmemBytes(int mode) {
@@ -231,18 +234,25 @@ __device__ __forceinline__ float apply_update(float w, float x, float decay, flo
 }
 
 
+// Byte offset of 16-byte chunk q of row r in a 64-byte-row block with the
+// 64-byte swizzle that the bulk tensor store expects.
+__device__ __forceinline__ uint32_t sw64(uint32_t r, uint32_t q) { return r * 64u + ((q ^ ((r >> 1) & 3u)) << 4); }
+
+// Byte offset of 16-byte chunk q of row r in a 128-byte-row block of W.
+__device__ __forceinline__ uint32_t sw128w(uint32_t r, uint32_t q) { return r * 128u + ((q ^ (r & 7u)) << 4); }
+
 // Final apply: W <- W*(1 - lr*wd) - lr*scale*X_N in the caller's fp32 weights,
-// run by each epilogue warp over its four 32-column chunks of every tile.
+// run by each epilogue warp over its 32-column chunks of every tile.
 //
-// The chunk's 32 x 32 block of W (in W's own orientation: transposed back
-// when the unit was tall) comes into one of two shared-memory buffers by
-// 16-byte asynchronous copies, 8 lanes per 128-byte row. The first two chunks
-// of a tile are fetched before the accumulator is ready, and each later chunk
-// while the one before it is being computed, so the weights' DRAM latency
-// hides behind the main loop without holding registers. Each lane then
-// updates its own row (or, transposed, its own column) of the block in place
-// from X_N in its registers, and the block goes back to W with coalesced
-// 16-byte stores.
+// For each chunk, the 32 x 32 block of W (in W's own orientation: transposed
+// back when the unit was tall) and the 32 x 32 block of X that the a*X term
+// needs come into shared memory by 16-byte asynchronous copies. The first two
+// chunks of a tile are fetched before the accumulator is ready, and each
+// later chunk while the one before it is being computed, so the DRAM latency
+// of both hides behind the main loop without holding registers. Each lane
+// then forms its row of X_N from the accumulator and X, updates its own row
+// (or, transposed, its own column) of the W block in place, and the block
+// goes back to W with coalesced 16-byte stores.
 template <bool PAIR>
 __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int npairs, uint32_t rank,
                                                uint32_t tmem_base, int warp, int lane, uint8_t* wbuf,
@@ -253,6 +263,7 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int 
     const long long limit = L.wait_limit_ns;
     const uint32_t acc_empty_leader0 = PAIR ? mapa_shared(smem_u32(&acc_empty[0]), 0) : 0u;
     const uint32_t acc_empty_leader1 = PAIR ? mapa_shared(smem_u32(&acc_empty[1]), 0) : 0u;
+    uint8_t* xbuf = wbuf + 2 * WBUF;
     int lt = 0;
     for (int t = pair; t < L.total_tiles; t += npairs, ++lt) {
         const JobTile jt = decode_job_tile(L, NS_FINAL, t);
@@ -260,11 +271,14 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int 
         const TileCoord tc = jt.tc;
         const int m = p.m, n = p.n;
         const float decay = p.decay, lrs = p.lr_s;
+        const float sa = p.first ? p.scale[tc.u] : 1.f;
+        const float ca = sa * p.a;
         const int acc = lt & 1;
         const uint32_t use = (uint32_t)(lt >> 1);
         const int row_lo = tc.ti * S::TM + (int)rank * HM + quad * 32;
         const int bidx = tc.u / p.heads, h = tc.u - bidx * p.heads;
         float* Wb = L.W[p.w0 + bidx] + (int64_t)h * p.Rh * p.C;
+        const __nv_bfloat16* Xin = reinterpret_cast<const __nv_bfloat16*>(p.xin) + (int64_t)tc.u * p.x_unit;
         // geometry of chunk c's W block: its first W row, first W column, and extents
         auto block = [&](int c, int& r0, int& c0, int& nr, int& rb) -> bool {
             const int col0 = tc.tj * S::TN + (half * CPW + c) * 32;
@@ -281,7 +295,16 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int 
                 for (int i = 0; i < 8; ++i) {
                     const int row = 4 * i + (lane >> 3), q = lane & 7;
                     if (row < nr && q * 16 < rb)
-                        cp_async16(buf + row * WROW + q * 16, Wb + (int64_t)(r0 + row) * p.C + c0 + q * 4);
+                        cp_async16(buf + sw128w(row, q), Wb + (int64_t)(r0 + row) * p.C + c0 + q * 4);
+                }
+                // X rows row_lo.., columns col0..: 8 bf16 per copy; the row stride is a multiple of 8
+                const int col0 = tc.tj * S::TN + (half * CPW + c) * 32;
+                uint8_t* xb = xbuf + (c & 1) * XBUF;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int row = 8 * i + (lane >> 2), q = lane & 3;
+                    if (row_lo + row < m && col0 + 8 * q < n)
+                        cp_async16(xb + sw64(row, q), Xin + (int64_t)(row_lo + row) * p.ldx + col0 + 8 * q);
                 }
             }
             cp_async_commit();  // one group per chunk, empty or not, so the counts line up
@@ -297,19 +320,29 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int 
         for (int c = 0; c < CPW; ++c) {
             int r0, c0, nr, rb;
             if (!block(c, r0, c0, nr, rb)) break;  // warp-uniform
-            const int col0 = tc.tj * S::TN + (half * CPW + c) * 32;
             uint8_t* buf = wbuf + (c & 1) * WBUF;
-            float v[32], o[32];
-            tmem_ld32(tmem_base + (uint32_t)(acc * S::TN + (half * CPW + c) * 32) + ((uint32_t)(quad * 32) << 16), v);
-            epilogue_values<NS_FINAL>(p, tc, row_lo + lane, col0, v, o);
+            const uint8_t* xb = xbuf + (c & 1) * XBUF;
+            float o[32];
+            tmem_ld32(tmem_base + (uint32_t)(acc * S::TN + (half * CPW + c) * 32) + ((uint32_t)(quad * 32) << 16), o);
             // chunk c's copies are the oldest group but one (chunk c + 1 was issued after it)
             cp_async_wait<1>();
             __syncwarp();
+            // X_N row of this lane: s*(a*X + (B X)), s only on the first iteration
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 w = *reinterpret_cast<const uint4*>(xb + sw64(lane, q));
+                const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    o[8 * q + 2 * e] = ca * bf16_lo(wv[e]) + sa * o[8 * q + 2 * e];
+                    o[8 * q + 2 * e + 1] = ca * bf16_hi(wv[e]) + sa * o[8 * q + 2 * e + 1];
+                }
+            }
             if (!p.transposed) {
                 // lane = row of W: 32 consecutive elements
 #pragma unroll
                 for (int q = 0; q < 8; ++q) {
-                    float4* wq = reinterpret_cast<float4*>(buf + lane * WROW + q * 16);
+                    float4* wq = reinterpret_cast<float4*>(buf + sw128w(lane, q));
                     float4 w = *wq;
                     w.x = apply_update(w.x, o[4 * q + 0], decay, lrs, p);
                     w.y = apply_update(w.y, o[4 * q + 1], decay, lrs, p);
@@ -321,7 +354,7 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int 
                 // lane = column of W: element t of the lane's X_N row is W[t][lane]
 #pragma unroll
                 for (int q = 0; q < 32; ++q) {
-                    float* wq = reinterpret_cast<float*>(buf + q * WROW + lane * 4);
+                    float* wq = reinterpret_cast<float*>(buf + sw128w(q, lane >> 2) + (lane & 3) * 4);
                     *wq = apply_update(*wq, o[q], decay, lrs, p);
                 }
             }
@@ -331,9 +364,9 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int 
                 const int row = 4 * i + (lane >> 3), q = lane & 7;
                 if (row < nr && q * 16 < rb)
                     *reinterpret_cast<float4*>(Wb + (int64_t)(r0 + row) * p.C + c0 + q * 4) =
-                        *reinterpret_cast<const float4*>(buf + row * WROW + q * 16);
+                        *reinterpret_cast<const float4*>(buf + sw128w(row, q));
             }
-            __syncwarp();  // the buffer is free again
+            __syncwarp();  // both buffers of chunk c are free again
             fetch(c + 2);
         }
         cp_async_wait<0>();  // drop the copies of chunks this tile does not use
@@ -348,9 +381,6 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int 
     cp_async_wait<0>();
 }
 
-// Byte offset of 16-byte chunk q of row r in a 64-byte-row block with the
-// 64-byte swizzle that the bulk tensor store expects.
-__device__ __forceinline__ uint32_t sw64(uint32_t r, uint32_t q) { return r * 64u + ((q ^ ((r >> 1) & 3u)) << 4); }
 
 template <int MODE, bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -525,7 +555,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
     } else if (MODE == NS_FINAL) {
-        final_epilogue<PAIR>(L, pair, npairs, rank, tmem_base, warp, lane, staging + (warp - 2) * 2 * WBUF,
+        final_epilogue<PAIR>(L, pair, npairs, rank, tmem_base, warp, lane, staging + (warp - 2) * FIN_WARP_BYTES,
                              acc_full, acc_empty, abort_flag);
     } else {
         const int quad = warp & 3;              // TMEM lanes [32*quad, 32*quad + 32)
