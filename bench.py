@@ -367,11 +367,15 @@ def main():
         ns_fl = sum(prof[c]["flops"] for c in ns_cls)
         ns_launches = sum(prof[c]["launches"] for c in ns_cls)
         ns_tflops = ns_fl / (ns_ms / 1000.0) / 1e12 if ns_ms > 0 else None
-        peak_t = peaks["bf16_tflops_sustained"]
+        # The sustained (power-capped) GEMM peak applies when the power cap held
+        # the SM clock down during the timed region; at full clock, the burst one.
+        capped = bool(clk and clk.get("sm_mhz") and clk.get("sm_max_mhz")
+                      and clk["sm_mhz"] < 0.95 * clk["sm_max_mhz"])
+        peak_t = peaks["bf16_tflops_sustained"] if capped else peaks["bf16_tflops"]
         roofline = {"kernel": "ns_tc_kernel (Newton-Schulz Gram + apply, tcgen05)", "bound": "tensor",
                     "achieved": ns_tflops, "peak": peak_t, "unit": "TFLOP/s",
                     "frac": ns_tflops / peak_t if ns_tflops else None,
-                    "peak_kind": f"bf16 dense, sustained ({peaks['source']})",
+                    "peak_kind": f"bf16 dense, {'sustained' if capped else 'burst'} ({peaks['source']})",
                     "traffic": NS_TRAFFIC_BYTES_PER_LAUNCH,
                     "launches": ns_launches, "avg_launch_ms": ns_ms / max(1, ns_launches),
                     "flops_per_launch": ns_fl / max(1, ns_launches)}
