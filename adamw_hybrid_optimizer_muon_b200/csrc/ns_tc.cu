@@ -455,6 +455,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int kblocks = L.job[jt.j].kblocks;
                 const int arow = tc.ti * S::TM + (int)rank * HM;
                 const int bcol = tc.tj * S::TN + (int)rank * S::CN;
+                // a diagonal Gram tile multiplies a block of rows by itself: B is A's smem
+                const bool diag = !kApply && tc.ti == tc.tj;
+                const uint32_t stage_tx = diag ? A_BYTES : S::STAGE;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit, L.status)) {
                         ok = false;
@@ -463,21 +466,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                     uint8_t* sa = smem + stage * S::STAGE;
                     uint8_t* sb = sa + A_BYTES;
                     if (PAIR) {
-                        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * S::STAGE);
+                        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * stage_tx);
                         const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
                         tma_load_3d_pair(sa, mapA, fb, kb * BK, arow, tc.u);
                         if (!kApply) {
-                            tma_load_3d_pair(sb, mapB, fb, kb * BK, bcol, tc.u);
+                            if (!diag) tma_load_3d_pair(sb, mapB, fb, kb * BK, bcol, tc.u);
                         } else {
 #pragma unroll
                             for (int q = 0; q < S::CN / 64; ++q)
                                 tma_load_3d_pair(sb + q * (64 * BK * 2), mapB, fb, bcol + q * 64, kb * BK, tc.u);
                         }
                     } else {
-                        mbar_arrive_expect_tx(&full[stage], S::STAGE);
+                        mbar_arrive_expect_tx(&full[stage], stage_tx);
                         tma_load_3d(sa, mapA, &full[stage], kb * BK, arow, tc.u);
                         if (!kApply) {
-                            tma_load_3d(sb, mapB, &full[stage], kb * BK, bcol, tc.u);  // CN = 128 rows
+                            if (!diag) tma_load_3d(sb, mapB, &full[stage], kb * BK, bcol, tc.u);  // CN = 128 rows
                         } else {
 #pragma unroll
                             for (int q = 0; q < S::CN / 64; ++q)
@@ -516,7 +519,9 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
                 tc_fence_after();
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * S::TN);
-                const int kblocks = L.job[decode_job_tile(L, MODE, t).j].kblocks;
+                const JobTile jt = decode_job_tile(L, MODE, t);
+                const int kblocks = L.job[jt.j].kblocks;
+                const bool diag = !kApply && jt.tc.ti == jt.tc.tj;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait_bounded(&full[stage], phase, abort_flag, limit, L.status)) {
                         ok = false;
@@ -524,7 +529,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                     }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(smem + stage * S::STAGE);
-                    const uint32_t b0 = a0 + A_BYTES;
+                    const uint32_t b0 = diag ? a0 : a0 + A_BYTES;
 #pragma unroll
                     for (int kk = 0; kk < BK / 16; ++kk) {
                         const uint64_t adesc = smem_desc_sw128(a0 + kk * 32, 16, 1024);
