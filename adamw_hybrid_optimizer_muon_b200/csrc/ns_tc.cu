@@ -156,8 +156,11 @@ __device__ __forceinline__ TileCoord decode_tile(int mode, int t, int tiles_per_
         c.ti = r;
         c.tj = tj;
     } else {
-        c.ti = r / nt;
-        c.tj = r - c.ti * nt;
+        // column by column: the pairs working at the same time share the few
+        // column strips of X (the B operand) they read, and all of them read the
+        // m x m Gram, the smaller operand when n > m
+        c.tj = r / mt;
+        c.ti = r - c.tj * mt;
     }
     return c;
 }
@@ -444,6 +447,10 @@ __global__ void __launch_bounds__(THREADS, 1)
 
     if (warp == 0) {
         if (lane == 0) {
+            // In the applies every pair working at the same time reads all of
+            // the m x m Gram (the A operand), one wave after another: keep it in
+            // L2 ahead of the X strips, which each wave reads once.
+            const uint64_t keep = l2_evict_last_policy();
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -468,7 +475,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                     if (PAIR) {
                         if (leader) mbar_arrive_expect_tx(&full[stage], 2 * stage_tx);
                         const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
-                        tma_load_3d_pair(sa, mapA, fb, kb * BK, arow, tc.u);
+                        if (kApply) tma_load_3d_pair_hint(sa, mapA, fb, kb * BK, arow, tc.u, keep);
+                        else tma_load_3d_pair(sa, mapA, fb, kb * BK, arow, tc.u);
                         if (!kApply) {
                             if (!diag) tma_load_3d_pair(sb, mapB, fb, kb * BK, bcol, tc.u);
                         } else {
@@ -478,7 +486,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                         }
                     } else {
                         mbar_arrive_expect_tx(&full[stage], stage_tx);
-                        tma_load_3d(sa, mapA, &full[stage], kb * BK, arow, tc.u);
+                        if (kApply) tma_load_3d_hint(sa, mapA, &full[stage], kb * BK, arow, tc.u, keep);
+                        else tma_load_3d(sa, mapA, &full[stage], kb * BK, arow, tc.u);
                         if (!kApply) {
                             if (!diag) tma_load_3d(sb, mapB, &full[stage], kb * BK, bcol, tc.u);  // CN = 128 rows
                         } else {
@@ -566,6 +575,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int quad = warp & 3;              // TMEM lanes [32*quad, 32*quad + 32)
         const int half = (warp - 2) / 4;        // which half of the 256 columns
         uint8_t* stg = staging + (warp - 2) * 2 * STG_BLOCK;
+        // outputs are read only by the next launch, long after L2 has turned over
+        const uint64_t stream_out = l2_evict_first_policy();
         const uint32_t acc_empty_leader0 = PAIR ? mapa_shared(smem_u32(&acc_empty[0]), 0) : 0u;
         const uint32_t acc_empty_leader1 = PAIR ? mapa_shared(smem_u32(&acc_empty[1]), 0) : 0u;
         int lt = 0;
@@ -618,8 +629,8 @@ __global__ void __launch_bounds__(THREADS, 1)
                 fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_3d(mapOut, stg, col0, row_lo, tc.u);
-                    if (mirror) tma_store_3d(mapOut, stg + STG_BLOCK, row_lo, col0, tc.u);
+                    tma_store_3d_hint(mapOut, stg, col0, row_lo, tc.u, stream_out);
+                    if (mirror) tma_store_3d_hint(mapOut, stg + STG_BLOCK, row_lo, col0, tc.u, stream_out);
                     bulk_commit_group();
                 }
             }
