@@ -18,11 +18,13 @@
 //           X_N is never rounded or stored.
 //
 // Kernel structure: CTA pairs (clusters of 2), persistent over the 256 x 256
-// output tiles of all units of a batch, 320 threads per CTA:
+// output tiles of every unit of the launch's jobs (up to eight batches of
+// one mode, tiles numbered job after job), 320 threads per CTA:
 //   warp 0      TMA producer in each CTA: this CTA's half of the A tile
 //               (128 rows x 64) and of the B tile (128 columns x 64), bf16,
-//               128B swizzle, 6 stages of 32 KB. Both CTAs' loads complete on
-//               the leader CTA's stage barrier; there is no multicast.
+//               128B swizzle, 6 stages of 32 KB (4 in the final apply). Both
+//               CTAs' loads complete on the leader CTA's stage barrier; there
+//               is no multicast. A diagonal Gram tile loads only A.
 //   warp 1      TMEM allocation in both CTAs (cta_group::2, 2 x 256 fp32
 //               columns). In the leader only, MMA issue:
 //               tcgen05.mma.cta_group::2.kind::f16, M = 256 (128 rows in each
@@ -32,10 +34,16 @@
 //               warps, each taking half of the 256 columns, 32 at a time.
 // Per unit of tile work, the pair moves (256 + 256) x 64 x 2 bytes from L2 for
 // 256 x 256 x 64 multiply-adds: one third fewer bytes per flop than a
-// single-CTA 128 x 256 tile.
+// single-CTA 128 x 256 tile. Units with m <= 128 would fill half of that tile;
+// they run on a single-CTA instance of the same template (cta_group::1,
+// 128 x 256 tiles, 128 x 128 for the Gram).
 // B operand major-ness: for GRAM and GRAMSQ both operands are K-major rows of
 // the same matrix. For APPLY the B operand is X itself, read MN-major (the
 // contraction runs over X's rows), so no transposed copy is ever made.
+// Tile order and L2: the applies walk each unit's tiles column by column, so
+// the pairs running at the same time share a few column strips of X and all
+// of the m x m Gram, which they load with an evict-last L2 policy; every
+// bulk tensor store is evict-first (only the next launch reads it).
 #include <climits>
 #include <cstring>
 
