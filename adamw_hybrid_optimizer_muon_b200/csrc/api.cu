@@ -279,6 +279,17 @@ int muon_prep(const MuonJob& j, cudaStream_t s, int* launches) {
     return MA_OK;
 }
 
+// Algorithmic DRAM bytes of one Newton-Schulz launch: each operand read once
+// and each result written once (esz bytes per element: 2 for bf16, 4 in fp32
+// mode). The final apply also reads and writes the fp32 weights.
+double ns_bytes(int mode, int64_t units, int64_t m, int64_t n, int esz) {
+    const double u = (double)units, M = (double)m, N = (double)n, e = (double)esz;
+    if (mode == NS_GRAM) return u * e * (M * N + M * M);
+    if (mode == NS_GRAMSQ) return u * e * 2.0 * M * M;
+    if (mode == NS_APPLY) return u * e * (M * M + 2.0 * M * N);
+    return u * (e * (M * M + M * N) + 8.0 * M * N);
+}
+
 // All checks passed; launch the whole Muon chain for a set of jobs that are
 // pairwise ns_compatible (or a single job). Each Newton-Schulz step is one
 // launch over every job's tiles on the tensor-core path; per job in fp32 mode.
@@ -332,11 +343,13 @@ int run_muon_jobs(const MuonJob* jobs_in, int njobs_in, cudaStream_t s, int sms,
     std::vector<NsJobIn> in(nj);
     auto launch = [&](int mode, const std::vector<void*>& xb, const std::vector<void*>& gb) -> int {
         const int pr = prof_begin(ns_prof_class(mode), s);
-        double flops = 0.0;
+        double flops = 0.0, bytes = 0.0;
         cudaError_t e = cudaSuccess;
         for (int i = 0; i < nj; ++i) {
             in[i] = {&p[i], xb[i], gb[i]};
-            flops += ns_flops(mode, jobs[i]->g.units, jobs[i]->g.m, jobs[i]->g.n);
+            const MuonGeom& g = jobs[i]->g;
+            flops += ns_flops(mode, g.units, g.m, g.n);
+            bytes += ns_bytes(mode, g.units, g.m, g.n, g.esz);
         }
         if (hp0.precision) {
             for (int i = 0; i < nj && e == cudaSuccess; ++i) {
@@ -346,7 +359,7 @@ int run_muon_jobs(const MuonJob* jobs_in, int njobs_in, cudaStream_t s, int sms,
         } else {
             e = launch_ns_tc_group(mode, in.data(), nj, sms, s, launches);
         }
-        prof_end(pr, s, flops, 0.0);
+        prof_end(pr, s, flops, bytes);
         return cuda_status(e);
     };
 

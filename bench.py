@@ -42,9 +42,11 @@ import synth  # noqa: E402
 METRIC = "MuonAdamW step ms & params/s; NS TFLOP/s vs bf16 peak; AdamW GB/s vs HBM"
 UNIT = "params/s"
 
-# ncu DRAM traffic per launch of the dominant kernel, from the capture summarised
-# under profiles/ (None until a capture of the current kernel exists).
-NS_TRAFFIC_BYTES_PER_LAUNCH = None
+# ncu DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per
+# Newton-Schulz launch, averaged over the 60 ns_tc_kernel launches of two 7B
+# steps in one capture of the current kernel (profiles/launches_7b_step.md).
+# Workloads without a capture report None.
+NS_TRAFFIC_BYTES_PER_LAUNCH = {"7b": 20.25e9}
 
 
 def env_int(name, default):
@@ -140,9 +142,10 @@ def blas_threads():
     return os.cpu_count()
 
 
-def oracle_sample(wl):
-    """A bounded slice of the workload for the oracle: one Muon matrix of the most
-    common shape plus AdamW elements in the workload's AdamW:Muon proportion."""
+def oracle_sample(wl, n_matrices=1):
+    """A bounded slice of the workload for the oracle: n_matrices Muon matrices of
+    the most common shape plus AdamW elements in the workload's AdamW:Muon
+    proportion."""
     import oracle
     kinds = oracle.partition([(t.shape, t.role) for t in wl.tensors])
     muon = [i for i, k in enumerate(kinds) if k == 0]
@@ -150,19 +153,19 @@ def oracle_sample(wl):
     shapes = {}
     for i in muon:
         shapes.setdefault(wl.tensors[i].shape, []).append(i)
-    mi = max(shapes.values(), key=len)[0] if muon else None
+    mis = max(shapes.values(), key=len)[:n_matrices] if muon else []
     n_muon = sum(wl.tensors[i].numel for i in muon)
     n_adamw = sum(wl.tensors[i].numel for i in adamw)
-    mat = wl.tensors[mi].numel if mi is not None else 0
+    mat = sum(wl.tensors[i].numel for i in mis)
     k_adamw = int(round(n_adamw * mat / n_muon)) if n_muon else min(n_adamw, 4_000_000)
-    return mi, adamw, k_adamw
+    return mis, adamw, k_adamw
 
 
-def time_oracle_step(wl, mi, adamw, k_adamw, step=2):
+def time_oracle_step(wl, mis, adamw, k_adamw, step=2):
     import oracle
     elapsed = 0.0
     params = 0
-    if mi is not None:
+    for mi in mis:
         spec = wl.tensors[mi]
         g = wl.groups[spec.group].muon
         W = synth.initial_weight(spec, mi)
@@ -191,11 +194,11 @@ def time_oracle_step(wl, mi, adamw, k_adamw, step=2):
     return params, elapsed
 
 
-def cpu_baseline(wl):
-    mi, adamw, k = oracle_sample(wl)
-    params, secs = time_oracle_step(wl, mi, adamw, k)
-    desc = (f"oracle fp64 on 1 Muon matrix {wl.tensors[mi].shape} + {k} AdamW elements "
-            f"({params} params, {secs:.1f} s)") if mi is not None else f"oracle fp64 on {params} AdamW elements"
+def cpu_baseline(wl, n_matrices=4):
+    mis, adamw, k = oracle_sample(wl, n_matrices)
+    params, secs = time_oracle_step(wl, mis, adamw, k)
+    desc = (f"oracle fp64 on {len(mis)} Muon matrices {wl.tensors[mis[0]].shape} + {k} AdamW elements "
+            f"({params} params, {secs:.1f} s)") if mis else f"oracle fp64 on {params} AdamW elements"
     return {"value": params / secs, "unit": UNIT, "cores": blas_threads(), "kind": "oracle", "sample": desc}
 
 
@@ -205,16 +208,17 @@ def run_reference(args, rank, world):
     if rank != 0:
         return 0
     wl = synth.WORKLOADS[args.workload]()
-    mi, adamw, k = oracle_sample(wl)
+    mis, adamw, k = oracle_sample(wl)
     for _ in range(args.warmup):
-        time_oracle_step(wl, mi, adamw, k)
+        time_oracle_step(wl, mis, adamw, k)
     tot_params, tot_s = 0, 0.0
     for _ in range(args.steps):
-        p, s = time_oracle_step(wl, mi, adamw, k)
+        p, s = time_oracle_step(wl, mis, adamw, k)
         tot_params += p
         tot_s += s
     value = tot_params / tot_s
-    sample = f"per step: oracle fp64 on 1 Muon matrix {wl.tensors[mi].shape} + {k} AdamW elements"
+    sample = (f"per step: oracle fp64 on 1 Muon matrix {wl.tensors[mis[0]].shape} + {k} AdamW elements"
+              if mis else f"per step: oracle fp64 on {k} AdamW elements")
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 * tot_s / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
@@ -365,6 +369,7 @@ def main():
         ns_cls = ("ns_gram", "ns_apply", "ns_gramsq", "ns_final")
         ns_ms = sum(prof[c]["ms"] for c in ns_cls)
         ns_fl = sum(prof[c]["flops"] for c in ns_cls)
+        ns_bytes = sum(prof[c]["bytes"] for c in ns_cls)
         ns_launches = sum(prof[c]["launches"] for c in ns_cls)
         ns_tflops = ns_fl / (ns_ms / 1000.0) / 1e12 if ns_ms > 0 else None
         # The sustained (power-capped) GEMM peak applies when the power cap held
@@ -376,7 +381,8 @@ def main():
                     "achieved": ns_tflops, "peak": peak_t, "unit": "TFLOP/s",
                     "frac": ns_tflops / peak_t if ns_tflops else None,
                     "peak_kind": f"bf16 dense, {'sustained' if capped else 'burst'} ({peaks['source']})",
-                    "traffic": NS_TRAFFIC_BYTES_PER_LAUNCH,
+                    "traffic": NS_TRAFFIC_BYTES_PER_LAUNCH.get(args.workload),
+                    "traffic_algorithmic": ns_bytes / max(1, ns_launches),
                     "launches": ns_launches, "avg_launch_ms": ns_ms / max(1, ns_launches),
                     "flops_per_launch": ns_fl / max(1, ns_launches)}
         kernels = {}
@@ -387,7 +393,9 @@ def main():
             d = {"ms_per_step": pc["ms"] / args.steps, "launches_per_step": pc["launches"] / args.steps}
             if pc["flops"] > 0:
                 d["tflops"] = pc["flops"] / (pc["ms"] / 1000.0) / 1e12
-            if pc["bytes"] > 0:
+            if pc["bytes"] > 0 and pc["flops"] > 0:
+                d["algorithmic_gbs"] = pc["bytes"] / (pc["ms"] / 1000.0) / 1e9  # tensor-bound: context only
+            elif pc["bytes"] > 0:
                 d["gbs"] = pc["bytes"] / (pc["ms"] / 1000.0) / 1e9
                 d["frac_hbm"] = d["gbs"] / peaks["hbm_gbs"]
             kernels[c] = d

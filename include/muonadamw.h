@@ -285,7 +285,9 @@ int ma_profile_enable(int on);
  * Newton-Schulz classes (symmetric Gram counted as m(m+1)n, apply as 2m^2n,
  * per unit), DRAM bytes for the memory-bound classes (AdamW 26 B/element with
  * bf16 gradients and 28 with fp32; momentum pass 12 / 14 B/element, +2 when X
- * is fp32). Clears the record. */
+ * is fp32), and for the Newton-Schulz classes the bytes of reading each
+ * operand and writing each result once (the final apply adds 8 B per weight).
+ * Clears the record. */
 int ma_profile_collect(double* ms_out, int64_t* launches_out, double* flops_out, double* bytes_out);
 
 /* ---------------------------------------------------------------- status */
