@@ -84,7 +84,7 @@ constexpr size_t kAlign = 256;
 // Muon sub-batch sizes when gradients stream in from the host: the first
 // sub-batch is small so that compute starts after a short copy, the others
 // large enough to keep every GEMM launch many waves deep.
-constexpr int kFromHostFirstBatch = 8;
+constexpr int kFromHostFirstBatch = 2;
 constexpr int kFromHostBatch = 32;
 // Workspace that a plan may use, beyond its largest sub-batch, to run small
 // Muon buckets through shared Newton-Schulz launches.
@@ -610,8 +610,11 @@ size_t part_ws(const ma_plan* plan, const ma_group_t* groups, const Part& pt) {
     return g.total;
 }
 
-// Segments in launch order. first_cap / cap bound the Muon sub-batch sizes
-// (0 = the plan's own sub-batch size); AdamW goes first or last. With
+// Segments in launch order. cap bounds the Muon sub-batch sizes (0 = the
+// plan's own sub-batch size); with first_cap > 0 the first sub-batch holds at
+// most first_cap matrices and each later one at most twice the one before,
+// up to cap, so that the first copy of a host-gradient step is short. AdamW
+// goes first or last. With
 // group_limit > 0, consecutive sub-batches whose Newton-Schulz chains take
 // the same kernels are merged into one segment while their summed workspace
 // stays within group_limit and the launch tables have room (jobs, weights).
@@ -619,7 +622,7 @@ std::vector<Segment> step_segments(const ma_plan* plan, const ma_group_t* groups
                                    bool adamw_last, size_t group_limit) {
     std::vector<Segment> segs;
     if (!adamw_last && !plan->adamw_idx.empty()) segs.push_back({1, {}});
-    bool first = true;
+    int ramp = first_cap;  // 0 once the ramp has reached cap
     size_t seg_ws = 0;
     int seg_w = 0;
     for (int bi = 0; bi < (int)plan->buckets.size(); ++bi) {
@@ -628,7 +631,7 @@ std::vector<Segment> step_segments(const ma_plan* plan, const ma_group_t* groups
         for (int s0 = 0; s0 < nb;) {
             int lim = b.sub;
             if (cap > 0) lim = std::min(lim, cap);
-            if (first && first_cap > 0) lim = std::min(lim, first_cap);
+            if (ramp > 0) lim = std::min(lim, ramp);
             const int cnt = std::min(lim, nb - s0);
             const Part pt{bi, s0, cnt};
             const size_t ws = part_ws(plan, groups, pt);
@@ -651,7 +654,7 @@ std::vector<Segment> step_segments(const ma_plan* plan, const ma_group_t* groups
                 seg_w = nw;
             }
             s0 += cnt;
-            first = false;
+            if (ramp > 0) ramp = (cap > 0 && 2 * ramp >= cap) || ramp >= (1 << 20) ? 0 : 2 * ramp;
         }
     }
     if (adamw_last && !plan->adamw_idx.empty()) segs.push_back({1, {}});
