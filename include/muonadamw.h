@@ -230,7 +230,11 @@ int adamw_step_fused(int n, float* const* P, const void* const* G, int gdt, floa
  * partition, same-shape Muon buckets (first-appearance order), batching and
  * workspace sizing. t, groups: host arrays, copied. *ws_bytes: in = largest
  * workspace the caller will provide (0 = no limit), out = the bytes that
- * muonadamw_step needs (Muon buckets are split into sub-batches to fit). */
+ * muonadamw_step needs (Muon buckets are split into sub-batches to fit).
+ * Consecutive sub-batches whose Newton-Schulz chains take the same kernels
+ * (tensor-core path, same iteration count, same iterations with c != 0) share
+ * launches when their summed workspace fits: within the cap when one is given,
+ * else within the larger of the biggest sub-batch and 4 GiB. */
 int ma_plan_create(const ma_tensor_t* t, int n, const ma_group_t* groups, int ngroups,
                    ma_plan_t** out, size_t* ws_bytes);
 
