@@ -16,7 +16,7 @@ __all__ = [
     "LibraryMissing", "MAError", "lib", "MuonHParams", "AdamWHParams", "Group", "Tensor",
     "MA_OK", "MA_F32", "MA_BF16", "MA_MUON", "MA_ADAMW", "ROLE_HIDDEN", "ROLE_EMBED", "ROLE_UNEMBED",
     "ROLE_FORCE_ADAMW", "ma_partition", "ma_assign_owners", "muon_workspace_bytes", "muon_step_batched",
-    "ns_iterate_workspace_bytes", "ns_iterate_bf16", "adamw_step_fused", "ma_plan_create", "muonadamw_step",
+    "ns_iterate_workspace_bytes", "ns_iterate_bf16", "adamw_step_fused", "ma_plan_create", "muonadamw_step", "muonadamw_step_graph",
     "ma_plan_destroy", "ma_device_status", "ma_set_wait_limit_ns", "ma_selftest_wait_timeout", "Plan",
     "MuonAdamW", "muon_hparams", "adamw_hparams", "ma_profile_enable", "ma_profile_collect", "PROF_CLASSES",
     "muon_step_batched_noalloc", "STATIC_SCRATCH_BYTES", "muonadamw_step_from_host",
@@ -105,6 +105,8 @@ def lib() -> ctypes.CDLL:
         "muonadamw_step": (i32, [vp, ctypes.POINTER(Group), vp, sz, vp]),
         "muonadamw_step_from_host": (i32, [vp, ctypes.POINTER(Group), pp, vp, sz, vp, vp]),
         "ma_plan_last_launches": (i32, [vp]),
+        "muonadamw_step_graph": (i32, [vp, ctypes.POINTER(Group), vp, sz, vp]),
+        "ma_plan_graph_captures": (i32, [vp]),
         "ma_plan_destroy": (None, [vp]),
         "ma_device_status": (i32, [vp, i32]),
         "ma_set_wait_limit_ns": (i32, [i64]),
@@ -298,6 +300,12 @@ def muonadamw_step(plan, groups: Sequence[Group], ws, ws_bytes: int, stream=None
     _check(lib().muonadamw_step(plan, garr, _ptr(ws), int(ws_bytes), _stream(stream)), "muonadamw_step")
 
 
+def muonadamw_step_graph(plan, groups: Sequence[Group], ws, ws_bytes: int, stream=None) -> None:
+    """muonadamw_step replayed from a CUDA graph the plan captures and keeps."""
+    garr = (Group * max(1, len(groups)))(*groups)
+    _check(lib().muonadamw_step_graph(plan, garr, _ptr(ws), int(ws_bytes), _stream(stream)), "muonadamw_step_graph")
+
+
 def muonadamw_step_from_host(plan, groups: Sequence[Group], host_grads, ws, ws_bytes: int, stream=None,
                              copy_stream=None) -> None:
     """One step whose gradients are copied from host memory (pinned tensors or host pointers) on copy_stream,
@@ -353,8 +361,9 @@ class Plan:
         self.handle, self.ws_bytes = ma_plan_create(self.tensors, self.groups, ws_cap)
         self.ws = torch.empty(max(self.ws_bytes, 256), dtype=torch.uint8, device=device or "cuda")
 
-    def step(self, groups: Sequence[Group] | None = None, stream=None) -> None:
-        muonadamw_step(self.handle, groups if groups is not None else self.groups, self.ws, self.ws.numel(), stream)
+    def step(self, groups: Sequence[Group] | None = None, stream=None, graph: bool = False) -> None:
+        fn = muonadamw_step_graph if graph else muonadamw_step
+        fn(self.handle, groups if groups is not None else self.groups, self.ws, self.ws.numel(), stream)
 
     def step_from_host(self, host_grads, groups: Sequence[Group] | None = None, stream=None,
                        copy_stream=None) -> None:
@@ -364,6 +373,10 @@ class Plan:
     @property
     def launches(self) -> int:
         return int(lib().ma_plan_last_launches(self.handle))
+
+    @property
+    def graph_captures(self) -> int:
+        return int(lib().ma_plan_graph_captures(self.handle))
 
     def close(self) -> None:
         if self.handle is not None and self.handle.value:
@@ -443,12 +456,16 @@ class MuonAdamW:
             if g.kind == MA_ADAMW:
                 g.adamw.step = self.step_count
 
-    def step(self, grads=None, stream=None) -> None:
+    def step(self, grads=None, stream=None, graph: bool = False) -> None:
+        """One step. graph=True replays the step from a CUDA graph that the plan
+        captures on first use (same results; one launch instead of one per kernel).
+        A plan, and with it the graph, belongs to one set of gradient buffers:
+        keep them at fixed addresses (as persistent ``.grad`` tensors are)."""
         if grads is None:
             grads = [p.grad for p, _, _ in self.entries]
         self._ensure_plan(grads)
         self._advance()
-        self._plan.step(self.groups, stream)
+        self._plan.step(self.groups, stream, graph)
 
     def step_from_host(self, host_grads, device_grads, stream=None, copy_stream=None) -> None:
         """One step whose gradients arrive from host memory.
@@ -471,3 +488,8 @@ class MuonAdamW:
     @property
     def launches(self) -> int:
         return self._plan.launches if self._plan is not None else 0
+
+    @property
+    def graph_captures(self) -> int:
+        """How many times the plan captured its CUDA graph (graph steps only)."""
+        return self._plan.graph_captures if self._plan is not None else 0

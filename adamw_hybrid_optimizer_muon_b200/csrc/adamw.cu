@@ -92,6 +92,8 @@ __global__ void __launch_bounds__(256) adamw_kernel(const __grid_constant__ Adam
 
 }  // namespace
 
+const void* adamw_kernel_func() { return reinterpret_cast<const void*>(adamw_kernel); }
+
 cudaError_t launch_adamw(const AdamwLaunch& L, cudaStream_t s) {
     if (L.nchunks <= 0 || L.ntensors <= 0) return cudaSuccess;
     adamw_kernel<<<dim3((unsigned)L.nchunks), dim3(256), 0, s>>>(L);

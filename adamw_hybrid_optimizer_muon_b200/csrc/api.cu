@@ -17,6 +17,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <new>
+#include <unordered_map>
 #include <vector>
 
 #include "common.cuh"
@@ -551,8 +552,36 @@ struct ma_plan {
     size_t ws_bytes = 0;
     int last_launches = 0;
     std::vector<cudaEvent_t> events;  // segment-ready events of muonadamw_step_from_host
+    // muonadamw_step_graph: the captured step and the kernel nodes whose
+    // parameters follow the per-step hyperparameters
+    struct GraphNode {
+        cudaGraphNode_t node;
+        cudaKernelNodeParams params;  // func, launch shape; kernelParams replaced on update
+        std::vector<uint8_t> arg;     // the kernel's single by-value parameter
+        int final_apply;              // 0: AdamW launch, 1: Newton-Schulz final apply
+    };
+    struct Graph {
+        cudaGraph_t graph = nullptr;
+        cudaGraphExec_t exec = nullptr;
+        cudaStream_t capture = nullptr;
+        int capture_dev = -1;  // device of `capture`
+        std::vector<uint8_t> key;
+        std::vector<GraphNode> nodes;
+        int launches = 0;
+        int captures = 0;
+        void release() {
+            if (exec) cudaGraphExecDestroy(exec);
+            if (graph) cudaGraphDestroy(graph);
+            exec = nullptr;
+            graph = nullptr;
+            nodes.clear();
+            key.clear();
+        }
+    } g;
     ~ma_plan() {
         for (cudaEvent_t e : events) cudaEventDestroy(e);
+        g.release();
+        if (g.capture) cudaStreamDestroy(g.capture);
     }
 };
 
@@ -1041,6 +1070,181 @@ int muonadamw_step(ma_plan_t* plan, const ma_group_t* groups, void* ws, size_t w
     return MA_OK;
 }
 
+}  // extern "C"
+
+namespace ma {
+namespace {
+
+// What a captured step depends on beyond the per-step values that are patched
+// into its nodes (AdamW hyperparameters and step, Muon lr and weight decay on
+// the tensor-core path): the workspace, the device and the rest of every Muon
+// group's hyperparameters.
+std::vector<uint8_t> graph_key(const ma_plan* plan, const ma_group_t* groups, const void* ws, int dev) {
+    std::vector<uint8_t> k;
+    auto put = [&k](const void* p, size_t n) {
+        const uint8_t* b = reinterpret_cast<const uint8_t*>(p);
+        k.insert(k.end(), b, b + n);
+    };
+    put(&ws, sizeof(ws));
+    put(&dev, sizeof(dev));
+    for (size_t i = 0; i < plan->group_kind.size(); ++i) {
+        put(&groups[i].kind, sizeof(groups[i].kind));
+        if (groups[i].kind != MA_MUON) continue;
+        const ma_muon_hparams_t& h = groups[i].muon;
+        const float lr = h.precision ? h.lr : 0.f, wd = h.precision ? h.weight_decay : 0.f;
+        put(&lr, sizeof(lr));
+        put(&wd, sizeof(wd));
+        put(&h.beta, sizeof(h.beta));
+        put(&h.eps, sizeof(h.eps));
+        put(&h.nesterov, sizeof(h.nesterov));
+        put(&h.ns_steps, sizeof(h.ns_steps));
+        put(&h.n_coeffs, sizeof(h.n_coeffs));
+        for (int c = 0; c < h.n_coeffs && c < MA_MAX_NS_STEPS; ++c) put(h.coeffs[c], 3 * sizeof(float));
+        put(&h.scale_mode, sizeof(h.scale_mode));
+        put(&h.heads, sizeof(h.heads));
+        put(&h.precision, sizeof(h.precision));
+        put(&h.cautious, sizeof(h.cautious));
+    }
+    return k;
+}
+
+struct FinalPatchCtx {
+    const ma_plan* plan;
+    const ma_group_t* groups;
+    std::unordered_map<const float*, int> tensor_of;  // Muon weight -> table index
+};
+
+// The decay terms of one final-apply job, as run_muon_jobs computes them.
+int patch_final_job(void* ctx, const float* W, int64_t Rh, int64_t C, float* decay, float* lr_s, float* lr_wd) {
+    const FinalPatchCtx& c = *reinterpret_cast<const FinalPatchCtx*>(ctx);
+    const auto it = c.tensor_of.find(W);
+    if (it == c.tensor_of.end()) return MA_ERR_ARG;
+    const ma_muon_hparams_t& hp = c.groups[c.plan->t[it->second].group].muon;
+    *decay = 1.f - hp.lr * hp.weight_decay;
+    *lr_s = hp.lr * shape_scale(Rh, C, hp.scale_mode);
+    *lr_wd = hp.lr * hp.weight_decay;
+    return MA_OK;
+}
+
+// Write this step's hyperparameters into the captured AdamW and final-apply nodes.
+int graph_patch(ma_plan* plan, const ma_group_t* groups) {
+    const int ngroups = (int)plan->group_kind.size();
+    AdamwGroupConst gc[MA_MAX_GROUPS];
+    std::memset(gc, 0, sizeof(gc));
+    for (int k = 0; k < ngroups; ++k)
+        if (groups[k].kind == MA_ADAMW) gc[k] = adamw_const(groups[k].adamw);
+    FinalPatchCtx ctx{plan, groups, {}};
+    for (size_t i = 0; i < plan->t.size(); ++i)
+        if (plan->kind[i] == MA_MUON) ctx.tensor_of[plan->t[i].param] = (int)i;
+    for (ma_plan::GraphNode& n : plan->g.nodes) {
+        if (n.final_apply) {
+            const int st = ns_tc_patch_final(n.arg.data(), patch_final_job, &ctx);
+            if (st) return st;
+        } else {
+            AdamwLaunch* L = reinterpret_cast<AdamwLaunch*>(n.arg.data());
+            for (int k = 0; k < ngroups; ++k) L->grp[k] = gc[k];
+        }
+        cudaKernelNodeParams p = n.params;
+        void* args[1] = {n.arg.data()};
+        p.kernelParams = args;
+        p.extra = nullptr;
+        if (cudaGraphExecKernelNodeSetParams(plan->g.exec, n.node, &p) != cudaSuccess) return MA_ERR_CUDA;
+    }
+    return MA_OK;
+}
+
+// Capture one whole step on the plan's own stream and instantiate it.
+int graph_capture(ma_plan* plan, const ma_group_t* groups, void* ws, int sms, int dev) {
+    ma_plan::Graph& G = plan->g;
+    G.release();
+    if (G.capture && G.capture_dev != dev) {
+        int cur = dev;
+        cudaSetDevice(G.capture_dev);
+        cudaStreamDestroy(G.capture);
+        cudaSetDevice(cur);
+        G.capture = nullptr;
+    }
+    if (!G.capture) {
+        if (cudaStreamCreateWithFlags(&G.capture, cudaStreamNonBlocking) != cudaSuccess) return MA_ERR_CUDA;
+        G.capture_dev = dev;
+    }
+    // everything that must not happen inside a capture: attribute set-up,
+    // driver entry points, the status-word address
+    if (ns_tc_setup(sms) != cudaSuccess || !device_status_ptr()) return MA_ERR_CUDA;
+    const bool prof = g_prof_on;
+    g_prof_on = false;
+    if (cudaStreamBeginCapture(G.capture, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
+        g_prof_on = prof;
+        return MA_ERR_CUDA;
+    }
+    int launches = 0, st = MA_OK;
+    for (const Segment& sg : step_segments(plan, groups, 0, 0, false, plan->ws_bytes))
+        if ((st = launch_segment(plan, groups, sg, ws, G.capture, sms, &launches))) break;
+    cudaGraph_t graph = nullptr;
+    const cudaError_t ec = cudaStreamEndCapture(G.capture, &graph);
+    g_prof_on = prof;
+    if (st || ec != cudaSuccess) {
+        if (graph) cudaGraphDestroy(graph);
+        return st ? st : MA_ERR_CUDA;
+    }
+    G.graph = graph;
+    if (cudaGraphInstantiate(&G.exec, graph, 0) != cudaSuccess) {
+        G.release();
+        return MA_ERR_CUDA;
+    }
+    size_t n = 0;
+    if (cudaGraphGetNodes(graph, nullptr, &n) != cudaSuccess) {
+        G.release();
+        return MA_ERR_CUDA;
+    }
+    std::vector<cudaGraphNode_t> nodes(n);
+    if (n > 0 && cudaGraphGetNodes(graph, nodes.data(), &n) != cudaSuccess) {
+        G.release();
+        return MA_ERR_CUDA;
+    }
+    for (cudaGraphNode_t node : nodes) {
+        cudaGraphNodeType type;
+        if (cudaGraphNodeGetType(node, &type) != cudaSuccess || type != cudaGraphNodeTypeKernel) continue;
+        cudaKernelNodeParams p;
+        if (cudaGraphKernelNodeGetParams(node, &p) != cudaSuccess) {
+            G.release();
+            return MA_ERR_CUDA;
+        }
+        const bool adamw = p.func == adamw_kernel_func();
+        const bool fin = ns_tc_is_final(p.func);
+        if (!adamw && !fin) continue;
+        const size_t bytes = adamw ? sizeof(AdamwLaunch) : ns_tc_launch_bytes();
+        const uint8_t* a = reinterpret_cast<const uint8_t*>(p.kernelParams[0]);
+        G.nodes.push_back({node, p, std::vector<uint8_t>(a, a + bytes), fin ? 1 : 0});
+    }
+    G.launches = launches;
+    ++G.captures;
+    return MA_OK;
+}
+
+}  // namespace
+}  // namespace ma
+
+extern "C" {
+
+int muonadamw_step_graph(ma_plan_t* plan, const ma_group_t* groups, void* ws, size_t ws_bytes, void* stream) {
+    int sms = 0;
+    int st = check_step(plan, groups, ws, ws_bytes, &sms);
+    if (st) return st;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MA_ERR_CUDA;
+    std::vector<uint8_t> key = graph_key(plan, groups, ws, dev);
+    if (!plan->g.exec || key != plan->g.key) {
+        if ((st = graph_capture(plan, groups, ws, sms, dev))) return st;
+        plan->g.key = std::move(key);
+    } else if ((st = graph_patch(plan, groups))) {
+        return st;
+    }
+    if (cudaGraphLaunch(plan->g.exec, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return MA_ERR_CUDA;
+    plan->last_launches = plan->g.launches;
+    return MA_OK;
+}
+
 int muonadamw_step_from_host(ma_plan_t* plan, const ma_group_t* groups, const void* const* host_grads, void* ws,
                              size_t ws_bytes, void* stream, void* copy_stream) {
     int sms = 0;
@@ -1095,6 +1299,8 @@ int muonadamw_step_from_host(ma_plan_t* plan, const ma_group_t* groups, const vo
 }
 
 int ma_plan_last_launches(const ma_plan_t* plan) { return plan ? plan->last_launches : 0; }
+
+int ma_plan_graph_captures(const ma_plan_t* plan) { return plan ? plan->g.captures : 0; }
 
 void ma_plan_destroy(ma_plan_t* plan) { delete plan; }
 

@@ -45,6 +45,7 @@ struct AdamwLaunch {
 };
 
 cudaError_t launch_adamw(const AdamwLaunch& L, cudaStream_t s);
+const void* adamw_kernel_func();  // the kernel's host-side handle (CUDA-graph node matching)
 
 // ------------------------------------------------------------------ Muon: momentum + norm
 
@@ -115,6 +116,17 @@ cudaError_t launch_ns_tc_group(int mode, const NsJobIn* jobs, int njobs, int num
                                int* launched);
 int ns_tc_max_jobs();
 int ns_tc_max_weights();
+// Per-device kernel attributes of every instance, ahead of a stream capture.
+cudaError_t ns_tc_setup(int num_sms);
+// CUDA-graph support: whether a kernel node's function is a final apply, the
+// size of its single (by value) parameter, and an in-place update of the
+// decay terms of each of its jobs. f(ctx, first weight of the job, rows per
+// unit, columns, &decay, &lr_s, &lr_wd) returns nonzero to stop with that code.
+typedef int (*NsFinalPatchFn)(void* ctx, const float* W, int64_t Rh, int64_t C, float* decay, float* lr_s,
+                              float* lr_wd);
+bool ns_tc_is_final(const void* func);
+size_t ns_tc_launch_bytes();
+int ns_tc_patch_final(void* launch, NsFinalPatchFn f, void* ctx);
 
 // fp32 SIMT path (precision mode 1).
 cudaError_t launch_ns_simt(int mode, const NsParams& p, const void* x_buf, const void* g_buf, cudaStream_t s);

@@ -701,6 +701,51 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Once per device and kernel instance: allow its dynamic shared memory and
+// find how many pairs (or CTAs) can be resident at once. Not legal inside a
+// stream capture the first time; ns_tc_setup runs it for every instance.
+template <int MODE, bool PAIR>
+cudaError_t setup_mode(int num_sms, int* max_units_out) {
+    using S = Shape<MODE, PAIR>;
+    static unsigned long long attr_set = 0;  // one bit per device
+    static int max_units[64] = {0};          // resident pairs (or CTAs) per device
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+    if (!(attr_set & (1ull << dev))) {
+        e = cudaFuncSetAttribute(ns_tc_kernel<MODE, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM);
+        if (e != cudaSuccess) return e;
+        if (PAIR) {
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = 2;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cudaLaunchConfig_t qc = {};
+            qc.gridDim = dim3(2 * (unsigned)(num_sms / 2));
+            qc.blockDim = dim3(THREADS);
+            qc.dynamicSmemBytes = S::SMEM;
+            qc.attrs = attr;
+            qc.numAttrs = 1;
+            int nclusters = 0;
+            e = cudaOccupancyMaxActiveClusters(&nclusters, ns_tc_kernel<MODE, PAIR>, &qc);
+            if (e != cudaSuccess) return e;
+            if (nclusters < 1) return cudaErrorInvalidConfiguration;
+            max_units[dev] = nclusters;
+        } else {
+            int per_sm = 0;
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ns_tc_kernel<MODE, PAIR>, THREADS, S::SMEM);
+            if (e != cudaSuccess) return e;
+            if (per_sm < 1) return cudaErrorInvalidConfiguration;
+            max_units[dev] = per_sm * num_sms;
+        }
+        attr_set |= 1ull << dev;
+    }
+    *max_units_out = max_units[dev];
+    return cudaSuccess;
+}
+
 template <int MODE, bool PAIR>
 cudaError_t launch_mode(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_t s) {
     using S = Shape<MODE, PAIR>;
@@ -763,42 +808,15 @@ cudaError_t launch_mode(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_
     L.wait_limit_ns = jobs[0].p->wait_limit_ns;
     L.status = jobs[0].p->status;
     if (tile0 <= 0) return cudaSuccess;
-    static unsigned long long attr_set = 0;  // one bit per device
-    static int max_units[64] = {0};          // resident pairs (or CTAs) per device
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
+    int max_units = 0;
+    cudaError_t e = setup_mode<MODE, PAIR>(num_sms, &max_units);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 2;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
-    if (!(attr_set & (1ull << dev))) {
-        e = cudaFuncSetAttribute(ns_tc_kernel<MODE, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM);
-        if (e != cudaSuccess) return e;
-        if (PAIR) {
-            cudaLaunchConfig_t qc = {};
-            qc.gridDim = dim3(2 * (unsigned)(num_sms / 2));
-            qc.blockDim = dim3(THREADS);
-            qc.dynamicSmemBytes = S::SMEM;
-            qc.attrs = attr;
-            qc.numAttrs = 1;
-            int nclusters = 0;
-            e = cudaOccupancyMaxActiveClusters(&nclusters, ns_tc_kernel<MODE, PAIR>, &qc);
-            if (e != cudaSuccess) return e;
-            if (nclusters < 1) return cudaErrorInvalidConfiguration;
-            max_units[dev] = nclusters;
-        } else {
-            int per_sm = 0;
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ns_tc_kernel<MODE, PAIR>, THREADS, S::SMEM);
-            if (e != cudaSuccess) return e;
-            if (per_sm < 1) return cudaErrorInvalidConfiguration;
-            max_units[dev] = per_sm * num_sms;
-        }
-        attr_set |= 1ull << dev;
-    }
-    const long long units = tile0 < max_units[dev] ? tile0 : max_units[dev];
+    const long long units = tile0 < max_units ? tile0 : max_units;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((PAIR ? 2 : 1) * units));
     cfg.blockDim = dim3(THREADS);
@@ -839,6 +857,35 @@ cudaError_t launch_split(const NsJobIn* jobs, int njobs, int num_sms, cudaStream
 }  // namespace
 
 size_t ns_tc_smem_bytes() { return SMEM_BYTES; }
+
+cudaError_t ns_tc_setup(int num_sms) {
+    if (!encode_fn()) return cudaErrorNotSupported;
+    int u = 0;
+    cudaError_t e;
+#define MA_SETUP(M, P) \
+    if ((e = setup_mode<M, P>(num_sms, &u)) != cudaSuccess) return e;
+    MA_SETUP(NS_GRAM, true) MA_SETUP(NS_GRAM, false) MA_SETUP(NS_GRAMSQ, true) MA_SETUP(NS_GRAMSQ, false)
+    MA_SETUP(NS_APPLY, true) MA_SETUP(NS_APPLY, false) MA_SETUP(NS_FINAL, true) MA_SETUP(NS_FINAL, false)
+#undef MA_SETUP
+    return cudaSuccess;
+}
+
+bool ns_tc_is_final(const void* func) {
+    return func == reinterpret_cast<const void*>(ns_tc_kernel<NS_FINAL, true>) ||
+           func == reinterpret_cast<const void*>(ns_tc_kernel<NS_FINAL, false>);
+}
+
+size_t ns_tc_launch_bytes() { return sizeof(NsLaunch); }
+
+int ns_tc_patch_final(void* launch, NsFinalPatchFn f, void* ctx) {
+    NsLaunch* L = reinterpret_cast<NsLaunch*>(launch);
+    for (int j = 0; j < L->njobs; ++j) {
+        NsJob& J = L->job[j];
+        const int st = f(ctx, L->W[J.w0], J.Rh, J.C, &J.decay, &J.lr_s, &J.lr_wd);
+        if (st) return st;
+    }
+    return 0;
+}
 int ns_tc_max_jobs() { return kMaxJobs; }
 int ns_tc_max_weights() { return kMaxW; }
 

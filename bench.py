@@ -230,14 +230,24 @@ def run_reference(args, rank, world):
     return 0
 
 
+L2_BYTES = 126 << 20
+
+
+def small_inputs(wl):
+    """Whether one step's data (fp32 params and state, bf16 grads) fits in twice the L2."""
+    return wl.numel * 14 < 2 * L2_BYTES
+
+
 def workload_config(wl, n_gpus):
     import oracle
     kinds = oracle.partition([(t.shape, t.role) for t in wl.tensors])
+    l2 = ("inputs smaller than L2: a 512 MB buffer is written between timed steps, outside their events"
+          if small_inputs(wl) else "inputs larger than L2 (no flush needed)")
     return {"workload": f"{wl.name}: {wl.description}", "params": wl.numel,
             "muon_matrices": kinds.count(0), "adamw_tensors": kinds.count(1),
             "ns_steps": wl.groups[0].muon.ns_steps if wl.groups[0].kind == 0 else None,
             "ns_coeffs": [list(c) for c in wl.groups[0].muon.coeffs] if wl.groups[0].kind == 0 else None,
-            "l2": "inputs larger than L2 (no flush needed)", "parallelism": f"replicas x{n_gpus}"}
+            "l2": l2, "parallelism": f"replicas x{n_gpus}"}
 
 
 # ----------------------------------------------------------------------------- our arm
@@ -251,6 +261,9 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--graph", action="store_true",
+                    help="time the step replayed from a CUDA graph (muonadamw_step_graph); the per-kernel "
+                         "profile then comes from an extra, untimed pass of eager steps")
     ap.add_argument("--coeffs", default=None,
                     help="Newton-Schulz polynomial per iteration, 'a,b,c[;a,b,c...]' (default: the cubic 1.5,-0.5,0)")
     args = ap.parse_args()
@@ -296,7 +309,7 @@ def main():
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
-        opt.step(grads)
+        opt.step(grads, graph=args.graph)
     torch.cuda.synchronize(dev)
     st = ma.ma_device_status(stream)
     if st != ma.MA_OK:
@@ -308,18 +321,38 @@ def main():
     time.sleep(0.5)
     barrier()
     torch.cuda.synchronize(dev)
-    ma.ma_profile_enable(True)
-    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    t0.record(stream)
-    for _ in range(args.steps):
-        opt.step(grads)
-    t1.record(stream)
-    torch.cuda.synchronize(dev)
+    ma.ma_profile_enable(not args.graph)
+    if small_inputs(wl):
+        # flush L2 between steps; each step is timed by its own pair of events
+        flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for a, b in evs:
+            flush.zero_()
+            a.record(stream)
+            opt.step(grads, graph=args.graph)
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        step_ms = sum(a.elapsed_time(b) for a, b in evs)
+        del flush
+    else:
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        t0.record(stream)
+        for _ in range(args.steps):
+            opt.step(grads, graph=args.graph)
+        t1.record(stream)
+        torch.cuda.synchronize(dev)
+        step_ms = t0.elapsed_time(t1)
     barrier()
+    clk = clocks.stop()
+    if args.graph:  # graph replays record no per-kernel events: profile eager steps, untimed
+        ma.ma_profile_enable(True)
+        for _ in range(args.steps):
+            opt.step(grads)
+        torch.cuda.synchronize(dev)
     ma.ma_profile_enable(False)
     prof = ma.ma_profile_collect()
-    clk = clocks.stop()
-    ms = t0.elapsed_time(t1) / args.steps
+    ms = step_ms / args.steps
     launches_per_step = opt.launches
     if world > 1:
         tt = torch.tensor([ms], device=dev, dtype=torch.float64)

@@ -261,7 +261,27 @@ int muonadamw_step(ma_plan_t* plan, const ma_group_t* groups, void* ws, size_t w
 int muonadamw_step_from_host(ma_plan_t* plan, const ma_group_t* groups, const void* const* host_grads, void* ws,
                              size_t ws_bytes, void* stream, void* copy_stream);
 
-/* Number of kernel launches the last muonadamw_step or muonadamw_step_from_host issued (for benchmarks). */
+/* The same step as muonadamw_step, replayed from a CUDA graph (the launch
+ * cost of a whole step is one graph launch; for small parameter sets the step
+ * is launch-bound). The first call, and any call whose workspace, device or
+ * Muon hyperparameters other than lr and weight_decay differ from those of the
+ * captured step, captures the step on a stream the plan owns and instantiates
+ * it (host cost of an eager step plus instantiation; nothing runs until the
+ * launch). Every other call writes the new AdamW hyperparameters and step and
+ * the new Muon lr and weight_decay into the captured kernels' parameters and
+ * launches the graph on `stream`. Results are bit-identical to those of
+ * muonadamw_step with the same arguments. In fp32 mode (precision 1) a change
+ * of a Muon lr or weight_decay also re-captures. Must not be called while
+ * `stream` or this thread is capturing. The plan keeps the graph until it is
+ * destroyed. */
+int muonadamw_step_graph(ma_plan_t* plan, const ma_group_t* groups, void* ws, size_t ws_bytes, void* stream);
+
+/* How many times muonadamw_step_graph captured this plan's graph (tests,
+ * benchmarks). 0 for a NULL plan. */
+int ma_plan_graph_captures(const ma_plan_t* plan);
+
+/* Number of kernel launches the last muonadamw_step, muonadamw_step_graph or
+ * muonadamw_step_from_host issued (for a graph step: the kernels in the graph). */
 int ma_plan_last_launches(const ma_plan_t* plan);
 
 void ma_plan_destroy(ma_plan_t* plan);
