@@ -43,10 +43,10 @@ METRIC = "MuonAdamW step ms & params/s; NS TFLOP/s vs bf16 peak; AdamW GB/s vs H
 UNIT = "params/s"
 
 # ncu DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per
-# Newton-Schulz launch, averaged over the 60 ns_tc_kernel launches of two 7B
+# Newton-Schulz launch, averaged over the 200 ns_tc_kernel launches of two 7B
 # steps in one capture of the current kernel (profiles/launches_7b_step.md).
 # Workloads without a capture report None.
-NS_TRAFFIC_BYTES_PER_LAUNCH = {"7b": 20.25e9}
+NS_TRAFFIC_BYTES_PER_LAUNCH = {"7b": 5.771e9}
 
 
 def env_int(name, default):

@@ -178,8 +178,14 @@ def test_plan_sizing_on_host():
         descs.append(d)
     plan, ws = ma.ma_plan_create(descs, _groups_for(wl))
     hp = ma.muon_hparams()
-    expect = max(ma.muon_workspace_bytes(128, 4096, 4096, hp), ma.muon_workspace_bytes(64, 4096, 11008, hp),
-                 ma.muon_workspace_bytes(32, 11008, 4096, hp))
+
+    def sub(n, R, C):  # without a cap, sub-batches are halved to at most 4 GiB of workspace
+        while ma.muon_workspace_bytes(n, R, C, hp) > 4 << 30 and n > 1:
+            n //= 2
+        return n
+    assert (sub(128, 4096, 4096), sub(64, 4096, 11008), sub(32, 11008, 4096)) == (32, 16, 16)
+    expect = max(ma.muon_workspace_bytes(32, 4096, 4096, hp), ma.muon_workspace_bytes(16, 4096, 11008, hp),
+                 ma.muon_workspace_bytes(16, 11008, 4096, hp))
     assert ws == expect
     ma.ma_plan_destroy(plan)
     # a cap splits buckets into sub-batches
