@@ -5,12 +5,16 @@
 // Optimizer", "The MuonAdamW Class Architecture": one step() that dispatches
 // on each group's kind):
 //   1. one multi-tensor AdamW launch over every AdamW tensor (adamw.cu)
-//   2. per Muon bucket of same-shape matrices ("Muon Step Implementation":
-//      stacked batches): momentum + norm (muon_prep.cu), norm finalize, then
-//      the Newton-Schulz chain (ns_tc.cu, or ns_simt.cu in fp32 mode), whose
-//      last GEMM writes the decayed, updated weights.
-// The host never synchronises. Every argument is checked before the first
-// launch, so a failing call changes nothing.
+//   2. per Muon sub-batch of same-shape matrices ("Muon Step Implementation":
+//      stacked batches): momentum + norm (muon_prep.cu) and the norm
+//      finalize, then the Newton-Schulz chain (ns_tc.cu, or ns_simt.cu in
+//      fp32 mode), whose last GEMM writes the decayed, updated weights.
+//      Consecutive sub-batches whose chains take the same kernels share each
+//      Newton-Schulz launch.
+// The plan splits buckets into sub-batches (workspace within the caller's cap,
+// or 4 GiB), groups small ones, and can replay the whole step from a CUDA
+// graph. The host never synchronises. Every argument is checked before the
+// first launch, so a failing call changes nothing.
 #include <algorithm>
 #include <climits>
 #include <cmath>
