@@ -48,6 +48,8 @@ __device__ __forceinline__ float load_g1(const void* g, int gdt, int64_t i) {
 }
 
 __global__ void __launch_bounds__(256) adamw_kernel(const __grid_constant__ AdamwLaunch L) {
+    griddep_launch_dependents();
+    griddep_wait();
     const int64_t chunk = blockIdx.x;
     int lo = 0, hi = L.ntensors - 1;
     while (lo < hi) {  // last tensor whose first chunk is <= this chunk
@@ -96,8 +98,7 @@ const void* adamw_kernel_func() { return reinterpret_cast<const void*>(adamw_ker
 
 cudaError_t launch_adamw(const AdamwLaunch& L, cudaStream_t s) {
     if (L.nchunks <= 0 || L.ntensors <= 0) return cudaSuccess;
-    adamw_kernel<<<dim3((unsigned)L.nchunks), dim3(256), 0, s>>>(L);
-    return cudaGetLastError();
+    return launch_pdl(adamw_kernel, dim3((unsigned)L.nchunks), dim3(256), 0, s, L);
 }
 
 }  // namespace ma

@@ -10,6 +10,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <utility>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -172,6 +173,48 @@ __device__ __forceinline__ void bulk_wait_group0() { asm volatile("cp.async.bulk
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
+}
+
+// ------------------------------------------------------------------ programmatic dependent launch
+//
+// Every kernel of the library is launched with programmatic stream
+// serialisation. A kernel lets the next one be scheduled as soon as it starts
+// (griddep_launch_dependents), and waits for the one before it to complete,
+// with its memory visible, before it touches global memory (griddep_wait).
+// Work before the wait (barrier set-up, TMEM allocation, tensor-map prefetch)
+// overlaps the previous kernel's tail. With a predecessor that was launched
+// without the attribute, the wait returns at once.
+#ifndef MA_PDL
+#define MA_PDL 1
+#endif
+
+__device__ __forceinline__ void griddep_wait() {
+#if MA_PDL
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+#endif
+}
+
+__device__ __forceinline__ void griddep_launch_dependents() {
+#if MA_PDL
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+#endif
+}
+
+// Host: launch `kernel` with programmatic stream serialisation.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute a[1];
+    a[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a[0].val.programmaticStreamSerializationAllowed = MA_PDL;
+    cfg.attrs = a;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
 // ------------------------------------------------------------------ tcgen05

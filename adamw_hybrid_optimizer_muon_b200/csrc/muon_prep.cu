@@ -89,6 +89,8 @@ __device__ __forceinline__ void store_x8(void* X, int64_t i, const float (&d)[8]
 // so each thread keeps 12 independent 16-byte loads in flight.
 template <bool GBF16, bool XF32>
 __global__ void __launch_bounds__(256) prep_flat_kernel(const __grid_constant__ MuonPrepLaunch L) {
+    griddep_launch_dependents();
+    griddep_wait();
     __shared__ float red[8];
     constexpr int kIter = kPrepChunk / (8 * 256);
     const int u = blockIdx.y;
@@ -148,6 +150,8 @@ __global__ void __launch_bounds__(256) prep_flat_kernel(const __grid_constant__ 
 // consecutive values (128 bytes of bf16) written as 16-byte vectors.
 template <bool GBF16, bool XF32>
 __global__ void __launch_bounds__(256) prep_transpose_kernel(const __grid_constant__ MuonPrepLaunch L) {
+    griddep_launch_dependents();
+    griddep_wait();
     __shared__ float tile[kPrepTile][kPrepTile + 1];  // [column of u][row of u]
     __shared__ float red[8];
     const int u = blockIdx.y;
@@ -246,6 +250,8 @@ __global__ void __launch_bounds__(256) prep_transpose_kernel(const __grid_consta
 // butterfly, so the result does not depend on scheduling.
 __global__ void __launch_bounds__(256) norm_finalize_kernel(const double* __restrict__ partials, int64_t parts,
                                                             int units, float eps, float* __restrict__ scale) {
+    griddep_launch_dependents();
+    griddep_wait();
     const int u = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int l = threadIdx.x & 31;
     if (u >= units) return;
@@ -268,25 +274,26 @@ cudaError_t launch_muon_prep(const MuonPrepLaunch& L, cudaStream_t s) {
     if (units == 0 || L.parts == 0) return cudaSuccess;
     dim3 grid((unsigned)L.parts, (unsigned)units);
     const bool gb = L.gdt == MA_BF16, xf = L.x_f32 != 0;
+    cudaError_t e;
     if (L.transposed) {
-        if (gb && !xf) prep_transpose_kernel<true, false><<<grid, 256, 0, s>>>(L);
-        else if (gb) prep_transpose_kernel<true, true><<<grid, 256, 0, s>>>(L);
-        else if (!xf) prep_transpose_kernel<false, false><<<grid, 256, 0, s>>>(L);
-        else prep_transpose_kernel<false, true><<<grid, 256, 0, s>>>(L);
+        if (gb && !xf) e = launch_pdl(prep_transpose_kernel<true, false>, grid, dim3(256), 0, s, L);
+        else if (gb) e = launch_pdl(prep_transpose_kernel<true, true>, grid, dim3(256), 0, s, L);
+        else if (!xf) e = launch_pdl(prep_transpose_kernel<false, false>, grid, dim3(256), 0, s, L);
+        else e = launch_pdl(prep_transpose_kernel<false, true>, grid, dim3(256), 0, s, L);
     } else {
-        if (gb && !xf) prep_flat_kernel<true, false><<<grid, 256, 0, s>>>(L);
-        else if (gb) prep_flat_kernel<true, true><<<grid, 256, 0, s>>>(L);
-        else if (!xf) prep_flat_kernel<false, false><<<grid, 256, 0, s>>>(L);
-        else prep_flat_kernel<false, true><<<grid, 256, 0, s>>>(L);
+        if (gb && !xf) e = launch_pdl(prep_flat_kernel<true, false>, grid, dim3(256), 0, s, L);
+        else if (gb) e = launch_pdl(prep_flat_kernel<true, true>, grid, dim3(256), 0, s, L);
+        else if (!xf) e = launch_pdl(prep_flat_kernel<false, false>, grid, dim3(256), 0, s, L);
+        else e = launch_pdl(prep_flat_kernel<false, true>, grid, dim3(256), 0, s, L);
     }
-    return cudaGetLastError();
+    return e;
 }
 
 cudaError_t launch_norm_finalize(const double* partials, int64_t parts, int units, float eps, float* scale,
                                  cudaStream_t s) {
     if (units == 0) return cudaSuccess;
-    norm_finalize_kernel<<<(units + 7) / 8, 256, 0, s>>>(partials, parts, units, eps, scale);
-    return cudaGetLastError();
+    return launch_pdl(norm_finalize_kernel, dim3((units + 7) / 8), dim3(256), 0, s, partials, parts, units, eps,
+                      scale);
 }
 
 }  // namespace ma

@@ -21,6 +21,8 @@ __global__ void __launch_bounds__(256) ns_simt_kernel(const __grid_constant__ Ns
                                                       const float* __restrict__ gb) {
     __shared__ float As[TK][TS + 4];
     __shared__ float Bs[TK][TS + 4];
+    griddep_launch_dependents();
+    griddep_wait();
     const int u = blockIdx.z;
     const int i0 = blockIdx.y * TS, j0 = blockIdx.x * TS;
     const bool gram = (MODE == NS_GRAM || MODE == NS_GRAMSQ);
@@ -128,13 +130,12 @@ cudaError_t launch_ns_simt(int mode, const NsParams& p, const void* x_buf, const
     const float* xb = reinterpret_cast<const float*>(x_buf);
     const float* gb = reinterpret_cast<const float*>(g_buf);
     switch (mode) {
-        case NS_GRAM: ns_simt_kernel<NS_GRAM><<<grid, 256, 0, s>>>(p, xb, gb); break;
-        case NS_GRAMSQ: ns_simt_kernel<NS_GRAMSQ><<<grid, 256, 0, s>>>(p, xb, gb); break;
-        case NS_APPLY: ns_simt_kernel<NS_APPLY><<<grid, 256, 0, s>>>(p, xb, gb); break;
-        case NS_FINAL: ns_simt_kernel<NS_FINAL><<<grid, 256, 0, s>>>(p, xb, gb); break;
+        case NS_GRAM: return launch_pdl(ns_simt_kernel<NS_GRAM>, grid, dim3(256), 0, s, p, xb, gb);
+        case NS_GRAMSQ: return launch_pdl(ns_simt_kernel<NS_GRAMSQ>, grid, dim3(256), 0, s, p, xb, gb);
+        case NS_APPLY: return launch_pdl(ns_simt_kernel<NS_APPLY>, grid, dim3(256), 0, s, p, xb, gb);
+        case NS_FINAL: return launch_pdl(ns_simt_kernel<NS_FINAL>, grid, dim3(256), 0, s, p, xb, gb);
         default: return cudaErrorInvalidValue;
     }
-    return cudaGetLastError();
 }
 
 }  // namespace ma

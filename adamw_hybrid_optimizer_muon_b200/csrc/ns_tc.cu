@@ -411,6 +411,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    griddep_launch_dependents();
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = leader of the pair
     const bool leader = rank == 0;
     const int pair = PAIR ? (int)cluster_id_x() : (int)blockIdx.x;
@@ -452,6 +453,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     else __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_holder;
+    griddep_wait();  // the previous kernel's results (and its reads of our outputs) are complete
 
     if (warp == 0) {
         if (lane == 0) {
@@ -811,19 +813,21 @@ cudaError_t launch_mode(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_
     int max_units = 0;
     cudaError_t e = setup_mode<MODE, PAIR>(num_sms, &max_units);
     if (e != cudaSuccess) return e;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = 2;
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = MA_PDL;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     const long long units = tile0 < max_units ? tile0 : max_units;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)((PAIR ? 2 : 1) * units));
     cfg.blockDim = dim3(THREADS);
     cfg.dynamicSmemBytes = S::SMEM;
     cfg.stream = s;
-    cfg.attrs = PAIR ? attr : nullptr;
-    cfg.numAttrs = PAIR ? 1 : 0;
+    cfg.attrs = attr;
+    cfg.numAttrs = PAIR ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, ns_tc_kernel<MODE, PAIR>, L);
 }
 
