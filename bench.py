@@ -46,7 +46,7 @@ UNIT = "params/s"
 # Newton-Schulz launch, averaged over the 200 ns_tc_kernel launches of two 7B
 # steps in one capture of the current kernel (profiles/launches_7b_step.md).
 # Workloads without a capture report None.
-NS_TRAFFIC_BYTES_PER_LAUNCH = {"7b": 5.771e9}
+NS_TRAFFIC_BYTES_PER_LAUNCH = {"7b": 5.015e9}
 
 
 def env_int(name, default):
