@@ -114,12 +114,14 @@ int device_ok_and_sms(int* sms) {
     if (cudaGetDevice(&dev) != cudaSuccess) return MA_ERR_CUDA;
     if (dev < 0 || dev >= 64) return MA_ERR_UNSUPPORTED;
     if (!cached_ok[dev]) {
-        int maj = 0, min = 0, n = 0;
+        int maj = 0, min = 0, n = 0, smem = 0;
         if (cudaDeviceGetAttribute(&maj, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&min, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
             return MA_ERR_CUDA;
         if (maj != 10 || min != 0) return MA_ERR_UNSUPPORTED;
+        if ((size_t)smem < ns_tc_smem_bytes() || n < 2) return MA_ERR_UNSUPPORTED;
         cached_sms[dev] = n;
         cached_ok[dev] = 1;
     }

@@ -60,8 +60,6 @@ namespace {
 constexpr int BM = 256, BN = 256, BK = 64, STAGES = MA_NS_STAGES;
 constexpr int HM = BM / 2, HN = BN / 2;                // rows of A / columns of B held by each CTA
 constexpr uint32_t A_BYTES = HM * BK * 2;              // 16 KB
-constexpr uint32_t B_BYTES = HN * BK * 2;              // 16 KB
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;    // 32 KB per CTA
 constexpr int EPI_WARPS = 8;
 constexpr int THREADS = 32 * (2 + EPI_WARPS);
 // Epilogue staging: per epilogue warp one 32 x 32 bf16 block for the tile and
@@ -86,10 +84,6 @@ constexpr uint32_t FIN_WARP_BYTES = 2 * WBUF + 2 * XBUF;         // 12 KB
 constexpr uint32_t WBUF_BYTES = EPI_WARPS * FIN_WARP_BYTES;      // 96 KB
 constexpr int kStages(int mode) { return mode == NS_FINAL ? 4 : STAGES; }
 constexpr uint32_t kEpiBytes(int mode) { return mode == NS_FINAL ? WBUF_BYTES : STG_BYTES; }
-constexpr size_t kSmemBytes(int mode) {
-    return (size_t)kStages(mode) * STAGE_BYTES + kEpiBytes(mode) + 1024 /*align*/ + 512 /*barriers*/;
-}
-constexpr size_t SMEM_BYTES = kSmemBytes(NS_GRAM);
 
 // Tile shape of one kernel instance. PAIR: a CTA pair computes a 256 x 256
 // tile (cta_group::2, each CTA holding 128 rows of A and 128 columns of B).
@@ -860,7 +854,14 @@ cudaError_t launch_split(const NsJobIn* jobs, int njobs, int num_sms, cudaStream
 
 }  // namespace
 
-size_t ns_tc_smem_bytes() { return SMEM_BYTES; }
+size_t ns_tc_smem_bytes() {  // the largest dynamic shared memory of any instance
+    size_t m = 0;
+#define MA_MAXS(M, P) m = Shape<M, P>::SMEM > m ? Shape<M, P>::SMEM : m;
+    MA_MAXS(NS_GRAM, true) MA_MAXS(NS_GRAM, false) MA_MAXS(NS_GRAMSQ, true) MA_MAXS(NS_GRAMSQ, false)
+    MA_MAXS(NS_APPLY, true) MA_MAXS(NS_APPLY, false) MA_MAXS(NS_FINAL, true) MA_MAXS(NS_FINAL, false)
+#undef MA_MAXS
+    return m;
+}
 
 cudaError_t ns_tc_setup(int num_sms) {
     if (!encode_fn()) return cudaErrorNotSupported;
