@@ -1040,6 +1040,23 @@ int ma_plan_create(const ma_tensor_t* t, int n, const ma_group_t* groups, int ng
             if (!found) plan->buckets.push_back({x.group, x.shape[0], x.shape[1], {i}, 0});
         }
     }
+    // Buffers the step writes (params and optimizer state) must not overlap:
+    // a tensor listed twice, or state sharing memory with a parameter, would be
+    // updated twice or read after being overwritten.
+    {
+        std::vector<std::pair<uintptr_t, uintptr_t>> w;  // [begin, end) of every written buffer
+        for (int i = 0; i < n; ++i) {
+            const int64_t numel = tensor_numel(t[i]);
+            if (numel == 0) continue;
+            const uintptr_t bytes = (uintptr_t)numel * 4;
+            w.push_back({(uintptr_t)t[i].param, (uintptr_t)t[i].param + bytes});
+            w.push_back({(uintptr_t)t[i].state0, (uintptr_t)t[i].state0 + bytes});
+            if (kind[i] == MA_ADAMW) w.push_back({(uintptr_t)t[i].state1, (uintptr_t)t[i].state1 + bytes});
+        }
+        std::sort(w.begin(), w.end());
+        for (size_t k = 1; k < w.size(); ++k)
+            if (w[k].first < w[k - 1].second) return fail(MA_ERR_ARG);
+    }
     size_t need = 0;
     for (auto& b : plan->buckets) {
         const ma_muon_hparams_t& hp = groups[b.group].muon;

@@ -234,7 +234,9 @@ int adamw_step_fused(int n, float* const* P, const void* const* G, int gdt, floa
  * Consecutive sub-batches whose Newton-Schulz chains take the same kernels
  * (tensor-core path, same iteration count, same iterations with c != 0) share
  * launches when their summed workspace fits: within the cap when one is given,
- * else within the larger of the biggest sub-batch and 4 GiB. */
+ * else within the larger of the biggest sub-batch and 4 GiB. Parameters and
+ * optimizer state of different tensors (and a tensor's own state buffers)
+ * must not overlap: MA_ERR_ARG otherwise. */
 int ma_plan_create(const ma_tensor_t* t, int n, const ma_group_t* groups, int ngroups,
                    ma_plan_t** out, size_t* ws_bytes);
 

@@ -173,7 +173,7 @@ def test_plan_sizing_on_host():
     descs = []
     for i, t in enumerate(wl.tensors):
         d = _desc(t.shape, t.role, t.group)
-        d.param = d.state0 = d.state1 = d.grad = 0x100000 + 0x1000 * i
+        d.param, d.state0, d.state1, d.grad = (((4 * i + k + 1) << 32) for k in range(4))  # disjoint fake buffers
         d.grad_dtype = ma.MA_BF16
         descs.append(d)
     plan, ws = ma.ma_plan_create(descs, _groups_for(wl))
@@ -195,6 +195,32 @@ def test_plan_sizing_on_host():
     with pytest.raises(ma.MAError) as e:
         ma.ma_plan_create(descs, _groups_for(wl), ws_cap=1 << 20)
     assert e.value.code == ma.MA_ERR_WORKSPACE
+
+
+def test_plan_rejects_overlapping_written_buffers():
+    wl = synth.tiny()
+
+    def desc(shape, role, group, base):
+        d = _desc(shape, role, group)
+        d.param, d.state0, d.state1, d.grad = base, base + (1 << 30), base + (2 << 30), base + (3 << 30)
+        return d
+    a = desc((256, 512), ma.ROLE_HIDDEN, 0, 1 << 36)
+    b = desc((512,), ma.ROLE_HIDDEN, 1, 2 << 36)
+    plan, _ = ma.ma_plan_create([a, b], _groups_for(wl))  # disjoint: accepted
+    ma.ma_plan_destroy(plan)
+    c = desc((512,), ma.ROLE_HIDDEN, 1, 2 << 36)
+    c.param = a.param + 256 * 512 * 4 - 4  # starts inside the last element of a's parameter
+    with pytest.raises(ma.MAError) as e:
+        ma.ma_plan_create([a, c], _groups_for(wl))
+    assert e.value.code == ma.MA_ERR_ARG
+    with pytest.raises(ma.MAError) as e:
+        ma.ma_plan_create([a, a], _groups_for(wl))  # the same tensor twice
+    assert e.value.code == ma.MA_ERR_ARG
+    d = desc((512,), ma.ROLE_HIDDEN, 1, 3 << 36)
+    d.state1 = d.state0  # exp_avg and exp_avg_sq in one buffer
+    with pytest.raises(ma.MAError) as e:
+        ma.ma_plan_create([a, d], _groups_for(wl))
+    assert e.value.code == ma.MA_ERR_ARG
 
 
 def test_plan_rejects_kind_mismatch():
