@@ -428,6 +428,15 @@ int check_ptr_array(const void* const* a, int n, size_t align) {
     return MA_OK;
 }
 
+// MA_ERR_ARG if any two of the [begin, end) byte ranges overlap (buffers that
+// one call writes must be disjoint). Sorts w.
+int check_disjoint(std::vector<std::pair<uintptr_t, uintptr_t>>& w) {
+    std::sort(w.begin(), w.end());
+    for (size_t k = 1; k < w.size(); ++k)
+        if (w[k].first < w[k - 1].second) return MA_ERR_ARG;
+    return MA_OK;
+}
+
 int check_muon_call(int batch, int64_t R, int64_t C, float* const* W, const void* const* G, int gdt,
                     float* const* M, const ma_muon_hparams_t* hp, MuonGeom* g) {
     int st = check_muon_hp(hp);
@@ -442,7 +451,13 @@ int check_muon_call(int batch, int64_t R, int64_t C, float* const* W, const void
     if ((st = check_ptr_array(reinterpret_cast<const void* const*>(M), batch, 16))) return st;
     if (C % 8 != 0) return MA_ERR_ALIGN;
     if (g->units > 65535 || g->m > INT_MAX || g->n > INT_MAX || g->parts > INT_MAX) return MA_ERR_UNSUPPORTED;
-    return MA_OK;
+    std::vector<std::pair<uintptr_t, uintptr_t>> w;
+    const uintptr_t bytes = (uintptr_t)(R * C) * 4;
+    for (int b = 0; b < batch; ++b) {
+        w.push_back({(uintptr_t)W[b], (uintptr_t)W[b] + bytes});
+        w.push_back({(uintptr_t)M[b], (uintptr_t)M[b] + bytes});
+    }
+    return check_disjoint(w);
 }
 
 // ------------------------------------------------------------------ AdamW helpers
@@ -969,6 +984,12 @@ int adamw_step_fused(int n, float* const* P, const void* const* G, int gdt, floa
         items.push_back({P[i], G[i], M[i], V[i], numel[i], 0});
     }
     if (items.empty()) return MA_OK;
+    std::vector<std::pair<uintptr_t, uintptr_t>> w;
+    for (const AdamwItem& it : items) {
+        const uintptr_t bytes = (uintptr_t)it.numel * 4;
+        for (const float* q : {it.p, it.m, it.v}) w.push_back({(uintptr_t)q, (uintptr_t)q + bytes});
+    }
+    if ((st = check_disjoint(w))) return st;
     if ((st = device_ok_and_sms(nullptr))) return st;
     AdamwGroupConst c = adamw_const(*hp);
     int launches = 0;
@@ -1053,9 +1074,7 @@ int ma_plan_create(const ma_tensor_t* t, int n, const ma_group_t* groups, int ng
             w.push_back({(uintptr_t)t[i].state0, (uintptr_t)t[i].state0 + bytes});
             if (kind[i] == MA_ADAMW) w.push_back({(uintptr_t)t[i].state1, (uintptr_t)t[i].state1 + bytes});
         }
-        std::sort(w.begin(), w.end());
-        for (size_t k = 1; k < w.size(); ++k)
-            if (w[k].first < w[k - 1].second) return fail(MA_ERR_ARG);
+        if ((st = check_disjoint(w))) return fail(st);
     }
     size_t need = 0;
     for (auto& b : plan->buckets) {

@@ -120,38 +120,48 @@ def test_validation_before_any_device_call():
     hp = ma.muon_hparams()
     L = ma.lib()
     fake = ctypes.c_void_p(0x1000)
-    arr = (ctypes.c_void_p * 1)(0x1000)
+    arr = (ctypes.c_void_p * 1)(0x100000)   # weights / AdamW params
+    garr = (ctypes.c_void_p * 1)(0x200000)  # gradients
+    marr = (ctypes.c_void_p * 1)(0x300000)  # momentum / exp_avg
+    varr = (ctypes.c_void_p * 1)(0x400000)  # exp_avg_sq
     null = (ctypes.c_void_p * 1)(0)
     # C % 8 != 0
-    rc = L.muon_step_batched(1, 16, 12, arr, arr, ma.MA_F32, arr, ctypes.byref(hp), fake, 1 << 30, None)
+    rc = L.muon_step_batched(1, 16, 12, arr, garr, ma.MA_F32, marr, ctypes.byref(hp), fake, 1 << 30, None)
     assert rc == ma.MA_ERR_ALIGN
     # null pointer entry
-    rc = L.muon_step_batched(1, 16, 16, null, arr, ma.MA_F32, arr, ctypes.byref(hp), fake, 1 << 30, None)
+    rc = L.muon_step_batched(1, 16, 16, null, garr, ma.MA_F32, marr, ctypes.byref(hp), fake, 1 << 30, None)
     assert rc == ma.MA_ERR_NULL
     # heads must divide R
     hp3 = ma.muon_hparams(heads=3)
-    rc = L.muon_step_batched(1, 16, 16, arr, arr, ma.MA_F32, arr, ctypes.byref(hp3), fake, 1 << 30, None)
+    rc = L.muon_step_batched(1, 16, 16, arr, garr, ma.MA_F32, marr, ctypes.byref(hp3), fake, 1 << 30, None)
     assert rc == ma.MA_ERR_SHAPE
     # bad dtype, bad steps, bad coefficient count
-    assert L.muon_step_batched(1, 16, 16, arr, arr, 7, arr, ctypes.byref(hp), fake, 1 << 30, None) == ma.MA_ERR_DTYPE
+    assert L.muon_step_batched(1, 16, 16, arr, garr, 7, marr, ctypes.byref(hp), fake, 1 << 30, None) == ma.MA_ERR_DTYPE
     bad = ma.muon_hparams(ns_steps=0)
-    assert L.muon_step_batched(1, 16, 16, arr, arr, 0, arr, ctypes.byref(bad), fake, 1 << 30, None) == ma.MA_ERR_ARG
+    assert L.muon_step_batched(1, 16, 16, arr, garr, 0, marr, ctypes.byref(bad), fake, 1 << 30, None) == ma.MA_ERR_ARG
     bad = ma.muon_hparams(ns_steps=3, coeffs=((1.5, -0.5, 0), (1.5, -0.5, 0)))
-    assert L.muon_step_batched(1, 16, 16, arr, arr, 0, arr, ctypes.byref(bad), fake, 1 << 30, None) == ma.MA_ERR_ARG
+    assert L.muon_step_batched(1, 16, 16, arr, garr, 0, marr, ctypes.byref(bad), fake, 1 << 30, None) == ma.MA_ERR_ARG
     # workspace too small / misaligned
-    assert L.muon_step_batched(1, 16, 16, arr, arr, 0, arr, ctypes.byref(hp), fake, 16, None) == ma.MA_ERR_WORKSPACE
-    assert L.muon_step_batched(1, 16, 16, arr, arr, 0, arr, ctypes.byref(hp), ctypes.c_void_p(0x1008), 1 << 30,
+    assert L.muon_step_batched(1, 16, 16, arr, garr, 0, marr, ctypes.byref(hp), fake, 16, None) == ma.MA_ERR_WORKSPACE
+    assert L.muon_step_batched(1, 16, 16, arr, garr, 0, marr, ctypes.byref(hp), ctypes.c_void_p(0x1008), 1 << 30,
                                None) == ma.MA_ERR_WORKSPACE
     # empty batch is a no-op
-    assert L.muon_step_batched(0, 16, 16, arr, arr, 0, arr, ctypes.byref(hp), None, 0, None) == ma.MA_OK
+    assert L.muon_step_batched(0, 16, 16, arr, garr, 0, marr, ctypes.byref(hp), None, 0, None) == ma.MA_OK
     # AdamW: bad step, bad betas
     ahp = ma.adamw_hparams(step=0)
     n1 = (ctypes.c_int64 * 1)(4)
-    assert L.adamw_step_fused(1, arr, arr, 0, arr, arr, n1, ctypes.byref(ahp), None) == ma.MA_ERR_ARG
+    assert L.adamw_step_fused(1, arr, garr, 0, marr, varr, n1, ctypes.byref(ahp), None) == ma.MA_ERR_ARG
     ahp = ma.adamw_hparams(beta2=1.0)
-    assert L.adamw_step_fused(1, arr, arr, 0, arr, arr, n1, ctypes.byref(ahp), None) == ma.MA_ERR_ARG
+    assert L.adamw_step_fused(1, arr, garr, 0, marr, varr, n1, ctypes.byref(ahp), None) == ma.MA_ERR_ARG
     ahp = ma.adamw_hparams()
-    assert L.adamw_step_fused(1, null, arr, 0, arr, arr, n1, ctypes.byref(ahp), None) == ma.MA_ERR_NULL
+    assert L.adamw_step_fused(1, null, garr, 0, marr, varr, n1, ctypes.byref(ahp), None) == ma.MA_ERR_NULL
+    # buffers the call writes must be disjoint
+    assert L.muon_step_batched(1, 16, 16, arr, garr, 0, arr, ctypes.byref(hp), fake, 1 << 30, None) == ma.MA_ERR_ARG
+    two = (ctypes.c_void_p * 2)(0x100000, 0x100000 + 512)  # second matrix starts inside the first
+    m2 = (ctypes.c_void_p * 2)(0x300000, 0x310000)
+    g2 = (ctypes.c_void_p * 2)(0x200000, 0x210000)
+    assert L.muon_step_batched(2, 16, 16, two, g2, 0, m2, ctypes.byref(hp), fake, 1 << 30, None) == ma.MA_ERR_ARG
+    assert L.adamw_step_fused(1, arr, garr, 0, marr, marr, n1, ctypes.byref(ahp), None) == ma.MA_ERR_ARG
 
 
 def test_valid_call_without_gpu_fails_loudly():
