@@ -173,8 +173,8 @@ def test_valid_call_without_gpu_fails_loudly():
         pass
     hp = ma.muon_hparams()
     L = ma.lib()
-    arr = (ctypes.c_void_p * 1)(0x1000)
-    rc = L.muon_step_batched(1, 16, 16, arr, arr, 0, arr, ctypes.byref(hp), ctypes.c_void_p(0x10000), 1 << 30, None)
+    w, g, m = ((ctypes.c_void_p * 1)(a) for a in (0x100000, 0x200000, 0x300000))
+    rc = L.muon_step_batched(1, 16, 16, w, g, 0, m, ctypes.byref(hp), ctypes.c_void_p(0x10000), 1 << 30, None)
     assert rc in (ma.MA_ERR_CUDA, ma.MA_ERR_UNSUPPORTED)
 
 
