@@ -25,7 +25,7 @@ method as these pages describe it:
   Design", "Confirmed": per-head orthogonalisation, and forcing AdamW on
   some projections.
 
-Readings where the pages are silent (each one is listed in the design notes):
+Readings where the pages are silent:
 
 * Frobenius normalisation ``X0 = u / (||u||_F + eps)`` with eps = 1e-7.
 * Nesterov form ``u = beta*m_new + (1-beta)*g``.
