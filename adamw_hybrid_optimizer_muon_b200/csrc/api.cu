@@ -885,8 +885,24 @@ int muon_step_batched(int batch, int64_t R, int64_t C, float* const* W, const vo
     if (!ws || !aligned(ws, kAlign) || ws_bytes < g.total) return MA_ERR_WORKSPACE;
     int sms = 0;
     if ((st = device_ok_and_sms(&sms))) return st;
+    // a large batch runs as consecutive sub-batches of at most kSubBatchBytes of
+    // workspace each (fewer units per launch; the workspace is reused)
+    int sub = batch;
+    MuonGeom gs = g;
+    while (gs.total > kSubBatchBytes && sub > 1) {
+        sub = std::max(1, sub / 2);
+        muon_geom(sub, R, C, *hp, &gs);
+    }
     int launches = 0;
-    return run_muon(batch, g, W, G, gdt, M, *hp, ws, reinterpret_cast<cudaStream_t>(stream), sms, &launches);
+    for (int s0 = 0; s0 < batch; s0 += sub) {
+        const int cnt = std::min(sub, batch - s0);
+        MuonGeom gc;
+        muon_geom(cnt, R, C, *hp, &gc);
+        if ((st = run_muon(cnt, gc, W + s0, G + s0, gdt, M + s0, *hp, ws, reinterpret_cast<cudaStream_t>(stream),
+                           sms, &launches)))
+            return st;
+    }
+    return MA_OK;
 }
 
 size_t ns_iterate_workspace_bytes(int batch, int64_t m, int64_t n) {

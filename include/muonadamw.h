@@ -174,7 +174,10 @@ size_t muon_workspace_bytes(int batch, int64_t R, int64_t C, const ma_muon_hpara
  *  G:    host array of `batch` device pointers to R x C gradients (gdt), read only.
  *  hp:   host pointer. ws: device workspace of ws_bytes >= muon_workspace_bytes(),
  *        256-byte aligned, contents scratch.
- * Requires C % 8 == 0 and 16-byte aligned W/M/G; R % hp->heads == 0. */
+ * Requires C % 8 == 0 and 16-byte aligned W/M/G; R % hp->heads == 0, and
+ * W and M buffers that do not overlap (MA_ERR_ARG). A batch whose workspace
+ * exceeds 4 GiB runs as consecutive sub-batches (halved until each fits),
+ * reusing the start of ws; the results are the same. */
 int muon_step_batched(int batch, int64_t R, int64_t C, float* const* W, const void* const* G,
                       int gdt, float* const* M, const ma_muon_hparams_t* hp, void* ws,
                       size_t ws_bytes, void* stream);

@@ -234,3 +234,27 @@ def test_grouped_newton_schulz_launches_match_per_bucket_calls():
         return int(any(small)) + int(not all(small))
     sets = [(range(0, 8), 2), (range(8, 9), 2), (range(9, 11), 3)]
     assert grouped == 2 * len(shapes) + sum(5 * per * kinds(b) for b, per in sets)
+
+
+def test_batched_call_beyond_4gib_runs_in_sub_batches():
+    """muon_step_batched on 48 matrices of 4096 x 4096 (4.6 GB of workspace)
+    runs as two sub-batches of 24 inside the caller's workspace; the result
+    must equal two calls of 24, bit for bit."""
+    R = C = 4096
+    n = 48
+    hp = ma.muon_hparams()
+    assert ma.muon_workspace_bytes(n, R, C, hp) > 4 << 30 >= ma.muon_workspace_bytes(n // 2, R, C, hp)
+    gen = torch.Generator(device="cuda").manual_seed(5)
+    W0 = torch.randn(n, R, C, device="cuda", generator=gen) * 0.02
+    G = (torch.randn(n, R, C, device="cuda", generator=gen) * 1e-3).to(torch.bfloat16)
+    Wa, Ma = W0.clone(), torch.zeros_like(W0)
+    ws = torch.empty(ma.muon_workspace_bytes(n, R, C, hp), dtype=torch.uint8, device="cuda")
+    ma.muon_step_batched(list(Wa), list(G), list(Ma), hp, ws)
+    Wb, Mb = W0.clone(), torch.zeros_like(W0)
+    for s0 in (0, n // 2):
+        sl = slice(s0, s0 + n // 2)
+        ma.muon_step_batched(list(Wb[sl]), list(G[sl]), list(Mb[sl]), hp, ws)
+    torch.cuda.synchronize()
+    assert ma.ma_device_status() == ma.MA_OK
+    assert torch.equal(Wa, Wb) and torch.equal(Ma, Mb)
+    assert not torch.equal(Wa, W0)
