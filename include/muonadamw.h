@@ -151,10 +151,15 @@ size_t ma_struct_size(int which);
  * array of n ints. Host-only, no CUDA call, bit-exact and deterministic. */
 int ma_partition(const ma_tensor_t* t, int n, int32_t* kind_out);
 
-/* Owner rank per tensor for a data-parallel step over `world_size` ranks: Muon
- * matrices by greedy largest-Newton-Schulz-flops-first onto the least-loaded
- * rank, AdamW tensors the same way by element count, ties to the lower rank and
- * the lower tensor index. Every tensor gets exactly one owner. Host-only. */
+/* Owner rank per tensor for a data-parallel step over `world_size` ranks
+ * [P1 "Distributed Training Support": each rank updates its share of the
+ * parameters; P3: matrix batches are independent]: Muon matrices by greedy
+ * largest-Newton-Schulz-flops-first onto the least-loaded rank, AdamW tensors
+ * the same way by element count, ties to the lower rank and the lower tensor
+ * index. Every tensor gets exactly one owner. t, groups: host arrays (shapes,
+ * roles, groups and each Muon group's heads/ns_steps are read). owner_out:
+ * host array of n ints. Errors as ma_partition, MA_ERR_ARG for world_size < 1
+ * or a bad group index. Host-only, no CUDA call. */
 int ma_assign_owners(const ma_tensor_t* t, int n, const ma_group_t* groups, int ngroups,
                      int world_size, int32_t* owner_out);
 
