@@ -16,7 +16,7 @@ __all__ = [
     "LibraryMissing", "MAError", "lib", "MuonHParams", "AdamWHParams", "Group", "Tensor",
     "MA_OK", "MA_F32", "MA_BF16", "MA_MUON", "MA_ADAMW", "ROLE_HIDDEN", "ROLE_EMBED", "ROLE_UNEMBED",
     "ROLE_FORCE_ADAMW", "ma_partition", "ma_assign_owners", "muon_workspace_bytes", "muon_step_batched",
-    "ns_iterate_workspace_bytes", "ns_iterate_bf16", "adamw_step_fused", "ma_plan_create", "muonadamw_step", "muonadamw_step_graph",
+    "ns_iterate_workspace_bytes", "ns_iterate_bf16", "adamw_step_fused", "ma_plan_create", "muonadamw_step", "muonadamw_step_graph", "ma_plan_describe",
     "ma_plan_destroy", "ma_device_status", "ma_set_wait_limit_ns", "ma_selftest_wait_timeout", "Plan",
     "MuonAdamW", "muon_hparams", "adamw_hparams", "ma_profile_enable", "ma_profile_collect", "PROF_CLASSES",
     "muon_step_batched_noalloc", "STATIC_SCRATCH_BYTES", "muonadamw_step_from_host",
@@ -107,6 +107,7 @@ def lib() -> ctypes.CDLL:
         "ma_plan_last_launches": (i32, [vp]),
         "muonadamw_step_graph": (i32, [vp, ctypes.POINTER(Group), vp, sz, vp]),
         "ma_plan_graph_captures": (i32, [vp]),
+        "ma_plan_describe": (i32, [vp, ctypes.POINTER(Group), ctypes.c_char_p, sz]),
         "ma_plan_destroy": (None, [vp]),
         "ma_device_status": (i32, [vp, i32]),
         "ma_set_wait_limit_ns": (i32, [i64]),
@@ -300,6 +301,19 @@ def muonadamw_step(plan, groups: Sequence[Group], ws, ws_bytes: int, stream=None
     _check(lib().muonadamw_step(plan, garr, _ptr(ws), int(ws_bytes), _stream(stream)), "muonadamw_step")
 
 
+def ma_plan_describe(plan, groups: Sequence[Group]) -> str:
+    """Text description of the plan's buckets, sub-batches and launch segments (host-only)."""
+    garr = (Group * max(1, len(groups)))(*groups)
+    size = 1 << 14
+    while True:
+        buf = ctypes.create_string_buffer(size)
+        rc = lib().ma_plan_describe(plan, garr, buf, size)
+        if rc != MA_ERR_SHAPE or size >= 1 << 24:
+            _check(rc, "ma_plan_describe")
+            return buf.value.decode()
+        size *= 4
+
+
 def muonadamw_step_graph(plan, groups: Sequence[Group], ws, ws_bytes: int, stream=None) -> None:
     """muonadamw_step replayed from a CUDA graph the plan captures and keeps."""
     garr = (Group * max(1, len(groups)))(*groups)
@@ -377,6 +391,10 @@ class Plan:
     @property
     def graph_captures(self) -> int:
         return int(lib().ma_plan_graph_captures(self.handle))
+
+    def describe(self, groups: Sequence[Group] | None = None) -> str:
+        """What a step runs: workspace, buckets, sub-batches and shared launches."""
+        return ma_plan_describe(self.handle, groups if groups is not None else self.groups)
 
     def close(self) -> None:
         if self.handle is not None and self.handle.value:
@@ -493,3 +511,9 @@ class MuonAdamW:
     def graph_captures(self) -> int:
         """How many times the plan captured its CUDA graph (graph steps only)."""
         return self._plan.graph_captures if self._plan is not None else 0
+
+    def describe(self) -> str:
+        """What a step runs (buckets, sub-batches, shared launches); needs one step first."""
+        if self._plan is None:
+            raise RuntimeError("no plan yet: the plan is built on the first step")
+        return self._plan.describe(self.groups)

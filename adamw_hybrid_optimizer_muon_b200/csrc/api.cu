@@ -19,8 +19,10 @@
 #include <climits>
 #include <cmath>
 #include <cstdlib>
+#include <cstdio>
 #include <cstring>
 #include <new>
+#include <string>
 #include <unordered_map>
 #include <vector>
 
@@ -1367,6 +1369,51 @@ int muonadamw_step_from_host(ma_plan_t* plan, const ma_group_t* groups, const vo
 int ma_plan_last_launches(const ma_plan_t* plan) { return plan ? plan->last_launches : 0; }
 
 int ma_plan_graph_captures(const ma_plan_t* plan) { return plan ? plan->g.captures : 0; }
+
+int ma_plan_describe(const ma_plan_t* plan, const ma_group_t* groups, char* buf, size_t len) {
+    if (!plan || !buf || len == 0) return MA_ERR_NULL;
+    const int ngroups = (int)plan->group_kind.size();
+    if (ngroups > 0 && !groups) return MA_ERR_NULL;
+    for (int k = 0; k < ngroups; ++k) {
+        if (groups[k].kind != plan->group_kind[k]) return MA_ERR_ARG;
+        if (groups[k].kind == MA_MUON && check_muon_hp(&groups[k].muon)) return MA_ERR_ARG;
+    }
+    std::string out;
+    char line[256];
+    int64_t adamw_elems = 0;
+    for (int i : plan->adamw_idx) adamw_elems += tensor_numel(plan->t[i]);
+    std::snprintf(line, sizeof(line), "workspace %zu bytes; AdamW: %zu tensors, %lld elements\n", plan->ws_bytes,
+                  plan->adamw_idx.size(), (long long)adamw_elems);
+    out += line;
+    for (size_t bi = 0; bi < plan->buckets.size(); ++bi) {
+        const auto& b = plan->buckets[bi];
+        const ma_muon_hparams_t& hp = groups[b.group].muon;
+        std::snprintf(line, sizeof(line), "bucket %zu: group %d, %lld x %lld, %zu matrices (%s grads), heads %d, "
+                      "sub-batches of %d\n", bi, b.group, (long long)b.R, (long long)b.C, b.members.size(),
+                      plan->t[b.members[0]].grad_dtype == MA_BF16 ? "bf16" : "fp32", hp.heads, b.sub);
+        out += line;
+    }
+    int si = 0;
+    for (const Segment& sg : step_segments(plan, groups, 0, 0, false, plan->ws_bytes)) {
+        if (sg.adamw) {
+            std::snprintf(line, sizeof(line), "segment %d: AdamW\n", si++);
+            out += line;
+            continue;
+        }
+        std::snprintf(line, sizeof(line), "segment %d: Newton-Schulz launches shared by", si++);
+        out += line;
+        for (const Part& pt : sg.parts) {
+            std::snprintf(line, sizeof(line), " [bucket %d, matrices %d..%d]", pt.bucket, pt.start,
+                          pt.start + pt.count - 1);
+            out += line;
+        }
+        out += "\n";
+    }
+    const size_t n = std::min(len - 1, out.size());
+    std::memcpy(buf, out.data(), n);
+    buf[n] = 0;
+    return out.size() < len ? MA_OK : MA_ERR_SHAPE;
+}
 
 void ma_plan_destroy(ma_plan_t* plan) { delete plan; }
 

@@ -290,6 +290,14 @@ int muonadamw_step_graph(ma_plan_t* plan, const ma_group_t* groups, void* ws, si
  * benchmarks). 0 for a NULL plan. */
 int ma_plan_graph_captures(const ma_plan_t* plan);
 
+/* A text description of what muonadamw_step runs for this plan with these
+ * hyperparameters: the workspace, the AdamW tensors, each Muon bucket (group,
+ * shape, count, gradient dtype, heads, sub-batch size) and each segment of
+ * launches (which sub-batches share Newton-Schulz launches). buf: host buffer
+ * of len bytes, always NUL-terminated; MA_ERR_SHAPE when the text was cut to
+ * fit. Host-only, no CUDA call. */
+int ma_plan_describe(const ma_plan_t* plan, const ma_group_t* groups, char* buf, size_t len);
+
 /* Number of kernel launches the last muonadamw_step, muonadamw_step_graph or
  * muonadamw_step_from_host issued (for a graph step: the kernels in the graph). */
 int ma_plan_last_launches(const ma_plan_t* plan);

@@ -207,6 +207,36 @@ def test_plan_sizing_on_host():
     assert e.value.code == ma.MA_ERR_WORKSPACE
 
 
+def _fake_descs(wl):
+    descs = []
+    for i, t in enumerate(wl.tensors):
+        d = _desc(t.shape, t.role, t.group)
+        d.param, d.state0, d.state1, d.grad = (((4 * i + k + 1) << 32) for k in range(4))
+        d.grad_dtype = ma.MA_BF16
+        descs.append(d)
+    return descs
+
+
+def test_plan_describe():
+    wl = synth.llama7b()
+    plan, ws = ma.ma_plan_create(_fake_descs(wl), _groups_for(wl))
+    text = ma.ma_plan_describe(plan, _groups_for(wl))
+    ma.ma_plan_destroy(plan)
+    assert text.startswith(f"workspace {ws} bytes; AdamW: 67 tensors, ")
+    assert "4096 x 4096, 128 matrices (bf16 grads), heads 1, sub-batches of 32" in text
+    assert "4096 x 11008, 64 matrices (bf16 grads), heads 1, sub-batches of 16" in text
+    assert "11008 x 4096, 32 matrices (bf16 grads), heads 1, sub-batches of 16" in text
+    segs = [ln for ln in text.splitlines() if ln.startswith("segment")]
+    assert segs[0] == "segment 0: AdamW" and len(segs) == 1 + 4 + 4 + 2  # no sharing at this size
+    # the d20 set: its three buckets share one chain of Newton-Schulz launches
+    wl = synth.d20()
+    plan, _ = ma.ma_plan_create(_fake_descs(wl), _groups_for(wl))
+    text = ma.ma_plan_describe(plan, _groups_for(wl))
+    ma.ma_plan_destroy(plan)
+    segs = [ln for ln in text.splitlines() if ln.startswith("segment")]
+    assert len(segs) == 2 and segs[1].count("[bucket") == 3, text
+
+
 def test_plan_rejects_overlapping_written_buffers():
     wl = synth.tiny()
 
