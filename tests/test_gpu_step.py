@@ -48,8 +48,12 @@ def oracle_groups(wl, precision=0):
     return out
 
 
-@pytest.mark.parametrize("precision", [0, 1])
-def test_tiny_two_steps_every_element(precision):
+@pytest.mark.parametrize("precision,graph", [(0, False), (1, False), (0, True)])
+def test_tiny_twelve_steps_every_element(precision, graph):
+    """Twelve steps (the AdamW bias corrections and the momentum carry over),
+    each checked element by element against one oracle step from the GPU's
+    own pre-step values; eagerly, in fp32 mode, and replayed from a CUDA graph
+    whose AdamW step counter is patched every step."""
     wl = synth.tiny()
     W0 = [synth.initial_weight(t, i) for i, t in enumerate(wl.tensors)]
     params = [torch.from_numpy(w).cuda() for w in W0]
@@ -58,12 +62,14 @@ def test_tiny_two_steps_every_element(precision):
     groups = oracle_groups(wl)
     state = [{} for _ in wl.tensors]
     ref = [w.astype(np.float64) for w in W0]
-    for step in (1, 2):
+    gd = [torch.empty(t.shape, device="cuda") for t in wl.tensors]  # fixed buffers (one plan, one graph)
+    for step in range(1, 13):
         G = [synth.gradient(wl, i, step) for i in range(len(wl.tensors))]
-        gd = [torch.from_numpy(g).cuda() for g in G]  # fp32 gradients in this config
+        for d, g in zip(gd, G):
+            d.copy_(torch.from_numpy(g))  # fp32 gradients in this config
         before_p = [host(p) for p in params]
         before_s = [(host(s0), None if s1 is None else host(s1)) for s0, s1 in opt.state]
-        opt.step(gd)
+        opt.step(gd, graph=graph)
         torch.cuda.synchronize()
         assert ma.ma_device_status() == ma.MA_OK
         # one oracle step from exactly the GPU's pre-step values
@@ -79,6 +85,7 @@ def test_tiny_two_steps_every_element(precision):
         check_state(host(opt.state[1][0]), st[1]["exp_avg"], tm, what="exp_avg")
         check_state(host(opt.state[1][1]), st[1]["exp_avg_sq"], tv, what="exp_avg_sq")
     assert opt.launches == 1 + 2 + 2 * 5  # AdamW, momentum+norm, finalize, 5 x (Gram, apply)
+    assert opt.graph_captures == (1 if graph else 0)
 
 
 def _full_size_check(name, n_muon_samples=1, adamw_samples=200_000, seed=0):
