@@ -1,6 +1,6 @@
 """The whole MuonAdamW step through the plan (muonadamw_step) against the oracle.
 
-* tiny: every element of every tensor, two steps.
+* tiny: every element of every tensor, twelve steps (eager, fp32 mode, CUDA graph).
 * d20 and the 7B-shaped set at full size, in the same launch configuration
   bench.py times. The oracle recomputes sampled matrices in full (one of each
   bucket) and sampled elements of the AdamW tensors and of every momentum
