@@ -237,6 +237,38 @@ def test_plan_describe():
     assert len(segs) == 2 and segs[1].count("[bucket") == 3, text
 
 
+def test_plan_group_table_limits():
+    """MA_MAX_GROUPS groups are accepted, one more is refused before anything is built."""
+    def groups(k):
+        out = []
+        for i in range(k):
+            G = ma.Group()
+            G.kind = ma.MA_ADAMW if i % 2 else ma.MA_MUON
+            if G.kind == ma.MA_MUON:
+                G.muon = ma.muon_hparams(lr=0.01 * (i + 1))
+            else:
+                G.adamw = ma.adamw_hparams(lr=0.001 * (i + 1))
+            out.append(G)
+        return out
+    descs = []
+    for i in range(32):
+        d = _desc((64, 128) if i % 2 == 0 else (128,), ma.ROLE_HIDDEN, i)
+        d.param, d.state0, d.state1, d.grad = (((4 * i + k + 1) << 32) for k in range(4))
+        d.grad_dtype = ma.MA_BF16
+        descs.append(d)
+    plan, ws = ma.ma_plan_create(descs, groups(32))
+    text = ma.ma_plan_describe(plan, groups(32))
+    ma.ma_plan_destroy(plan)
+    lines = text.splitlines()
+    assert sum(ln.startswith("bucket ") for ln in lines) == 16  # one 64 x 128 bucket per Muon group
+    segs = [ln for ln in lines if ln.startswith("segment")]
+    # the 16 small buckets share launches, eight jobs at most per launch
+    assert len(segs) == 3 and segs[1].count("[bucket") == 8 and segs[2].count("[bucket") == 8
+    with pytest.raises(ma.MAError) as e:
+        ma.ma_plan_create(descs, groups(33))
+    assert e.value.code == ma.MA_ERR_UNSUPPORTED
+
+
 def test_plan_rejects_overlapping_written_buffers():
     wl = synth.tiny()
 
