@@ -1,15 +1,17 @@
 #!/usr/bin/env python
 """Benchmark of one MuonAdamW optimizer step on a B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 7b|d20|square|aspect|tiny]
-                    [--impl ours|reference] [--no-e2e]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 7b|d20|square|aspect|tiny|square8]
+                    [--impl ours|reference] [--no-e2e] [--no-cpu-baseline] [--graph] [--coeffs a,b,c;...]
 
-A step is one muonadamw_step over a synthetic parameter set. Each step runs
-AdamW on every 0-D/1-D tensor and on the embedding/unembedding, and the
-momentum/norm pass plus 5 Newton-Schulz iterations on every hidden matrix,
-with the final decay and apply. The default workload is the 7B-shaped set.
-Its inputs (params, grads, state: ~80 GB) are far larger than the 126 MB L2,
-so no flush is needed between steps.
+A step is one muonadamw_step over a synthetic parameter set (with --graph,
+the same step replayed from a CUDA graph). Each step runs AdamW on every
+0-D/1-D tensor and on the embedding/unembedding, and the momentum/norm pass
+plus 5 Newton-Schulz iterations on every hidden matrix, with the final decay
+and apply. The default workload is the 7B-shaped set. Its inputs (params,
+grads, state: ~70 GB) are far larger than the 126 MB L2, so no flush is
+needed between steps; sets smaller than twice the L2 get a 512 MB write
+between timed steps, outside their events.
 
 Printed (rank 0): one JSON line with the metric (params/s), ms per step, the
 end-to-end number through the C ABI with host buffers, the roofline of the
