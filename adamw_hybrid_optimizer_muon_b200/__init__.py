@@ -17,7 +17,7 @@ __all__ = [
     "MA_OK", "MA_F32", "MA_BF16", "MA_MUON", "MA_ADAMW", "ROLE_HIDDEN", "ROLE_EMBED", "ROLE_UNEMBED",
     "ROLE_FORCE_ADAMW", "ma_partition", "ma_assign_owners", "muon_workspace_bytes", "muon_step_batched",
     "ns_iterate_workspace_bytes", "ns_iterate_bf16", "adamw_step_fused", "ma_plan_create", "muonadamw_step", "muonadamw_step_graph", "ma_plan_describe",
-    "ma_plan_destroy", "ma_device_status", "ma_set_wait_limit_ns", "ma_selftest_wait_timeout", "Plan",
+    "ma_plan_destroy", "ma_device_status", "ma_device_status_async", "ma_set_wait_limit_ns", "ma_selftest_wait_timeout", "Plan",
     "MuonAdamW", "muon_hparams", "adamw_hparams", "ma_profile_enable", "ma_profile_collect", "PROF_CLASSES",
     "muon_step_batched_noalloc", "STATIC_SCRATCH_BYTES", "muonadamw_step_from_host",
 ]
@@ -110,6 +110,7 @@ def lib() -> ctypes.CDLL:
         "ma_plan_describe": (i32, [vp, ctypes.POINTER(Group), ctypes.c_char_p, sz]),
         "ma_plan_destroy": (None, [vp]),
         "ma_device_status": (i32, [vp, i32]),
+        "ma_device_status_async": (i32, [vp, vp]),
         "ma_set_wait_limit_ns": (i32, [i64]),
         "ma_selftest_wait_timeout": (i32, [i64, vp]),
         "muon_step_batched_noalloc": (i32, [i32, i64, i64, pp, pp, i32, pp, ctypes.POINTER(MuonHParams), vp]),
@@ -336,6 +337,11 @@ def ma_plan_destroy(plan) -> None:
 
 def ma_device_status(stream=None, reset: bool = True) -> int:
     return int(lib().ma_device_status(_stream(stream), int(bool(reset))))
+
+
+def ma_device_status_async(host_dst, stream=None) -> None:
+    """Enqueue a copy of the device status word into host_dst (a pinned int32 tensor element or address)."""
+    _check(lib().ma_device_status_async(_ptr(host_dst), _stream(stream)), "ma_device_status_async")
 
 
 def ma_set_wait_limit_ns(limit_ns: int) -> None:

@@ -1463,6 +1463,16 @@ int ma_device_status(void* stream, int reset) {
     return v;
 }
 
+int ma_device_status_async(int32_t* host_dst, void* stream) {
+    if (!host_dst) return MA_ERR_NULL;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MA_ERR_CUDA;
+    return cudaMemcpyFromSymbolAsync(host_dst, g_status, sizeof(int32_t), 0, cudaMemcpyDeviceToHost,
+                                     reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+               ? MA_OK
+               : MA_ERR_CUDA;
+}
+
 int ma_set_wait_limit_ns(int64_t limit_ns) {
     if (limit_ns <= 0) return MA_ERR_ARG;
     g_host_wait_limit_ns = limit_ns;

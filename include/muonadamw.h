@@ -338,6 +338,13 @@ int ma_profile_collect(double* ms_out, int64_t* launches_out, double* flops_out,
  * device-side error recorded since the last reset) and, if reset != 0, clear it. */
 int ma_device_status(void* stream, int reset);
 
+/* Enqueue on `stream` a copy of the current device's status word into
+ * host_dst (one int32, host; page-locked memory makes the copy asynchronous).
+ * The value is valid once the stream has passed the copy; the word is not
+ * reset. Lets a training loop read every step's status without stalling the
+ * host. MA_ERR_NULL for a NULL destination. */
+int ma_device_status_async(int32_t* host_dst, void* stream);
+
 /* Set the limit, in nanoseconds, of every device-side bounded wait (default
  * 2e9). Takes effect for launches issued after the call. */
 int ma_set_wait_limit_ns(int64_t limit_ns);
