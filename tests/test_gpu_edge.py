@@ -258,3 +258,21 @@ def test_batched_call_beyond_4gib_runs_in_sub_batches():
     assert ma.ma_device_status() == ma.MA_OK
     assert torch.equal(Wa, Wb) and torch.equal(Ma, Mb)
     assert not torch.equal(Wa, W0)
+
+
+@pytest.mark.parametrize("shape", [(1, 64), (1, 4096), (8, 8), (4096, 8), (8, 4096), (200, 8), (3, 1000 * 8)])
+def test_extreme_shapes(shape):
+    """Degenerate Muon shapes: a single row (m = 1), an 8 x 8 matrix, very
+    tall and very wide ones (m = 8 against n = 4096 or 8000), each through the
+    single-CTA tensor-core path, against the oracle."""
+    r = np.random.default_rng(sum(shape))
+    W0 = (r.standard_normal(shape) * 0.02).astype(np.float32)
+    g = bf16_round(r.standard_normal(shape) * 1e-3)
+    hp = ma.muon_hparams()
+    Wd, Md = [dev_f32(W0)], [torch.zeros(shape, device="cuda")]
+    ws = torch.empty(ma.muon_workspace_bytes(1, *shape, hp), dtype=torch.uint8, device="cuda")
+    ma.muon_step_batched(Wd, [dev_grad(g, "bf16")], Md, hp, ws)
+    torch.cuda.synchronize()
+    assert ma.ma_device_status() == ma.MA_OK
+    rw, _ = oracle.muon_update(W0, g, np.zeros(shape), f32(0.02), f32(0.95), f32(0.01), eps=f32(1e-7))
+    check_muon(W0, host(Wd[0]), rw, f32(0.02), f32(0.01), TOL_BF16, what=str(shape))
