@@ -7,7 +7,12 @@
   than 256 matrices: results bit-identical to the unsplit plan;
 * 1 and 16 Newton-Schulz iterations;
 * resume: k steps, state copied into fresh buffers, more steps, bit for bit;
-* fp32 mode on larger matrices (1e-5).
+* fp32 mode on larger matrices (1e-5);
+* shared Newton-Schulz launches (grouped buckets) against one call per bucket,
+  bit for bit;
+* a muon_step_batched call beyond 4 GiB of workspace (run as sub-batches)
+  against two smaller calls, bit for bit;
+* degenerate shapes: a single row, 8 x 8, very tall and very wide matrices.
 """
 import numpy as np
 import pytest
