@@ -126,31 +126,6 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
         : "memory");
 }
 
-// 3-D tiled bulk tensor store shared -> global (out-of-bounds parts of the box
-// are not written), tracked by the issuing thread's bulk async-group.
-__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* smem_src, int c0, int c1, int c2) {
-    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
-                     reinterpret_cast<uint64_t>(map)),
-                 "r"(smem_u32(smem_src)), "r"(c0), "r"(c1), "r"(c2)
-                 : "memory");
-}
-
-// Untiled bulk copy global -> this CTA's shared memory of `bytes` (a multiple
-// of 16, both addresses 16-byte aligned), completing on `bar`.
-__device__ __forceinline__ void bulk_load(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
-    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                     smem_u32(smem_dst)),
-                 "l"(reinterpret_cast<uint64_t>(gsrc)), "r"(bytes), "r"(smem_u32(bar))
-                 : "memory");
-}
-
-// Untiled bulk copy shared -> global, tracked by the issuing thread's bulk async-group.
-__device__ __forceinline__ void bulk_store(void* gdst, const void* smem_src, uint32_t bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(gdst)),
-                 "r"(smem_u32(smem_src)), "r"(bytes)
-                 : "memory");
-}
-
 // 16-byte asynchronous copy global -> shared by this thread (cached in L2 only).
 __device__ __forceinline__ void cp_async16(void* smem_dst, const void* gsrc) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)),
@@ -352,7 +327,9 @@ __device__ __forceinline__ void tma_load_3d_hint(void* smem_dst, const CUtensorM
         : "memory");
 }
 
-// tma_store_3d with an L2 eviction-priority policy.
+// 3-D tiled bulk tensor store shared -> global (out-of-bounds parts of the box
+// are not written), tracked by the issuing thread's bulk async-group, with an
+// L2 eviction-priority policy.
 __device__ __forceinline__ void tma_store_3d_hint(const CUtensorMap* map, const void* smem_src, int c0, int c1, int c2,
                                                   uint64_t policy) {
     asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group.L2::cache_hint [%0, {%2, %3, %4}], [%1], %5;" ::"l"(
