@@ -148,6 +148,21 @@ def muon_heads_by_columns(W, g, m, lr, beta, weight_decay, nesterov=True, steps=
     return W * (1 - lr * weight_decay) - lr * O, m_new
 
 
+def muon_cautious_inverted(W, g, m, lr, beta, weight_decay, nesterov=True, steps=5, coeffs=(CUBIC,), eps=1e-7,
+                           scale_mode=0, heads=1, cautious=False):
+    if not cautious:
+        return oracle_muon_update(W, g, m, lr, beta, weight_decay, nesterov, steps, coeffs, eps, scale_mode, heads)
+    Wn, mn = oracle_muon_update(W, g, m, lr, beta, 0.0, nesterov, steps, coeffs, eps, scale_mode, heads)
+    W = np.asarray(W, dtype=np.float64)
+    O = (W - Wn) / lr  # the scaled update
+    return W - lr * weight_decay * W * (O * W < 0) - lr * O, mn  # decays where the signs differ
+
+
+def muon_cautious_ignored(W, g, m, lr, beta, weight_decay, nesterov=True, steps=5, coeffs=(CUBIC,), eps=1e-7,
+                          scale_mode=0, heads=1, cautious=False):
+    return oracle_muon_update(W, g, m, lr, beta, weight_decay, nesterov, steps, coeffs, eps, scale_mode, heads)
+
+
 def kind_embed_to_muon(ndim, role):
     if ndim == 2 and role == oracle.ROLE_EMBED:
         return oracle.KIND_MUON
@@ -179,6 +194,7 @@ ADAMW_PINS = [(pins.test_adamw_closed_form_constant_grad, dict(wd=wd, gscale=gs)
               for wd in (0.0, 0.3) for gs in (1e-3, 1e-9)] + [(pins.test_adamw_first_step_is_sign_like, {})]
 MUON_PINS = [(pins.test_muon_one_step_closed_form, dict(shape=s, heads=h, nesterov=True, mode=0))
              for s, h in [((16, 40), 1), ((40, 16), 1), ((32, 24), 2)]] + [(pins.test_shape_scale_values, {})]
+CAUTIOUS_PINS = [(pins.test_cautious_decay_closed_form, dict(shape=s)) for s in [(16, 40), (40, 16)]]
 PART_PINS = [(pins.test_partition_rules, {}),
              (pins.test_partition_counts_and_exactly_once, dict(name="7b", muon=224, adamw=67, buckets=3))]
 
@@ -199,6 +215,8 @@ MUTATIONS = [
     ("shape_scale", scale_inverted, MUON_PINS),
     ("muon_update", muon_decay_no_lr, MUON_PINS),
     ("muon_update", muon_heads_by_columns, MUON_PINS),
+    ("muon_update", muon_cautious_inverted, CAUTIOUS_PINS),
+    ("muon_update", muon_cautious_ignored, CAUTIOUS_PINS),
     ("kind_of", kind_embed_to_muon, PART_PINS),
 ]
 
