@@ -1324,8 +1324,8 @@ int muonadamw_step_from_host(ma_plan_t* plan, const ma_group_t* groups, const vo
         if (tensor_numel(plan->t[i]) > 0 && !host_grads[i]) return MA_ERR_NULL;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(copy_stream);
-    // Muon sub-batches first (the first one small, so the compute starts early),
-    // the AdamW tensors last: every later copy overlaps earlier compute.
+    // Muon sub-batches first (2, 4, 8, ... matrices, so the compute starts
+    // early), the AdamW tensors last: every later copy overlaps earlier compute.
     const std::vector<Segment> segs = step_segments(plan, groups, kFromHostFirstBatch, kFromHostBatch, true, 0);
     while (plan->events.size() < segs.size() + 1) {
         cudaEvent_t e;
