@@ -36,10 +36,11 @@ MAX_BATCH = 256
 
 
 class LibraryMissing(RuntimeError):
-    pass
+    """The compiled library is absent or cannot be loaded (there is no CPU fallback)."""
 
 
 class MAError(RuntimeError):
+    """A C entry point returned a nonzero status; ``code`` holds it."""
     def __init__(self, code: int, what: str = ""):
         self.code = int(code)
         msg = _lib_status_string(code)
@@ -49,6 +50,8 @@ class MAError(RuntimeError):
 # ---------------------------------------------------------------------------- structs (mirror muonadamw.h)
 
 class MuonHParams(ctypes.Structure):
+    """ma_muon_hparams_t: Muon hyperparameters (lr, beta, weight decay, eps, Nesterov,
+    Newton-Schulz schedule, scale mode, heads, precision, cautious decay)."""
     _fields_ = [("lr", ctypes.c_float), ("beta", ctypes.c_float), ("weight_decay", ctypes.c_float),
                 ("eps", ctypes.c_float), ("nesterov", ctypes.c_int32), ("ns_steps", ctypes.c_int32),
                 ("n_coeffs", ctypes.c_int32), ("coeffs", (ctypes.c_float * 3) * MAX_NS_STEPS),
@@ -57,15 +60,18 @@ class MuonHParams(ctypes.Structure):
 
 
 class AdamWHParams(ctypes.Structure):
+    """ma_adamw_hparams_t: AdamW hyperparameters and the 1-based step being taken."""
     _fields_ = [("lr", ctypes.c_float), ("beta1", ctypes.c_float), ("beta2", ctypes.c_float),
                 ("eps", ctypes.c_float), ("weight_decay", ctypes.c_float), ("step", ctypes.c_int64)]
 
 
 class Group(ctypes.Structure):
+    """ma_group_t: one parameter group, Muon or AdamW by ``kind``."""
     _fields_ = [("kind", ctypes.c_int32), ("muon", MuonHParams), ("adamw", AdamWHParams)]
 
 
 class Tensor(ctypes.Structure):
+    """ma_tensor_t: one tensor of the table (device pointers, gradient dtype, shape, role, group)."""
     _fields_ = [("param", ctypes.c_void_p), ("grad", ctypes.c_void_p), ("grad_dtype", ctypes.c_int32),
                 ("state0", ctypes.c_void_p), ("state1", ctypes.c_void_p), ("ndim", ctypes.c_int32),
                 ("shape", ctypes.c_int64 * 2), ("role", ctypes.c_int32), ("group", ctypes.c_int32)]
@@ -179,6 +185,7 @@ def _dtype_code(t) -> int:
 
 def muon_hparams(lr=0.02, beta=0.95, weight_decay=0.01, eps=1e-7, nesterov=True, ns_steps=5,
                  coeffs=((1.5, -0.5, 0.0),), scale_mode=0, heads=1, precision=0, cautious=False) -> MuonHParams:
+    """Build Muon hyperparameters; ``coeffs`` is one (a, b, c) triple for every iteration or one per iteration."""
     hp = MuonHParams()
     hp.lr, hp.beta, hp.weight_decay, hp.eps = lr, beta, weight_decay, eps
     hp.nesterov, hp.ns_steps, hp.n_coeffs = int(bool(nesterov)), int(ns_steps), len(coeffs)
@@ -192,6 +199,7 @@ def muon_hparams(lr=0.02, beta=0.95, weight_decay=0.01, eps=1e-7, nesterov=True,
 
 
 def adamw_hparams(lr=0.02, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.01, step=1) -> AdamWHParams:
+    """Build AdamW hyperparameters."""
     hp = AdamWHParams()
     hp.lr, hp.beta1, hp.beta2, hp.eps, hp.weight_decay, hp.step = lr, beta1, beta2, eps, weight_decay, int(step)
     return hp
@@ -200,6 +208,7 @@ def adamw_hparams(lr=0.02, beta1=0.9, beta2=0.95, eps=1e-8, weight_decay=0.01, s
 # ---------------------------------------------------------------------------- entry points
 
 def ma_partition(tensors: Sequence[Tensor]) -> list:
+    """Kind (MA_MUON or MA_ADAMW) of each tensor descriptor, by rank and role (host-only)."""
     n = len(tensors)
     arr = (Tensor * max(1, n))(*tensors)
     out = (ctypes.c_int32 * max(1, n))()
@@ -208,6 +217,7 @@ def ma_partition(tensors: Sequence[Tensor]) -> list:
 
 
 def ma_assign_owners(tensors: Sequence[Tensor], groups: Sequence[Group], world_size: int) -> list:
+    """Owner rank of each tensor for a sharded data-parallel step over ``world_size`` ranks (host-only)."""
     n = len(tensors)
     arr = (Tensor * max(1, n))(*tensors)
     garr = (Group * max(1, len(groups)))(*groups)
@@ -217,6 +227,7 @@ def ma_assign_owners(tensors: Sequence[Tensor], groups: Sequence[Group], world_s
 
 
 def muon_workspace_bytes(batch: int, R: int, C: int, hp: MuonHParams) -> int:
+    """Workspace bytes muon_step_batched needs for ``batch`` R x C matrices."""
     v = lib().muon_workspace_bytes(int(batch), int(R), int(C), ctypes.byref(hp))
     if v == ctypes.c_size_t(-1).value:
         raise MAError(MA_ERR_ARG, "muon_workspace_bytes")
@@ -262,6 +273,7 @@ def muon_step_batched_noalloc(W, G, M, hp: MuonHParams, stream=None, gdt: int | 
 
 
 def ns_iterate_workspace_bytes(batch: int, m: int, n: int) -> int:
+    """Workspace bytes ns_iterate_bf16 needs for ``batch`` m x n matrices."""
     return int(lib().ns_iterate_workspace_bytes(int(batch), int(m), int(n)))
 
 
@@ -277,6 +289,7 @@ def ns_iterate_bf16(X_in, X_out, coeffs, steps: int, ws, ws_bytes: int | None = 
 
 
 def adamw_step_fused(P, G, M, V, hp: AdamWHParams, stream=None, gdt: int | None = None, numel=None) -> None:
+    """One multi-tensor AdamW step over parallel lists of fp32 params, gradients, exp_avg and exp_avg_sq."""
     n = len(P)
     if gdt is None:
         gdt = _dtype_code(G[0]) if n else MA_F32
@@ -288,6 +301,7 @@ def adamw_step_fused(P, G, M, V, hp: AdamWHParams, stream=None, gdt: int | None 
 
 
 def ma_plan_create(tensors: Sequence[Tensor], groups: Sequence[Group], ws_cap: int = 0):
+    """Plan a parameter table; returns (plan handle, workspace bytes the step needs)."""
     n = len(tensors)
     arr = (Tensor * max(1, n))(*tensors)
     garr = (Group * max(1, len(groups)))(*groups)
@@ -298,6 +312,7 @@ def ma_plan_create(tensors: Sequence[Tensor], groups: Sequence[Group], ws_cap: i
 
 
 def muonadamw_step(plan, groups: Sequence[Group], ws, ws_bytes: int, stream=None) -> None:
+    """One MuonAdamW step over the planned table, gradients already on the device."""
     garr = (Group * max(1, len(groups)))(*groups)
     _check(lib().muonadamw_step(plan, garr, _ptr(ws), int(ws_bytes), _stream(stream)), "muonadamw_step")
 
@@ -332,10 +347,12 @@ def muonadamw_step_from_host(plan, groups: Sequence[Group], host_grads, ws, ws_b
 
 
 def ma_plan_destroy(plan) -> None:
+    """Free a plan (and its CUDA graph, if one was captured)."""
     lib().ma_plan_destroy(plan)
 
 
 def ma_device_status(stream=None, reset: bool = True) -> int:
+    """Wait for ``stream``, then read (and by default reset) this device's status word."""
     return int(lib().ma_device_status(_stream(stream), int(bool(reset))))
 
 
@@ -345,10 +362,12 @@ def ma_device_status_async(host_dst, stream=None) -> None:
 
 
 def ma_set_wait_limit_ns(limit_ns: int) -> None:
+    """Time limit of the kernels' bounded waits, in nanoseconds (default 2 s)."""
     _check(lib().ma_set_wait_limit_ns(int(limit_ns)), "ma_set_wait_limit_ns")
 
 
 def ma_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
+    """Launch a block whose wait can only time out; the status word must then read MA_ERR_TIMEOUT."""
     _check(lib().ma_selftest_wait_timeout(int(limit_ns), _stream(stream)), "ma_selftest_wait_timeout")
 
 
@@ -356,6 +375,7 @@ PROF_CLASSES = ("adamw", "momentum", "finalize", "ns_gram", "ns_apply", "ns_gram
 
 
 def ma_profile_enable(on: bool) -> None:
+    """Bracket every later launch of this thread with CUDA events (ma_profile_collect reads them)."""
     _check(lib().ma_profile_enable(int(bool(on))), "ma_profile_enable")
 
 
