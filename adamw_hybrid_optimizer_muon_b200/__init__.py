@@ -16,10 +16,11 @@ __all__ = [
     "LibraryMissing", "MAError", "lib", "MuonHParams", "AdamWHParams", "Group", "Tensor",
     "MA_OK", "MA_F32", "MA_BF16", "MA_MUON", "MA_ADAMW", "ROLE_HIDDEN", "ROLE_EMBED", "ROLE_UNEMBED",
     "ROLE_FORCE_ADAMW", "ma_partition", "ma_assign_owners", "muon_workspace_bytes", "muon_step_batched",
-    "ns_iterate_workspace_bytes", "ns_iterate_bf16", "adamw_step_fused", "ma_plan_create", "muonadamw_step", "muonadamw_step_graph", "ma_plan_describe",
-    "ma_plan_destroy", "ma_device_status", "ma_device_status_async", "ma_set_wait_limit_ns", "ma_selftest_wait_timeout", "Plan",
-    "MuonAdamW", "muon_hparams", "adamw_hparams", "ma_profile_enable", "ma_profile_collect", "PROF_CLASSES",
-    "muon_step_batched_noalloc", "STATIC_SCRATCH_BYTES", "muonadamw_step_from_host",
+    "muon_step_batched_noalloc", "STATIC_SCRATCH_BYTES", "ns_iterate_workspace_bytes", "ns_iterate_bf16",
+    "adamw_step_fused", "ma_plan_create", "muonadamw_step", "muonadamw_step_graph", "muonadamw_step_from_host",
+    "ma_plan_describe", "ma_plan_destroy", "ma_device_status", "ma_device_status_async", "ma_set_wait_limit_ns",
+    "ma_selftest_wait_timeout", "ma_profile_enable", "ma_profile_collect", "PROF_CLASSES", "Plan", "MuonAdamW",
+    "muon_hparams", "adamw_hparams",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
