@@ -15,12 +15,13 @@ from typing import Sequence
 __all__ = [
     "LibraryMissing", "MAError", "lib", "MuonHParams", "AdamWHParams", "Group", "Tensor",
     "MA_OK", "MA_F32", "MA_BF16", "MA_MUON", "MA_ADAMW", "ROLE_HIDDEN", "ROLE_EMBED", "ROLE_UNEMBED",
-    "ROLE_FORCE_ADAMW", "ma_partition", "ma_assign_owners", "muon_workspace_bytes", "muon_step_batched",
+    "ROLE_FORCE_ADAMW", "ShardSlot", "ShardBucket", "SHARD_ALIGN", "ma_partition", "ma_assign_owners",
+    "ma_shard_layout", "muon_workspace_bytes", "muon_step_batched",
     "muon_step_batched_noalloc", "STATIC_SCRATCH_BYTES", "ns_iterate_workspace_bytes", "ns_iterate_bf16",
     "adamw_step_fused", "ma_plan_create", "muonadamw_step", "muonadamw_step_graph", "muonadamw_step_from_host",
     "ma_plan_describe", "ma_plan_destroy", "ma_device_status", "ma_device_status_async", "ma_set_wait_limit_ns",
-    "ma_selftest_wait_timeout", "ma_profile_enable", "ma_profile_collect", "PROF_CLASSES", "Plan", "MuonAdamW",
-    "muon_hparams", "adamw_hparams",
+    "ma_selftest_wait_timeout", "ma_profile_enable", "ma_profile_collect", "PROF_CLASSES", "group_table", "Plan",
+    "MuonAdamW", "muon_hparams", "adamw_hparams",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -78,6 +79,17 @@ class Tensor(ctypes.Structure):
                 ("shape", ctypes.c_int64 * 2), ("role", ctypes.c_int32), ("group", ctypes.c_int32)]
 
 
+class ShardSlot(ctypes.Structure):
+    """ma_shard_slot_t: where a tensor sits in the flat buffers of a sharded step."""
+    _fields_ = [("bucket", ctypes.c_int32), ("owner", ctypes.c_int32), ("offset", ctypes.c_int64)]
+
+
+class ShardBucket(ctypes.Structure):
+    """ma_shard_bucket_t: one bucket of a sharded step (kind, tensors, start, per-rank segment)."""
+    _fields_ = [("kind", ctypes.c_int32), ("count", ctypes.c_int32), ("start", ctypes.c_int64),
+                ("seg", ctypes.c_int64)]
+
+
 _LIB = None
 
 
@@ -101,6 +113,9 @@ def lib() -> ctypes.CDLL:
         "ma_partition": (i32, [ctypes.POINTER(Tensor), i32, ctypes.POINTER(ctypes.c_int32)]),
         "ma_assign_owners": (i32, [ctypes.POINTER(Tensor), i32, ctypes.POINTER(Group), i32, i32,
                                    ctypes.POINTER(ctypes.c_int32)]),
+        "ma_shard_layout": (i32, [ctypes.POINTER(Tensor), i32, ctypes.POINTER(Group), i32, i32, i64,
+                                  ctypes.POINTER(ShardSlot), ctypes.POINTER(ShardBucket), ctypes.POINTER(i32),
+                                  ctypes.POINTER(i64)]),
         "muon_workspace_bytes": (sz, [i32, i64, i64, ctypes.POINTER(MuonHParams)]),
         "muon_step_batched": (i32, [i32, i64, i64, pp, pp, i32, pp, ctypes.POINTER(MuonHParams), vp, sz, vp]),
         "ns_iterate_workspace_bytes": (sz, [i32, i64, i64]),
@@ -129,7 +144,7 @@ def lib() -> ctypes.CDLL:
         fn = getattr(L, name)
         fn.restype = res
         fn.argtypes = args
-    for which, cls in enumerate((Tensor, Group, MuonHParams, AdamWHParams)):
+    for which, cls in enumerate((Tensor, Group, MuonHParams, AdamWHParams, ShardSlot, ShardBucket)):
         if L.ma_struct_size(which) != ctypes.sizeof(cls):
             raise LibraryMissing(f"ABI mismatch for {cls.__name__}: C {L.ma_struct_size(which)} "
                                  f"vs Python {ctypes.sizeof(cls)}")
@@ -225,6 +240,29 @@ def ma_assign_owners(tensors: Sequence[Tensor], groups: Sequence[Group], world_s
     out = (ctypes.c_int32 * max(1, n))()
     _check(lib().ma_assign_owners(arr, n, garr, len(groups), int(world_size), out), "ma_assign_owners")
     return [int(out[i]) for i in range(n)]
+
+
+SHARD_ALIGN = 64  # MA_SHARD_ALIGN
+
+
+def ma_shard_layout(tensors: Sequence[Tensor], groups: Sequence[Group], world_size: int, seg_cap: int):
+    """Flat-buffer layout of a sharded data-parallel step (host-only).
+
+    Returns (slots, buckets, total): per tensor a (bucket, owner, offset) tuple
+    (owner -1 for AdamW tensors, which are split by element range), per bucket
+    a (kind, count, start, seg) tuple, and the flat buffers' length in elements.
+    """
+    n = len(tensors)
+    arr = (Tensor * max(1, n))(*tensors)
+    garr = (Group * max(1, len(groups)))(*groups)
+    slots = (ShardSlot * max(1, n))()
+    buckets = (ShardBucket * max(1, n))()
+    nb, total = ctypes.c_int(0), ctypes.c_int64(0)
+    _check(lib().ma_shard_layout(arr, n, garr, len(groups), int(world_size), int(seg_cap), slots, buckets,
+                                 ctypes.byref(nb), ctypes.byref(total)), "ma_shard_layout")
+    return ([(int(s.bucket), int(s.owner), int(s.offset)) for s in slots[:n]],
+            [(int(b.kind), int(b.count), int(b.start), int(b.seg)) for b in buckets[:nb.value]],
+            int(total.value))
 
 
 def muon_workspace_bytes(batch: int, R: int, C: int, hp: MuonHParams) -> int:
@@ -392,6 +430,20 @@ def ma_profile_collect() -> dict:
 
 # ---------------------------------------------------------------------------- user-level wrappers
 
+def group_table(groups) -> list:
+    """ma_group_t entries from ("muon", MuonHParams) / ("adamw", AdamWHParams) pairs."""
+    table = []
+    for kind, hp in groups:
+        g = Group()
+        g.kind = MA_MUON if kind == "muon" else MA_ADAMW
+        if g.kind == MA_MUON:
+            g.muon = hp
+        else:
+            g.adamw = hp
+        table.append(g)
+    return table
+
+
 class Plan:
     """Owns an ma_plan_t and its device workspace (a torch uint8 buffer)."""
 
@@ -449,15 +501,7 @@ class MuonAdamW:
     def __init__(self, params, groups, ws_cap: int = 0):
         import torch
         self.entries = list(params)
-        self.groups = []
-        for kind, hp in groups:
-            g = Group()
-            g.kind = MA_MUON if kind == "muon" else MA_ADAMW
-            if g.kind == MA_MUON:
-                g.muon = hp
-            else:
-                g.adamw = hp
-            self.groups.append(g)
+        self.groups = group_table(groups)
         self.state = []
         self.step_count = 0
         self._ws_cap = ws_cap

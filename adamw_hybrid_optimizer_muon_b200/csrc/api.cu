@@ -804,6 +804,8 @@ size_t ma_struct_size(int which) {
         case 1: return sizeof(ma_group_t);
         case 2: return sizeof(ma_muon_hparams_t);
         case 3: return sizeof(ma_adamw_hparams_t);
+        case 4: return sizeof(ma_shard_slot_t);
+        case 5: return sizeof(ma_shard_bucket_t);
         default: return 0;
     }
 }
@@ -868,6 +870,186 @@ int ma_assign_owners(const ma_tensor_t* t, int n, const ma_group_t* groups, int 
             load[best] += cost[i];
         }
     }
+    return MA_OK;
+}
+
+namespace {
+
+int64_t shard_align(int64_t x) { return (x + MA_SHARD_ALIGN - 1) / MA_SHARD_ALIGN * MA_SHARD_ALIGN; }
+
+struct ShardBucket {
+    int first;                 // lowest tensor index in the bucket (orders the buckets)
+    int kind;
+    std::vector<int> members;  // tensor indices, ascending
+};
+
+}  // namespace
+
+int ma_shard_layout(const ma_tensor_t* t, int n, const ma_group_t* groups, int ngroups, int world_size,
+                    int64_t seg_cap, ma_shard_slot_t* slots, ma_shard_bucket_t* buckets, int* nbuckets,
+                    int64_t* total) {
+    if (n < 0 || ngroups < 0) return MA_ERR_SHAPE;
+    if (world_size < 1 || seg_cap < 1) return MA_ERR_ARG;
+    if (!nbuckets || !total) return MA_ERR_NULL;
+    *nbuckets = 0;
+    *total = 0;
+    if (n == 0) return MA_OK;
+    if (!t || !slots || !buckets || !groups) return MA_ERR_NULL;
+    std::vector<int32_t> kind(n);
+    int st = ma_partition(t, n, kind.data());
+    if (st) return st;
+    const int64_t kMaxElems = int64_t(1) << 50;
+    std::vector<int64_t> numel(n, 1);
+    for (int i = 0; i < n; ++i) {
+        if (t[i].group < 0 || t[i].group >= ngroups) return MA_ERR_ARG;
+        if (groups[t[i].group].kind != kind[i]) return MA_ERR_ARG;
+        for (int d = 0; d < t[i].ndim; ++d) {
+            if (t[i].shape[d] < 0 || t[i].shape[d] > kMaxElems) return MA_ERR_SHAPE;
+            numel[i] *= t[i].shape[d];
+            if (numel[i] > kMaxElems) return MA_ERR_SHAPE;
+        }
+    }
+
+    // Muon, first pass: matrices of one shape and group, in order of
+    // appearance, are cut into buckets of world_size * k matrices, k = as many
+    // as fit one rank's segment cap (at least one). Matrix j of such a bucket
+    // belongs to rank j % world_size, so every segment holds k matrices. The
+    // last c % world_size matrices of a class of c are left over.
+    std::vector<ShardBucket> bl;
+    std::vector<int> leftover;
+    std::vector<bool> placed(n, false);
+    for (int i = 0; i < n; ++i) {
+        if (kind[i] != MA_MUON || placed[i]) continue;
+        std::vector<int> cls;
+        for (int j = i; j < n; ++j)
+            if (kind[j] == MA_MUON && !placed[j] && t[j].shape[0] == t[i].shape[0] &&
+                t[j].shape[1] == t[i].shape[1] && t[j].group == t[i].group) {
+                cls.push_back(j);
+                placed[j] = true;
+            }
+        const size_t full = cls.size() / (size_t)world_size * (size_t)world_size;
+        const int64_t a = shard_align(numel[i]);
+        const int64_t per_rank = std::min<int64_t>(n, std::max<int64_t>(1, a > 0 ? seg_cap / a : seg_cap));
+        const size_t k = (size_t)per_rank * (size_t)world_size;
+        for (size_t b = 0; b < full; b += k) {
+            ShardBucket sb{cls[b], MA_MUON, {}};
+            for (size_t j = b; j < std::min(full, b + k); ++j) sb.members.push_back(cls[j]);
+            bl.push_back(std::move(sb));
+        }
+        for (size_t j = full; j < cls.size(); ++j) leftover.push_back(cls[j]);
+    }
+    // Muon, second pass: the leftovers, in order of appearance, fill mixed
+    // buckets; one closes before the matrix that would take the bucket's
+    // average per-rank share past the cap. Their owners are set below,
+    // largest matrix first onto the least-loaded rank.
+    std::sort(leftover.begin(), leftover.end());
+    {
+        ShardBucket cur{-1, MA_MUON, {}};
+        int64_t run = 0;
+        for (int i : leftover) {
+            const int64_t next = run + shard_align(numel[i]);
+            if (!cur.members.empty() && (next + world_size - 1) / world_size > seg_cap) {
+                bl.push_back(std::move(cur));
+                cur = ShardBucket{-1, MA_MUON, {}};
+                run = 0;
+            }
+            if (cur.members.empty()) cur.first = i;
+            cur.members.push_back(i);
+            run += shard_align(numel[i]);
+            if (run > kMaxElems) return MA_ERR_SHAPE;
+        }
+        if (!cur.members.empty()) bl.push_back(std::move(cur));
+    }
+    // AdamW: tensors in order of appearance; a bucket closes before the
+    // tensor that would take its per-rank share past the cap (a bucket always
+    // takes at least one tensor). Its elements are split evenly by range.
+    {
+        ShardBucket cur{-1, MA_ADAMW, {}};
+        int64_t run = 0;
+        for (int i = 0; i < n; ++i) {
+            if (kind[i] != MA_ADAMW) continue;
+            const int64_t next = run + shard_align(numel[i]);
+            if (!cur.members.empty() && (next + world_size - 1) / world_size > seg_cap) {
+                bl.push_back(std::move(cur));
+                cur = ShardBucket{-1, MA_ADAMW, {}};
+                run = 0;
+            }
+            if (cur.members.empty()) cur.first = i;
+            cur.members.push_back(i);
+            run += shard_align(numel[i]);
+            if (run > kMaxElems) return MA_ERR_SHAPE;
+        }
+        if (!cur.members.empty()) bl.push_back(std::move(cur));
+    }
+    std::stable_sort(bl.begin(), bl.end(), [](const ShardBucket& x, const ShardBucket& y) { return x.first < y.first; });
+
+    // Owners and segment lengths first, so that an oversized layout is
+    // refused before any output is written. A bucket whose matrices all share
+    // one shape and whose count is a multiple of world_size is dealt round
+    // robin; any other Muon bucket is packed largest first onto the
+    // least-loaded rank (ties: lower rank, then lower tensor index). Within a
+    // segment, matrices sit in order of appearance.
+    std::vector<int> owner(n, -1);
+    std::vector<int64_t> segs(bl.size());
+    int64_t end = 0;
+    for (size_t b = 0; b < bl.size(); ++b) {
+        const ShardBucket& sb = bl[b];
+        if (sb.kind == MA_MUON) {
+            bool uniform = sb.members.size() % (size_t)world_size == 0;
+            for (int i : sb.members)
+                uniform = uniform && t[i].shape[0] == t[sb.members[0]].shape[0] &&
+                          t[i].shape[1] == t[sb.members[0]].shape[1];
+            std::vector<int64_t> load(world_size, 0);
+            if (uniform) {
+                for (size_t j = 0; j < sb.members.size(); ++j) {
+                    owner[sb.members[j]] = (int)(j % (size_t)world_size);
+                    load[j % (size_t)world_size] += shard_align(numel[sb.members[j]]);
+                }
+            } else {
+                std::vector<int> order = sb.members;
+                std::stable_sort(order.begin(), order.end(),
+                                 [&](int x, int y) { return numel[x] > numel[y]; });
+                for (int i : order) {
+                    int r = 0;
+                    for (int q = 1; q < world_size; ++q)
+                        if (load[q] < load[r]) r = q;
+                    owner[i] = r;
+                    load[r] += shard_align(numel[i]);
+                }
+            }
+            segs[b] = *std::max_element(load.begin(), load.end());
+        } else {
+            int64_t len = 0;
+            for (int i : sb.members) len += shard_align(numel[i]);
+            segs[b] = shard_align((len + world_size - 1) / world_size);
+        }
+        if (segs[b] > kMaxElems / world_size) return MA_ERR_SHAPE;
+        end += segs[b] * world_size;
+        if (end > kMaxElems) return MA_ERR_SHAPE;
+    }
+    int64_t start = 0;
+    for (size_t b = 0; b < bl.size(); ++b) {
+        const ShardBucket& sb = bl[b];
+        const int64_t seg = segs[b];
+        if (sb.kind == MA_MUON) {
+            std::vector<int64_t> fill(world_size, 0);
+            for (int i : sb.members) {
+                const int r = owner[i];
+                slots[i] = ma_shard_slot_t{(int32_t)b, r, start + r * seg + fill[r]};
+                fill[r] += shard_align(numel[i]);
+            }
+        } else {
+            int64_t off = 0;
+            for (int i : sb.members) {
+                slots[i] = ma_shard_slot_t{(int32_t)b, -1, start + off};
+                off += shard_align(numel[i]);
+            }
+        }
+        buckets[b] = ma_shard_bucket_t{sb.kind, (int32_t)sb.members.size(), start, seg};
+        start += seg * world_size;
+    }
+    *nbuckets = (int)bl.size();
+    *total = start;
     return MA_OK;
 }
 

@@ -2,7 +2,8 @@
 """Benchmark of one MuonAdamW optimizer step on a B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 7b|d20|square|aspect|tiny|square8]
-                    [--impl ours|reference] [--no-e2e] [--no-cpu-baseline] [--graph] [--coeffs a,b,c;...]
+                    [--impl ours|reference] [--no-e2e] [--no-cpu-baseline] [--graph] [--sharded]
+                    [--coeffs a,b,c;...]
 
 A step is one muonadamw_step over a synthetic parameter set (with --graph,
 the same step replayed from a CUDA graph). Each step runs AdamW on every
@@ -18,6 +19,10 @@ end-to-end number through the C ABI with host buffers, the roofline of the
 dominant kernel (Newton-Schulz GEMMs, measured live with CUDA events on their
 launch stream), the clocks seen during the timed region, and a CPU baseline
 (the fp64 oracle on a bounded sample, host cores).
+
+``--sharded`` times the sharded data-parallel step instead (DistMuonAdamW:
+the ranks share one step of the set, so its scaling is strong; with one GPU
+the collectives move each bucket onto itself).
 
 ``--impl reference`` times that same oracle (there is no other implementation
 of this method to run) on a bounded sample per step and prints the same line
@@ -56,6 +61,15 @@ def env_int(name, default):
         return int(os.environ.get(name, default))
     except ValueError:
         return default
+
+
+def free_port():
+    import socket
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
 
 
 def load_peaks():
@@ -266,6 +280,9 @@ def main():
     ap.add_argument("--graph", action="store_true",
                     help="time the step replayed from a CUDA graph (muonadamw_step_graph); the per-kernel "
                          "profile then comes from an extra, untimed pass of eager steps")
+    ap.add_argument("--sharded", action="store_true",
+                    help="time the sharded data-parallel step (DistMuonAdamW: reduce-scatter of the gradients, "
+                         "each rank's share of the update, all-gather of the parameters) instead of N replicas")
     ap.add_argument("--coeffs", default=None,
                     help="Newton-Schulz polynomial per iteration, 'a,b,c[;a,b,c...]' (default: the cubic 1.5,-0.5,0)")
     args = ap.parse_args()
@@ -281,8 +298,13 @@ def main():
 
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    if args.sharded and args.graph:
+        raise SystemExit("--sharded steps run collectives and are not captured in a graph")
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    elif args.sharded:  # one rank: a process group of its own
+        dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{free_port()}", rank=0, world_size=1,
+                                timeout=datetime.timedelta(seconds=300), device_id=dev)
 
     def barrier():
         if world > 1:
@@ -307,11 +329,29 @@ def main():
         else:
             h = g.adamw
             groups.append(("adamw", ma.adamw_hparams(h.lr, h.beta1, h.beta2, h.eps, h.weight_decay, 1)))
-    opt = ma.MuonAdamW([(p, t.role, t.group) for p, t in zip(params, wl.tensors)], groups)
+    table = [(p, t.role, t.group) for p, t in zip(params, wl.tensors)]
+    if args.sharded:
+        from adamw_hybrid_optimizer_muon_b200.dist import DistMuonAdamW
+        gdts = {g.dtype for g in grads}
+        if len(gdts) != 1:
+            raise SystemExit("--sharded needs one gradient dtype across the workload")
+        opt = DistMuonAdamW(table, groups, grad_dtype=gdts.pop())
+        for gv, g in zip(opt.grads, grads):
+            gv.copy_(g)
+        del grads, params, table
+        grads = None
+
+        def do_step():
+            opt.step()
+    else:
+        opt = ma.MuonAdamW(table, groups)
+
+        def do_step():
+            opt.step(grads, graph=args.graph)
     stream = torch.cuda.current_stream(dev)
 
     for _ in range(args.warmup):
-        opt.step(grads, graph=args.graph)
+        do_step()
     torch.cuda.synchronize(dev)
     st = ma.ma_device_status(stream)
     if st != ma.MA_OK:
@@ -332,7 +372,7 @@ def main():
         for a, b in evs:
             flush.zero_()
             a.record(stream)
-            opt.step(grads, graph=args.graph)
+            do_step()
             b.record(stream)
         torch.cuda.synchronize(dev)
         step_ms = sum(a.elapsed_time(b) for a, b in evs)
@@ -341,7 +381,7 @@ def main():
         t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         t0.record(stream)
         for _ in range(args.steps):
-            opt.step(grads, graph=args.graph)
+            do_step()
         t1.record(stream)
         torch.cuda.synchronize(dev)
         step_ms = t0.elapsed_time(t1)
@@ -364,13 +404,47 @@ def main():
     if st != ma.MA_OK:
         raise SystemExit(f"device status after the timed steps: {st}")
     n_params = wl.numel
-    value = world * n_params / (ms / 1000.0)
+    # replicas: each rank steps its own copy of the set (weak scaling); sharded:
+    # the ranks share one step of the set (strong scaling)
+    jobs = 1 if args.sharded else world
+    value = jobs * n_params / (ms / 1000.0)
 
     # ---- end to end through the public API: every step the gradients come from
     # pinned host memory (copied by the library on its own stream, overlapped with
     # the compute), then the device status word (the step's result) is read back
     e2e = None
-    if not args.no_e2e:
+    if not args.no_e2e and args.sharded:
+        # the gradients of the whole set arrive in the flat gradient buffer from
+        # pinned host memory every step; the status word is read back after it
+        host_flat = torch.empty(opt.flat_grad.shape, dtype=opt.flat_grad.dtype, pin_memory=True)
+        host_flat.copy_(opt.flat_grad)
+        h2d = host_flat.numel() * host_flat.element_size()
+        k_e2e = max(1, min(args.steps, 5))
+        status = torch.full((k_e2e,), -1, dtype=torch.int32, pin_memory=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(k_e2e):
+            opt.flat_grad.copy_(host_flat, non_blocking=True)
+            opt.step()
+            ma.ma_device_status_async(status.data_ptr() + 4 * i, stream)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier()
+        if int(status.abs().max()) != ma.MA_OK:
+            raise SystemExit(f"device status error in the end-to-end loop: {status.tolist()}")
+        ems = e0.elapsed_time(e1) / k_e2e
+        if world > 1:
+            tt = torch.tensor([ems], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ems = float(tt.item())
+        e2e = {"value": n_params / (ems / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": 4, "ms_per_step": ems,
+               "path": "DistMuonAdamW.step after a copy of the flat gradient buffer from pinned host memory; "
+                       "each step's status word read back asynchronously"}
+        del host_flat
+    elif not args.no_e2e:
         host_grads = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in grads]
         for hg, g in zip(host_grads, grads):
             hg.copy_(g)
@@ -439,18 +513,26 @@ def main():
                 d["gbs"] = pc["bytes"] / (pc["ms"] / 1000.0) / 1e9
                 d["frac_hbm"] = d["gbs"] / peaks["hbm_gbs"]
             kernels[c] = d
+        config = workload_config(wl, world)
+        if args.sharded:
+            config["parallelism"] = (f"sharded dp{world}: reduce-scatter, each rank's share of the update, "
+                                     f"all-gather ({len(opt.buckets)} buckets)")
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "strong" if args.sharded else "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,0.02^2) weights, "
-                "N(0,1e-3^2) bf16 grads)", "config": workload_config(wl, world),
+                "N(0,1e-3^2) bf16 grads)", "config": config,
                 "e2e": e2e, "gpu_launches": launches_per_step * args.steps, "roofline": roofline,
                 "kernels": kernels, "clocks": clk,
                 "precision": {"ns_operands": "bf16", "accumulate": "fp32", "state": "fp32"}}
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(wl)
         print(json.dumps(line))
-    opt._plan.close()
-    if world > 1:
+    if args.sharded:
+        opt.close()
+    else:
+        opt._plan.close()
+    if dist.is_initialized():
         dist.destroy_process_group()
     return 0
 

@@ -141,7 +141,8 @@ const char* ma_status_string(int status);
 int ma_version(void);
 
 /* sizeof of the ABI structs, for bindings to check their layouts:
- * 0 ma_tensor_t, 1 ma_group_t, 2 ma_muon_hparams_t, 3 ma_adamw_hparams_t; else 0. */
+ * 0 ma_tensor_t, 1 ma_group_t, 2 ma_muon_hparams_t, 3 ma_adamw_hparams_t,
+ * 4 ma_shard_slot_t, 5 ma_shard_bucket_t; else 0. */
 size_t ma_struct_size(int which);
 
 /* Partition by tensor rank [P1 "Parameter Grouping Strategy"; P4]:
@@ -162,6 +163,62 @@ int ma_partition(const ma_tensor_t* t, int n, int32_t* kind_out);
  * or a bad group index. Host-only, no CUDA call. */
 int ma_assign_owners(const ma_tensor_t* t, int n, const ma_group_t* groups, int ngroups,
                      int world_size, int32_t* owner_out);
+
+/* Flat-buffer layout of a sharded data-parallel step [P1 "Distributed
+ * Training Support": each rank reduces the gradients it needs, updates its
+ * share of the parameters and passes the result on; P3: matrix batches are
+ * independent, and a matrix must be complete on the rank that orthogonalises
+ * it].
+ *
+ * Every rank keeps the parameters (and, with the same element offsets, the
+ * gradients) of the whole model in one flat buffer of `total` elements, cut
+ * into buckets. Bucket b spans [start, start + world_size * seg) and rank r's
+ * segment of it is [start + r * seg, start + (r + 1) * seg): the part that
+ * rank r receives from a reduce-scatter of the bucket's gradients, updates,
+ * and hands to an all-gather of the bucket's parameters.
+ *  - Muon matrices are owned whole. Matrices of one shape and group (in
+ *    order of appearance) fill buckets of world_size * k of them, k as many
+ *    as fit seg_cap (at least one); matrix j of such a bucket belongs to rank
+ *    j % world_size. The last (count % world_size) matrices of each class
+ *    are left over and fill mixed buckets, in order of appearance, each
+ *    closing before the matrix that would take its average per-rank share
+ *    past seg_cap; a mixed bucket is packed largest matrix first onto the
+ *    least-loaded rank (ties: lower rank, then lower index). A Muon segment
+ *    is as long as its bucket's most loaded rank needs; within it, matrices
+ *    sit in order of appearance.
+ *  - An AdamW bucket holds AdamW tensors in order of appearance, laid end to
+ *    end; AdamW is elementwise, so its segments split them by element range
+ *    and a tensor may straddle segments (owner -1).
+ * Buckets are ordered by their first tensor's index. Every tensor offset,
+ * bucket start and segment length is a multiple of MA_SHARD_ALIGN elements,
+ * so every piece a rank updates starts 16-byte aligned for fp32 and bf16.
+ * Padding elements belong to no tensor. An AdamW bucket closes before the
+ * tensor that would take its per-rank share past seg_cap. Every bucket holds
+ * at least one tensor.
+ *  t, groups: host arrays (shape, ndim, role and group are read).
+ *  slots: host array of n entries (out). buckets: host array of at least n
+ *  entries (out); nbuckets, total (out).
+ * Errors: as ma_partition; MA_ERR_ARG for world_size < 1, seg_cap < 1, a bad
+ * group index or a group whose kind differs from the tensor's; MA_ERR_SHAPE
+ * for a negative extent or a layout beyond 2^50 elements. Host-only. */
+#define MA_SHARD_ALIGN 64
+
+typedef struct {
+    int32_t bucket;   /* index of the bucket that holds the tensor        */
+    int32_t owner;    /* owning rank of a Muon matrix; -1 for AdamW       */
+    int64_t offset;   /* element offset of the tensor in the flat buffers */
+} ma_shard_slot_t;
+
+typedef struct {
+    int32_t kind;     /* MA_MUON or MA_ADAMW                              */
+    int32_t count;    /* tensors in the bucket                            */
+    int64_t start;    /* element offset of the bucket                     */
+    int64_t seg;      /* elements of one rank's segment                   */
+} ma_shard_bucket_t;
+
+int ma_shard_layout(const ma_tensor_t* t, int n, const ma_group_t* groups, int ngroups,
+                    int world_size, int64_t seg_cap, ma_shard_slot_t* slots,
+                    ma_shard_bucket_t* buckets, int* nbuckets, int64_t* total);
 
 /* ---------------------------------------------------------------- Muon */
 

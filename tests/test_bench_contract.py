@@ -1,7 +1,8 @@
 """bench.py's JSON line: the keys and types the benchmark contract asks for.
 
 The reference arm (the oracle on the host cores) runs anywhere; the GPU arm
-runs on a B200 only. Both run bench.py as a subprocess on the tiny set.
+(replicas, from a CUDA graph, and the sharded step on one NCCL rank) runs on
+a B200 only. All run bench.py as a subprocess on the tiny set.
 """
 import json
 import os
@@ -73,3 +74,16 @@ def test_gpu_arm_line(graph):
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] > 0
     assert {"sm_mhz", "sm_max_mhz", "reasons"} <= set(d["clocks"])
     assert "L2" in d["config"]["l2"]
+
+
+@pytest.mark.gpu
+def test_gpu_arm_line_sharded():
+    # one NCCL rank: the sharded step (reduce-scatter, local update, all-gather)
+    (line,) = _run(["--workload", "tiny", "--steps", "3", "--warmup", "3", "--sharded", "--no-cpu-baseline"])
+    d = json.loads(line)
+    assert d["scaling"] == "strong" and d["config"]["parallelism"].startswith("sharded dp1")
+    assert d["value"] > 0 and d["n_gpus"] == 1
+    assert d["gpu_launches"] == 3 * 13  # a Muon bucket (12 launches) and an AdamW bucket (1)
+    e = d["e2e"]
+    assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] == 4
+    assert d["roofline"]["achieved"] > 0
