@@ -11,10 +11,11 @@ overlapping the compute. Here the three phases are:
    receives the averaged gradients of its own segment of the bucket; every
    bucket's reduction is queued at once;
 2. as each bucket's reduction completes, the library's MuonAdamW step on
-   that rank's segment: the Muon matrices it owns whole (a matrix must be
-   complete on the rank that orthogonalises it; matrices are independent,
-   per "nemo_automodel.components.optim.muown_triton"), and its element range
-   of the bucket's AdamW tensors (AdamW is elementwise);
+   that rank's segment: the Muon matrices it owns whole (Newton-Schulz mixes
+   all rows of a matrix, and "nemo_automodel.components.optim.muown_triton"
+   treats batched matrices as independent and wants the input axis complete
+   on the rank), and its element range of the bucket's AdamW tensors (AdamW
+   is elementwise);
 3. all-gather of each bucket's updated segments into every rank's replica,
    queued right after that bucket's step, so it overlaps the next bucket's.
 
@@ -211,11 +212,53 @@ class DistMuonAdamW:
 
     def step(self) -> None:
         """One data-parallel step: reduce-scatter, local update, all-gather (all asynchronous on the device)."""
+        self._run(None)
+
+    def step_from_host(self, host_flat: torch.Tensor) -> None:
+        """One step whose gradients come from ``host_flat``, a pinned CPU tensor
+        shaped and typed like ``flat_grad`` (``host_views`` gives its per-tensor
+        views). Each bucket's gradients are copied on a side stream and that
+        bucket's reduce-scatter starts as soon as its copy lands, so the copies
+        overlap the reductions and the updates of the buckets before it."""
+        if host_flat.shape != self.flat_grad.shape or host_flat.dtype != self.flat_grad.dtype:
+            raise ValueError("host_flat must match flat_grad in shape and dtype")
+        self._run(host_flat)
+
+    def host_views(self, host_flat: torch.Tensor) -> list:
+        """Per-tensor views of a flat host gradient buffer (same offsets as ``grads``)."""
+        return [host_flat[off:off + g.numel()].view(g.shape) for g, (_, _, off) in zip(self.grads, self.slots)]
+
+    def _run(self, host_flat) -> None:
         self._advance()
+        cuda = self.flat_grad.is_cuda
+        if not cuda and host_flat is not None:
+            self.flat_grad.copy_(host_flat)
+            host_flat = None
+        side = None
+        if cuda:
+            # the reductions are issued from a side stream, which first waits
+            # for everything queued so far (the gradients' producers, the last
+            # step's reads of flat_grad); NCCL then waits on the side stream
+            # only, so a copy or reduction never waits for an update
+            if getattr(self, "_side", None) is None:
+                self._side = torch.cuda.Stream(device=self.flat_grad.device)
+            side = self._side
+            side.wait_stream(torch.cuda.current_stream(self.flat_grad.device))
         reduces = []
         for bv in self.buckets:
-            reduces.append(dist.reduce_scatter_tensor(bv.grad_shard, bv.grad_bucket, op=dist.ReduceOp.AVG,
-                                                      group=self.pg, async_op=True) if bv.seg else None)
+            if not bv.seg:
+                reduces.append(None)
+                continue
+            if side is None:
+                reduces.append(dist.reduce_scatter_tensor(bv.grad_shard, bv.grad_bucket, op=dist.ReduceOp.AVG,
+                                                          group=self.pg, async_op=True))
+                continue
+            with torch.cuda.stream(side):
+                if host_flat is not None:
+                    n = self.world * bv.seg
+                    bv.grad_bucket.copy_(host_flat[bv.start:bv.start + n], non_blocking=True)
+                reduces.append(dist.reduce_scatter_tensor(bv.grad_shard, bv.grad_bucket, op=dist.ReduceOp.AVG,
+                                                          group=self.pg, async_op=True))
         gathers = []
         for b, bv in enumerate(self.buckets):
             if reduces[b] is not None:

@@ -415,7 +415,9 @@ def main():
     e2e = None
     if not args.no_e2e and args.sharded:
         # the gradients of the whole set arrive in the flat gradient buffer from
-        # pinned host memory every step; the status word is read back after it
+        # pinned host memory every step (bucket by bucket on a side stream, each
+        # bucket's reduce-scatter starting when its copy lands); the status word
+        # is read back after it
         host_flat = torch.empty(opt.flat_grad.shape, dtype=opt.flat_grad.dtype, pin_memory=True)
         host_flat.copy_(opt.flat_grad)
         h2d = host_flat.numel() * host_flat.element_size()
@@ -426,8 +428,7 @@ def main():
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for i in range(k_e2e):
-            opt.flat_grad.copy_(host_flat, non_blocking=True)
-            opt.step()
+            opt.step_from_host(host_flat)
             ma.ma_device_status_async(status.data_ptr() + 4 * i, stream)
         e1.record(stream)
         torch.cuda.synchronize(dev)
@@ -441,8 +442,8 @@ def main():
             ems = float(tt.item())
         e2e = {"value": n_params / (ems / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": 4, "ms_per_step": ems,
-               "path": "DistMuonAdamW.step after a copy of the flat gradient buffer from pinned host memory; "
-                       "each step's status word read back asynchronously"}
+               "path": "DistMuonAdamW.step_from_host (pinned host gradients copied bucket by bucket, overlapped "
+                       "with the reductions and updates; each step's status word read back asynchronously)"}
         del host_flat
     elif not args.no_e2e:
         host_grads = [torch.empty(g.shape, dtype=g.dtype, pin_memory=True) for g in grads]

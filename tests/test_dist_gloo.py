@@ -17,6 +17,7 @@ buckets), a per-head group, an embedding that straddles AdamW segments, 1-D
 and 0-D tensors, and a small segment cap so that there are many buckets.
 The gradients must be left as they were, the initial parameters must come
 from rank 0, and each rank must hold only its share of the optimizer state.
+The second step takes its gradients from a host buffer (step_from_host).
 """
 import datetime
 import os
@@ -280,12 +281,19 @@ def _worker(rank, world, port, q):
         start = [p.clone() for p in params]
         out = {"start": [p.numpy().copy() for p in start], "steps": [], "state_elems": opt.state0.numel(),
                "nbuckets": len(opt.buckets), "pieces": [(pc.index, pc.lo, pc.hi) for pc in opt.pieces()]}
+        host_flat = torch.zeros_like(opt.flat_grad)
         for step in (1, 2):
             G = _grads(step, rank, world)
-            for g, v in zip(opt.grads, G):
-                g.copy_(torch.from_numpy(v))
-            flat_before = opt.flat_grad.clone()
-            opt.step()
+            if step == 1:
+                for g, v in zip(opt.grads, G):
+                    g.copy_(torch.from_numpy(v))
+                flat_before = opt.flat_grad.clone()
+                opt.step()
+            else:  # the second step takes its gradients from a host buffer
+                for h, v in zip(opt.host_views(host_flat), G):
+                    h.copy_(torch.from_numpy(v))
+                opt.step_from_host(host_flat)
+                flat_before = host_flat
             out["steps"].append({"params": [p.numpy().copy() for p in params],
                                  "grads_kept": bool(torch.equal(flat_before, opt.flat_grad)),
                                  "views": all(p.data_ptr() == opt.flat_param[s[2]:].data_ptr()

@@ -6,9 +6,10 @@ on the same table: each tensor's arithmetic does not depend on the plan (or
 the launch) it runs in, and an average over one rank is the value itself.
 The table has several buckets (a small segment cap), Muon classes of one and
 of several matrices, a per-head group, bf16 gradients, an embedding, 1-D and
-0-D tensors. The first step is also checked against the oracle. Multi-rank
-runs of the same code are the gloo tests (the collectives are the only
-difference).
+0-D tensors. The first step is also checked against the oracle, and the
+step with gradients copied from pinned host memory against the
+device-resident one, bit for bit. Multi-rank runs of the same code are the
+gloo tests (the collectives are the only difference).
 """
 import datetime
 import socket
@@ -96,3 +97,37 @@ def test_one_rank_matches_muonadamw_bit_for_bit(one_rank_group):
     finally:
         opt.close()
         ref._plan.close()
+
+
+def test_one_rank_step_from_host_matches_step(one_rank_group):
+    # gradients from pinned host memory, copied bucket by bucket on a side
+    # stream: the same bits as the device-resident step
+    from adamw_hybrid_optimizer_muon_b200.dist import DistMuonAdamW
+
+    r = np.random.default_rng(78)
+    P0 = [np.asarray(r.standard_normal(s) * 0.02, dtype=np.float32) for s, _, _ in TABLE]
+    pa = [dev_f32(p) for p in P0]
+    pb = [dev_f32(p) for p in P0]
+    oa = DistMuonAdamW([(p, role, g) for p, (_, role, g) in zip(pa, TABLE)], _groups(),
+                       grad_dtype=torch.bfloat16, seg_cap=1 << 16)
+    ob = DistMuonAdamW([(p, role, g) for p, (_, role, g) in zip(pb, TABLE)], _groups(),
+                       grad_dtype=torch.bfloat16, seg_cap=1 << 16)
+    host_flat = torch.zeros(ob.flat_grad.shape, dtype=torch.bfloat16, pin_memory=True)
+    hv = ob.host_views(host_flat)
+    try:
+        for step in (1, 2, 3):
+            G = [dev_grad(bf16_round(r.standard_normal(s) * 1e-3), "bf16") for s, _, _ in TABLE]
+            for gv, h, g in zip(oa.grads, hv, G):
+                gv.copy_(g)
+                h.copy_(g.cpu())
+            oa.step()
+            ob.step_from_host(host_flat)
+            torch.cuda.synchronize()
+            assert ma.ma_device_status() == ma.MA_OK
+            assert torch.equal(oa.flat_grad, ob.flat_grad)
+            for i, (a, b) in enumerate(zip(pa, pb)):
+                assert torch.equal(a, b), f"step {step} tensor {i}"
+    finally:
+        oa.close()
+        ob.close()
+
