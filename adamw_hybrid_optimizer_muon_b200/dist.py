@@ -170,6 +170,7 @@ class DistMuonAdamW:
                                    self.grad_shard[r0:r1].view(shape), self.state0[r0:r1].view(shape), s1))
         self._plans = None
         self._ws = None
+        self._side = None   # stream the reductions are issued from (CUDA only)
 
     # ------------------------------------------------------------------ step
 
@@ -240,7 +241,7 @@ class DistMuonAdamW:
             # for everything queued so far (the gradients' producers, the last
             # step's reads of flat_grad); NCCL then waits on the side stream
             # only, so a copy or reduction never waits for an update
-            if getattr(self, "_side", None) is None:
+            if self._side is None:
                 self._side = torch.cuda.Stream(device=self.flat_grad.device)
             side = self._side
             side.wait_stream(torch.cuda.current_stream(self.flat_grad.device))
