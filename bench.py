@@ -14,7 +14,8 @@ grads, state: ~70 GB) are far larger than the 126 MB L2, so no flush is
 needed between steps; sets smaller than twice the L2 get a 512 MB write
 between timed steps, outside their events.
 
-Printed (rank 0): one JSON line with the metric (params/s), ms per step, the
+Printed (rank 0): one JSON line with the metric (params/s), ms per step (the
+mean over the K timed steps, plus the median and range of the per-step times), the
 end-to-end number through the C ABI with host buffers, the roofline of the
 dominant kernel (Newton-Schulz GEMMs, measured live with CUDA events on their
 launch stream), the clocks seen during the timed region, and a CPU baseline
@@ -271,7 +272,7 @@ def workload_config(wl, n_gpus):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--workload", default="7b", choices=sorted(synth.WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
@@ -375,16 +376,20 @@ def main():
             do_step()
             b.record(stream)
         torch.cuda.synchronize(dev)
-        step_ms = sum(a.elapsed_time(b) for a, b in evs)
+        per_step = [a.elapsed_time(b) for a, b in evs]
+        step_ms = sum(per_step)
         del flush
     else:
-        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        t0.record(stream)
-        for _ in range(args.steps):
+        # one event before each step and one after the last: the steps run
+        # back to back, and each one's time is read between its two events
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps + 1)]
+        evs[0].record(stream)
+        for i in range(args.steps):
             do_step()
-        t1.record(stream)
+            evs[i + 1].record(stream)
         torch.cuda.synchronize(dev)
-        step_ms = t0.elapsed_time(t1)
+        per_step = [evs[i].elapsed_time(evs[i + 1]) for i in range(args.steps)]
+        step_ms = evs[0].elapsed_time(evs[-1])
     barrier()
     clk = clocks.stop()
     if args.graph:  # graph replays record no per-kernel events: profile eager steps, untimed
@@ -519,7 +524,9 @@ def main():
             config["parallelism"] = (f"sharded dp{world}: reduce-scatter, each rank's share of the update, "
                                      f"all-gather ({len(opt.buckets)} buckets)")
         line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-                "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "warmup": args.warmup, "ms_per_step": ms,
+                "ms_per_step_median": statistics.median(per_step),
+                "ms_per_step_range": [min(per_step), max(per_step)], "higher_is_better": True,
                 "scaling": "strong" if args.sharded else "weak",
                 "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded N(0,0.02^2) weights, "
                 "N(0,1e-3^2) bf16 grads)", "config": config,

@@ -63,6 +63,8 @@ def test_gpu_arm_line(graph):
     d = json.loads(line)
     _check_base(d, 3, 3)
     assert d["n_gpus"] == 1 and d["dtype"] == "bf16"
+    lo, hi = d["ms_per_step_range"]
+    assert 0 < lo <= d["ms_per_step_median"] <= hi
     r = d["roofline"]
     assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
     assert r["achieved"] > 0 and r["peak"] > 0 and abs(r["frac"] - r["achieved"] / r["peak"]) < 1e-9
