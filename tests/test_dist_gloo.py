@@ -357,3 +357,43 @@ def test_dist_step_matches_single_process_oracle(world):
     _, buckets, total = ma.ma_shard_layout(descs, ma.group_table(_groups()), world, 2048)
     assert results[0]["nbuckets"] == len(buckets)
     assert sum(results[r]["state_elems"] for r in range(world)) == total
+
+
+@pytest.fixture
+def gloo_one_rank():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        yield
+    finally:
+        dist.destroy_process_group()
+
+
+def test_dist_host_side_one_rank(gloo_one_rank):
+    from adamw_hybrid_optimizer_muon_b200.dist import DistMuonAdamW
+
+    params = [torch.full(s, float(i), dtype=torch.float32) for i, (s, _, _) in enumerate(TABLE)]
+    opt = DistMuonAdamW([(p, role, g) for p, (_, role, g) in zip(params, TABLE)], _groups(), seg_cap=2048)
+    # the parameters moved into the flat buffer, values kept, tensors now views of it
+    for i, (p, (_, _, off)) in enumerate(zip(params, opt.slots)):
+        assert p.data_ptr() == opt.flat_param[off:].data_ptr() and bool((p == float(i)).all())
+    # one rank updates everything: its pieces are whole tensors, its state is the flat buffer
+    assert sorted(pc.index for pc in opt.pieces()) == list(range(len(TABLE)))
+    assert all(pc.lo == 0 and pc.hi == _numel(TABLE[pc.index][0]) for pc in opt.pieces())
+    assert opt.state0.numel() == opt.flat_param.numel()
+    assert opt.state_bytes == 4 * (opt.state0.numel() + opt.state1.numel())
+    host = torch.zeros_like(opt.flat_grad)
+    views = opt.host_views(host)
+    assert [tuple(v.shape) for v in views] == [tuple(g.shape) for g in opt.grads]
+    text = opt.describe()
+    assert text.startswith("rank 0 of 1:") and text.count("bucket ") == len(opt.buckets)
+    with pytest.raises(ValueError):
+        opt.step_from_host(torch.zeros(3))
+    with pytest.raises(ValueError):
+        DistMuonAdamW([(torch.zeros(8, 8, dtype=torch.float16), H, 0)], _groups())
+    with pytest.raises(ValueError):
+        DistMuonAdamW([], _groups())
