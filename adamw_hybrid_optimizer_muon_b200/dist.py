@@ -271,6 +271,12 @@ class DistMuonAdamW:
         for w in gathers:
             w.wait()
 
+    def zero_grad(self) -> None:
+        """Zero the flat gradient buffer. The ``.grad`` views stay in place, so
+        that backward keeps accumulating into the buffer (setting ``.grad`` to
+        None instead would detach the parameters from it)."""
+        self.flat_grad.zero_()
+
     # ------------------------------------------------------------------ introspection
 
     @property

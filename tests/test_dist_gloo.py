@@ -397,3 +397,24 @@ def test_dist_host_side_one_rank(gloo_one_rank):
         DistMuonAdamW([(torch.zeros(8, 8, dtype=torch.float16), H, 0)], _groups())
     with pytest.raises(ValueError):
         DistMuonAdamW([], _groups())
+
+
+def test_dist_backward_accumulates_into_flat_buffer(gloo_one_rank):
+    # with fp32 gradients the parameters' .grad are views of the flat buffer:
+    # backward writes (and accumulates) there, and zero_grad keeps the views
+    from adamw_hybrid_optimizer_muon_b200.dist import DistMuonAdamW
+
+    torch.manual_seed(0)
+    lin = torch.nn.Linear(32, 16, bias=True)
+    opt = DistMuonAdamW([(lin.weight, H, 0), (lin.bias, H, 1)],
+                        [("muon", ma.muon_hparams()), ("adamw", ma.adamw_hparams())])
+    x = torch.randn(8, 32)
+    lin(x).square().sum().backward()
+    g1 = [lin.weight.grad.clone(), lin.bias.grad.clone()]
+    assert lin.weight.grad.data_ptr() == opt.grads[0].data_ptr()
+    assert torch.equal(opt.grads[0], g1[0]) and torch.equal(opt.grads[1], g1[1])
+    lin(x).square().sum().backward()
+    assert torch.allclose(opt.grads[0], 2 * g1[0]) and torch.allclose(opt.grads[1], 2 * g1[1])
+    opt.zero_grad()
+    assert float(opt.flat_grad.abs().sum()) == 0.0
+    assert lin.weight.grad.data_ptr() == opt.grads[0].data_ptr()
