@@ -26,6 +26,8 @@
 #include <unordered_map>
 #include <vector>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 #include "internal.h"
 
@@ -720,8 +722,18 @@ std::vector<Segment> step_segments(const ma_plan* plan, const ma_group_t* groups
     return segs;
 }
 
+// An NVTX range over a scope (host-side markers for timeline tools such as
+// Nsight Systems; without a tool attached the calls do nothing).
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
 int launch_segment(ma_plan* plan, const ma_group_t* groups, const Segment& sg, void* ws, cudaStream_t s, int sms,
                    int* launches) {
+    NvtxRange range(sg.adamw ? "ma.adamw" : "ma.muon");
     const int ngroups = (int)plan->group_kind.size();
     int st;
     if (sg.adamw) {
@@ -1309,6 +1321,7 @@ int ma_plan_create(const ma_tensor_t* t, int n, const ma_group_t* groups, int ng
 }
 
 int muonadamw_step(ma_plan_t* plan, const ma_group_t* groups, void* ws, size_t ws_bytes, void* stream) {
+    ma::NvtxRange range("ma.step");
     int sms = 0;
     int st = check_step(plan, groups, ws, ws_bytes, &sms);
     if (st) return st;
