@@ -103,6 +103,8 @@ class DistMuonAdamW:
             raise ValueError("no parameters")
         device = self.entries[0][0].device
         gdt = grad_dtype or torch.float32
+        if gdt not in (torch.float32, torch.bfloat16):
+            raise ValueError("gradients must be fp32 or bf16")
         descs = []
         for p, role, grp in self.entries:
             if p.dtype != torch.float32 or p.device != device:

@@ -397,6 +397,8 @@ def test_dist_host_side_one_rank(gloo_one_rank):
         DistMuonAdamW([(torch.zeros(8, 8, dtype=torch.float16), H, 0)], _groups())
     with pytest.raises(ValueError):
         DistMuonAdamW([], _groups())
+    with pytest.raises(ValueError):
+        DistMuonAdamW([(torch.zeros(8, 8), H, 0)], _groups(), grad_dtype=torch.float16)
 
 
 def test_dist_backward_accumulates_into_flat_buffer(gloo_one_rank):
