@@ -164,7 +164,7 @@ def test_shard_layout_random_tables():
         shapes, descs, kinds = [], [], []
         for _ in range(n):
             nd = int(r.integers(0, 3))
-            shape = tuple(int(x) for x in r.choice([1, 3, 8, 16, 40], size=nd))
+            shape = tuple(int(x) for x in r.choice([0, 1, 3, 8, 16, 40], size=nd))
             role = int(r.choice([H, H, E]))
             kind = ma.MA_MUON if nd == 2 and role == H else ma.MA_ADAMW
             shapes.append(shape)
@@ -202,6 +202,7 @@ TABLE = [  # (shape, role, group)
     ((96,), H, 2), ((), H, 3), ((7,), H, 3),
     ((48, 96), H, 0),
     ((40, 96), H, 0),
+    ((0, 16), H, 0), ((0,), H, 2),                           # empty tensors: placed, never updated
 ]
 
 
@@ -297,7 +298,7 @@ def _worker(rank, world, port, q):
             out["steps"].append({"params": [p.numpy().copy() for p in params],
                                  "grads_kept": bool(torch.equal(flat_before, opt.flat_grad)),
                                  "views": all(p.data_ptr() == opt.flat_param[s[2]:].data_ptr()
-                                              for p, s in zip(params, opt.slots))})
+                                              for p, s in zip(params, opt.slots) if p.numel())})
         q.put((rank, out))
     finally:
         dist.destroy_process_group()
@@ -312,6 +313,8 @@ def _reference(world, start):
     for step in (1, 2):
         avg = _average(step, world)
         for i, (s, _, g) in enumerate(TABLE):
+            if _numel(s) == 0:
+                continue
             P[i], S0[i], v = _oracle_update(groups[g], P[i], avg[i], S0[i], S1[i], step)
             if v is not None:
                 S1[i] = v
@@ -380,9 +383,12 @@ def test_dist_host_side_one_rank(gloo_one_rank):
     opt = DistMuonAdamW([(p, role, g) for p, (_, role, g) in zip(params, TABLE)], _groups(), seg_cap=2048)
     # the parameters moved into the flat buffer, values kept, tensors now views of it
     for i, (p, (_, _, off)) in enumerate(zip(params, opt.slots)):
-        assert p.data_ptr() == opt.flat_param[off:].data_ptr() and bool((p == float(i)).all())
-    # one rank updates everything: its pieces are whole tensors, its state is the flat buffer
-    assert sorted(pc.index for pc in opt.pieces()) == list(range(len(TABLE)))
+        assert bool((p == float(i)).all())
+        if p.numel():
+            assert p.data_ptr() == opt.flat_param[off:].data_ptr()
+    # one rank updates everything: its pieces are whole tensors (empty ones have
+    # none), its state is the flat buffer
+    assert sorted(pc.index for pc in opt.pieces()) == [i for i, (s, _, _) in enumerate(TABLE) if _numel(s)]
     assert all(pc.lo == 0 and pc.hi == _numel(TABLE[pc.index][0]) for pc in opt.pieces())
     assert opt.state0.numel() == opt.flat_param.numel()
     assert opt.state_bytes == 4 * (opt.state0.numel() + opt.state1.numel())
