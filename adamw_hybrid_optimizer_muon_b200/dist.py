@@ -32,6 +32,7 @@ the library's kernels. Tests on CPU ranks replace ``_local_step``.
 """
 from __future__ import annotations
 
+import hashlib
 from dataclasses import dataclass, field
 
 import torch
@@ -118,6 +119,7 @@ class DistMuonAdamW:
         self.kinds = ma_partition(descs)
         slots, buckets, total = ma_shard_layout(descs, self.groups, self.world, seg_cap)
         self.slots = slots
+        self._layout_key = hashlib.sha256(repr((slots, buckets, total, str(gdt))).encode()).hexdigest()
         self.flat_param = torch.zeros(total, dtype=torch.float32, device=device)
         self.flat_grad = torch.zeros(total, dtype=gdt, device=device)
         self.grads = []
@@ -272,6 +274,22 @@ class DistMuonAdamW:
                                                            async_op=True))
         for w in gathers:
             w.wait()
+
+    def state_dict(self) -> dict:
+        """This rank's optimizer state: the step count, its state buffers (the
+        tensors themselves, not copies) and a key of the layout they belong to.
+        Each rank saves its own; a resumed run needs the same table, world size
+        and segment cap."""
+        return {"step": self.step_count, "world": self.world, "rank": self.rank, "layout": self._layout_key,
+                "state0": self.state0, "state1": self.state1}
+
+    def load_state_dict(self, sd: dict) -> None:
+        """Restore what :meth:`state_dict` returned on this rank of an identical setup."""
+        if (sd["world"], sd["rank"], sd["layout"]) != (self.world, self.rank, self._layout_key):
+            raise ValueError("optimizer state of another layout, world size or rank")
+        self.state0.copy_(sd["state0"])
+        self.state1.copy_(sd["state1"])
+        self.step_count = int(sd["step"])
 
     def zero_grad(self) -> None:
         """Zero the flat gradient buffer. The ``.grad`` views stay in place, so

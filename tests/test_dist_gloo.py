@@ -17,7 +17,9 @@ buckets), a per-head group, an embedding that straddles AdamW segments, 1-D
 and 0-D tensors, and a small segment cap so that there are many buckets.
 The gradients must be left as they were, the initial parameters must come
 from rank 0, and each rank must hold only its share of the optimizer state.
-The second step takes its gradients from a host buffer (step_from_host).
+The second step takes its gradients from a host buffer (step_from_host). A
+run resumed from a state_dict after its first step must match the
+uninterrupted run bit for bit.
 """
 import datetime
 import os
@@ -426,3 +428,75 @@ def test_dist_backward_accumulates_into_flat_buffer(gloo_one_rank):
     opt.zero_grad()
     assert float(opt.flat_grad.abs().sum()) == 0.0
     assert lin.weight.grad.data_ptr() == opt.grads[0].data_ptr()
+
+
+def _resume_worker(rank, world, port, q):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        from adamw_hybrid_optimizer_muon_b200.dist import DistMuonAdamW
+
+        class OracleDist(DistMuonAdamW):
+            def _local_step(self, b):
+                for pc in self.buckets[b].pieces:
+                    grp = self.groups[pc.group]
+                    s1 = None if pc.state1 is None else pc.state1.numpy()
+                    W1, a, v = _oracle_update(grp, pc.param.numpy(), pc.grad.numpy(), pc.state0.numpy(), s1,
+                                              grp.adamw.step)
+                    pc.param.copy_(torch.from_numpy(W1))
+                    pc.state0.copy_(torch.from_numpy(a))
+                    if v is not None:
+                        pc.state1.copy_(torch.from_numpy(v))
+
+        def make(start):
+            params = [torch.from_numpy(x.copy()) for x in start]
+            return params, OracleDist([(p, role, g) for p, (_, role, g) in zip(params, TABLE)], _groups(),
+                                      seg_cap=2048)
+
+        init = np.random.default_rng(5)
+        start = [np.asarray(init.standard_normal(s) * 0.02, dtype=np.float32) for s, _, _ in TABLE]
+        steps = 3
+        # uninterrupted
+        pa, oa = make(start)
+        for step in range(1, steps + 1):
+            for g, v in zip(oa.grads, _grads(step, rank, world)):
+                g.copy_(torch.from_numpy(v))
+            oa.step()
+            if step == 1:
+                saved = {k: (v.clone() if torch.is_tensor(v) else v) for k, v in oa.state_dict().items()}
+                mid = [p.numpy().copy() for p in pa]
+        # resumed after step 1 from the saved parameters and state
+        pb, ob = make(mid)
+        ob.load_state_dict(saved)
+        for step in range(2, steps + 1):
+            for g, v in zip(ob.grads, _grads(step, rank, world)):
+                g.copy_(torch.from_numpy(v))
+            ob.step()
+        same = all(torch.equal(a, b) for a, b in zip(pa, pb))
+        refused = False
+        try:
+            ob.load_state_dict(dict(saved, layout="other"))
+        except ValueError:
+            refused = True
+        q.put((rank, same and refused and ob.step_count == steps))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_dist_resume_from_state_dict():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    procs = [ctx.Process(target=_resume_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    results = dict(q.get(timeout=300) for _ in range(2))
+    for p in procs:
+        p.join(60)
+    assert all(p.exitcode == 0 for p in procs)
+    assert results == {0: True, 1: True}
+
