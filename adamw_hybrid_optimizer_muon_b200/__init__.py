@@ -574,6 +574,24 @@ class MuonAdamW:
         self._advance()
         self._plan.step_from_host(host_grads, self.groups, stream, copy_stream)
 
+    def state_dict(self) -> dict:
+        """The step count and the state buffers (the tensors themselves, not
+        copies): per entry (momentum, None) for Muon, (exp_avg, exp_avg_sq)
+        for AdamW."""
+        return {"step": self.step_count, "state": list(self.state)}
+
+    def load_state_dict(self, sd: dict) -> None:
+        """Copy a state_dict of an optimizer over the same table into this one."""
+        if len(sd["state"]) != len(self.state):
+            raise ValueError("state of another parameter table")
+        for (a0, a1), (b0, b1) in zip(self.state, sd["state"]):
+            if a0.shape != b0.shape or (a1 is None) != (b1 is None):
+                raise ValueError("state of another parameter table")
+            a0.copy_(b0)
+            if a1 is not None:
+                a1.copy_(b1)
+        self.step_count = int(sd["step"])
+
     @property
     def launches(self) -> int:
         return self._plan.launches if self._plan is not None else 0

@@ -302,3 +302,28 @@ def test_plan_rejects_kind_mismatch():
     with pytest.raises(ma.MAError) as e:
         ma.ma_plan_create([d0], _groups_for(wl))
     assert e.value.code == ma.MA_ERR_ARG
+
+
+def test_muonadamw_state_dict_roundtrip_on_host():
+    # the optimizer object and its state buffers can be built without a GPU
+    # (the plan, and with it the library's device work, is made on the first step)
+    import torch
+    params = [torch.randn(16, 32), torch.randn(32), torch.randn(8, 16)]
+    table = [(params[0], ma.ROLE_HIDDEN, 0), (params[1], ma.ROLE_HIDDEN, 1), (params[2], ma.ROLE_EMBED, 1)]
+    groups = [("muon", ma.muon_hparams()), ("adamw", ma.adamw_hparams())]
+    a = ma.MuonAdamW(table, groups)
+    assert [s1 is None for _, s1 in a.state] == [True, False, False]
+    for s0, s1 in a.state:
+        s0.normal_()
+        if s1 is not None:
+            s1.uniform_()
+    a.step_count = 7
+    b = ma.MuonAdamW(table, groups)
+    b.load_state_dict(a.state_dict())
+    assert b.step_count == 7
+    for (a0, a1), (b0, b1) in zip(a.state, b.state):
+        assert torch.equal(a0, b0) and a0.data_ptr() != b0.data_ptr()
+        assert (a1 is None and b1 is None) or torch.equal(a1, b1)
+    c = ma.MuonAdamW(table[:2], groups)
+    with pytest.raises(ValueError):
+        c.load_state_dict(a.state_dict())
