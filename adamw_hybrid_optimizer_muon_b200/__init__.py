@@ -19,7 +19,8 @@ __all__ = [
     "ma_shard_layout", "muon_workspace_bytes", "muon_step_batched",
     "muon_step_batched_noalloc", "STATIC_SCRATCH_BYTES", "ns_iterate_workspace_bytes", "ns_iterate_bf16",
     "adamw_step_fused", "ma_plan_create", "muonadamw_step", "muonadamw_step_graph", "muonadamw_step_from_host",
-    "ma_plan_describe", "ma_plan_destroy", "ma_device_status", "ma_device_status_async", "ma_set_wait_limit_ns",
+    "ma_plan_describe", "ma_plan_destroy", "ma_plan_status", "ma_device_status", "ma_device_status_async",
+    "ma_set_wait_limit_ns",
     "ma_selftest_wait_timeout", "ma_profile_enable", "ma_profile_collect", "PROF_CLASSES", "group_table", "Plan",
     "MuonAdamW", "muon_hparams", "adamw_hparams",
 ]
@@ -133,6 +134,7 @@ def lib() -> ctypes.CDLL:
         "ma_plan_destroy": (None, [vp]),
         "ma_device_status": (i32, [vp, i32]),
         "ma_device_status_async": (i32, [vp, vp]),
+        "ma_plan_status": (i32, [vp, vp]),
         "ma_set_wait_limit_ns": (i32, [i64]),
         "ma_selftest_wait_timeout": (i32, [i64, vp]),
         "muon_step_batched_noalloc": (i32, [i32, i64, i64, pp, pp, i32, pp, ctypes.POINTER(MuonHParams), vp]),
@@ -395,6 +397,11 @@ def ma_device_status(stream=None, reset: bool = True) -> int:
     return int(lib().ma_device_status(_stream(stream), int(bool(reset))))
 
 
+def ma_plan_status(plan, stream=None) -> int:
+    """Wait for ``stream``, then read and clear the status word of the device the plan's steps ran on."""
+    return int(lib().ma_plan_status(plan, _stream(stream)))
+
+
 def ma_device_status_async(host_dst, stream=None) -> None:
     """Enqueue a copy of the device status word into host_dst (a pinned int32 tensor element or address)."""
     _check(lib().ma_device_status_async(_ptr(host_dst), _stream(stream)), "ma_device_status_async")
@@ -470,6 +477,10 @@ class Plan:
     @property
     def graph_captures(self) -> int:
         return int(lib().ma_plan_graph_captures(self.handle))
+
+    def status(self, stream=None) -> int:
+        """Wait for ``stream``; MA_OK or the first device-side error of the steps since the last read."""
+        return ma_plan_status(self.handle, stream)
 
     def describe(self, groups: Sequence[Group] | None = None) -> str:
         """What a step runs: workspace, buckets, sub-batches and shared launches."""

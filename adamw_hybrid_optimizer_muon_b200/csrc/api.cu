@@ -1658,6 +1658,11 @@ int ma_device_status(void* stream, int reset) {
     return v;
 }
 
+int ma_plan_status(ma_plan_t* plan, void* stream) {
+    if (!plan) return MA_ERR_NULL;
+    return ma_device_status(stream, 1);
+}
+
 int ma_device_status_async(int32_t* host_dst, void* stream) {
     if (!host_dst) return MA_ERR_NULL;
     int dev = 0;

@@ -395,6 +395,13 @@ int ma_profile_collect(double* ms_out, int64_t* launches_out, double* flops_out,
  * device-side error recorded since the last reset) and, if reset != 0, clear it. */
 int ma_device_status(void* stream, int reset);
 
+/* The status of a plan's steps: synchronise `stream` (the stream the plan's
+ * steps were launched on), then read and clear the status word of the current
+ * device, as ma_device_status(stream, 1) does. Returns MA_ERR_NULL for a NULL
+ * plan, MA_ERR_CUDA when the device cannot be reached, else MA_OK or the
+ * first device-side error (MA_ERR_TIMEOUT) since the last read. */
+int ma_plan_status(ma_plan_t* plan, void* stream);
+
 /* Enqueue on `stream` a copy of the current device's status word into
  * host_dst (one int32, host; page-locked memory makes the copy asynchronous).
  * The value is valid once the stream has passed the copy; the word is not

@@ -327,3 +327,13 @@ def test_muonadamw_state_dict_roundtrip_on_host():
     c = ma.MuonAdamW(table[:2], groups)
     with pytest.raises(ValueError):
         c.load_state_dict(a.state_dict())
+
+
+def test_plan_status_without_gpu_fails_loudly():
+    assert ma.lib().ma_plan_status(None, None) == ma.MA_ERR_NULL
+    wl = synth.tiny()
+    plan, _ = ma.ma_plan_create(_fake_descs(wl), _groups_for(wl))
+    try:
+        assert ma.ma_plan_status(plan, 0) == ma.MA_ERR_CUDA  # no device: an error, never a fake OK
+    finally:
+        ma.ma_plan_destroy(plan)
