@@ -19,7 +19,8 @@ The gradients must be left as they were, the initial parameters must come
 from rank 0, and each rank must hold only its share of the optimizer state.
 The second step takes its gradients from a host buffer (step_from_host). A
 run resumed from a state_dict after its first step must match the
-uninterrupted run bit for bit.
+uninterrupted run bit for bit. Two mistakes planted in the exchange (a sum
+instead of an average, a missing all-gather) must each break the comparison.
 """
 import datetime
 import os
@@ -258,10 +259,30 @@ def _oracle_update(group, W, g, s0, s1, step):
     return p1.astype(np.float32), m1.astype(np.float32), v1.astype(np.float32)
 
 
-def _worker(rank, world, port, q):
+class _DoneWork:
+    def wait(self):
+        return True
+
+
+def _plant(mutation):
+    """A planted mistake in the exchange (for the test that the comparison catches it)."""
+    if mutation == "sum":  # gradients summed instead of averaged
+        orig = dist.reduce_scatter_tensor
+
+        def reduce_scatter_sum(out, inp, op=None, group=None, async_op=False):
+            return orig(out, inp, op=dist.ReduceOp.SUM, group=group, async_op=async_op)
+        dist.reduce_scatter_tensor = reduce_scatter_sum
+    elif mutation == "no_gather":  # updated segments never leave their rank
+        def skip_gather(out, inp, group=None, async_op=False):
+            return _DoneWork()
+        dist.all_gather_into_tensor = skip_gather
+
+
+def _worker(rank, world, port, q, mutation=None):
     os.environ["MASTER_ADDR"] = "127.0.0.1"
     os.environ["MASTER_PORT"] = str(port)
     dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    _plant(mutation)
     try:
         from adamw_hybrid_optimizer_muon_b200.dist import DistMuonAdamW
 
@@ -324,20 +345,36 @@ def _reference(world, start):
     return out
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_dist_step_matches_single_process_oracle(world):
+def _run_ranks(world, mutation=None):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     s = socket.socket()
     s.bind(("127.0.0.1", 0))
     port = s.getsockname()[1]
     s.close()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q, mutation)) for r in range(world)]
     for p in procs:
         p.start()
     results = dict(q.get(timeout=300) for _ in range(world))
     for p in procs:
         p.join(60)
+    return procs, results
+
+
+@pytest.mark.parametrize("mutation", ["sum", "no_gather"])
+def test_dist_comparison_catches_a_planted_exchange_mistake(mutation):
+    procs, results = _run_ranks(2, mutation)
+    assert all(p.exitcode == 0 for p in procs)
+    ref = _reference(2, results[0]["start"])
+    same = all(np.array_equal(got, want)
+               for r in range(2) for k, st in enumerate(results[r]["steps"])
+               for got, want in zip(st["params"], ref[k]))
+    assert not same, f"planted mistake {mutation!r} went unnoticed"
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_dist_step_matches_single_process_oracle(world):
+    procs, results = _run_ranks(world)
     assert all(p.exitcode == 0 for p in procs), [p.exitcode for p in procs]
 
     start = results[0]["start"]
