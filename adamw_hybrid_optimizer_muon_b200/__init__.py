@@ -417,7 +417,8 @@ def ma_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
     _check(lib().ma_selftest_wait_timeout(int(limit_ns), _stream(stream)), "ma_selftest_wait_timeout")
 
 
-PROF_CLASSES = ("adamw", "momentum", "finalize", "ns_gram", "ns_apply", "ns_gramsq", "ns_final")
+PROF_CLASSES = ("adamw", "momentum", "finalize", "ns_gram", "ns_apply", "ns_gramsq", "ns_final", "momentum_side",
+                "ns_cluster")
 
 
 def ma_profile_enable(on: bool) -> None:
@@ -575,6 +576,11 @@ class MuonAdamW:
         dtypes); the library copies each group of gradients on copy_stream
         (default: a stream owned by this optimizer) and overlaps the copies
         with the compute on stream.
+
+        The call returns before the copies have read host_grads: do not write
+        to them until ``host_copies_done`` (a CUDA event recorded on the copy
+        stream after the last copy) has completed, e.g.
+        ``opt.host_copies_done.synchronize()``.
         """
         import torch
         self._ensure_plan(device_grads)
@@ -584,6 +590,9 @@ class MuonAdamW:
             copy_stream = self._copy_stream
         self._advance()
         self._plan.step_from_host(host_grads, self.groups, stream, copy_stream)
+        cs = copy_stream if isinstance(copy_stream, torch.cuda.Stream) else torch.cuda.ExternalStream(int(copy_stream))
+        self.host_copies_done = torch.cuda.Event()
+        self.host_copies_done.record(cs)
 
     def state_dict(self) -> dict:
         """The step count and the state buffers (the tensors themselves, not

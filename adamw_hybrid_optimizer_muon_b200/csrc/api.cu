@@ -16,6 +16,7 @@
 // graph. The host never synchronises. Every argument is checked before the
 // first launch, so a failing call changes nothing.
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstdlib>
@@ -35,19 +36,21 @@ namespace ma {
 
 __device__ int g_status = 0;
 
-static long long g_host_wait_limit_ns = 2000000000LL;
-long long host_wait_limit_ns() { return g_host_wait_limit_ns; }
+static std::atomic<long long> g_host_wait_limit_ns{2000000000LL};
+long long host_wait_limit_ns() { return g_host_wait_limit_ns.load(std::memory_order_relaxed); }
 
 int* device_status_ptr() {
-    static int* cached[64] = {nullptr};
+    static PerDevice<int*> cache;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!cached[dev]) {
-        void* ptr = nullptr;
-        if (cudaGetSymbolAddress(&ptr, g_status) != cudaSuccess) return nullptr;
-        cached[dev] = reinterpret_cast<int*>(ptr);
-    }
-    return cached[dev];
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    int* ptr = nullptr;
+    const cudaError_t e = cache.get(dev, &ptr, [](int** v) {
+        void* p = nullptr;
+        const cudaError_t r = cudaGetSymbolAddress(&p, g_status);
+        *v = reinterpret_cast<int*>(p);
+        return r;
+    });
+    return e == cudaSuccess ? ptr : nullptr;
 }
 
 namespace {
@@ -112,24 +115,26 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 
 // sm_100a code runs only on compute capability 10.0; cache per device.
 int device_ok_and_sms(int* sms) {
-    static int cached_sms[64] = {0};
-    static int cached_ok[64] = {0};
+    // per device: the SM count, or -MA_ERR_* when the device cannot run this library
+    static PerDevice<int> cache;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return MA_ERR_CUDA;
-    if (dev < 0 || dev >= 64) return MA_ERR_UNSUPPORTED;
-    if (!cached_ok[dev]) {
+    if (dev < 0 || dev >= kMaxDevices) return MA_ERR_UNSUPPORTED;
+    int v = 0;
+    const cudaError_t e = cache.get(dev, &v, [dev](int* out) {
         int maj = 0, min = 0, n = 0, smem = 0;
         if (cudaDeviceGetAttribute(&maj, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&min, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
             cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
-            return MA_ERR_CUDA;
-        if (maj != 10 || min != 0) return MA_ERR_UNSUPPORTED;
-        if ((size_t)smem < ns_tc_smem_bytes() || n < 2) return MA_ERR_UNSUPPORTED;
-        cached_sms[dev] = n;
-        cached_ok[dev] = 1;
-    }
-    if (sms) *sms = cached_sms[dev];
+            return cudaErrorUnknown;  // not cached: the next call asks again
+        if (maj != 10 || min != 0 || (size_t)smem < ns_tc_smem_bytes() || n < 2) *out = -MA_ERR_UNSUPPORTED;
+        else *out = n;
+        return cudaSuccess;
+    });
+    if (e != cudaSuccess) return MA_ERR_CUDA;
+    if (v < 0) return -v;
+    if (sms) *sms = v;
     return MA_OK;
 }
 
@@ -143,7 +148,7 @@ struct MuonGeom {
     int64_t parts;
     int esz;
     bool quintic;
-    size_t off_x0, off_x1, off_g, off_g2, off_part, off_scale, total;
+    size_t off_x0, off_x1, off_g, off_g2, off_part, off_scale, off_ctr, total;
 };
 
 bool any_c(const ma_muon_hparams_t& hp) {
@@ -199,6 +204,8 @@ int muon_geom(int batch, int64_t R, int64_t C, const ma_muon_hparams_t& hp, Muon
     off = align_up(off + (size_t)g->units * g->parts * sizeof(double), kAlign);
     g->off_scale = off;
     off = align_up(off + (size_t)g->units * sizeof(float), kAlign);
+    g->off_ctr = off;  // tile counters of the Newton-Schulz launches
+    off = align_up(off + kNsCounterBytes, kAlign);
     g->total = (batch == 0 || R == 0 || C == 0) ? 0 : off;
     return MA_OK;
 }
@@ -257,7 +264,7 @@ bool ns_compatible(const ma_muon_hparams_t& x, const ma_muon_hparams_t& y) {
 }
 
 // Momentum + norm partials, then the norm finalize, of one job.
-int muon_prep(const MuonJob& j, cudaStream_t s, int* launches) {
+int muon_prep(const MuonJob& j, cudaStream_t s, int max_blocks, bool side, int* launches) {
     const MuonGeom& g = j.g;
     const ma_muon_hparams_t& hp = *j.hp;
     double* part = reinterpret_cast<double*>(j.ws + g.off_part);
@@ -285,12 +292,13 @@ int muon_prep(const MuonJob& j, cudaStream_t s, int* launches) {
         P.M[b] = j.M[b];
     }
     const double elems = (double)g.units * (double)g.Rh * (double)g.C;
-    int pr = prof_begin(MA_PROF_MOMENTUM, s);
-    int st = cuda_status(launch_muon_prep(P, s));
+    int pr = prof_begin(side ? MA_PROF_MOMENTUM_SIDE : MA_PROF_MOMENTUM, s);
+    int st = cuda_status(launch_muon_prep(P, max_blocks, s));
     prof_end(pr, s, 0.0, elems * ((j.gdt == MA_BF16 ? 2 : 4) + 8 + (hp.precision ? 4 : 2)));
     if (st) return st;
     pr = prof_begin(MA_PROF_FINALIZE, s);
-    st = cuda_status(launch_norm_finalize(part, g.parts, (int)g.units, hp.eps, scale, s));
+    st = cuda_status(launch_norm_finalize(part, g.parts, (int)g.units, hp.eps, scale,
+                                          reinterpret_cast<unsigned int*>(j.ws + g.off_ctr), kNsCounters, s));
     prof_end(pr, s, 0.0, (double)g.units * g.parts * 8.0 + g.units * 4.0);
     if (st) return st;
     *launches += 2;
@@ -313,16 +321,83 @@ double ns_bytes(int mode, int64_t units, int64_t m, int64_t n, int esz) {
 // launch over every job's tiles on the tensor-core path; per job in fp32 mode.
 // A tile's arithmetic does not depend on the launch it is in, so grouping
 // gives the same bits as running the jobs one by one.
-int run_muon_jobs(const MuonJob* jobs_in, int njobs_in, cudaStream_t s, int sms, int* launches) {
+// Grid of the flat momentum kernel on the caller's stream: six blocks per SM
+// (as many as its registers let reside), each walking many chunks, so that
+// the pass is not bound by the rate at which blocks start.
+constexpr int kPrepBlocksPerSm = 6;
+
+// The momentum passes (and norm finalizes) of a set of jobs. max_blocks > 0
+// bounds the flat momentum kernel's grid (see launch_muon_prep).
+int prep_jobs(const MuonJob* jobs, int njobs, cudaStream_t s, int max_blocks, int* launches, bool side = false) {
+    int st;
+    for (int j = 0; j < njobs; ++j)
+        if (jobs[j].g.total > 0 && (st = muon_prep(jobs[j], s, max_blocks, side, launches))) return st;
+    return MA_OK;
+}
+
+// Whether a job's chain runs as one cluster-resident launch (ns_cluster.cu):
+// bf16 operands, no A^2 term, short unrolled units (m <= 128, rows <= columns,
+// n <= 4096).
+// Off until the kernel has passed its GPU tests.
+constexpr bool kClusterChain = false;
+
+bool cluster_job(const MuonJob& j) {
+    return kClusterChain && j.g.total > 0 && j.hp->precision == 0 && !j.g.quintic &&
+           ns_cluster_eligible((int)j.g.m, (int)j.g.n, j.g.transposed);
+}
+
+// The whole chain of one job in one cluster launch.
+int chain_cluster(const MuonJob& J, cudaStream_t s, int* launches) {
+    const MuonGeom& g = J.g;
+    const ma_muon_hparams_t& hp = *J.hp;
+    NsClusterIn in;
+    std::memset(&in, 0, sizeof(in));
+    in.x = J.ws + g.off_x0;
+    in.ldx = g.ldx;
+    in.x_unit = g.m * g.ldx;
+    in.units = (int)g.units;
+    in.m = (int)g.m;
+    in.n = (int)g.n;
+    in.steps = hp.ns_steps;
+    for (int k = 0; k < hp.ns_steps; ++k) {
+        const float* cf = hp.coeffs[hp.n_coeffs == 1 ? 0 : k];
+        in.coef[k][0] = cf[0];
+        in.coef[k][1] = cf[1];
+    }
+    in.scale = reinterpret_cast<const float*>(J.ws + g.off_scale);
+    in.heads = g.heads;
+    in.Rh = g.Rh;
+    in.C = g.C;
+    in.decay = 1.f - hp.lr * hp.weight_decay;
+    in.lr_s = hp.lr * shape_scale(g.Rh, g.C, hp.scale_mode);
+    in.lr_wd = hp.lr * hp.weight_decay;
+    in.cautious = hp.cautious ? 1 : 0;
+    in.wait_limit_ns = host_wait_limit_ns();
+    in.status = device_status_ptr();
+    in.W = J.W;
+    const int pr = prof_begin(MA_PROF_NS_CLUSTER, s);
+    const cudaError_t e = launch_ns_cluster(in, s);
+    const double u = (double)g.units, m = (double)g.m, n = (double)g.n;
+    prof_end(pr, s, (double)hp.ns_steps * u * (m * (m + 1.0) * n + 2.0 * m * m * n), u * m * n * (2.0 + 8.0));
+    ++*launches;
+    return cuda_status(e);
+}
+
+// The Newton-Schulz chain of a set of jobs whose momentum passes are done.
+int chain_jobs(const MuonJob* jobs_in, int njobs_in, cudaStream_t s, int sms, int* launches) {
     std::vector<const MuonJob*> jobs;
-    for (int j = 0; j < njobs_in; ++j)
-        if (jobs_in[j].g.total > 0) jobs.push_back(&jobs_in[j]);
+    int st;
+    for (int j = 0; j < njobs_in; ++j) {
+        if (jobs_in[j].g.total == 0) continue;
+        if (cluster_job(jobs_in[j])) {
+            if ((st = chain_cluster(jobs_in[j], s, launches))) return st;
+        } else {
+            jobs.push_back(&jobs_in[j]);
+        }
+    }
     const int nj = (int)jobs.size();
     if (nj == 0) return MA_OK;
     if (nj > ns_tc_max_jobs()) return MA_ERR_UNSUPPORTED;
-    int st;
-    for (const MuonJob* j : jobs)
-        if ((st = muon_prep(*j, s, launches))) return st;
 
     const ma_muon_hparams_t& hp0 = *jobs[0]->hp;
     std::vector<NsParams> p(nj);
@@ -359,11 +434,17 @@ int run_muon_jobs(const MuonJob* jobs_in, int njobs_in, cudaStream_t s, int sms,
     }
 
     std::vector<NsJobIn> in(nj);
+    // each launch of the chain takes its own two tile counters (the first job's,
+    // zeroed by its norm finalize)
+    unsigned int* ctr = reinterpret_cast<unsigned int*>(jobs[0]->ws + jobs[0]->g.off_ctr);
+    int nlaunch = 0;
     auto launch = [&](int mode, const std::vector<void*>& xb, const std::vector<void*>& gb) -> int {
         const int pr = prof_begin(ns_prof_class(mode), s);
         double flops = 0.0, bytes = 0.0;
         cudaError_t e = cudaSuccess;
+        if (2 * nlaunch + 2 > kNsCounters) return MA_ERR_UNSUPPORTED;
         for (int i = 0; i < nj; ++i) {
+            p[i].tile_ctr = ctr + 2 * nlaunch;
             in[i] = {&p[i], xb[i], gb[i]};
             const MuonGeom& g = jobs[i]->g;
             flops += ns_flops(mode, g.units, g.m, g.n);
@@ -378,6 +459,7 @@ int run_muon_jobs(const MuonJob* jobs_in, int njobs_in, cudaStream_t s, int sms,
             e = launch_ns_tc_group(mode, in.data(), nj, sms, s, launches);
         }
         prof_end(pr, s, flops, bytes);
+        ++nlaunch;
         return cuda_status(e);
     };
 
@@ -414,6 +496,12 @@ int run_muon_jobs(const MuonJob* jobs_in, int njobs_in, cudaStream_t s, int sms,
         if (!last) std::swap(cur, nxt);
     }
     return MA_OK;
+}
+
+int run_muon_jobs(const MuonJob* jobs, int njobs, cudaStream_t s, int sms, int* launches) {
+    if (njobs > ns_tc_max_jobs()) return MA_ERR_UNSUPPORTED;
+    const int st = prep_jobs(jobs, njobs, s, kPrepBlocksPerSm * sms, launches);
+    return st ? st : chain_jobs(jobs, njobs, s, sms, launches);
 }
 
 // One batch with workspace ws.
@@ -582,15 +670,22 @@ struct ma_plan {
     };
     std::vector<Bucket> buckets;
     size_t ws_bytes = 0;
+    // > 0: the workspace holds two halves of this many bytes, used by the Muon
+    // segments in turn, so that a segment's momentum pass can run under the
+    // chain of the one before it (on the side stream)
+    size_t region = 0;
     int last_launches = 0;
     std::vector<cudaEvent_t> events;  // segment-ready events of muonadamw_step_from_host
+    cudaStream_t side = nullptr;      // the momentum passes that run under a chain
+    int side_dev = -1;
+    std::vector<cudaEvent_t> side_events;
     // muonadamw_step_graph: the captured step and the kernel nodes whose
     // parameters follow the per-step hyperparameters
     struct GraphNode {
         cudaGraphNode_t node;
         cudaKernelNodeParams params;  // func, launch shape; kernelParams replaced on update
         std::vector<uint8_t> arg;     // the kernel's single by-value parameter
-        int final_apply;              // 0: AdamW launch, 1: Newton-Schulz final apply
+        int final_apply;              // 0: AdamW launch, 1: Newton-Schulz final apply, 2: cluster chain
     };
     struct Graph {
         cudaGraph_t graph = nullptr;
@@ -612,8 +707,10 @@ struct ma_plan {
     } g;
     ~ma_plan() {
         for (cudaEvent_t e : events) cudaEventDestroy(e);
+        for (cudaEvent_t e : side_events) cudaEventDestroy(e);
         g.release();
         if (g.capture) cudaStreamDestroy(g.capture);
+        if (side) cudaStreamDestroy(side);
     }
 };
 
@@ -636,6 +733,10 @@ int64_t tensor_numel(const ma_tensor_t& x) {
     return n;
 }
 
+// The workspace one Muon segment may use: half of the plan's workspace when
+// it is split in two (see run_segments), else all of it.
+size_t seg_limit(const ma_plan* plan) { return plan->region ? plan->region : plan->ws_bytes; }
+
 // Shared checks of a step over a plan; fills *sms.
 int check_step(ma_plan* plan, const ma_group_t* groups, void* ws, size_t ws_bytes, int* sms) {
     if (!plan) return MA_ERR_NULL;
@@ -654,7 +755,7 @@ int check_step(ma_plan* plan, const ma_group_t* groups, void* ws, size_t ws_byte
     for (auto& b : plan->buckets) {
         MuonGeom g;
         if ((st = muon_geom(b.sub, b.R, b.C, groups[b.group].muon, &g))) return st;
-        if (g.total > plan->ws_bytes) return MA_ERR_ARG;
+        if (g.total > seg_limit(plan)) return MA_ERR_ARG;
     }
     if (plan->ws_bytes > 0 && (!ws || !aligned(ws, kAlign) || ws_bytes < plan->ws_bytes)) return MA_ERR_WORKSPACE;
     *sms = 0;
@@ -731,60 +832,190 @@ struct NvtxRange {
     NvtxRange& operator=(const NvtxRange&) = delete;
 };
 
-int launch_segment(ma_plan* plan, const ma_group_t* groups, const Segment& sg, void* ws, cudaStream_t s, int sms,
-                   int* launches) {
-    NvtxRange range(sg.adamw ? "ma.adamw" : "ma.muon");
-    const int ngroups = (int)plan->group_kind.size();
-    int st;
-    if (sg.adamw) {
-        AdamwGroupConst gc[MA_MAX_GROUPS];
-        std::memset(gc, 0, sizeof(gc));
-        for (int k = 0; k < ngroups; ++k)
-            if (groups[k].kind == MA_ADAMW) gc[k] = adamw_const(groups[k].adamw);
-        for (int dt = 0; dt < 2; ++dt) {
-            std::vector<AdamwItem> items;
-            for (int i : plan->adamw_idx) {
-                const ma_tensor_t& x = plan->t[i];
-                if (x.grad_dtype != dt) continue;
-                items.push_back({x.param, x.grad, x.state0, x.state1, tensor_numel(x), x.group});
-            }
-            if (!items.empty() && (st = run_adamw(items, dt, gc, ngroups, s, launches))) return st;
-        }
-        return MA_OK;
-    }
-    const int np = (int)sg.parts.size();
-    std::vector<MuonJob> jobs(np);
+// The jobs of one Muon segment, with the pointer tables they point into.
+struct SegJobs {
+    std::vector<MuonJob> jobs;
     std::vector<float*> W, M;
     std::vector<const void*> G;
+};
+
+// Jobs of Muon segment sg with their workspaces laid out from base.
+void build_jobs(const ma_plan* plan, const ma_group_t* groups, const Segment& sg, uint8_t* base, SegJobs& out) {
+    const int np = (int)sg.parts.size();
+    out.jobs.assign(np, MuonJob{});
     int total = 0;
     for (const Part& pt : sg.parts) total += pt.count;
-    W.reserve(total);
-    M.reserve(total);
-    G.reserve(total);
-    uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+    out.W.clear();
+    out.M.clear();
+    out.G.clear();
+    out.W.reserve(total);  // no reallocation below: the jobs keep pointers into these tables
+    out.M.reserve(total);
+    out.G.reserve(total);
     for (int q = 0; q < np; ++q) {
         const Part& pt = sg.parts[q];
         const auto& b = plan->buckets[pt.bucket];
         const ma_muon_hparams_t& hp = groups[b.group].muon;
-        MuonJob& J = jobs[q];
+        MuonJob& J = out.jobs[q];
         J.batch = pt.count;
         muon_geom(pt.count, b.R, b.C, hp, &J.g);
         J.gdt = plan->t[b.members[0]].grad_dtype;
         J.hp = &hp;
         J.ws = base;
         base += J.g.total;  // a multiple of the workspace alignment
-        const size_t off = W.size();
+        const size_t off = out.W.size();
         for (int k = 0; k < pt.count; ++k) {
             const ma_tensor_t& x = plan->t[b.members[pt.start + k]];
-            W.push_back(x.param);
-            G.push_back(x.grad);
-            M.push_back(x.state0);
+            out.W.push_back(x.param);
+            out.G.push_back(x.grad);
+            out.M.push_back(x.state0);
         }
-        J.W = W.data() + off;
-        J.G = G.data() + off;
-        J.M = M.data() + off;
+        J.W = out.W.data() + off;
+        J.G = out.G.data() + off;
+        J.M = out.M.data() + off;
     }
-    return run_muon_jobs(jobs.data(), np, s, sms, launches);
+}
+
+int run_adamw_segment(ma_plan* plan, const ma_group_t* groups, cudaStream_t s, int* launches) {
+    NvtxRange range("ma.adamw");
+    const int ngroups = (int)plan->group_kind.size();
+    AdamwGroupConst gc[MA_MAX_GROUPS];
+    std::memset(gc, 0, sizeof(gc));
+    for (int k = 0; k < ngroups; ++k)
+        if (groups[k].kind == MA_ADAMW) gc[k] = adamw_const(groups[k].adamw);
+    int st;
+    for (int dt = 0; dt < 2; ++dt) {
+        std::vector<AdamwItem> items;
+        for (int i : plan->adamw_idx) {
+            const ma_tensor_t& x = plan->t[i];
+            if (x.grad_dtype != dt) continue;
+            items.push_back({x.param, x.grad, x.state0, x.state1, tensor_numel(x), x.group});
+        }
+        if (!items.empty() && (st = run_adamw(items, dt, gc, ngroups, s, launches))) return st;
+    }
+    return MA_OK;
+}
+
+// Whether a segment's momentum passes may run on the side stream under the
+// Newton-Schulz chain of the segment before it: every unit flat (the flat
+// momentum kernel fits beside a Newton-Schulz CTA on an SM; the transposing
+// one needs a shared-memory tile that does not) and bf16 operands.
+bool side_prep_ok(const SegJobs& sj) {
+    for (const MuonJob& j : sj.jobs)
+        if (j.g.total > 0 && (j.g.transposed || j.hp->precision)) return false;
+    return true;
+}
+
+// Whether a segment's chain runs on the tensor cores (the CTAs the side
+// stream's momentum kernel is sized to run beside).
+bool tc_chain(const SegJobs& sj) {
+    for (const MuonJob& j : sj.jobs)
+        if (j.g.total > 0 && j.hp->precision) return false;
+    return true;
+}
+
+// The plan's side stream and an event pool on the current device.
+int side_resources(ma_plan* plan, int dev, size_t nevents, cudaStream_t* side) {
+    if (plan->side && plan->side_dev != dev) {
+        int cur = dev;
+        cudaSetDevice(plan->side_dev);
+        cudaStreamDestroy(plan->side);
+        for (cudaEvent_t e : plan->side_events) cudaEventDestroy(e);
+        cudaSetDevice(cur);
+        plan->side = nullptr;
+        plan->side_events.clear();
+    }
+    if (!plan->side) {
+        int lo = 0, hi = 0;
+        if (cudaDeviceGetStreamPriorityRange(&lo, &hi) != cudaSuccess) return MA_ERR_CUDA;
+        // the least priority: the Newton-Schulz kernels of the caller's stream go first
+        if (cudaStreamCreateWithPriority(&plan->side, cudaStreamNonBlocking, lo) != cudaSuccess) return MA_ERR_CUDA;
+        plan->side_dev = dev;
+    }
+    while (plan->side_events.size() < nevents) {
+        cudaEvent_t e;
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return MA_ERR_CUDA;
+        plan->side_events.push_back(e);
+    }
+    *side = plan->side;
+    return MA_OK;
+}
+
+// One step over segments, on stream s. ready (may be null): per segment, an
+// event its work must wait for (the host copies of its gradients).
+//
+// With the plan's double workspace (plan->region > 0), the Muon segments use
+// its two halves in turn, and the momentum pass of segment q + 1 runs on the
+// plan's side stream, on a small grid that fits beside the Newton-Schulz
+// CTAs, while segment q's chain runs: the HBM-bound pass hides under the
+// tensor-core work. The side stream starts after all work queued on s before
+// the step; segment q + 1's momentum pass waits for the chain of segment
+// q - 1, the last user of its workspace half; segment q + 1's chain waits for
+// its momentum pass; s waits for the side stream at the end. Every kernel
+// does the same arithmetic as on one stream, so the results are the same bits.
+int run_segments(ma_plan* plan, const ma_group_t* groups, const std::vector<Segment>& segs, void* ws, cudaStream_t s,
+                 int sms, int* launches, const cudaEvent_t* ready) {
+    std::vector<int> mi;  // Muon segments, in order
+    for (int k = 0; k < (int)segs.size(); ++k)
+        if (!segs[k].adamw) mi.push_back(k);
+    const int nm = (int)mi.size();
+    uint8_t* base = reinterpret_cast<uint8_t*>(ws);
+    const size_t region = plan->region;
+    std::vector<SegJobs> sj(nm);
+    for (int q = 0; q < nm; ++q) build_jobs(plan, groups, segs[mi[q]], base + (region ? (q & 1) * region : 0), sj[q]);
+    std::vector<char> on_side(nm, 0);
+    bool any_side = false;
+    for (int q = 1; q < nm && region; ++q) {
+        on_side[q] = side_prep_ok(sj[q]) && tc_chain(sj[q - 1]);
+        any_side = any_side || on_side[q];
+    }
+    cudaStream_t side = nullptr;
+    cudaEvent_t *ev_fork = nullptr, *ev_prep = nullptr, *ev_chain = nullptr;
+    int st;
+    if (any_side) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return MA_ERR_CUDA;
+        if ((st = side_resources(plan, dev, 2 + 2 * (size_t)nm, &side))) return st;
+        ev_fork = &plan->side_events[0];
+        ev_prep = &plan->side_events[1];
+        ev_chain = &plan->side_events[1 + nm];
+        if (cudaEventRecord(*ev_fork, s) != cudaSuccess || cudaStreamWaitEvent(side, *ev_fork, 0) != cudaSuccess)
+            return MA_ERR_CUDA;
+    }
+    bool side_work = false;
+    int q = 0;
+    for (int k = 0; k < (int)segs.size(); ++k) {
+        if (ready && cudaStreamWaitEvent(s, ready[k], 0) != cudaSuccess) return MA_ERR_CUDA;
+        if (segs[k].adamw) {
+            if ((st = run_adamw_segment(plan, groups, s, launches))) return st;
+            continue;
+        }
+        NvtxRange range("ma.muon");
+        SegJobs& cur = sj[q];
+        if (!on_side[q]) {
+            if ((st = prep_jobs(cur.jobs.data(), (int)cur.jobs.size(), s, kPrepBlocksPerSm * sms, launches)))
+                return st;
+        } else if (cudaStreamWaitEvent(s, ev_prep[q], 0) != cudaSuccess) {
+            return MA_ERR_CUDA;
+        }
+        if (q + 1 < nm && on_side[q + 1]) {
+            SegJobs& nx = sj[q + 1];
+            if (ready && cudaStreamWaitEvent(side, ready[mi[q + 1]], 0) != cudaSuccess) return MA_ERR_CUDA;
+            if (q >= 1 && cudaStreamWaitEvent(side, ev_chain[q - 1], 0) != cudaSuccess) return MA_ERR_CUDA;
+            // one block per SM: each sits beside that SM's Newton-Schulz CTA
+            if ((st = prep_jobs(nx.jobs.data(), (int)nx.jobs.size(), side, sms, launches, true))) return st;
+            if (cudaEventRecord(ev_prep[q + 1], side) != cudaSuccess) return MA_ERR_CUDA;
+            side_work = true;
+        }
+        if ((st = chain_jobs(cur.jobs.data(), (int)cur.jobs.size(), s, sms, launches))) return st;
+        if (any_side && cudaEventRecord(ev_chain[q], s) != cudaSuccess) return MA_ERR_CUDA;
+        ++q;
+    }
+    if (side_work) {
+        // join: s continues after everything queued on the side stream
+        if (cudaEventRecord(*ev_fork, side) != cudaSuccess || cudaStreamWaitEvent(s, *ev_fork, 0) != cudaSuccess)
+            return MA_ERR_CUDA;
+    }
+    return MA_OK;
 }
 
 }  // namespace
@@ -1105,7 +1336,7 @@ size_t ns_iterate_workspace_bytes(int batch, int64_t m, int64_t n) {
     if (batch < 0 || m < 0 || n < 0) return SIZE_MAX;
     const size_t x = align_up((size_t)batch * m * n * 2, kAlign);
     const size_t gm = align_up((size_t)batch * m * round8(m) * 2, kAlign);
-    return x + 2 * gm;
+    return x + 2 * gm + align_up(kNsCounterBytes, kAlign);  // + the launches' tile counters
 }
 
 int ns_iterate_bf16(int batch, int64_t m, int64_t n, const uint16_t* X_in, uint16_t* X_out, const float* coeffs,
@@ -1130,6 +1361,10 @@ int ns_iterate_bf16(int batch, int64_t m, int64_t n, const uint16_t* X_in, uint1
     void* T = base;
     void* Gb = base + align_up((size_t)batch * m * n * 2, kAlign);
     void* G2 = reinterpret_cast<uint8_t*>(Gb) + align_up((size_t)batch * m * round8(m) * 2, kAlign);
+    unsigned int* ctr =
+        reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(G2) + align_up((size_t)batch * m * round8(m) * 2, kAlign));
+    if (cudaMemsetAsync(ctr, 0, kNsCounterBytes, s) != cudaSuccess) return MA_ERR_CUDA;
+    int nlaunch = 0;
     NsParams p;
     std::memset(&p, 0, sizeof(p));
     p.units = batch;
@@ -1152,6 +1387,7 @@ int ns_iterate_bf16(int batch, int64_t m, int64_t n, const uint16_t* X_in, uint1
         const bool quint = cf[2] != 0.f;
         p.coef_gram = quint ? 1.f : cf[1];
         auto launch = [&](int mode, const void* xb, const void* gb) -> int {
+            p.tile_ctr = ctr + 2 * nlaunch++;
             const int pr = prof_begin(ns_prof_class(mode), s);
             cudaError_t e = launch_ns_tc(mode, p, xb, gb, sms, s);
             prof_end(pr, s, ns_flops(mode, batch, m, n), 0.0);
@@ -1288,34 +1524,60 @@ int ma_plan_create(const ma_tensor_t* t, int n, const ma_group_t* groups, int ng
         }
         if ((st = check_disjoint(w))) return fail(st);
     }
-    size_t need = 0;
-    for (auto& b : plan->buckets) {
-        const ma_muon_hparams_t& hp = groups[b.group].muon;
-        const int nb = (int)b.members.size();
-        int sub = std::min(nb, (int)MA_MAX_BATCH);
-        MuonGeom g;
-        if ((st = muon_geom(sub, b.R, b.C, hp, &g))) return fail(st);
-        const size_t target = cap > 0 ? cap : kSubBatchBytes;
-        while (g.total > target && sub > 1) {
-            sub = std::max(1, sub / 2);
-            muon_geom(sub, b.R, b.C, hp, &g);
+    // Sub-batch sizes for a per-segment workspace budget `target` (halving a
+    // bucket's sub-batch until it fits), then the workspace the step's
+    // segments need (small buckets share Newton-Schulz launches within
+    // `group` bytes) and how many Muon segments a step has. Returns nonzero
+    // when a bucket does not fit even one matrix at a time.
+    auto size_plan = [&](size_t target, size_t group, size_t* need_out, int* nseg) -> int {
+        size_t need = 0;
+        for (auto& b : plan->buckets) {
+            const ma_muon_hparams_t& hp = groups[b.group].muon;
+            const int nb = (int)b.members.size();
+            int sub = std::min(nb, (int)MA_MAX_BATCH);
+            MuonGeom g;
+            int r = muon_geom(sub, b.R, b.C, hp, &g);
+            if (r) return r;
+            while (g.total > target && sub > 1) {
+                sub = std::max(1, sub / 2);
+                muon_geom(sub, b.R, b.C, hp, &g);
+            }
+            if (g.total > target) return MA_ERR_WORKSPACE;
+            if (g.units > 65535 || g.m > INT_MAX || g.n > INT_MAX || g.parts > INT_MAX) return MA_ERR_UNSUPPORTED;
+            b.sub = sub;
+            need = std::max(need, g.total);
         }
-        if (cap > 0 && g.total > cap) return fail(MA_ERR_WORKSPACE);
-        if (g.units > 65535 || g.m > INT_MAX || g.n > INT_MAX || g.parts > INT_MAX) return fail(MA_ERR_UNSUPPORTED);
-        b.sub = sub;
-        need = std::max(need, g.total);
-    }
-    // Small buckets share Newton-Schulz launches (more tiles per launch, fewer
-    // launches) when the grouped workspace stays within the cap, or without a
-    // cap within the larger of the biggest single sub-batch and kGroupWsBytes.
-    const size_t limit = cap > 0 ? cap : std::max(need, kGroupWsBytes);
-    for (const Segment& sg : step_segments(plan, groups, 0, 0, false, limit)) {
-        size_t tot = 0;
-        for (const Part& pt : sg.parts) tot += part_ws(plan, groups, pt);
-        need = std::max(need, tot);
+        const size_t limit = group ? group : std::max(need, kGroupWsBytes);
+        int muon_segments = 0;
+        for (const Segment& sg : step_segments(plan, groups, 0, 0, false, limit)) {
+            size_t tot = 0;
+            for (const Part& pt : sg.parts) tot += part_ws(plan, groups, pt);
+            need = std::max(need, tot);
+            muon_segments += sg.adamw ? 0 : 1;
+        }
+        *need_out = need;
+        *nseg = muon_segments;
+        return MA_OK;
+    };
+    // A step with two or more Muon segments gets a workspace of two halves,
+    // so that one segment's momentum pass can run under the chain of the one
+    // before it: without a cap, halves of at most kSubBatchBytes (the
+    // sub-batch budget) each; with a cap, halves of at most half the cap when
+    // every bucket fits in that, else one workspace of at most the cap.
+    size_t need = 0;
+    int nseg = 0;
+    if (cap == 0) {
+        if ((st = size_plan(kSubBatchBytes, 0, &need, &nseg))) return fail(st);
+    } else if (size_plan(cap / 2, cap / 2, &need, &nseg) != MA_OK || nseg < 2) {
+        if ((st = size_plan(cap, cap, &need, &nseg))) return fail(st);
+        nseg = 0;  // no halves: one workspace within the cap
     }
     plan->ws_bytes = need;
-    *ws_bytes = need;
+    if (nseg >= 2 && need > 0) {
+        plan->region = align_up(need, kAlign);
+        plan->ws_bytes = 2 * plan->region;
+    }
+    *ws_bytes = plan->ws_bytes;
     *out = plan;
     return MA_OK;
 }
@@ -1327,8 +1589,9 @@ int muonadamw_step(ma_plan_t* plan, const ma_group_t* groups, void* ws, size_t w
     if (st) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     int launches = 0;
-    for (const Segment& sg : step_segments(plan, groups, 0, 0, false, plan->ws_bytes))
-        if ((st = launch_segment(plan, groups, sg, ws, s, sms, &launches))) return st;
+    st = run_segments(plan, groups, step_segments(plan, groups, 0, 0, false, seg_limit(plan)), ws, s, sms, &launches,
+                      nullptr);
+    if (st) return st;
     plan->last_launches = launches;
     return MA_OK;
 }
@@ -1400,8 +1663,11 @@ int graph_patch(ma_plan* plan, const ma_group_t* groups) {
     for (size_t i = 0; i < plan->t.size(); ++i)
         if (plan->kind[i] == MA_MUON) ctx.tensor_of[plan->t[i].param] = (int)i;
     for (ma_plan::GraphNode& n : plan->g.nodes) {
-        if (n.final_apply) {
+        if (n.final_apply == 1) {
             const int st = ns_tc_patch_final(n.arg.data(), patch_final_job, &ctx);
+            if (st) return st;
+        } else if (n.final_apply == 2) {
+            const int st = ns_cluster_patch(n.arg.data(), patch_final_job, &ctx);
             if (st) return st;
         } else {
             AdamwLaunch* L = reinterpret_cast<AdamwLaunch*>(n.arg.data());
@@ -1432,17 +1698,27 @@ int graph_capture(ma_plan* plan, const ma_group_t* groups, void* ws, int sms, in
         G.capture_dev = dev;
     }
     // everything that must not happen inside a capture: attribute set-up,
-    // driver entry points, the status-word address
-    if (ns_tc_setup(sms) != cudaSuccess || !device_status_ptr()) return MA_ERR_CUDA;
+    // driver entry points, the status-word address, the side stream
+    if (ns_tc_setup(sms) != cudaSuccess || prep_setup() != cudaSuccess || ns_cluster_setup() != cudaSuccess ||
+        !device_status_ptr())
+        return MA_ERR_CUDA;
+    if (plan->region) {
+        size_t nm = 0;
+        for (const Segment& sg : step_segments(plan, groups, 0, 0, false, seg_limit(plan))) nm += sg.adamw ? 0 : 1;
+        cudaStream_t side;
+        const int st0 = side_resources(plan, dev, 2 + 2 * nm, &side);
+        if (st0) return st0;
+    }
     const bool prof = g_prof_on;
     g_prof_on = false;
     if (cudaStreamBeginCapture(G.capture, cudaStreamCaptureModeThreadLocal) != cudaSuccess) {
         g_prof_on = prof;
         return MA_ERR_CUDA;
     }
-    int launches = 0, st = MA_OK;
-    for (const Segment& sg : step_segments(plan, groups, 0, 0, false, plan->ws_bytes))
-        if ((st = launch_segment(plan, groups, sg, ws, G.capture, sms, &launches))) break;
+    int launches = 0;
+    const int st =
+        run_segments(plan, groups, step_segments(plan, groups, 0, 0, false, seg_limit(plan)), ws, G.capture, sms,
+                     &launches, nullptr);
     cudaGraph_t graph = nullptr;
     const cudaError_t ec = cudaStreamEndCapture(G.capture, &graph);
     g_prof_on = prof;
@@ -1475,10 +1751,11 @@ int graph_capture(ma_plan* plan, const ma_group_t* groups, void* ws, int sms, in
         }
         const bool adamw = p.func == adamw_kernel_func();
         const bool fin = ns_tc_is_final(p.func);
-        if (!adamw && !fin) continue;
-        const size_t bytes = adamw ? sizeof(AdamwLaunch) : ns_tc_launch_bytes();
+        const bool chain = ns_cluster_is_kernel(p.func);  // a whole chain, final update included
+        if (!adamw && !fin && !chain) continue;
+        const size_t bytes = adamw ? sizeof(AdamwLaunch) : fin ? ns_tc_launch_bytes() : ns_cluster_launch_bytes();
         const uint8_t* a = reinterpret_cast<const uint8_t*>(p.kernelParams[0]);
-        G.nodes.push_back({node, p, std::vector<uint8_t>(a, a + bytes), fin ? 1 : 0});
+        G.nodes.push_back({node, p, std::vector<uint8_t>(a, a + bytes), fin ? 1 : chain ? 2 : 0});
     }
     G.launches = launches;
     ++G.captures;
@@ -1553,10 +1830,7 @@ int muonadamw_step_from_host(ma_plan_t* plan, const ma_group_t* groups, const vo
         if (cudaEventRecord(plan->events[k], cs) != cudaSuccess) return MA_ERR_CUDA;
     }
     int launches = 0;
-    for (size_t k = 0; k < segs.size(); ++k) {
-        if (cudaStreamWaitEvent(s, plan->events[k], 0) != cudaSuccess) return MA_ERR_CUDA;
-        if ((st = launch_segment(plan, groups, segs[k], ws, s, sms, &launches))) return st;
-    }
+    if ((st = run_segments(plan, groups, segs, ws, s, sms, &launches, plan->events.data()))) return st;
     plan->last_launches = launches;
     return MA_OK;
 }
@@ -1577,8 +1851,14 @@ int ma_plan_describe(const ma_plan_t* plan, const ma_group_t* groups, char* buf,
     char line[256];
     int64_t adamw_elems = 0;
     for (int i : plan->adamw_idx) adamw_elems += tensor_numel(plan->t[i]);
-    std::snprintf(line, sizeof(line), "workspace %zu bytes; AdamW: %zu tensors, %lld elements\n", plan->ws_bytes,
-                  plan->adamw_idx.size(), (long long)adamw_elems);
+    if (plan->region)
+        std::snprintf(line, sizeof(line),
+                      "workspace %zu bytes in two halves of %zu (momentum passes under the previous chain); "
+                      "AdamW: %zu tensors, %lld elements\n",
+                      plan->ws_bytes, plan->region, plan->adamw_idx.size(), (long long)adamw_elems);
+    else
+        std::snprintf(line, sizeof(line), "workspace %zu bytes; AdamW: %zu tensors, %lld elements\n", plan->ws_bytes,
+                      plan->adamw_idx.size(), (long long)adamw_elems);
     out += line;
     for (size_t bi = 0; bi < plan->buckets.size(); ++bi) {
         const auto& b = plan->buckets[bi];
@@ -1589,7 +1869,7 @@ int ma_plan_describe(const ma_plan_t* plan, const ma_group_t* groups, char* buf,
         out += line;
     }
     int si = 0;
-    for (const Segment& sg : step_segments(plan, groups, 0, 0, false, plan->ws_bytes)) {
+    for (const Segment& sg : step_segments(plan, groups, 0, 0, false, seg_limit(plan))) {
         if (sg.adamw) {
             std::snprintf(line, sizeof(line), "segment %d: AdamW\n", si++);
             out += line;
@@ -1675,7 +1955,7 @@ int ma_device_status_async(int32_t* host_dst, void* stream) {
 
 int ma_set_wait_limit_ns(int64_t limit_ns) {
     if (limit_ns <= 0) return MA_ERR_ARG;
-    g_host_wait_limit_ns = limit_ns;
+    g_host_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
     return MA_OK;
 }
 
@@ -1703,17 +1983,16 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[MA_STATIC_SCRAT
 
 // Device address of g_noalloc_scratch on the current device, looked up once per
 // device (host code only has a host-side stand-in for the symbol, which must
-// never be handed to a kernel). NULL if the lookup fails.
+// never be handed to a kernel). NULL if the lookup fails. Host threads making
+// their first call on a device at the same time are serialised by the cache.
 static void* noalloc_scratch_ptr() {
-    static void* cached[64] = {nullptr};
+    static ma::PerDevice<void*> cache;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!cached[dev]) {
-        void* ptr = nullptr;
-        if (cudaGetSymbolAddress((void**)&ptr, g_noalloc_scratch) != cudaSuccess) return nullptr;
-        cached[dev] = ptr;
-    }
-    return cached[dev];
+    if (cudaGetDevice(&dev) != cudaSuccess) return nullptr;
+    void* ptr = nullptr;
+    const cudaError_t e =
+        cache.get(dev, &ptr, [](void** v) { return cudaGetSymbolAddress(v, g_noalloc_scratch); });
+    return e == cudaSuccess ? ptr : nullptr;
 }
 
 extern "C" int muon_step_batched_noalloc(int batch, int64_t R, int64_t C, float* const* W, const void* const* G,

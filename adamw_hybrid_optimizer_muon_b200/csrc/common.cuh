@@ -114,6 +114,80 @@ __device__ __forceinline__ bool mbar_wait_bounded(uint64_t* bar, uint32_t parity
     }
 }
 
+// Same as mbar_try_wait, with acquire semantics at cluster scope: for a
+// barrier whose arrivals come from the peer CTA of a pair and publish data
+// (release at cluster scope on the arriving side).
+__device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar_addr, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar_addr), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// The block-local abort of a bounded wait, raised in this CTA and, for a CTA
+// pair, in the peer CTA too (so that both wind down together).
+struct AbortCtl {
+    volatile int* flag;  // this CTA's flag (shared memory)
+    uint32_t peer;       // shared::cluster address of the peer CTA's flag; 0 without a peer
+};
+
+__device__ __forceinline__ void st_cluster_s32(uint32_t cluster_addr, int v) {
+    asm volatile("st.shared::cluster.s32 [%0], %1;" ::"r"(cluster_addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int ld_cluster_s32(uint32_t cluster_addr) {
+    int v;
+    asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(cluster_addr) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void raise_abort(const AbortCtl& a) {
+    *a.flag = 1;
+    if (a.peer) st_cluster_s32(a.peer, 1);
+}
+
+// Bounded wait for the phase with the given parity of `bar`. Returns false
+// after recording MA_ERR_TIMEOUT and raising the abort (here and in the peer)
+// when the wait exceeds limit_ns, and, unless ignore_abort, as soon as the
+// abort is raised by any thread of the pair. cluster_acq: acquire at cluster
+// scope (arrivals from the peer CTA that publish data). sleep_ns > 0 lets the
+// thread sleep inside the wait instead of polling it.
+__device__ __forceinline__ bool mbar_wait_ctl(uint64_t* bar, uint32_t parity, const AbortCtl& ab, long long limit_ns,
+                                              int* status, uint32_t sleep_ns = 0, bool cluster_acq = false,
+                                              bool ignore_abort = false) {
+    const uint32_t a = smem_u32(bar);
+    auto probe = [&]() {
+        if (cluster_acq) return mbar_try_wait_cluster(a, parity, sleep_ns ? sleep_ns : 1u);
+        return sleep_ns ? mbar_try_wait_sleep(a, parity, sleep_ns) : mbar_try_wait(a, parity);
+    };
+    if (probe()) return true;
+    const uint64_t t0 = globaltimer();
+    for (uint32_t it = 0;; ++it) {
+        if (probe()) return true;
+        if (sleep_ns || cluster_acq || (it & 63u) == 63u) {
+            if (!ignore_abort && *ab.flag) return false;
+            if ((long long)(globaltimer() - t0) > limit_ns) {
+                record_error(status, MA_ERR_TIMEOUT);
+                raise_abort(ab);
+                return false;
+            }
+        }
+    }
+}
+
+// Complete `bytes` of the pending transaction count of the current phase of a
+// barrier of this CTA, as a bulk copy's arrival would (the abort drain uses it
+// for copies that were expected but never issued).
+__device__ __forceinline__ void mbar_complete_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.complete_tx.relaxed.cta.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+
 // ------------------------------------------------------------------ TMA
 
 // 3-D tiled bulk tensor load global -> shared, completing on `bar`.

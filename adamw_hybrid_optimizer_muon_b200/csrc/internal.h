@@ -9,9 +9,50 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "../../include/muonadamw.h"
 
 namespace ma {
+
+// ------------------------------------------------------------------ per-device host caches
+
+constexpr int kMaxDevices = 64;
+
+// A value looked up once per device (a symbol address, an occupancy figure,
+// kernel attributes set), safe when several host threads make their first
+// call on a device at the same time: the lookup runs under a mutex, at most
+// once per device while it succeeds, and readers after that take no lock.
+// A failed lookup is not cached, so the next call tries again. Objects of
+// this type live in static storage (zero-initialised before any call).
+template <typename T>
+class PerDevice {
+  public:
+    // *out = the cached value of device `dev`, computed by init(&value) (which
+    // returns a cudaError_t) on the first successful call.
+    template <typename Init>
+    cudaError_t get(int dev, T* out, Init init) {
+        if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+        if (!ready_[dev].load(std::memory_order_acquire)) {
+            std::lock_guard<std::mutex> lock(mu_);
+            if (!ready_[dev].load(std::memory_order_relaxed)) {
+                T v{};
+                const cudaError_t e = init(&v);
+                if (e != cudaSuccess) return e;
+                val_[dev] = v;
+                ready_[dev].store(1, std::memory_order_release);
+            }
+        }
+        *out = val_[dev];
+        return cudaSuccess;
+    }
+
+  private:
+    std::mutex mu_;
+    std::atomic<int> ready_[kMaxDevices];
+    T val_[kMaxDevices];
+};
 
 // ------------------------------------------------------------------ AdamW
 
@@ -49,8 +90,9 @@ const void* adamw_kernel_func();  // the kernel's host-side handle (CUDA-graph n
 
 // ------------------------------------------------------------------ Muon: momentum + norm
 
-constexpr int kPrepChunk = 8192;  // elements per block, flat path
-constexpr int kPrepTile = 64;     // tile edge, transposing path
+constexpr int kPrepChunk = 4096;   // elements per chunk (one partial sum each), flat path
+constexpr int kPrepThreads = 128;  // threads per block, flat path
+constexpr int kPrepTile = 64;      // tile edge, transposing path
 
 struct MuonPrepLaunch {
     int32_t batch, heads, transposed, gdt, nesterov, x_f32;
@@ -69,14 +111,27 @@ struct MuonPrepLaunch {
 // Number of per-block partial sums the momentum pass writes for one unit.
 int64_t prep_parts_per_unit(int64_t Rh, int64_t C, int transposed);
 
-cudaError_t launch_muon_prep(const MuonPrepLaunch& L, cudaStream_t s);
+// max_blocks > 0 bounds the flat path's grid (its blocks then walk the chunks
+// grid-stride; a small grid runs beside the Newton-Schulz kernels of another
+// batch); 0: one block per chunk. The transposing path ignores it.
+cudaError_t launch_muon_prep(const MuonPrepLaunch& L, int max_blocks, cudaStream_t s);
+// Per-device kernel attributes of the momentum kernels, ahead of a stream capture.
+cudaError_t prep_setup();
 // scale[u] = 1 / (sqrt(sum of the unit's partials) + eps), deterministic order.
+// Also zeroes the nctr tile counters of the Newton-Schulz launches that follow.
 cudaError_t launch_norm_finalize(const double* partials, int64_t parts, int units, float eps, float* scale,
-                                 cudaStream_t s);
+                                 unsigned int* ctr, int nctr, cudaStream_t s);
 
 // ------------------------------------------------------------------ Newton-Schulz
 
 enum NsMode { NS_GRAM = 0, NS_APPLY = 1, NS_FINAL = 2, NS_GRAMSQ = 3 };
+
+// Tile counters of one Newton-Schulz chain (in the workspace): two per launch
+// (the CTA-pair kernel and the single-CTA kernel of a grouped launch), at most
+// three launches per iteration.
+constexpr int kNsCounters = 2 * 3 * MA_MAX_NS_STEPS;
+constexpr size_t kNsCounterBytes = 512;
+static_assert(kNsCounters * sizeof(unsigned int) <= kNsCounterBytes, "tile counters");
 
 struct NsParams {
     int32_t units, m, n;
@@ -96,6 +151,7 @@ struct NsParams {
     int32_t cautious;        // decay only where X_N * W > 0
     long long wait_limit_ns;
     int* status;             // per-device status word
+    unsigned int* tile_ctr;  // two zeroed counters of this launch (tcgen05 path)
     float* W[MA_MAX_BATCH];
 };
 
@@ -127,6 +183,43 @@ typedef int (*NsFinalPatchFn)(void* ctx, const float* W, int64_t Rh, int64_t C, 
 bool ns_tc_is_final(const void* func);
 size_t ns_tc_launch_bytes();
 int ns_tc_patch_final(void* launch, NsFinalPatchFn f, void* ctx);
+
+// Cluster-resident chain for short units (m <= 128, rows <= columns, n <= 4096,
+// no A^2 term): one launch runs all iterations of a batch and the final
+// update of W (ns_cluster.cu).
+struct NsClusterIn {
+    const void* x;             // X0, bf16 [units][m][ldx]
+    int64_t ldx, x_unit;
+    int32_t units, m, n, steps;
+    float coef[MA_MAX_NS_STEPS][2];  // (a, b) of each iteration
+    const float* scale;        // per-unit 1 / (||u|| + eps)
+    int32_t heads;
+    int64_t Rh, C;
+    float decay, lr_s, lr_wd;
+    int32_t cautious;
+    long long wait_limit_ns;
+    int* status;
+    float* const* W;           // units / heads weight matrices
+};
+struct NsClusterLaunch {
+    CUtensorMap mapX;
+    int32_t m, n, nc, steps;
+    float coef[MA_MAX_NS_STEPS][2];
+    const float* scale;
+    int32_t heads, cautious;
+    int64_t Rh, C;
+    float decay, lr_s, lr_wd;
+    long long wait_limit_ns;
+    int* status;
+    float* W[MA_MAX_BATCH];
+};
+bool ns_cluster_eligible(int m, int n, int transposed);
+int ns_cluster_cols(int n);  // columns of X each CTA of a unit's cluster holds
+cudaError_t ns_cluster_setup();
+cudaError_t launch_ns_cluster(const NsClusterIn& in, cudaStream_t s);
+bool ns_cluster_is_kernel(const void* func);
+size_t ns_cluster_launch_bytes();
+int ns_cluster_patch(void* launch, NsFinalPatchFn f, void* ctx);
 
 // fp32 SIMT path (precision mode 1).
 cudaError_t launch_ns_simt(int mode, const NsParams& p, const void* x_buf, const void* g_buf, cudaStream_t s);

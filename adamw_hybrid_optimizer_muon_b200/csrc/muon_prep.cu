@@ -28,7 +28,11 @@ namespace ma {
 
 namespace {
 
-__device__ __forceinline__ float block_sum_256(float v, float* red) {
+// Sum of v over the block's NT threads in a fixed order (a butterfly within
+// each warp, then the warps in order); thread 0 gets it. `red` may be reused
+// by the next call, hence the trailing barrier.
+template <int NT>
+__device__ __forceinline__ float block_sum(float v, float* red) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
     const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
@@ -37,8 +41,9 @@ __device__ __forceinline__ float block_sum_256(float v, float* red) {
     float t = 0.f;
     if (threadIdx.x == 0) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) t += red[i];
+        for (int i = 0; i < NT / 32; ++i) t += red[i];
     }
+    __syncthreads();
     return t;
 }
 
@@ -84,64 +89,73 @@ __device__ __forceinline__ void store_x8(void* X, int64_t i, const float (&d)[8]
     }
 }
 
-// Flat path: one block per 8192-element chunk of one unit. A full chunk issues
+// Flat path: blocks of kPrepThreads threads walk the (unit, chunk) pairs of
+// the launch, kPrepChunk elements per chunk, grid-stride. A full chunk issues
 // all of its loads (4 groups of 8 elements per thread) before any arithmetic,
-// so each thread keeps 12 independent 16-byte loads in flight.
+// so each thread keeps 12 independent 16-byte loads in flight. The launch
+// bounds keep the kernel at most 85 registers a thread, and it uses 16 bytes
+// of shared memory: a block fits on an SM beside a Newton-Schulz CTA, so a
+// small grid of it can run under the tensor-core kernels of another batch.
+// The partial of a chunk does not depend on the grid size.
 template <bool GBF16, bool XF32>
-__global__ void __launch_bounds__(256) prep_flat_kernel(const __grid_constant__ MuonPrepLaunch L) {
+__global__ void __launch_bounds__(kPrepThreads, 6) prep_flat_kernel(const __grid_constant__ MuonPrepLaunch L) {
     griddep_launch_dependents();
     griddep_wait();
-    __shared__ float red[8];
-    constexpr int kIter = kPrepChunk / (8 * 256);
-    const int u = blockIdx.y;
-    const int b = u / L.heads, h = u % L.heads;
+    __shared__ float red[kPrepThreads / 32];
+    constexpr int kIter = kPrepChunk / (8 * kPrepThreads);
     const int64_t unit_elems = L.Rh * L.C;
-    const int64_t off = (int64_t)h * unit_elems;
-    const int64_t start = (int64_t)blockIdx.x * kPrepChunk;
-    const int64_t end = min(start + (int64_t)kPrepChunk, unit_elems);
-    float* M = L.M[b] + off;
-    const void* G = GBF16 ? static_cast<const void*>(reinterpret_cast<const uint16_t*>(L.G[b]) + off)
-                          : static_cast<const void*>(reinterpret_cast<const float*>(L.G[b]) + off);
-    void* X = XF32 ? static_cast<void*>(reinterpret_cast<float*>(L.X) + (int64_t)u * L.x_unit)
-                   : static_cast<void*>(reinterpret_cast<uint16_t*>(L.X) + (int64_t)u * L.x_unit);
+    const int64_t items = (int64_t)L.batch * L.heads * L.parts;
     const float beta = L.beta, omb = L.omb;
     const bool nest = L.nesterov != 0;
-    float ss = 0.f;
-    if (end - start == kPrepChunk) {
-        float g[kIter][8], m[kIter][8];
+    for (int64_t w = blockIdx.x; w < items; w += gridDim.x) {
+        const int u = (int)(w / L.parts);
+        const int64_t part = w - (int64_t)u * L.parts;
+        const int b = u / L.heads, h = u % L.heads;
+        const int64_t off = (int64_t)h * unit_elems;
+        const int64_t start = part * kPrepChunk;
+        const int64_t end = min(start + (int64_t)kPrepChunk, unit_elems);
+        float* M = L.M[b] + off;
+        const void* G = GBF16 ? static_cast<const void*>(reinterpret_cast<const uint16_t*>(L.G[b]) + off)
+                              : static_cast<const void*>(reinterpret_cast<const float*>(L.G[b]) + off);
+        void* X = XF32 ? static_cast<void*>(reinterpret_cast<float*>(L.X) + (int64_t)u * L.x_unit)
+                       : static_cast<void*>(reinterpret_cast<uint16_t*>(L.X) + (int64_t)u * L.x_unit);
+        float ss = 0.f;
+        if (end - start == kPrepChunk) {
+            float g[kIter][8], m[kIter][8];
 #pragma unroll
-        for (int k = 0; k < kIter; ++k) {
-            const int64_t i = start + 8 * ((int64_t)k * 256 + threadIdx.x);
-            load_g8<GBF16>(G, i, g[k]);
-            const float4 a = __ldcs(reinterpret_cast<const float4*>(M + i));
-            const float4 c = __ldcs(reinterpret_cast<const float4*>(M + i + 4));
-            m[k][0] = a.x; m[k][1] = a.y; m[k][2] = a.z; m[k][3] = a.w;
-            m[k][4] = c.x; m[k][5] = c.y; m[k][6] = c.z; m[k][7] = c.w;
-        }
+            for (int k = 0; k < kIter; ++k) {
+                const int64_t i = start + 8 * ((int64_t)k * kPrepThreads + threadIdx.x);
+                load_g8<GBF16>(G, i, g[k]);
+                const float4 a = __ldcs(reinterpret_cast<const float4*>(M + i));
+                const float4 c = __ldcs(reinterpret_cast<const float4*>(M + i + 4));
+                m[k][0] = a.x; m[k][1] = a.y; m[k][2] = a.z; m[k][3] = a.w;
+                m[k][4] = c.x; m[k][5] = c.y; m[k][6] = c.z; m[k][7] = c.w;
+            }
 #pragma unroll
-        for (int k = 0; k < kIter; ++k) {
-            const int64_t i = start + 8 * ((int64_t)k * 256 + threadIdx.x);
-            float d[8];
-            ss += momentum8(m[k], g[k], d, beta, omb, nest);
-            __stcs(reinterpret_cast<float4*>(M + i), make_float4(m[k][0], m[k][1], m[k][2], m[k][3]));
-            __stcs(reinterpret_cast<float4*>(M + i + 4), make_float4(m[k][4], m[k][5], m[k][6], m[k][7]));
-            store_x8<XF32>(X, i, d);
+            for (int k = 0; k < kIter; ++k) {
+                const int64_t i = start + 8 * ((int64_t)k * kPrepThreads + threadIdx.x);
+                float d[8];
+                ss += momentum8(m[k], g[k], d, beta, omb, nest);
+                __stcs(reinterpret_cast<float4*>(M + i), make_float4(m[k][0], m[k][1], m[k][2], m[k][3]));
+                __stcs(reinterpret_cast<float4*>(M + i + 4), make_float4(m[k][4], m[k][5], m[k][6], m[k][7]));
+                store_x8<XF32>(X, i, d);
+            }
+        } else {
+            for (int64_t i = start + 8 * (int64_t)threadIdx.x; i < end; i += 8 * kPrepThreads) {
+                float g[8], m[8], d[8];
+                load_g8<GBF16>(G, i, g);
+                const float4 a = __ldcs(reinterpret_cast<const float4*>(M + i));
+                const float4 c = __ldcs(reinterpret_cast<const float4*>(M + i + 4));
+                m[0] = a.x; m[1] = a.y; m[2] = a.z; m[3] = a.w; m[4] = c.x; m[5] = c.y; m[6] = c.z; m[7] = c.w;
+                ss += momentum8(m, g, d, beta, omb, nest);
+                __stcs(reinterpret_cast<float4*>(M + i), make_float4(m[0], m[1], m[2], m[3]));
+                __stcs(reinterpret_cast<float4*>(M + i + 4), make_float4(m[4], m[5], m[6], m[7]));
+                store_x8<XF32>(X, i, d);
+            }
         }
-    } else {
-        for (int64_t i = start + 8 * (int64_t)threadIdx.x; i < end; i += 8 * 256) {
-            float g[8], m[8], d[8];
-            load_g8<GBF16>(G, i, g);
-            const float4 a = __ldcs(reinterpret_cast<const float4*>(M + i));
-            const float4 c = __ldcs(reinterpret_cast<const float4*>(M + i + 4));
-            m[0] = a.x; m[1] = a.y; m[2] = a.z; m[3] = a.w; m[4] = c.x; m[5] = c.y; m[6] = c.z; m[7] = c.w;
-            ss += momentum8(m, g, d, beta, omb, nest);
-            __stcs(reinterpret_cast<float4*>(M + i), make_float4(m[0], m[1], m[2], m[3]));
-            __stcs(reinterpret_cast<float4*>(M + i + 4), make_float4(m[4], m[5], m[6], m[7]));
-            store_x8<XF32>(X, i, d);
-        }
+        const float tot = block_sum<kPrepThreads>(ss, red);
+        if (threadIdx.x == 0) L.partials[(int64_t)u * L.parts + part] = (double)tot;
     }
-    const float tot = block_sum_256(ss, red);
-    if (threadIdx.x == 0) L.partials[(int64_t)u * L.parts + blockIdx.x] = (double)tot;
 }
 
 // Transposing path (tall units, X = u^T). A 64 x 64 tile: each thread reads
@@ -242,16 +256,19 @@ __global__ void __launch_bounds__(256) prep_transpose_kernel(const __grid_consta
             }
         }
     }
-    const float tot = block_sum_256(ss, red);
+    const float tot = block_sum<256>(ss, red);
     if (threadIdx.x == 0) L.partials[(int64_t)u * L.parts + blockIdx.x] = (double)tot;
 }
 
 // One warp per unit: lane-strided sum of the unit's partials, then a fixed
-// butterfly, so the result does not depend on scheduling.
+// butterfly, so the result does not depend on scheduling. Block 0 also zeroes
+// the tile counters of the Newton-Schulz launches that follow.
 __global__ void __launch_bounds__(256) norm_finalize_kernel(const double* __restrict__ partials, int64_t parts,
-                                                            int units, float eps, float* __restrict__ scale) {
+                                                            int units, float eps, float* __restrict__ scale,
+                                                            unsigned int* __restrict__ ctr, int nctr) {
     griddep_launch_dependents();
     griddep_wait();
+    if (blockIdx.x == 0 && (int)threadIdx.x < nctr) ctr[threadIdx.x] = 0u;
     const int u = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int l = threadIdx.x & 31;
     if (u >= units) return;
@@ -269,31 +286,62 @@ int64_t prep_parts_per_unit(int64_t Rh, int64_t C, int transposed) {
     return (Rh * C + kPrepChunk - 1) / kPrepChunk;
 }
 
-cudaError_t launch_muon_prep(const MuonPrepLaunch& L, cudaStream_t s) {
+// The flat kernels prefer the largest shared-memory carveout, the one a
+// Newton-Schulz CTA sets on its SM, so that their blocks can join that SM.
+// Once per device; the attribute is set before any stream capture by the
+// library's set-up (the first call on a device).
+cudaError_t prep_setup() {
+    static PerDevice<int> cache;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    int done = 0;
+    return cache.get(dev, &done, [](int* v) -> cudaError_t {
+        const void* fns[4] = {reinterpret_cast<const void*>(prep_flat_kernel<true, false>),
+                              reinterpret_cast<const void*>(prep_flat_kernel<true, true>),
+                              reinterpret_cast<const void*>(prep_flat_kernel<false, false>),
+                              reinterpret_cast<const void*>(prep_flat_kernel<false, true>)};
+        for (const void* f : fns) {
+            const cudaError_t r = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                                       cudaSharedmemCarveoutMaxShared);
+            if (r != cudaSuccess) return r;
+        }
+        *v = 1;
+        return cudaSuccess;
+    });
+}
+
+cudaError_t launch_muon_prep(const MuonPrepLaunch& L, int max_blocks, cudaStream_t s) {
     const int units = L.batch * L.heads;
     if (units == 0 || L.parts == 0) return cudaSuccess;
-    dim3 grid((unsigned)L.parts, (unsigned)units);
     const bool gb = L.gdt == MA_BF16, xf = L.x_f32 != 0;
     cudaError_t e;
     if (L.transposed) {
+        const dim3 grid((unsigned)L.parts, (unsigned)units);
         if (gb && !xf) e = launch_pdl(prep_transpose_kernel<true, false>, grid, dim3(256), 0, s, L);
         else if (gb) e = launch_pdl(prep_transpose_kernel<true, true>, grid, dim3(256), 0, s, L);
         else if (!xf) e = launch_pdl(prep_transpose_kernel<false, false>, grid, dim3(256), 0, s, L);
         else e = launch_pdl(prep_transpose_kernel<false, true>, grid, dim3(256), 0, s, L);
     } else {
-        if (gb && !xf) e = launch_pdl(prep_flat_kernel<true, false>, grid, dim3(256), 0, s, L);
-        else if (gb) e = launch_pdl(prep_flat_kernel<true, true>, grid, dim3(256), 0, s, L);
-        else if (!xf) e = launch_pdl(prep_flat_kernel<false, false>, grid, dim3(256), 0, s, L);
-        else e = launch_pdl(prep_flat_kernel<false, true>, grid, dim3(256), 0, s, L);
+        if ((e = prep_setup()) != cudaSuccess) return e;
+        int64_t items = (int64_t)units * L.parts;
+        if (max_blocks > 0 && items > max_blocks) items = max_blocks;
+        if (items > INT32_MAX) items = INT32_MAX;
+        const dim3 grid((unsigned)items), block(kPrepThreads);
+        if (gb && !xf) e = launch_pdl(prep_flat_kernel<true, false>, grid, block, 0, s, L);
+        else if (gb) e = launch_pdl(prep_flat_kernel<true, true>, grid, block, 0, s, L);
+        else if (!xf) e = launch_pdl(prep_flat_kernel<false, false>, grid, block, 0, s, L);
+        else e = launch_pdl(prep_flat_kernel<false, true>, grid, block, 0, s, L);
     }
     return e;
 }
 
 cudaError_t launch_norm_finalize(const double* partials, int64_t parts, int units, float eps, float* scale,
-                                 cudaStream_t s) {
+                                 unsigned int* ctr, int nctr, cudaStream_t s) {
     if (units == 0) return cudaSuccess;
+    if (nctr < 0 || nctr > 256 || (nctr > 0 && !ctr)) return cudaErrorInvalidValue;
     return launch_pdl(norm_finalize_kernel, dim3((units + 7) / 8), dim3(256), 0, s, partials, parts, units, eps,
-                      scale);
+                      scale, ctr, nctr);
 }
 
 }  // namespace ma

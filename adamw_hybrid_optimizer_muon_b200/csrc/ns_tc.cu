@@ -85,6 +85,46 @@ constexpr uint32_t WBUF_BYTES = EPI_WARPS * FIN_WARP_BYTES;      // 96 KB
 constexpr int kStages(int mode) { return mode == NS_FINAL ? 4 : STAGES; }
 constexpr uint32_t kEpiBytes(int mode) { return mode == NS_FINAL ? WBUF_BYTES : STG_BYTES; }
 
+// Tiles are handed out at run time: the leader's producer thread takes the
+// next tile index from the launch's counter (one atomic add per tile, ahead
+// of need) and publishes it to the pair's other roles through a ring of
+// kRing slots in shared memory, two tiles ahead of its own loads. The pairs
+// running at any moment therefore work on a contiguous window of the
+// launch's tile order, whatever their speed, which keeps the operand strips
+// that window shares in L2. A tile's arithmetic does not depend on which pair
+// computes it.
+//
+// A slot needs no "consumed" barrier: when the leader writes the slot of tile
+// s + 2 (about to load tile s), it has issued every load of tile s - 1, so the
+// MMA thread has consumed a stage use of tile s - 1 - NST or later (the stage
+// ring allows no more), which it did after taking that tile and after the
+// epilogue warps of both CTAs released tile s - 3 - NST; each epilogue warp
+// takes its next tile before it releases the current one, so all of them
+// have taken tile s - 2 - NST; the peer's producer issued the loads the MMA
+// thread consumed. Every consumer has therefore taken tile s + 2 - kRing
+// whenever kRing >= NST + 4.
+constexpr int kMaxStages = 8;
+constexpr int kRing = kMaxStages + 4;
+// Wind-down after an abort: waits for the pair's own work in flight (issued
+// MMAs, bulk loads) are bounded by at least this, whatever the wait limit.
+constexpr long long kDrainNs = 50000000LL;
+
+// Control block in shared memory, after the stage ring and the epilogue
+// buffers. Its offsets are the same in both CTAs of a pair.
+struct Ctl {
+    uint64_t full[kMaxStages], empty[kMaxStages];  // stage ring: data landed / stage released by the MMAs
+    uint64_t acc_full[2], acc_empty[2];            // TMEM accumulators: ready for the epilogue / free again
+    uint64_t drain;                                // the MMA thread's last commit before an aborted exit
+    uint64_t tile_full[kRing];                     // tile ring: index published
+    int32_t tile_id[kRing];                        // tile index of each ring slot, -1 = no more tiles
+    uint32_t tmem_base;
+    int32_t abort_flag;
+    int32_t issued;                    // producer: stage uses armed and loaded so far
+    int32_t consumed;                  // MMA thread: stage uses whose data it has waited for
+    uint32_t stage_tx[kMaxStages];     // producer: bytes per CTA of the latest use of each stage
+};
+static_assert(sizeof(Ctl) <= 512, "control block");
+
 // Tile shape of one kernel instance. PAIR: a CTA pair computes a 256 x 256
 // tile (cta_group::2, each CTA holding 128 rows of A and 128 columns of B).
 // Single CTA (for units with m <= 128, where a 256-row tile would be half
@@ -104,6 +144,7 @@ struct Shape {
     static constexpr int CPW = TN / 64;                             // 32-column chunks per epilogue warp
     static constexpr size_t SMEM = (size_t)NST * STAGE + EPI + 1024 + 512;
     static_assert(SMEM <= 232448, "shared memory");
+    static_assert(NST <= kMaxStages, "stage ring");
 };
 
 struct TileCoord {
@@ -135,6 +176,7 @@ struct NsLaunch {
     int32_t njobs, total_tiles;
     long long wait_limit_ns;
     int* status;
+    unsigned int* tile_ctr;  // zero before the launch; one atomic add per tile handed out
     float* W[kMaxW];
 };
 
@@ -246,6 +288,49 @@ __device__ __forceinline__ uint32_t sw64(uint32_t r, uint32_t q) { return r * 64
 // Byte offset of 16-byte chunk q of row r in a 128-byte-row block of W.
 __device__ __forceinline__ uint32_t sw128w(uint32_t r, uint32_t q) { return r * 128u + ((q ^ (r & 7u)) << 4); }
 
+// ------------------------------------------------------------------ tile ring
+
+// Leader's producer: publish tile index t (-1: no more tiles) as sequence
+// number seq, in this CTA and in the peer CTA of the pair. Every consumer is
+// done with the slot's previous use (see kRing).
+template <bool PAIR>
+__device__ __forceinline__ void ring_publish(Ctl* ctl, int seq, int t) {
+    const int slot = seq % kRing;
+    ctl->tile_id[slot] = t;
+    if (PAIR) {
+        st_cluster_s32(mapa_shared(smem_u32(&ctl->tile_id[slot]), 1), t);
+        mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->tile_full[slot]), 1));  // release: the store above first
+    }
+    mbar_arrive(&ctl->tile_full[slot]);
+}
+
+// Consumer (one thread): the tile index of sequence number seq. Returns -1
+// with *ok = false when the wait gave up (timeout or abort).
+template <bool PAIR>
+__device__ __forceinline__ int ring_take(Ctl* ctl, int seq, uint32_t rank, const AbortCtl& ab, const NsLaunch& L,
+                                         uint32_t sleep_ns, bool* ok) {
+    const int slot = seq % kRing;
+    const uint32_t par = (uint32_t)(seq / kRing) & 1u;
+    const bool remote = PAIR && rank != 0;
+    if (!mbar_wait_ctl(&ctl->tile_full[slot], par, ab, L.wait_limit_ns, L.status, sleep_ns, remote)) {
+        *ok = false;
+        return -1;
+    }
+    *ok = true;
+    return reinterpret_cast<volatile int32_t*>(ctl->tile_id)[slot];
+}
+
+// Epilogue warp: the tile of sequence number seq (lane 0 takes it from the
+// ring, the warp shares it); -1 when there are no more tiles or on an abort.
+template <bool PAIR>
+__device__ __forceinline__ int epi_take(Ctl* ctl, int seq, uint32_t rank, const AbortCtl& ab, const NsLaunch& L,
+                                        int lane) {
+    int t = -1;
+    bool ok = true;
+    if (lane == 0) t = ring_take<PAIR>(ctl, seq, rank, ab, L, kEpiSleepNs, &ok);
+    return __shfl_sync(0xffffffffu, t, 0);
+}
+
 // Final apply: W <- W*(1 - lr*wd) - lr*scale*X_N in the caller's fp32 weights,
 // run by each epilogue warp over its 32-column chunks of every tile.
 //
@@ -259,18 +344,18 @@ __device__ __forceinline__ uint32_t sw128w(uint32_t r, uint32_t q) { return r * 
 // (or, transposed, its own column) of the W block in place, and the block
 // goes back to W with coalesced 16-byte stores.
 template <bool PAIR>
-__device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int npairs, uint32_t rank,
-                                               uint32_t tmem_base, int warp, int lane, uint8_t* wbuf,
-                                               uint64_t* acc_full, uint64_t* acc_empty, volatile int* abort_flag) {
+__device__ __forceinline__ void final_epilogue(const NsLaunch& L, Ctl* ctl, uint32_t rank, uint32_t tmem_base,
+                                               int warp, int lane, uint8_t* wbuf, const AbortCtl& ab) {
     using S = Shape<NS_FINAL, PAIR>;
     constexpr int CPW = S::CPW;
     const int quad = warp & 3, half = (warp - 2) / 4;
     const long long limit = L.wait_limit_ns;
-    const uint32_t acc_empty_leader0 = PAIR ? mapa_shared(smem_u32(&acc_empty[0]), 0) : 0u;
-    const uint32_t acc_empty_leader1 = PAIR ? mapa_shared(smem_u32(&acc_empty[1]), 0) : 0u;
+    const uint32_t acc_empty_leader0 = PAIR ? mapa_shared(smem_u32(&ctl->acc_empty[0]), 0) : 0u;
+    const uint32_t acc_empty_leader1 = PAIR ? mapa_shared(smem_u32(&ctl->acc_empty[1]), 0) : 0u;
     uint8_t* xbuf = wbuf + 2 * WBUF;
-    int lt = 0;
-    for (int t = pair; t < L.total_tiles; t += npairs, ++lt) {
+    // each tile is taken before the previous accumulator is released (see kRing)
+    int t = epi_take<PAIR>(ctl, 0, rank, ab, L, lane);
+    for (int lt = 0; t >= 0; ++lt) {  // -1: no more tiles, or an abort
         const JobTile jt = decode_job_tile(L, NS_FINAL, t);
         const NsJob& p = L.job[jt.j];
         const TileCoord tc = jt.tc;
@@ -317,7 +402,8 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int 
         fetch(0);
         fetch(1);
         int ok = 1;
-        if (lane == 0) ok = mbar_wait_bounded(&acc_full[acc], use & 1u, abort_flag, limit, L.status, kEpiSleepNs) ? 1 : 0;
+        if (lane == 0)
+            ok = mbar_wait_ctl(&ctl->acc_full[acc], use & 1u, ab, limit, L.status, kEpiSleepNs) ? 1 : 0;
         ok = __shfl_sync(0xffffffffu, ok, 0);
         if (!ok) break;
         tc_fence_after();
@@ -367,25 +453,63 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, int pair, int 
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int row = 4 * i + (lane >> 3), q = lane & 7;
+                // streaming stores (evict-first in L2): the updated weights are not
+                // read again in this launch, unlike the Gram and X strips
                 if (row < nr && q * 16 < rb)
-                    *reinterpret_cast<float4*>(Wb + (int64_t)(r0 + row) * p.C + c0 + q * 4) =
-                        *reinterpret_cast<const float4*>(buf + sw128w(row, q));
+                    __stcs(reinterpret_cast<float4*>(Wb + (int64_t)(r0 + row) * p.C + c0 + q * 4),
+                           *reinterpret_cast<const float4*>(buf + sw128w(row, q)));
             }
             __syncwarp();  // both buffers of chunk c are free again
             fetch(c + 2);
         }
         cp_async_wait<0>();  // drop the copies of chunks this tile does not use
-        if (!ok) break;
+        t = epi_take<PAIR>(ctl, lt + 1, rank, ab, L, lane);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
             if (PAIR) mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);
-            else mbar_arrive(&acc_empty[acc]);
+            else mbar_arrive(&ctl->acc_empty[acc]);
         }
     }
     cp_async_wait<0>();
 }
 
+// After an abort, with every role of both CTAs stopped (no thread issues
+// anything more), the leader's MMA thread waits for the pair's work in
+// flight, bounded by the drain limit but not cut short by the abort:
+//  * every MMA it issued (one more commit, on the drain barrier);
+//  * every bulk load either producer issued that the MMAs never consumed.
+//    Each such stage use has at most one outstanding phase. Where both
+//    producers issued it, the phase completes when the bytes land. Where only
+//    the leader did (it armed the barrier for both CTAs' bytes), the peer's
+//    missing bytes are completed by hand; where only the peer did (the leader
+//    never armed it), the leader arms it for the peer's bytes. Either way the
+//    phase then completes exactly when the issued copies have landed.
+// Returns normally in every case; a drain wait that runs out records
+// MA_ERR_TIMEOUT like any other wait.
+template <int NST, bool PAIR>
+__device__ __forceinline__ void abort_drain(Ctl* ctl, const AbortCtl& ab, const NsLaunch& L) {
+    const long long lim = L.wait_limit_ns > kDrainNs ? L.wait_limit_ns : kDrainNs;
+    if (PAIR) tc_commit_pair(&ctl->drain);
+    else tc_commit(&ctl->drain);
+    mbar_wait_ctl(&ctl->drain, 0, ab, lim, L.status, 0, false, true);
+    const int consumed = ctl->consumed;
+    const int own = ctl->issued;
+    const int peer = PAIR ? ld_cluster_s32(mapa_shared(smem_u32(&ctl->issued), 1)) : own;
+    const int last = own > peer ? own : peer;
+    for (int u = consumed; u < last; ++u) {
+        const int st = u % NST;
+        const uint32_t par = (uint32_t)(u / NST) & 1u;
+        const bool mine = u < own, theirs = u < peer;
+        if (PAIR && mine && !theirs) {
+            mbar_complete_tx(&ctl->full[st], ctl->stage_tx[st]);
+        } else if (PAIR && theirs && !mine) {
+            const uint32_t tx = (uint32_t)ld_cluster_s32(mapa_shared(smem_u32(&ctl->stage_tx[st]), 1));
+            mbar_arrive_expect_tx(&ctl->full[st], tx);
+        }
+        mbar_wait_ctl(&ctl->full[st], par, ab, lim, L.status, 0, PAIR, true);
+    }
+}
 
 template <int MODE, bool PAIR>
 __global__ void __launch_bounds__(THREADS, 1)
@@ -395,37 +519,31 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int NST = S::NST;
     uint8_t* staging = smem + NST * S::STAGE;
-    uint64_t* full = reinterpret_cast<uint64_t*>(staging + S::EPI);
-    uint64_t* empty = full + NST;
-    uint64_t* acc_full = empty + NST;
-    uint64_t* acc_empty = acc_full + 2;
-    uint64_t* drain = acc_empty + 2;
-    uint64_t* wbar = drain + 1;  // final apply: 2 per epilogue warp
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(wbar + 2 * EPI_WARPS);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+    Ctl* ctl = reinterpret_cast<Ctl*>(staging + S::EPI);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     griddep_launch_dependents();
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = leader of the pair
     const bool leader = rank == 0;
-    const int pair = PAIR ? (int)cluster_id_x() : (int)blockIdx.x;
-    const int npairs = PAIR ? (int)cluster_count_x() : (int)gridDim.x;
     const int total_tiles = L.total_tiles;
     const long long limit = L.wait_limit_ns;
     constexpr bool kApply = (MODE == NS_APPLY || MODE == NS_FINAL);
+    const AbortCtl ab{&ctl->abort_flag, PAIR ? mapa_shared(smem_u32(&ctl->abort_flag), rank ^ 1u) : 0u};
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < NST; ++s) {
-            mbar_init(&full[s], 1);   // leader: its own arrive.expect_tx + both CTAs' bytes
-            mbar_init(&empty[s], 1);  // both: one multicast commit per use
+            mbar_init(&ctl->full[s], 1);   // leader: its own arrive.expect_tx + both CTAs' bytes
+            mbar_init(&ctl->empty[s], 1);  // both: one multicast commit per use
         }
-        for (int w = 0; w < 2 * EPI_WARPS; ++w) mbar_init(&wbar[w], 1);
         for (int a = 0; a < 2; ++a) {
-            mbar_init(&acc_full[a], 1);                  // both: one multicast commit per tile
-            mbar_init(&acc_empty[a], (PAIR ? 2 : 1) * EPI_WARPS);  // leader: every epilogue warp of the pair
+            mbar_init(&ctl->acc_full[a], 1);                              // both: one multicast commit per tile
+            mbar_init(&ctl->acc_empty[a], (PAIR ? 2 : 1) * EPI_WARPS);  // leader: every epilogue warp of the pair
         }
-        mbar_init(drain, 1);
-        *abort_flag = 0;
+        mbar_init(&ctl->drain, 1);
+        for (int r = 0; r < kRing; ++r) mbar_init(&ctl->tile_full[r], 1);  // the leader's publish
+        ctl->abort_flag = 0;
+        ctl->issued = 0;
+        ctl->consumed = 0;
         fence_barrier_init();
         for (int j = 0; j < L.njobs; ++j) {
             prefetch_tensormap(&L.mA[j]);
@@ -435,10 +553,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     if (warp == 1) {
         if (PAIR) {
-            tmem_alloc_pair(tmem_holder, S::TMEM);
+            tmem_alloc_pair(&ctl->tmem_base, S::TMEM);
             tmem_relinquish_pair();
         } else {
-            tmem_alloc(tmem_holder, S::TMEM);
+            tmem_alloc(&ctl->tmem_base, S::TMEM);
             tmem_relinquish();
         }
     }
@@ -446,19 +564,50 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (PAIR) cluster_sync_all();  // barriers of both CTAs initialised, TMEM allocated in both
     else __syncthreads();
     tc_fence_after();
-    const uint32_t tmem_base = *tmem_holder;
+    const uint32_t tmem_base = ctl->tmem_base;
     griddep_wait();  // the previous kernel's results (and its reads of our outputs) are complete
 
     if (warp == 0) {
         if (lane == 0) {
             // In the applies every pair working at the same time reads all of
-            // the m x m Gram (the A operand), one wave after another: keep it in
-            // L2 ahead of the X strips, which each wave reads once.
+            // the m x m Gram (the A operand): keep it in L2 ahead of the X
+            // strips, which the window of running tiles reads once.
             const uint64_t keep = l2_evict_last_policy();
             int stage = 0;
             uint32_t phase = 0;
+            int issued = 0;
             bool ok = true;
-            for (int t = pair; t < total_tiles && ok; t += npairs) {
+            // The leader publishes each tile index two tiles ahead of its own
+            // loads (the peer's producer, the MMA thread and the epilogue warps
+            // find it waiting at every tile boundary), and takes indices from
+            // the counter one further ahead, so that the atomic's latency hides
+            // behind a whole tile of loads. -1 ends the sequence.
+            auto take_next = [&](int prev) -> int {
+                if (prev < 0) return -1;
+                const unsigned int v = atomicAdd(L.tile_ctr, 1u);
+                return v < (unsigned int)total_tiles ? (int)v : -1;
+            };
+            int cur0 = -1, cur1 = -1, nxt = -1;  // leader: tiles seq, seq + 1 (published), seq + 2 (taken)
+            if (leader) {
+                cur0 = take_next(0);
+                cur1 = take_next(cur0);
+                nxt = take_next(cur1);
+                ring_publish<PAIR>(ctl, 0, cur0);  // the ring is fresh
+                if (cur0 >= 0) ring_publish<PAIR>(ctl, 1, cur1);
+            }
+            for (int seq = 0; ok; ++seq) {
+                int t;
+                if (leader) {
+                    t = cur0;
+                    if (t < 0) break;
+                    if (cur1 >= 0) ring_publish<PAIR>(ctl, seq + 2, nxt);  // tile seq + 2, before loading tile seq
+                    cur0 = cur1;
+                    cur1 = nxt;
+                    nxt = take_next(nxt);
+                } else {
+                    t = ring_take<PAIR>(ctl, seq, rank, ab, L, 0, &ok);
+                }
+                if (t < 0) break;
                 const JobTile jt = decode_job_tile(L, MODE, t);
                 const TileCoord tc = jt.tc;
                 const CUtensorMap* mapA = &L.mA[jt.j];
@@ -470,15 +619,15 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const bool diag = !kApply && tc.ti == tc.tj;
                 const uint32_t stage_tx = diag ? A_BYTES : S::STAGE;
                 for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit, L.status)) {
+                    if (!mbar_wait_ctl(&ctl->empty[stage], phase ^ 1u, ab, limit, L.status)) {
                         ok = false;
                         break;
                     }
                     uint8_t* sa = smem + stage * S::STAGE;
                     uint8_t* sb = sa + A_BYTES;
                     if (PAIR) {
-                        if (leader) mbar_arrive_expect_tx(&full[stage], 2 * stage_tx);
-                        const uint32_t fb = mapa_shared(smem_u32(&full[stage]), 0);
+                        if (leader) mbar_arrive_expect_tx(&ctl->full[stage], 2 * stage_tx);
+                        const uint32_t fb = mapa_shared(smem_u32(&ctl->full[stage]), 0);
                         if (kApply) tma_load_3d_pair_hint(sa, mapA, fb, kb * BK, arow, tc.u, keep);
                         else tma_load_3d_pair(sa, mapA, fb, kb * BK, arow, tc.u);
                         if (!kApply) {
@@ -489,17 +638,21 @@ __global__ void __launch_bounds__(THREADS, 1)
                                 tma_load_3d_pair(sb + q * (64 * BK * 2), mapB, fb, bcol + q * 64, kb * BK, tc.u);
                         }
                     } else {
-                        mbar_arrive_expect_tx(&full[stage], stage_tx);
-                        if (kApply) tma_load_3d_hint(sa, mapA, &full[stage], kb * BK, arow, tc.u, keep);
-                        else tma_load_3d(sa, mapA, &full[stage], kb * BK, arow, tc.u);
+                        mbar_arrive_expect_tx(&ctl->full[stage], stage_tx);
+                        if (kApply) tma_load_3d_hint(sa, mapA, &ctl->full[stage], kb * BK, arow, tc.u, keep);
+                        else tma_load_3d(sa, mapA, &ctl->full[stage], kb * BK, arow, tc.u);
                         if (!kApply) {
-                            if (!diag) tma_load_3d(sb, mapB, &full[stage], kb * BK, bcol, tc.u);  // CN = 128 rows
+                            if (!diag) tma_load_3d(sb, mapB, &ctl->full[stage], kb * BK, bcol, tc.u);  // CN = 128 rows
                         } else {
 #pragma unroll
                             for (int q = 0; q < S::CN / 64; ++q)
-                                tma_load_3d(sb + q * (64 * BK * 2), mapB, &full[stage], bcol + q * 64, kb * BK, tc.u);
+                                tma_load_3d(sb + q * (64 * BK * 2), mapB, &ctl->full[stage], bcol + q * 64, kb * BK,
+                                            tc.u);
                         }
                     }
+                    // what the abort drain needs: this use is armed (leader) and its loads issued
+                    ctl->stage_tx[stage] = stage_tx;
+                    ctl->issued = ++issued;
                     if (++stage == NST) {
                         stage = 0;
                         phase ^= 1u;
@@ -509,7 +662,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             // Tail: wait until the MMAs have released every stage this CTA filled,
             // so that no commit arrives on this CTA's barriers after it exits.
             for (int i = 0; i < NST && ok; ++i) {
-                ok = mbar_wait_bounded(&empty[stage], phase ^ 1u, abort_flag, limit, L.status);
+                ok = mbar_wait_ctl(&ctl->empty[stage], phase ^ 1u, ab, limit, L.status);
                 if (++stage == NST) {
                     stage = 0;
                     phase ^= 1u;
@@ -521,12 +674,14 @@ __global__ void __launch_bounds__(THREADS, 1)
             constexpr uint32_t IDESC = idesc_bf16_f32(S::TM, S::TN, kApply ? 1 : 0);
             int stage = 0;
             uint32_t phase = 0;
-            int lt = 0;
+            int consumed = 0;
             bool ok = true;
-            for (int t = pair; t < total_tiles && ok; t += npairs, ++lt) {
+            for (int lt = 0; ok; ++lt) {
+                const int t = ring_take<PAIR>(ctl, lt, rank, ab, L, 0, &ok);
+                if (t < 0) break;
                 const int acc = lt & 1;
                 const uint32_t use = (uint32_t)(lt >> 1);
-                if (!mbar_wait_bounded(&acc_empty[acc], (use & 1u) ^ 1u, abort_flag, limit, L.status)) {
+                if (!mbar_wait_ctl(&ctl->acc_empty[acc], (use & 1u) ^ 1u, ab, limit, L.status)) {
                     ok = false;
                     break;
                 }
@@ -536,10 +691,11 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int kblocks = L.job[jt.j].kblocks;
                 const bool diag = !kApply && jt.tc.ti == jt.tc.tj;
                 for (int kb = 0; kb < kblocks; ++kb) {
-                    if (!mbar_wait_bounded(&full[stage], phase, abort_flag, limit, L.status)) {
+                    if (!mbar_wait_ctl(&ctl->full[stage], phase, ab, limit, L.status)) {
                         ok = false;
                         break;
                     }
+                    ctl->consumed = ++consumed;
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(smem + stage * S::STAGE);
                     const uint32_t b0 = diag ? a0 : a0 + A_BYTES;
@@ -554,37 +710,31 @@ __global__ void __launch_bounds__(THREADS, 1)
                         if (PAIR) tc_mma_f16_pair(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
                         else tc_mma_f16(d_tmem, adesc, bdesc, IDESC, (kb | kk) != 0 ? 1u : 0u);
                     }
-                    if (PAIR) tc_commit_pair_mc(&empty[stage], 0x3);
-                    else tc_commit(&empty[stage]);
+                    if (PAIR) tc_commit_pair_mc(&ctl->empty[stage], 0x3);
+                    else tc_commit(&ctl->empty[stage]);
                     if (++stage == NST) {
                         stage = 0;
                         phase ^= 1u;
                     }
                 }
                 if (!ok) break;
-                if (PAIR) tc_commit_pair_mc(&acc_full[acc], 0x3);
-                else tc_commit(&acc_full[acc]);
-            }
-            if (!ok) {
-                // let every MMA issued so far finish before TMEM is released
-                if (PAIR) tc_commit_pair(drain);
-                else tc_commit(drain);
-                mbar_wait_bounded(drain, 0, abort_flag, limit, L.status);
+                if (PAIR) tc_commit_pair_mc(&ctl->acc_full[acc], 0x3);
+                else tc_commit(&ctl->acc_full[acc]);
             }
         }
     } else if (MODE == NS_FINAL) {
-        final_epilogue<PAIR>(L, pair, npairs, rank, tmem_base, warp, lane, staging + (warp - 2) * FIN_WARP_BYTES,
-                             acc_full, acc_empty, abort_flag);
+        final_epilogue<PAIR>(L, ctl, rank, tmem_base, warp, lane, staging + (warp - 2) * FIN_WARP_BYTES, ab);
     } else {
         const int quad = warp & 3;              // TMEM lanes [32*quad, 32*quad + 32)
         const int half = (warp - 2) / 4;        // which half of the 256 columns
         uint8_t* stg = staging + (warp - 2) * 2 * STG_BLOCK;
         // outputs are read only by the next launch, long after L2 has turned over
         const uint64_t stream_out = l2_evict_first_policy();
-        const uint32_t acc_empty_leader0 = PAIR ? mapa_shared(smem_u32(&acc_empty[0]), 0) : 0u;
-        const uint32_t acc_empty_leader1 = PAIR ? mapa_shared(smem_u32(&acc_empty[1]), 0) : 0u;
-        int lt = 0;
-        for (int t = pair; t < total_tiles; t += npairs, ++lt) {
+        const uint32_t acc_empty_leader0 = PAIR ? mapa_shared(smem_u32(&ctl->acc_empty[0]), 0) : 0u;
+        const uint32_t acc_empty_leader1 = PAIR ? mapa_shared(smem_u32(&ctl->acc_empty[1]), 0) : 0u;
+        // each tile is taken before the previous accumulator is released (see kRing)
+        int t = epi_take<PAIR>(ctl, 0, rank, ab, L, lane);
+        for (int lt = 0; t >= 0; ++lt) {  // -1: no more tiles, or an abort
             const JobTile jt = decode_job_tile(L, MODE, t);
             const NsJob& p = L.job[jt.j];
             const CUtensorMap* mapOut = &L.mO[jt.j];
@@ -595,7 +745,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const int row = row_lo + lane;
             int ok = 1;
             if (lane == 0)
-                ok = mbar_wait_bounded(&acc_full[acc], use & 1u, abort_flag, limit, L.status, kEpiSleepNs) ? 1 : 0;
+                ok = mbar_wait_ctl(&ctl->acc_full[acc], use & 1u, ab, limit, L.status, kEpiSleepNs) ? 1 : 0;
             ok = __shfl_sync(0xffffffffu, ok, 0);
             if (!ok) break;
             tc_fence_after();
@@ -638,26 +788,32 @@ __global__ void __launch_bounds__(THREADS, 1)
                     bulk_commit_group();
                 }
             }
+            t = epi_take<PAIR>(ctl, lt + 1, rank, ab, L, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
                 if (PAIR) mbar_arrive_cluster(acc ? acc_empty_leader1 : acc_empty_leader0);
-                else mbar_arrive(&acc_empty[acc]);
+                else mbar_arrive(&ctl->acc_empty[acc]);
             }
         }
         if (lane == 0) bulk_wait_group0();  // every bulk store of this warp has completed
     }
 
+    // Every role of this CTA has stopped issuing; wait for the peer's too. The
+    // normal path is drained by construction (the producers waited for the
+    // MMAs to release their stages, the epilogues for every accumulator).
+    // After an abort, which reached both CTAs before this barrier, the leader
+    // drains the pair's MMAs and bulk loads before either CTA releases TMEM
+    // or exits.
+    __syncwarp();
     __syncthreads();
-    if (threadIdx.x == 0 && *abort_flag) {
-        // give this CTA's own bulk copies that may still be in flight time to land
-        const uint64_t t0 = globaltimer();
-        while (globaltimer() - t0 < 200000ull) {
-        }
-    }
+    tc_fence_before();
+    if (PAIR) cluster_sync_all();
+    if (ctl->abort_flag && leader && warp == 1 && lane == 0) abort_drain<NST, PAIR>(ctl, ab, L);
+    __syncwarp();
+    __syncthreads();
     tc_fence_before();
     if (PAIR) cluster_sync_all();  // neither CTA leaves while the pair may still touch its memory
-    else __syncthreads();
     if (warp == 1) {
         tc_fence_after();
         if (PAIR) tmem_dealloc_pair(tmem_base, S::TMEM);
@@ -669,15 +825,17 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
+// The driver's tensor-map encoder, looked up once (thread-safe static
+// initialisation); NULL when the driver does not provide it.
 EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
+    static const EncodeTiledFn fn = []() -> EncodeTiledFn {
         void* ptr = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(ptr);
-    }
+            return reinterpret_cast<EncodeTiledFn>(ptr);
+        return nullptr;
+    }();
     return fn;
 }
 
@@ -700,17 +858,18 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
 // Once per device and kernel instance: allow its dynamic shared memory and
 // find how many pairs (or CTAs) can be resident at once. Not legal inside a
 // stream capture the first time; ns_tc_setup runs it for every instance.
+// Concurrent first calls from several host threads are serialised per
+// instance, and a launch never sees a device whose attribute is not yet set.
 template <int MODE, bool PAIR>
 cudaError_t setup_mode(int num_sms, int* max_units_out) {
     using S = Shape<MODE, PAIR>;
-    static unsigned long long attr_set = 0;  // one bit per device
-    static int max_units[64] = {0};          // resident pairs (or CTAs) per device
+    static PerDevice<int> cache;  // resident pairs (or CTAs) per device, once its attributes are set
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-    if (!(attr_set & (1ull << dev))) {
-        e = cudaFuncSetAttribute(ns_tc_kernel<MODE, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM);
+    return cache.get(dev, max_units_out, [num_sms](int* max_units) -> cudaError_t {
+        cudaError_t e =
+            cudaFuncSetAttribute(ns_tc_kernel<MODE, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM);
         if (e != cudaSuccess) return e;
         if (PAIR) {
             cudaLaunchAttribute attr[1];
@@ -728,18 +887,16 @@ cudaError_t setup_mode(int num_sms, int* max_units_out) {
             e = cudaOccupancyMaxActiveClusters(&nclusters, ns_tc_kernel<MODE, PAIR>, &qc);
             if (e != cudaSuccess) return e;
             if (nclusters < 1) return cudaErrorInvalidConfiguration;
-            max_units[dev] = nclusters;
+            *max_units = nclusters;
         } else {
             int per_sm = 0;
             e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ns_tc_kernel<MODE, PAIR>, THREADS, S::SMEM);
             if (e != cudaSuccess) return e;
             if (per_sm < 1) return cudaErrorInvalidConfiguration;
-            max_units[dev] = per_sm * num_sms;
+            *max_units = per_sm * num_sms;
         }
-        attr_set |= 1ull << dev;
-    }
-    *max_units_out = max_units[dev];
-    return cudaSuccess;
+        return cudaSuccess;
+    });
 }
 
 template <int MODE, bool PAIR>
@@ -803,7 +960,11 @@ cudaError_t launch_mode(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_
     L.total_tiles = tile0;
     L.wait_limit_ns = jobs[0].p->wait_limit_ns;
     L.status = jobs[0].p->status;
+    // the launch's own counter: the first of the pair for the CTA-pair kernel,
+    // the second for the single-CTA kernel of the same grouped launch
+    L.tile_ctr = jobs[0].p->tile_ctr ? jobs[0].p->tile_ctr + (PAIR ? 0 : 1) : nullptr;
     if (tile0 <= 0) return cudaSuccess;
+    if (!L.tile_ctr) return cudaErrorInvalidValue;
     int max_units = 0;
     cudaError_t e = setup_mode<MODE, PAIR>(num_sms, &max_units);
     if (e != cudaSuccess) return e;

@@ -224,7 +224,12 @@ class DistMuonAdamW:
         shaped and typed like ``flat_grad`` (``host_views`` gives its per-tensor
         views). Each bucket's gradients are copied on a side stream and that
         bucket's reduce-scatter starts as soon as its copy lands, so the copies
-        overlap the reductions and the updates of the buckets before it."""
+        overlap the reductions and the updates of the buckets before it.
+
+        The call returns before the copies have read ``host_flat``: do not
+        write to it until ``host_copies_done`` (a CUDA event recorded after the
+        last copy) has completed, e.g. ``opt.host_copies_done.synchronize()``,
+        or the step may read the new values for some buckets."""
         if host_flat.shape != self.flat_grad.shape or host_flat.dtype != self.flat_grad.dtype:
             raise ValueError("host_flat must match flat_grad in shape and dtype")
         self._run(host_flat)
@@ -264,6 +269,10 @@ class DistMuonAdamW:
                     bv.grad_bucket.copy_(host_flat[bv.start:bv.start + n], non_blocking=True)
                 reduces.append(dist.reduce_scatter_tensor(bv.grad_shard, bv.grad_bucket, op=dist.ReduceOp.AVG,
                                                           group=self.pg, async_op=True))
+        if side is not None and host_flat is not None:
+            # every copy from host_flat is queued on `side` before this event
+            self.host_copies_done = torch.cuda.Event()
+            self.host_copies_done.record(side)
         gathers = []
         for b, bv in enumerate(self.buckets):
             if reduces[b] is not None:

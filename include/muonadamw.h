@@ -371,7 +371,11 @@ void ma_plan_destroy(ma_plan_t* plan);
 #define MA_PROF_NS_APPLY 4      /* Newton-Schulz X' = aX + BX (not the last)   */
 #define MA_PROF_NS_GRAMSQ 5     /* Newton-Schulz A^2 (c != 0 only)             */
 #define MA_PROF_NS_FINAL 6      /* last apply, fused with decay and W update   */
-#define MA_PROF_CLASSES 7
+#define MA_PROF_MOMENTUM_SIDE 7 /* momentum pass run under the Newton-Schulz   */
+                                /* chain of the batch before it (side stream)  */
+#define MA_PROF_NS_CLUSTER 8    /* whole chain of short units (m <= 128) in    */
+                                /* one cluster-resident launch                 */
+#define MA_PROF_CLASSES 9
 
 /* When on != 0, every kernel the library launches on this thread's current
  * device is bracketed by two CUDA events recorded on its launch stream. Off by

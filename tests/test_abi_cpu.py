@@ -35,6 +35,25 @@ def test_header_symbols_exported():
         assert hasattr(L, n), f"{n} declared in muonadamw.h but not exported"
 
 
+def test_binding_constants_match_header_macros():
+    # the binding's copies of the header's size constants (the allocation-free
+    # entry point's scratch size among them) must be the header's values
+    src = open(HEADER).read()
+
+    def macro(name):
+        m = re.search(r"#define\s+" + name + r"\s+(.+)", src)
+        assert m, name
+        expr = re.sub(r"\((?:size_t|int64_t|int)\)", "", m.group(1).split("/*")[0])
+        return int(eval(expr, {"__builtins__": {}}))  # plain integer arithmetic of the macro
+
+    assert ma.STATIC_SCRATCH_BYTES == macro("MA_STATIC_SCRATCH_BYTES")
+    assert ma.SHARD_ALIGN == macro("MA_SHARD_ALIGN")
+    assert ma.MAX_NS_STEPS == macro("MA_MAX_NS_STEPS")
+    assert ma.MAX_GROUPS == macro("MA_MAX_GROUPS")
+    assert ma.MAX_BATCH == macro("MA_MAX_BATCH")
+    assert len(ma.PROF_CLASSES) == macro("MA_PROF_CLASSES")
+
+
 def test_struct_layouts_match():
     L = ma.lib()
     for which, cls in enumerate((ma.Tensor, ma.Group, ma.MuonHParams, ma.AdamWHParams)):
@@ -196,11 +215,21 @@ def test_plan_sizing_on_host():
     assert (sub(128, 4096, 4096), sub(64, 4096, 11008), sub(32, 11008, 4096)) == (32, 16, 16)
     expect = max(ma.muon_workspace_bytes(32, 4096, 4096, hp), ma.muon_workspace_bytes(16, 4096, 11008, hp),
                  ma.muon_workspace_bytes(16, 11008, 4096, hp))
-    assert ws == expect
+    # ten Muon sub-batches: two halves, so that each sub-batch's momentum pass
+    # can run under the chain of the one before it
+    assert ws == 2 * ((expect + 255) // 256 * 256)
     ma.ma_plan_destroy(plan)
-    # a cap splits buckets into sub-batches
+    # a cap splits buckets into sub-batches, and the two halves fit in it
     plan, ws2 = ma.ma_plan_create(descs, _groups_for(wl), ws_cap=4 << 30)
     assert 0 < ws2 <= 4 << 30
+    ma.ma_plan_destroy(plan)
+    plan, ws3 = ma.ma_plan_create(descs, _groups_for(wl), ws_cap=2 * ((expect + 255) // 256 * 256))
+    assert ws3 == 2 * ((expect + 255) // 256 * 256)
+    ma.ma_plan_destroy(plan)
+    # a cap below two halves of the largest single matrix: one workspace
+    one = ma.muon_workspace_bytes(1, 4096, 11008, hp)
+    plan, ws4 = ma.ma_plan_create(descs, _groups_for(wl), ws_cap=one + 4096)
+    assert ws4 <= one + 4096
     ma.ma_plan_destroy(plan)
     with pytest.raises(ma.MAError) as e:
         ma.ma_plan_create(descs, _groups_for(wl), ws_cap=1 << 20)
@@ -222,7 +251,8 @@ def test_plan_describe():
     plan, ws = ma.ma_plan_create(_fake_descs(wl), _groups_for(wl))
     text = ma.ma_plan_describe(plan, _groups_for(wl))
     ma.ma_plan_destroy(plan)
-    assert text.startswith(f"workspace {ws} bytes; AdamW: 67 tensors, ")
+    assert text.startswith(f"workspace {ws} bytes in two halves of {ws // 2} (momentum passes under the previous "
+                           f"chain); AdamW: 67 tensors, ")
     assert "4096 x 4096, 128 matrices (bf16 grads), heads 1, sub-batches of 32" in text
     assert "4096 x 11008, 64 matrices (bf16 grads), heads 1, sub-batches of 16" in text
     assert "11008 x 4096, 32 matrices (bf16 grads), heads 1, sub-batches of 16" in text

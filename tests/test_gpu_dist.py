@@ -122,6 +122,12 @@ def test_one_rank_step_from_host_matches_step(one_rank_group):
                 h.copy_(g.cpu())
             oa.step()
             ob.step_from_host(host_flat)
+            # the caller refills its pinned buffer as soon as the copies have
+            # read it, while the step may still run (every tensor's range; the
+            # alignment gaps between tensors keep their zeros)
+            ob.host_copies_done.synchronize()
+            for h in hv:
+                h.fill_(1e3)
             torch.cuda.synchronize()
             assert ma.ma_device_status() == ma.MA_OK
             assert torch.equal(oa.flat_grad, ob.flat_grad)

@@ -175,6 +175,28 @@ def test_resume_from_copied_state_is_bit_identical():
         assert torch.equal(s0, t0) and (s1 is None or torch.equal(s1, t1))
 
 
+@pytest.mark.parametrize("shape", [(4096, 11008), (11008, 4096)])
+def test_fp32_mode_7b_mlp_shapes_exact_update(shape):
+    """fp32 mode on the 7B-shaped set's MLP matrices (the longest K loops of the
+    fp32 kernels; 11008 x 4096 takes the transpose path), at the 1e-5 bound
+    with no allowance: from W = 0 the step writes W_new = -lr * scale * X_N,
+    whose only rounding beyond the update itself is one fp32 product, so the
+    fp32 storage of the weights puts no floor under the measured error."""
+    r = np.random.default_rng(21)
+    W0 = np.zeros(shape, np.float32)
+    g = (r.standard_normal(shape) * 1e-3).astype(np.float32)
+    hp = ma.muon_hparams(precision=1)
+    Wd, Md = [dev_f32(W0)], [torch.zeros(shape, device="cuda")]
+    ws = torch.empty(ma.muon_workspace_bytes(1, *shape, hp), dtype=torch.uint8, device="cuda")
+    ma.muon_step_batched(Wd, [dev_f32(g)], Md, hp, ws)
+    torch.cuda.synchronize()
+    assert ma.ma_device_status() == ma.MA_OK
+    rw, _ = oracle.muon_update(W0, g, np.zeros(shape), f32(0.02), f32(0.95), f32(0.01), eps=f32(1e-7))
+    d_gpu, d_ref = host(Wd[0]), rw  # W_old = 0: the update is W_new itself
+    err = np.linalg.norm(d_gpu - d_ref) / np.linalg.norm(d_ref)
+    assert err <= TOL_F32, f"fp32-mode update relative error {err:.3e} > {TOL_F32}"
+
+
 @pytest.mark.parametrize("shape", [(1024, 2048), (2048, 1024)])
 def test_fp32_mode_larger(shape):
     r = np.random.default_rng(20)

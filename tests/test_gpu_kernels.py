@@ -273,3 +273,35 @@ def test_bounded_wait_times_out_and_context_survives():
     x = torch.ones(1024, device="cuda")
     assert float(x.sum()) == 1024.0
     _muon_run((128, 256), 1, True, 0, (oracle.CUBIC,), precision=0, gdt="bf16", batch=1, steps=1)
+
+
+@pytest.mark.parametrize("heads", [1, 32])
+def test_newton_schulz_wait_timeout_winds_down_and_context_survives(heads):
+    """A wait limit far below one tile's main loop makes the bounded waits
+    inside real Newton-Schulz launches run out: 4096 x 4096 matrices on the
+    CTA-pair kernel (heads = 1) and their 128-row head slices on the
+    single-CTA kernel (heads = 32). Every launch of the step must record
+    MA_ERR_TIMEOUT, wind down (the leader drains the issued MMAs and the bulk
+    loads in flight, then both CTAs release TMEM) and return; with the default
+    limit back, ordinary steps on the same context, on both kernels, match the
+    oracle."""
+    shape, batch = (4096, 4096), 2
+    hp = ma.muon_hparams(heads=heads)
+    W = [torch.zeros(shape, device="cuda") for _ in range(batch)]
+    M = [torch.zeros(shape, device="cuda") for _ in range(batch)]
+    g = torch.Generator(device="cuda").manual_seed(3)
+    G = [(torch.randn(shape, device="cuda", generator=g) * 1e-3).bfloat16() for _ in range(batch)]
+    ws = torch.empty(ma.muon_workspace_bytes(batch, *shape, hp), dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    ma.ma_device_status(reset=True)
+    try:
+        ma.ma_set_wait_limit_ns(2_000)  # 2 us: a 256 x 256 tile's main loop takes tens of microseconds
+        ma.muon_step_batched(W, G, M, hp, ws)
+        torch.cuda.synchronize()
+    finally:
+        ma.ma_set_wait_limit_ns(2_000_000_000)  # the library's default
+    assert ma.ma_device_status(reset=True) == ma.MA_ERR_TIMEOUT
+    assert ma.ma_device_status(reset=True) == ma.MA_OK
+    # the context, the kernels' TMEM and the workspace are usable again
+    _muon_run((512, 1024), 1, True, 0, (oracle.CUBIC,), precision=0, gdt="bf16", batch=2, steps=1)
+    _muon_run((2048, 128), 4, True, 0, (oracle.CUBIC,), precision=0, gdt="bf16", batch=1, steps=1)

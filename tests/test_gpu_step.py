@@ -2,8 +2,9 @@
 
 * tiny: every element of every tensor, twelve steps (eager, fp32 mode, CUDA graph).
 * d20 and the 7B-shaped set at full size, in the same launch configuration
-  bench.py times. The oracle recomputes sampled matrices in full (one of each
-  bucket) and sampled elements of the AdamW tensors and of every momentum
+  bench.py times. The oracle recomputes sampled matrices in full (one or two
+  of each bucket; on the 7B set the first and the last, which lie in different
+  sub-batches) and sampled elements of the AdamW tensors and of every momentum
   buffer, two steps from zero state.
 """
 import numpy as np
@@ -89,12 +90,21 @@ def test_tiny_twelve_steps_every_element(precision, graph):
 
 
 def _full_size_check(name, n_muon_samples=1, adamw_samples=200_000, seed=0):
+    """n_muon_samples matrices of every bucket are recomputed in full: the
+    bucket's first matrix and, for two or more, its last one (which the plan
+    puts in the bucket's last sub-batch), then evenly spaced members."""
     wl = synth.WORKLOADS[name]()
     params = sdev.weights(wl)
     opt = build_optimizer(wl, params)
     kinds = oracle.partition([(t.shape, t.role) for t in wl.tensors])
     buckets = oracle.muon_buckets([(t.shape, t.role) for t in wl.tensors], [t.group for t in wl.tensors])
-    sample_mats = [idx for b in buckets for idx in b[3][:n_muon_samples]]
+
+    def pick(members):
+        k = min(n_muon_samples, len(members))
+        pos = sorted({round(j * (len(members) - 1) / max(1, k - 1)) for j in range(k)}) if k > 1 else [0]
+        return [members[p] for p in pos]
+
+    sample_mats = [idx for b in buckets for idx in pick(b[3])]
     r = np.random.default_rng(seed)
     grads = None
     for step in (1, 2):
@@ -147,7 +157,10 @@ def test_d20_full_size_sampled():
 
 @pytest.mark.slow
 def test_7b_full_size_sampled():
-    _full_size_check("7b", n_muon_samples=1, adamw_samples=100_000)
+    # two matrices of each of the three buckets: the first and the last (which
+    # lies in a later sub-batch: 32 matrices per sub-batch of the 4096^2 bucket,
+    # 16 of the 4096x11008 and 11008x4096 buckets)
+    _full_size_check("7b", n_muon_samples=2, adamw_samples=100_000)
 
 
 @pytest.mark.slow
@@ -178,6 +191,11 @@ def test_step_from_host_equals_resident_step(name):
         host_g = [x.cpu().pin_memory() for x in g]
         opt_a.step(dev_a)
         opt_b.step_from_host(host_g, dev_b)
+        # once the copies have read the host buffers, the caller may reuse them
+        # while the step still runs
+        opt_b.host_copies_done.synchronize()
+        for h in host_g:
+            h.fill_(float("nan"))
         torch.cuda.synchronize()
         assert ma.ma_device_status() == ma.MA_OK
         for x, y in zip(pa, pb):
