@@ -148,7 +148,10 @@ struct MuonGeom {
     int64_t parts;
     int esz;
     bool quintic;
-    size_t off_x0, off_x1, off_g, off_g2, off_part, off_scale, off_ctr, total;
+    bool gspace;  // the chain runs in Gram space (gram_space below)
+    // standard chain: X0, X1 (ping-pong), Gram, Gram2 (c != 0); Gram-space
+    // chain: X0, and four m x m buffers A0 (off_g), A1 (off_g2), Q0, Q1
+    size_t off_x0, off_x1, off_g, off_g2, off_q0, off_q1, off_part, off_scale, total;
 };
 
 bool any_c(const ma_muon_hparams_t& hp) {
@@ -173,6 +176,22 @@ int check_muon_hp(const ma_muon_hparams_t* hp) {
     return MA_OK;
 }
 
+// Whether a unit's Newton-Schulz chain runs in Gram space. The iteration
+// X_{k+1} = P_k X_k, P_k = a_k I + b_k A_k, A_k = X_k X_k^T, gives
+// X_N = Q_N X_0 with Q_N = P_{N-1} ... P_0, and A_{k+1} = P_k A_k P_k: every
+// factor is a polynomial in A_0, so all of them are symmetric and commute.
+// The chain then forms A_0 (one Gram, m(m+1)n flops), updates Q, A and
+// Y = A P with symmetric m x m products (m(m+1)m flops each, 3N - 3 of them)
+// and applies Q_N to X_0 once (2m^2 n): for N = 5 and n = 2.69 m (the 7B
+// set's MLP matrices, or 128 x 4096 head slices) a fraction of the flops of
+// N Grams and N applies. Taken for bf16 operands without an A^2 term when
+// n >= 1.25 m, m >= 128 and m n >= 2^19 (on smaller units the 3N + 1
+// launches cost more than the flops saved); exact in real arithmetic, and
+// within the same bf16 error as the direct iteration.
+bool gram_space(int64_t m, int64_t n, const ma_muon_hparams_t& hp) {
+    return hp.precision == 0 && !any_c(hp) && m >= 128 && 4 * n >= 5 * m && m * n >= (int64_t(1) << 19);
+}
+
 int muon_geom(int batch, int64_t R, int64_t C, const ma_muon_hparams_t& hp, MuonGeom* g) {
     if (batch < 0 || R < 0 || C < 0) return MA_ERR_SHAPE;
     if (hp.heads < 1 || (R > 0 && R % hp.heads != 0)) return MA_ERR_SHAPE;
@@ -189,23 +208,35 @@ int muon_geom(int batch, int64_t R, int64_t C, const ma_muon_hparams_t& hp, Muon
     g->parts = (g->Rh > 0 && C > 0) ? prep_parts_per_unit(g->Rh, C, g->transposed) : 0;
     g->esz = hp.precision ? 4 : 2;
     g->quintic = any_c(hp);
+    g->gspace = gram_space(g->m, g->n, hp);
     size_t off = 0;
     const size_t xbytes = (size_t)g->units * g->m * g->ldx * g->esz;
     const size_t gbytes = (size_t)g->units * g->m * g->ldg * g->esz;
     g->off_x0 = off;
     off = align_up(off + xbytes, kAlign);
-    g->off_x1 = off;
-    if (hp.ns_steps >= 2) off = align_up(off + xbytes, kAlign);
-    g->off_g = off;
-    off = align_up(off + gbytes, kAlign);
-    g->off_g2 = off;
-    if (g->quintic) off = align_up(off + gbytes, kAlign);
+    if (!g->gspace) {
+        g->off_x1 = off;
+        if (hp.ns_steps >= 2) off = align_up(off + xbytes, kAlign);
+        g->off_g = off;
+        off = align_up(off + gbytes, kAlign);
+        g->off_g2 = off;
+        if (g->quintic) off = align_up(off + gbytes, kAlign);
+        g->off_q0 = g->off_q1 = off;  // unused
+    } else {
+        g->off_x1 = g->off_x0;  // unused
+        g->off_g = off;
+        off = align_up(off + gbytes, kAlign);
+        g->off_g2 = off;
+        off = align_up(off + gbytes, kAlign);
+        g->off_q0 = off;
+        off = align_up(off + gbytes, kAlign);
+        g->off_q1 = off;
+        off = align_up(off + gbytes, kAlign);
+    }
     g->off_part = off;
     off = align_up(off + (size_t)g->units * g->parts * sizeof(double), kAlign);
     g->off_scale = off;
     off = align_up(off + (size_t)g->units * sizeof(float), kAlign);
-    g->off_ctr = off;  // tile counters of the Newton-Schulz launches
-    off = align_up(off + kNsCounterBytes, kAlign);
     g->total = (batch == 0 || R == 0 || C == 0) ? 0 : off;
     return MA_OK;
 }
@@ -297,8 +328,7 @@ int muon_prep(const MuonJob& j, cudaStream_t s, int max_blocks, bool side, int* 
     prof_end(pr, s, 0.0, elems * ((j.gdt == MA_BF16 ? 2 : 4) + 8 + (hp.precision ? 4 : 2)));
     if (st) return st;
     pr = prof_begin(MA_PROF_FINALIZE, s);
-    st = cuda_status(launch_norm_finalize(part, g.parts, (int)g.units, hp.eps, scale,
-                                          reinterpret_cast<unsigned int*>(j.ws + g.off_ctr), kNsCounters, s));
+    st = cuda_status(launch_norm_finalize(part, g.parts, (int)g.units, hp.eps, scale, s));
     prof_end(pr, s, 0.0, (double)g.units * g.parts * 8.0 + g.units * 4.0);
     if (st) return st;
     *launches += 2;
@@ -311,7 +341,7 @@ int muon_prep(const MuonJob& j, cudaStream_t s, int max_blocks, bool side, int* 
 double ns_bytes(int mode, int64_t units, int64_t m, int64_t n, int esz) {
     const double u = (double)units, M = (double)m, N = (double)n, e = (double)esz;
     if (mode == NS_GRAM) return u * e * (M * N + M * M);
-    if (mode == NS_GRAMSQ) return u * e * 2.0 * M * M;
+    if (mode == NS_GRAMSQ) return u * e * 3.0 * M * M;  // A and Z read, the product written
     if (mode == NS_APPLY) return u * e * (M * M + 2.0 * M * N);
     return u * (e * (M * M + M * N) + 8.0 * M * N);
 }
@@ -321,11 +351,6 @@ double ns_bytes(int mode, int64_t units, int64_t m, int64_t n, int esz) {
 // launch over every job's tiles on the tensor-core path; per job in fp32 mode.
 // A tile's arithmetic does not depend on the launch it is in, so grouping
 // gives the same bits as running the jobs one by one.
-// Grid of the flat momentum kernel on the caller's stream: six blocks per SM
-// (as many as its registers let reside), each walking many chunks, so that
-// the pass is not bound by the rate at which blocks start.
-constexpr int kPrepBlocksPerSm = 6;
-
 // The momentum passes (and norm finalizes) of a set of jobs. max_blocks > 0
 // bounds the flat momentum kernel's grid (see launch_muon_prep).
 int prep_jobs(const MuonJob* jobs, int njobs, cudaStream_t s, int max_blocks, int* launches, bool side = false) {
@@ -335,66 +360,143 @@ int prep_jobs(const MuonJob* jobs, int njobs, cudaStream_t s, int max_blocks, in
     return MA_OK;
 }
 
-// Whether a job's chain runs as one cluster-resident launch (ns_cluster.cu):
-// bf16 operands, no A^2 term, short unrolled units (m <= 128, rows <= columns,
-// n <= 4096).
-// Off until the kernel has passed its GPU tests.
-constexpr bool kClusterChain = false;
-
-bool cluster_job(const MuonJob& j) {
-    return kClusterChain && j.g.total > 0 && j.hp->precision == 0 && !j.g.quintic &&
-           ns_cluster_eligible((int)j.g.m, (int)j.g.n, j.g.transposed);
-}
-
-// The whole chain of one job in one cluster launch.
-int chain_cluster(const MuonJob& J, cudaStream_t s, int* launches) {
+// Newton-Schulz parameters of a job that do not change along its chain:
+// geometry, the normalisation scales, the final decay and update.
+NsParams base_params(const MuonJob& J) {
     const MuonGeom& g = J.g;
     const ma_muon_hparams_t& hp = *J.hp;
-    NsClusterIn in;
-    std::memset(&in, 0, sizeof(in));
-    in.x = J.ws + g.off_x0;
-    in.ldx = g.ldx;
-    in.x_unit = g.m * g.ldx;
-    in.units = (int)g.units;
-    in.m = (int)g.m;
-    in.n = (int)g.n;
-    in.steps = hp.ns_steps;
-    for (int k = 0; k < hp.ns_steps; ++k) {
-        const float* cf = hp.coeffs[hp.n_coeffs == 1 ? 0 : k];
-        in.coef[k][0] = cf[0];
-        in.coef[k][1] = cf[1];
-    }
-    in.scale = reinterpret_cast<const float*>(J.ws + g.off_scale);
-    in.heads = g.heads;
-    in.Rh = g.Rh;
-    in.C = g.C;
-    in.decay = 1.f - hp.lr * hp.weight_decay;
-    in.lr_s = hp.lr * shape_scale(g.Rh, g.C, hp.scale_mode);
-    in.lr_wd = hp.lr * hp.weight_decay;
-    in.cautious = hp.cautious ? 1 : 0;
-    in.wait_limit_ns = host_wait_limit_ns();
-    in.status = device_status_ptr();
-    in.W = J.W;
-    const int pr = prof_begin(MA_PROF_NS_CLUSTER, s);
-    const cudaError_t e = launch_ns_cluster(in, s);
-    const double u = (double)g.units, m = (double)g.m, n = (double)g.n;
-    prof_end(pr, s, (double)hp.ns_steps * u * (m * (m + 1.0) * n + 2.0 * m * m * n), u * m * n * (2.0 + 8.0));
-    ++*launches;
-    return cuda_status(e);
+    NsParams q;
+    std::memset(&q, 0, sizeof(q));
+    q.units = (int)g.units;
+    q.m = (int)g.m;
+    q.n = (int)g.n;
+    q.ldx = g.ldx;
+    q.ldg = g.ldg;
+    q.x_unit = g.m * g.ldx;
+    q.g_unit = g.m * g.ldg;
+    q.scale = reinterpret_cast<float*>(J.ws + g.off_scale);
+    q.transposed = g.transposed;
+    q.heads = g.heads;
+    q.Rh = g.Rh;
+    q.C = g.C;
+    q.decay = 1.f - hp.lr * hp.weight_decay;
+    q.lr_s = hp.lr * shape_scale(g.Rh, g.C, hp.scale_mode);
+    q.lr_wd = hp.lr * hp.weight_decay;
+    q.cautious = hp.cautious ? 1 : 0;
+    q.wait_limit_ns = host_wait_limit_ns();
+    q.status = device_status_ptr();
+    for (int b = 0; b < J.batch; ++b) q.W[b] = J.W[b];
+    return q;
 }
 
-// The Newton-Schulz chain of a set of jobs whose momentum passes are done.
+// The Gram-space chain (gram_space) of a set of jobs, the launches shared:
+//   A_0 = s^2 X_0 X_0^T                       (Gram, into A)
+//   Q_1 = a_0 I + b_0 A_0                     (elementwise)
+//   per iteration k: Q_{k+1} = a_k Q_k + b_k A_k Q_k   (k >= 1)
+//                    Y = a_k A_k + b_k A_k A_k, A_{k+1} = a_k Y + b_k A_k Y   (k < N - 1)
+//   W <- W (1 - lr wd) - lr scale (s Q_N X_0)  (final apply)
+// Each m x m product is symmetric (all factors are polynomials in A_0): the
+// symmetric-product launches compute its upper tiles and mirror them. Y goes
+// to the Q buffer that the Q update has just freed, so four m x m buffers do.
+int chain_gspace(const std::vector<const MuonJob*>& jobs, cudaStream_t s, int sms, int* launches) {
+    const int nj = (int)jobs.size();
+    if (nj == 0) return MA_OK;
+    if (nj > ns_tc_max_jobs()) return MA_ERR_UNSUPPORTED;
+    const int steps = jobs[0]->hp->ns_steps;  // the same for every job of the set
+    std::vector<NsParams> p(nj);
+    std::vector<void*> X0(nj), Acur(nj), Anext(nj), Qcur(nj), Qfree(nj);
+    for (int i = 0; i < nj; ++i) {
+        const MuonJob& J = *jobs[i];
+        p[i] = base_params(J);
+        X0[i] = J.ws + J.g.off_x0;
+        Acur[i] = J.ws + J.g.off_g;
+        Anext[i] = J.ws + J.g.off_g2;
+        Qcur[i] = J.ws + J.g.off_q0;
+        Qfree[i] = J.ws + J.g.off_q1;
+    }
+    std::vector<NsJobIn> in(nj);
+    // one launch over every job; xb: the X operand (Gram and final apply), gb: the m x m operand
+    auto launch = [&](int mode, const std::vector<void*>& xb, const std::vector<void*>& gb) -> int {
+        const int pr = prof_begin(ns_prof_class(mode), s);
+        double flops = 0.0, bytes = 0.0;
+        for (int i = 0; i < nj; ++i) {
+            in[i] = {&p[i], xb[i], gb[i]};
+            const MuonGeom& g = jobs[i]->g;
+            flops += ns_flops(mode, g.units, g.m, g.n);
+            bytes += ns_bytes(mode, g.units, g.m, g.n, g.esz);
+        }
+        const cudaError_t e = launch_ns_tc_group(mode, in.data(), nj, sms, s, launches);
+        prof_end(pr, s, flops, bytes);
+        return cuda_status(e);
+    };
+    auto coef = [&](int i, int k, int which) {
+        const ma_muon_hparams_t& hp = *jobs[i]->hp;
+        return hp.coeffs[hp.n_coeffs == 1 ? 0 : k][which];
+    };
+    int st;
+    // A_0, normalised: the Gram with multiplier 1 (times s^2 on the first iteration)
+    for (int i = 0; i < nj; ++i) {
+        p[i].first = 1;
+        p[i].coef_gram = 1.f;
+        p[i].out = Acur[i];
+    }
+    if ((st = launch(NS_GRAM, X0, Acur))) return st;
+    for (int i = 0; i < nj; ++i) {
+        const MuonGeom& g = jobs[i]->g;
+        const cudaError_t e = launch_ns_q1(Acur[i], Qcur[i], (int)g.m, g.ldg, g.m * g.ldg, (int)g.units,
+                                           coef(i, 0, 0), coef(i, 0, 1), sms, s);
+        if (e != cudaSuccess) return MA_ERR_CUDA;
+        ++*launches;
+    }
+    // a symmetric product out = alpha Z + beta A Z over every job (Z = A when z is null)
+    auto symprod = [&](const std::vector<void*>& A, const std::vector<void*>* Z, const std::vector<void*>& out,
+                       int k) -> int {
+        for (int i = 0; i < nj; ++i) {
+            p[i].first = 0;
+            p[i].xin = A[i];
+            p[i].zin = Z ? (*Z)[i] : nullptr;
+            p[i].out = out[i];
+            p[i].b = coef(i, k, 0);
+            p[i].c = coef(i, k, 1);
+        }
+        return launch(NS_GRAMSQ, X0, A);
+    };
+    for (int k = 0; k < steps; ++k) {
+        if (k >= 1) {
+            if ((st = symprod(Acur, &Qcur, Qfree, k))) return st;  // Q_{k+1}
+            std::swap(Qcur, Qfree);                                  // Qfree: Q_k, no longer needed
+        }
+        if (k + 1 < steps) {
+            if ((st = symprod(Acur, nullptr, Qfree, k))) return st;  // Y = A P, in the free Q buffer
+            if ((st = symprod(Acur, &Qfree, Anext, k))) return st;   // A_{k+1} = P Y
+            std::swap(Acur, Anext);
+        }
+    }
+    // X_N = s Q_N X_0, written into W by the final apply (a = 0: no a X term)
+    for (int i = 0; i < nj; ++i) {
+        p[i].first = 1;
+        p[i].a = 0.f;
+        p[i].b = 1.f;
+        p[i].c = 0.f;
+        p[i].zin = nullptr;
+        p[i].xin = X0[i];
+        p[i].out = nullptr;
+    }
+    return launch(NS_FINAL, X0, Qcur);
+}
+
+// The Newton-Schulz chain of a set of jobs whose momentum passes are done:
+// the Gram-space chain where it pays (gram_space), the direct iteration for
+// the rest.
 int chain_jobs(const MuonJob* jobs_in, int njobs_in, cudaStream_t s, int sms, int* launches) {
-    std::vector<const MuonJob*> jobs;
+    std::vector<const MuonJob*> jobs, gjobs;
     int st;
     for (int j = 0; j < njobs_in; ++j) {
         if (jobs_in[j].g.total == 0) continue;
-        if (cluster_job(jobs_in[j])) {
-            if ((st = chain_cluster(jobs_in[j], s, launches))) return st;
-        } else {
-            jobs.push_back(&jobs_in[j]);
-        }
+        if (jobs_in[j].g.gspace) gjobs.push_back(&jobs_in[j]);
+        else jobs.push_back(&jobs_in[j]);
     }
+    if ((st = chain_gspace(gjobs, s, sms, launches))) return st;
     const int nj = (int)jobs.size();
     if (nj == 0) return MA_OK;
     if (nj > ns_tc_max_jobs()) return MA_ERR_UNSUPPORTED;
@@ -405,28 +507,7 @@ int chain_jobs(const MuonJob* jobs_in, int njobs_in, cudaStream_t s, int sms, in
     for (int i = 0; i < nj; ++i) {
         const MuonJob& J = *jobs[i];
         const MuonGeom& g = J.g;
-        const ma_muon_hparams_t& hp = *J.hp;
-        NsParams& q = p[i];
-        std::memset(&q, 0, sizeof(q));
-        q.units = (int)g.units;
-        q.m = (int)g.m;
-        q.n = (int)g.n;
-        q.ldx = g.ldx;
-        q.ldg = g.ldg;
-        q.x_unit = g.m * g.ldx;
-        q.g_unit = g.m * g.ldg;
-        q.scale = reinterpret_cast<float*>(J.ws + g.off_scale);
-        q.transposed = g.transposed;
-        q.heads = g.heads;
-        q.Rh = g.Rh;
-        q.C = g.C;
-        q.decay = 1.f - hp.lr * hp.weight_decay;
-        q.lr_s = hp.lr * shape_scale(g.Rh, g.C, hp.scale_mode);
-        q.lr_wd = hp.lr * hp.weight_decay;
-        q.cautious = hp.cautious ? 1 : 0;
-        q.wait_limit_ns = host_wait_limit_ns();
-        q.status = device_status_ptr();
-        for (int b = 0; b < J.batch; ++b) q.W[b] = J.W[b];
+        p[i] = base_params(J);
         cur[i] = J.ws + g.off_x0;
         nxt[i] = J.ws + g.off_x1;
         Gb[i] = J.ws + g.off_g;
@@ -434,17 +515,11 @@ int chain_jobs(const MuonJob* jobs_in, int njobs_in, cudaStream_t s, int sms, in
     }
 
     std::vector<NsJobIn> in(nj);
-    // each launch of the chain takes its own two tile counters (the first job's,
-    // zeroed by its norm finalize)
-    unsigned int* ctr = reinterpret_cast<unsigned int*>(jobs[0]->ws + jobs[0]->g.off_ctr);
-    int nlaunch = 0;
     auto launch = [&](int mode, const std::vector<void*>& xb, const std::vector<void*>& gb) -> int {
         const int pr = prof_begin(ns_prof_class(mode), s);
         double flops = 0.0, bytes = 0.0;
         cudaError_t e = cudaSuccess;
-        if (2 * nlaunch + 2 > kNsCounters) return MA_ERR_UNSUPPORTED;
         for (int i = 0; i < nj; ++i) {
-            p[i].tile_ctr = ctr + 2 * nlaunch;
             in[i] = {&p[i], xb[i], gb[i]};
             const MuonGeom& g = jobs[i]->g;
             flops += ns_flops(mode, g.units, g.m, g.n);
@@ -459,7 +534,6 @@ int chain_jobs(const MuonJob* jobs_in, int njobs_in, cudaStream_t s, int sms, in
             e = launch_ns_tc_group(mode, in.data(), nj, sms, s, launches);
         }
         prof_end(pr, s, flops, bytes);
-        ++nlaunch;
         return cuda_status(e);
     };
 
@@ -500,7 +574,7 @@ int chain_jobs(const MuonJob* jobs_in, int njobs_in, cudaStream_t s, int sms, in
 
 int run_muon_jobs(const MuonJob* jobs, int njobs, cudaStream_t s, int sms, int* launches) {
     if (njobs > ns_tc_max_jobs()) return MA_ERR_UNSUPPORTED;
-    const int st = prep_jobs(jobs, njobs, s, kPrepBlocksPerSm * sms, launches);
+    const int st = prep_jobs(jobs, njobs, s, 0, launches);
     return st ? st : chain_jobs(jobs, njobs, s, sms, launches);
 }
 
@@ -685,7 +759,7 @@ struct ma_plan {
         cudaGraphNode_t node;
         cudaKernelNodeParams params;  // func, launch shape; kernelParams replaced on update
         std::vector<uint8_t> arg;     // the kernel's single by-value parameter
-        int final_apply;              // 0: AdamW launch, 1: Newton-Schulz final apply, 2: cluster chain
+        int final_apply;              // 0: AdamW launch, 1: Newton-Schulz final apply
     };
     struct Graph {
         cudaGraph_t graph = nullptr;
@@ -992,8 +1066,7 @@ int run_segments(ma_plan* plan, const ma_group_t* groups, const std::vector<Segm
         NvtxRange range("ma.muon");
         SegJobs& cur = sj[q];
         if (!on_side[q]) {
-            if ((st = prep_jobs(cur.jobs.data(), (int)cur.jobs.size(), s, kPrepBlocksPerSm * sms, launches)))
-                return st;
+            if ((st = prep_jobs(cur.jobs.data(), (int)cur.jobs.size(), s, 0, launches))) return st;
         } else if (cudaStreamWaitEvent(s, ev_prep[q], 0) != cudaSuccess) {
             return MA_ERR_CUDA;
         }
@@ -1336,7 +1409,7 @@ size_t ns_iterate_workspace_bytes(int batch, int64_t m, int64_t n) {
     if (batch < 0 || m < 0 || n < 0) return SIZE_MAX;
     const size_t x = align_up((size_t)batch * m * n * 2, kAlign);
     const size_t gm = align_up((size_t)batch * m * round8(m) * 2, kAlign);
-    return x + 2 * gm + align_up(kNsCounterBytes, kAlign);  // + the launches' tile counters
+    return x + 2 * gm;
 }
 
 int ns_iterate_bf16(int batch, int64_t m, int64_t n, const uint16_t* X_in, uint16_t* X_out, const float* coeffs,
@@ -1361,10 +1434,6 @@ int ns_iterate_bf16(int batch, int64_t m, int64_t n, const uint16_t* X_in, uint1
     void* T = base;
     void* Gb = base + align_up((size_t)batch * m * n * 2, kAlign);
     void* G2 = reinterpret_cast<uint8_t*>(Gb) + align_up((size_t)batch * m * round8(m) * 2, kAlign);
-    unsigned int* ctr =
-        reinterpret_cast<unsigned int*>(reinterpret_cast<uint8_t*>(G2) + align_up((size_t)batch * m * round8(m) * 2, kAlign));
-    if (cudaMemsetAsync(ctr, 0, kNsCounterBytes, s) != cudaSuccess) return MA_ERR_CUDA;
-    int nlaunch = 0;
     NsParams p;
     std::memset(&p, 0, sizeof(p));
     p.units = batch;
@@ -1387,7 +1456,6 @@ int ns_iterate_bf16(int batch, int64_t m, int64_t n, const uint16_t* X_in, uint1
         const bool quint = cf[2] != 0.f;
         p.coef_gram = quint ? 1.f : cf[1];
         auto launch = [&](int mode, const void* xb, const void* gb) -> int {
-            p.tile_ctr = ctr + 2 * nlaunch++;
             const int pr = prof_begin(ns_prof_class(mode), s);
             cudaError_t e = launch_ns_tc(mode, p, xb, gb, sms, s);
             prof_end(pr, s, ns_flops(mode, batch, m, n), 0.0);
@@ -1666,9 +1734,6 @@ int graph_patch(ma_plan* plan, const ma_group_t* groups) {
         if (n.final_apply == 1) {
             const int st = ns_tc_patch_final(n.arg.data(), patch_final_job, &ctx);
             if (st) return st;
-        } else if (n.final_apply == 2) {
-            const int st = ns_cluster_patch(n.arg.data(), patch_final_job, &ctx);
-            if (st) return st;
         } else {
             AdamwLaunch* L = reinterpret_cast<AdamwLaunch*>(n.arg.data());
             for (int k = 0; k < ngroups; ++k) L->grp[k] = gc[k];
@@ -1699,9 +1764,7 @@ int graph_capture(ma_plan* plan, const ma_group_t* groups, void* ws, int sms, in
     }
     // everything that must not happen inside a capture: attribute set-up,
     // driver entry points, the status-word address, the side stream
-    if (ns_tc_setup(sms) != cudaSuccess || prep_setup() != cudaSuccess || ns_cluster_setup() != cudaSuccess ||
-        !device_status_ptr())
-        return MA_ERR_CUDA;
+    if (ns_tc_setup(sms) != cudaSuccess || prep_setup() != cudaSuccess || !device_status_ptr()) return MA_ERR_CUDA;
     if (plan->region) {
         size_t nm = 0;
         for (const Segment& sg : step_segments(plan, groups, 0, 0, false, seg_limit(plan))) nm += sg.adamw ? 0 : 1;
@@ -1751,11 +1814,10 @@ int graph_capture(ma_plan* plan, const ma_group_t* groups, void* ws, int sms, in
         }
         const bool adamw = p.func == adamw_kernel_func();
         const bool fin = ns_tc_is_final(p.func);
-        const bool chain = ns_cluster_is_kernel(p.func);  // a whole chain, final update included
-        if (!adamw && !fin && !chain) continue;
-        const size_t bytes = adamw ? sizeof(AdamwLaunch) : fin ? ns_tc_launch_bytes() : ns_cluster_launch_bytes();
+        if (!adamw && !fin) continue;
+        const size_t bytes = adamw ? sizeof(AdamwLaunch) : ns_tc_launch_bytes();
         const uint8_t* a = reinterpret_cast<const uint8_t*>(p.kernelParams[0]);
-        G.nodes.push_back({node, p, std::vector<uint8_t>(a, a + bytes), fin ? 1 : chain ? 2 : 0});
+        G.nodes.push_back({node, p, std::vector<uint8_t>(a, a + bytes), fin ? 1 : 0});
     }
     G.launches = launches;
     ++G.captures;
@@ -1863,9 +1925,12 @@ int ma_plan_describe(const ma_plan_t* plan, const ma_group_t* groups, char* buf,
     for (size_t bi = 0; bi < plan->buckets.size(); ++bi) {
         const auto& b = plan->buckets[bi];
         const ma_muon_hparams_t& hp = groups[b.group].muon;
+        MuonGeom g;
+        muon_geom(b.sub, b.R, b.C, hp, &g);
         std::snprintf(line, sizeof(line), "bucket %zu: group %d, %lld x %lld, %zu matrices (%s grads), heads %d, "
-                      "sub-batches of %d\n", bi, b.group, (long long)b.R, (long long)b.C, b.members.size(),
-                      plan->t[b.members[0]].grad_dtype == MA_BF16 ? "bf16" : "fp32", hp.heads, b.sub);
+                      "sub-batches of %d, %s\n", bi, b.group, (long long)b.R, (long long)b.C, b.members.size(),
+                      plan->t[b.members[0]].grad_dtype == MA_BF16 ? "bf16" : "fp32", hp.heads, b.sub,
+                      g.gspace ? "Gram-space chain" : "direct chain");
         out += line;
     }
     int si = 0;

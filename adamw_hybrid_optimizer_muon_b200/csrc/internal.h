@@ -90,8 +90,8 @@ const void* adamw_kernel_func();  // the kernel's host-side handle (CUDA-graph n
 
 // ------------------------------------------------------------------ Muon: momentum + norm
 
-constexpr int kPrepChunk = 4096;   // elements per chunk (one partial sum each), flat path
-constexpr int kPrepThreads = 128;  // threads per block, flat path
+constexpr int kPrepChunk = 8192;      // elements per chunk (one partial sum each), flat path
+constexpr int kPrepSideThreads = 128;  // threads per block of the side-stream flat kernel
 constexpr int kPrepTile = 64;      // tile edge, transposing path
 
 struct MuonPrepLaunch {
@@ -111,27 +111,21 @@ struct MuonPrepLaunch {
 // Number of per-block partial sums the momentum pass writes for one unit.
 int64_t prep_parts_per_unit(int64_t Rh, int64_t C, int transposed);
 
-// max_blocks > 0 bounds the flat path's grid (its blocks then walk the chunks
-// grid-stride; a small grid runs beside the Newton-Schulz kernels of another
-// batch); 0: one block per chunk. The transposing path ignores it.
+// max_blocks > 0: the flat path runs its side-stream kernel on at most that
+// many blocks (a small grid that runs beside the Newton-Schulz kernels of
+// another batch, with the same partial sums); 0: one block per chunk. The
+// transposing path ignores it.
 cudaError_t launch_muon_prep(const MuonPrepLaunch& L, int max_blocks, cudaStream_t s);
 // Per-device kernel attributes of the momentum kernels, ahead of a stream capture.
 cudaError_t prep_setup();
 // scale[u] = 1 / (sqrt(sum of the unit's partials) + eps), deterministic order.
-// Also zeroes the nctr tile counters of the Newton-Schulz launches that follow.
 cudaError_t launch_norm_finalize(const double* partials, int64_t parts, int units, float eps, float* scale,
-                                 unsigned int* ctr, int nctr, cudaStream_t s);
+                                 cudaStream_t s);
 
 // ------------------------------------------------------------------ Newton-Schulz
 
 enum NsMode { NS_GRAM = 0, NS_APPLY = 1, NS_FINAL = 2, NS_GRAMSQ = 3 };
 
-// Tile counters of one Newton-Schulz chain (in the workspace): two per launch
-// (the CTA-pair kernel and the single-CTA kernel of a grouped launch), at most
-// three launches per iteration.
-constexpr int kNsCounters = 2 * 3 * MA_MAX_NS_STEPS;
-constexpr size_t kNsCounterBytes = 512;
-static_assert(kNsCounters * sizeof(unsigned int) <= kNsCounterBytes, "tile counters");
 
 struct NsParams {
     int32_t units, m, n;
@@ -141,7 +135,9 @@ struct NsParams {
     float a, b, c;           // this iteration's polynomial coefficients
     float coef_gram;         // GRAM epilogue multiplier (b, or 1 when c != 0)
     const float* scale;      // per-unit 1 / (||u|| + eps); may be NULL when first == 0
-    const void* xin;         // APPLY/FINAL: X of this iteration; GRAMSQ: the Gram input
+    const void* xin;         // APPLY/FINAL: X of this iteration; GRAMSQ: the Gram input A
+    const void* zin;         // GRAMSQ: second operand Z, symmetric and commuting with A (NULL: A itself);
+                             // the launch computes b*Z + c*(A Z) on the upper tiles and mirrors them
     void* out;               // GRAM/GRAMSQ: Gram output; APPLY: next X
     // FINAL: W <- W * decay - lr_s * X_N, written through W[] in the original orientation
     int32_t transposed, heads;
@@ -151,7 +147,6 @@ struct NsParams {
     int32_t cautious;        // decay only where X_N * W > 0
     long long wait_limit_ns;
     int* status;             // per-device status word
-    unsigned int* tile_ctr;  // two zeroed counters of this launch (tcgen05 path)
     float* W[MA_MAX_BATCH];
 };
 
@@ -184,42 +179,9 @@ bool ns_tc_is_final(const void* func);
 size_t ns_tc_launch_bytes();
 int ns_tc_patch_final(void* launch, NsFinalPatchFn f, void* ctx);
 
-// Cluster-resident chain for short units (m <= 128, rows <= columns, n <= 4096,
-// no A^2 term): one launch runs all iterations of a batch and the final
-// update of W (ns_cluster.cu).
-struct NsClusterIn {
-    const void* x;             // X0, bf16 [units][m][ldx]
-    int64_t ldx, x_unit;
-    int32_t units, m, n, steps;
-    float coef[MA_MAX_NS_STEPS][2];  // (a, b) of each iteration
-    const float* scale;        // per-unit 1 / (||u|| + eps)
-    int32_t heads;
-    int64_t Rh, C;
-    float decay, lr_s, lr_wd;
-    int32_t cautious;
-    long long wait_limit_ns;
-    int* status;
-    float* const* W;           // units / heads weight matrices
-};
-struct NsClusterLaunch {
-    CUtensorMap mapX;
-    int32_t m, n, nc, steps;
-    float coef[MA_MAX_NS_STEPS][2];
-    const float* scale;
-    int32_t heads, cautious;
-    int64_t Rh, C;
-    float decay, lr_s, lr_wd;
-    long long wait_limit_ns;
-    int* status;
-    float* W[MA_MAX_BATCH];
-};
-bool ns_cluster_eligible(int m, int n, int transposed);
-int ns_cluster_cols(int n);  // columns of X each CTA of a unit's cluster holds
-cudaError_t ns_cluster_setup();
-cudaError_t launch_ns_cluster(const NsClusterIn& in, cudaStream_t s);
-bool ns_cluster_is_kernel(const void* func);
-size_t ns_cluster_launch_bytes();
-int ns_cluster_patch(void* launch, NsFinalPatchFn f, void* ctx);
+// Q = a*I + b*A (bf16 m x m per unit, row stride ldg, unit stride g_unit).
+cudaError_t launch_ns_q1(const void* A, void* Q, int m, int64_t ldg, int64_t g_unit, int units, float a, float b,
+                         int num_sms, cudaStream_t s);
 
 // fp32 SIMT path (precision mode 1).
 cudaError_t launch_ns_simt(int mode, const NsParams& p, const void* x_buf, const void* g_buf, cudaStream_t s);

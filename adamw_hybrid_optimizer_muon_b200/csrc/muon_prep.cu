@@ -89,72 +89,121 @@ __device__ __forceinline__ void store_x8(void* X, int64_t i, const float (&d)[8]
     }
 }
 
-// Flat path: blocks of kPrepThreads threads walk the (unit, chunk) pairs of
-// the launch, kPrepChunk elements per chunk, grid-stride. A full chunk issues
-// all of its loads (4 groups of 8 elements per thread) before any arithmetic,
-// so each thread keeps 12 independent 16-byte loads in flight. The launch
-// bounds keep the kernel at most 85 registers a thread, and it uses 16 bytes
-// of shared memory: a block fits on an SM beside a Newton-Schulz CTA, so a
-// small grid of it can run under the tensor-core kernels of another batch.
-// The partial of a chunk does not depend on the grid size.
+// The chunk of a flat unit that one 256-thread block of prep_flat_kernel
+// covers: pass vt (0..255) handles the 8-element groups vt, vt + 256, ...;
+// returns its sum of squares, accumulated in that order. Loads for a full
+// chunk are all issued before any arithmetic (12 independent 16-byte loads
+// in flight per pass).
 template <bool GBF16, bool XF32>
-__global__ void __launch_bounds__(kPrepThreads, 6) prep_flat_kernel(const __grid_constant__ MuonPrepLaunch L) {
-    griddep_launch_dependents();
-    griddep_wait();
-    __shared__ float red[kPrepThreads / 32];
-    constexpr int kIter = kPrepChunk / (8 * kPrepThreads);
+__device__ __forceinline__ float prep_flat_pass(const MuonPrepLaunch& L, int u, int64_t part, int vt) {
+    constexpr int kIter = kPrepChunk / (8 * 256);
+    const int b = u / L.heads, h = u % L.heads;
     const int64_t unit_elems = L.Rh * L.C;
-    const int64_t items = (int64_t)L.batch * L.heads * L.parts;
+    const int64_t off = (int64_t)h * unit_elems;
+    const int64_t start = part * kPrepChunk;
+    const int64_t end = min(start + (int64_t)kPrepChunk, unit_elems);
+    float* M = L.M[b] + off;
+    const void* G = GBF16 ? static_cast<const void*>(reinterpret_cast<const uint16_t*>(L.G[b]) + off)
+                          : static_cast<const void*>(reinterpret_cast<const float*>(L.G[b]) + off);
+    void* X = XF32 ? static_cast<void*>(reinterpret_cast<float*>(L.X) + (int64_t)u * L.x_unit)
+                   : static_cast<void*>(reinterpret_cast<uint16_t*>(L.X) + (int64_t)u * L.x_unit);
     const float beta = L.beta, omb = L.omb;
     const bool nest = L.nesterov != 0;
-    for (int64_t w = blockIdx.x; w < items; w += gridDim.x) {
-        const int u = (int)(w / L.parts);
-        const int64_t part = w - (int64_t)u * L.parts;
-        const int b = u / L.heads, h = u % L.heads;
-        const int64_t off = (int64_t)h * unit_elems;
-        const int64_t start = part * kPrepChunk;
-        const int64_t end = min(start + (int64_t)kPrepChunk, unit_elems);
-        float* M = L.M[b] + off;
-        const void* G = GBF16 ? static_cast<const void*>(reinterpret_cast<const uint16_t*>(L.G[b]) + off)
-                              : static_cast<const void*>(reinterpret_cast<const float*>(L.G[b]) + off);
-        void* X = XF32 ? static_cast<void*>(reinterpret_cast<float*>(L.X) + (int64_t)u * L.x_unit)
-                       : static_cast<void*>(reinterpret_cast<uint16_t*>(L.X) + (int64_t)u * L.x_unit);
-        float ss = 0.f;
-        if (end - start == kPrepChunk) {
-            float g[kIter][8], m[kIter][8];
+    float ss = 0.f;
+    if (end - start == kPrepChunk) {
+        float g[kIter][8], m[kIter][8];
 #pragma unroll
-            for (int k = 0; k < kIter; ++k) {
-                const int64_t i = start + 8 * ((int64_t)k * kPrepThreads + threadIdx.x);
-                load_g8<GBF16>(G, i, g[k]);
-                const float4 a = __ldcs(reinterpret_cast<const float4*>(M + i));
-                const float4 c = __ldcs(reinterpret_cast<const float4*>(M + i + 4));
-                m[k][0] = a.x; m[k][1] = a.y; m[k][2] = a.z; m[k][3] = a.w;
-                m[k][4] = c.x; m[k][5] = c.y; m[k][6] = c.z; m[k][7] = c.w;
-            }
-#pragma unroll
-            for (int k = 0; k < kIter; ++k) {
-                const int64_t i = start + 8 * ((int64_t)k * kPrepThreads + threadIdx.x);
-                float d[8];
-                ss += momentum8(m[k], g[k], d, beta, omb, nest);
-                __stcs(reinterpret_cast<float4*>(M + i), make_float4(m[k][0], m[k][1], m[k][2], m[k][3]));
-                __stcs(reinterpret_cast<float4*>(M + i + 4), make_float4(m[k][4], m[k][5], m[k][6], m[k][7]));
-                store_x8<XF32>(X, i, d);
-            }
-        } else {
-            for (int64_t i = start + 8 * (int64_t)threadIdx.x; i < end; i += 8 * kPrepThreads) {
-                float g[8], m[8], d[8];
-                load_g8<GBF16>(G, i, g);
-                const float4 a = __ldcs(reinterpret_cast<const float4*>(M + i));
-                const float4 c = __ldcs(reinterpret_cast<const float4*>(M + i + 4));
-                m[0] = a.x; m[1] = a.y; m[2] = a.z; m[3] = a.w; m[4] = c.x; m[5] = c.y; m[6] = c.z; m[7] = c.w;
-                ss += momentum8(m, g, d, beta, omb, nest);
-                __stcs(reinterpret_cast<float4*>(M + i), make_float4(m[0], m[1], m[2], m[3]));
-                __stcs(reinterpret_cast<float4*>(M + i + 4), make_float4(m[4], m[5], m[6], m[7]));
-                store_x8<XF32>(X, i, d);
-            }
+        for (int k = 0; k < kIter; ++k) {
+            const int64_t i = start + 8 * ((int64_t)k * 256 + vt);
+            load_g8<GBF16>(G, i, g[k]);
+            const float4 a = __ldcs(reinterpret_cast<const float4*>(M + i));
+            const float4 c = __ldcs(reinterpret_cast<const float4*>(M + i + 4));
+            m[k][0] = a.x; m[k][1] = a.y; m[k][2] = a.z; m[k][3] = a.w;
+            m[k][4] = c.x; m[k][5] = c.y; m[k][6] = c.z; m[k][7] = c.w;
         }
-        const float tot = block_sum<kPrepThreads>(ss, red);
-        if (threadIdx.x == 0) L.partials[(int64_t)u * L.parts + part] = (double)tot;
+#pragma unroll
+        for (int k = 0; k < kIter; ++k) {
+            const int64_t i = start + 8 * ((int64_t)k * 256 + vt);
+            float d[8];
+            ss += momentum8(m[k], g[k], d, beta, omb, nest);
+            __stcs(reinterpret_cast<float4*>(M + i), make_float4(m[k][0], m[k][1], m[k][2], m[k][3]));
+            __stcs(reinterpret_cast<float4*>(M + i + 4), make_float4(m[k][4], m[k][5], m[k][6], m[k][7]));
+            store_x8<XF32>(X, i, d);
+        }
+    } else {
+        for (int64_t i = start + 8 * (int64_t)vt; i < end; i += 8 * 256) {
+            float g[8], m[8], d[8];
+            load_g8<GBF16>(G, i, g);
+            const float4 a = __ldcs(reinterpret_cast<const float4*>(M + i));
+            const float4 c = __ldcs(reinterpret_cast<const float4*>(M + i + 4));
+            m[0] = a.x; m[1] = a.y; m[2] = a.z; m[3] = a.w; m[4] = c.x; m[5] = c.y; m[6] = c.z; m[7] = c.w;
+            ss += momentum8(m, g, d, beta, omb, nest);
+            __stcs(reinterpret_cast<float4*>(M + i), make_float4(m[0], m[1], m[2], m[3]));
+            __stcs(reinterpret_cast<float4*>(M + i + 4), make_float4(m[4], m[5], m[6], m[7]));
+            store_x8<XF32>(X, i, d);
+        }
+    }
+    return ss;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// Flat path, on the caller's stream: one block of 256 threads per chunk of
+// kPrepChunk elements of one unit. The chunk's partial is the sum over the
+// block in a fixed order: each warp's butterfly, then the eight warps in order.
+template <bool GBF16, bool XF32>
+__global__ void __launch_bounds__(256) prep_flat_kernel(const __grid_constant__ MuonPrepLaunch L) {
+    griddep_launch_dependents();
+    griddep_wait();
+    __shared__ float red[8];
+    const int u = blockIdx.y;
+    const float s = warp_sum(prep_flat_pass<GBF16, XF32>(L, u, blockIdx.x, threadIdx.x));
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) t += red[w];
+        L.partials[(int64_t)u * L.parts + blockIdx.x] = (double)t;
+    }
+}
+
+// Flat path under another batch's Newton-Schulz kernels (a side stream): a
+// small grid of kPrepSideThreads-thread blocks walks the (unit, chunk) pairs
+// grid-stride. At most 85 registers a thread and 32 bytes of shared memory:
+// a block fits on an SM beside a Newton-Schulz CTA. Each thread makes the
+// passes of two of prep_flat_kernel's threads (vt and vt + 128, one after the
+// other) and keeps their sums apart, and the warps' butterflies and the final
+// sum run in prep_flat_kernel's order: every partial, and so every scale, is
+// the same bits on either path.
+template <bool GBF16, bool XF32>
+__global__ void __launch_bounds__(kPrepSideThreads, 6) prep_flat_side_kernel(const __grid_constant__ MuonPrepLaunch L) {
+    griddep_launch_dependents();
+    griddep_wait();
+    __shared__ float red[8];
+    const int64_t items = (int64_t)L.batch * L.heads * L.parts;
+    const int w = threadIdx.x >> 5;
+    for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+        const int u = (int)(it / L.parts);
+        const int64_t part = it - (int64_t)u * L.parts;
+        const float lo = warp_sum(prep_flat_pass<GBF16, XF32>(L, u, part, threadIdx.x));        // warps 0..3
+        const float hi = warp_sum(prep_flat_pass<GBF16, XF32>(L, u, part, threadIdx.x + 128));  // warps 4..7
+        if ((threadIdx.x & 31) == 0) {
+            red[w] = lo;
+            red[4 + w] = hi;
+        }
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float t = 0.f;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) t += red[q];
+            L.partials[(int64_t)u * L.parts + part] = (double)t;
+        }
+        __syncthreads();  // red is reused by the next chunk
     }
 }
 
@@ -261,14 +310,11 @@ __global__ void __launch_bounds__(256) prep_transpose_kernel(const __grid_consta
 }
 
 // One warp per unit: lane-strided sum of the unit's partials, then a fixed
-// butterfly, so the result does not depend on scheduling. Block 0 also zeroes
-// the tile counters of the Newton-Schulz launches that follow.
+// butterfly, so the result does not depend on scheduling.
 __global__ void __launch_bounds__(256) norm_finalize_kernel(const double* __restrict__ partials, int64_t parts,
-                                                            int units, float eps, float* __restrict__ scale,
-                                                            unsigned int* __restrict__ ctr, int nctr) {
+                                                            int units, float eps, float* __restrict__ scale) {
     griddep_launch_dependents();
     griddep_wait();
-    if (blockIdx.x == 0 && (int)threadIdx.x < nctr) ctr[threadIdx.x] = 0u;
     const int u = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int l = threadIdx.x & 31;
     if (u >= units) return;
@@ -286,8 +332,9 @@ int64_t prep_parts_per_unit(int64_t Rh, int64_t C, int transposed) {
     return (Rh * C + kPrepChunk - 1) / kPrepChunk;
 }
 
-// The flat kernels prefer the largest shared-memory carveout, the one a
-// Newton-Schulz CTA sets on its SM, so that their blocks can join that SM.
+// The side-stream flat kernels prefer the largest shared-memory carveout,
+// the one a Newton-Schulz CTA sets on its SM, so that their blocks can join
+// that SM.
 // Once per device; the attribute is set before any stream capture by the
 // library's set-up (the first call on a device).
 cudaError_t prep_setup() {
@@ -297,10 +344,10 @@ cudaError_t prep_setup() {
     if (e != cudaSuccess) return e;
     int done = 0;
     return cache.get(dev, &done, [](int* v) -> cudaError_t {
-        const void* fns[4] = {reinterpret_cast<const void*>(prep_flat_kernel<true, false>),
-                              reinterpret_cast<const void*>(prep_flat_kernel<true, true>),
-                              reinterpret_cast<const void*>(prep_flat_kernel<false, false>),
-                              reinterpret_cast<const void*>(prep_flat_kernel<false, true>)};
+        const void* fns[4] = {reinterpret_cast<const void*>(prep_flat_side_kernel<true, false>),
+                              reinterpret_cast<const void*>(prep_flat_side_kernel<true, true>),
+                              reinterpret_cast<const void*>(prep_flat_side_kernel<false, false>),
+                              reinterpret_cast<const void*>(prep_flat_side_kernel<false, true>)};
         for (const void* f : fns) {
             const cudaError_t r = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
                                                        cudaSharedmemCarveoutMaxShared);
@@ -322,26 +369,30 @@ cudaError_t launch_muon_prep(const MuonPrepLaunch& L, int max_blocks, cudaStream
         else if (gb) e = launch_pdl(prep_transpose_kernel<true, true>, grid, dim3(256), 0, s, L);
         else if (!xf) e = launch_pdl(prep_transpose_kernel<false, false>, grid, dim3(256), 0, s, L);
         else e = launch_pdl(prep_transpose_kernel<false, true>, grid, dim3(256), 0, s, L);
+    } else if (max_blocks <= 0) {
+        const dim3 grid((unsigned)L.parts, (unsigned)units);
+        if (gb && !xf) e = launch_pdl(prep_flat_kernel<true, false>, grid, dim3(256), 0, s, L);
+        else if (gb) e = launch_pdl(prep_flat_kernel<true, true>, grid, dim3(256), 0, s, L);
+        else if (!xf) e = launch_pdl(prep_flat_kernel<false, false>, grid, dim3(256), 0, s, L);
+        else e = launch_pdl(prep_flat_kernel<false, true>, grid, dim3(256), 0, s, L);
     } else {
         if ((e = prep_setup()) != cudaSuccess) return e;
         int64_t items = (int64_t)units * L.parts;
-        if (max_blocks > 0 && items > max_blocks) items = max_blocks;
-        if (items > INT32_MAX) items = INT32_MAX;
-        const dim3 grid((unsigned)items), block(kPrepThreads);
-        if (gb && !xf) e = launch_pdl(prep_flat_kernel<true, false>, grid, block, 0, s, L);
-        else if (gb) e = launch_pdl(prep_flat_kernel<true, true>, grid, block, 0, s, L);
-        else if (!xf) e = launch_pdl(prep_flat_kernel<false, false>, grid, block, 0, s, L);
-        else e = launch_pdl(prep_flat_kernel<false, true>, grid, block, 0, s, L);
+        if (items > max_blocks) items = max_blocks;
+        const dim3 grid((unsigned)items), block(kPrepSideThreads);
+        if (gb && !xf) e = launch_pdl(prep_flat_side_kernel<true, false>, grid, block, 0, s, L);
+        else if (gb) e = launch_pdl(prep_flat_side_kernel<true, true>, grid, block, 0, s, L);
+        else if (!xf) e = launch_pdl(prep_flat_side_kernel<false, false>, grid, block, 0, s, L);
+        else e = launch_pdl(prep_flat_side_kernel<false, true>, grid, block, 0, s, L);
     }
     return e;
 }
 
 cudaError_t launch_norm_finalize(const double* partials, int64_t parts, int units, float eps, float* scale,
-                                 unsigned int* ctr, int nctr, cudaStream_t s) {
+                                 cudaStream_t s) {
     if (units == 0) return cudaSuccess;
-    if (nctr < 0 || nctr > 256 || (nctr > 0 && !ctr)) return cudaErrorInvalidValue;
     return launch_pdl(norm_finalize_kernel, dim3((units + 7) / 8), dim3(256), 0, s, partials, parts, units, eps,
-                      scale, ctr, nctr);
+                      scale);
 }
 
 }  // namespace ma

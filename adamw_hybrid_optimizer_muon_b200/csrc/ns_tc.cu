@@ -85,26 +85,7 @@ constexpr uint32_t WBUF_BYTES = EPI_WARPS * FIN_WARP_BYTES;      // 96 KB
 constexpr int kStages(int mode) { return mode == NS_FINAL ? 4 : STAGES; }
 constexpr uint32_t kEpiBytes(int mode) { return mode == NS_FINAL ? WBUF_BYTES : STG_BYTES; }
 
-// Tiles are handed out at run time: the leader's producer thread takes the
-// next tile index from the launch's counter (one atomic add per tile, ahead
-// of need) and publishes it to the pair's other roles through a ring of
-// kRing slots in shared memory, two tiles ahead of its own loads. The pairs
-// running at any moment therefore work on a contiguous window of the
-// launch's tile order, whatever their speed, which keeps the operand strips
-// that window shares in L2. A tile's arithmetic does not depend on which pair
-// computes it.
-//
-// A slot needs no "consumed" barrier: when the leader writes the slot of tile
-// s + 2 (about to load tile s), it has issued every load of tile s - 1, so the
-// MMA thread has consumed a stage use of tile s - 1 - NST or later (the stage
-// ring allows no more), which it did after taking that tile and after the
-// epilogue warps of both CTAs released tile s - 3 - NST; each epilogue warp
-// takes its next tile before it releases the current one, so all of them
-// have taken tile s - 2 - NST; the peer's producer issued the loads the MMA
-// thread consumed. Every consumer has therefore taken tile s + 2 - kRing
-// whenever kRing >= NST + 4.
 constexpr int kMaxStages = 8;
-constexpr int kRing = kMaxStages + 4;
 // Wind-down after an abort: waits for the pair's own work in flight (issued
 // MMAs, bulk loads) are bounded by at least this, whatever the wait limit.
 constexpr long long kDrainNs = 50000000LL;
@@ -115,8 +96,6 @@ struct Ctl {
     uint64_t full[kMaxStages], empty[kMaxStages];  // stage ring: data landed / stage released by the MMAs
     uint64_t acc_full[2], acc_empty[2];            // TMEM accumulators: ready for the epilogue / free again
     uint64_t drain;                                // the MMA thread's last commit before an aborted exit
-    uint64_t tile_full[kRing];                     // tile ring: index published
-    int32_t tile_id[kRing];                        // tile index of each ring slot, -1 = no more tiles
     uint32_t tmem_base;
     int32_t abort_flag;
     int32_t issued;                    // producer: stage uses armed and loaded so far
@@ -163,8 +142,10 @@ struct NsJob {
     float a, b, c, coef_gram;
     const float* scale;
     const void* xin;
+    const void* zin;    // GRAMSQ: the second operand Z (and the combine input); xin when it is A itself
     void* out;
     int32_t transposed, heads, cautious, w0;
+    int32_t same;       // GRAM/GRAMSQ: both operands are rows of one matrix (a diagonal tile loads it once)
     int64_t Rh, C;
     float decay, lr_s, lr_wd;
     int32_t tiles_per_unit, mt, nt, kblocks, tile0;
@@ -176,7 +157,6 @@ struct NsLaunch {
     int32_t njobs, total_tiles;
     long long wait_limit_ns;
     int* status;
-    unsigned int* tile_ctr;  // zero before the launch; one atomic add per tile handed out
     float* W[kMaxW];
 };
 
@@ -260,11 +240,11 @@ __device__ __forceinline__ void epilogue_values(const NsJob& p, const TileCoord&
 #pragma unroll
         for (int t = 0; t < 32; ++t) o[t] = coef * v[t];
     } else if (MODE == NS_GRAMSQ) {
-        // acc = A^2; A is read back from the Gram buffer, 8 values at a time
+        // acc = A Z^T (= A Z: both symmetric); out = b*Z + c*acc, Z read back 8 values at a time
         const int m = p.m;
         const float b = p.b, c = p.c;
-        const __nv_bfloat16* Gin = reinterpret_cast<const __nv_bfloat16*>(p.xin) + (int64_t)tc.u * p.g_unit;
-        combine_row(Gin + (int64_t)row * p.ldg + col0, row < m, m - col0, b, c, v, o);
+        const __nv_bfloat16* Zin = reinterpret_cast<const __nv_bfloat16*>(p.zin) + (int64_t)tc.u * p.g_unit;
+        combine_row(Zin + (int64_t)row * p.ldg + col0, row < m, m - col0, b, c, v, o);
     } else {
         const int m = p.m, n = p.n;
         const float sa = p.first ? p.scale[tc.u] : 1.f;
@@ -288,49 +268,6 @@ __device__ __forceinline__ uint32_t sw64(uint32_t r, uint32_t q) { return r * 64
 // Byte offset of 16-byte chunk q of row r in a 128-byte-row block of W.
 __device__ __forceinline__ uint32_t sw128w(uint32_t r, uint32_t q) { return r * 128u + ((q ^ (r & 7u)) << 4); }
 
-// ------------------------------------------------------------------ tile ring
-
-// Leader's producer: publish tile index t (-1: no more tiles) as sequence
-// number seq, in this CTA and in the peer CTA of the pair. Every consumer is
-// done with the slot's previous use (see kRing).
-template <bool PAIR>
-__device__ __forceinline__ void ring_publish(Ctl* ctl, int seq, int t) {
-    const int slot = seq % kRing;
-    ctl->tile_id[slot] = t;
-    if (PAIR) {
-        st_cluster_s32(mapa_shared(smem_u32(&ctl->tile_id[slot]), 1), t);
-        mbar_arrive_cluster(mapa_shared(smem_u32(&ctl->tile_full[slot]), 1));  // release: the store above first
-    }
-    mbar_arrive(&ctl->tile_full[slot]);
-}
-
-// Consumer (one thread): the tile index of sequence number seq. Returns -1
-// with *ok = false when the wait gave up (timeout or abort).
-template <bool PAIR>
-__device__ __forceinline__ int ring_take(Ctl* ctl, int seq, uint32_t rank, const AbortCtl& ab, const NsLaunch& L,
-                                         uint32_t sleep_ns, bool* ok) {
-    const int slot = seq % kRing;
-    const uint32_t par = (uint32_t)(seq / kRing) & 1u;
-    const bool remote = PAIR && rank != 0;
-    if (!mbar_wait_ctl(&ctl->tile_full[slot], par, ab, L.wait_limit_ns, L.status, sleep_ns, remote)) {
-        *ok = false;
-        return -1;
-    }
-    *ok = true;
-    return reinterpret_cast<volatile int32_t*>(ctl->tile_id)[slot];
-}
-
-// Epilogue warp: the tile of sequence number seq (lane 0 takes it from the
-// ring, the warp shares it); -1 when there are no more tiles or on an abort.
-template <bool PAIR>
-__device__ __forceinline__ int epi_take(Ctl* ctl, int seq, uint32_t rank, const AbortCtl& ab, const NsLaunch& L,
-                                        int lane) {
-    int t = -1;
-    bool ok = true;
-    if (lane == 0) t = ring_take<PAIR>(ctl, seq, rank, ab, L, kEpiSleepNs, &ok);
-    return __shfl_sync(0xffffffffu, t, 0);
-}
-
 // Final apply: W <- W*(1 - lr*wd) - lr*scale*X_N in the caller's fp32 weights,
 // run by each epilogue warp over its 32-column chunks of every tile.
 //
@@ -344,8 +281,9 @@ __device__ __forceinline__ int epi_take(Ctl* ctl, int seq, uint32_t rank, const 
 // (or, transposed, its own column) of the W block in place, and the block
 // goes back to W with coalesced 16-byte stores.
 template <bool PAIR>
-__device__ __forceinline__ void final_epilogue(const NsLaunch& L, Ctl* ctl, uint32_t rank, uint32_t tmem_base,
-                                               int warp, int lane, uint8_t* wbuf, const AbortCtl& ab) {
+__device__ __forceinline__ void final_epilogue(const NsLaunch& L, Ctl* ctl, int pair, int npairs, uint32_t rank,
+                                               uint32_t tmem_base, int warp, int lane, uint8_t* wbuf,
+                                               const AbortCtl& ab) {
     using S = Shape<NS_FINAL, PAIR>;
     constexpr int CPW = S::CPW;
     const int quad = warp & 3, half = (warp - 2) / 4;
@@ -353,9 +291,8 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, Ctl* ctl, uint
     const uint32_t acc_empty_leader0 = PAIR ? mapa_shared(smem_u32(&ctl->acc_empty[0]), 0) : 0u;
     const uint32_t acc_empty_leader1 = PAIR ? mapa_shared(smem_u32(&ctl->acc_empty[1]), 0) : 0u;
     uint8_t* xbuf = wbuf + 2 * WBUF;
-    // each tile is taken before the previous accumulator is released (see kRing)
-    int t = epi_take<PAIR>(ctl, 0, rank, ab, L, lane);
-    for (int lt = 0; t >= 0; ++lt) {  // -1: no more tiles, or an abort
+    int lt = 0;
+    for (int t = pair; t < L.total_tiles; t += npairs, ++lt) {
         const JobTile jt = decode_job_tile(L, NS_FINAL, t);
         const NsJob& p = L.job[jt.j];
         const TileCoord tc = jt.tc;
@@ -463,7 +400,6 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, Ctl* ctl, uint
             fetch(c + 2);
         }
         cp_async_wait<0>();  // drop the copies of chunks this tile does not use
-        t = epi_take<PAIR>(ctl, lt + 1, rank, ab, L, lane);
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
@@ -525,6 +461,8 @@ __global__ void __launch_bounds__(THREADS, 1)
     griddep_launch_dependents();
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;  // 0 = leader of the pair
     const bool leader = rank == 0;
+    const int pair = PAIR ? (int)cluster_id_x() : (int)blockIdx.x;
+    const int npairs = PAIR ? (int)cluster_count_x() : (int)gridDim.x;
     const int total_tiles = L.total_tiles;
     const long long limit = L.wait_limit_ns;
     constexpr bool kApply = (MODE == NS_APPLY || MODE == NS_FINAL);
@@ -540,7 +478,6 @@ __global__ void __launch_bounds__(THREADS, 1)
             mbar_init(&ctl->acc_empty[a], (PAIR ? 2 : 1) * EPI_WARPS);  // leader: every epilogue warp of the pair
         }
         mbar_init(&ctl->drain, 1);
-        for (int r = 0; r < kRing; ++r) mbar_init(&ctl->tile_full[r], 1);  // the leader's publish
         ctl->abort_flag = 0;
         ctl->issued = 0;
         ctl->consumed = 0;
@@ -570,44 +507,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     if (warp == 0) {
         if (lane == 0) {
             // In the applies every pair working at the same time reads all of
-            // the m x m Gram (the A operand): keep it in L2 ahead of the X
-            // strips, which the window of running tiles reads once.
+            // the m x m Gram (the A operand), one wave after another: keep it in
+            // L2 ahead of the X strips, which each wave reads once.
             const uint64_t keep = l2_evict_last_policy();
             int stage = 0;
             uint32_t phase = 0;
             int issued = 0;
             bool ok = true;
-            // The leader publishes each tile index two tiles ahead of its own
-            // loads (the peer's producer, the MMA thread and the epilogue warps
-            // find it waiting at every tile boundary), and takes indices from
-            // the counter one further ahead, so that the atomic's latency hides
-            // behind a whole tile of loads. -1 ends the sequence.
-            auto take_next = [&](int prev) -> int {
-                if (prev < 0) return -1;
-                const unsigned int v = atomicAdd(L.tile_ctr, 1u);
-                return v < (unsigned int)total_tiles ? (int)v : -1;
-            };
-            int cur0 = -1, cur1 = -1, nxt = -1;  // leader: tiles seq, seq + 1 (published), seq + 2 (taken)
-            if (leader) {
-                cur0 = take_next(0);
-                cur1 = take_next(cur0);
-                nxt = take_next(cur1);
-                ring_publish<PAIR>(ctl, 0, cur0);  // the ring is fresh
-                if (cur0 >= 0) ring_publish<PAIR>(ctl, 1, cur1);
-            }
-            for (int seq = 0; ok; ++seq) {
-                int t;
-                if (leader) {
-                    t = cur0;
-                    if (t < 0) break;
-                    if (cur1 >= 0) ring_publish<PAIR>(ctl, seq + 2, nxt);  // tile seq + 2, before loading tile seq
-                    cur0 = cur1;
-                    cur1 = nxt;
-                    nxt = take_next(nxt);
-                } else {
-                    t = ring_take<PAIR>(ctl, seq, rank, ab, L, 0, &ok);
-                }
-                if (t < 0) break;
+            for (int t = pair; t < total_tiles && ok; t += npairs) {
                 const JobTile jt = decode_job_tile(L, MODE, t);
                 const TileCoord tc = jt.tc;
                 const CUtensorMap* mapA = &L.mA[jt.j];
@@ -616,7 +523,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const int arow = tc.ti * S::TM + (int)rank * HM;
                 const int bcol = tc.tj * S::TN + (int)rank * S::CN;
                 // a diagonal Gram tile multiplies a block of rows by itself: B is A's smem
-                const bool diag = !kApply && tc.ti == tc.tj;
+                const bool diag = !kApply && tc.ti == tc.tj && L.job[jt.j].same;
                 const uint32_t stage_tx = diag ? A_BYTES : S::STAGE;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait_ctl(&ctl->empty[stage], phase ^ 1u, ab, limit, L.status)) {
@@ -676,9 +583,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             uint32_t phase = 0;
             int consumed = 0;
             bool ok = true;
-            for (int lt = 0; ok; ++lt) {
-                const int t = ring_take<PAIR>(ctl, lt, rank, ab, L, 0, &ok);
-                if (t < 0) break;
+            int lt = 0;
+            for (int t = pair; t < total_tiles && ok; t += npairs, ++lt) {
                 const int acc = lt & 1;
                 const uint32_t use = (uint32_t)(lt >> 1);
                 if (!mbar_wait_ctl(&ctl->acc_empty[acc], (use & 1u) ^ 1u, ab, limit, L.status)) {
@@ -689,7 +595,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 const uint32_t d_tmem = tmem_base + (uint32_t)(acc * S::TN);
                 const JobTile jt = decode_job_tile(L, MODE, t);
                 const int kblocks = L.job[jt.j].kblocks;
-                const bool diag = !kApply && jt.tc.ti == jt.tc.tj;
+                const bool diag = !kApply && jt.tc.ti == jt.tc.tj && L.job[jt.j].same;
                 for (int kb = 0; kb < kblocks; ++kb) {
                     if (!mbar_wait_ctl(&ctl->full[stage], phase, ab, limit, L.status)) {
                         ok = false;
@@ -723,7 +629,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
     } else if (MODE == NS_FINAL) {
-        final_epilogue<PAIR>(L, ctl, rank, tmem_base, warp, lane, staging + (warp - 2) * FIN_WARP_BYTES, ab);
+        final_epilogue<PAIR>(L, ctl, pair, npairs, rank, tmem_base, warp, lane, staging + (warp - 2) * FIN_WARP_BYTES,
+                             ab);
     } else {
         const int quad = warp & 3;              // TMEM lanes [32*quad, 32*quad + 32)
         const int half = (warp - 2) / 4;        // which half of the 256 columns
@@ -732,9 +639,8 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint64_t stream_out = l2_evict_first_policy();
         const uint32_t acc_empty_leader0 = PAIR ? mapa_shared(smem_u32(&ctl->acc_empty[0]), 0) : 0u;
         const uint32_t acc_empty_leader1 = PAIR ? mapa_shared(smem_u32(&ctl->acc_empty[1]), 0) : 0u;
-        // each tile is taken before the previous accumulator is released (see kRing)
-        int t = epi_take<PAIR>(ctl, 0, rank, ab, L, lane);
-        for (int lt = 0; t >= 0; ++lt) {  // -1: no more tiles, or an abort
+        int lt = 0;
+        for (int t = pair; t < total_tiles; t += npairs, ++lt) {
             const JobTile jt = decode_job_tile(L, MODE, t);
             const NsJob& p = L.job[jt.j];
             const CUtensorMap* mapOut = &L.mO[jt.j];
@@ -788,7 +694,6 @@ __global__ void __launch_bounds__(THREADS, 1)
                     bulk_commit_group();
                 }
             }
-            t = epi_take<PAIR>(ctl, lt + 1, rank, ab, L, lane);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
@@ -924,7 +829,16 @@ cudaError_t launch_mode(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_
                 if (!make_map(&L.mA[j], p.xin, p.m, p.m, p.units, p.ldg, p.g_unit, BK, HM))
                     return cudaErrorInvalidValue;
             }
-            L.mB[j] = L.mA[j];  // both operands are 128-row, 64-deep K-major boxes of the same matrix
+            // both operands are 128-row, 64-deep K-major boxes: of the same matrix,
+            // or (GRAMSQ with a second operand) of Z
+            if (MODE == NS_GRAMSQ && p.zin && p.zin != p.xin) {
+                if (!make_map(&L.mB[j], p.zin, p.m, p.m, p.units, p.ldg, p.g_unit, BK, HM))
+                    return cudaErrorInvalidValue;
+                J.same = 0;
+            } else {
+                L.mB[j] = L.mA[j];
+                J.same = 1;
+            }
             if (!make_map(&L.mO[j], p.out, p.m, p.m, p.units, p.ldg, p.g_unit, 32, 32, CU_TENSOR_MAP_SWIZZLE_64B))
                 return cudaErrorInvalidValue;
         } else {
@@ -941,6 +855,7 @@ cudaError_t launch_mode(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_
         J.ldx = p.ldx; J.ldg = p.ldg; J.x_unit = p.x_unit; J.g_unit = p.g_unit;
         J.a = p.a; J.b = p.b; J.c = p.c; J.coef_gram = p.coef_gram;
         J.scale = p.scale; J.xin = p.xin; J.out = p.out;
+        J.zin = (MODE == NS_GRAMSQ && p.zin) ? p.zin : p.xin;
         J.transposed = p.transposed; J.heads = p.heads; J.cautious = p.cautious;
         J.Rh = p.Rh; J.C = p.C; J.decay = p.decay; J.lr_s = p.lr_s; J.lr_wd = p.lr_wd;
         J.tiles_per_unit = tiles; J.mt = mt; J.nt = nt; J.kblocks = kblocks;
@@ -960,11 +875,7 @@ cudaError_t launch_mode(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_
     L.total_tiles = tile0;
     L.wait_limit_ns = jobs[0].p->wait_limit_ns;
     L.status = jobs[0].p->status;
-    // the launch's own counter: the first of the pair for the CTA-pair kernel,
-    // the second for the single-CTA kernel of the same grouped launch
-    L.tile_ctr = jobs[0].p->tile_ctr ? jobs[0].p->tile_ctr + (PAIR ? 0 : 1) : nullptr;
     if (tile0 <= 0) return cudaSuccess;
-    if (!L.tile_ctr) return cudaErrorInvalidValue;
     int max_units = 0;
     cudaError_t e = setup_mode<MODE, PAIR>(num_sms, &max_units);
     if (e != cudaSuccess) return e;
@@ -1013,7 +924,57 @@ cudaError_t launch_split(const NsJobIn* jobs, int njobs, int num_sms, cudaStream
     return cudaSuccess;
 }
 
+// Q = a*I + b*A for every unit: the first factor of the Gram-space chain.
+// Eight bf16 elements per thread and step, grid-stride over units and rows.
+__global__ void __launch_bounds__(256) ns_q1_kernel(const __nv_bfloat16* __restrict__ A, __nv_bfloat16* __restrict__ Q,
+                                                    int m, int64_t ldg, int64_t g_unit, int units, float a, float b) {
+    griddep_launch_dependents();
+    griddep_wait();
+    const int64_t per_row = (m + 7) / 8;
+    const int64_t total = (int64_t)units * m * per_row;
+    for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < total; w += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t u = w / ((int64_t)m * per_row);
+        const int64_t rem = w - u * m * per_row;
+        const int row = (int)(rem / per_row);
+        const int c0 = (int)(rem - (int64_t)row * per_row) * 8;
+        const int64_t off = u * g_unit + (int64_t)row * ldg + c0;
+        if (c0 + 8 <= m) {
+            const uint4 v = *reinterpret_cast<const uint4*>(A + off);
+            const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+            float f[8];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                f[2 * e] = b * bf16_lo(x[e]);
+                f[2 * e + 1] = b * bf16_hi(x[e]);
+            }
+            if (row >= c0 && row < c0 + 8) f[row - c0] += a;
+            uint4 o;
+            o.x = pack_bf16x2(f[0], f[1]);
+            o.y = pack_bf16x2(f[2], f[3]);
+            o.z = pack_bf16x2(f[4], f[5]);
+            o.w = pack_bf16x2(f[6], f[7]);
+            *reinterpret_cast<uint4*>(Q + off) = o;
+        } else {
+            for (int e = 0; c0 + e < m; ++e) {
+                const float f = b * __bfloat162float(A[off + e]) + (row == c0 + e ? a : 0.f);
+                Q[off + e] = __float2bfloat16_rn(f);
+            }
+        }
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_ns_q1(const void* A, void* Q, int m, int64_t ldg, int64_t g_unit, int units, float a, float b,
+                         int num_sms, cudaStream_t s) {
+    if (units <= 0 || m <= 0) return cudaSuccess;
+    const int64_t total = (int64_t)units * m * ((m + 7) / 8);
+    int64_t blocks = (total + 255) / 256;
+    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
+    return launch_pdl(ns_q1_kernel, dim3((unsigned)blocks), dim3(256), 0, s,
+                      reinterpret_cast<const __nv_bfloat16*>(A), reinterpret_cast<__nv_bfloat16*>(Q), m, ldg, g_unit,
+                      units, a, b);
+}
 
 size_t ns_tc_smem_bytes() {  // the largest dynamic shared memory of any instance
     size_t m = 0;

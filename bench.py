@@ -282,6 +282,19 @@ def small_inputs(wl):
     return wl.numel * 14 < 2 * L2_BYTES
 
 
+def _descs_for(wl, ma):
+    """Host-only tensor descriptors of a workload (shapes and roles) for ma_partition."""
+    out = []
+    for t in wl.tensors:
+        d = ma.Tensor()
+        d.ndim = len(t.shape)
+        for k, v in enumerate(t.shape[:2]):
+            d.shape[k] = v
+        d.role = t.role
+        out.append(d)
+    return out
+
+
 def workload_config(wl, n_gpus):
     import oracle
     kinds = oracle.partition([(t.shape, t.role) for t in wl.tensors])
@@ -513,7 +526,7 @@ def main():
 
     if rank == 0:
         peaks = load_peaks()
-        ns_cls = ("ns_gram", "ns_apply", "ns_gramsq", "ns_final", "ns_cluster")
+        ns_cls = ("ns_gram", "ns_apply", "ns_gramsq", "ns_final")
         ns_ms = sum(prof[c]["ms"] for c in ns_cls)
         ns_fl = sum(prof[c]["flops"] for c in ns_cls)
         ns_bytes = sum(prof[c]["bytes"] for c in ns_cls)
@@ -524,6 +537,17 @@ def main():
         capped = bool(clk and clk.get("sm_mhz") and clk.get("sm_max_mhz")
                       and clk["sm_mhz"] < 0.95 * clk["sm_max_mhz"])
         peak_t = peaks["bf16_tflops_sustained"] if capped else peaks["bf16_tflops"]
+        # the flops the pages' iteration itself would take (N Grams, symmetric,
+        # and N applies per matrix); the achieved rate counts the flops executed,
+        # which the Gram-space chain of wide matrices makes fewer
+        direct = 0.0
+        for t, kd in zip(wl.tensors, ma.ma_partition(_descs_for(wl, ma))):
+            if kd != ma.MA_MUON:
+                continue
+            g = wl.groups[t.group].muon
+            rh = t.shape[0] // g.heads
+            m_, n_ = min(rh, t.shape[1]), max(rh, t.shape[1])
+            direct += g.heads * g.ns_steps * (m_ * (m_ + 1) * n_ + 2 * m_ * m_ * n_)
         roofline = {"kernel": "ns_tc_kernel (Newton-Schulz Gram + apply, tcgen05)", "bound": "tensor",
                     "achieved": ns_tflops, "peak": peak_t, "unit": "TFLOP/s",
                     "frac": ns_tflops / peak_t if ns_tflops else None,
@@ -531,7 +555,8 @@ def main():
                     "traffic": ns_traffic(args.workload, ns_launches / args.steps),
                     "traffic_algorithmic": ns_bytes / max(1, ns_launches),
                     "launches": ns_launches, "avg_launch_ms": ns_ms / max(1, ns_launches),
-                    "flops_per_launch": ns_fl / max(1, ns_launches)}
+                    "flops_per_launch": ns_fl / max(1, ns_launches),
+                    "flops_per_step_executed": ns_fl / args.steps, "flops_per_step_direct_iteration": direct}
         kernels = {}
         for c in ma.PROF_CLASSES:
             pc = prof[c]

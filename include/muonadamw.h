@@ -369,13 +369,12 @@ void ma_plan_destroy(ma_plan_t* plan);
 #define MA_PROF_FINALIZE 2      /* norm finalize                               */
 #define MA_PROF_NS_GRAM 3       /* Newton-Schulz A = X X^T (tcgen05 or fp32)   */
 #define MA_PROF_NS_APPLY 4      /* Newton-Schulz X' = aX + BX (not the last)   */
-#define MA_PROF_NS_GRAMSQ 5     /* Newton-Schulz A^2 (c != 0 only)             */
+#define MA_PROF_NS_GRAMSQ 5     /* symmetric m x m products: A^2 (c != 0), and */
+                                /* the Gram-space chain's Q, A P and P A P     */
 #define MA_PROF_NS_FINAL 6      /* last apply, fused with decay and W update   */
 #define MA_PROF_MOMENTUM_SIDE 7 /* momentum pass run under the Newton-Schulz   */
                                 /* chain of the batch before it (side stream)  */
-#define MA_PROF_NS_CLUSTER 8    /* whole chain of short units (m <= 128) in    */
-                                /* one cluster-resident launch                 */
-#define MA_PROF_CLASSES 9
+#define MA_PROF_CLASSES 8
 
 /* When on != 0, every kernel the library launches on this thread's current
  * device is bracketed by two CUDA events recorded on its launch stream. Off by

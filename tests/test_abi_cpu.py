@@ -227,7 +227,7 @@ def test_plan_sizing_on_host():
     assert ws3 == 2 * ((expect + 255) // 256 * 256)
     ma.ma_plan_destroy(plan)
     # a cap below two halves of the largest single matrix: one workspace
-    one = ma.muon_workspace_bytes(1, 4096, 11008, hp)
+    one = max(ma.muon_workspace_bytes(1, 4096, 11008, hp), ma.muon_workspace_bytes(1, 11008, 4096, hp))
     plan, ws4 = ma.ma_plan_create(descs, _groups_for(wl), ws_cap=one + 4096)
     assert ws4 <= one + 4096
     ma.ma_plan_destroy(plan)
@@ -253,9 +253,9 @@ def test_plan_describe():
     ma.ma_plan_destroy(plan)
     assert text.startswith(f"workspace {ws} bytes in two halves of {ws // 2} (momentum passes under the previous "
                            f"chain); AdamW: 67 tensors, ")
-    assert "4096 x 4096, 128 matrices (bf16 grads), heads 1, sub-batches of 32" in text
-    assert "4096 x 11008, 64 matrices (bf16 grads), heads 1, sub-batches of 16" in text
-    assert "11008 x 4096, 32 matrices (bf16 grads), heads 1, sub-batches of 16" in text
+    assert "4096 x 4096, 128 matrices (bf16 grads), heads 1, sub-batches of 32, direct chain" in text
+    assert "4096 x 11008, 64 matrices (bf16 grads), heads 1, sub-batches of 16, Gram-space chain" in text
+    assert "11008 x 4096, 32 matrices (bf16 grads), heads 1, sub-batches of 16, Gram-space chain" in text
     segs = [ln for ln in text.splitlines() if ln.startswith("segment")]
     assert segs[0] == "segment 0: AdamW" and len(segs) == 1 + 4 + 4 + 2  # no sharing at this size
     # the d20 set: its three buckets share one chain of Newton-Schulz launches

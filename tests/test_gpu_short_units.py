@@ -1,13 +1,12 @@
-"""The cluster-resident Newton-Schulz chain for short units (m <= 128) against the oracle.
+"""Short units (at most 128 rows) against the oracle.
 
-Units with at most 128 rows, no more rows than columns and at most 4096
-columns (the per-head slices of Q/K/V among them) run their whole chain in
-one launch: a cluster of eight CTAs keeps the unit's X in shared memory and
-reduces the Gram partials over distributed shared memory. Cases span one to
-eight CTAs holding columns, ragged column counts (a CTA with a partial block,
-CTAs with none), fewer than 128 rows, single rows, head slices, and the
-per-iteration coefficient table. Results are compared with the fp64 oracle at
-the bf16 tolerance, and two calls on the same inputs must agree bit for bit.
+Units with m <= 128 run on the single-CTA instance of the Newton-Schulz
+kernels: the per-head slices of Q/K/V (128 x 4096, 128 x 1024) and small
+matrices. The 128 x 4096 slices take the Gram-space chain (one Gram, 128 x 128
+symmetric products, one final apply); the others the direct iteration.
+Cases: ragged column counts, fewer than 128 rows, a single row, head
+slices, and a per-iteration coefficient table, compared with the fp64 oracle
+at the bf16 tolerance; two calls on the same inputs agree bit for bit.
 """
 import numpy as np
 import pytest
@@ -22,24 +21,24 @@ pytestmark = pytest.mark.gpu
 
 CASES = [
     # (R, C), heads, batch
-    ((128, 4096), 1, 2),    # every CTA holds 512 columns
-    ((4096, 4096), 32, 1),  # 32 head slices of 128 x 4096
+    ((128, 4096), 1, 2),    # Gram space: 128 x 128 products
+    ((4096, 4096), 32, 1),  # 32 head slices of 128 x 4096 (Gram space)
     ((64, 1024), 1, 3),     # 64 rows: the rest of the 128-row tile is zero
-    ((96, 520), 1, 2),      # 128-column blocks: four full, one of 8 columns, three empty
-    ((128, 256), 1, 1),     # 64-column blocks in four CTAs, four empty
-    ((1, 64), 1, 2),        # one row, one CTA
+    ((96, 520), 1, 2),      # ragged rows and columns
+    ((128, 256), 1, 1),     # one 128 x 256 tile
+    ((1, 64), 1, 2),        # one row
     ((384, 1024), 3, 2),    # three head slices of 128 x 1024
 ]
 
 
-def _hp(coeffs):
-    return ma.muon_hparams(coeffs=coeffs, ns_steps=len(coeffs) if len(coeffs) > 1 else 5)
+def _hp(coeffs, heads=1):
+    return ma.muon_hparams(coeffs=coeffs, ns_steps=len(coeffs) if len(coeffs) > 1 else 5, heads=heads)
 
 
 @pytest.mark.parametrize("case", CASES, ids=lambda c: f"{c[0][0]}x{c[0][1]}h{c[1]}b{c[2]}")
-def test_cluster_chain_matches_oracle(case):
+def test_short_units_match_oracle(case):
     (R, C), heads, batch = case
-    hp = _hp(((1.5, -0.5, 0.0),))
+    hp = _hp(((1.5, -0.5, 0.0),), heads)
     r = np.random.default_rng(R * 7 + C)
     W0 = [(r.standard_normal((R, C)) * 0.02).astype(np.float32) for _ in range(batch)]
     Wd = [dev_f32(w) for w in W0]
@@ -58,11 +57,11 @@ def test_cluster_chain_matches_oracle(case):
             check_muon(w0, host(w), rw, f32(0.02), f32(0.01), TOL_BF16, what=f"{R}x{C} heads {heads}")
 
 
-def test_cluster_chain_coefficient_table_and_repeatability():
+def test_short_units_coefficient_table_and_repeatability():
     # a different (a, b) per iteration; the same inputs twice give the same bits
     R, C, heads = 512, 2048, 4
     co = ((2.0, -1.0, 0.0), (1.75, -0.75, 0.0), (1.5, -0.5, 0.0), (1.5, -0.5, 0.0))  # p(1) = 1 each
-    hp = _hp(co)
+    hp = _hp(co, heads)
     r = np.random.default_rng(5)
     W0 = (r.standard_normal((R, C)) * 0.02).astype(np.float32)
     g = bf16_round(r.standard_normal((R, C)) * 1e-3)
