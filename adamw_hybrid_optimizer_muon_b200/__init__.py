@@ -20,7 +20,7 @@ __all__ = [
     "muon_step_batched_noalloc", "STATIC_SCRATCH_BYTES", "ns_iterate_workspace_bytes", "ns_iterate_bf16",
     "adamw_step_fused", "ma_plan_create", "muonadamw_step", "muonadamw_step_graph", "muonadamw_step_from_host",
     "ma_plan_describe", "ma_plan_destroy", "ma_plan_status", "ma_device_status", "ma_device_status_async",
-    "ma_set_wait_limit_ns",
+    "ma_set_wait_limit_ns", "ma_set_momentum_overlap",
     "ma_selftest_wait_timeout", "ma_profile_enable", "ma_profile_collect", "PROF_CLASSES", "group_table", "Plan",
     "MuonAdamW", "muon_hparams", "adamw_hparams",
 ]
@@ -136,6 +136,7 @@ def lib() -> ctypes.CDLL:
         "ma_device_status_async": (i32, [vp, vp]),
         "ma_plan_status": (i32, [vp, vp]),
         "ma_set_wait_limit_ns": (i32, [i64]),
+        "ma_set_momentum_overlap": (i32, [i32]),
         "ma_selftest_wait_timeout": (i32, [i64, vp]),
         "muon_step_batched_noalloc": (i32, [i32, i64, i64, pp, pp, i32, pp, ctypes.POINTER(MuonHParams), vp]),
         "ma_profile_enable": (i32, [i32]),
@@ -410,6 +411,12 @@ def ma_device_status_async(host_dst, stream=None) -> None:
 def ma_set_wait_limit_ns(limit_ns: int) -> None:
     """Time limit of the kernels' bounded waits, in nanoseconds (default 2 s)."""
     _check(lib().ma_set_wait_limit_ns(int(limit_ns)), "ma_set_wait_limit_ns")
+
+
+def ma_set_momentum_overlap(on: bool) -> None:
+    """Momentum passes under the previous sub-batch's chain, on a side stream, for plans created
+    after the call (default off: slower on a B200, see the header)."""
+    _check(lib().ma_set_momentum_overlap(1 if on else 0), "ma_set_momentum_overlap")
 
 
 def ma_selftest_wait_timeout(limit_ns: int, stream=None) -> None:

@@ -37,6 +37,9 @@ namespace ma {
 __device__ int g_status = 0;
 
 static std::atomic<long long> g_host_wait_limit_ns{2000000000LL};
+// Plans created while this is set get two workspace halves and run momentum
+// passes on a side stream (ma_set_momentum_overlap).
+static std::atomic<int> g_momentum_overlap{0};
 long long host_wait_limit_ns() { return g_host_wait_limit_ns.load(std::memory_order_relaxed); }
 
 int* device_status_ptr() {
@@ -313,7 +316,7 @@ int muon_prep(const MuonJob& j, cudaStream_t s, int max_blocks, bool side, int* 
     P.ldx = g.ldx;
     P.x_unit = g.m * g.ldx;
     P.parts = g.parts;
-    P.tiles_c = (g.C + kPrepTile - 1) / kPrepTile;
+    P.tiles_c = (g.C + kPrepTCols - 1) / kPrepTCols;
     P.beta = hp.beta;
     P.omb = 1.f - hp.beta;
     P.X = j.ws + g.off_x0;
@@ -327,7 +330,8 @@ int muon_prep(const MuonJob& j, cudaStream_t s, int max_blocks, bool side, int* 
     int st = cuda_status(launch_muon_prep(P, max_blocks, s));
     prof_end(pr, s, 0.0, elems * ((j.gdt == MA_BF16 ? 2 : 4) + 8 + (hp.precision ? 4 : 2)));
     if (st) return st;
-    pr = prof_begin(MA_PROF_FINALIZE, s);
+    // on the side stream the finalize shares the SMs with the chain before it, like the pass
+    pr = prof_begin(side ? MA_PROF_MOMENTUM_SIDE : MA_PROF_FINALIZE, s);
     st = cuda_status(launch_norm_finalize(part, g.parts, (int)g.units, hp.eps, scale, s));
     prof_end(pr, s, 0.0, (double)g.units * g.parts * 8.0 + g.units * 4.0);
     if (st) return st;
@@ -970,12 +974,11 @@ int run_adamw_segment(ma_plan* plan, const ma_group_t* groups, cudaStream_t s, i
 }
 
 // Whether a segment's momentum passes may run on the side stream under the
-// Newton-Schulz chain of the segment before it: every unit flat (the flat
-// momentum kernel fits beside a Newton-Schulz CTA on an SM; the transposing
-// one needs a shared-memory tile that does not) and bf16 operands.
+// Newton-Schulz chain of the segment before it: bf16 operands (both momentum
+// kernels then fit beside a Newton-Schulz CTA on an SM).
 bool side_prep_ok(const SegJobs& sj) {
     for (const MuonJob& j : sj.jobs)
-        if (j.g.total > 0 && (j.g.transposed || j.hp->precision)) return false;
+        if (j.g.total > 0 && j.hp->precision) return false;
     return true;
 }
 
@@ -1627,21 +1630,24 @@ int ma_plan_create(const ma_tensor_t* t, int n, const ma_group_t* groups, int ng
         *nseg = muon_segments;
         return MA_OK;
     };
-    // A step with two or more Muon segments gets a workspace of two halves,
-    // so that one segment's momentum pass can run under the chain of the one
-    // before it: without a cap, halves of at most kSubBatchBytes (the
-    // sub-batch budget) each; with a cap, halves of at most half the cap when
-    // every bucket fits in that, else one workspace of at most the cap.
+    // With momentum overlap on, a step with two or more Muon segments gets a
+    // workspace of two halves, so that one segment's momentum pass can run
+    // under the chain of the one before it: without a cap, halves of at most
+    // kSubBatchBytes (the sub-batch budget) each; with a cap, halves of at
+    // most half the cap when every bucket fits in that, else one workspace of
+    // at most the cap. Otherwise one workspace, sub-batches within
+    // kSubBatchBytes or the cap.
+    const bool halves = g_momentum_overlap.load(std::memory_order_relaxed) != 0;
     size_t need = 0;
     int nseg = 0;
     if (cap == 0) {
         if ((st = size_plan(kSubBatchBytes, 0, &need, &nseg))) return fail(st);
-    } else if (size_plan(cap / 2, cap / 2, &need, &nseg) != MA_OK || nseg < 2) {
+    } else if (!halves || size_plan(cap / 2, cap / 2, &need, &nseg) != MA_OK || nseg < 2) {
         if ((st = size_plan(cap, cap, &need, &nseg))) return fail(st);
         nseg = 0;  // no halves: one workspace within the cap
     }
     plan->ws_bytes = need;
-    if (nseg >= 2 && need > 0) {
+    if (halves && nseg >= 2 && need > 0) {
         plan->region = align_up(need, kAlign);
         plan->ws_bytes = 2 * plan->region;
     }
@@ -2021,6 +2027,12 @@ int ma_device_status_async(int32_t* host_dst, void* stream) {
 int ma_set_wait_limit_ns(int64_t limit_ns) {
     if (limit_ns <= 0) return MA_ERR_ARG;
     g_host_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
+    return MA_OK;
+}
+
+int ma_set_momentum_overlap(int on) {
+    if (on != 0 && on != 1) return MA_ERR_ARG;
+    g_momentum_overlap.store(on, std::memory_order_relaxed);
     return MA_OK;
 }
 

@@ -92,7 +92,8 @@ const void* adamw_kernel_func();  // the kernel's host-side handle (CUDA-graph n
 
 constexpr int kPrepChunk = 8192;      // elements per chunk (one partial sum each), flat path
 constexpr int kPrepSideThreads = 128;  // threads per block of the side-stream flat kernel
-constexpr int kPrepTile = 64;      // tile edge, transposing path
+constexpr int kPrepTRows = 32;        // transposing path: rows of u per warp block
+constexpr int kPrepTCols = 128;       // transposing path: columns of u per thread block (four warps)
 
 struct MuonPrepLaunch {
     int32_t batch, heads, transposed, gdt, nesterov, x_f32;
@@ -100,7 +101,7 @@ struct MuonPrepLaunch {
     int64_t ldx;          // row stride (elements) of the NS operand X
     int64_t x_unit;       // elements between consecutive units of X
     int64_t parts;        // partial sums per unit
-    int64_t tiles_c;      // transposing path: tiles along C
+    int64_t tiles_c;      // transposing path: blocks of kPrepTCols columns along C
     float beta, omb;
     void* X;
     double* partials;
@@ -111,10 +112,9 @@ struct MuonPrepLaunch {
 // Number of per-block partial sums the momentum pass writes for one unit.
 int64_t prep_parts_per_unit(int64_t Rh, int64_t C, int transposed);
 
-// max_blocks > 0: the flat path runs its side-stream kernel on at most that
-// many blocks (a small grid that runs beside the Newton-Schulz kernels of
-// another batch, with the same partial sums); 0: one block per chunk. The
-// transposing path ignores it.
+// max_blocks > 0: at most that many blocks (a small grid that runs beside the
+// Newton-Schulz kernels of another batch, with the same partial sums; the
+// flat path then takes its side-stream kernel); 0: one block per chunk.
 cudaError_t launch_muon_prep(const MuonPrepLaunch& L, int max_blocks, cudaStream_t s);
 // Per-device kernel attributes of the momentum kernels, ahead of a stream capture.
 cudaError_t prep_setup();

@@ -207,106 +207,100 @@ __global__ void __launch_bounds__(kPrepSideThreads, 6) prep_flat_side_kernel(con
     }
 }
 
-// Transposing path (tall units, X = u^T). A 64 x 64 tile: each thread reads
-// four 4-wide vectors along a row of u (a warp covers two 256-byte row
-// segments), the tile turns in shared memory, and each row of X gets 64
-// consecutive values (128 bytes of bf16) written as 16-byte vectors.
+// Transposing path (tall units, X = u^T), without shared memory: each warp
+// takes a 32-row x 32-column block of u, lane l owning column c0 + l. Row by
+// row the warp reads 32 consecutive gradients and momenta (64- and 128-byte
+// segments), updates the momentum in place and keeps the direction in a
+// register, so that after the 32 rows lane l holds 32 consecutive elements of
+// row c0 + l of X, which it writes as 16-byte vectors. A block is four warps
+// side by side (32 x 128 of u); its partial is the warps' sums in order, each
+// a butterfly over lanes that added their 32 values in row order. Blocks walk
+// the (unit, block) pairs grid-stride: one block per pair on the caller's
+// stream, or a small grid on a side stream, where a block (at most 64
+// registers a thread, 16 bytes of shared memory) fits beside a Newton-Schulz
+// CTA. The partials do not depend on the grid.
 template <bool GBF16, bool XF32>
-__global__ void __launch_bounds__(256) prep_transpose_kernel(const __grid_constant__ MuonPrepLaunch L) {
+__global__ void __launch_bounds__(kPrepSideThreads, 8) prep_transpose_kernel(const __grid_constant__ MuonPrepLaunch L) {
     griddep_launch_dependents();
     griddep_wait();
-    __shared__ float tile[kPrepTile][kPrepTile + 1];  // [column of u][row of u]
-    __shared__ float red[8];
-    const int u = blockIdx.y;
-    const int b = u / L.heads, h = u % L.heads;
-    const int64_t off = (int64_t)h * L.Rh * L.C;
-    const int64_t tr = blockIdx.x / L.tiles_c, tc = blockIdx.x % L.tiles_c;
-    const int64_t r0 = tr * kPrepTile, c0 = tc * kPrepTile;
-    const int t = threadIdx.x;
-    float* M = L.M[b] + off;
+    __shared__ float red[kPrepSideThreads / 32];
+    const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t items = (int64_t)L.batch * L.heads * L.parts;
     const float beta = L.beta, omb = L.omb;
     const bool nest = L.nesterov != 0;
-    float ss = 0.f;
-    {
-        const int cl = (t & 15) * 4;  // C % 8 == 0, so a 4-wide vector never straddles the row end
-        const int64_t c = c0 + cl;
-        float g[4][4], m[4][4];
-        bool in[4];
+    for (int64_t it = blockIdx.x; it < items; it += gridDim.x) {
+        const int u = (int)(it / L.parts);
+        const int64_t part = it - (int64_t)u * L.parts;
+        const int b = u / L.heads, h = u % L.heads;
+        const int64_t off = (int64_t)h * L.Rh * L.C;
+        const int64_t r0 = (part / L.tiles_c) * kPrepTRows;
+        const int64_t c = (part % L.tiles_c) * kPrepTCols + 32 * w + lane;  // this lane's column of u
+        float d[kPrepTRows];
+        float ss = 0.f;
+        const bool col_ok = c < L.C;
+        const int rows = col_ok ? (int)min((int64_t)kPrepTRows, L.Rh - r0) : 0;  // rows of this block in range
+        // running pointers to row r0 + i, column c, of the momentum and the gradient
+        float* mp = L.M[b] + off + r0 * L.C + c;
+        const float* gpf = reinterpret_cast<const float*>(L.G[b]) + off + r0 * L.C + c;
+        const unsigned short* gph = reinterpret_cast<const unsigned short*>(L.G[b]) + off + r0 * L.C + c;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int rl = (t >> 4) + 16 * k;
-            const int64_t r = r0 + rl;
-            in[k] = (r < L.Rh) && (c < L.C);
-            if (in[k]) {
-                const int64_t idx = r * L.C + c;
-                if (GBF16) {
-                    const uint2 w = __ldcs(reinterpret_cast<const uint2*>(reinterpret_cast<const uint16_t*>(L.G[b]) +
-                                                                          off + idx));
-                    g[k][0] = bf16_lo(w.x); g[k][1] = bf16_hi(w.x); g[k][2] = bf16_lo(w.y); g[k][3] = bf16_hi(w.y);
-                } else {
-                    const float4 w =
-                        __ldcs(reinterpret_cast<const float4*>(reinterpret_cast<const float*>(L.G[b]) + off + idx));
-                    g[k][0] = w.x; g[k][1] = w.y; g[k][2] = w.z; g[k][3] = w.w;
+        for (int i0 = 0; i0 < kPrepTRows; i0 += 4) {
+            float g[4], m[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {  // four rows' loads in flight before any arithmetic
+                const int64_t o = (int64_t)(i0 + i) * L.C;
+                g[i] = 0.f;
+                m[i] = 0.f;
+                if (i0 + i < rows) {
+                    g[i] = GBF16 ? __uint_as_float((uint32_t)__ldcs(gph + o) << 16) : __ldcs(gpf + o);
+                    m[i] = __ldcs(mp + o);
                 }
-                const float4 mv = __ldcs(reinterpret_cast<const float4*>(M + idx));
-                m[k][0] = mv.x; m[k][1] = mv.y; m[k][2] = mv.z; m[k][3] = mv.w;
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int rl = (t >> 4) + 16 * k;
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-            if (in[k]) {
-                const int64_t idx = (r0 + rl) * L.C + c;
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    m[k][j] = beta * m[k][j] + omb * g[k][j];
-                    d[j] = nest ? beta * m[k][j] + omb * g[k][j] : m[k][j];
-                    ss += d[j] * d[j];
-                }
-                __stcs(reinterpret_cast<float4*>(M + idx), make_float4(m[k][0], m[k][1], m[k][2], m[k][3]));
             }
 #pragma unroll
-            for (int j = 0; j < 4; ++j) tile[cl + j][rl] = d[j];
+            for (int i = 0; i < 4; ++i) {
+                d[i0 + i] = 0.f;
+                if (i0 + i < rows) {
+                    const float mn = beta * m[i] + omb * g[i];
+                    const float di = nest ? beta * mn + omb * g[i] : mn;
+                    __stcs(mp + (int64_t)(i0 + i) * L.C, mn);
+                    d[i0 + i] = di;
+                    ss += di * di;
+                }
+            }
         }
-    }
-    __syncthreads();
-    {
-        const int xr_l = t >> 2;         // row of X within the tile (a column of u)
-        const int seg = (t & 3) * 16;    // 16 consecutive values of that row
-        const int64_t xr = c0 + xr_l, xc = r0 + seg;
-        if (xr < L.C) {
-            float d[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j) d[j] = tile[xr_l][seg + j];
-            const int64_t xi = (int64_t)u * L.x_unit + xr * L.ldx + xc;
-            if (xc + 16 <= L.Rh) {
+        // row c of X, elements r0 .. r0 + 31
+        if (col_ok) {
+            const int64_t xi = (int64_t)u * L.x_unit + c * L.ldx + r0;
+            if (r0 + kPrepTRows <= L.Rh) {
                 if (XF32) {
                     float4* xp = reinterpret_cast<float4*>(reinterpret_cast<float*>(L.X) + xi);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) __stcs(xp + q, make_float4(d[4 * q], d[4 * q + 1], d[4 * q + 2], d[4 * q + 3]));
+                    for (int q = 0; q < 8; ++q) __stcs(xp + q, make_float4(d[4 * q], d[4 * q + 1], d[4 * q + 2], d[4 * q + 3]));
                 } else {
                     uint4* xp = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(L.X) + xi);
 #pragma unroll
-                    for (int q = 0; q < 2; ++q) {
-                        uint4 w;
-                        w.x = pack_bf16x2(d[8 * q + 0], d[8 * q + 1]);
-                        w.y = pack_bf16x2(d[8 * q + 2], d[8 * q + 3]);
-                        w.z = pack_bf16x2(d[8 * q + 4], d[8 * q + 5]);
-                        w.w = pack_bf16x2(d[8 * q + 6], d[8 * q + 7]);
-                        __stcs(xp + q, w);
+                    for (int q = 0; q < 4; ++q) {
+                        uint4 v;
+                        v.x = pack_bf16x2(d[8 * q + 0], d[8 * q + 1]);
+                        v.y = pack_bf16x2(d[8 * q + 2], d[8 * q + 3]);
+                        v.z = pack_bf16x2(d[8 * q + 4], d[8 * q + 5]);
+                        v.w = pack_bf16x2(d[8 * q + 6], d[8 * q + 7]);
+                        __stcs(xp + q, v);
                     }
                 }
             } else {
-                for (int j = 0; j < 16 && xc + j < L.Rh; ++j) {
-                    if (XF32) reinterpret_cast<float*>(L.X)[xi + j] = d[j];
-                    else reinterpret_cast<__nv_bfloat16*>(L.X)[xi + j] = __float2bfloat16_rn(d[j]);
+#pragma unroll
+                for (int i = 0; i < kPrepTRows; ++i) {
+                    if (r0 + i < L.Rh) {
+                        if (XF32) reinterpret_cast<float*>(L.X)[xi + i] = d[i];
+                        else reinterpret_cast<__nv_bfloat16*>(L.X)[xi + i] = __float2bfloat16_rn(d[i]);
+                    }
                 }
             }
         }
+        const float tot = block_sum<kPrepSideThreads>(ss, red);
+        if (threadIdx.x == 0) L.partials[(int64_t)u * L.parts + part] = (double)tot;
     }
-    const float tot = block_sum<256>(ss, red);
-    if (threadIdx.x == 0) L.partials[(int64_t)u * L.parts + blockIdx.x] = (double)tot;
 }
 
 // One warp per unit: lane-strided sum of the unit's partials, then a fixed
@@ -328,13 +322,13 @@ __global__ void __launch_bounds__(256) norm_finalize_kernel(const double* __rest
 }  // namespace
 
 int64_t prep_parts_per_unit(int64_t Rh, int64_t C, int transposed) {
-    if (transposed) return ((Rh + kPrepTile - 1) / kPrepTile) * ((C + kPrepTile - 1) / kPrepTile);
+    if (transposed) return ((Rh + kPrepTRows - 1) / kPrepTRows) * ((C + kPrepTCols - 1) / kPrepTCols);
     return (Rh * C + kPrepChunk - 1) / kPrepChunk;
 }
 
-// The side-stream flat kernels prefer the largest shared-memory carveout,
-// the one a Newton-Schulz CTA sets on its SM, so that their blocks can join
-// that SM.
+// The kernels that run beside Newton-Schulz CTAs prefer the largest
+// shared-memory carveout, the one those CTAs set on their SMs, so that their
+// blocks can join those SMs.
 // Once per device; the attribute is set before any stream capture by the
 // library's set-up (the first call on a device).
 cudaError_t prep_setup() {
@@ -344,10 +338,14 @@ cudaError_t prep_setup() {
     if (e != cudaSuccess) return e;
     int done = 0;
     return cache.get(dev, &done, [](int* v) -> cudaError_t {
-        const void* fns[4] = {reinterpret_cast<const void*>(prep_flat_side_kernel<true, false>),
+        const void* fns[8] = {reinterpret_cast<const void*>(prep_flat_side_kernel<true, false>),
                               reinterpret_cast<const void*>(prep_flat_side_kernel<true, true>),
                               reinterpret_cast<const void*>(prep_flat_side_kernel<false, false>),
-                              reinterpret_cast<const void*>(prep_flat_side_kernel<false, true>)};
+                              reinterpret_cast<const void*>(prep_flat_side_kernel<false, true>),
+                              reinterpret_cast<const void*>(prep_transpose_kernel<true, false>),
+                              reinterpret_cast<const void*>(prep_transpose_kernel<true, true>),
+                              reinterpret_cast<const void*>(prep_transpose_kernel<false, false>),
+                              reinterpret_cast<const void*>(prep_transpose_kernel<false, true>)};
         for (const void* f : fns) {
             const cudaError_t r = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
                                                        cudaSharedmemCarveoutMaxShared);
@@ -364,11 +362,15 @@ cudaError_t launch_muon_prep(const MuonPrepLaunch& L, int max_blocks, cudaStream
     const bool gb = L.gdt == MA_BF16, xf = L.x_f32 != 0;
     cudaError_t e;
     if (L.transposed) {
-        const dim3 grid((unsigned)L.parts, (unsigned)units);
-        if (gb && !xf) e = launch_pdl(prep_transpose_kernel<true, false>, grid, dim3(256), 0, s, L);
-        else if (gb) e = launch_pdl(prep_transpose_kernel<true, true>, grid, dim3(256), 0, s, L);
-        else if (!xf) e = launch_pdl(prep_transpose_kernel<false, false>, grid, dim3(256), 0, s, L);
-        else e = launch_pdl(prep_transpose_kernel<false, true>, grid, dim3(256), 0, s, L);
+        if ((e = prep_setup()) != cudaSuccess) return e;
+        int64_t items = (int64_t)units * L.parts;
+        if (max_blocks > 0 && items > max_blocks) items = max_blocks;
+        if (items > INT32_MAX) items = INT32_MAX;
+        const dim3 grid((unsigned)items), block(kPrepSideThreads);
+        if (gb && !xf) e = launch_pdl(prep_transpose_kernel<true, false>, grid, block, 0, s, L);
+        else if (gb) e = launch_pdl(prep_transpose_kernel<true, true>, grid, block, 0, s, L);
+        else if (!xf) e = launch_pdl(prep_transpose_kernel<false, false>, grid, block, 0, s, L);
+        else e = launch_pdl(prep_transpose_kernel<false, true>, grid, block, 0, s, L);
     } else if (max_blocks <= 0) {
         const dim3 grid((unsigned)L.parts, (unsigned)units);
         if (gb && !xf) e = launch_pdl(prep_flat_kernel<true, false>, grid, dim3(256), 0, s, L);

@@ -53,8 +53,7 @@ UNIT = "params/s"
 # Sources of the Newton-Schulz kernel: a DRAM-traffic record (ncu's
 # dram__bytes_read.sum + dram__bytes_write.sum per launch) applies only to the
 # kernel built from exactly these files.
-NS_KERNEL_SOURCES = ("adamw_hybrid_optimizer_muon_b200/csrc/ns_tc.cu", "adamw_hybrid_optimizer_muon_b200/csrc/common.cuh",
-                     "adamw_hybrid_optimizer_muon_b200/csrc/internal.h")
+NS_KERNEL_SOURCES = ("adamw_hybrid_optimizer_muon_b200/csrc/ns_tc.cu", "adamw_hybrid_optimizer_muon_b200/csrc/common.cuh")
 NS_TRAFFIC_RECORD = os.path.join("profiles", "ns_tc_kernel_traffic.json")
 
 
@@ -82,6 +81,68 @@ def ns_traffic(workload, ns_launches_per_step):
     if not w or w.get("ns_launches_per_step") != ns_launches_per_step:
         return None
     return float(w["bytes_per_launch"])
+
+
+def _ncu_ns_launch_bytes(csv_path):
+    """DRAM bytes (read + write) of each ns_tc_kernel launch in an ncu --csv
+    launch list taken with --metrics dram__bytes_read.sum,dram__bytes_write.sum."""
+    import csv
+    scale = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "Tbyte": 1e12}
+    with open(csv_path) as f:
+        lines = [ln for ln in f if ln.startswith('"')]
+    per = {}
+    for r in csv.DictReader(lines):
+        if "ns_tc_kernel" not in r["Kernel Name"]:
+            continue
+        if r["Metric Name"] in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+            v = float(r["Metric Value"].replace(",", "")) * scale[r["Metric Unit"]]
+            per[int(r["ID"])] = per.get(int(r["ID"]), 0.0) + v
+    return [per[k] for k in sorted(per)]
+
+
+def write_traffic_record(square_csv, rect_csv, bench_7b_log):
+    """Write the DRAM-traffic record for the current kernel sources from ncu
+    launch lists of one step of the square8 and rect8 workloads (every
+    ns_tc_kernel launch of the step) and a bench.py line of the 7b workload
+    (for its Newton-Schulz launches per step). The 7b figure scales the two
+    8-matrix chains' traffic per unit to the 7b step's units: square units
+    take the 4096 x 4096 chain, the 4096 x 11008 and 11008 x 4096 units the
+    rectangular one (their chains differ only in the transposition of the
+    momentum pass and of the final store)."""
+    sq, rc = _ncu_ns_launch_bytes(square_csv), _ncu_ns_launch_bytes(rect_csv)
+    n_sq = len(synth.WORKLOADS["square8"]().tensors)
+    n_rc = len(synth.WORKLOADS["rect8"]().tensors)
+    units = {}
+    for t in synth.WORKLOADS["7b"]().tensors:
+        if t.role == synth.ROLE_HIDDEN and len(t.shape) == 2:
+            units[tuple(sorted(t.shape))] = units.get(tuple(sorted(t.shape)), 0) + 1
+    u_sq, u_rc = units.get((4096, 4096), 0), units.get((4096, 11008), 0)
+    if set(units) - {(4096, 4096), (4096, 11008)}:
+        raise SystemExit(f"7b hidden matrices of shapes this record does not cover: {sorted(units)}")
+    with open(bench_7b_log) as f:
+        line = json.loads([ln for ln in f if ln.startswith("{")][-1])
+    if not line["config"]["workload"].startswith("7b"):
+        raise SystemExit("the bench line is not the 7b workload's")
+    n7 = int(round(sum(line["kernels"][c]["launches_per_step"]
+                       for c in ("ns_gram", "ns_apply", "ns_gramsq", "ns_final") if c in line["kernels"])))
+    step_7b = u_sq * sum(sq) / n_sq + u_rc * sum(rc) / n_rc
+    rec = {
+        "kernel_sha16": ns_kernel_sha16(),
+        "source": "ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum (one pass), "
+                  "every ns_tc_kernel launch of one step of bench.py --workload square8 and --workload rect8",
+        "workloads": {
+            "square8": {"bytes_per_launch": sum(sq) / len(sq), "ns_launches_per_step": len(sq)},
+            "rect8": {"bytes_per_launch": sum(rc) / len(rc), "ns_launches_per_step": len(rc)},
+            "7b": {"bytes_per_launch": step_7b / n7, "ns_launches_per_step": n7,
+                   "derivation": f"per-unit traffic of the 8-matrix chains scaled to the 7B step's units: "
+                                 f"{u_sq} x (4096 x 4096 chain) + {u_rc} x (4096 x 11008 chain, wide and tall "
+                                 f"alike), over its {n7} Newton-Schulz launches"},
+        },
+    }
+    with open(os.path.join(ROOT, NS_TRAFFIC_RECORD), "w") as f:
+        json.dump(rec, f, indent=1)
+    print(json.dumps({"square8_per_launch": sq, "rect8_per_launch": rc, "7b_step_bytes": step_7b,
+                      "7b_ns_launches": n7}))
 
 
 def env_int(name, default):
@@ -326,7 +387,15 @@ def main():
                          "each rank's share of the update, all-gather of the parameters) instead of N replicas")
     ap.add_argument("--coeffs", default=None,
                     help="Newton-Schulz polynomial per iteration, 'a,b,c[;a,b,c...]' (default: the cubic 1.5,-0.5,0)")
+    ap.add_argument("--momentum-overlap", action="store_true",
+                    help="run each Muon sub-batch's momentum pass on a side stream under the previous sub-batch's "
+                         "Newton-Schulz chain (ma_set_momentum_overlap; off by default, slower on a B200)")
+    ap.add_argument("--write-traffic-record", nargs=3, metavar=("SQUARE8_CSV", "RECT8_CSV", "BENCH_7B_LOG"),
+                    default=None, help="host only: write the Newton-Schulz DRAM-traffic record for the current "
+                                       "kernel sources from ncu launch lists and a 7b bench line, then exit")
     args = ap.parse_args()
+    if args.write_traffic_record:
+        return write_traffic_record(*args.write_traffic_record)
     rank, world, local = env_int("RANK", 0), env_int("WORLD_SIZE", 1), env_int("LOCAL_RANK", 0)
     if args.impl == "reference":
         return run_reference(args, rank, world)
@@ -371,6 +440,7 @@ def main():
             h = g.adamw
             groups.append(("adamw", ma.adamw_hparams(h.lr, h.beta1, h.beta2, h.eps, h.weight_decay, 1)))
     table = [(p, t.role, t.group) for p, t in zip(params, wl.tensors)]
+    ma.ma_set_momentum_overlap(args.momentum_overlap)  # read when the plans are made
     if args.sharded:
         from adamw_hybrid_optimizer_muon_b200.dist import DistMuonAdamW
         gdts = {g.dtype for g in grads}
@@ -571,10 +641,13 @@ def main():
                 d["gbs"] = pc["bytes"] / (pc["ms"] / 1000.0) / 1e9
                 d["frac_hbm"] = d["gbs"] / peaks["hbm_gbs"]
             if c == "momentum_side":
-                d["note"] = ("momentum passes run on a side stream, one block per SM beside the Newton-Schulz "
-                             "CTAs of the previous sub-batch: their time is hidden, not a bandwidth target")
+                d["note"] = ("momentum passes and their norm finalizes run on a side stream, one block per SM "
+                             "beside the Newton-Schulz CTAs of the previous sub-batch: their time is hidden, "
+                             "not a bandwidth target")
             kernels[c] = d
         config = workload_config(wl, world)
+        if args.momentum_overlap:
+            config["momentum_overlap"] = "momentum passes on a side stream under the previous sub-batch's chain"
         if args.sharded:
             config["parallelism"] = (f"sharded dp{world}: reduce-scatter, each rank's share of the update, "
                                      f"all-gather ({len(opt.buckets)} buckets)")

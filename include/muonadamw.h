@@ -372,8 +372,9 @@ void ma_plan_destroy(ma_plan_t* plan);
 #define MA_PROF_NS_GRAMSQ 5     /* symmetric m x m products: A^2 (c != 0), and */
                                 /* the Gram-space chain's Q, A P and P A P     */
 #define MA_PROF_NS_FINAL 6      /* last apply, fused with decay and W update   */
-#define MA_PROF_MOMENTUM_SIDE 7 /* momentum pass run under the Newton-Schulz   */
-                                /* chain of the batch before it (side stream)  */
+#define MA_PROF_MOMENTUM_SIDE 7 /* momentum pass and norm finalize run under   */
+                                /* the Newton-Schulz chain of the batch before */
+                                /* it (side stream)                            */
 #define MA_PROF_CLASSES 8
 
 /* When on != 0, every kernel the library launches on this thread's current
@@ -415,6 +416,19 @@ int ma_device_status_async(int32_t* host_dst, void* stream);
 /* Set the limit, in nanoseconds, of every device-side bounded wait (default
  * 2e9). Takes effect for launches issued after the call. */
 int ma_set_wait_limit_ns(int64_t limit_ns);
+
+/* Momentum overlap for plans created after the call (on: 1, off: 0, the
+ * default; MA_ERR_ARG otherwise). A plan created with it on, whose step has
+ * two or more Muon sub-batches, takes a workspace of two halves used by the
+ * sub-batches in turn, and runs each sub-batch's momentum pass and norm
+ * finalize on a low-priority stream of its own while the Newton-Schulz chain
+ * of the sub-batch before it runs (a cap then bounds the two halves
+ * together). Results are bit-identical either way. It is off by default
+ * because it is slower on a B200: the side kernels' blocks share SMs with the
+ * persistent Newton-Schulz CTA pairs, each pair walks a fixed share of the
+ * tiles, and every launch then ends with its slowest pair; on the 7B-shaped
+ * set the step took 270 ms with it and 251.5 ms without on the same GPU. */
+int ma_set_momentum_overlap(int on);
 
 /* Self-test of the bounded wait: launch one block that waits on a barrier
  * phase that nothing completes, with a wait limit of limit_ns. The kernel

@@ -215,25 +215,40 @@ def test_plan_sizing_on_host():
     assert (sub(128, 4096, 4096), sub(64, 4096, 11008), sub(32, 11008, 4096)) == (32, 16, 16)
     expect = max(ma.muon_workspace_bytes(32, 4096, 4096, hp), ma.muon_workspace_bytes(16, 4096, 11008, hp),
                  ma.muon_workspace_bytes(16, 11008, 4096, hp))
-    # ten Muon sub-batches: two halves, so that each sub-batch's momentum pass
-    # can run under the chain of the one before it
-    assert ws == 2 * ((expect + 255) // 256 * 256)
+    # one workspace for the largest sub-batch, used by the sub-batches in turn
+    assert ws == expect
     ma.ma_plan_destroy(plan)
-    # a cap splits buckets into sub-batches, and the two halves fit in it
-    plan, ws2 = ma.ma_plan_create(descs, _groups_for(wl), ws_cap=4 << 30)
-    assert 0 < ws2 <= 4 << 30
-    ma.ma_plan_destroy(plan)
-    plan, ws3 = ma.ma_plan_create(descs, _groups_for(wl), ws_cap=2 * ((expect + 255) // 256 * 256))
-    assert ws3 == 2 * ((expect + 255) // 256 * 256)
-    ma.ma_plan_destroy(plan)
-    # a cap below two halves of the largest single matrix: one workspace
-    one = max(ma.muon_workspace_bytes(1, 4096, 11008, hp), ma.muon_workspace_bytes(1, 11008, 4096, hp))
-    plan, ws4 = ma.ma_plan_create(descs, _groups_for(wl), ws_cap=one + 4096)
-    assert ws4 <= one + 4096
+    # a cap splits buckets into sub-batches that fit in it
+    plan, ws2 = ma.ma_plan_create(descs, _groups_for(wl), ws_cap=1 << 30)
+    assert 0 < ws2 <= 1 << 30
     ma.ma_plan_destroy(plan)
     with pytest.raises(ma.MAError) as e:
         ma.ma_plan_create(descs, _groups_for(wl), ws_cap=1 << 20)
     assert e.value.code == ma.MA_ERR_WORKSPACE
+    # momentum overlap: ten Muon sub-batches get two halves, so that each
+    # sub-batch's momentum pass can run under the chain of the one before it
+    ma.ma_set_momentum_overlap(True)
+    try:
+        plan, ws = ma.ma_plan_create(descs, _groups_for(wl))
+        assert ws == 2 * ((expect + 255) // 256 * 256)
+        ma.ma_plan_destroy(plan)
+        # a cap bounds the two halves together
+        plan, ws2 = ma.ma_plan_create(descs, _groups_for(wl), ws_cap=4 << 30)
+        assert 0 < ws2 <= 4 << 30
+        ma.ma_plan_destroy(plan)
+        plan, ws3 = ma.ma_plan_create(descs, _groups_for(wl), ws_cap=2 * ((expect + 255) // 256 * 256))
+        assert ws3 == 2 * ((expect + 255) // 256 * 256)
+        ma.ma_plan_destroy(plan)
+        # a cap below two halves of the largest single matrix: one workspace
+        one = max(ma.muon_workspace_bytes(1, 4096, 11008, hp), ma.muon_workspace_bytes(1, 11008, 4096, hp))
+        plan, ws4 = ma.ma_plan_create(descs, _groups_for(wl), ws_cap=one + 4096)
+        assert ws4 <= one + 4096
+        ma.ma_plan_destroy(plan)
+    finally:
+        ma.ma_set_momentum_overlap(False)
+    with pytest.raises(ma.MAError) as e:
+        ma._check(ma.lib().ma_set_momentum_overlap(2), "ma_set_momentum_overlap")
+    assert e.value.code == ma.MA_ERR_ARG
 
 
 def _fake_descs(wl):
@@ -251,13 +266,21 @@ def test_plan_describe():
     plan, ws = ma.ma_plan_create(_fake_descs(wl), _groups_for(wl))
     text = ma.ma_plan_describe(plan, _groups_for(wl))
     ma.ma_plan_destroy(plan)
-    assert text.startswith(f"workspace {ws} bytes in two halves of {ws // 2} (momentum passes under the previous "
-                           f"chain); AdamW: 67 tensors, ")
+    assert text.startswith(f"workspace {ws} bytes; AdamW: 67 tensors, ")
     assert "4096 x 4096, 128 matrices (bf16 grads), heads 1, sub-batches of 32, direct chain" in text
     assert "4096 x 11008, 64 matrices (bf16 grads), heads 1, sub-batches of 16, Gram-space chain" in text
     assert "11008 x 4096, 32 matrices (bf16 grads), heads 1, sub-batches of 16, Gram-space chain" in text
     segs = [ln for ln in text.splitlines() if ln.startswith("segment")]
     assert segs[0] == "segment 0: AdamW" and len(segs) == 1 + 4 + 4 + 2  # no sharing at this size
+    ma.ma_set_momentum_overlap(True)
+    try:
+        plan, ws = ma.ma_plan_create(_fake_descs(wl), _groups_for(wl))
+        text = ma.ma_plan_describe(plan, _groups_for(wl))
+        ma.ma_plan_destroy(plan)
+    finally:
+        ma.ma_set_momentum_overlap(False)
+    assert text.startswith(f"workspace {ws} bytes in two halves of {ws // 2} (momentum passes under the previous "
+                           f"chain); AdamW: 67 tensors, ")
     # the d20 set: its three buckets share one chain of Newton-Schulz launches
     wl = synth.d20()
     plan, _ = ma.ma_plan_create(_fake_descs(wl), _groups_for(wl))

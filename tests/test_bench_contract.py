@@ -89,3 +89,55 @@ def test_gpu_arm_line_sharded():
     e = d["e2e"]
     assert e["value"] > 0 and e["h2d_bytes_per_step"] > 0 and e["d2h_bytes_per_step"] == 4
     assert d["roofline"]["achieved"] > 0
+
+
+def _ncu_csv(path, launches):
+    # an ncu --csv launch list: preamble lines, a header, one row per launch and metric
+    head = ('"ID","Process ID","Process Name","Host Name","Kernel Name","Context","Stream","Block Size",'
+            '"Grid Size","Device","CC","Section Name","Metric Name","Metric Unit","Metric Value"\n')
+    with open(path, "w") as f:
+        f.write("==PROF== Connected to process 1 (python)\n" + head)
+        for i, (kern, rd, wr, unit) in enumerate(launches):
+            for name, v in (("dram__bytes_read.sum", rd), ("dram__bytes_write.sum", wr),
+                            ("gpu__time_duration.sum", "1,000")):
+                u = "nsecond" if name.startswith("gpu__") else unit
+                f.write(f'"{i}","1","python","h","{kern}","1","7","(320, 1, 1)","(148, 1, 1)","0","10.0",'
+                        f'"Command line profiler metrics","{name}","{u}","{v}"\n')
+
+
+def test_traffic_record_writer_scales_captures_to_the_7b_step(tmp_path, monkeypatch):
+    sys.path.insert(0, ROOT)
+    import bench
+    import synth
+    sq = tmp_path / "sq.csv"
+    rc = tmp_path / "rc.csv"
+    # square8: two Newton-Schulz launches (MB units) and a launch of another kernel that must be ignored
+    _ncu_csv(sq, [("void ns_tc_kernel<0, 1>(NsLaunch)", "300", "100", "Mbyte"),
+                  ("void adamw_kernel(Args)", "999", "999", "Mbyte"),
+                  ("void ns_tc_kernel<3, 1>(NsLaunch)", "1,200,000,000", "400,000,000", "byte")])
+    # rect8: three launches
+    _ncu_csv(rc, [("void ns_tc_kernel<0, 1>(NsLaunch)", "1.5", "0.5", "Gbyte")] * 3)
+    log = tmp_path / "b.log"
+    line = {"config": {"workload": "7b: 32 layers"},
+            "kernels": {"ns_gram": {"launches_per_step": 26.0}, "ns_final": {"launches_per_step": 10.0},
+                        "momentum": {"launches_per_step": 3.0}}}
+    log.write_text("noise\n" + json.dumps(line) + "\n")
+    rec_path = tmp_path / "rec.json"
+    monkeypatch.setattr(bench, "NS_TRAFFIC_RECORD", str(rec_path))
+    bench.write_traffic_record(str(sq), str(rc), str(log))
+    rec = json.loads(rec_path.read_text())
+    w = rec["workloads"]
+    assert w["square8"] == {"bytes_per_launch": (4e8 + 1.6e9) / 2, "ns_launches_per_step": 2}
+    assert w["rect8"] == {"bytes_per_launch": 2e9, "ns_launches_per_step": 3}
+    # 7b: 128 square and 96 rectangular units; each 8-matrix chain's traffic per unit
+    hidden = [t for t in synth.WORKLOADS["7b"]().tensors if t.role == synth.ROLE_HIDDEN and len(t.shape) == 2]
+    assert len(hidden) == 224
+    step = 128 * 2e9 / 8 + 96 * 6e9 / 8
+    assert w["7b"]["ns_launches_per_step"] == 36
+    assert w["7b"]["bytes_per_launch"] == pytest.approx(step / 36, rel=1e-12)
+    # read back while the kernel sources match; not for another launch structure
+    assert bench.ns_traffic("7b", 36) == pytest.approx(step / 36, rel=1e-12)
+    assert bench.ns_traffic("7b", 35) is None
+    rec["kernel_sha16"] = "0" * 16
+    rec_path.write_text(json.dumps(rec))
+    assert bench.ns_traffic("7b", 36) is None

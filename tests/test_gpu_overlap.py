@@ -1,13 +1,14 @@
 """Momentum passes on a side stream, under the Newton-Schulz chain of the
 sub-batch before them, against separate calls, bit for bit.
 
-A plan whose step has several Muon sub-batches splits its workspace in two
-halves. Each sub-batch of wide (flat) matrices then has its momentum pass run
-on the plan's side stream, one block per SM beside the Newton-Schulz CTAs of
-the sub-batch before it, while tall (transposing) sub-batches keep theirs on
-the caller's stream. Every kernel does the same arithmetic as in a call of its
-own, so the parameters and momentum must equal those of one
-muon_step_batched call per matrix, eagerly and replayed from a CUDA graph.
+With momentum overlap on (ma_set_momentum_overlap; off by default), a plan
+whose step has several Muon sub-batches splits its workspace in two halves.
+Each sub-batch then has its momentum pass (flat for wide matrices,
+transposing for tall ones) run on the plan's side stream, one block per SM
+beside the Newton-Schulz CTAs of the sub-batch before it. Every kernel does
+the same arithmetic as in a call of its own, so the parameters and momentum
+must equal those of one muon_step_batched call per matrix, eagerly and
+replayed from a CUDA graph.
 """
 import numpy as np
 import pytest
@@ -36,8 +37,15 @@ def _cap():
     return 2 * max(ma.muon_workspace_bytes(2, 512, 1024, hp), ma.muon_workspace_bytes(2, 1024, 512, hp))
 
 
+@pytest.fixture
+def overlap_on():
+    ma.ma_set_momentum_overlap(True)
+    yield
+    ma.ma_set_momentum_overlap(False)
+
+
 @pytest.mark.parametrize("graph", [False, True])
-def test_side_stream_momentum_matches_separate_calls(graph):
+def test_side_stream_momentum_matches_separate_calls(graph, overlap_on):
     r = np.random.default_rng(41)
     P0 = [(r.standard_normal(s) * 0.02).astype(np.float32) for s, _ in TABLE]
     pa = [dev_f32(p) for p in P0]
