@@ -273,7 +273,8 @@ __device__ __forceinline__ uint32_t sw128w(uint32_t r, uint32_t q) { return r * 
 //
 // For each chunk, the 32 x 32 block of W (in W's own orientation: transposed
 // back when the unit was tall) and the 32 x 32 block of X that the a*X term
-// needs come into shared memory by 16-byte asynchronous copies. The first two
+// needs (none when a = 0) come into shared memory by 16-byte asynchronous
+// copies. The first two
 // chunks of a tile are fetched before the accumulator is ready, and each
 // later chunk while the one before it is being computed, so the DRAM latency
 // of both hides behind the main loop without holding registers. Each lane
@@ -300,6 +301,7 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, Ctl* ctl, int 
         const float decay = p.decay, lrs = p.lr_s;
         const float sa = p.first ? p.scale[tc.u] : 1.f;
         const float ca = sa * p.a;
+        const bool ax = p.a != 0.f;  // a = 0 (the Gram-space chain's X_N = s Q_N X_0): no X block needed
         const int acc = lt & 1;
         const uint32_t use = (uint32_t)(lt >> 1);
         const int row_lo = tc.ti * S::TM + (int)rank * HM + quad * 32;
@@ -327,11 +329,13 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, Ctl* ctl, int 
                 // X rows row_lo.., columns col0..: 8 bf16 per copy; the row stride is a multiple of 8
                 const int col0 = tc.tj * S::TN + (half * CPW + c) * 32;
                 uint8_t* xb = xbuf + (c & 1) * XBUF;
+                if (ax) {
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int row = 8 * i + (lane >> 2), q = lane & 3;
-                    if (row_lo + row < m && col0 + 8 * q < n)
-                        cp_async16(xb + sw64(row, q), Xin + (int64_t)(row_lo + row) * p.ldx + col0 + 8 * q);
+                    for (int i = 0; i < 4; ++i) {
+                        const int row = 8 * i + (lane >> 2), q = lane & 3;
+                        if (row_lo + row < m && col0 + 8 * q < n)
+                            cp_async16(xb + sw64(row, q), Xin + (int64_t)(row_lo + row) * p.ldx + col0 + 8 * q);
+                    }
                 }
             }
             cp_async_commit();  // one group per chunk, empty or not, so the counts line up
@@ -356,15 +360,20 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, Ctl* ctl, int 
             cp_async_wait<1>();
             __syncwarp();
             // X_N row of this lane: s*(a*X + (B X)), s only on the first iteration
+            if (ax) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint4 w = *reinterpret_cast<const uint4*>(xb + sw64(lane, q));
-                const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+                for (int q = 0; q < 4; ++q) {
+                    const uint4 w = *reinterpret_cast<const uint4*>(xb + sw64(lane, q));
+                    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    o[8 * q + 2 * e] = ca * bf16_lo(wv[e]) + sa * o[8 * q + 2 * e];
-                    o[8 * q + 2 * e + 1] = ca * bf16_hi(wv[e]) + sa * o[8 * q + 2 * e + 1];
+                    for (int e = 0; e < 4; ++e) {
+                        o[8 * q + 2 * e] = ca * bf16_lo(wv[e]) + sa * o[8 * q + 2 * e];
+                        o[8 * q + 2 * e + 1] = ca * bf16_hi(wv[e]) + sa * o[8 * q + 2 * e + 1];
+                    }
                 }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) o[e] *= sa;
             }
             if (!p.transposed) {
                 // lane = row of W: 32 consecutive elements
