@@ -424,7 +424,8 @@ def ma_selftest_wait_timeout(limit_ns: int, stream=None) -> None:
     _check(lib().ma_selftest_wait_timeout(int(limit_ns), _stream(stream)), "ma_selftest_wait_timeout")
 
 
-PROF_CLASSES = ("adamw", "momentum", "finalize", "ns_gram", "ns_apply", "ns_gramsq", "ns_final", "momentum_side")
+PROF_CLASSES = ("adamw", "momentum", "finalize", "ns_gram", "ns_apply", "ns_gramsq", "ns_final", "momentum_side",
+                "ns_q1")
 
 
 def ma_profile_enable(on: bool) -> None:

@@ -447,8 +447,10 @@ int chain_gspace(const std::vector<const MuonJob*>& jobs, cudaStream_t s, int sm
     if ((st = launch(NS_GRAM, X0, Acur))) return st;
     for (int i = 0; i < nj; ++i) {
         const MuonGeom& g = jobs[i]->g;
+        const int pr = prof_begin(MA_PROF_NS_Q1, s);
         const cudaError_t e = launch_ns_q1(Acur[i], Qcur[i], (int)g.m, g.ldg, g.m * g.ldg, (int)g.units,
                                            coef(i, 0, 0), coef(i, 0, 1), sms, s);
+        prof_end(pr, s, 0.0, 4.0 * (double)g.units * (double)g.m * (double)g.m);  // A read, Q written (bf16)
         if (e != cudaSuccess) return MA_ERR_CUDA;
         ++*launches;
     }

@@ -92,8 +92,8 @@ const void* adamw_kernel_func();  // the kernel's host-side handle (CUDA-graph n
 
 constexpr int kPrepChunk = 8192;      // elements per chunk (one partial sum each), flat path
 constexpr int kPrepSideThreads = 128;  // threads per block of the side-stream flat kernel
-constexpr int kPrepTRows = 32;        // transposing path: rows of u per warp block
-constexpr int kPrepTCols = 128;       // transposing path: columns of u per thread block (four warps)
+constexpr int kPrepTRows = 64;        // transposing path: rows of u per thread block (16 per warp)
+constexpr int kPrepTCols = 64;        // transposing path: columns of u per thread block (2 per lane)
 
 struct MuonPrepLaunch {
     int32_t batch, heads, transposed, gdt, nesterov, x_f32;

@@ -207,22 +207,28 @@ __global__ void __launch_bounds__(kPrepSideThreads, 6) prep_flat_side_kernel(con
     }
 }
 
-// Transposing path (tall units, X = u^T), without shared memory: each warp
-// takes a 32-row x 32-column block of u, lane l owning column c0 + l. Row by
-// row the warp reads 32 consecutive gradients and momenta (64- and 128-byte
-// segments), updates the momentum in place and keeps the direction in a
-// register, so that after the 32 rows lane l holds 32 consecutive elements of
-// row c0 + l of X, which it writes as 16-byte vectors. A block is four warps
-// side by side (32 x 128 of u); its partial is the warps' sums in order, each
-// a butterfly over lanes that added their 32 values in row order. Blocks walk
-// the (unit, block) pairs grid-stride: one block per pair on the caller's
-// stream, or a small grid on a side stream, where a block (at most 64
-// registers a thread, 16 bytes of shared memory) fits beside a Newton-Schulz
-// CTA. The partials do not depend on the grid.
+// Transposing path (tall units, X = u^T), without shared memory: a block
+// takes a 64-row x 64-column block of u, warp w its rows 16w .. 16w + 15 and
+// lane l columns 2l and 2l + 1. Row by row a warp reads 256 bytes of momentum
+// and 128 of bf16 gradient as 8- and 4-byte vectors, all sixteen rows' loads
+// in flight before any arithmetic (fp32 gradients: two batches of eight);
+// the direction overwrites the momentum in registers once the new momentum
+// has gone out. Lane l then holds 16 consecutive elements of rows c0 + 2l
+// and c0 + 2l + 1 of X: one whole 32-byte sector each (bf16), which the four
+// warps of the block complete to whole 128-byte lines. The block's partial
+// is the warps' sums in order, each a butterfly over lanes that added their
+// 32 values row by row. Blocks walk the (unit, block) pairs grid-stride: one
+// block per pair on the caller's stream, or a small grid on a side stream,
+// where a block (at most 80 registers a thread, 16 bytes of shared memory)
+// fits beside a Newton-Schulz CTA. The partials do not depend on the grid.
 template <bool GBF16, bool XF32>
-__global__ void __launch_bounds__(kPrepSideThreads, 8) prep_transpose_kernel(const __grid_constant__ MuonPrepLaunch L) {
+__global__ void __launch_bounds__(kPrepSideThreads, 6) prep_transpose_kernel(const __grid_constant__ MuonPrepLaunch L) {
     griddep_launch_dependents();
     griddep_wait();
+    constexpr int RW = kPrepTRows / (kPrepSideThreads / 32);  // rows per warp
+    static_assert(RW == 16 && kPrepTCols == 2 * 32, "block shape");
+    constexpr int RB = GBF16 ? RW : RW / 2;  // rows whose loads are in flight together
+    constexpr int GW = GBF16 ? 1 : 2;        // gradient words per row and lane
     __shared__ float red[kPrepSideThreads / 32];
     const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int64_t items = (int64_t)L.batch * L.heads * L.parts;
@@ -233,67 +239,82 @@ __global__ void __launch_bounds__(kPrepSideThreads, 8) prep_transpose_kernel(con
         const int64_t part = it - (int64_t)u * L.parts;
         const int b = u / L.heads, h = u % L.heads;
         const int64_t off = (int64_t)h * L.Rh * L.C;
-        const int64_t r0 = (part / L.tiles_c) * kPrepTRows;
-        const int64_t c = (part % L.tiles_c) * kPrepTCols + 32 * w + lane;  // this lane's column of u
-        float d[kPrepTRows];
+        const int64_t r0 = (part / L.tiles_c) * kPrepTRows + RW * w;  // this warp's first row of u
+        const int64_t c = (part % L.tiles_c) * kPrepTCols + 2 * lane;  // this lane's first column of u
+        // C % 8 == 0: a lane's two columns are both in range or both out of it
+        const int rows = c < L.C ? (int)max((int64_t)0, min((int64_t)RW, L.Rh - r0)) : 0;
+        const int64_t e0 = off + r0 * L.C + c;  // element index of (r0, c)
+        float* mp = L.M[b] + e0;
+        const uint32_t* gp = reinterpret_cast<const uint32_t*>(L.G[b]) + (GBF16 ? e0 / 2 : e0);
+        const int64_t gstride = GBF16 ? L.C / 2 : L.C;  // words per row
+        float d[RW][2];  // momentum in, then the direction
         float ss = 0.f;
-        const bool col_ok = c < L.C;
-        const int rows = col_ok ? (int)min((int64_t)kPrepTRows, L.Rh - r0) : 0;  // rows of this block in range
-        // running pointers to row r0 + i, column c, of the momentum and the gradient
-        float* mp = L.M[b] + off + r0 * L.C + c;
-        const float* gpf = reinterpret_cast<const float*>(L.G[b]) + off + r0 * L.C + c;
-        const unsigned short* gph = reinterpret_cast<const unsigned short*>(L.G[b]) + off + r0 * L.C + c;
 #pragma unroll
-        for (int i0 = 0; i0 < kPrepTRows; i0 += 4) {
-            float g[4], m[4];
+        for (int i0 = 0; i0 < RW; i0 += RB) {
+            uint32_t g[RB][GW];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {  // four rows' loads in flight before any arithmetic
-                const int64_t o = (int64_t)(i0 + i) * L.C;
-                g[i] = 0.f;
-                m[i] = 0.f;
-                if (i0 + i < rows) {
-                    g[i] = GBF16 ? __uint_as_float((uint32_t)__ldcs(gph + o) << 16) : __ldcs(gpf + o);
-                    m[i] = __ldcs(mp + o);
+            for (int i = i0; i < i0 + RB; ++i) {
+                d[i][0] = d[i][1] = 0.f;
+#pragma unroll
+                for (int k = 0; k < GW; ++k) g[i - i0][k] = 0u;
+                if (i < rows) {
+                    const float2 mv = __ldcs(reinterpret_cast<const float2*>(mp + (int64_t)i * L.C));
+                    d[i][0] = mv.x;
+                    d[i][1] = mv.y;
+                    if (GBF16) {
+                        g[i - i0][0] = __ldcs(gp + (int64_t)i * gstride);
+                    } else {
+                        const uint2 gv = __ldcs(reinterpret_cast<const uint2*>(gp + (int64_t)i * gstride));
+                        g[i - i0][0] = gv.x;
+                        g[i - i0][GW - 1] = gv.y;
+                    }
                 }
             }
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                d[i0 + i] = 0.f;
-                if (i0 + i < rows) {
-                    const float mn = beta * m[i] + omb * g[i];
-                    const float di = nest ? beta * mn + omb * g[i] : mn;
-                    __stcs(mp + (int64_t)(i0 + i) * L.C, mn);
-                    d[i0 + i] = di;
-                    ss += di * di;
+            for (int i = i0; i < i0 + RB; ++i) {
+                if (i < rows) {
+                    const float g0 = GBF16 ? bf16_lo(g[i - i0][0]) : __uint_as_float(g[i - i0][0]);
+                    const float g1 = GBF16 ? bf16_hi(g[i - i0][0]) : __uint_as_float(g[i - i0][GW - 1]);
+                    const float mn0 = beta * d[i][0] + omb * g0;
+                    const float mn1 = beta * d[i][1] + omb * g1;
+                    d[i][0] = nest ? beta * mn0 + omb * g0 : mn0;
+                    d[i][1] = nest ? beta * mn1 + omb * g1 : mn1;
+                    ss += d[i][0] * d[i][0];
+                    ss += d[i][1] * d[i][1];
+                    __stcs(reinterpret_cast<float2*>(mp + (int64_t)i * L.C), make_float2(mn0, mn1));
                 }
             }
         }
-        // row c of X, elements r0 .. r0 + 31
-        if (col_ok) {
-            const int64_t xi = (int64_t)u * L.x_unit + c * L.ldx + r0;
-            if (r0 + kPrepTRows <= L.Rh) {
-                if (XF32) {
-                    float4* xp = reinterpret_cast<float4*>(reinterpret_cast<float*>(L.X) + xi);
+        // rows c and c + 1 of X, elements r0 .. r0 + 15
+        if (rows > 0) {
 #pragma unroll
-                    for (int q = 0; q < 8; ++q) __stcs(xp + q, make_float4(d[4 * q], d[4 * q + 1], d[4 * q + 2], d[4 * q + 3]));
-                } else {
-                    uint4* xp = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(L.X) + xi);
+            for (int j = 0; j < 2; ++j) {
+                const int64_t xi = (int64_t)u * L.x_unit + (c + j) * L.ldx + r0;
+                if (rows == RW) {
+                    if (XF32) {
+                        float4* xp = reinterpret_cast<float4*>(reinterpret_cast<float*>(L.X) + xi);
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        uint4 v;
-                        v.x = pack_bf16x2(d[8 * q + 0], d[8 * q + 1]);
-                        v.y = pack_bf16x2(d[8 * q + 2], d[8 * q + 3]);
-                        v.z = pack_bf16x2(d[8 * q + 4], d[8 * q + 5]);
-                        v.w = pack_bf16x2(d[8 * q + 6], d[8 * q + 7]);
-                        __stcs(xp + q, v);
+                        for (int q = 0; q < RW / 4; ++q)
+                            __stcs(xp + q, make_float4(d[4 * q][j], d[4 * q + 1][j], d[4 * q + 2][j], d[4 * q + 3][j]));
+                    } else {
+                        uint4* xp = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(L.X) + xi);
+#pragma unroll
+                        for (int q = 0; q < RW / 8; ++q) {
+                            uint4 v;
+                            v.x = pack_bf16x2(d[8 * q + 0][j], d[8 * q + 1][j]);
+                            v.y = pack_bf16x2(d[8 * q + 2][j], d[8 * q + 3][j]);
+                            v.z = pack_bf16x2(d[8 * q + 4][j], d[8 * q + 5][j]);
+                            v.w = pack_bf16x2(d[8 * q + 6][j], d[8 * q + 7][j]);
+                            __stcs(xp + q, v);
+                        }
                     }
-                }
-            } else {
+                } else {
 #pragma unroll
-                for (int i = 0; i < kPrepTRows; ++i) {
-                    if (r0 + i < L.Rh) {
-                        if (XF32) reinterpret_cast<float*>(L.X)[xi + i] = d[i];
-                        else reinterpret_cast<__nv_bfloat16*>(L.X)[xi + i] = __float2bfloat16_rn(d[i]);
+                    for (int i = 0; i < RW; ++i) {
+                        if (i < rows) {
+                            if (XF32) reinterpret_cast<float*>(L.X)[xi + i] = d[i][j];
+                            else reinterpret_cast<__nv_bfloat16*>(L.X)[xi + i] = __float2bfloat16_rn(d[i][j]);
+                        }
                     }
                 }
             }

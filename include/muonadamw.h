@@ -375,7 +375,8 @@ void ma_plan_destroy(ma_plan_t* plan);
 #define MA_PROF_MOMENTUM_SIDE 7 /* momentum pass and norm finalize run under   */
                                 /* the Newton-Schulz chain of the batch before */
                                 /* it (side stream)                            */
-#define MA_PROF_CLASSES 8
+#define MA_PROF_NS_Q1 8         /* Gram-space chain: Q_1 = a I + b A_0         */
+#define MA_PROF_CLASSES 9
 
 /* When on != 0, every kernel the library launches on this thread's current
  * device is bracketed by two CUDA events recorded on its launch stream. Off by
