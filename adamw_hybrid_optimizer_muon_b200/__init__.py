@@ -20,16 +20,19 @@ __all__ = [
     "muon_step_batched_noalloc", "STATIC_SCRATCH_BYTES", "ns_iterate_workspace_bytes", "ns_iterate_bf16",
     "adamw_step_fused", "ma_plan_create", "muonadamw_step", "muonadamw_step_graph", "muonadamw_step_from_host",
     "ma_plan_describe", "ma_plan_destroy", "ma_plan_status", "ma_device_status", "ma_device_status_async",
-    "ma_set_wait_limit_ns", "ma_set_momentum_overlap",
+    "ma_set_wait_limit_ns", "ma_set_momentum_overlap", "ma_debug_build", "MA_ERR_BOUNDS",
     "ma_selftest_wait_timeout", "ma_profile_enable", "ma_profile_collect", "PROF_CLASSES", "group_table", "Plan",
     "MuonAdamW", "muon_hparams", "adamw_hparams",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(HERE, "lib", "libmuonadamw.so")
+# The release library, or (MA_LIBRARY=debug) the build with guarded device
+# indexing, lib/libmuonadamw_debug.so; both are compiled by build.py.
+LIB_PATH = os.path.join(HERE, "lib", "libmuonadamw_debug.so" if os.environ.get("MA_LIBRARY") == "debug"
+                        else "libmuonadamw.so")
 
 MA_OK, MA_ERR_NULL, MA_ERR_SHAPE, MA_ERR_DTYPE, MA_ERR_ALIGN, MA_ERR_WORKSPACE = 0, 1, 2, 3, 4, 5
-MA_ERR_UNSUPPORTED, MA_ERR_CUDA, MA_ERR_TIMEOUT, MA_ERR_ARG = 6, 7, 8, 9
+MA_ERR_UNSUPPORTED, MA_ERR_CUDA, MA_ERR_TIMEOUT, MA_ERR_ARG, MA_ERR_BOUNDS = 6, 7, 8, 9, 10
 MA_F32, MA_BF16 = 0, 1
 MA_MUON, MA_ADAMW = 0, 1
 ROLE_HIDDEN, ROLE_EMBED, ROLE_UNEMBED, ROLE_FORCE_ADAMW = 0, 1, 2, 3
@@ -137,6 +140,7 @@ def lib() -> ctypes.CDLL:
         "ma_plan_status": (i32, [vp, vp]),
         "ma_set_wait_limit_ns": (i32, [i64]),
         "ma_set_momentum_overlap": (i32, [i32]),
+        "ma_debug_build": (i32, []),
         "ma_selftest_wait_timeout": (i32, [i64, vp]),
         "muon_step_batched_noalloc": (i32, [i32, i64, i64, pp, pp, i32, pp, ctypes.POINTER(MuonHParams), vp]),
         "ma_profile_enable": (i32, [i32]),
@@ -411,6 +415,11 @@ def ma_device_status_async(host_dst, stream=None) -> None:
 def ma_set_wait_limit_ns(limit_ns: int) -> None:
     """Time limit of the kernels' bounded waits, in nanoseconds (default 2 s)."""
     _check(lib().ma_set_wait_limit_ns(int(limit_ns)), "ma_set_wait_limit_ns")
+
+
+def ma_debug_build() -> bool:
+    """Whether the loaded library is the build with guarded device indexing."""
+    return bool(lib().ma_debug_build())
 
 
 def ma_set_momentum_overlap(on: bool) -> None:

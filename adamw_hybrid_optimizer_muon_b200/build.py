@@ -1,13 +1,18 @@
 """Build the MuonAdamW CUDA library in-tree for sm_100a.
 
-    python -m adamw_hybrid_optimizer_muon_b200.build [--verbose]
+    python -m adamw_hybrid_optimizer_muon_b200.build [--verbose] [--force]
 
 Compiles every ``csrc/*.cu`` with nvcc (``-gencode arch=compute_100a,code=sm_100a``)
-into ``lib/libmuonadamw.so``. Each object is rebuilt only when a source or header
-is newer than it. nvcc cross-compiles, so no GPU is needed.
+into ``lib/libmuonadamw.so``, and once more with ``-DMA_DEBUG`` into
+``lib/libmuonadamw_debug.so``: the debug build checks every hand-computed device
+index against the extent of its buffer (a failed check records MA_ERR_BOUNDS
+and skips the access) and otherwise computes the same bits. Each object is
+rebuilt only when a source or header is newer than it; the objects compile in
+parallel. nvcc cross-compiles, so no GPU is needed.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import glob
 import os
 import shutil
@@ -20,6 +25,8 @@ CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(HERE, "_build")
 LIB_DIR = os.path.join(HERE, "lib")
 LIB = os.path.join(LIB_DIR, "libmuonadamw.so")
+LIB_DEBUG = os.path.join(LIB_DIR, "libmuonadamw_debug.so")
+VARIANTS = (("release", LIB, []), ("debug", LIB_DEBUG, ["-DMA_DEBUG"]))
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O3",
@@ -39,28 +46,45 @@ def _headers():
 
 
 def build(verbose: bool = False, force: bool = False) -> str:
-    os.makedirs(OBJ, exist_ok=True)
+    """Build both libraries; returns the release library's path."""
     os.makedirs(LIB_DIR, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
     hdr_mtime = max([os.path.getmtime(h) for h in _headers()] + [0.0])
-    objs = []
-    for src in srcs:
-        obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
-        objs.append(obj)
-        if not force and os.path.exists(obj) and os.path.getmtime(obj) >= max(os.path.getmtime(src), hdr_mtime):
-            continue
-        cmd = [nvcc()] + ARCH + FLAGS + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
-        res = subprocess.run(cmd, capture_output=True, text=True)
-        if verbose or res.returncode != 0:
-            sys.stderr.write(res.stdout + res.stderr)
-        if res.returncode != 0:
-            raise RuntimeError(f"nvcc failed on {os.path.basename(src)}")
-    if force or not os.path.exists(LIB) or os.path.getmtime(LIB) < max(os.path.getmtime(o) for o in objs):
-        cmd = [nvcc()] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-o", LIB] + objs
-        res = subprocess.run(cmd, capture_output=True, text=True)
-        if res.returncode != 0:
-            sys.stderr.write(res.stdout + res.stderr)
-            raise RuntimeError("link failed")
+    jobs = []  # (source, object, extra flags)
+    objs = {}
+    for name, _, extra in VARIANTS:
+        odir = os.path.join(OBJ, name)
+        os.makedirs(odir, exist_ok=True)
+        objs[name] = []
+        for src in srcs:
+            obj = os.path.join(odir, os.path.basename(src)[:-3] + ".o")
+            objs[name].append(obj)
+            if force or not os.path.exists(obj) or os.path.getmtime(obj) < max(os.path.getmtime(src), hdr_mtime):
+                jobs.append((src, obj, extra))
+
+    def compile_one(job):
+        src, obj, extra = job
+        cmd = [nvcc()] + ARCH + FLAGS + extra + (["-Xptxas", "-v"] if verbose else []) + ["-c", src, "-o", obj]
+        return job, subprocess.run(cmd, capture_output=True, text=True)
+
+    workers = max(1, min(len(jobs), os.cpu_count() or 1))
+    failed = []
+    with concurrent.futures.ThreadPoolExecutor(max_workers=workers) as pool:
+        for (src, obj, extra), res in pool.map(compile_one, jobs):
+            if verbose or res.returncode != 0:
+                sys.stderr.write(res.stdout + res.stderr)
+            if res.returncode != 0:
+                failed.append(os.path.basename(src) + (" (debug)" if extra else ""))
+    if failed:
+        raise RuntimeError("nvcc failed on " + ", ".join(failed))
+    for name, lib_path, _ in VARIANTS:
+        o = objs[name]
+        if force or not os.path.exists(lib_path) or os.path.getmtime(lib_path) < max(os.path.getmtime(x) for x in o):
+            cmd = [nvcc()] + ARCH + ["-shared", "-Xcompiler", "-fPIC", "-o", lib_path] + o
+            res = subprocess.run(cmd, capture_output=True, text=True)
+            if res.returncode != 0:
+                sys.stderr.write(res.stdout + res.stderr)
+                raise RuntimeError(f"link failed ({name})")
     return LIB
 
 

@@ -68,6 +68,7 @@ __global__ void __launch_bounds__(256) adamw_kernel(const __grid_constant__ Adam
         const int64_t nvec_end = start + ((end - start) & ~int64_t(3));
 #pragma unroll 2
         for (int64_t i = start + 4 * (int64_t)threadIdx.x; i < nvec_end; i += 4 * 256) {
+            if (!MA_INB(i, 4, T.numel, L.status)) continue;
             float4 p = *reinterpret_cast<const float4*>(T.p + i);
             float4 m = *reinterpret_cast<const float4*>(T.m + i);
             float4 v = *reinterpret_cast<const float4*>(T.v + i);
@@ -84,6 +85,7 @@ __global__ void __launch_bounds__(256) adamw_kernel(const __grid_constant__ Adam
         scalar_from = nvec_end;
     }
     for (int64_t i = scalar_from + threadIdx.x; i < end; i += 256) {
+        if (!MA_INB(i, 1, T.numel, L.status)) continue;
         float p = T.p[i], m = T.m[i], v = T.v[i];
         adamw_elem(p, m, v, load_g1(T.g, L.gdt, i), H);
         T.p[i] = p;

@@ -306,6 +306,7 @@ int muon_prep(const MuonJob& j, cudaStream_t s, int max_blocks, bool side, int* 
     MuonPrepLaunch P;
     std::memset(&P, 0, sizeof(P));
     P.batch = j.batch;
+    P.status = device_status_ptr();
     P.heads = g.heads;
     P.transposed = g.transposed;
     P.gdt = j.gdt;
@@ -449,7 +450,7 @@ int chain_gspace(const std::vector<const MuonJob*>& jobs, cudaStream_t s, int sm
         const MuonGeom& g = jobs[i]->g;
         const int pr = prof_begin(MA_PROF_NS_Q1, s);
         const cudaError_t e = launch_ns_q1(Acur[i], Qcur[i], (int)g.m, g.ldg, g.m * g.ldg, (int)g.units,
-                                           coef(i, 0, 0), coef(i, 0, 1), sms, s);
+                                           coef(i, 0, 0), coef(i, 0, 1), device_status_ptr(), sms, s);
         prof_end(pr, s, 0.0, 4.0 * (double)g.units * (double)g.m * (double)g.m);  // A read, Q written (bf16)
         if (e != cudaSuccess) return MA_ERR_CUDA;
         ++*launches;
@@ -674,6 +675,7 @@ int run_adamw(const std::vector<AdamwItem>& items, int gdt, const AdamwGroupCons
     while (i < items.size()) {
         std::memset(&L, 0, sizeof(L));
         L.gdt = gdt;
+        L.status = device_status_ptr();
         for (int k = 0; k < ngroups; ++k) L.grp[k] = grp[k];
         int64_t chunk = 0;
         int nt = 0;
@@ -1113,6 +1115,7 @@ const char* ma_status_string(int s) {
         case MA_ERR_CUDA: return "CUDA runtime error";
         case MA_ERR_TIMEOUT: return "device wait timed out";
         case MA_ERR_ARG: return "hyperparameter out of range";
+        case MA_ERR_BOUNDS: return "guarded device index out of bounds (debug build)";
         default: return "unknown status";
     }
 }
@@ -2030,6 +2033,14 @@ int ma_set_wait_limit_ns(int64_t limit_ns) {
     if (limit_ns <= 0) return MA_ERR_ARG;
     g_host_wait_limit_ns.store(limit_ns, std::memory_order_relaxed);
     return MA_OK;
+}
+
+int ma_debug_build(void) {
+#ifdef MA_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
 }
 
 int ma_set_momentum_overlap(int on) {

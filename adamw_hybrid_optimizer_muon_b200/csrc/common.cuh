@@ -31,6 +31,23 @@ __device__ __forceinline__ void record_error(int* status, int code) {
     if (status) atomicCAS(status, 0, code);
 }
 
+// Guarded indexing, in debug builds (-DMA_DEBUG): each hand-computed global
+// access is checked against the extent of its buffer. An access of k elements
+// at element i of a buffer of n elements needs 0 <= i and i + k <= n; a check
+// that fails records MA_ERR_BOUNDS in the status word and the access is
+// skipped. Other builds compile the checks to nothing (MA_INB is true).
+#ifdef MA_DEBUG
+static __device__ __noinline__ void bounds_fail(int* status) { record_error(status, MA_ERR_BOUNDS); }
+__device__ __forceinline__ bool in_bounds(int64_t i, int64_t k, int64_t n, int* status) {
+    const bool ok = i >= 0 && i + k <= n;
+    if (!ok) bounds_fail(status);
+    return ok;
+}
+#define MA_INB(i, k, n, status) ::ma::in_bounds((int64_t)(i), (int64_t)(k), (int64_t)(n), (status))
+#else
+#define MA_INB(i, k, n, status) true
+#endif
+
 __device__ __forceinline__ uint64_t globaltimer() {
     uint64_t t;
     asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

@@ -81,6 +81,7 @@ struct AdamwLaunch {
     int32_t ntensors;
     int32_t gdt;  // ma_dtype_t of every gradient in this launch
     int64_t nchunks;
+    int* status;  // device status word (guarded indexing in debug builds)
     AdamwGroupConst grp[MA_MAX_GROUPS];
     AdamwTensorDesc t[kAdamwMaxTensorsPerLaunch];
 };
@@ -97,6 +98,7 @@ constexpr int kPrepTCols = 64;        // transposing path: columns of u per thre
 
 struct MuonPrepLaunch {
     int32_t batch, heads, transposed, gdt, nesterov, x_f32;
+    int* status;          // device status word (guarded indexing in debug builds)
     int64_t C, Rh;        // matrix columns, rows per head slice
     int64_t ldx;          // row stride (elements) of the NS operand X
     int64_t x_unit;       // elements between consecutive units of X
@@ -180,8 +182,9 @@ size_t ns_tc_launch_bytes();
 int ns_tc_patch_final(void* launch, NsFinalPatchFn f, void* ctx);
 
 // Q = a*I + b*A (bf16 m x m per unit, row stride ldg, unit stride g_unit).
+// status: the device status word (guarded indexing in debug builds).
 cudaError_t launch_ns_q1(const void* A, void* Q, int m, int64_t ldg, int64_t g_unit, int units, float a, float b,
-                         int num_sms, cudaStream_t s);
+                         int* status, int num_sms, cudaStream_t s);
 
 // fp32 SIMT path (precision mode 1).
 cudaError_t launch_ns_simt(int mode, const NsParams& p, const void* x_buf, const void* g_buf, cudaStream_t s);

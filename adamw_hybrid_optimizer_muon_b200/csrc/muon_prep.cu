@@ -109,12 +109,20 @@ __device__ __forceinline__ float prep_flat_pass(const MuonPrepLaunch& L, int u, 
                    : static_cast<void*>(reinterpret_cast<uint16_t*>(L.X) + (int64_t)u * L.x_unit);
     const float beta = L.beta, omb = L.omb;
     const bool nest = L.nesterov != 0;
+    // buffer extents for the guarded build: a matrix's G and M, and the workspace's X
+    const int64_t mat_elems = (int64_t)L.heads * unit_elems, x_elems = (int64_t)L.batch * L.heads * L.x_unit;
+    const int64_t xu = (int64_t)u * L.x_unit;
     float ss = 0.f;
     if (end - start == kPrepChunk) {
         float g[kIter][8], m[kIter][8];
+        bool ok[kIter];
 #pragma unroll
         for (int k = 0; k < kIter; ++k) {
             const int64_t i = start + 8 * ((int64_t)k * 256 + vt);
+            ok[k] = MA_INB(off + i, 8, mat_elems, L.status) && MA_INB(xu + i, 8, x_elems, L.status);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) g[k][e] = m[k][e] = 0.f;
+            if (!ok[k]) continue;
             load_g8<GBF16>(G, i, g[k]);
             const float4 a = __ldcs(reinterpret_cast<const float4*>(M + i));
             const float4 c = __ldcs(reinterpret_cast<const float4*>(M + i + 4));
@@ -126,12 +134,14 @@ __device__ __forceinline__ float prep_flat_pass(const MuonPrepLaunch& L, int u, 
             const int64_t i = start + 8 * ((int64_t)k * 256 + vt);
             float d[8];
             ss += momentum8(m[k], g[k], d, beta, omb, nest);
+            if (!ok[k]) continue;
             __stcs(reinterpret_cast<float4*>(M + i), make_float4(m[k][0], m[k][1], m[k][2], m[k][3]));
             __stcs(reinterpret_cast<float4*>(M + i + 4), make_float4(m[k][4], m[k][5], m[k][6], m[k][7]));
             store_x8<XF32>(X, i, d);
         }
     } else {
         for (int64_t i = start + 8 * (int64_t)vt; i < end; i += 8 * 256) {
+            if (!(MA_INB(off + i, 8, mat_elems, L.status) && MA_INB(xu + i, 8, x_elems, L.status))) continue;
             float g[8], m[8], d[8];
             load_g8<GBF16>(G, i, g);
             const float4 a = __ldcs(reinterpret_cast<const float4*>(M + i));
@@ -244,6 +254,8 @@ __global__ void __launch_bounds__(kPrepSideThreads, 6) prep_transpose_kernel(con
         // C % 8 == 0: a lane's two columns are both in range or both out of it
         const int rows = c < L.C ? (int)max((int64_t)0, min((int64_t)RW, L.Rh - r0)) : 0;
         const int64_t e0 = off + r0 * L.C + c;  // element index of (r0, c)
+        // buffer extents for the guarded build: a matrix's G and M, and the workspace's X
+        const int64_t mat_elems = (int64_t)L.heads * L.Rh * L.C, x_elems = (int64_t)L.batch * L.heads * L.x_unit;
         float* mp = L.M[b] + e0;
         const uint32_t* gp = reinterpret_cast<const uint32_t*>(L.G[b]) + (GBF16 ? e0 / 2 : e0);
         const int64_t gstride = GBF16 ? L.C / 2 : L.C;  // words per row
@@ -257,7 +269,7 @@ __global__ void __launch_bounds__(kPrepSideThreads, 6) prep_transpose_kernel(con
                 d[i][0] = d[i][1] = 0.f;
 #pragma unroll
                 for (int k = 0; k < GW; ++k) g[i - i0][k] = 0u;
-                if (i < rows) {
+                if (i < rows && MA_INB(e0 + (int64_t)i * L.C, 2, mat_elems, L.status)) {
                     const float2 mv = __ldcs(reinterpret_cast<const float2*>(mp + (int64_t)i * L.C));
                     d[i][0] = mv.x;
                     d[i][1] = mv.y;
@@ -272,7 +284,7 @@ __global__ void __launch_bounds__(kPrepSideThreads, 6) prep_transpose_kernel(con
             }
 #pragma unroll
             for (int i = i0; i < i0 + RB; ++i) {
-                if (i < rows) {
+                if (i < rows && MA_INB(e0 + (int64_t)i * L.C, 2, mat_elems, L.status)) {
                     const float g0 = GBF16 ? bf16_lo(g[i - i0][0]) : __uint_as_float(g[i - i0][0]);
                     const float g1 = GBF16 ? bf16_hi(g[i - i0][0]) : __uint_as_float(g[i - i0][GW - 1]);
                     const float mn0 = beta * d[i][0] + omb * g0;
@@ -290,6 +302,7 @@ __global__ void __launch_bounds__(kPrepSideThreads, 6) prep_transpose_kernel(con
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
                 const int64_t xi = (int64_t)u * L.x_unit + (c + j) * L.ldx + r0;
+                if (!MA_INB(xi, rows, x_elems, L.status)) continue;
                 if (rows == RW) {
                     if (XF32) {
                         float4* xp = reinterpret_cast<float4*>(reinterpret_cast<float*>(L.X) + xi);

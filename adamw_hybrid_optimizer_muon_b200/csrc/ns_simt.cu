@@ -33,16 +33,21 @@ __global__ void __launch_bounds__(256) ns_simt_kernel(const __grid_constant__ Ns
     const float* SA;
     const float* SB;
     int64_t lda, ldb;
+    int64_t a_unit, b_unit;  // elements per unit of the operands' buffers (guarded build)
     if (MODE == NS_GRAM) {
-        SA = xb + (int64_t)u * p.x_unit; lda = p.ldx;
-        SB = SA; ldb = p.ldx;
+        SA = xb + (int64_t)u * p.x_unit; lda = p.ldx; a_unit = p.x_unit;
+        SB = SA; ldb = p.ldx; b_unit = p.x_unit;
     } else if (MODE == NS_GRAMSQ) {
-        SA = reinterpret_cast<const float*>(p.xin) + (int64_t)u * p.g_unit; lda = p.ldg;
-        SB = SA; ldb = p.ldg;
+        SA = reinterpret_cast<const float*>(p.xin) + (int64_t)u * p.g_unit; lda = p.ldg; a_unit = p.g_unit;
+        SB = SA; ldb = p.ldg; b_unit = p.g_unit;
     } else {
-        SA = gb + (int64_t)u * p.g_unit; lda = p.ldg;
-        SB = xb + (int64_t)u * p.x_unit; ldb = p.ldx;
+        SA = gb + (int64_t)u * p.g_unit; lda = p.ldg; a_unit = p.g_unit;
+        SB = xb + (int64_t)u * p.x_unit; ldb = p.ldx; b_unit = p.x_unit;
     }
+    // element offsets from the buffers' starts, and their extents
+    const int64_t a0 = (int64_t)u * a_unit, a_ext = (int64_t)p.units * a_unit;
+    const int64_t b0 = (int64_t)u * b_unit, b_ext = (int64_t)p.units * b_unit;
+    (void)a0; (void)a_ext; (void)b0; (void)b_ext;
     const int tid = threadIdx.x;
     const int ty = tid >> 4, tx = tid & 15;
     float acc[4][4] = {};
@@ -52,7 +57,8 @@ __global__ void __launch_bounds__(256) ns_simt_kernel(const __grid_constant__ Ns
             const int idx = tid * 4 + e;
             const int ii = idx >> 4, kk = idx & 15;
             const int gi = i0 + ii, gk = k0 + kk;
-            As[kk][ii] = (gi < M && gk < K) ? SA[(int64_t)gi * lda + gk] : 0.f;
+            As[kk][ii] = (gi < M && gk < K && MA_INB(a0 + (int64_t)gi * lda + gk, 1, a_ext, p.status))
+                             ? SA[(int64_t)gi * lda + gk] : 0.f;
         }
         if (gram) {
 #pragma unroll
@@ -60,7 +66,8 @@ __global__ void __launch_bounds__(256) ns_simt_kernel(const __grid_constant__ Ns
                 const int idx = tid * 4 + e;
                 const int jj = idx >> 4, kk = idx & 15;
                 const int gj = j0 + jj, gk = k0 + kk;
-                Bs[kk][jj] = (gj < N && gk < K) ? SB[(int64_t)gj * ldb + gk] : 0.f;
+                Bs[kk][jj] = (gj < N && gk < K && MA_INB(b0 + (int64_t)gj * ldb + gk, 1, b_ext, p.status))
+                                 ? SB[(int64_t)gj * ldb + gk] : 0.f;
             }
         } else {
 #pragma unroll
@@ -68,7 +75,8 @@ __global__ void __launch_bounds__(256) ns_simt_kernel(const __grid_constant__ Ns
                 const int idx = tid * 4 + e;
                 const int kk = idx >> 6, jj = idx & 63;
                 const int gj = j0 + jj, gk = k0 + kk;
-                Bs[kk][jj] = (gj < N && gk < K) ? SB[(int64_t)gk * ldb + gj] : 0.f;
+                Bs[kk][jj] = (gj < N && gk < K && MA_INB(b0 + (int64_t)gk * ldb + gj, 1, b_ext, p.status))
+                                 ? SB[(int64_t)gk * ldb + gj] : 0.f;
             }
         }
         __syncthreads();
@@ -96,22 +104,28 @@ __global__ void __launch_bounds__(256) ns_simt_kernel(const __grid_constant__ Ns
             const int j = j0 + tx * 4 + c;
             if (j >= N) continue;
             const float v = acc[r][c];
+            const int64_t gi = (int64_t)u * p.g_unit + (int64_t)i * p.ldg + j;  // (i, j) in a Gram buffer
+            const int64_t xi = (int64_t)u * p.x_unit + (int64_t)i * p.ldx + j;  // (i, j) in an X buffer
+            const int64_t g_ext = (int64_t)p.units * p.g_unit, x_ext = (int64_t)p.units * p.x_unit;
             if (MODE == NS_GRAM) {
                 float coef = p.coef_gram;
                 if (p.first) coef *= sa * sa;
-                reinterpret_cast<float*>(p.out)[(int64_t)u * p.g_unit + (int64_t)i * p.ldg + j] = coef * v;
+                if (MA_INB(gi, 1, g_ext, p.status)) reinterpret_cast<float*>(p.out)[gi] = coef * v;
             } else if (MODE == NS_GRAMSQ) {
+                if (!MA_INB(gi, 1, g_ext, p.status)) continue;
                 const float ain = SA[(int64_t)i * lda + j];
-                reinterpret_cast<float*>(p.out)[(int64_t)u * p.g_unit + (int64_t)i * p.ldg + j] = p.b * ain + p.c * v;
+                reinterpret_cast<float*>(p.out)[gi] = p.b * ain + p.c * v;
             } else {
-                const float x = xb[(int64_t)u * p.x_unit + (int64_t)i * p.ldx + j];
+                if (!MA_INB(xi, 1, x_ext, p.status)) continue;
+                const float x = xb[xi];
                 const float o = sa * (p.a * x + v);
                 if (MODE == NS_APPLY) {
-                    reinterpret_cast<float*>(p.out)[(int64_t)u * p.x_unit + (int64_t)i * p.ldx + j] = o;
+                    reinterpret_cast<float*>(p.out)[xi] = o;
                 } else {
                     const int bidx = u / p.heads, h = u - bidx * p.heads;
-                    float* Wb = p.W[bidx] + (int64_t)h * p.Rh * p.C;
-                    float* w = p.transposed ? Wb + (int64_t)j * p.C + i : Wb + (int64_t)i * p.C + j;
+                    const int64_t wi = (int64_t)h * p.Rh * p.C + (p.transposed ? (int64_t)j * p.C + i : (int64_t)i * p.C + j);
+                    if (!MA_INB(wi, 1, (int64_t)p.heads * p.Rh * p.C, p.status)) continue;
+                    float* w = p.W[bidx] + wi;
                     const float wv = *w;
                     *w = p.cautious ? (o * wv > 0.f ? wv - p.lr_wd * wv : wv) - p.lr_s * o : wv * p.decay - p.lr_s * o;
                 }

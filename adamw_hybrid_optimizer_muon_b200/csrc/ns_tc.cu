@@ -75,15 +75,26 @@ constexpr uint32_t STG_BLOCK = 32 * 32 * 2;
 constexpr uint32_t kEpiSleepNs = MA_EPI_SLEEP_NS;
 constexpr uint32_t STG_BYTES = EPI_WARPS * 2 * STG_BLOCK;  // 32 KB
 // Final apply: each epilogue warp double-buffers a 32 x 32 fp32 block of W
-// (128-byte rows) and the matching 32 x 32 bf16 block of X (64-byte rows).
-// The 16-byte chunks of each row are XOR-swizzled by the row index, which
-// keeps row-wise and column-wise accesses free of bank conflicts.
+// (128-byte rows) and, in the shallow variant, the matching 32 x 32 bf16
+// block of X (64-byte rows). The 16-byte chunks of each row are XOR-swizzled
+// by the row index, which keeps row-wise and column-wise accesses free of
+// bank conflicts. Two variants share the code:
+//  * shallow (DEEP = false): W and X staged, 96 KB, a 4-stage ring. For short
+//    K loops (m < 2048), where the epilogue's latency is on the critical path
+//    and the W stream nearly fills HBM;
+//  * deep (DEEP = true): W staged, each lane reads its row of X straight from
+//    global memory, 64 KB, a 5-stage ring. For m >= 2048, where the main loop
+//    is long and more loads in flight keep the tensor pipe busier.
 constexpr uint32_t WBUF = 32 * 128;                              // 4 KB
 constexpr uint32_t XBUF = 32 * 64;                               // 2 KB
-constexpr uint32_t FIN_WARP_BYTES = 2 * WBUF + 2 * XBUF;         // 12 KB
-constexpr uint32_t WBUF_BYTES = EPI_WARPS * FIN_WARP_BYTES;      // 96 KB
-constexpr int kStages(int mode) { return mode == NS_FINAL ? 4 : STAGES; }
-constexpr uint32_t kEpiBytes(int mode) { return mode == NS_FINAL ? WBUF_BYTES : STG_BYTES; }
+constexpr uint32_t fin_warp_bytes(bool deep) { return deep ? 2 * WBUF : 2 * WBUF + 2 * XBUF; }  // 8 / 12 KB
+constexpr int kStages(int mode, bool deep) { return mode == NS_FINAL ? (deep ? 5 : 4) : STAGES; }
+constexpr uint32_t kEpiBytes(int mode, bool deep) {
+    return mode == NS_FINAL ? EPI_WARPS * fin_warp_bytes(deep) : STG_BYTES;
+}
+// Final-apply launches whose units all have at least this many rows (the K
+// of the main loop) take the deep variant.
+constexpr int kDeepFinalMinM = 2048;
 
 constexpr int kMaxStages = 8;
 // Wind-down after an abort: waits for the pair's own work in flight (issued
@@ -109,16 +120,17 @@ static_assert(sizeof(Ctl) <= 512, "control block");
 // Single CTA (for units with m <= 128, where a 256-row tile would be half
 // empty): a 128-row tile, 256 columns for the applies and 128 for the Gram,
 // cta_group::1.
-template <int MODE, bool PAIR>
+template <int MODE, bool PAIR, bool DEEP = false>
 struct Shape {
+    static_assert(!DEEP || MODE == NS_FINAL, "only the final apply has a deep variant");
     static constexpr bool kApply = MODE == NS_APPLY || MODE == NS_FINAL;
     static constexpr int TM = PAIR ? BM : HM;                       // output tile rows
     static constexpr int TN = PAIR ? BN : (kApply ? BN : HN);       // output tile columns
     static constexpr int CN = PAIR ? TN / 2 : TN;                   // B columns staged by each CTA
     static constexpr uint32_t STAGE = A_BYTES + (uint32_t)CN * BK * 2;
-    static constexpr uint32_t EPI = kEpiBytes(MODE);
+    static constexpr uint32_t EPI = kEpiBytes(MODE, DEEP);
     static constexpr int FIT = (int)((232448u - EPI - 1536u) / STAGE);  // 227 KB of shared memory per CTA
-    static constexpr int NST = PAIR ? kStages(MODE) : (FIT < STAGES ? FIT : STAGES);
+    static constexpr int NST = PAIR ? kStages(MODE, DEEP) : (FIT < STAGES ? FIT : STAGES);
     static constexpr uint32_t TMEM = 2 * TN;                        // two fp32 accumulators
     static constexpr int CPW = TN / 64;                             // 32-column chunks per epilogue warp
     static constexpr size_t SMEM = (size_t)NST * STAGE + EPI + 1024 + 512;
@@ -229,7 +241,7 @@ __device__ __forceinline__ void combine_row(const __nv_bfloat16* in, bool row_ok
 // col0..col0+31), before rounding: GRAM b*A (x s^2 on the first iteration),
 // GRAMSQ b*A + c*A^2, APPLY/FINAL s*(a*X + B*X).
 template <int MODE>
-__device__ __forceinline__ void epilogue_values(const NsJob& p, const TileCoord& tc, int row, int col0,
+__device__ __forceinline__ void epilogue_values(const NsJob& p, const TileCoord& tc, int row, int col0, int* status,
                                                 const float (&v)[32], float (&o)[32]) {  // o may alias v
     if (MODE == NS_GRAM) {
         float coef = p.coef_gram;
@@ -244,12 +256,16 @@ __device__ __forceinline__ void epilogue_values(const NsJob& p, const TileCoord&
         const int m = p.m;
         const float b = p.b, c = p.c;
         const __nv_bfloat16* Zin = reinterpret_cast<const __nv_bfloat16*>(p.zin) + (int64_t)tc.u * p.g_unit;
-        combine_row(Zin + (int64_t)row * p.ldg + col0, row < m, m - col0, b, c, v, o);
+        const bool ok = row < m && MA_INB((int64_t)tc.u * p.g_unit + (int64_t)row * p.ldg + col0, min(32, m - col0),
+                                          (int64_t)p.units * p.g_unit, status);
+        combine_row(Zin + (int64_t)row * p.ldg + col0, ok, m - col0, b, c, v, o);
     } else {
         const int m = p.m, n = p.n;
         const float sa = p.first ? p.scale[tc.u] : 1.f;
         const __nv_bfloat16* Xin = reinterpret_cast<const __nv_bfloat16*>(p.xin) + (int64_t)tc.u * p.x_unit;
-        combine_row(Xin + (int64_t)row * p.ldx + col0, row < m, n - col0, sa * p.a, sa, v, o);
+        const bool ok = row < m && MA_INB((int64_t)tc.u * p.x_unit + (int64_t)row * p.ldx + col0, min(32, n - col0),
+                                          (int64_t)p.units * p.x_unit, status);
+        combine_row(Xin + (int64_t)row * p.ldx + col0, ok, n - col0, sa * p.a, sa, v, o);
     }
 }
 
@@ -272,26 +288,28 @@ __device__ __forceinline__ uint32_t sw128w(uint32_t r, uint32_t q) { return r * 
 // run by each epilogue warp over its 32-column chunks of every tile.
 //
 // For each chunk, the 32 x 32 block of W (in W's own orientation: transposed
-// back when the unit was tall) and the 32 x 32 block of X that the a*X term
-// needs (none when a = 0) come into shared memory by 16-byte asynchronous
-// copies. The first two
-// chunks of a tile are fetched before the accumulator is ready, and each
-// later chunk while the one before it is being computed, so the DRAM latency
-// of both hides behind the main loop without holding registers. Each lane
-// then forms its row of X_N from the accumulator and X, updates its own row
-// (or, transposed, its own column) of the W block in place, and the block
-// goes back to W with coalesced 16-byte stores.
-template <bool PAIR>
+// back when the unit was tall) comes into shared memory by 16-byte
+// asynchronous copies, and so does, in the shallow variant, the 32 x 32 block
+// of X that the a*X term needs (none when a = 0). The first two chunks of a
+// tile are fetched before the accumulator is ready, and each later chunk
+// while the one before it is being computed, so the DRAM latency hides
+// behind the main loop without holding registers. In the deep variant each
+// lane reads the 32 values of its row of X straight from global memory, as
+// the other epilogues read theirs. Each lane forms its row of X_N from the
+// accumulator and X, updates its own row (or, transposed, its own column) of
+// the W block in place, and the block goes back to W with coalesced 16-byte
+// stores.
+template <bool PAIR, bool DEEP>
 __device__ __forceinline__ void final_epilogue(const NsLaunch& L, Ctl* ctl, int pair, int npairs, uint32_t rank,
                                                uint32_t tmem_base, int warp, int lane, uint8_t* wbuf,
                                                const AbortCtl& ab) {
-    using S = Shape<NS_FINAL, PAIR>;
+    using S = Shape<NS_FINAL, PAIR, DEEP>;
+    uint8_t* xbuf = wbuf + 2 * WBUF;  // shallow variant only
     constexpr int CPW = S::CPW;
     const int quad = warp & 3, half = (warp - 2) / 4;
     const long long limit = L.wait_limit_ns;
     const uint32_t acc_empty_leader0 = PAIR ? mapa_shared(smem_u32(&ctl->acc_empty[0]), 0) : 0u;
     const uint32_t acc_empty_leader1 = PAIR ? mapa_shared(smem_u32(&ctl->acc_empty[1]), 0) : 0u;
-    uint8_t* xbuf = wbuf + 2 * WBUF;
     int lt = 0;
     for (int t = pair; t < L.total_tiles; t += npairs, ++lt) {
         const JobTile jt = decode_job_tile(L, NS_FINAL, t);
@@ -308,6 +326,10 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, Ctl* ctl, int 
         const int bidx = tc.u / p.heads, h = tc.u - bidx * p.heads;
         float* Wb = L.W[p.w0 + bidx] + (int64_t)h * p.Rh * p.C;
         const __nv_bfloat16* Xin = reinterpret_cast<const __nv_bfloat16*>(p.xin) + (int64_t)tc.u * p.x_unit;
+        // element offsets and extents of this unit's W (in its matrix) and X (guarded build)
+        const int64_t wbase = (int64_t)h * p.Rh * p.C, w_ext = (int64_t)p.heads * p.Rh * p.C;
+        const int64_t xbase = (int64_t)tc.u * p.x_unit, x_ext = (int64_t)p.units * p.x_unit;
+        (void)wbase; (void)w_ext; (void)xbase; (void)x_ext;
         // geometry of chunk c's W block: its first W row, first W column, and extents
         auto block = [&](int c, int& r0, int& c0, int& nr, int& rb) -> bool {
             const int col0 = tc.tj * S::TN + (half * CPW + c) * 32;
@@ -323,17 +345,19 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, Ctl* ctl, int 
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
                     const int row = 4 * i + (lane >> 3), q = lane & 7;
-                    if (row < nr && q * 16 < rb)
+                    if (row < nr && q * 16 < rb &&
+                        MA_INB(wbase + (int64_t)(r0 + row) * p.C + c0 + q * 4, 4, w_ext, L.status))
                         cp_async16(buf + sw128w(row, q), Wb + (int64_t)(r0 + row) * p.C + c0 + q * 4);
                 }
-                // X rows row_lo.., columns col0..: 8 bf16 per copy; the row stride is a multiple of 8
-                const int col0 = tc.tj * S::TN + (half * CPW + c) * 32;
-                uint8_t* xb = xbuf + (c & 1) * XBUF;
-                if (ax) {
+                if (!DEEP && ax) {
+                    // X rows row_lo.., columns col0..: 8 bf16 per copy; the row stride is a multiple of 8
+                    const int col0 = tc.tj * S::TN + (half * CPW + c) * 32;
+                    uint8_t* xb = xbuf + (c & 1) * XBUF;
 #pragma unroll
                     for (int i = 0; i < 4; ++i) {
                         const int row = 8 * i + (lane >> 2), q = lane & 3;
-                        if (row_lo + row < m && col0 + 8 * q < n)
+                        if (row_lo + row < m && col0 + 8 * q < n &&
+                            MA_INB(xbase + (int64_t)(row_lo + row) * p.ldx + col0 + 8 * q, 8, x_ext, L.status))
                             cp_async16(xb + sw64(row, q), Xin + (int64_t)(row_lo + row) * p.ldx + col0 + 8 * q);
                     }
                 }
@@ -353,18 +377,36 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, Ctl* ctl, int 
             int r0, c0, nr, rb;
             if (!block(c, r0, c0, nr, rb)) break;  // warp-uniform
             uint8_t* buf = wbuf + (c & 1) * WBUF;
-            const uint8_t* xb = xbuf + (c & 1) * XBUF;
+            // this lane's 32 values of X (row row_lo + lane), loaded before the accumulator
+            // read; the row stride is a multiple of 8 and n - col0 of 8, so a group of 8
+            // is wholly in range or out of it
+            const int col0 = tc.tj * S::TN + (half * CPW + c) * 32;
+            uint4 xv[4];
+            if (DEEP && ax) {
+                const bool xrow = row_lo + lane < m;
+                const uint4* xs = reinterpret_cast<const uint4*>(Xin + (int64_t)(row_lo + lane) * p.ldx + col0);
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    xv[q] = (xrow && col0 + 8 * q < n &&
+                             MA_INB(xbase + (int64_t)(row_lo + lane) * p.ldx + col0 + 8 * q, 8, x_ext, L.status))
+                                ? __ldg(xs + q)
+                                : make_uint4(0u, 0u, 0u, 0u);
+            }
             float o[32];
             tmem_ld32(tmem_base + (uint32_t)(acc * S::TN + (half * CPW + c) * 32) + ((uint32_t)(quad * 32) << 16), o);
             // chunk c's copies are the oldest group but one (chunk c + 1 was issued after it)
             cp_async_wait<1>();
             __syncwarp();
+            if (!DEEP && ax) {
+                const uint8_t* xb = xbuf + (c & 1) * XBUF;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) xv[q] = *reinterpret_cast<const uint4*>(xb + sw64(lane, q));
+            }
             // X_N row of this lane: s*(a*X + (B X)), s only on the first iteration
             if (ax) {
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const uint4 w = *reinterpret_cast<const uint4*>(xb + sw64(lane, q));
-                    const uint32_t wv[4] = {w.x, w.y, w.z, w.w};
+                    const uint32_t wv[4] = {xv[q].x, xv[q].y, xv[q].z, xv[q].w};
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
                         o[8 * q + 2 * e] = ca * bf16_lo(wv[e]) + sa * o[8 * q + 2 * e];
@@ -401,7 +443,8 @@ __device__ __forceinline__ void final_epilogue(const NsLaunch& L, Ctl* ctl, int 
                 const int row = 4 * i + (lane >> 3), q = lane & 7;
                 // streaming stores (evict-first in L2): the updated weights are not
                 // read again in this launch, unlike the Gram and X strips
-                if (row < nr && q * 16 < rb)
+                if (row < nr && q * 16 < rb &&
+                    MA_INB(wbase + (int64_t)(r0 + row) * p.C + c0 + q * 4, 4, w_ext, L.status))
                     __stcs(reinterpret_cast<float4*>(Wb + (int64_t)(r0 + row) * p.C + c0 + q * 4),
                            *reinterpret_cast<const float4*>(buf + sw128w(row, q)));
             }
@@ -456,10 +499,10 @@ __device__ __forceinline__ void abort_drain(Ctl* ctl, const AbortCtl& ab, const 
     }
 }
 
-template <int MODE, bool PAIR>
+template <int MODE, bool PAIR, bool DEEP = false>
 __global__ void __launch_bounds__(THREADS, 1)
     ns_tc_kernel(const __grid_constant__ NsLaunch L) {
-    using S = Shape<MODE, PAIR>;
+    using S = Shape<MODE, PAIR, DEEP>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     constexpr int NST = S::NST;
@@ -638,8 +681,8 @@ __global__ void __launch_bounds__(THREADS, 1)
             }
         }
     } else if (MODE == NS_FINAL) {
-        final_epilogue<PAIR>(L, ctl, pair, npairs, rank, tmem_base, warp, lane, staging + (warp - 2) * FIN_WARP_BYTES,
-                             ab);
+        final_epilogue<PAIR, DEEP>(L, ctl, pair, npairs, rank, tmem_base, warp, lane,
+                                   staging + (warp - 2) * fin_warp_bytes(DEEP), ab);
     } else {
         const int quad = warp & 3;              // TMEM lanes [32*quad, 32*quad + 32)
         const int half = (warp - 2) / 4;        // which half of the 256 columns
@@ -673,7 +716,7 @@ __global__ void __launch_bounds__(THREADS, 1)
                 if (!kApply && col0 < row_lo) continue;                          // below the diagonal
                 float o[32];
                 tmem_ld32(tmem_base + (uint32_t)(acc * S::TN + cc * 32) + ((uint32_t)(quad * 32) << 16), o);
-                epilogue_values<MODE>(p, tc, row, col0, o, o);  // in place
+                epilogue_values<MODE>(p, tc, row, col0, L.status, o, o);  // in place
                 // Stage this warp's 32 x 32 block (and, for an off-diagonal Gram
                 // chunk, its transpose), then write both with bulk tensor stores:
                 // each leaves shared memory as contiguous 64-byte rows.
@@ -774,16 +817,17 @@ bool make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows,
 // stream capture the first time; ns_tc_setup runs it for every instance.
 // Concurrent first calls from several host threads are serialised per
 // instance, and a launch never sees a device whose attribute is not yet set.
-template <int MODE, bool PAIR>
+template <int MODE, bool PAIR, bool DEEP = false>
 cudaError_t setup_mode(int num_sms, int* max_units_out) {
-    using S = Shape<MODE, PAIR>;
+    using S = Shape<MODE, PAIR, DEEP>;
     static PerDevice<int> cache;  // resident pairs (or CTAs) per device, once its attributes are set
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
     return cache.get(dev, max_units_out, [num_sms](int* max_units) -> cudaError_t {
         cudaError_t e =
-            cudaFuncSetAttribute(ns_tc_kernel<MODE, PAIR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)S::SMEM);
+            cudaFuncSetAttribute(ns_tc_kernel<MODE, PAIR, DEEP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)S::SMEM);
         if (e != cudaSuccess) return e;
         if (PAIR) {
             cudaLaunchAttribute attr[1];
@@ -798,13 +842,14 @@ cudaError_t setup_mode(int num_sms, int* max_units_out) {
             qc.attrs = attr;
             qc.numAttrs = 1;
             int nclusters = 0;
-            e = cudaOccupancyMaxActiveClusters(&nclusters, ns_tc_kernel<MODE, PAIR>, &qc);
+            e = cudaOccupancyMaxActiveClusters(&nclusters, ns_tc_kernel<MODE, PAIR, DEEP>, &qc);
             if (e != cudaSuccess) return e;
             if (nclusters < 1) return cudaErrorInvalidConfiguration;
             *max_units = nclusters;
         } else {
             int per_sm = 0;
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ns_tc_kernel<MODE, PAIR>, THREADS, S::SMEM);
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, ns_tc_kernel<MODE, PAIR, DEEP>, THREADS,
+                                                              S::SMEM);
             if (e != cudaSuccess) return e;
             if (per_sm < 1) return cudaErrorInvalidConfiguration;
             *max_units = per_sm * num_sms;
@@ -813,9 +858,9 @@ cudaError_t setup_mode(int num_sms, int* max_units_out) {
     });
 }
 
-template <int MODE, bool PAIR>
+template <int MODE, bool PAIR, bool DEEP = false>
 cudaError_t launch_mode(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_t s) {
-    using S = Shape<MODE, PAIR>;
+    using S = Shape<MODE, PAIR, DEEP>;
     if (njobs < 1 || njobs > kMaxJobs) return cudaErrorInvalidValue;
     static thread_local NsLaunch L;  // ~9 KB parameter block, copied at launch
     std::memset(&L, 0, sizeof(L));
@@ -886,7 +931,7 @@ cudaError_t launch_mode(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_
     L.status = jobs[0].p->status;
     if (tile0 <= 0) return cudaSuccess;
     int max_units = 0;
-    cudaError_t e = setup_mode<MODE, PAIR>(num_sms, &max_units);
+    cudaError_t e = setup_mode<MODE, PAIR, DEEP>(num_sms, &max_units);
     if (e != cudaSuccess) return e;
     cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -903,7 +948,7 @@ cudaError_t launch_mode(const NsJobIn* jobs, int njobs, int num_sms, cudaStream_
     cfg.stream = s;
     cfg.attrs = attr;
     cfg.numAttrs = PAIR ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, ns_tc_kernel<MODE, PAIR>, L);
+    return cudaLaunchKernelEx(&cfg, ns_tc_kernel<MODE, PAIR, DEEP>, L);
 }
 
 // Units with m <= 128 fill only half of a pair's 256-row tile: they take the
@@ -921,7 +966,11 @@ cudaError_t launch_split(const NsJobIn* jobs, int njobs, int num_sms, cudaStream
     if (njobs > kMaxJobs) return cudaErrorInvalidValue;
     cudaError_t e = cudaSuccess;
     if (nb > 0) {
-        e = launch_mode<MODE, true>(big, nb, num_sms, s);
+        // the final apply takes its deep variant when every unit's K loop is long
+        bool deep = MODE == NS_FINAL;
+        for (int j = 0; j < nb; ++j) deep = deep && big[j].p->m >= kDeepFinalMinM;
+        if (MODE == NS_FINAL && deep) e = launch_mode<NS_FINAL, true, true>(big, nb, num_sms, s);
+        else e = launch_mode<MODE, true>(big, nb, num_sms, s);
         if (e != cudaSuccess) return e;
         ++*launched;
     }
@@ -934,39 +983,59 @@ cudaError_t launch_split(const NsJobIn* jobs, int njobs, int num_sms, cudaStream
 }
 
 // Q = a*I + b*A for every unit: the first factor of the Gram-space chain.
-// Eight bf16 elements per thread and step, grid-stride over units and rows.
+// One warp per row of a unit (grid-stride over units x rows); lanes take the
+// row's 16-byte groups of eight bf16 values, four groups in flight at a time.
+__device__ __forceinline__ uint4 q1_group(uint4 v, int row, int c0, float a, float b) {
+    const uint32_t x[4] = {v.x, v.y, v.z, v.w};
+    float f[8];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        f[2 * e] = b * bf16_lo(x[e]);
+        f[2 * e + 1] = b * bf16_hi(x[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+        if (row == c0 + e) f[e] += a;
+    uint4 o;
+    o.x = pack_bf16x2(f[0], f[1]);
+    o.y = pack_bf16x2(f[2], f[3]);
+    o.z = pack_bf16x2(f[4], f[5]);
+    o.w = pack_bf16x2(f[6], f[7]);
+    return o;
+}
+
 __global__ void __launch_bounds__(256) ns_q1_kernel(const __nv_bfloat16* __restrict__ A, __nv_bfloat16* __restrict__ Q,
-                                                    int m, int64_t ldg, int64_t g_unit, int units, float a, float b) {
+                                                    int m, int64_t ldg, int64_t g_unit, int units, float a, float b,
+                                                    int* status) {
     griddep_launch_dependents();
     griddep_wait();
-    const int64_t per_row = (m + 7) / 8;
-    const int64_t total = (int64_t)units * m * per_row;
-    for (int64_t w = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; w < total; w += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t u = w / ((int64_t)m * per_row);
-        const int64_t rem = w - u * m * per_row;
-        const int row = (int)(rem / per_row);
-        const int c0 = (int)(rem - (int64_t)row * per_row) * 8;
-        const int64_t off = u * g_unit + (int64_t)row * ldg + c0;
-        if (c0 + 8 <= m) {
-            const uint4 v = *reinterpret_cast<const uint4*>(A + off);
-            const uint32_t x[4] = {v.x, v.y, v.z, v.w};
-            float f[8];
+    const int lane = threadIdx.x & 31;
+    const int64_t rows = (int64_t)units * m;
+    const int64_t nwarps = (int64_t)gridDim.x * (blockDim.x / 32);
+    const int full = m / 8;  // whole 16-byte groups in a row (the row stride is a multiple of 8)
+    for (int64_t r = (int64_t)blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5); r < rows; r += nwarps) {
+        const int64_t u = r / m;
+        const int row = (int)(r - u * m);
+        const int64_t off = u * g_unit + (int64_t)row * ldg;
+        const uint4* src = reinterpret_cast<const uint4*>(A + off);
+        uint4* dst = reinterpret_cast<uint4*>(Q + off);
+        const int64_t ext = (int64_t)units * g_unit;  // elements of A and of Q (guarded build)
+        (void)ext;
+        int q = lane;
+        for (; q + 96 < full; q += 128) {
+            if (!MA_INB(off + 8 * q, 8 * 97, ext, status)) break;  // groups q .. q + 96
+            uint4 v[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                f[2 * e] = b * bf16_lo(x[e]);
-                f[2 * e + 1] = b * bf16_hi(x[e]);
-            }
-            if (row >= c0 && row < c0 + 8) f[row - c0] += a;
-            uint4 o;
-            o.x = pack_bf16x2(f[0], f[1]);
-            o.y = pack_bf16x2(f[2], f[3]);
-            o.z = pack_bf16x2(f[4], f[5]);
-            o.w = pack_bf16x2(f[6], f[7]);
-            *reinterpret_cast<uint4*>(Q + off) = o;
-        } else {
-            for (int e = 0; c0 + e < m; ++e) {
-                const float f = b * __bfloat162float(A[off + e]) + (row == c0 + e ? a : 0.f);
-                Q[off + e] = __float2bfloat16_rn(f);
+            for (int k = 0; k < 4; ++k) v[k] = __ldcs(src + q + 32 * k);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) __stcs(dst + q + 32 * k, q1_group(v[k], row, 8 * (q + 32 * k), a, b));
+        }
+        for (; q < full; q += 32)
+            if (MA_INB(off + 8 * q, 8, ext, status)) __stcs(dst + q, q1_group(__ldcs(src + q), row, 8 * q, a, b));
+        if (lane == 0 && MA_INB(off, m, ext, status)) {
+            for (int c = 8 * full; c < m; ++c) {
+                const float f = b * __bfloat162float(A[off + c]) + (row == c ? a : 0.f);
+                Q[off + c] = __float2bfloat16_rn(f);
             }
         }
     }
@@ -975,14 +1044,14 @@ __global__ void __launch_bounds__(256) ns_q1_kernel(const __nv_bfloat16* __restr
 }  // namespace
 
 cudaError_t launch_ns_q1(const void* A, void* Q, int m, int64_t ldg, int64_t g_unit, int units, float a, float b,
-                         int num_sms, cudaStream_t s) {
+                         int* status, int num_sms, cudaStream_t s) {
     if (units <= 0 || m <= 0) return cudaSuccess;
-    const int64_t total = (int64_t)units * m * ((m + 7) / 8);
-    int64_t blocks = (total + 255) / 256;
+    const int64_t rows = (int64_t)units * m;
+    int64_t blocks = (rows + 7) / 8;  // eight warps a block, one row each
     if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
     return launch_pdl(ns_q1_kernel, dim3((unsigned)blocks), dim3(256), 0, s,
                       reinterpret_cast<const __nv_bfloat16*>(A), reinterpret_cast<__nv_bfloat16*>(Q), m, ldg, g_unit,
-                      units, a, b);
+                      units, a, b, status);
 }
 
 size_t ns_tc_smem_bytes() {  // the largest dynamic shared memory of any instance
@@ -990,6 +1059,7 @@ size_t ns_tc_smem_bytes() {  // the largest dynamic shared memory of any instanc
 #define MA_MAXS(M, P) m = Shape<M, P>::SMEM > m ? Shape<M, P>::SMEM : m;
     MA_MAXS(NS_GRAM, true) MA_MAXS(NS_GRAM, false) MA_MAXS(NS_GRAMSQ, true) MA_MAXS(NS_GRAMSQ, false)
     MA_MAXS(NS_APPLY, true) MA_MAXS(NS_APPLY, false) MA_MAXS(NS_FINAL, true) MA_MAXS(NS_FINAL, false)
+    m = Shape<NS_FINAL, true, true>::SMEM > m ? Shape<NS_FINAL, true, true>::SMEM : m;
 #undef MA_MAXS
     return m;
 }
@@ -1002,12 +1072,14 @@ cudaError_t ns_tc_setup(int num_sms) {
     if ((e = setup_mode<M, P>(num_sms, &u)) != cudaSuccess) return e;
     MA_SETUP(NS_GRAM, true) MA_SETUP(NS_GRAM, false) MA_SETUP(NS_GRAMSQ, true) MA_SETUP(NS_GRAMSQ, false)
     MA_SETUP(NS_APPLY, true) MA_SETUP(NS_APPLY, false) MA_SETUP(NS_FINAL, true) MA_SETUP(NS_FINAL, false)
+    if ((e = setup_mode<NS_FINAL, true, true>(num_sms, &u)) != cudaSuccess) return e;
 #undef MA_SETUP
     return cudaSuccess;
 }
 
 bool ns_tc_is_final(const void* func) {
     return func == reinterpret_cast<const void*>(ns_tc_kernel<NS_FINAL, true>) ||
+           func == reinterpret_cast<const void*>(ns_tc_kernel<NS_FINAL, true, true>) ||
            func == reinterpret_cast<const void*>(ns_tc_kernel<NS_FINAL, false>);
 }
 

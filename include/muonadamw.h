@@ -52,7 +52,9 @@ typedef enum {
     MA_ERR_UNSUPPORTED = 6, /* a valid request this build does not implement      */
     MA_ERR_CUDA = 7,        /* a CUDA runtime call failed                         */
     MA_ERR_TIMEOUT = 8,     /* a device-side bounded wait ran out (status word)   */
-    MA_ERR_ARG = 9          /* a hyperparameter is out of its domain              */
+    MA_ERR_ARG = 9,         /* a hyperparameter is out of its domain              */
+    MA_ERR_BOUNDS = 10      /* debug builds: a guarded device index fell outside  */
+                            /* its buffer and the access was skipped (status word) */
 } ma_status_t;
 
 typedef enum { MA_F32 = 0, MA_BF16 = 1 } ma_dtype_t;
@@ -430,6 +432,13 @@ int ma_set_wait_limit_ns(int64_t limit_ns);
  * tiles, and every launch then ends with its slowest pair; on the 7B-shaped
  * set the step took 270 ms with it and 251.5 ms without on the same GPU. */
 int ma_set_momentum_overlap(int on);
+
+/* 1 in the debug build of the library (libmuonadamw_debug.so, compiled with
+ * -DMA_DEBUG), else 0. The debug build checks every hand-computed device
+ * index against the extent of its buffer before the access; a failed check
+ * records MA_ERR_BOUNDS in the status word and skips the access. Its results
+ * are otherwise bit-identical to the release build's. */
+int ma_debug_build(void);
 
 /* Self-test of the bounded wait: launch one block that waits on a barrier
  * phase that nothing completes, with a wait limit of limit_ns. The kernel

@@ -215,16 +215,17 @@ def aspect(d: int = 4096, ff: int = 14336, heads: int = 32) -> Workload:
 
 
 def rect(batch: int = 8, R: int = 4096, C: int = 11008) -> Workload:
-    """Batch of the 7B-shaped set's wide MLP matrices (4096 x 11008), grads N(0, 1e-3^2) in bf16."""
+    """Batch of the 7B-shaped set's MLP matrices (4096 x 11008 by default; 11008 x 4096 is the tall
+    one), grads N(0, 1e-3^2) in bf16."""
     groups = [_muon_group(lr=0.02, beta=0.95, weight_decay=0.01, nesterov=True, ns_steps=5)]
     t = [TensorSpec(f"mlp{i}", (R, C), ROLE_HIDDEN, 0) for i in range(batch)]
     return Workload(f"rect{batch}x{R}x{C}", t, groups, f"{batch} matrices {R}x{C}, bf16 grads N(0,1e-3^2)")
 
 
 WORKLOADS = {"tiny": tiny, "d20": d20, "square": square, "aspect": aspect, "7b": llama7b,
-             # few-GB cases for profiler captures: 8 square 4096x4096 matrices, and
-             # 8 of the 7B set's 4096x11008 MLP matrices
-             "square8": lambda: square(8), "rect8": lambda: rect(8)}
+             # few-GB cases for profiler captures: 8 square 4096x4096 matrices, 8 of
+             # the 7B set's 4096x11008 MLP matrices, and 8 of its 11008x4096 ones
+             "square8": lambda: square(8), "rect8": lambda: rect(8), "tall8": lambda: rect(8, 11008, 4096)}
 
 
 # ---------------------------------------------------------------------------

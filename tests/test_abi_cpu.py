@@ -35,6 +35,21 @@ def test_header_symbols_exported():
         assert hasattr(L, n), f"{n} declared in muonadamw.h but not exported"
 
 
+def test_debug_build_loads_and_exports_the_same_abi():
+    # the debug library (guarded device indexing) is built beside the release
+    # one; each reports which it is, and the debug one exports every symbol too
+    assert ma.ma_debug_build() == (os.environ.get("MA_LIBRARY") == "debug")
+    dbg = os.path.join(os.path.dirname(ma.LIB_PATH), "libmuonadamw_debug.so")
+    D = ctypes.CDLL(dbg)
+    for n in declared_functions():
+        assert hasattr(D, n), f"{n} not exported by the debug build"
+    D.ma_debug_build.restype = ctypes.c_int
+    D.ma_status_string.restype = ctypes.c_char_p
+    assert D.ma_debug_build() == 1
+    assert D.ma_status_string(ma.MA_ERR_BOUNDS) == b"guarded device index out of bounds (debug build)"
+    assert ma.lib().ma_status_string(ma.MA_ERR_BOUNDS) == b"guarded device index out of bounds (debug build)"
+
+
 def test_binding_constants_match_header_macros():
     # the binding's copies of the header's size constants (the allocation-free
     # entry point's scratch size among them) must be the header's values

@@ -97,3 +97,38 @@ def test_graph_step_equals_eager_step():
             assert torch.equal(s0, t0) and (s1 is None or torch.equal(s1, t1)), f"step {step}: state {i}"
         assert graph.launches == eager.launches
         assert graph.graph_captures == CAPTURES_AFTER[step], f"step {step}"
+
+
+def test_graph_patches_the_deep_final_apply():
+    # matrices with m >= 2048 only, so that the final applies take the deep
+    # variant (5-stage ring): a square one (a*X term) and a wide one
+    # (Gram-space chain, a = 0); lr and decay change every step and must be
+    # patched into the deep kernel's parameter block, with no re-capture
+    table = [((2048, 2048), H, 0), ((2048, 2560), H, 0)]
+    r = np.random.default_rng(78)
+    P0 = [(r.standard_normal(s) * 0.02).astype(np.float32) for s, *_ in table]
+    lrs = [(0.02, 0.01), (0.015, 0.02), (0.01, 0.0)]
+
+    def make():
+        params = [dev_f32(p) for p in P0]
+        return params, ma.MuonAdamW([(p, role, g) for p, (_, role, g) in zip(params, table)],
+                                    [("muon", ma.muon_hparams(lr=lrs[0][0], weight_decay=lrs[0][1]))])
+
+    pa, eager = make()
+    pb, graph = make()
+    ga = [dev_grad(np.zeros(s), "bf16") for s, *_ in table]
+    gb = [dev_grad(np.zeros(s), "bf16") for s, *_ in table]
+    for step, (lr, wd) in enumerate(lrs, start=1):
+        G = [bf16_round(r.standard_normal(s) * 1e-3) for s, *_ in table]
+        for a, b, g in zip(ga, gb, G):
+            a.copy_(dev_grad(g, "bf16"))
+            b.copy_(a)
+        for opt in (eager, graph):
+            opt.groups[0].muon = ma.muon_hparams(lr=lr, weight_decay=wd)
+        eager.step(ga)
+        graph.step(gb, graph=True)
+        torch.cuda.synchronize()
+        assert ma.ma_device_status() == ma.MA_OK
+        for i, (x, y) in enumerate(zip(pa, pb)):
+            assert torch.equal(x, y), f"step {step}: parameter {i}"
+        assert graph.graph_captures == 1
