@@ -110,8 +110,9 @@ __device__ __forceinline__ float prep_flat_pass(const MuonPrepLaunch& L, int u, 
     const float beta = L.beta, omb = L.omb;
     const bool nest = L.nesterov != 0;
     // buffer extents for the guarded build: a matrix's G and M, and the workspace's X
-    const int64_t mat_elems = (int64_t)L.heads * unit_elems, x_elems = (int64_t)L.batch * L.heads * L.x_unit;
-    const int64_t xu = (int64_t)u * L.x_unit;
+    [[maybe_unused]] const int64_t mat_elems = (int64_t)L.heads * unit_elems;
+    [[maybe_unused]] const int64_t x_elems = (int64_t)L.batch * L.heads * L.x_unit;
+    [[maybe_unused]] const int64_t xu = (int64_t)u * L.x_unit;
     float ss = 0.f;
     if (end - start == kPrepChunk) {
         float g[kIter][8], m[kIter][8];
@@ -255,7 +256,8 @@ __global__ void __launch_bounds__(kPrepSideThreads, 6) prep_transpose_kernel(con
         const int rows = c < L.C ? (int)max((int64_t)0, min((int64_t)RW, L.Rh - r0)) : 0;
         const int64_t e0 = off + r0 * L.C + c;  // element index of (r0, c)
         // buffer extents for the guarded build: a matrix's G and M, and the workspace's X
-        const int64_t mat_elems = (int64_t)L.heads * L.Rh * L.C, x_elems = (int64_t)L.batch * L.heads * L.x_unit;
+        [[maybe_unused]] const int64_t mat_elems = (int64_t)L.heads * L.Rh * L.C;
+        [[maybe_unused]] const int64_t x_elems = (int64_t)L.batch * L.heads * L.x_unit;
         float* mp = L.M[b] + e0;
         const uint32_t* gp = reinterpret_cast<const uint32_t*>(L.G[b]) + (GBF16 ? e0 / 2 : e0);
         const int64_t gstride = GBF16 ? L.C / 2 : L.C;  // words per row

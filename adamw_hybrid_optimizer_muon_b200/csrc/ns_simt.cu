@@ -45,9 +45,8 @@ __global__ void __launch_bounds__(256) ns_simt_kernel(const __grid_constant__ Ns
         SB = xb + (int64_t)u * p.x_unit; ldb = p.ldx; b_unit = p.x_unit;
     }
     // element offsets from the buffers' starts, and their extents
-    const int64_t a0 = (int64_t)u * a_unit, a_ext = (int64_t)p.units * a_unit;
-    const int64_t b0 = (int64_t)u * b_unit, b_ext = (int64_t)p.units * b_unit;
-    (void)a0; (void)a_ext; (void)b0; (void)b_ext;
+    [[maybe_unused]] const int64_t a0 = (int64_t)u * a_unit, a_ext = (int64_t)p.units * a_unit;
+    [[maybe_unused]] const int64_t b0 = (int64_t)u * b_unit, b_ext = (int64_t)p.units * b_unit;
     const int tid = threadIdx.x;
     const int ty = tid >> 4, tx = tid & 15;
     float acc[4][4] = {};
@@ -106,7 +105,8 @@ __global__ void __launch_bounds__(256) ns_simt_kernel(const __grid_constant__ Ns
             const float v = acc[r][c];
             const int64_t gi = (int64_t)u * p.g_unit + (int64_t)i * p.ldg + j;  // (i, j) in a Gram buffer
             const int64_t xi = (int64_t)u * p.x_unit + (int64_t)i * p.ldx + j;  // (i, j) in an X buffer
-            const int64_t g_ext = (int64_t)p.units * p.g_unit, x_ext = (int64_t)p.units * p.x_unit;
+            [[maybe_unused]] const int64_t g_ext = (int64_t)p.units * p.g_unit;
+            [[maybe_unused]] const int64_t x_ext = (int64_t)p.units * p.x_unit;
             if (MODE == NS_GRAM) {
                 float coef = p.coef_gram;
                 if (p.first) coef *= sa * sa;
