@@ -1024,15 +1024,18 @@ int side_resources(ma_plan* plan, int dev, size_t nevents, cudaStream_t* side) {
 // One step over segments, on stream s. ready (may be null): per segment, an
 // event its work must wait for (the host copies of its gradients).
 //
-// With the plan's double workspace (plan->region > 0), the Muon segments use
-// its two halves in turn, and the momentum pass of segment q + 1 runs on the
-// plan's side stream, on a small grid that fits beside the Newton-Schulz
-// CTAs, while segment q's chain runs: the HBM-bound pass hides under the
-// tensor-core work. The side stream starts after all work queued on s before
-// the step; segment q + 1's momentum pass waits for the chain of segment
-// q - 1, the last user of its workspace half; segment q + 1's chain waits for
-// its momentum pass; s waits for the side stream at the end. Every kernel
-// does the same arithmetic as on one stream, so the results are the same bits.
+// With the plan's double workspace (plan->region > 0, only for plans made
+// with ma_set_momentum_overlap on), the Muon segments use its two halves in
+// turn, and the momentum pass of segment q + 1 runs on the plan's side
+// stream, on a small grid that fits beside the Newton-Schulz CTAs, while
+// segment q's chain runs. It is off by default: on a B200 the side blocks
+// slow the CTA pairs they share SMs with by more than the pass costs inline,
+// and every launch ends with its slowest pair. The side stream starts after
+// all work queued on s before the step; segment q + 1's momentum pass waits
+// for the chain of segment q - 1, the last user of its workspace half;
+// segment q + 1's chain waits for its momentum pass; s waits for the side
+// stream at the end. Every kernel does the same arithmetic as on one stream,
+// so the results are the same bits.
 int run_segments(ma_plan* plan, const ma_group_t* groups, const std::vector<Segment>& segs, void* ws, cudaStream_t s,
                  int sms, int* launches, const cudaEvent_t* ready) {
     std::vector<int> mi;  // Muon segments, in order
