@@ -141,3 +141,15 @@ def test_traffic_record_writer_scales_captures_to_the_7b_step(tmp_path, monkeypa
     rec["kernel_sha16"] = "0" * 16
     rec_path.write_text(json.dumps(rec))
     assert bench.ns_traffic("7b", 36) is None
+
+
+def test_committed_traffic_record_matches_the_kernel_sources():
+    # the per-launch DRAM record must belong to the kernel sources in the tree,
+    # or bench.py prints no traffic: re-capture it after changing the kernel
+    sys.path.insert(0, ROOT)
+    import bench
+    with open(os.path.join(ROOT, bench.NS_TRAFFIC_RECORD)) as f:
+        rec = json.load(f)
+    assert rec["kernel_sha16"] == bench.ns_kernel_sha16()
+    assert rec["workloads"]["7b"]["ns_launches_per_step"] > 0
+    assert 1.0 < rec["workloads"]["7b"]["bytes_per_launch"] / 2.38e9 < 1.5  # within 1-1.5x the algorithmic bytes
