@@ -76,3 +76,28 @@ def test_gram_space_chain_is_taken_and_repeatable():
         assert opt.launches == 2 + 1 + 1 + 12 + 1
         outs.append(p.clone())
     assert torch.equal(outs[0], outs[1])
+
+
+@pytest.mark.parametrize("shape", [(2056, 2600), (2056, 2056)], ids=["gram_space", "direct"])
+def test_deep_final_apply_ragged_matches_oracle(shape):
+    # m = 2056 >= 2048 takes the deep final-apply variant (5-stage ring, X read
+    # per lane) with a ragged last tile row (2056 = 8 x 256 + 8): on the
+    # Gram-space chain (a = 0, no X term) and on the direct chain (a * X term)
+    R, C = shape
+    hp = ma.muon_hparams()
+    r = np.random.default_rng(R + C)
+    batch = 2
+    W0 = [(r.standard_normal((R, C)) * 0.02).astype(np.float32) for _ in range(batch)]
+    Wd = [dev_f32(w) for w in W0]
+    Md = [torch.zeros((R, C), device="cuda") for _ in range(batch)]
+    ws = torch.empty(ma.muon_workspace_bytes(batch, R, C, hp), dtype=torch.uint8, device="cuda")
+    G = [bf16_round(r.standard_normal((R, C)) * 1e-3) for _ in range(batch)]
+    ma.muon_step_batched(Wd, [dev_grad(g, "bf16") for g in G], Md, hp, ws)
+    torch.cuda.synchronize()
+    assert ma.ma_device_status() == ma.MA_OK
+    co32 = ((f32(1.5), f32(-0.5), f32(0.0)),)
+    for w0, g, w, m in zip(W0, G, Wd, Md):
+        rw, rm = oracle.muon_update(w0, g, np.zeros_like(w0), f32(0.02), f32(0.95), f32(0.01), True, 5, co32,
+                                    f32(1e-7), 0, 1, False)
+        check_state(host(m), rm, momentum_terms(np.zeros_like(w0), g, f32(0.95)), what="momentum")
+        check_muon(w0, host(w), rw, f32(0.02), f32(0.01), TOL_BF16, what=f"{R}x{C} deep final")
