@@ -5,8 +5,9 @@ X_N = Q_N X_0 with Q and A updated by symmetric m x m products (upper tiles,
 mirrored) instead of N Grams and N applies on X. The oracle runs the pages'
 iteration itself, so these cases check the reformulation end to end: wide
 and tall (transposed) matrices, ragged sizes on both sides, the 1.25 ratio
-at its boundary, head slices, one iteration, a per-iteration coefficient
-table, cautious decay, two steps (momentum carried), and repeatability.
+at its boundary, wide and tall head slices, one iteration, a per-iteration
+coefficient table, cautious decay, two steps (momentum carried), and
+repeatability.
 """
 import numpy as np
 import pytest
@@ -26,6 +27,7 @@ CASES = [
     ((640, 800), 1, ((1.5, -0.5, 0.0),), False),        # n = 1.25 m, m = 2.5 tiles
     ((520, 2056), 1, ((1.5, -0.5, 0.0),), True),        # ragged both ways, cautious decay
     ((1536, 4096), 3, ((1.5, -0.5, 0.0),), False),      # three head slices of 512 x 4096
+    ((2048, 512), 2, ((1.5, -0.5, 0.0),), False),       # two tall head slices of 1024 x 512 (transposed)
     ((768, 2048), 1, ((2.0, -1.0, 0.0), (1.75, -0.75, 0.0), (1.5, -0.5, 0.0)), False),  # 3 iterations, a table
     ((512, 1536), 1, ((1.5, -0.5, 0.0),) * 1, False),   # steps = 1 below
 ]
