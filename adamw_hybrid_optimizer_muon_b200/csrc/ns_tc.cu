@@ -10,7 +10,11 @@
 //                                  writes its elements and their mirror)
 //           epilogue: B = coef * A, coef = b * s^2 on the first iteration
 //           (s = 1/(||u||_F + eps), the Frobenius normalisation), else b.
-//   GRAMSQ  (only when c != 0) B = b*A + c*A*A, with A*A = A A^T by symmetry
+//   GRAMSQ  a symmetric m x m product out = b*Z + c*A Z (Z = A: b*A + c*A^2,
+//           the extra term when c != 0; Z a second symmetric matrix that
+//           commutes with A: the Gram-space chain's Q and A updates, which
+//           reach X_N = Q_N X_0 from m x m products only); A Z = A Z^T by
+//           symmetry, and only tiles touching the upper triangle run
 //   APPLY   X' = s * (a X + B X)  (s only on the first iteration)
 //   FINAL   the last APPLY. Its epilogue does the decoupled decay and the
 //           update, W <- W*(1 - lr*wd) - lr*scale*X_N, straight into the
@@ -22,7 +26,8 @@
 // one mode, tiles numbered job after job), 320 threads per CTA:
 //   warp 0      TMA producer in each CTA: this CTA's half of the A tile
 //               (128 rows x 64) and of the B tile (128 columns x 64), bf16,
-//               128B swizzle, 6 stages of 32 KB (4 in the final apply). Both
+//               128B swizzle, 6 stages of 32 KB (the final apply: 4, or 5 in
+//               its deep variant for m >= 2048). Both
 //               CTAs' loads complete on the leader CTA's stage barrier; there
 //               is no multicast. A diagonal Gram tile loads only A.
 //   warp 1      TMEM allocation in both CTAs (cta_group::2, 2 x 256 fp32
@@ -37,9 +42,10 @@
 // single-CTA 128 x 256 tile. Units with m <= 128 would fill half of that tile;
 // they run on a single-CTA instance of the same template (cta_group::1,
 // 128 x 256 tiles, 128 x 128 for the Gram).
-// B operand major-ness: for GRAM and GRAMSQ both operands are K-major rows of
-// the same matrix. For APPLY the B operand is X itself, read MN-major (the
-// contraction runs over X's rows), so no transposed copy is ever made.
+// B operand major-ness: for GRAM and GRAMSQ both operands are K-major rows
+// (of the same matrix, or of A and Z). For APPLY the B operand is X itself,
+// read MN-major (the contraction runs over X's rows), so no transposed copy
+// is ever made.
 // Tile order and L2: the applies walk each unit's tiles column by column, so
 // the pairs running at the same time share a few column strips of X and all
 // of the m x m Gram, which they load with an evict-last L2 policy; every
