@@ -405,3 +405,32 @@ def test_plan_status_without_gpu_fails_loudly():
         assert ma.ma_plan_status(plan, 0) == ma.MA_ERR_CUDA  # no device: an error, never a fake OK
     finally:
         ma.ma_plan_destroy(plan)
+
+
+@pytest.mark.parametrize("shape,heads,kw,gspace", [
+    ((512, 1024), 1, {}, True),                      # m n = 2^19 exactly, n = 2 m
+    ((1024, 512), 1, {}, True),                      # tall: the unit is its transpose
+    ((512, 1016), 1, {}, False),                     # m n below 2^19
+    ((672, 840), 1, {}, True),                       # 4 n = 5 m exactly (m n above 2^19)
+    ((672, 832), 1, {}, False),                      # 4 n < 5 m
+    ((1024, 1024), 1, {}, False),                    # square
+    ((128, 4096), 1, {}, True),                      # m = 128
+    ((120, 4400), 1, {}, False),                     # m < 128
+    ((4096, 4096), 32, {}, True),                    # head slices of 128 x 4096
+    ((512, 1024), 1, {"precision": 1}, False),       # fp32 mode keeps the direct chain
+    ((512, 1024), 1, {"coeffs": ((2.0, -1.5, 0.5),)}, False),  # c != 0
+])
+def test_gram_space_selection(shape, heads, kw, gspace):
+    # which units take the Gram-space chain: m >= 128, 4 n >= 5 m and
+    # m n >= 2^19 (m the short side of a unit), bf16 operands, no c term
+    d = _desc(shape, ma.ROLE_HIDDEN, 0)
+    d.param, d.state0, d.state1, d.grad = (1 << 32), (2 << 32), (3 << 32), (4 << 32)
+    d.grad_dtype = ma.MA_BF16
+    G = ma.Group()
+    G.kind = ma.MA_MUON
+    G.muon = ma.muon_hparams(heads=heads, **kw)
+    plan, _ = ma.ma_plan_create([d], [G])
+    text = ma.ma_plan_describe(plan, [G])
+    ma.ma_plan_destroy(plan)
+    assert ("Gram-space chain" in text) == gspace, text
+    assert ("direct chain" in text) == (not gspace), text

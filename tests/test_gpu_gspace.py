@@ -24,7 +24,7 @@ CASES = [
     # (R, C), heads, coefficient table, cautious
     ((512, 1024), 1, ((1.5, -0.5, 0.0),), False),
     ((1024, 512), 1, ((1.5, -0.5, 0.0),), False),       # tall: X = u^T, written back transposed
-    ((640, 800), 1, ((1.5, -0.5, 0.0),), False),        # n = 1.25 m, m = 2.5 tiles
+    ((672, 840), 1, ((1.5, -0.5, 0.0),), False),        # n = 1.25 m exactly, m = 2.6 tiles
     ((520, 2056), 1, ((1.5, -0.5, 0.0),), True),        # ragged both ways, cautious decay
     ((1536, 4096), 3, ((1.5, -0.5, 0.0),), False),      # three head slices of 512 x 4096
     ((2048, 512), 2, ((1.5, -0.5, 0.0),), False),       # two tall head slices of 1024 x 512 (transposed)
